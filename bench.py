@@ -1,0 +1,397 @@
+"""Benchmark of the fused EAAS + on-the-fly equivariant attention hot path.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one pass of the whole hot path over one synthetic system:
+radius graph (egat_build_graph) -> EAAS source coupling (egat_eaas_couple)
+-> on-the-fly attention with the target coupling fused (egat_otf_attention_coupled).
+The default workload is the 32,768-atom, K = 256, ℓmax = 2, bf16-storage
+system.  Inputs are resident in HBM when the timed region starts; L2 is
+flushed (a 256 MiB write) before every timed step, outside the step's events.
+
+Prints ONE JSON line (rank 0).  ``value`` is atoms/s over all ranks; edges/s,
+per-kernel times, the roofline of the dominant kernel, the CPU oracle baseline
+and an end-to-end figure through host buffers ride along.
+
+Multi-GPU (torchrun): every rank runs its own independent system (same shape,
+seeded by rank) — the units are independent problems, so there is no
+data-path collective; timing is the max over ranks.  ``--impl reference``
+times the CPU oracle on the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from equivariant_graph_attention_b200 import synth  # noqa: E402
+
+METRIC = "atoms/s & edges/s, fused EAAS+on-the-fly attention; % of HBM roofline"
+DEFAULT_WORKLOAD = "uniform32768_K256_l2_bf16"
+FLUSH_BYTES = 256 << 20
+#: kernels this library launches per step: graph (assign, scan x3, scatter,
+#: count, fill) + source coupling + fused attention
+LAUNCHES_PER_STEP = 9
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attention_traffic.json")
+KERNEL_SOURCES = ["equivariant_graph_attention_b200/csrc/attention.cu",
+                  "equivariant_graph_attention_b200/csrc/egat_device.cuh"]
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def algorithmic_bytes(wl: synth.Workload, cnt: np.ndarray) -> dict:
+    """Bytes the method itself moves, per kernel (each counted once).
+
+    attention (steps 3+4): per target the padded list row (K*4) and count (4),
+    q_i, r_i (12) and the float32 output row; per real edge the neighbour's
+    key and value rows.  source coupling (step 2): read h, write h', r.
+    """
+    s = 2 if wl.dtype == "bf16" else 4
+    N, D, C, H, dk, K = wl.n, wl.D, wl.C, wl.H, wl.dk, wl.K
+    E = int(cnt.sum())
+    attn = N * (K * 4 + 4 + H * dk * s + 12 + D * C * 4) + E * (D * C * s + H * dk * s)
+    eaas = N * (2 * D * C * s + 12)
+    return {"attention": attn, "eaas": eaas, "edges": E}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- oracle
+def oracle_sample(wl: synth.Workload, data: dict, n_targets: int, seed: int = 0) -> float:
+    """Seconds the CPU oracle takes for the forward pass of ``n_targets``
+    sampled targets (their brute-force neighbour rows, the source coupling of
+    the atoms they need, two-pass attention and target coupling)."""
+    from oracle.attention import forward
+    from oracle.graph import radius_graph
+
+    rows = np.random.default_rng(seed).choice(wl.n, size=n_targets, replace=False)
+    t0 = time.perf_counter()
+    lists, _ = radius_graph(data["pos_q"], wl.cutoff_q, K=wl.K, rows=rows)
+    forward(data["h"], data["pos"], data["q"], data["k"], data["w1"], data["w2"], wl.lmax,
+            lists, targets=rows)
+    return time.perf_counter() - t0
+
+
+def cpu_threads_used() -> int:
+    # numpy einsum and the integer neighbour search run on one thread
+    return 1
+
+
+# ---------------------------------------------------------------------------- distributed
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def run_reference(args, wl: synth.Workload):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    data = synth.make(wl)
+    per_step_targets = args.ref_targets
+    for _ in range(args.warmup):
+        oracle_sample(wl, data, max(1, per_step_targets // 4), seed=99)
+    secs = [oracle_sample(wl, data, per_step_targets, seed=s) for s in range(args.steps)]
+    total = float(sum(secs))
+    value = per_step_targets * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "atoms/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "atoms": wl.n, "K": wl.K, "lmax": wl.lmax, "C": wl.C,
+                   "H": wl.H, "dk": wl.dk, "cutoff_A": wl.cutoff},
+        "cpu_baseline": {"value": value, "unit": "atoms/s", "cores": cpu_threads_used(),
+                         "kind": "oracle",
+                         "sample": f"{per_step_targets} random target atoms per step of the "
+                                   f"{wl.n}-atom system (neighbour rows, source coupling of "
+                                   f"their neighbours, attention, target coupling)"},
+        "e2e": {"value": value, "unit": "atoms/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=synth.WORKLOAD_ORDER)
+    ap.add_argument("--impl", default="egat", choices=["egat", "reference"])
+    ap.add_argument("--ref-targets", type=int, default=64)
+    ap.add_argument("--cpu-targets", type=int, default=256)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from equivariant_graph_attention_b200 import egat
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=dev)
+    egat.load_library()
+
+    data = synth.make(wl, seed=rank)
+    st = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+
+    def td(x, dt):
+        return torch.from_numpy(np.ascontiguousarray(x)).to(dev, dtype=dt)
+
+    h, q, k = td(data["h"], st), td(data["q"], st), td(data["k"], st)
+    pos, pos_q = td(data["pos"], torch.float32), td(data["pos_q"], torch.int32)
+    w1, w2 = td(data["w1"], torch.float32), td(data["w2"], torch.float32)
+    shape = egat.Shape(n=wl.n, lmax=wl.lmax, C=wl.C, H=wl.H, dk=wl.dk, K=wl.K, dtype=wl.dtype)
+    gws = torch.empty(egat.egat_graph_workspace_bytes(wl.n), dtype=torch.uint8, device=dev)
+    nbr = torch.empty((wl.n, wl.K), dtype=torch.int32, device=dev)
+    cnt = torch.empty(wl.n, dtype=torch.int32, device=dev)
+    order = torch.empty(wl.n, dtype=torch.int32, device=dev)
+    ovf = torch.zeros(1, dtype=torch.int32, device=dev)
+    hp = torch.empty((wl.n, wl.D, wl.C), dtype=st, device=dev)
+    out = torch.empty((wl.n, wl.D, wl.C), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    lib = egat.load_library()
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    cshape = shape.c()
+    import ctypes
+
+    def graph():
+        rc = lib.egat_build_graph(pos_q.data_ptr(), wl.n, wl.cutoff_q, wl.K, 0, nbr.data_ptr(),
+                                  cnt.data_ptr(), 0, order.data_ptr(), ovf.data_ptr(),
+                                  gws.data_ptr(), gws.numel(), sp)
+        egat._check("egat_build_graph", rc)
+
+    def couple():
+        rc = lib.egat_eaas_couple(ctypes.byref(cshape), h.data_ptr(), pos.data_ptr(),
+                                  w1.data_ptr(), hp.data_ptr(), sp)
+        egat._check("egat_eaas_couple", rc)
+
+    def attend():
+        rc = lib.egat_otf_attention_coupled(ctypes.byref(cshape), q.data_ptr(), k.data_ptr(),
+                                            hp.data_ptr(), nbr.data_ptr(), cnt.data_ptr(),
+                                            order.data_ptr(), pos.data_ptr(), w2.data_ptr(),
+                                            out.data_ptr(), sp)
+        egat._check("egat_otf_attention_coupled", rc)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        graph()
+        couple()
+        attend()
+    torch.cuda.synchronize(dev)
+    cnt_host = cnt.cpu().numpy()
+    alg = algorithmic_bytes(wl, cnt_host)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    for s in range(args.steps):
+        flush.fill_(s & 0xff)
+        e = ev[s]
+        e[0].record(stream)
+        graph()
+        e[1].record(stream)
+        couple()
+        e[2].record(stream)
+        attend()
+        e[3].record(stream)
+    torch.cuda.synchronize(dev)
+    if ws > 1:
+        dist.barrier()
+    clk = clocks.stop()
+
+    t_graph = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    t_eaas = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    t_attn = sum(e[2].elapsed_time(e[3]) for e in ev) / args.steps
+    t_step = sum(e[0].elapsed_time(e[3]) for e in ev) / args.steps      # ms
+    total_ms = t_step * args.steps
+    if ws > 1:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    atoms_total = wl.n * ws * args.steps
+    value = atoms_total / (total_ms / 1000.0)
+    edges_per_s = alg["edges"] * ws * args.steps / (total_ms / 1000.0)
+
+    # ------------------------------------------------------------------ e2e
+    # the same step through the C ABI with the inputs in pinned host memory:
+    # copies in, graph, fused forward, copy of the result out
+    host = {nm: torch.from_numpy(np.ascontiguousarray(data[nm])).to(
+        dtype=(st if nm in ("h", "q", "k") else (torch.int32 if nm == "pos_q" else torch.float32))
+    ).pin_memory() for nm in ("h", "q", "k", "pos", "pos_q", "w1", "w2")}
+    dmap = {"h": h, "q": q, "k": k, "pos": pos, "pos_q": pos_q, "w1": w1, "w2": w2}
+    out_host = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    fws = torch.empty(egat.egat_forward_workspace_bytes(shape), dtype=torch.uint8, device=dev)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        for nm, t in host.items():
+            dmap[nm].copy_(t, non_blocking=True)
+        graph()
+        rc = lib.egat_forward(ctypes.byref(cshape), h.data_ptr(), pos.data_ptr(), q.data_ptr(),
+                              k.data_ptr(), nbr.data_ptr(), cnt.data_ptr(), order.data_ptr(),
+                              w1.data_ptr(), w2.data_ptr(), fws.data_ptr(), fws.numel(),
+                              out.data_ptr(), sp)
+        egat._check("egat_forward", rc)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if ws > 1:
+        dist.barrier()
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ea.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    eb.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = ea.elapsed_time(eb)
+    if ws > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e_value = wl.n * ws * args.e2e_steps / (e2e_ms / 1000.0)
+
+    # ------------------------------------------------------------------ roofline
+    peaks = measured_peaks()
+    achieved = alg["attention"] / (t_attn / 1000.0) / 1e9      # GB/s
+    traffic = None
+    if os.path.exists(TRAFFIC_FILE):
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+        if rec.get("source_sha") == kernel_source_sha() and rec.get("workload") == wl.name:
+            traffic = rec.get("dram_bytes_per_launch")
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        oracle_sample(wl, data, 4, seed=123)        # warm caches / imports
+        secs = oracle_sample(wl, data, args.cpu_targets, seed=7)
+        cpu = {"value": args.cpu_targets / secs, "unit": "atoms/s", "cores": cpu_threads_used(),
+               "kind": "oracle",
+               "sample": f"{args.cpu_targets} random target atoms of the {wl.n}-atom system "
+                         f"(brute-force neighbour rows, dense source coupling of their "
+                         f"neighbours, two-pass attention, dense target coupling), "
+                         f"{secs:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "atoms/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": wl.dtype, "data": "synthetic",
+            "config": {"workload": wl.name, "atoms": wl.n, "edges": alg["edges"], "K": wl.K,
+                       "lmax": wl.lmax, "C": wl.C, "H": wl.H, "dk": wl.dk,
+                       "cutoff_A": wl.cutoff, "accumulate": "f32",
+                       "l2": "flushed before every timed step (256 MiB write, untimed)",
+                       "parallelism": f"{ws} independent systems (one per GPU)"},
+            "edges_per_s": edges_per_s,
+            "kernel_ms": {"build_graph": t_graph, "eaas_couple": t_eaas,
+                          "otf_attention_coupled": t_attn},
+            "roofline": {"bound": "hbm", "kernel": "otf_attention_coupled",
+                         "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                         "algorithmic_bytes": alg["attention"], "peak_source": peaks["source"]},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "atoms/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.e2e_steps},
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,173 @@
+// extern "C" entry points of libegat.so: argument validation, workspace
+// carving and dispatch to the kernels.  The ABI itself is documented in
+// include/egat.h.
+#include <cstring>
+
+#include "egat_device.cuh"
+#include "egat_host.h"
+
+using namespace egat;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+// Shape checks common to steps 2-4 (supported set stated in egat.h).
+int check_shape(const egat_shape* s, bool need_graph) {
+  if (!s) return EGAT_ERR_ARG;
+  if (s->n < 0) return EGAT_ERR_ARG;
+  if (s->dtype != EGAT_F32 && s->dtype != EGAT_BF16) return EGAT_ERR_ARG;
+  if (s->lmax < 1 || s->lmax > kMaxL) return EGAT_ERR_UNSUPPORTED;
+  if (s->C != 16 && s->C != 32 && s->C != 64 && s->C != 128) return EGAT_ERR_UNSUPPORTED;
+  if (need_graph) {
+    if (!pow2(s->H) || s->C % s->H != 0 || (s->C / s->H) % 8 != 0) return EGAT_ERR_UNSUPPORTED;
+    if (s->dk != 8 && s->dk != 16 && s->dk != 32) return EGAT_ERR_UNSUPPORTED;
+    if (s->H * s->dk > 256) return EGAT_ERR_UNSUPPORTED;
+    if (s->graph_mode == EGAT_GRAPH_PADDED) {
+      if (s->K < 1 || s->K > 1024) return EGAT_ERR_ARG;
+    } else if (s->graph_mode == EGAT_GRAPH_CSR) {
+      if (s->n_edges < 0) return EGAT_ERR_ARG;
+    } else {
+      return EGAT_ERR_ARG;
+    }
+  }
+  return EGAT_OK;
+}
+
+size_t hp_bytes(const egat_shape& s) {
+  const size_t D = size_t(s.lmax + 1) * (s.lmax + 1);
+  return (size_t(s.n) * D * s.C * storage_bytes(s.dtype) + 255) & ~size_t(255);
+}
+
+}  // namespace
+
+extern "C" {
+
+int egat_version(void) { return EGAT_VERSION; }
+
+const char* egat_strerror(int code) {
+  switch (code) {
+    case EGAT_OK: return "success";
+    case EGAT_ERR_ARG: return "invalid argument (null pointer, size or alignment)";
+    case EGAT_ERR_UNSUPPORTED: return "shape outside the supported set";
+    case EGAT_ERR_CUDA: return "CUDA launch or runtime error";
+    case EGAT_ERR_WORKSPACE: return "workspace too small";
+    default: return "unknown egat status";
+  }
+}
+
+int egat_num_paths(int lmax) {
+  if (lmax < 0 || lmax > kMaxL) return 0;
+  return num_paths(lmax);
+}
+
+int egat_graph_workspace_bytes(int32_t n, size_t* bytes) {
+  if (!bytes || n < 0) return EGAT_ERR_ARG;
+  *bytes = graph_workspace_bytes(n);
+  return EGAT_OK;
+}
+
+int egat_build_graph(const int32_t* d_pos_q, int32_t n, int32_t cutoff_q, int32_t K, int32_t mode,
+                     int32_t* d_nbr_or_rowptr, int32_t* d_cnt_or_col, int64_t col_capacity,
+                     int32_t* d_order, int32_t* d_overflow, void* d_ws, size_t ws_bytes,
+                     void* stream) {
+  if (n < 0 || cutoff_q <= 0 || !d_overflow) return EGAT_ERR_ARG;
+  if (mode == EGAT_GRAPH_PADDED) {
+    if (K < 1 || K > 1024) return EGAT_ERR_ARG;
+  } else if (mode == EGAT_GRAPH_CSR) {
+    if (col_capacity < 0) return EGAT_ERR_ARG;
+  } else {
+    return EGAT_ERR_ARG;
+  }
+  // keys are (d^2 << ceil(log2 n)) | j in 64 bits
+  int shift = 1;
+  while ((int64_t(1) << shift) < int64_t(n)) ++shift;
+  const unsigned __int128 top = (unsigned __int128)((uint64_t)cutoff_q * (uint64_t)cutoff_q) << shift;
+  if (top >> 64) return EGAT_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (n == 0) {
+    if (mode == EGAT_GRAPH_CSR && d_nbr_or_rowptr &&
+        cudaMemsetAsync(d_nbr_or_rowptr, 0, sizeof(int32_t), st) != cudaSuccess)
+      return EGAT_ERR_CUDA;
+    return cudaMemsetAsync(d_overflow, 0, sizeof(int32_t), st) == cudaSuccess ? EGAT_OK
+                                                                              : EGAT_ERR_CUDA;
+  }
+  if (!d_pos_q || !d_nbr_or_rowptr || !d_ws) return EGAT_ERR_ARG;
+  if (!d_cnt_or_col && !(mode == EGAT_GRAPH_CSR && col_capacity == 0)) return EGAT_ERR_ARG;
+  if (!aligned4(d_pos_q) || !aligned4(d_nbr_or_rowptr) || !aligned4(d_overflow)) return EGAT_ERR_ARG;
+  if (!aligned16(d_ws)) return EGAT_ERR_ARG;
+  return build_graph(d_pos_q, n, cutoff_q, K, mode, d_nbr_or_rowptr, d_cnt_or_col, col_capacity,
+                     d_order, d_overflow, d_ws, ws_bytes, st);
+}
+
+int egat_eaas_couple(const egat_shape* s, const void* d_x, const float* d_pos, const float* d_w,
+                     void* d_y, void* stream) {
+  const int rc = check_shape(s, false);
+  if (rc != EGAT_OK) return rc;
+  if (s->n == 0) return EGAT_OK;
+  if (!d_x || !d_pos || !d_w || !d_y) return EGAT_ERR_ARG;
+  if (!aligned16(d_x) || !aligned16(d_y) || !aligned4(d_pos) || !aligned4(d_w)) return EGAT_ERR_ARG;
+  return launch_eaas_source(*s, d_x, d_pos, d_w, d_y, static_cast<cudaStream_t>(stream));
+}
+
+int egat_otf_attention(const egat_shape* s, const void* d_q, const void* d_k, const void* d_hp,
+                       const int32_t* d_nbr_or_rowptr, const int32_t* d_cnt_or_col,
+                       const int32_t* d_order, float* d_m, void* stream) {
+  const int rc = check_shape(s, true);
+  if (rc != EGAT_OK) return rc;
+  if (s->n == 0) return EGAT_OK;
+  if (!d_q || !d_k || !d_hp || !d_nbr_or_rowptr || !d_m) return EGAT_ERR_ARG;
+  if (s->graph_mode == EGAT_GRAPH_CSR && !d_cnt_or_col && s->n_edges > 0) return EGAT_ERR_ARG;
+  if (!aligned16(d_q) || !aligned16(d_k) || !aligned16(d_hp) || !aligned16(d_m)) return EGAT_ERR_ARG;
+  return launch_attention(*s, false, d_q, d_k, d_hp, d_nbr_or_rowptr, d_cnt_or_col, d_order,
+                          nullptr, nullptr, d_m, static_cast<cudaStream_t>(stream));
+}
+
+int egat_otf_attention_coupled(const egat_shape* s, const void* d_q, const void* d_k,
+                               const void* d_hp, const int32_t* d_nbr_or_rowptr,
+                               const int32_t* d_cnt_or_col, const int32_t* d_order,
+                               const float* d_pos, const float* d_w2, float* d_out, void* stream) {
+  const int rc = check_shape(s, true);
+  if (rc != EGAT_OK) return rc;
+  if (s->n == 0) return EGAT_OK;
+  if (!d_q || !d_k || !d_hp || !d_nbr_or_rowptr || !d_pos || !d_w2 || !d_out) return EGAT_ERR_ARG;
+  if (s->graph_mode == EGAT_GRAPH_CSR && !d_cnt_or_col && s->n_edges > 0) return EGAT_ERR_ARG;
+  if (!aligned16(d_q) || !aligned16(d_k) || !aligned16(d_hp) || !aligned16(d_out) ||
+      !aligned4(d_pos) || !aligned4(d_w2))
+    return EGAT_ERR_ARG;
+  return launch_attention(*s, true, d_q, d_k, d_hp, d_nbr_or_rowptr, d_cnt_or_col, d_order, d_pos,
+                          d_w2, d_out, static_cast<cudaStream_t>(stream));
+}
+
+int egat_forward_workspace_bytes(const egat_shape* s, size_t* bytes) {
+  if (!bytes) return EGAT_ERR_ARG;
+  const int rc = check_shape(s, true);
+  if (rc != EGAT_OK) return rc;
+  *bytes = hp_bytes(*s);
+  return EGAT_OK;
+}
+
+int egat_forward(const egat_shape* s, const void* d_h, const float* d_pos, const void* d_q,
+                 const void* d_k, const int32_t* d_nbr_or_rowptr, const int32_t* d_cnt_or_col,
+                 const int32_t* d_order, const float* d_w1, const float* d_w2, void* d_ws,
+                 size_t ws_bytes, float* d_out, void* stream) {
+  const int rc = check_shape(s, true);
+  if (rc != EGAT_OK) return rc;
+  if (s->n == 0) return EGAT_OK;
+  if (!d_h || !d_pos || !d_q || !d_k || !d_nbr_or_rowptr || !d_w1 || !d_w2 || !d_ws || !d_out)
+    return EGAT_ERR_ARG;
+  if (s->graph_mode == EGAT_GRAPH_CSR && !d_cnt_or_col && s->n_edges > 0) return EGAT_ERR_ARG;
+  if (!aligned16(d_h) || !aligned16(d_q) || !aligned16(d_k) || !aligned16(d_ws) ||
+      !aligned16(d_out) || !aligned4(d_pos) || !aligned4(d_w1) || !aligned4(d_w2))
+    return EGAT_ERR_ARG;
+  if (ws_bytes < hp_bytes(*s)) return EGAT_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int e = launch_eaas_source(*s, d_h, d_pos, d_w1, d_ws, st);
+  if (e != EGAT_OK) return e;
+  return launch_attention(*s, true, d_q, d_k, d_ws, d_nbr_or_rowptr, d_cnt_or_col, d_order, d_pos,
+                          d_w2, d_out, st);
+}
+
+}  // extern "C"

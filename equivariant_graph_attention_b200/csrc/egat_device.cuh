@@ -1,0 +1,298 @@
+// Device-side building blocks shared by the egat kernels: storage loads,
+// compile-time coupling-path enumeration, real Wigner-D matrices and the
+// per-channel EAAS operator.
+//
+// Pages cited (by title):
+//  [EX] "E2Former-V2：突破等变图神经网络计算瓶颈的创新架构"
+//  [TS] "E2Former-V2: On-the-Fly Equivariant Attention with Linear Activation Memory"
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <type_traits>
+
+namespace egat {
+
+constexpr int kMaxL = 3;
+constexpr int kMaxPaths = 34;
+constexpr int kMaxDim = (kMaxL + 1) * (kMaxL + 1);
+
+// ---------------------------------------------------------------------------
+// compile-time helpers
+// ---------------------------------------------------------------------------
+template <int I, int N, typename F>
+__device__ __forceinline__ void static_for(F&& f) {
+  if constexpr (I < N) {
+    f(std::integral_constant<int, I>{});
+    static_for<I + 1, N>(f);
+  }
+}
+
+__host__ __device__ constexpr int iabs(int x) { return x < 0 ? -x : x; }
+
+// Coupling paths (li, lf, lo): every triple <= L with |li-lf| <= lo <= li+lf,
+// ordered by lo, then li, then lf ascending ([EX] §2.2 keeps both parities of
+// li+lf+lo).  which: 0 -> li, 1 -> lf, 2 -> lo; p == -1 counts the paths.
+__host__ __device__ constexpr int path_info(int L, int p, int which) {
+  int n = 0;
+  for (int lo = 0; lo <= L; ++lo)
+    for (int li = 0; li <= L; ++li)
+      for (int lf = 0; lf <= L; ++lf)
+        if (iabs(li - lf) <= lo && lo <= li + lf) {
+          if (n == p) return which == 0 ? li : (which == 1 ? lf : lo);
+          ++n;
+        }
+  return p < 0 ? n : -1;
+}
+__host__ __device__ constexpr int num_paths(int L) { return path_info(L, -1, 0); }
+
+// Offset of D^l inside the concatenated Wigner-D block (D^0, D^1, ...).
+__host__ __device__ constexpr int wig_off(int l) {
+  int o = 0;
+  for (int k = 0; k < l; ++k) o += (2 * k + 1) * (2 * k + 1);
+  return o;
+}
+__host__ __device__ constexpr int wig_size(int L) { return wig_off(L + 1); }
+
+// Axis-frame re-index factors: for path p and output m_o, the factor that
+// multiplies the rotated input component.  Filled on the host from
+// Clebsch–Gordan coefficients; which input component it reads is fixed at
+// compile time by the parity of li+lf+lo ([EX] §2.2; [TS] Eq. 13).
+struct EaasTable {
+  float f[kMaxPaths][2 * kMaxL + 1];
+};
+
+// ---------------------------------------------------------------------------
+// storage loads / stores
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&o)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    o[2 * i] = __uint_as_float(w[i] << 16);
+    o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// 8 consecutive elements starting at an element offset that is a multiple of 8.
+template <typename T>
+struct Chunk8;
+
+template <>
+struct Chunk8<__nv_bfloat16> {
+  uint4 v;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) {
+    v = __ldg(reinterpret_cast<const uint4*>(p));
+  }
+  __device__ __forceinline__ void zero() { v = make_uint4(0, 0, 0, 0); }
+  __device__ __forceinline__ void to_f32(float (&o)[8]) const { bf16x8_to_f32(v, o); }
+};
+
+template <>
+struct Chunk8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* p) {
+    a = __ldg(reinterpret_cast<const float4*>(p));
+    b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  }
+  __device__ __forceinline__ void zero() {
+    a = make_float4(0.f, 0.f, 0.f, 0.f);
+    b = a;
+  }
+  __device__ __forceinline__ void to_f32(float (&o)[8]) const {
+    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+    o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+  }
+};
+
+template <typename T>
+__device__ __forceinline__ float load_one(const T* p);
+template <>
+__device__ __forceinline__ float load_one<float>(const float* p) { return __ldg(p); }
+template <>
+__device__ __forceinline__ float load_one<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat162float(__ldg(p));
+}
+
+template <typename T>
+__device__ __forceinline__ void store_one(T* p, float v);
+template <>
+__device__ __forceinline__ void store_one<float>(float* p, float v) { *p = v; }
+template <>
+__device__ __forceinline__ void store_one<__nv_bfloat16>(__nv_bfloat16* p, float v) {
+  *p = __float2bfloat16_rn(v);
+}
+
+// 2^x on the special-function unit (PTX ex2.approx).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// ---------------------------------------------------------------------------
+// alignment rotation and real Wigner-D matrices
+// ---------------------------------------------------------------------------
+// Q = R_z(phi) R_y(theta), (theta, phi) the polar angles of r, so Q z = r/|r|
+// ([EX] §2.1 "compute_alignment_rotation"); identity for r = 0.  Written with
+// cos/sin of the angles taken directly from the coordinates.  Also returns
+// |r|.  Row-major Q[3][3].
+__device__ __forceinline__ float alignment_rotation(float x, float y, float z, float (&Q)[9]) {
+  const float rho2 = x * x + y * y;
+  const float r = sqrtf(rho2 + z * z);
+  if (r == 0.f) {
+    Q[0] = 1.f; Q[1] = 0.f; Q[2] = 0.f;
+    Q[3] = 0.f; Q[4] = 1.f; Q[5] = 0.f;
+    Q[6] = 0.f; Q[7] = 0.f; Q[8] = 1.f;
+    return 0.f;
+  }
+  const float rho = sqrtf(rho2);
+  const float ct = z / r, st = rho / r;
+  float cp = 1.f, sp = 0.f;
+  if (rho > 0.f) {
+    cp = x / rho;
+    sp = y / rho;
+  }
+  Q[0] = cp * ct; Q[1] = -sp; Q[2] = cp * st;
+  Q[3] = sp * ct; Q[4] = cp;  Q[5] = sp * st;
+  Q[6] = -st;     Q[7] = 0.f; Q[8] = ct;
+  return r;
+}
+
+// Degree-1 real Wigner-D: the rotation in (y, z, x) component order.
+__device__ __forceinline__ float wig1_from_Q(const float (&Q)[9], int e) {
+  const int perm[3] = {1, 2, 0};
+  const int a = e / 3, b = e % 3;
+  return Q[perm[a] * 3 + perm[b]];
+}
+
+// One entry D^l[m][mp] (m, mp in -l..l) of the real Wigner-D matrix of degree
+// l >= 2, from D^1 and D^{l-1} by the recursion of Ivanic and Ruedenberg
+// ("Rotation matrices for real spherical harmonics. Direct determination by
+// recursion", J. Phys. Chem. 100 (1996) 6342; erratum 102 (1998) 9099).
+// D1 and Dp are row-major with rows/cols indexed m + 1 and m + l - 1.
+__device__ __forceinline__ float ir_entry(int l, int m, int mp, const float* D1,
+                                          const float* Dp) {
+  const int wp = 2 * l - 1;  // width of D^{l-1}
+  auto r1 = [&](int i, int j) { return D1[(i + 1) * 3 + (j + 1)]; };
+  auto rp = [&](int a, int b) { return Dp[(a + l - 1) * wp + (b + l - 1)]; };
+  auto P = [&](int i, int a, int b) -> float {
+    if (b == l) return r1(i, 1) * rp(a, l - 1) - r1(i, -1) * rp(a, -l + 1);
+    if (b == -l) return r1(i, 1) * rp(a, -l + 1) + r1(i, -1) * rp(a, l - 1);
+    return r1(i, 0) * rp(a, b);
+  };
+  const float d = (iabs(mp) == l) ? float((2 * l) * (2 * l - 1)) : float((l + mp) * (l - mp));
+  const int am = iabs(m);
+  const bool m0 = (m == 0);
+  float val = 0.f;
+  // u-term
+  if (am < l) val += sqrtf(float((l + m) * (l - m)) / d) * P(0, m, mp);
+  // v-term
+  {
+    const float v = 0.5f * sqrtf(float((m0 ? 2 : 1) * (l + am - 1) * (l + am)) / d) * (m0 ? -1.f : 1.f);
+    float V;
+    if (m0) {
+      V = P(1, 1, mp) + P(-1, -1, mp);
+    } else if (m > 0) {
+      V = P(1, m - 1, mp) * (m == 1 ? 1.41421356237309515f : 1.f) -
+          (m == 1 ? 0.f : P(-1, -m + 1, mp));
+    } else {
+      V = (m == -1 ? 0.f : P(1, m + 1, mp)) +
+          P(-1, -m - 1, mp) * (m == -1 ? 1.41421356237309515f : 1.f);
+    }
+    val += v * V;
+  }
+  // w-term (vanishes for m = 0 and |m| >= l-1)
+  if (!m0 && am < l - 1) {
+    const float w = -0.5f * sqrtf(float((l - am - 1) * (l - am)) / d);
+    const float W = (m > 0) ? (P(1, m + 1, mp) + P(-1, -m - 1, mp))
+                            : (P(1, m - 1, mp) - P(-1, -m + 1, mp));
+    val += w * W;
+  }
+  return val;
+}
+
+// Build D^0..D^L for one rotation into Dsm (wig_size(L) floats) using
+// `nthreads` cooperating threads (thread index `tid`); `sync` is called
+// between degrees.  Dsm must be visible to all cooperating threads.
+template <int L, typename Sync>
+__device__ __forceinline__ void wigner_build(const float (&Q)[9], float* Dsm, int tid,
+                                             int nthreads, Sync sync) {
+  if (tid == 0) Dsm[0] = 1.f;
+  for (int e = tid; e < 9; e += nthreads) Dsm[wig_off(1) + e] = wig1_from_Q(Q, e);
+  sync();
+#pragma unroll
+  for (int l = 2; l <= L; ++l) {
+    const int w = 2 * l + 1;
+    for (int e = tid; e < w * w; e += nthreads) {
+      const int m = e / w - l, mp = e % w - l;
+      Dsm[wig_off(l) + e] = ir_entry(l, m, mp, Dsm + wig_off(1), Dsm + wig_off(l - 1));
+    }
+    sync();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// EAAS on one channel ([EX] §2.3, Proposition 4.3)
+// ---------------------------------------------------------------------------
+// y = sum_p w_p (x^{li} (x) R^{lf}(r))^{lo}, computed as
+//   xt^l = D^l(Q)^T x^l                       (into the frame with z along r)
+//   t^{lo}_m += w_p |r|^{lf} f_p(m) xt^{li}_{m or -m}   (only m_f = 0 survives)
+//   y^l = D^l(Q) t^l                          (back to the global frame)
+// `wgt(p)` returns w[p] for this channel; Dsm holds D^0..D^L.
+template <int L, typename WFn>
+__device__ __forceinline__ void eaas_channel(const float (&x)[(L + 1) * (L + 1)],
+                                             float (&y)[(L + 1) * (L + 1)],
+                                             const float* __restrict__ Dsm,
+                                             const float (&rpow)[L + 1], const EaasTable& tab,
+                                             WFn wgt) {
+  constexpr int D = (L + 1) * (L + 1);
+  float xt[D];
+  float t[D];
+#pragma unroll
+  for (int i = 0; i < D; ++i) t[i] = 0.f;
+  xt[0] = x[0];
+  static_for<1, L + 1>([&](auto lc) {
+    constexpr int l = decltype(lc)::value;
+    constexpr int w = 2 * l + 1;
+    const float* Dl = Dsm + wig_off(l);
+#pragma unroll
+    for (int a = 0; a < w; ++a) {
+      float s = 0.f;
+#pragma unroll
+      for (int b = 0; b < w; ++b) s = fmaf(Dl[b * w + a], x[l * l + b], s);
+      xt[l * l + a] = s;
+    }
+  });
+  static_for<0, num_paths(L)>([&](auto pc) {
+    constexpr int p = decltype(pc)::value;
+    constexpr int li = path_info(L, p, 0);
+    constexpr int lf = path_info(L, p, 1);
+    constexpr int lo = path_info(L, p, 2);
+    constexpr bool even = ((li + lf + lo) % 2) == 0;
+    const float wp = wgt(p) * rpow[lf];
+#pragma unroll
+    for (int mo = -lo; mo <= lo; ++mo) {
+      const int src = even ? mo : -mo;
+      const bool live = (iabs(mo) <= li) && (even || mo != 0);
+      if (live) t[lo * lo + lo + mo] = fmaf(wp * tab.f[p][mo + lo], xt[li * li + li + src],
+                                            t[lo * lo + lo + mo]);
+    }
+  });
+  y[0] = t[0];
+  static_for<1, L + 1>([&](auto lc) {
+    constexpr int l = decltype(lc)::value;
+    constexpr int w = 2 * l + 1;
+    const float* Dl = Dsm + wig_off(l);
+#pragma unroll
+    for (int a = 0; a < w; ++a) {
+      float s = 0.f;
+#pragma unroll
+      for (int b = 0; b < w; ++b) s = fmaf(Dl[a * w + b], t[l * l + b], s);
+      y[l * l + a] = s;
+    }
+  });
+}
+
+}  // namespace egat

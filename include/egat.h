@@ -1,0 +1,199 @@
+/*
+ * egat — equivariant graph attention hot path for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of the library libegat.so.  Every entry point takes plain pointers and
+ * sizes; "d_" pointers are CUDA device pointers, everything else is host
+ * memory.  The caller allocates every buffer (inputs, outputs and scratch
+ * "workspace", sized by the *_workspace_bytes queries); the library allocates
+ * no memory of its own.  All work is enqueued asynchronously on the given
+ * stream (a cudaStream_t passed as void*, NULL = legacy default stream); no
+ * call synchronises the device.  Calls report errors by return code and never
+ * abort, trap or print.
+ *
+ * Pages cited (by title):
+ *  [EX] "E2Former-V2：突破等变图神经网络计算瓶颈的创新架构" (explainer)
+ *  [TS] "E2Former-V2: On-the-Fly Equivariant Attention with Linear Activation
+ *       Memory" (technical summary)
+ *
+ * The four steps ([EX] §3.1 node-centric factorisation, [EX] §2 EAAS):
+ *  1. egat_build_graph    radius graph from positions (cell list);
+ *  2. egat_eaas_couple    h'_j = h_j (x) R(r_j) by EAAS;
+ *  3. egat_otf_attention  m_i = sum_j softmax_j(q_i.k_j/sqrt(dk)) h'_j, streamed;
+ *  4. egat_otf_attention_coupled  3 with the target coupling ^h_i = m_i (x) R(r_i)
+ *                         fused into the attention epilogue;
+ *     egat_forward        2 then 3+4.
+ *
+ * Conventions shared by all calls
+ *  - Irrep features are row-major [n][D][C], D = (lmax+1)^2, component index
+ *    l*l + l + m (m = -l..l), channel fastest.  Real spherical-harmonic basis
+ *    (Condon–Shortley phase cancelled), degree 1 ordered (y, z, x).
+ *  - R^l(r) are Racah-normalised solid harmonics of the position vector r as
+ *    given (callers centre positions on the system centroid).
+ *  - Coupling paths (li, lf, lo) are all triples <= lmax with
+ *    |li-lf| <= lo <= li+lf (odd li+lf+lo included), ordered by lo, then li,
+ *    then lf ascending; egat_num_paths(lmax) of them (5, 15, 34 for lmax 1-3).
+ *    Weights are float32 [P][C]: w[p][c] scales path p of channel c.
+ *  - Channel c belongs to head floor(c*H/C); logits are per head.
+ *  - Positions for the graph are int32 grid coordinates [n][3]; the float32
+ *    positions used for geometry [n][3] must equal them times the grid step
+ *    the caller chose (2^-16 Å in this project's inputs).
+ *  - Supported shapes: 1 <= lmax <= 3; C in {16, 32, 64, 128}; H a power of
+ *    two with C/H a multiple of 8; dk in {8, 16, 32} with H*dk <= 256;
+ *    1 <= K <= 1024.  Feature pointers must be 16-byte aligned.
+ */
+#ifndef EGAT_H
+#define EGAT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define EGAT_VERSION 1
+
+#if defined(__GNUC__)
+#define EGAT_API __attribute__((visibility("default")))
+#else
+#define EGAT_API
+#endif
+
+/* return codes: 0 success, negative errors */
+enum {
+  EGAT_OK = 0,
+  EGAT_ERR_ARG = -1,          /* null pointer, bad size or misaligned pointer */
+  EGAT_ERR_UNSUPPORTED = -2,  /* shape outside the supported set above */
+  EGAT_ERR_CUDA = -3,         /* a CUDA launch or runtime call failed */
+  EGAT_ERR_WORKSPACE = -4     /* workspace smaller than the query returned */
+};
+
+/* storage type of h, q, k and h' (accumulation and outputs are float32) */
+enum { EGAT_F32 = 0, EGAT_BF16 = 1 };
+
+/* neighbour-list format */
+enum {
+  EGAT_GRAPH_PADDED = 0,  /* nbr int32 [n][K] (unused slots -1) + cnt int32 [n] */
+  EGAT_GRAPH_CSR = 1      /* rowptr int32 [n+1] + col int32 [n_edges] */
+};
+
+typedef struct egat_shape {
+  int32_t n;           /* atoms */
+  int32_t lmax;        /* highest irrep degree, 1..3 */
+  int32_t C;           /* channels per degree */
+  int32_t H;           /* attention heads */
+  int32_t dk;          /* query/key width per head */
+  int32_t K;           /* padded neighbour slots (PADDED) */
+  int32_t dtype;       /* EGAT_F32 or EGAT_BF16 */
+  int32_t graph_mode;  /* EGAT_GRAPH_PADDED or EGAT_GRAPH_CSR */
+  int64_t n_edges;     /* CSR: length of col (row ranges are clamped to it) */
+} egat_shape;
+
+/* Library version (EGAT_VERSION). */
+EGAT_API int egat_version(void);
+
+/* Static description of a return code. */
+EGAT_API const char* egat_strerror(int code);
+
+/* Number of coupling paths P for lmax (0 if lmax is out of range). */
+EGAT_API int egat_num_paths(int lmax);
+
+/*
+ * Step 1 — radius graph ([EX] §5.1 edge_cutoff, §5.2 neighbour-list check).
+ * Atom j != i is a neighbour of i when |p_j - p_i|^2 <= cutoff_q^2, computed
+ * exactly in 64-bit integers on grid coordinates (inclusive cutoff).  Cells
+ * of edge cutoff_q are hashed to a power-of-two table by a Morton code of the
+ * cell coordinates, so memory depends only on n, not on the box.
+ *
+ *  d_pos_q       int32 [n][3] grid coordinates
+ *  cutoff_q      cutoff in grid units, > 0
+ *  mode          EGAT_GRAPH_PADDED:
+ *                  d_nbr_or_rowptr = nbr int32 [n][K]: the K nearest
+ *                  neighbours ordered by (squared distance, index), then -1;
+ *                  d_cnt_or_col = cnt int32 [n] = min(degree, K);
+ *                  *d_overflow = number of neighbours dropped by the
+ *                  truncation (ties at the K-th distance keep smaller j).
+ *                EGAT_GRAPH_CSR:
+ *                  d_nbr_or_rowptr = rowptr int32 [n+1];
+ *                  d_cnt_or_col = col int32 [col_capacity]; each row ordered
+ *                  by (squared distance, index) when its degree is <= 1024,
+ *                  otherwise in unspecified order; entries past col_capacity
+ *                  are not written and *d_overflow = their number.
+ *  d_order       optional int32 [n]: atoms listed cell by cell (Morton
+ *                order of cells) — a traversal order with spatial locality
+ *                for egat_otf_attention / egat_forward.  May be NULL.
+ *  d_overflow    int32 [1], zeroed and then set by this call.
+ *  d_ws, ws_bytes  scratch of at least egat_graph_workspace_bytes(n).
+ * Returns EGAT_ERR_UNSUPPORTED when cutoff_q^2 * 2^ceil(log2 n) >= 2^64.
+ */
+EGAT_API int egat_graph_workspace_bytes(int32_t n, size_t* bytes);
+EGAT_API int egat_build_graph(const int32_t* d_pos_q, int32_t n, int32_t cutoff_q, int32_t K,
+                     int32_t mode, int32_t* d_nbr_or_rowptr, int32_t* d_cnt_or_col,
+                     int64_t col_capacity, int32_t* d_order, int32_t* d_overflow,
+                     void* d_ws, size_t ws_bytes, void* stream);
+
+/*
+ * Step 2 — EAAS coupling ([EX] §2.1-§2.3, Proposition 4.3; [TS] §2.1, Lemma
+ * 4.1, Eq. 13):
+ *   y_j^{lo} = sum_{p=(li,lf,lo)} w[p][c] (x_j^{li} (x) R^{lf}(r_j))^{lo}
+ * evaluated by rotating x_j into the frame whose z axis is r_j (real Wigner-D
+ * matrices by the Ivanic–Ruedenberg recursion), keeping only m_i = m_o (even
+ * li+lf+lo) or m_i = -m_o with sign sgn(m_o) (odd) times the Clebsch–Gordan
+ * factor <li |m|; lf 0 | lo |m|> |r_j|^lf, and rotating back.
+ *  d_x     [n][D][C] in s->dtype        d_pos  float32 [n][3]
+ *  d_w     float32 [P][C]               d_y    [n][D][C] in s->dtype
+ *                                              (bf16: round to nearest even)
+ */
+EGAT_API int egat_eaas_couple(const egat_shape* s, const void* d_x, const float* d_pos,
+                     const float* d_w, void* d_y, void* stream);
+
+/*
+ * Step 3 — on-the-fly attention ([EX] §3.2; [TS] §2.2):
+ *   s_ij^h = q_i^h . k_j^h / sqrt(dk),  alpha = softmax over j in N(i),
+ *   m_i^{l}[m][c] = sum_j alpha_ij^{head(c)} h'_j^{l}[m][c]
+ * streamed with an online softmax (running max and normaliser per head); each
+ * neighbour's key and value rows are read once and nothing of size n*K is
+ * written.  An atom without neighbours gets m_i = 0.  Neighbour entries that
+ * are negative or >= n are skipped.
+ *  d_q, d_k  [n][H][dk] in s->dtype      d_hp  [n][D][C] in s->dtype
+ *  graph     as produced by egat_build_graph in s->graph_mode
+ *            (PADDED: d_cnt may be NULL, then all K slots are scanned)
+ *  d_order   optional int32 [n] traversal order (a permutation); NULL = 0..n-1
+ *  d_m       float32 [n][D][C]
+ */
+EGAT_API int egat_otf_attention(const egat_shape* s, const void* d_q, const void* d_k,
+                       const void* d_hp, const int32_t* d_nbr_or_rowptr,
+                       const int32_t* d_cnt_or_col, const int32_t* d_order, float* d_m,
+                       void* stream);
+
+/*
+ * Steps 3+4 fused — on-the-fly attention whose epilogue applies the target
+ * coupling ^h_i = EAAS(m_i, r_i, w2) ([EX] §3.1 step 3) to the on-chip m_i
+ * (m_i never reaches memory).  Arguments as egat_otf_attention, plus
+ *  d_pos   float32 [n][3]      d_w2  float32 [P][C]
+ *  d_out   float32 [n][D][C]   ^h
+ */
+EGAT_API int egat_otf_attention_coupled(const egat_shape* s, const void* d_q, const void* d_k,
+                                        const void* d_hp, const int32_t* d_nbr_or_rowptr,
+                                        const int32_t* d_cnt_or_col, const int32_t* d_order,
+                                        const float* d_pos, const float* d_w2, float* d_out,
+                                        void* stream);
+
+/*
+ * Steps 2-4 — the fused forward pass ([EX] §3.1):
+ *   h' = EAAS(h, r, w1) into workspace;  then one kernel per target streams
+ *   its neighbours (step 3) and applies ^h_i = EAAS(m_i, r_i, w2) to the
+ *   on-chip m_i before writing ^h_i.
+ *  d_out  float32 [n][D][C];  d_ws at least egat_forward_workspace_bytes(s).
+ */
+EGAT_API int egat_forward_workspace_bytes(const egat_shape* s, size_t* bytes);
+EGAT_API int egat_forward(const egat_shape* s, const void* d_h, const float* d_pos, const void* d_q,
+                 const void* d_k, const int32_t* d_nbr_or_rowptr, const int32_t* d_cnt_or_col,
+                 const int32_t* d_order, const float* d_w1, const float* d_w2, void* d_ws,
+                 size_t ws_bytes, float* d_out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EGAT_H */

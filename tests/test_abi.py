@@ -1,0 +1,98 @@
+"""The C-ABI library on the CPU: it loads, exports every symbol the header
+declares, and rejects bad arguments on the host before touching a device.
+
+No call here reaches CUDA: each either is host-only (version, path count,
+workspace queries, status strings) or fails argument validation first.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from equivariant_graph_attention_b200 import egat
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from equivariant_graph_attention_b200.build import build
+    build()
+    return egat.load_library()
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "egat.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"EGAT_API\s+[\w\s\*]+?\b(egat_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert names == sorted(egat.EXPORTS)
+    for n in names:
+        assert hasattr(lib, n), n
+    # nothing else is exported: the internal C++ symbols are hidden
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", egat._LIB_PATH], capture_output=True,
+                         text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert {n for n in exported if n.startswith("egat_")} == set(names)
+
+
+def test_host_only_queries(lib):
+    assert egat.egat_version() == 1
+    assert [egat.egat_num_paths(l) for l in range(5)] == [1, 5, 15, 34, 0]
+    assert lib.egat_strerror(0) == b"success"
+    assert b"workspace" in lib.egat_strerror(egat.EGAT_ERR_WORKSPACE)
+    assert egat.egat_graph_workspace_bytes(1000) > 0
+    s = egat.Shape(n=32768, lmax=2, C=128, H=16, dk=16, K=256, dtype="bf16")
+    assert egat.egat_forward_workspace_bytes(s) == 32768 * 9 * 128 * 2
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("lmax", 4, egat.EGAT_ERR_UNSUPPORTED), ("lmax", 0, egat.EGAT_ERR_UNSUPPORTED),
+    ("C", 96, egat.EGAT_ERR_UNSUPPORTED), ("H", 3, egat.EGAT_ERR_UNSUPPORTED),
+    ("dk", 12, egat.EGAT_ERR_UNSUPPORTED), ("K", 0, egat.EGAT_ERR_ARG),
+    ("K", 2000, egat.EGAT_ERR_ARG), ("n", -1, egat.EGAT_ERR_ARG), ("dtype", "f16", None)])
+def test_shape_validation(lib, field, value, code):
+    base = dict(n=10, lmax=2, C=128, H=16, dk=16, K=64, dtype="f32")
+    base[field] = value
+    if value == "f16":
+        cs = egat.egat_shape(10, 2, 128, 16, 16, 64, 7, 0, 0)
+        code = egat.EGAT_ERR_ARG
+    else:
+        cs = egat.Shape(**base).c()
+    out = ctypes.c_size_t(0)
+    assert lib.egat_forward_workspace_bytes(ctypes.byref(cs), ctypes.byref(out)) == code
+    fake = ctypes.c_void_p(0x10000)
+    rc = lib.egat_forward(ctypes.byref(cs), fake, fake, fake, fake, fake, fake, None, fake, fake,
+                          fake, 1 << 30, fake, None)
+    assert rc == code
+
+
+def test_pointer_and_size_validation(lib):
+    cs = egat.Shape(n=10, lmax=2, C=128, H=16, dk=16, K=64, dtype="bf16").c()
+    ok = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)     # not 16-byte aligned
+    args = [ok, ok, ok, ok, ok, ok, None, ok, ok, ok, 1 << 30, ok, None]
+    for slot in (0, 2, 3, 9, 11):      # h, q, k, workspace, out
+        a = list(args)
+        a[slot] = odd
+        assert lib.egat_forward(ctypes.byref(cs), *a) == egat.EGAT_ERR_ARG
+        b = list(args)
+        b[slot] = None
+        assert lib.egat_forward(ctypes.byref(cs), *b) == egat.EGAT_ERR_ARG
+    small = list(args)
+    small[10] = 100
+    assert lib.egat_forward(ctypes.byref(cs), *small) == egat.EGAT_ERR_WORKSPACE
+    assert lib.egat_forward(None, *args) == egat.EGAT_ERR_ARG
+    # graph builder: bad cutoff, bad K, bad mode, missing overflow, key overflow
+    g = lambda n, cut, K, mode, ovf: lib.egat_build_graph(ok, n, cut, K, mode, ok, ok, 0, None,
+                                                          ovf, ok, 1 << 30, None)
+    assert g(10, 0, 8, 0, ok) == egat.EGAT_ERR_ARG
+    assert g(10, 100, 0, 0, ok) == egat.EGAT_ERR_ARG
+    assert g(10, 100, 8, 5, ok) == egat.EGAT_ERR_ARG
+    assert g(10, 100, 8, 0, None) == egat.EGAT_ERR_ARG
+    assert g(1 << 30, 2 ** 31 - 1, 8, 0, ok) == egat.EGAT_ERR_UNSUPPORTED

@@ -1,0 +1,292 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Pages: [EX] "E2Former-V2：突破等变图神经网络计算瓶颈的创新架构" §2-§3, §5;
+[TS] "E2Former-V2: On-the-Fly Equivariant Attention with Linear Activation
+Memory" §2.
+
+* Neighbour lists must match the oracle's brute force bit for bit (rows are
+  ordered by (squared distance, index) on both sides, so rows compare as-is).
+* Floating-point outputs must match within the per-(atom, degree) relative
+  error bar of ``parity_util`` (1e-4 float32 storage, 2e-2 bf16 storage).
+* Small workloads are compared on every atom; the 32,768- and 100,000-atom
+  workloads on a sample of targets that includes the truncated rows, in the
+  same launch configuration the benchmark times (graph -> fused forward with
+  the cell traversal order).
+"""
+import functools
+
+import numpy as np
+import pytest
+import torch
+from scipy.spatial import cKDTree
+
+from oracle.attention import aggregate, forward as oracle_forward, source_coupling
+from oracle.graph import radius_graph
+from equivariant_graph_attention_b200 import synth
+from tests.parity_util import TOL, block_rel_error, device_inputs, sample_targets, shape_of
+
+pytestmark = pytest.mark.gpu
+
+SMALL = ["uniform64_l1_f32", "water216_l2_f32", "uniform4096_l2_bf16"]
+LARGE = ["uniform32768_K256_l2_bf16", "uniform100000_l3_bf16"]
+
+
+@functools.lru_cache(maxsize=None)
+def _data(name):
+    wl = synth.WORKLOADS[name]
+    return wl, synth.make(wl)
+
+
+@functools.lru_cache(maxsize=None)
+def _full_degree(name):
+    wl, d = _data(name)
+    tree = cKDTree(d["pos_q"].astype(np.float64))
+    return np.array([len(x) - 1 for x in tree.query_ball_point(d["pos_q"].astype(np.float64),
+                                                               wl.cutoff_q)])
+
+
+def _egat():
+    from equivariant_graph_attention_b200 import egat
+    return egat
+
+
+# --------------------------------------------------------------------------- graph
+@pytest.mark.parametrize("name", SMALL)
+def test_graph_padded_bit_exact(name):
+    egat = _egat()
+    wl, d = _data(name)
+    dev = device_inputs(wl, d)
+    g = egat.egat_build_graph(dev["pos_q"], wl.cutoff_q, K=wl.K)
+    nbr = g["nbr"].cpu().numpy()
+    cnt = g["cnt"].cpu().numpy()
+    lists, full = radius_graph(d["pos_q"], wl.cutoff_q, K=wl.K)
+    for i, ref in enumerate(lists):
+        assert cnt[i] == len(ref)
+        assert np.array_equal(nbr[i, :cnt[i]], ref), i
+        assert np.all(nbr[i, cnt[i]:] == -1)
+    assert int(g["overflow"].item()) == int(np.maximum(full - wl.K, 0).sum())
+    order = g["order"].cpu().numpy()
+    assert np.array_equal(np.sort(order), np.arange(wl.n))
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_graph_csr_bit_exact(name):
+    egat = _egat()
+    wl, d = _data(name)
+    dev = device_inputs(wl, d)
+    lists, full = radius_graph(d["pos_q"], wl.cutoff_q)
+    E = int(full.sum())
+    g = egat.egat_build_graph(dev["pos_q"], wl.cutoff_q, mode="csr", col_capacity=E)
+    rowptr = g["rowptr"].cpu().numpy()
+    col = g["col"].cpu().numpy()
+    assert rowptr[0] == 0 and rowptr[-1] == E
+    for i, ref in enumerate(lists):
+        assert np.array_equal(col[rowptr[i]:rowptr[i + 1]], ref), i
+    assert int(g["overflow"].item()) == 0
+    # a short column buffer reports exactly the entries it could not hold
+    g2 = egat.egat_build_graph(dev["pos_q"], wl.cutoff_q, mode="csr", col_capacity=E - 5)
+    assert int(g2["overflow"].item()) == 5
+    assert np.array_equal(g2["col"].cpu().numpy(), col[:E - 5])
+
+
+@pytest.mark.parametrize("name", LARGE)
+def test_graph_full_size_sampled_rows(name):
+    egat = _egat()
+    wl, d = _data(name)
+    dev = device_inputs(wl, d)
+    g = egat.egat_build_graph(dev["pos_q"], wl.cutoff_q, K=wl.K)
+    nbr = g["nbr"].cpu().numpy()
+    cnt = g["cnt"].cpu().numpy()
+    full = _full_degree(name)
+    assert np.array_equal(cnt, np.minimum(full, wl.K))
+    assert int(g["overflow"].item()) == int(np.maximum(full - wl.K, 0).sum())
+    rows = sample_targets(wl, full)
+    lists, _ = radius_graph(d["pos_q"], wl.cutoff_q, K=wl.K, rows=rows)
+    for i, ref in zip(rows, lists):
+        assert np.array_equal(nbr[i, :cnt[i]], ref), i
+
+
+# --------------------------------------------------------------------------- steps 2, 3
+@pytest.mark.parametrize("name", SMALL + LARGE)
+def test_eaas_couple_parity(name):
+    egat = _egat()
+    wl, d = _data(name)
+    dev = device_inputs(wl, d)
+    hp = egat.egat_eaas_couple(shape_of(wl), dev["h"], dev["pos"], dev["w1"])
+    rows = np.arange(wl.n) if wl.n <= 4096 else np.array(sample_targets(wl, _full_degree(name), 300))
+    ref = source_coupling(d["h"][rows], d["pos"][rows], d["w1"], wl.lmax)
+    got = hp[torch.from_numpy(rows).cuda()].float().cpu().numpy()
+    assert block_rel_error(got, ref, wl.lmax) < TOL[wl.dtype]
+
+
+@pytest.mark.parametrize("name", SMALL + LARGE)
+def test_otf_attention_parity(name):
+    """Step 3 alone, on a value array drawn directly (the same values on both sides)."""
+    egat = _egat()
+    wl, d = _data(name)
+    dev = device_inputs(wl, d)
+    rng = np.random.default_rng(8)
+    vals = rng.standard_normal((wl.n, wl.D, wl.C)).astype(np.float32)
+    if wl.dtype == "bf16":
+        vals = synth.round_bf16(vals)
+    hp = torch.from_numpy(vals).to("cuda", dtype=dev["h"].dtype)
+    g = egat.egat_build_graph(dev["pos_q"], wl.cutoff_q, K=wl.K)
+    m = egat.egat_otf_attention(shape_of(wl), dev["q"], dev["k"], hp, g["nbr"], g["cnt"],
+                                order=g["order"])
+    rows = list(range(wl.n)) if wl.n <= 4096 else sample_targets(wl, _full_degree(name))
+    lists, _ = radius_graph(d["pos_q"], wl.cutoff_q, K=wl.K, rows=rows)
+    ref = aggregate(d["q"], d["k"], vals, lists, rows)
+    got = m[torch.tensor(rows).cuda()].cpu().numpy()
+    # inputs identical on both sides: only float32 accumulation differs
+    assert block_rel_error(got, ref, wl.lmax) < 1e-4
+
+
+# --------------------------------------------------------------------------- fused forward
+def _forward_case(name, mode="padded", use_order=True):
+    egat = _egat()
+    wl, d = _data(name)
+    dev = device_inputs(wl, d)
+    if mode == "padded":
+        g = egat.egat_build_graph(dev["pos_q"], wl.cutoff_q, K=wl.K)
+        shape = shape_of(wl)
+        a, b = g["nbr"], g["cnt"]
+    else:
+        E = int(_full_degree(name).sum()) if wl.n > 4096 else int(
+            radius_graph(d["pos_q"], wl.cutoff_q)[1].sum())
+        g = egat.egat_build_graph(dev["pos_q"], wl.cutoff_q, mode="csr", col_capacity=E)
+        shape = shape_of(wl, mode="csr", n_edges=E)
+        a, b = g["rowptr"], g["col"]
+    out = egat.egat_forward(shape, dev["h"], dev["pos"], dev["q"], dev["k"], a, b,
+                            dev["w1"], dev["w2"], order=g["order"] if use_order else None)
+    torch.cuda.synchronize()
+    return wl, d, out
+
+
+@pytest.mark.parametrize("name", SMALL + LARGE)
+def test_forward_parity(name):
+    wl, d, out = _forward_case(name)
+    if wl.n <= 4096:
+        rows = list(range(wl.n))
+    else:
+        rows = sample_targets(wl, _full_degree(name))
+    K = wl.K
+    lists, _ = radius_graph(d["pos_q"], wl.cutoff_q, K=K, rows=rows)
+    ref = oracle_forward(d["h"], d["pos"], d["q"], d["k"], d["w1"], d["w2"], wl.lmax, lists,
+                         targets=rows)
+    got = out[torch.tensor(rows).cuda()].cpu().numpy()
+    err = block_rel_error(got, ref, wl.lmax)
+    assert err < TOL[wl.dtype], err
+
+
+@pytest.mark.parametrize("name", ["water216_l2_f32", "uniform4096_l2_bf16"])
+def test_forward_csr_matches_padded_without_truncation(name):
+    wl, d, out_p = _forward_case(name, "padded")
+    _, _, out_c = _forward_case(name, "csr")
+    full = radius_graph(d["pos_q"], wl.cutoff_q)[1]
+    keep = full <= wl.K     # rows the padded list did not truncate
+    assert np.array_equal(out_p.cpu().numpy()[keep], out_c.cpu().numpy()[keep])
+
+
+def test_forward_order_does_not_change_results():
+    _, _, a = _forward_case("uniform4096_l2_bf16", use_order=True)
+    _, _, b = _forward_case("uniform4096_l2_bf16", use_order=False)
+    assert torch.equal(a, b)
+
+
+# --------------------------------------------------------------------------- edge cases
+def _tiny_problem(pos_list, lmax=2, C=16, H=2, dk=8, K=8, dtype="f32", cutoff=3.0, seed=4):
+    wl = synth.small_cube(len(pos_list), 1.0, cutoff, K, lmax, C, H, dk, dtype)
+    feats = synth.features(wl, seed)
+    pq = np.rint(np.asarray(pos_list, dtype=np.float64) / synth.GRID_QUANTUM).astype(np.int32)
+    pf = (pq.astype(np.float64) * synth.GRID_QUANTUM).astype(np.float32)
+    feats.update(pos_q=pq, pos=pf)
+    return wl, feats
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("lmax", [1, 2, 3])
+def test_special_geometry_and_isolated_atoms(lmax, dtype):
+    """Atoms at the origin (r = 0), on the -z and +z axes, an isolated atom
+    (no neighbours -> exactly zero output), and a ragged count of atoms."""
+    egat = _egat()
+    pts = [[0, 0, 0], [0, 0, -1.2], [0, 0, 1.1], [0.7, -0.4, 0.2], [-0.5, 0.9, -0.8],
+           [40.0, 40.0, 40.0], [1.3, 0.2, -0.1]]
+    wl, d = _tiny_problem(pts, lmax=lmax, dtype=dtype)
+    dev = device_inputs(wl, d)
+    g = egat.egat_build_graph(dev["pos_q"], wl.cutoff_q, K=wl.K)
+    out = egat.egat_forward(shape_of(wl), dev["h"], dev["pos"], dev["q"], dev["k"], g["nbr"],
+                            g["cnt"], dev["w1"], dev["w2"], order=g["order"]).cpu().numpy()
+    lists, _ = radius_graph(d["pos_q"], wl.cutoff_q, K=wl.K)
+    assert len(lists[5]) == 0
+    ref = oracle_forward(d["h"], d["pos"], d["q"], d["k"], d["w1"], d["w2"], lmax, lists)
+    assert np.all(out[5] == 0.0)
+    assert block_rel_error(out, ref, lmax) < TOL[dtype]
+
+
+@pytest.mark.parametrize("n", [1, 5, 37, 301])
+def test_ragged_sizes_and_no_count_array(n):
+    """Sizes that leave partial warps/tiles; the padded list scanned without
+    the count array (slots marked -1 are skipped)."""
+    egat = _egat()
+    wl = synth.small_cube(n, max(3.0, (n / 0.1) ** (1 / 3)), 4.0, 32, 2, 32, 4, 8, "f32")
+    d = synth.make(wl, seed=n)
+    dev = device_inputs(wl, d)
+    g = egat.egat_build_graph(dev["pos_q"], wl.cutoff_q, K=wl.K)
+    shape = shape_of(wl)
+    out = egat.egat_forward(shape, dev["h"], dev["pos"], dev["q"], dev["k"], g["nbr"], None,
+                            dev["w1"], dev["w2"]).cpu().numpy()
+    lists, _ = radius_graph(d["pos_q"], wl.cutoff_q, K=wl.K)
+    ref = oracle_forward(d["h"], d["pos"], d["q"], d["k"], d["w1"], d["w2"], wl.lmax, lists)
+    assert block_rel_error(out, ref, wl.lmax) < 1e-4
+
+
+def test_golden_tiny_forward():
+    """The stored oracle output for the tiny seeded system (tests/golden)."""
+    import json
+    import os
+    from tests.golden.make_golden import SPEC
+    egat = _egat()
+    with open(os.path.join(os.path.dirname(__file__), "golden", "forward_tiny.json")) as f:
+        rec = json.load(f)
+    s = SPEC
+    wl = synth.small_cube(s["n"], s["side"], s["cutoff"], s["K"], s["lmax"], s["C"], s["H"],
+                          s["dk"], s["dtype"])
+    d = synth.make(wl, s["seed"])
+    dev = device_inputs(wl, d)
+    g = egat.egat_build_graph(dev["pos_q"], wl.cutoff_q, K=wl.K)
+    cnt = g["cnt"].cpu().numpy()
+    nbr = g["nbr"].cpu().numpy()
+    assert [nbr[i, :cnt[i]].tolist() for i in range(wl.n)] == rec["neighbours"]
+    out = egat.egat_forward(shape_of(wl), dev["h"], dev["pos"], dev["q"], dev["k"], g["nbr"],
+                            g["cnt"], dev["w1"], dev["w2"], order=g["order"]).cpu().numpy()
+    assert block_rel_error(out, np.array(rec["out"]), wl.lmax) < 1e-4
+
+
+def test_empty_input_is_a_noop():
+    egat = _egat()
+    wl = synth.small_cube(0, 1.0, 1.0, 4, 1, 16, 2, 8)
+    shape = shape_of(wl, n=0)
+    z = torch.zeros(16, device="cuda")
+    pos_q = torch.zeros((0, 3), dtype=torch.int32, device="cuda")
+    g = egat.egat_build_graph(pos_q, wl.cutoff_q, K=4)
+    assert int(g["overflow"].item()) == 0
+    out = egat.egat_forward(shape, z, z, z, z, z.int(), z.int(), z, z, workspace=torch.zeros(
+        256, dtype=torch.uint8, device="cuda"))
+    assert out.shape == (0, 4, 16)
+
+
+def test_error_codes_from_the_device_path():
+    egat = _egat()
+    wl, d = _data("uniform64_l1_f32")
+    dev = device_inputs(wl, d)
+    g = egat.egat_build_graph(dev["pos_q"], wl.cutoff_q, K=wl.K)
+    with pytest.raises(egat.EgatError) as e:
+        egat.egat_forward(shape_of(wl), dev["h"], dev["pos"], dev["q"], dev["k"], g["nbr"], g["cnt"],
+                          dev["w1"], dev["w2"], workspace=torch.zeros(256, dtype=torch.uint8,
+                                                                      device="cuda"))
+    assert e.value.code == egat.EGAT_ERR_WORKSPACE
+    with pytest.raises(egat.EgatError) as e:
+        egat.egat_forward(shape_of(wl), dev["h"].reshape(-1)[1:], dev["pos"], dev["q"], dev["k"],
+                          g["nbr"], g["cnt"], dev["w1"], dev["w2"])
+    assert e.value.code == egat.EGAT_ERR_ARG     # misaligned feature pointer
+    torch.cuda.synchronize()
