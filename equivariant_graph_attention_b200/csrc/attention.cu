@@ -17,9 +17,12 @@
 // normaliser.  The key row is H*dk elements: lane r < H*dk/8 loads chunk r,
 // multiplies it with its register-resident slice of q_i and the dk/8 lanes of
 // a head reduce by shuffles; every lane then fetches its own head's logit
-// with one shuffle.  Neighbour indices are read two slots ahead and rows one
-// slot ahead (register double buffering) so the gathers overlap the FMAs.
-// Nothing per edge is written.  The fused variant writes m_i / z to shared
+// with one shuffle.  Neighbour indices are read four slots ahead and rows one
+// slot ahead into two register buffers used in ping-pong, so the gathers
+// overlap the arithmetic.  Accumulation uses the packed f32x2 FMA (two
+// channels per instruction); the online-softmax reference maximum is raised
+// lazily (only when a logit exceeds it by 2^8), which keeps the rescale of
+// the accumulators off the per-edge path.  Nothing per edge is written.  The fused variant writes m_i / z to shared
 // memory, rebuilds the target's Wigner-D matrices in shared memory, and lets
 // each lane apply EAAS to its channels before writing ^h_i.
 #include <cfloat>
@@ -63,7 +66,6 @@ struct Frag {
     for (int t = 0; t < TPL; ++t) {
       const int q = lane + 32 * t;
       if (q < NCH) hc[t].load(hp + (size_t)j * D * C + 8 * q);
-      else hc[t].zero();
     }
   }
 };
@@ -119,52 +121,71 @@ otf_attention_kernel(const __grid_constant__ AttnParams p) {
   }
   const int32_t* __restrict__ idx = (p.mode == EGAT_GRAPH_PADDED) ? p.nbr : p.cnt;
 
-  float acc[TPL][8];
+  // accumulators as packed float pairs: acc[t][e] holds elements 2e, 2e+1 of chunk t
+  f32x2 acc[TPL][4];
 #pragma unroll
   for (int t = 0; t < TPL; ++t)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[t][e] = 0.f;
-  float mrun = -INFINITY, z = 0.f;
+    for (int e = 0; e < 4; ++e) acc[t][e] = 0ull;
+  // Online softmax in the log2 domain.  mref is a running reference maximum
+  // that is raised only when a logit exceeds it by more than kLazy, so the
+  // O(D*C/32) rescale of the accumulators is rare; every weight is
+  // 2^(s - mref) <= 2^kLazy and z, acc share the same reference, so m = acc / z
+  // is the softmax average exactly as with the true running maximum.
+  constexpr float kLazy = 8.f;
+  float mref = -INFINITY, z = 0.f;
 
   auto valid = [&](int j) { return (unsigned)j < (unsigned)p.n; };
-  int j0 = beg < end ? __ldg(idx + beg) : -1;
-  int j1 = beg + 1 < end ? __ldg(idx + beg + 1) : -1;
-  Frag<L, C, T> f0, f1;
-  if (valid(j0)) f0.load(kp, hp, j0, lane, kch, hdk);
-
-  for (long long s = beg; s < end; ++s) {
-    const int j2 = s + 2 < end ? __ldg(idx + s + 2) : -1;
-    if (valid(j1)) f1.load(kp, hp, j1, lane, kch, hdk);
-    if (valid(j0)) {
-      float kf[8];
-      f0.kc.to_f32(kf);
-      float sp = 0.f;
+  auto idx_at = [&](long long s) { return s < end ? __ldg(idx + s) : -1; };
+  auto consume = [&](const Frag<L, C, T>& f) {
+    float kf[8];
+    f.kc.to_f32(kf);
+    float sp = 0.f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) sp = fmaf(qv[e], kf[e], sp);
-      for (int o = 1; o < G; o <<= 1) sp += __shfl_xor_sync(0xffffffffu, sp, o);
-      const float sl = __shfl_sync(0xffffffffu, sp, src_lane);  // log2-scaled logit
-      if (sl > mrun) {
-        const float sc = fast_exp2(mrun - sl);
-        z *= sc;
+    for (int e = 0; e < 8; ++e) sp = fmaf(qv[e], kf[e], sp);
+    for (int o = 1; o < G; o <<= 1) sp += __shfl_xor_sync(0xffffffffu, sp, o);
+    const float sl = __shfl_sync(0xffffffffu, sp, src_lane);  // log2-scaled logit
+    const bool raise = sl > mref + kLazy;
+    if (__any_sync(0xffffffffu, raise)) {
+      const float mnew = raise ? sl : mref;
+      const float sc = raise ? fast_exp2(mref - mnew) : 1.f;
+      z *= sc;
+      const f32x2 sc2 = f2_pack(sc, sc);
 #pragma unroll
-        for (int t = 0; t < TPL; ++t)
+      for (int t = 0; t < TPL; ++t)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[t][e] *= sc;
-        mrun = sl;
-      }
-      const float pw = fast_exp2(sl - mrun);
-      z += pw;
+        for (int e = 0; e < 4; ++e) acc[t][e] = f2_mul(acc[t][e], sc2);
+      mref = mnew;
+    }
+    const float pw = fast_exp2(sl - mref);
+    z += pw;
+    const f32x2 pw2 = f2_pack(pw, pw);
 #pragma unroll
-      for (int t = 0; t < TPL; ++t) {
-        float hv[8];
-        f0.hc[t].to_f32(hv);
+    for (int t = 0; t < TPL; ++t) {
+      if (lane + 32 * t < NCH) {
+        f32x2 hv[4];
+        f.hc[t].to_f2(hv);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[t][e] = fmaf(pw, hv[e], acc[t][e]);
+        for (int e = 0; e < 4; ++e) acc[t][e] = f2_fma(pw2, hv[e], acc[t][e]);
       }
     }
-    f0 = f1;
-    j0 = j1;
-    j1 = j2;
+  };
+
+  // Two row buffers in ping-pong; neighbour indices are read four slots ahead
+  // so the index load never sits on the path of a row gather.
+  Frag<L, C, T> fa, fb;
+  int j0 = idx_at(beg), j1 = idx_at(beg + 1), j2 = idx_at(beg + 2), j3 = idx_at(beg + 3);
+  if (valid(j0)) fa.load(kp, hp, j0, lane, kch, hdk);
+  for (long long s = beg; s < end; s += 2) {
+    const int j4 = idx_at(s + 4), j5 = idx_at(s + 5);
+    if (valid(j1)) fb.load(kp, hp, j1, lane, kch, hdk);
+    if (valid(j0)) consume(fa);
+    if (valid(j2)) fa.load(kp, hp, j2, lane, kch, hdk);
+    if (valid(j1)) consume(fb);
+    j0 = j2;
+    j1 = j3;
+    j2 = j4;
+    j3 = j5;
   }
 
   const float inv = z > 0.f ? 1.f / z : 0.f;
@@ -174,9 +195,12 @@ otf_attention_kernel(const __grid_constant__ AttnParams p) {
     for (int t = 0; t < TPL; ++t) {
       const int q = lane + 32 * t;
       if (q < NCH) {
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) f2_unpack(acc[t][e], v[2 * e], v[2 * e + 1]);
         float4* dst = reinterpret_cast<float4*>(o + 8 * q);
-        dst[0] = make_float4(acc[t][0] * inv, acc[t][1] * inv, acc[t][2] * inv, acc[t][3] * inv);
-        dst[1] = make_float4(acc[t][4] * inv, acc[t][5] * inv, acc[t][6] * inv, acc[t][7] * inv);
+        dst[0] = make_float4(v[0] * inv, v[1] * inv, v[2] * inv, v[3] * inv);
+        dst[1] = make_float4(v[4] * inv, v[5] * inv, v[6] * inv, v[7] * inv);
       }
     }
   } else {
@@ -187,8 +211,11 @@ otf_attention_kernel(const __grid_constant__ AttnParams p) {
     for (int t = 0; t < TPL; ++t) {
       const int q = lane + 32 * t;
       if (q < NCH) {
+        float v[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mbuf[8 * q + e] = acc[t][e] * inv;
+        for (int e = 0; e < 4; ++e) f2_unpack(acc[t][e], v[2 * e], v[2 * e + 1]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mbuf[8 * q + e] = v[e] * inv;
       }
     }
     float Q[9];
@@ -204,13 +231,12 @@ otf_attention_kernel(const __grid_constant__ AttnParams p) {
     for (int c0 = 0; c0 < C; c0 += 32) {
       const int c = c0 + lane;
       if (c < C) {
-        float xin[D], yout[D];
+        float xin[D];
 #pragma unroll
         for (int d = 0; d < D; ++d) xin[d] = mbuf[d * C + c];
-        eaas_channel<L>(xin, yout, Dsm, rpow, p.tab,
-                        [&](int pp) { return __ldg(p.w2 + pp * C + c); });
-#pragma unroll
-        for (int d = 0; d < D; ++d) o[d * C + c] = yout[d];
+        eaas_channel<L>(xin, Dsm, rpow, p.tab,
+                        [&](int pp) { return __ldg(p.w2 + pp * C + c); },
+                        [&](int d, float v) { o[d * C + c] = v; });
       }
     }
   }

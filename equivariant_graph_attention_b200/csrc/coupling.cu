@@ -6,14 +6,13 @@
 // Memory" §2.1 (Lemma 4.1: only m = 0 of the solid harmonic survives in the
 // aligned frame; Eq. 13: the re-index rule).
 //
-// Kernel layout: a 256-thread block takes tiles of 256/C atoms, one thread per
-// (atom, channel).  Per tile the block builds each atom's Wigner-D matrices
-// (degree 1 from the alignment rotation, higher degrees by the
-// Ivanic–Ruedenberg recursion, entries in parallel) in shared memory; each
-// thread then rotates its channel's components into the aligned frame,
-// applies the sparse re-index with the path weights, and rotates back.  The
-// weights of the thread's channel stay in registers across tiles.  Memory
-// traffic is one read of h and one write of h' (streaming, HBM-bound).
+// Kernel layout: one thread per (atom, channel); a warp covers 32 channels of
+// one atom (or all 16 channels of two atoms).  The warp builds the atom's
+// Wigner-D matrices (degree 1 from the alignment rotation, higher degrees by
+// the Ivanic–Ruedenberg recursion, entries in parallel) in shared memory;
+// each lane then rotates its channel's components into the aligned frame,
+// applies the sparse re-index with the path weights, and rotates back.
+// Memory traffic is one read of h and one write of h' (streaming, HBM-bound).
 #include <cmath>
 #include <mutex>
 
@@ -93,7 +92,7 @@ const EaasTable& eaas_table(int L) {
 // ---------------------------------------------------------------------------
 namespace {
 
-constexpr int kEaasThreads = 256;
+constexpr int kEaasWarps = 8;
 
 struct EaasParams {
   const void* x;
@@ -105,71 +104,95 @@ struct EaasParams {
   EaasTable tab;
 };
 
+// One warp owns a block of G = min(C, 32) channels of 32/G atoms at a time
+// (lane = channel, so every load and store of a component row is coalesced).
+// The warp's channel block is fixed, so the path weights of its lane's channel
+// stay in registers.  Each warp builds the Wigner-D matrices of its atoms in
+// its own shared-memory slot with warp-level synchronisation only, and the
+// next atom's position and features are fetched before the current atom is
+// coupled.
 template <int L, typename T>
-__global__ void __launch_bounds__(kEaasThreads)
+__global__ void __launch_bounds__(kEaasWarps * 32, (L >= 3 ? 1 : 2))
 eaas_source_kernel(const __grid_constant__ EaasParams p) {
   constexpr int D = (L + 1) * (L + 1);
   constexpr int NP = num_paths(L);
   constexpr int WS = wig_size(L);
-  constexpr int kMaxAtoms = kEaasThreads / 16;
-  __shared__ float Dsm[kMaxAtoms][WS];
-  __shared__ float Qs[kMaxAtoms][9];
-  __shared__ float rps[kMaxAtoms][L + 1];
+  __shared__ float Dsm[kEaasWarps][2][WS];   // up to 2 atoms per warp (C = 16)
 
+  const int lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
   const int C = p.C;
-  const int A = kEaasThreads / C;  // atoms per tile
-  const int tid = threadIdx.x;
-  const int a = tid / C;           // atom slot of this thread
-  const int c = tid % C;           // channel of this thread
+  const int G = C < 32 ? C : 32;          // lanes per atom
+  const int AW = 32 / G;                  // atoms per warp (1 or 2)
+  const int slot = lane / G;              // which of the warp's atoms
+  const int g = lane % G;
+  const int nblk = C / G;                 // channel blocks per atom
+  const long long gwarp = (long long)blockIdx.x * kEaasWarps + wib;
+  const long long nwarps = (long long)gridDim.x * kEaasWarps;
+  const int cb = int(gwarp % nblk);
+  const int c = cb * G + g;               // this lane's channel
+  const long long ngroups = ((long long)p.n + AW - 1) / AW;
   const T* __restrict__ x = static_cast<const T*>(p.x);
   T* __restrict__ y = static_cast<T*>(p.y);
 
-  float wreg[NP];
+  // weights of this lane's channel: registers up to lmax 2, L1-cached loads above
+  constexpr bool kRegW = NP <= 15;
+  float wreg[kRegW ? NP : 1];
 #pragma unroll
-  for (int q = 0; q < NP; ++q) wreg[q] = __ldg(p.w + q * C + c);
+  for (int q = 0; q < (kRegW ? NP : 0); ++q) wreg[q] = __ldg(p.w + q * C + c);
+  const float* __restrict__ wcol = p.w + c;
 
-  const int ntiles = (p.n + A - 1) / A;
-  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    const int atom0 = tile * A;
-    if (tid < A) {
-      const int at = atom0 + tid;
-      float Q[9];
-      float r = 0.f;
-      if (at < p.n) {
-        r = alignment_rotation(p.pos[3 * at], p.pos[3 * at + 1], p.pos[3 * at + 2], Q);
-      } else {
-        alignment_rotation(0.f, 0.f, 0.f, Q);
-      }
-#pragma unroll
-      for (int e = 0; e < 9; ++e) Qs[tid][e] = Q[e];
-      float rp = 1.f;
-#pragma unroll
-      for (int l = 0; l <= L; ++l) {
-        rps[tid][l] = rp;
-        rp *= r;
-      }
-    }
-    __syncthreads();
-    {
-      float Q[9];
-#pragma unroll
-      for (int e = 0; e < 9; ++e) Q[e] = Qs[a][e];
-      wigner_build<L>(Q, Dsm[a], c, C, [] { __syncthreads(); });
-    }
-    const int at = atom0 + a;
-    if (at < p.n) {
-      float xin[D], yout[D], rpow[L + 1];
-#pragma unroll
-      for (int l = 0; l <= L; ++l) rpow[l] = rps[a][l];
+  float* Dme = Dsm[wib][slot];
+  long long grp = gwarp / nblk;
+  const long long gstride = nwarps / nblk;   // launch keeps nwarps a multiple of nblk
+
+  // prefetch the first atom
+  float px = 0.f, py = 0.f, pz = 0.f, xin[D];
+  auto fetch = [&](long long gr, float& fx, float& fy, float& fz, float (&xv)[D]) {
+    const long long at = gr * AW + slot;
+    if (gr < ngroups && at < p.n) {
+      fx = __ldg(p.pos + 3 * at);
+      fy = __ldg(p.pos + 3 * at + 1);
+      fz = __ldg(p.pos + 3 * at + 2);
       const T* xr = x + (size_t)at * D * C + c;
 #pragma unroll
-      for (int d = 0; d < D; ++d) xin[d] = load_one<T>(xr + d * C);
-      eaas_channel<L>(xin, yout, Dsm[a], rpow, p.tab, [&](int q) { return wreg[q]; });
-      T* yr = y + (size_t)at * D * C + c;
-#pragma unroll
-      for (int d = 0; d < D; ++d) store_one<T>(yr + d * C, yout[d]);
+      for (int d = 0; d < D; ++d) xv[d] = load_one<T>(xr + d * C);
     }
-    __syncthreads();
+  };
+  fetch(grp, px, py, pz, xin);
+  // lmax 3 keeps no second feature row in flight (register budget)
+  constexpr bool kPrefetch = L <= 2;
+  for (; grp < ngroups; grp += gstride) {
+    const long long at = grp * AW + slot;
+    float nx = 0.f, ny = 0.f, nz = 0.f, xnext[kPrefetch ? D : 1];
+    if constexpr (kPrefetch) fetch(grp + gstride, nx, ny, nz, xnext);
+    float Q[9];
+    const float r = alignment_rotation(px, py, pz, Q);
+    float rpow[L + 1];
+    rpow[0] = 1.f;
+#pragma unroll
+    for (int l = 1; l <= L; ++l) rpow[l] = rpow[l - 1] * r;
+    __syncwarp();                             // previous atom's readers are done
+    wigner_build<L>(Q, Dme, g, G, [] { __syncwarp(); });
+    if (at < p.n) {
+      T* yr = y + (size_t)at * D * C + c;
+      eaas_channel<L>(
+          xin, Dme, rpow, p.tab,
+          [&](int q) {
+            if constexpr (kRegW) return wreg[q];
+            else return __ldg(wcol + q * C);
+          },
+          [&](int d, float v) { store_one<T>(yr + d * C, v); });
+    }
+    if constexpr (kPrefetch) {
+      px = nx;
+      py = ny;
+      pz = nz;
+#pragma unroll
+      for (int d = 0; d < D; ++d) xin[d] = xnext[d];
+    } else {
+      fetch(grp + gstride, px, py, pz, xin);
+    }
   }
 }
 
@@ -184,13 +207,18 @@ int launch_eaas_t(const egat_shape& s, const void* d_x, const float* d_pos, cons
   p.n = s.n;
   p.C = s.C;
   p.tab = eaas_table(L);
-  const int A = kEaasThreads / s.C;
-  const int ntiles = (s.n + A - 1) / A;
+  const int G = s.C < 32 ? s.C : 32;
+  const int nblk = s.C / G;
+  const long long groups = ((long long)s.n + (32 / G) - 1) / (32 / G);
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = std::max(1, std::min(ntiles, sms * 8));
-  eaas_source_kernel<L, T><<<grid, kEaasThreads, 0, st>>>(p);
+  // warps needed: one per (atom group, channel block); cap at 8 resident blocks per SM
+  const long long want = (groups * nblk + kEaasWarps - 1) / kEaasWarps;
+  int grid = int(std::max<long long>(1, std::min<long long>(want, (long long)sms * 8)));
+  // keep the total warp count a multiple of the channel-block count
+  while ((long long)grid * kEaasWarps % nblk) ++grid;
+  eaas_source_kernel<L, T><<<grid, kEaasWarps * 32, 0, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
 }
 

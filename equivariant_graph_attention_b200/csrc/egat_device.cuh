@@ -64,6 +64,37 @@ struct EaasTable {
 };
 
 // ---------------------------------------------------------------------------
+// packed float2 arithmetic (sm_100 f32x2 FMA / MUL on a 64-bit register pair)
+// ---------------------------------------------------------------------------
+typedef unsigned long long f32x2;
+
+__device__ __forceinline__ f32x2 f2_pack(float lo, float hi) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(f32x2 v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+// d = a * b + c, element-wise on (lo, hi)
+__device__ __forceinline__ f32x2 f2_fma(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f32x2 f2_mul(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// two bf16 in one 32-bit word (element 2i in the low half) -> (lo, hi) floats
+__device__ __forceinline__ f32x2 bf16x2_to_f2(uint32_t w) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(w << 16), "r"(w & 0xffff0000u));
+  return r;
+}
+
+// ---------------------------------------------------------------------------
 // storage loads / stores
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&o)[8]) {
@@ -87,6 +118,13 @@ struct Chunk8<__nv_bfloat16> {
   }
   __device__ __forceinline__ void zero() { v = make_uint4(0, 0, 0, 0); }
   __device__ __forceinline__ void to_f32(float (&o)[8]) const { bf16x8_to_f32(v, o); }
+  // element pairs (0,1), (2,3), (4,5), (6,7) as packed floats
+  __device__ __forceinline__ void to_f2(f32x2 (&o)[4]) const {
+    o[0] = bf16x2_to_f2(v.x);
+    o[1] = bf16x2_to_f2(v.y);
+    o[2] = bf16x2_to_f2(v.z);
+    o[3] = bf16x2_to_f2(v.w);
+  }
 };
 
 template <>
@@ -103,6 +141,12 @@ struct Chunk8<float> {
   __device__ __forceinline__ void to_f32(float (&o)[8]) const {
     o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
     o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+  }
+  __device__ __forceinline__ void to_f2(f32x2 (&o)[4]) const {
+    o[0] = f2_pack(a.x, a.y);
+    o[1] = f2_pack(a.z, a.w);
+    o[2] = f2_pack(b.x, b.y);
+    o[3] = f2_pack(b.z, b.w);
   }
 };
 
@@ -160,11 +204,9 @@ __device__ __forceinline__ float alignment_rotation(float x, float y, float z, f
   return r;
 }
 
-// Degree-1 real Wigner-D: the rotation in (y, z, x) component order.
-__device__ __forceinline__ float wig1_from_Q(const float (&Q)[9], int e) {
-  const int perm[3] = {1, 2, 0};
-  const int a = e / 3, b = e % 3;
-  return Q[perm[a] * 3 + perm[b]];
+// Degree-1 real Wigner-D entry e = 3a + b: the rotation in (y, z, x) order.
+__host__ __device__ constexpr int wig1_src(int e) {
+  return ((e / 3 + 1) % 3) * 3 + ((e % 3 + 1) % 3);
 }
 
 // One entry D^l[m][mp] (m, mp in -l..l) of the real Wigner-D matrix of degree
@@ -220,7 +262,9 @@ template <int L, typename Sync>
 __device__ __forceinline__ void wigner_build(const float (&Q)[9], float* Dsm, int tid,
                                              int nthreads, Sync sync) {
   if (tid == 0) Dsm[0] = 1.f;
-  for (int e = tid; e < 9; e += nthreads) Dsm[wig_off(1) + e] = wig1_from_Q(Q, e);
+#pragma unroll
+  for (int e = 0; e < 9; ++e)
+    if (e % nthreads == tid) Dsm[wig_off(1) + e] = Q[wig1_src(e)];
   sync();
 #pragma unroll
   for (int l = 2; l <= L; ++l) {
@@ -240,30 +284,33 @@ __device__ __forceinline__ void wigner_build(const float (&Q)[9], float* Dsm, in
 //   xt^l = D^l(Q)^T x^l                       (into the frame with z along r)
 //   t^{lo}_m += w_p |r|^{lf} f_p(m) xt^{li}_{m or -m}   (only m_f = 0 survives)
 //   y^l = D^l(Q) t^l                          (back to the global frame)
-// `wgt(p)` returns w[p] for this channel; Dsm holds D^0..D^L.
-template <int L, typename WFn>
-__device__ __forceinline__ void eaas_channel(const float (&x)[(L + 1) * (L + 1)],
-                                             float (&y)[(L + 1) * (L + 1)],
+// `wgt(p)` returns w[p] for this channel; Dsm holds D^0..D^L.  x is
+// overwritten (the rotation is done in place); each output component is
+// handed to `out(d, value)` as soon as its degree is finished, so only x, t and
+// one degree's worth of temporaries are live at a time.
+template <int L, typename WFn, typename OutFn>
+__device__ __forceinline__ void eaas_channel(float (&x)[(L + 1) * (L + 1)],
                                              const float* __restrict__ Dsm,
                                              const float (&rpow)[L + 1], const EaasTable& tab,
-                                             WFn wgt) {
+                                             WFn wgt, OutFn out) {
   constexpr int D = (L + 1) * (L + 1);
-  float xt[D];
   float t[D];
 #pragma unroll
   for (int i = 0; i < D; ++i) t[i] = 0.f;
-  xt[0] = x[0];
   static_for<1, L + 1>([&](auto lc) {
     constexpr int l = decltype(lc)::value;
     constexpr int w = 2 * l + 1;
     const float* Dl = Dsm + wig_off(l);
+    float tmp[w];
 #pragma unroll
     for (int a = 0; a < w; ++a) {
       float s = 0.f;
 #pragma unroll
       for (int b = 0; b < w; ++b) s = fmaf(Dl[b * w + a], x[l * l + b], s);
-      xt[l * l + a] = s;
+      tmp[a] = s;
     }
+#pragma unroll
+    for (int a = 0; a < w; ++a) x[l * l + a] = tmp[a];
   });
   static_for<0, num_paths(L)>([&](auto pc) {
     constexpr int p = decltype(pc)::value;
@@ -276,11 +323,11 @@ __device__ __forceinline__ void eaas_channel(const float (&x)[(L + 1) * (L + 1)]
     for (int mo = -lo; mo <= lo; ++mo) {
       const int src = even ? mo : -mo;
       const bool live = (iabs(mo) <= li) && (even || mo != 0);
-      if (live) t[lo * lo + lo + mo] = fmaf(wp * tab.f[p][mo + lo], xt[li * li + li + src],
+      if (live) t[lo * lo + lo + mo] = fmaf(wp * tab.f[p][mo + lo], x[li * li + li + src],
                                             t[lo * lo + lo + mo]);
     }
   });
-  y[0] = t[0];
+  out(0, t[0]);
   static_for<1, L + 1>([&](auto lc) {
     constexpr int l = decltype(lc)::value;
     constexpr int w = 2 * l + 1;
@@ -290,7 +337,7 @@ __device__ __forceinline__ void eaas_channel(const float (&x)[(L + 1) * (L + 1)]
       float s = 0.f;
 #pragma unroll
       for (int b = 0; b < w; ++b) s = fmaf(Dl[a * w + b], t[l * l + b], s);
-      y[l * l + a] = s;
+      out(l * l + a, s);
     }
   });
 }

@@ -8,10 +8,12 @@
 // Design (B200): cells of edge r_c are mapped to a power-of-two bucket table
 // by the Morton code of the low bits of their coordinates, so scratch memory
 // depends only on n and the bucket order is a space-filling-curve order.
-// Kernels: assign cells -> histogram -> exclusive scan -> scatter -> one warp
-// per atom counts candidates in the 27 surrounding cells -> one warp per atom
-// gathers (d^2, j) keys into shared memory, bitonic-sorts them and writes the
-// row.  No kernel waits on another block; there are no spin loops.
+// Kernels: assign cells -> histogram -> exclusive scan -> scatter -> rank
+// atoms inside their bucket by index (deterministic order) -> one warp per atom
+// sweeps the 27 surrounding cells, writes the row and counts (padded), or
+// counts, scans and writes (CSR).  Rows with more than K neighbours keep the K
+// nearest, found by bisection on the (d^2, j) key.  No kernel waits on another
+// block; every loop is bounded.
 #include "egat_device.cuh"
 #include "egat_host.h"
 
@@ -19,12 +21,12 @@ namespace egat {
 namespace {
 
 constexpr int kFillWarps = 4;
-constexpr int kSortCap = 1024;   // keys per warp held in shared memory
 
 struct GraphWs {
   int4* cell;          // [n] (cx, cy, cz, bucket)
-  int4* spos;          // [n] bucket-sorted (x, y, z, atom)
+  int4* spos;          // [n] bucket-sorted (x, y, z, atom), atoms of a bucket by index
   int4* scell;         // [n] bucket-sorted (cx, cy, cz, 0)
+  int4* tpos;          // [n] bucket-sorted in arrival order (before ranking)
   int* bucket_cnt;     // [M]
   int* bucket_start;   // [M + 1]
   int* cursor;         // [M]
@@ -58,6 +60,7 @@ GraphWs carve(void* base, int n) {
   w.cell = static_cast<int4*>(take(sizeof(int4) * size_t(n)));
   w.spos = static_cast<int4*>(take(sizeof(int4) * size_t(n)));
   w.scell = static_cast<int4*>(take(sizeof(int4) * size_t(n)));
+  w.tpos = static_cast<int4*>(take(sizeof(int4) * size_t(n)));
   w.bucket_cnt = static_cast<int*>(take(sizeof(int) * M));
   w.bucket_start = static_cast<int*>(take(sizeof(int) * (M + 1)));
   w.cursor = static_cast<int*>(take(sizeof(int) * M));
@@ -182,18 +185,35 @@ int launch_scan(const int* in, int n, int* partial, int* out, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
 }
 
+// Counting-sort scatter: slots within a bucket are taken in arrival order.
 __global__ void scatter_atoms(const int32_t* __restrict__ pos, int n,
                               const int4* __restrict__ cell,
                               const int* __restrict__ bucket_start, int* __restrict__ cursor,
-                              int4* __restrict__ spos, int4* __restrict__ scell,
-                              int32_t* __restrict__ order) {
+                              int4* __restrict__ tpos) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
   const int4 c = cell[i];
   const int slot = bucket_start[c.w] + atomicAdd(&cursor[c.w], 1);
-  spos[slot] = make_int4(pos[3 * i], pos[3 * i + 1], pos[3 * i + 2], i);
-  scell[slot] = make_int4(c.x, c.y, c.z, 0);
-  if (order) order[slot] = i;
+  tpos[slot] = make_int4(pos[3 * i], pos[3 * i + 1], pos[3 * i + 2], i);
+}
+
+// Deterministic order inside each bucket: an atom's final slot is the bucket
+// start plus the number of atoms of its bucket with a smaller index.
+__global__ void rank_in_bucket(int n, const int4* __restrict__ cell,
+                               const int* __restrict__ bucket_start,
+                               const int4* __restrict__ tpos, int4* __restrict__ spos,
+                               int4* __restrict__ scell, int32_t* __restrict__ order) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= n) return;
+  const int4 me = tpos[k];
+  const int4 c = cell[me.w];
+  const int beg = bucket_start[c.w], end = bucket_start[c.w + 1];
+  int rank = 0;
+  for (int t = beg; t < end; ++t) rank += tpos[t].w < me.w ? 1 : 0;
+  const int dst = beg + rank;
+  spos[dst] = me;
+  scell[dst] = make_int4(c.x, c.y, c.z, 0);
+  if (order) order[dst] = me.w;
 }
 
 struct Search {
@@ -249,117 +269,86 @@ __global__ void count_neighbours(Search s, int n, int* __restrict__ deg) {
   if ((threadIdx.x & 31) == 0) deg[p.w] = cnt;
 }
 
-__device__ __forceinline__ void warp_bitonic_sort(unsigned long long* keys, int size) {
-  // ascending sort of keys[0, size), size a power of two
+// K-th smallest key (d^2 << shift | j) among the atom's neighbours, by
+// bisection over the key range; every key is distinct because j is.
+__device__ unsigned long long kth_key(const Search& s, int4 p, int4 c, int K) {
+  const unsigned long long jmask = (1ull << s.key_shift) - 1ull;
+  unsigned long long lo = 0, hi = ((unsigned long long)s.rc2 << s.key_shift) | jmask;
+  while (lo < hi) {
+    const unsigned long long mid = lo + ((hi - lo) >> 1);
+    int cnt = 0;
+    for_each_neighbour(s, p, c, [&](bool hit, int j, long long d2) {
+      cnt += (hit && ((((unsigned long long)d2) << s.key_shift) | (unsigned long long)j) <= mid)
+                 ? 1 : 0;
+    });
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    if (cnt >= K) hi = mid; else lo = mid + 1;
+  }
+  return lo;
+}
+
+// Padded list, one warp per atom (atoms taken in cell order).  One sweep
+// writes the first K neighbours and counts all of them; a row with more than
+// K neighbours is rewritten with exactly the K nearest (ties to smaller j).
+// Row order is the sweep order: the 27 cells in a fixed order, atoms of a
+// cell by index — deterministic, independent of thread scheduling.
+__global__ void __launch_bounds__(kFillWarps * 32)
+fill_padded(Search s, int n, int K, int32_t* __restrict__ nbr, int32_t* __restrict__ cnt,
+            int* __restrict__ overflow) {
   const int lane = threadIdx.x & 31;
-  for (int k = 2; k <= size; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = lane; i < size; i += 32) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const unsigned long long a = keys[i], b = keys[ixj];
-          const bool up = (i & k) == 0;
-          if ((a > b) == up) {
-            keys[i] = b;
-            keys[ixj] = a;
-          }
-        }
-      }
-      __syncwarp();
-    }
+  const int w = blockIdx.x * kFillWarps + (threadIdx.x >> 5);
+  if (w >= n) return;
+  const int4 p = s.spos[w];
+  const int4 c = s.scell[w];
+  int32_t* row = nbr + (long long)p.w * K;
+  int total = 0;
+  for_each_neighbour(s, p, c, [&](bool hit, int j, long long) {
+    const unsigned m = __ballot_sync(0xffffffffu, hit);
+    const int pos = total + __popc(m & ((1u << lane) - 1u));
+    if (hit && pos < K) row[pos] = j;
+    total += __popc(m);
+  });
+  if (total > K) {
+    const unsigned long long thresh = kth_key(s, p, c, K);
+    int written = 0;
+    for_each_neighbour(s, p, c, [&](bool hit, int j, long long d2) {
+      const bool keep = hit && ((((unsigned long long)d2) << s.key_shift) |
+                                (unsigned long long)j) <= thresh;
+      const unsigned m = __ballot_sync(0xffffffffu, keep);
+      const int pos = written + __popc(m & ((1u << lane) - 1u));
+      if (keep && pos < K) row[pos] = j;
+      written += __popc(m);
+    });
+  }
+  const int take = total < K ? total : K;
+  for (int t = take + lane; t < K; t += 32) row[t] = -1;
+  if (lane == 0) {
+    cnt[p.w] = take;
+    if (total > K) atomicAdd(overflow, total - K);
   }
 }
 
-// One warp per atom: collect the atom's (d^2 << shift | j) keys, sort, write.
+// CSR rows (after count_neighbours and the scan): every neighbour, in sweep order.
 __global__ void __launch_bounds__(kFillWarps * 32)
-fill_neighbours(Search s, int n, int K, int mode, const int* __restrict__ deg,
-                const int* __restrict__ rowptr_in, int32_t* __restrict__ nbr_or_rowptr,
-                int32_t* __restrict__ cnt_or_col, long long col_capacity,
-                int* __restrict__ overflow) {
-  __shared__ unsigned long long keys_all[kFillWarps][kSortCap];
+fill_csr(Search s, int n, const int* __restrict__ rowptr, int32_t* __restrict__ col,
+         long long col_capacity, int* __restrict__ overflow) {
   const int lane = threadIdx.x & 31;
-  const int wib = threadIdx.x >> 5;
-  const int w = blockIdx.x * kFillWarps + wib;
+  const int w = blockIdx.x * kFillWarps + (threadIdx.x >> 5);
   if (w >= n) return;
-  unsigned long long* keys = keys_all[wib];
   const int4 p = s.spos[w];
   const int4 c = s.scell[w];
-  const int i = p.w;
-  const int d = deg[i];
-  const unsigned long long jmask = (1ull << s.key_shift) - 1ull;
-
-  long long out_base;
-  int take;
-  if (mode == EGAT_GRAPH_PADDED) {
-    out_base = (long long)i * K;
-    take = min(d, K);
-  } else {
-    out_base = rowptr_in[i];
-    take = d;
-  }
-
-  if (mode == EGAT_GRAPH_CSR && d > kSortCap) {
-    // very dense row: written in visiting order, without sorting
-    int written = 0;
-    for_each_neighbour(s, p, c, [&](bool hit, int j, long long) {
-      const unsigned m = __ballot_sync(0xffffffffu, hit);
-      const int pos = written + __popc(m & ((1u << lane) - 1u));
-      if (hit && out_base + pos < col_capacity) cnt_or_col[out_base + pos] = j;
-      written += __popc(m);
-    });
-    if (lane == 0 && out_base + d > col_capacity)
-      atomicAdd(overflow, int(out_base >= col_capacity ? (long long)d : out_base + d - col_capacity));
-    return;
-  }
-
-  unsigned long long thresh = ~0ull;  // keep keys <= thresh
-  if (d > kSortCap) {
-    // padded mode with more candidates than fit: the K-th smallest key by
-    // bisection over the key range (every key is distinct because j is).
-    unsigned long long lo = 0, hi = ((unsigned long long)s.rc2 << s.key_shift) | jmask;
-    while (lo < hi) {
-      const unsigned long long mid = lo + ((hi - lo) >> 1);
-      int cnt = 0;
-      for_each_neighbour(s, p, c, [&](bool hit, int j, long long d2) {
-        cnt += (hit && ((((unsigned long long)d2) << s.key_shift) | (unsigned long long)j) <= mid) ? 1 : 0;
-      });
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-      if (cnt >= K) hi = mid; else lo = mid + 1;
-    }
-    thresh = lo;
-  }
-
-  // gather keys
-  int filled = 0;
-  for_each_neighbour(s, p, c, [&](bool hit, int j, long long d2) {
-    const unsigned long long key = (((unsigned long long)d2) << s.key_shift) | (unsigned long long)j;
-    const bool keep = hit && key <= thresh;
-    const unsigned m = __ballot_sync(0xffffffffu, keep);
-    const int pos = filled + __popc(m & ((1u << lane) - 1u));
-    if (keep && pos < kSortCap) keys[pos] = key;
-    filled += __popc(m);
+  const long long base = rowptr[p.w];
+  int written = 0;
+  for_each_neighbour(s, p, c, [&](bool hit, int j, long long) {
+    const unsigned m = __ballot_sync(0xffffffffu, hit);
+    const long long pos = base + written + __popc(m & ((1u << lane) - 1u));
+    if (hit && pos < col_capacity) col[pos] = j;
+    written += __popc(m);
   });
-  filled = min(filled, kSortCap);
-  int size = 1;
-  while (size < filled) size <<= 1;
-  for (int t = filled + lane; t < size; t += 32) keys[t] = ~0ull;
-  __syncwarp();
-  warp_bitonic_sort(keys, size);
-
-  if (mode == EGAT_GRAPH_PADDED) {
-    for (int t = lane; t < K; t += 32)
-      nbr_or_rowptr[out_base + t] = t < take ? int32_t(keys[t] & jmask) : -1;
-    if (lane == 0) {
-      cnt_or_col[i] = take;
-      if (d > K) atomicAdd(overflow, d - K);
-    }
-  } else {
-    for (int t = lane; t < take; t += 32)
-      if (out_base + t < col_capacity) cnt_or_col[out_base + t] = int32_t(keys[t] & jmask);
-    if (lane == 0 && out_base + take > col_capacity)
-      atomicAdd(overflow, int(out_base >= col_capacity ? (long long)take : out_base + take - col_capacity));
-  }
+  if (lane == 0 && base + written > col_capacity)
+    atomicAdd(overflow, int(base >= col_capacity ? (long long)written
+                                                 : base + written - col_capacity));
 }
 
 }  // namespace
@@ -381,20 +370,21 @@ int build_graph(const int32_t* d_pos_q, int n, int cutoff_q, int K, int mode,
   if (cudaMemsetAsync(w.cursor, 0, sizeof(int) * M, st) != cudaSuccess) return EGAT_ERR_CUDA;
 
   const int tb = 256;
-  assign_cells<<<(n + tb - 1) / tb, tb, 0, st>>>(d_pos_q, n, cutoff_q, bits, w.cell, w.bucket_cnt);
+  const unsigned nb = unsigned((n + tb - 1) / tb);
+  assign_cells<<<nb, tb, 0, st>>>(d_pos_q, n, cutoff_q, bits, w.cell, w.bucket_cnt);
   if (launch_scan(w.bucket_cnt, M, w.partial, w.bucket_start, st) != EGAT_OK) return EGAT_ERR_CUDA;
-  scatter_atoms<<<(n + tb - 1) / tb, tb, 0, st>>>(d_pos_q, n, w.cell, w.bucket_start, w.cursor,
-                                                   w.spos, w.scell, d_order);
+  scatter_atoms<<<nb, tb, 0, st>>>(d_pos_q, n, w.cell, w.bucket_start, w.cursor, w.tpos);
+  rank_in_bucket<<<nb, tb, 0, st>>>(n, w.cell, w.bucket_start, w.tpos, w.spos, w.scell, d_order);
   Search s{w.spos, w.scell, w.bucket_start, bits, (long long)cutoff_q * cutoff_q, key_shift};
-  const long long nthreads = (long long)n * 32;
-  count_neighbours<<<unsigned((nthreads + tb - 1) / tb), tb, 0, st>>>(s, n, w.deg);
-  const int* rowptr = nullptr;
-  if (mode == EGAT_GRAPH_CSR) {
+  const unsigned nfill = unsigned((n + kFillWarps - 1) / kFillWarps);
+  if (mode == EGAT_GRAPH_PADDED) {
+    fill_padded<<<nfill, kFillWarps * 32, 0, st>>>(s, n, K, d_a, d_b, d_overflow);
+  } else {
+    const long long nthreads = (long long)n * 32;
+    count_neighbours<<<unsigned((nthreads + tb - 1) / tb), tb, 0, st>>>(s, n, w.deg);
     if (launch_scan(w.deg, n, w.partial, d_a, st) != EGAT_OK) return EGAT_ERR_CUDA;
-    rowptr = d_a;
+    fill_csr<<<nfill, kFillWarps * 32, 0, st>>>(s, n, d_a, d_b, col_capacity, d_overflow);
   }
-  fill_neighbours<<<(n + kFillWarps - 1) / kFillWarps, kFillWarps * 32, 0, st>>>(
-      s, n, K, mode, w.deg, rowptr, d_a, d_b, col_capacity, d_overflow);
   return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
 }
 

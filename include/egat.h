@@ -108,17 +108,19 @@ EGAT_API int egat_num_paths(int lmax);
  *  d_pos_q       int32 [n][3] grid coordinates
  *  cutoff_q      cutoff in grid units, > 0
  *  mode          EGAT_GRAPH_PADDED:
- *                  d_nbr_or_rowptr = nbr int32 [n][K]: the K nearest
- *                  neighbours ordered by (squared distance, index), then -1;
+ *                  d_nbr_or_rowptr = nbr int32 [n][K]: the neighbours, then
+ *                  -1; an atom with more than K keeps the K nearest (ties at
+ *                  the K-th distance keep the smaller index);
  *                  d_cnt_or_col = cnt int32 [n] = min(degree, K);
- *                  *d_overflow = number of neighbours dropped by the
- *                  truncation (ties at the K-th distance keep smaller j).
+ *                  *d_overflow = number of neighbours dropped.
  *                EGAT_GRAPH_CSR:
  *                  d_nbr_or_rowptr = rowptr int32 [n+1];
- *                  d_cnt_or_col = col int32 [col_capacity]; each row ordered
- *                  by (squared distance, index) when its degree is <= 1024,
- *                  otherwise in unspecified order; entries past col_capacity
- *                  are not written and *d_overflow = their number.
+ *                  d_cnt_or_col = col int32 [col_capacity]; entries past
+ *                  col_capacity are not written and *d_overflow = their
+ *                  number.
+ *                Row order, both modes: the 27 cells around the atom's cell
+ *                in a fixed sweep, atoms of one cell by index — a
+ *                deterministic order (the same arrays on every call).
  *  d_order       optional int32 [n]: atoms listed cell by cell (Morton
  *                order of cells) — a traversal order with spatial locality
  *                for egat_otf_attention / egat_forward.  May be NULL.

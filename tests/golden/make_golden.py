@@ -20,7 +20,7 @@ from oracle.attention import forward          # noqa: E402
 from oracle.graph import radius_graph         # noqa: E402
 from equivariant_graph_attention_b200 import synth   # noqa: E402
 
-SPEC = dict(n=12, side=5.0, cutoff=3.0, K=6, lmax=2, C=8, H=2, dk=8, dtype="f32", seed=11)
+SPEC = dict(n=12, side=5.0, cutoff=3.0, K=6, lmax=2, C=16, H=2, dk=8, dtype="f32", seed=11)
 
 
 def build():
