@@ -5,14 +5,14 @@
 // reading: j != i is a neighbour of i iff |p_j - p_i|^2 <= r_c^2 on integer
 // grid coordinates; a padded list keeps the K nearest, ties to smaller j.
 //
-// Design (B200): cells of edge r_c are mapped to a power-of-two bucket table
+// Design (B200): cells of edge r_c / 2 are mapped to a power-of-two bucket table
 // by the Morton code of the low bits of their coordinates, so scratch memory
 // depends only on n and the bucket order is a space-filling-curve order.
 // Kernels: assign cells -> histogram -> exclusive scan -> scatter -> rank
 // atoms inside their bucket by index (deterministic order) -> one warp per atom
-// sweeps the 27 surrounding cells, writes the row and counts (padded), or
+// sweeps the 125 surrounding cells, writes the row and counts (padded), or
 // counts, scans and writes (CSR).  Rows with more than K neighbours keep the K
-// nearest, found by bisection on the (d^2, j) key.  No kernel waits on another
+// nearest, selected on the (d^2, j) key.  No kernel waits on another
 // block; every loop is bounded.
 #include "egat_device.cuh"
 #include "egat_host.h"
@@ -21,6 +21,7 @@ namespace egat {
 namespace {
 
 constexpr int kFillWarps = 4;
+constexpr int kSelectCap = 1024;   // neighbour keys a warp can hold in shared memory
 
 struct GraphWs {
   int4* cell;          // [n] (cx, cy, cz, bucket)
@@ -38,8 +39,9 @@ struct GraphWs {
 constexpr int kScanTile = 4096;  // elements per scan block (1024 threads x 4)
 
 int bucket_bits(int n) {
-  // bits per axis b, table size M = 2^(3b) >= 2n, 2 <= b <= 8
-  int b = 2;
+  // bits per axis b, table size M = 2^(3b) >= 2n, 3 <= b <= 8 (2^b >= 5
+  // keeps the 5 x 5 x 5 cells around any cell in distinct buckets)
+  int b = 3;
   while (b < 8 && (int64_t(1) << (3 * b)) < 2 * int64_t(n)) ++b;
   return b;
 }
@@ -225,36 +227,72 @@ struct Search {
   int key_shift;
 };
 
-// Visit every candidate of atom (p, c, i) within the cutoff; lanes of a warp
-// split each cell's range.  f(j, d2) is called by the lane that owns the
-// candidate; all lanes return together.
+// Cells have edge ceil(r_c / 2), so every neighbour lies in the 5 x 5 x 5
+// block of cells around the atom's cell.
+constexpr int kSpan = 2;
+constexpr int kWidth = 2 * kSpan + 1;
+constexpr int kBlockCells = kWidth * kWidth * kWidth;
+
+// Visit every candidate of atom p (cell c) once; f(hit, j, d2) is called by
+// every lane of the warp together (full-warp ballots are allowed inside), hit
+// marking a neighbour within the cutoff.  Cells are taken 32 at a time: each
+// lane loads one cell's bucket range, a warp scan lays the ranges end to end,
+// and the warp walks that flat candidate list 32 at a time, each lane finding
+// its candidate's cell by a binary search over the scanned offsets.
 template <typename F>
 __device__ __forceinline__ void for_each_neighbour(const Search& s, int4 p, int4 c, F&& f) {
   const int lane = threadIdx.x & 31;
-  for (int dz = -1; dz <= 1; ++dz)
-    for (int dy = -1; dy <= 1; ++dy)
-      for (int dx = -1; dx <= 1; ++dx) {
-        const int cx = c.x + dx, cy = c.y + dy, cz = c.z + dz;
-        const int b = bucket_of(cx, cy, cz, s.bits);
-        const int beg = s.bucket_start[b], end = s.bucket_start[b + 1];
-        // warp-uniform trip count: callers use full-warp ballots
-        for (int base = beg; base < end; base += 32) {
-          const int k = base + lane;
-          bool hit = false;
-          int j = -1;
-          long long d2 = 0;
-          const int4 cc = k < end ? s.scell[k] : make_int4(0, 0, 0, 0);
-          if (k < end && cc.x == cx && cc.y == cy && cc.z == cz) {
-            const int4 q = s.spos[k];
-            j = q.w;
-            const long long ddx = (long long)q.x - p.x, ddy = (long long)q.y - p.y,
-                            ddz = (long long)q.z - p.z;
-            d2 = ddx * ddx + ddy * ddy + ddz * ddz;
-            hit = (j != p.w) && (d2 <= s.rc2);
-          }
-          f(hit, j, d2);
+  for (int r0 = 0; r0 < kBlockCells; r0 += 32) {
+    const int l = r0 + lane;
+    int beg = 0, len = 0, cx = 0, cy = 0, cz = 0;
+    if (l < kBlockCells) {
+      cx = c.x + l % kWidth - kSpan;
+      cy = c.y + (l / kWidth) % kWidth - kSpan;
+      cz = c.z + l / (kWidth * kWidth) - kSpan;
+      const int b = bucket_of(cx, cy, cz, s.bits);
+      beg = s.bucket_start[b];
+      len = s.bucket_start[b + 1] - beg;
+    }
+    int inc = len;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    const int total = __shfl_sync(0xffffffffu, inc, 31);
+    const int exc = inc - len;
+    for (int base = 0; base < total; base += 32) {
+      const int k = base + lane;
+      // owner: the last lane whose range starts at or before k
+      int own = 0;
+#pragma unroll
+      for (int step = 16; step > 0; step >>= 1) {
+        const int e = __shfl_sync(0xffffffffu, exc, own + step);
+        if (e <= k) own += step;
+      }
+      const int obeg = __shfl_sync(0xffffffffu, beg, own);
+      const int oexc = __shfl_sync(0xffffffffu, exc, own);
+      const int ocx = __shfl_sync(0xffffffffu, cx, own);
+      const int ocy = __shfl_sync(0xffffffffu, cy, own);
+      const int ocz = __shfl_sync(0xffffffffu, cz, own);
+      bool hit = false;
+      int j = -1;
+      long long d2 = 0;
+      if (k < total) {
+        const int slot = obeg + (k - oexc);
+        const int4 cc = s.scell[slot];
+        const int4 q = s.spos[slot];
+        if (cc.x == ocx && cc.y == ocy && cc.z == ocz) {
+          j = q.w;
+          const long long ddx = (long long)q.x - p.x, ddy = (long long)q.y - p.y,
+                          ddz = (long long)q.z - p.z;
+          d2 = ddx * ddx + ddy * ddy + ddz * ddz;
+          hit = (j != p.w) && (d2 <= s.rc2);
         }
       }
+      f(hit, j, d2);
+    }
+  }
 }
 
 __global__ void count_neighbours(Search s, int n, int* __restrict__ deg) {
@@ -288,16 +326,40 @@ __device__ unsigned long long kth_key(const Search& s, int4 p, int4 c, int K) {
   return lo;
 }
 
+__device__ __forceinline__ void warp_bitonic_sort(unsigned long long* keys, int size) {
+  // ascending sort of keys[0, size), size a power of two, one warp
+  const int lane = threadIdx.x & 31;
+  for (int k = 2; k <= size; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = lane; i < size; i += 32) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const unsigned long long a = keys[i], b = keys[ixj];
+          if ((a > b) == ((i & k) == 0)) {
+            keys[i] = b;
+            keys[ixj] = a;
+          }
+        }
+      }
+      __syncwarp();
+    }
+  }
+}
+
 // Padded list, one warp per atom (atoms taken in cell order).  One sweep
-// writes the first K neighbours and counts all of them; a row with more than
-// K neighbours is rewritten with exactly the K nearest (ties to smaller j).
-// Row order is the sweep order: the 27 cells in a fixed order, atoms of a
-// cell by index — deterministic, independent of thread scheduling.
+// writes the first K neighbours and counts all of them.  A row with more than
+// K neighbours finds the key (d^2 << shift | j) of its K-th nearest — by a
+// shared-memory sort of all its keys when they fit, by bisection otherwise —
+// and is rewritten with exactly the keys up to it (ties to smaller j).  Row
+// order is the sweep order: the 125 cells in a fixed order, atoms of a cell
+// by index — deterministic, independent of thread scheduling.
 __global__ void __launch_bounds__(kFillWarps * 32)
 fill_padded(Search s, int n, int K, int32_t* __restrict__ nbr, int32_t* __restrict__ cnt,
             int* __restrict__ overflow) {
+  __shared__ unsigned long long keys_all[kFillWarps][kSelectCap];
   const int lane = threadIdx.x & 31;
-  const int w = blockIdx.x * kFillWarps + (threadIdx.x >> 5);
+  const int wib = threadIdx.x >> 5;
+  const int w = blockIdx.x * kFillWarps + wib;
   if (w >= n) return;
   const int4 p = s.spos[w];
   const int4 c = s.scell[w];
@@ -310,7 +372,27 @@ fill_padded(Search s, int n, int K, int32_t* __restrict__ nbr, int32_t* __restri
     total += __popc(m);
   });
   if (total > K) {
-    const unsigned long long thresh = kth_key(s, p, c, K);
+    unsigned long long thresh;
+    if (total <= kSelectCap) {
+      unsigned long long* keys = keys_all[wib];
+      int filled = 0;
+      for_each_neighbour(s, p, c, [&](bool hit, int j, long long d2) {
+        const unsigned m = __ballot_sync(0xffffffffu, hit);
+        const int pos = filled + __popc(m & ((1u << lane) - 1u));
+        if (hit && pos < kSelectCap)
+          keys[pos] = (((unsigned long long)d2) << s.key_shift) | (unsigned long long)j;
+        filled += __popc(m);
+      });
+      int size = 1;
+      while (size < total) size <<= 1;
+      for (int t = total + lane; t < size; t += 32) keys[t] = ~0ull;
+      __syncwarp();
+      warp_bitonic_sort(keys, size);
+      thresh = keys[K - 1];
+      __syncwarp();
+    } else {
+      thresh = kth_key(s, p, c, K);
+    }
     int written = 0;
     for_each_neighbour(s, p, c, [&](bool hit, int j, long long d2) {
       const bool keep = hit && ((((unsigned long long)d2) << s.key_shift) |
@@ -371,7 +453,8 @@ int build_graph(const int32_t* d_pos_q, int n, int cutoff_q, int K, int mode,
 
   const int tb = 256;
   const unsigned nb = unsigned((n + tb - 1) / tb);
-  assign_cells<<<nb, tb, 0, st>>>(d_pos_q, n, cutoff_q, bits, w.cell, w.bucket_cnt);
+  const int cell_q = (cutoff_q + 1) / 2;   // cell edge ceil(r_c / 2)
+  assign_cells<<<nb, tb, 0, st>>>(d_pos_q, n, cell_q, bits, w.cell, w.bucket_cnt);
   if (launch_scan(w.bucket_cnt, M, w.partial, w.bucket_start, st) != EGAT_OK) return EGAT_ERR_CUDA;
   scatter_atoms<<<nb, tb, 0, st>>>(d_pos_q, n, w.cell, w.bucket_start, w.cursor, w.tpos);
   rank_in_bucket<<<nb, tb, 0, st>>>(n, w.cell, w.bucket_start, w.tpos, w.spos, w.scell, d_order);

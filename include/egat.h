@@ -102,8 +102,8 @@ EGAT_API int egat_num_paths(int lmax);
  * Step 1 — radius graph ([EX] §5.1 edge_cutoff, §5.2 neighbour-list check).
  * Atom j != i is a neighbour of i when |p_j - p_i|^2 <= cutoff_q^2, computed
  * exactly in 64-bit integers on grid coordinates (inclusive cutoff).  Cells
- * of edge cutoff_q are hashed to a power-of-two table by a Morton code of the
- * cell coordinates, so memory depends only on n, not on the box.
+ * of edge ceil(cutoff_q / 2) are hashed to a power-of-two table by a Morton
+ * code of the cell coordinates, so memory depends only on n, not on the box.
  *
  *  d_pos_q       int32 [n][3] grid coordinates
  *  cutoff_q      cutoff in grid units, > 0
@@ -118,8 +118,8 @@ EGAT_API int egat_num_paths(int lmax);
  *                  d_cnt_or_col = col int32 [col_capacity]; entries past
  *                  col_capacity are not written and *d_overflow = their
  *                  number.
- *                Row order, both modes: the 27 cells around the atom's cell
- *                in a fixed sweep, atoms of one cell by index — a
+ *                Row order, both modes: the 5 x 5 x 5 cells around the
+ *                atom's cell in a fixed sweep, atoms of one cell by index — a
  *                deterministic order (the same arrays on every call).
  *  d_order       optional int32 [n]: atoms listed cell by cell (Morton
  *                order of cells) — a traversal order with spatial locality
