@@ -54,6 +54,8 @@ const char* egat_strerror(int code) {
     case EGAT_ERR_UNSUPPORTED: return "shape outside the supported set";
     case EGAT_ERR_CUDA: return "CUDA launch or runtime error";
     case EGAT_ERR_WORKSPACE: return "workspace too small";
+    case EGAT_ERR_SCRATCH_LIMIT:
+      return "problem needs more scratch than egat_forward_noalloc's fixed array holds";
     default: return "unknown egat status";
   }
 }

@@ -25,6 +25,9 @@ EGAT_ERR_ARG = -1
 EGAT_ERR_UNSUPPORTED = -2
 EGAT_ERR_CUDA = -3
 EGAT_ERR_WORKSPACE = -4
+EGAT_ERR_SCRATCH_LIMIT = -5
+#: size of the fixed scratch array behind egat_forward_noalloc
+NOALLOC_SCRATCH_BYTES = 32 << 20
 EGAT_F32 = 0
 EGAT_BF16 = 1
 EGAT_GRAPH_PADDED = 0
@@ -34,7 +37,7 @@ EGAT_GRAPH_CSR = 1
 EXPORTS = ["egat_version", "egat_strerror", "egat_num_paths", "egat_graph_workspace_bytes",
            "egat_build_graph", "egat_eaas_couple", "egat_otf_attention",
            "egat_otf_attention_coupled",
-           "egat_forward_workspace_bytes", "egat_forward"]
+           "egat_forward_workspace_bytes", "egat_forward", "egat_forward_noalloc"]
 
 
 class EgatError(RuntimeError):
@@ -85,6 +88,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.egat_forward_workspace_bytes.argtypes = [sp, ctypes.POINTER(sz)]
     lib.egat_forward.restype = ctypes.c_int
     lib.egat_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
+    lib.egat_forward_noalloc.restype = ctypes.c_int
+    lib.egat_forward_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     if path is None:
         _lib = lib
     return lib
@@ -260,4 +265,24 @@ def egat_forward(shape: Shape, h: torch.Tensor, pos: torch.Tensor, q: torch.Tens
         _ptr(cnt_or_col), _ptr(order), _ptr(w1), _ptr(w2), _ptr(workspace), workspace.numel(),
         _ptr(out), _stream(stream))
     _check("egat_forward", rc)
+    return out
+
+
+def egat_forward_noalloc(shape: Shape, h: torch.Tensor, pos: torch.Tensor, q: torch.Tensor,
+                         k: torch.Tensor, nbr_or_rowptr: torch.Tensor,
+                         cnt_or_col: Optional[torch.Tensor], w1: torch.Tensor, w2: torch.Tensor,
+                         out: torch.Tensor, order: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """egat_forward without a workspace: the library's fixed scratch array holds h'.
+
+    For callers that may not allocate device memory at call time; ``out`` must
+    be provided by the caller.  Problems whose h' exceeds
+    ``NOALLOC_SCRATCH_BYTES`` raise EgatError(EGAT_ERR_SCRATCH_LIMIT).  Calls
+    that overlap on the GPU share the scratch and race; serialise them.
+    """
+    cs = shape.c()
+    rc = load_library().egat_forward_noalloc(
+        ctypes.byref(cs), _ptr(h), _ptr(pos), _ptr(q), _ptr(k), _ptr(nbr_or_rowptr),
+        _ptr(cnt_or_col), _ptr(order), _ptr(w1), _ptr(w2), _ptr(out), _stream(stream))
+    _check("egat_forward_noalloc", rc)
     return out

@@ -65,7 +65,8 @@ enum {
   EGAT_ERR_ARG = -1,          /* null pointer, bad size or misaligned pointer */
   EGAT_ERR_UNSUPPORTED = -2,  /* shape outside the supported set above */
   EGAT_ERR_CUDA = -3,         /* a CUDA launch or runtime call failed */
-  EGAT_ERR_WORKSPACE = -4     /* workspace smaller than the query returned */
+  EGAT_ERR_WORKSPACE = -4,    /* workspace smaller than the query returned */
+  EGAT_ERR_SCRATCH_LIMIT = -5 /* egat_forward_noalloc: problem larger than its fixed scratch */
 };
 
 /* storage type of h, q, k and h' (accumulation and outputs are float32) */
@@ -193,6 +194,32 @@ EGAT_API int egat_forward(const egat_shape* s, const void* d_h, const float* d_p
                  const void* d_k, const int32_t* d_nbr_or_rowptr, const int32_t* d_cnt_or_col,
                  const int32_t* d_order, const float* d_w1, const float* d_w2, void* d_ws,
                  size_t ws_bytes, float* d_out, void* stream);
+
+/*
+ * egat_forward_noalloc — egat_forward for callers that cannot allocate device
+ * memory at call time (a plugin inside a framework that owns all device
+ * allocations, a service whose memory footprint is fixed at start-up).  The
+ * pages have no counterpart: this is a library convenience, not a step of the
+ * method.  It takes the same arguments as egat_forward minus the workspace and
+ * computes the same result; its scratch (h') lives in a library-owned device
+ * array of EGAT_NOALLOC_SCRATCH_BYTES bytes that every GPU loading the library
+ * holds until the process exits.  It performs no allocation.
+ *  - Limit: egat_forward_workspace_bytes(s) <= EGAT_NOALLOC_SCRATCH_BYTES,
+ *    i.e. n * (lmax+1)^2 * C * (2 for bf16, 4 for f32) bytes rounded up to
+ *    256; larger problems return EGAT_ERR_SCRATCH_LIMIT without launching.
+ *  - The first call on a device, made with that device current, looks up the
+ *    array's device address once (cudaGetSymbolAddress); make that first call
+ *    before any stream capture.
+ *  - All calls share the array: calls whose work overlaps on the GPU race
+ *    on it and must be serialised by the caller.  Nothing in it needs
+ *    clearing between calls.
+ */
+#define EGAT_NOALLOC_SCRATCH_BYTES (32u << 20)
+EGAT_API int egat_forward_noalloc(const egat_shape* s, const void* d_h, const float* d_pos,
+                                  const void* d_q, const void* d_k,
+                                  const int32_t* d_nbr_or_rowptr, const int32_t* d_cnt_or_col,
+                                  const int32_t* d_order, const float* d_w1, const float* d_w2,
+                                  float* d_out, void* stream);
 
 #ifdef __cplusplus
 }
