@@ -3,8 +3,10 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
 One step = one pass of the whole hot path over one synthetic system:
-radius graph (egat_build_graph) -> EAAS source coupling (egat_eaas_couple)
--> on-the-fly attention with the target coupling fused (egat_otf_attention_coupled).
+radius graph (egat_build_graph) -> attention plan (egat_build_attention_plan,
+tensor-core shapes) -> EAAS source coupling (egat_eaas_couple) -> on-the-fly
+attention with the target coupling fused (egat_otf_attention_tiled on
+tensor-core shapes, egat_otf_attention_coupled otherwise).
 The default workload is the 32,768-atom, K = 256, ℓmax = 2, bf16-storage
 system.  Inputs are resident in HBM when the timed region starts; L2 is
 flushed (a 256 MiB write) before every timed step, outside the step's events.
@@ -40,10 +42,12 @@ METRIC = "atoms/s & edges/s, fused EAAS+on-the-fly attention; % of HBM roofline"
 DEFAULT_WORKLOAD = "uniform32768_K256_l2_bf16"
 FLUSH_BYTES = 256 << 20
 #: kernels this library launches per step: graph (assign, scan x3, scatter,
-#: count, fill) + source coupling + fused attention
-LAUNCHES_PER_STEP = 9
+#: rank, fill, truncated-row fix) + attention plan (tensor-core shapes) +
+#: source coupling + fused attention
+LAUNCHES_GRAPH = 8
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attention_traffic.json")
 KERNEL_SOURCES = ["equivariant_graph_attention_b200/csrc/attention.cu",
+                  "equivariant_graph_attention_b200/csrc/attention_tc.cu",
                   "equivariant_graph_attention_b200/csrc/egat_device.cuh"]
 
 
@@ -251,23 +255,44 @@ def main():
                                   w1.data_ptr(), hp.data_ptr(), sp)
         egat._check("egat_eaas_couple", rc)
 
+    plan_sz = ctypes.c_size_t(0)
+    tiled = (lib.egat_attention_plan_bytes(ctypes.byref(cshape), ctypes.byref(plan_sz)) == 0
+             and wl.dtype == "bf16" and wl.C == 128 and wl.H == 16 and wl.dk == 16)
+    plan = torch.empty(max(plan_sz.value, 16), dtype=torch.uint8, device=dev)
+
+    def build_plan():
+        if tiled:
+            rc = lib.egat_build_attention_plan(ctypes.byref(cshape), nbr.data_ptr(),
+                                               cnt.data_ptr(), order.data_ptr(), plan.data_ptr(),
+                                               plan.numel(), sp)
+            egat._check("egat_build_attention_plan", rc)
+
     def attend():
-        rc = lib.egat_otf_attention_coupled(ctypes.byref(cshape), q.data_ptr(), k.data_ptr(),
-                                            hp.data_ptr(), nbr.data_ptr(), cnt.data_ptr(),
-                                            order.data_ptr(), pos.data_ptr(), w2.data_ptr(),
-                                            out.data_ptr(), sp)
-        egat._check("egat_otf_attention_coupled", rc)
+        if tiled:
+            rc = lib.egat_otf_attention_tiled(ctypes.byref(cshape), q.data_ptr(), k.data_ptr(),
+                                              hp.data_ptr(), plan.data_ptr(), order.data_ptr(),
+                                              pos.data_ptr(), w2.data_ptr(), out.data_ptr(), 1, sp)
+            egat._check("egat_otf_attention_tiled", rc)
+        else:
+            rc = lib.egat_otf_attention_coupled(ctypes.byref(cshape), q.data_ptr(), k.data_ptr(),
+                                                hp.data_ptr(), nbr.data_ptr(), cnt.data_ptr(),
+                                                order.data_ptr(), pos.data_ptr(), w2.data_ptr(),
+                                                out.data_ptr(), sp)
+            egat._check("egat_otf_attention_coupled", rc)
+    attn_name = "otf_attention_tiled" if tiled else "otf_attention_coupled"
+    launches_per_step = LAUNCHES_GRAPH + (1 if tiled else 0) + 2
 
     for _ in range(args.warmup):
         flush.fill_(1)
         graph()
+        build_plan()
         couple()
         attend()
     torch.cuda.synchronize(dev)
     cnt_host = cnt.cpu().numpy()
     alg = algorithmic_bytes(wl, cnt_host)
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
     time.sleep(0.3)
     if ws > 1:
@@ -279,19 +304,22 @@ def main():
         e[0].record(stream)
         graph()
         e[1].record(stream)
-        couple()
+        build_plan()
         e[2].record(stream)
-        attend()
+        couple()
         e[3].record(stream)
+        attend()
+        e[4].record(stream)
     torch.cuda.synchronize(dev)
     if ws > 1:
         dist.barrier()
     clk = clocks.stop()
 
     t_graph = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
-    t_eaas = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
-    t_attn = sum(e[2].elapsed_time(e[3]) for e in ev) / args.steps
-    t_step = sum(e[0].elapsed_time(e[3]) for e in ev) / args.steps      # ms
+    t_plan = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    t_eaas = sum(e[2].elapsed_time(e[3]) for e in ev) / args.steps
+    t_attn = sum(e[3].elapsed_time(e[4]) for e in ev) / args.steps
+    t_step = sum(e[0].elapsed_time(e[4]) for e in ev) / args.steps      # ms
     total_ms = t_step * args.steps
     if ws > 1:
         tt = torch.tensor([total_ms], device=dev)
@@ -375,16 +403,16 @@ def main():
                        "l2": "flushed before every timed step (256 MiB write, untimed)",
                        "parallelism": f"{ws} independent systems (one per GPU)"},
             "edges_per_s": edges_per_s,
-            "kernel_ms": {"build_graph": t_graph, "eaas_couple": t_eaas,
-                          "otf_attention_coupled": t_attn},
-            "roofline": {"bound": "hbm", "kernel": "otf_attention_coupled",
+            "kernel_ms": {"build_graph": t_graph, "attention_plan": t_plan,
+                          "eaas_couple": t_eaas, attn_name: t_attn},
+            "roofline": {"bound": "hbm", "kernel": attn_name,
                          "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
                          "algorithmic_bytes": alg["attention"], "peak_source": peaks["source"]},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "atoms/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.e2e_steps},
-            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)

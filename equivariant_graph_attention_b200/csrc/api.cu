@@ -41,6 +41,13 @@ size_t hp_bytes(const egat_shape& s) {
   return (size_t(s.n) * D * s.C * storage_bytes(s.dtype) + 255) & ~size_t(255);
 }
 
+// forward workspace: h', then (tensor-core shapes) the attention plan
+size_t forward_ws_bytes(const egat_shape& s) {
+  size_t b = hp_bytes(s);
+  if (tc_attention_supported(s) && s.n > 0) b += plan_bytes(s.n, s.K);
+  return b;
+}
+
 }  // namespace
 
 extern "C" {
@@ -147,8 +154,51 @@ int egat_forward_workspace_bytes(const egat_shape* s, size_t* bytes) {
   if (!bytes) return EGAT_ERR_ARG;
   const int rc = check_shape(s, true);
   if (rc != EGAT_OK) return rc;
-  *bytes = hp_bytes(*s);
+  *bytes = forward_ws_bytes(*s);
   return EGAT_OK;
+}
+
+int egat_attention_plan_bytes(const egat_shape* s, size_t* bytes) {
+  if (!bytes) return EGAT_ERR_ARG;
+  const int rc = check_shape(s, true);
+  if (rc != EGAT_OK) return rc;
+  if (s->graph_mode != EGAT_GRAPH_PADDED) return EGAT_ERR_UNSUPPORTED;
+  if (plan_smem_bytes(s->n, s->K) > kPlanSmemLimit) return EGAT_ERR_UNSUPPORTED;
+  *bytes = s->n > 0 ? plan_bytes(s->n, s->K) : 0;
+  return EGAT_OK;
+}
+
+int egat_build_attention_plan(const egat_shape* s, const int32_t* d_nbr, const int32_t* d_cnt,
+                              const int32_t* d_order, void* d_plan, size_t plan_bytes_given,
+                              void* stream) {
+  const int rc = check_shape(s, true);
+  if (rc != EGAT_OK) return rc;
+  if (s->graph_mode != EGAT_GRAPH_PADDED) return EGAT_ERR_UNSUPPORTED;
+  if (plan_smem_bytes(s->n, s->K) > kPlanSmemLimit) return EGAT_ERR_UNSUPPORTED;
+  if (s->n == 0) return EGAT_OK;
+  if (!d_nbr || !d_plan) return EGAT_ERR_ARG;
+  if (!aligned16(d_plan) || !aligned4(d_nbr)) return EGAT_ERR_ARG;
+  if (plan_bytes_given < plan_bytes(s->n, s->K)) return EGAT_ERR_WORKSPACE;
+  return launch_build_plan(s->n, s->K, d_nbr, d_cnt, d_order, d_plan,
+                           static_cast<cudaStream_t>(stream));
+}
+
+int egat_otf_attention_tiled(const egat_shape* s, const void* d_q, const void* d_k,
+                             const void* d_hp, const void* d_plan, const int32_t* d_order,
+                             const float* d_pos, const float* d_w2, float* d_out, int32_t fused,
+                             void* stream) {
+  const int rc = check_shape(s, true);
+  if (rc != EGAT_OK) return rc;
+  if (!tc_attention_supported(*s)) return EGAT_ERR_UNSUPPORTED;
+  if (s->n == 0) return EGAT_OK;
+  if (!d_q || !d_k || !d_hp || !d_plan || !d_out) return EGAT_ERR_ARG;
+  if (fused && (!d_pos || !d_w2)) return EGAT_ERR_ARG;
+  if (!aligned16(d_q) || !aligned16(d_k) || !aligned16(d_hp) || !aligned16(d_plan) ||
+      !aligned16(d_out))
+    return EGAT_ERR_ARG;
+  if (fused && (!aligned4(d_pos) || !aligned4(d_w2))) return EGAT_ERR_ARG;
+  return launch_attention_tc(*s, fused != 0, d_q, d_k, d_hp, d_plan, d_order, d_pos, d_w2, d_out,
+                             static_cast<cudaStream_t>(stream));
 }
 
 int egat_forward(const egat_shape* s, const void* d_h, const float* d_pos, const void* d_q,
@@ -164,8 +214,16 @@ int egat_forward(const egat_shape* s, const void* d_h, const float* d_pos, const
   if (!aligned16(d_h) || !aligned16(d_q) || !aligned16(d_k) || !aligned16(d_ws) ||
       !aligned16(d_out) || !aligned4(d_pos) || !aligned4(d_w1) || !aligned4(d_w2))
     return EGAT_ERR_ARG;
-  if (ws_bytes < hp_bytes(*s)) return EGAT_ERR_WORKSPACE;
+  if (ws_bytes < forward_ws_bytes(*s)) return EGAT_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tc_attention_supported(*s)) {
+    void* plan = static_cast<char*>(d_ws) + hp_bytes(*s);
+    int e = launch_build_plan(s->n, s->K, d_nbr_or_rowptr, d_cnt_or_col, d_order, plan, st);
+    if (e != EGAT_OK) return e;
+    e = launch_eaas_source(*s, d_h, d_pos, d_w1, d_ws, st);
+    if (e != EGAT_OK) return e;
+    return launch_attention_tc(*s, true, d_q, d_k, d_ws, plan, d_order, d_pos, d_w2, d_out, st);
+  }
   int e = launch_eaas_source(*s, d_h, d_pos, d_w1, d_ws, st);
   if (e != EGAT_OK) return e;
   return launch_attention(*s, true, d_q, d_k, d_ws, d_nbr_or_rowptr, d_cnt_or_col, d_order, d_pos,

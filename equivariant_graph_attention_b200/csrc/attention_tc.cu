@@ -1,0 +1,443 @@
+// Step 3 (+4) on tensor cores: tiles of kTileM targets share one pass over
+// the union of their neighbours.
+//
+// What is computed is exactly the on-the-fly attention of
+// "E2Former-V2：突破等变图神经网络计算瓶颈的创新架构" §3.1-§3.2 and
+// "E2Former-V2: On-the-Fly Equivariant Attention with Linear Activation
+// Memory" §2.2: per target and head a softmax of q_i.k_j/sqrt(dk) over the
+// target's own neighbours, m_i = sum_j alpha_ij h'_j accumulated on chip with
+// an online softmax, and (fused) ^h_i = m_i (x) R(r_i) by EAAS.  Nothing per
+// edge reaches memory.
+//
+// How it maps to B200: a tile of 16 spatially adjacent targets (consecutive
+// in the cell order) reads each row of the union of their neighbour lists
+// once.  One warp per head; per k-step of 16 union atoms:
+//  * the tile's union indices and membership mask are copied to shared
+//    memory once; the 16 key rows and 16 value rows of a step are staged in
+//    shared memory with cp.async (32 threads per row; rows padded by 16 bytes
+//    so ldmatrix phases hit distinct banks), kept `STAGES` steps ahead;
+//  * S = Q_h K_h^T with two mma.sync m16n8k16 (bf16 in, f32 out), the key
+//    fragments by one ldmatrix.x4;
+//  * the plan's membership bits mask S to each target's own neighbours; the
+//    online softmax keeps a per-row reference maximum raised lazily (only by
+//    more than 2^8), so z and the accumulators share one reference;
+//  * the probabilities become the bf16 A fragment directly (the S fragment
+//    layout of two n8 tiles is the A layout of one k16 step) and P V_h runs
+//    as one mma.sync per component of the head's 8 channels, the value
+//    fragments by ldmatrix.trans from the staged rows.
+// The accumulator fragment of a lane holds, for targets g and g+8 and
+// channels 2t, 2t+1 of its head, every component d — exactly what the
+// per-channel EAAS epilogue needs, so the target coupling runs from registers.
+#include <cfloat>
+
+#include "egat_device.cuh"
+#include "egat_host.h"
+
+namespace egat {
+namespace {
+
+constexpr int kRowPad = 16;   // bytes of padding per staged row
+
+struct TcParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* hp;
+  PlanView plan;
+  const int32_t* order;
+  float* out;
+  const float* pos;
+  const float* w2;
+  int n;
+  float qscale;   // log2(e) / sqrt(dk)
+  EaasTable tab;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2_t(uint32_t (&r)[2], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(addr));
+}
+// D += A B for one m16n8k16 tile, bf16 inputs, f32 accumulators
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// two floats -> bf16x2 (lo in the low half), round to nearest even; also
+// returns the rounded values so the normaliser sums exactly what the mma uses
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi, float& rlo, float& rhi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  const uint32_t u = *reinterpret_cast<const uint32_t*>(&v);
+  rlo = __uint_as_float(u << 16);
+  rhi = __uint_as_float(u & 0xffff0000u);
+  return u;
+}
+
+template <int L>
+struct TcShape {
+  static constexpr int D = (L + 1) * (L + 1);
+  static constexpr int STAGES = L >= 3 ? 2 : 3;
+};
+
+// staging buffers, then the tile's Wigner-D / |r|^l / targets, then the tile's
+// union indices [cap] and membership mask [kTileM][cap / 32]
+template <int L, int H>
+constexpr size_t tc_smem_fixed() {
+  constexpr int D = (L + 1) * (L + 1);
+  constexpr int C = 8 * H;
+  constexpr int VSTR = D * C * 2 + kRowPad;
+  constexpr int KSTR = H * 16 * 2 + kRowPad;
+  return size_t(TcShape<L>::STAGES) * kTileK * (VSTR + KSTR) +
+         size_t(kTileM) * (wig_size(L) + L + 1) * sizeof(float) + kTileM * sizeof(int);
+}
+inline size_t tc_smem_plan(int cap) {
+  return size_t(cap) * sizeof(int) + size_t(kTileM) * (cap / 32) * sizeof(uint32_t);
+}
+
+template <int L, int H, bool FUSED>
+__global__ void __launch_bounds__(H * 32, 1)
+otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
+  constexpr int D = (L + 1) * (L + 1);
+  constexpr int C = 8 * H;
+  constexpr int ROW = D * C * 2;                  // value row bytes
+  constexpr int VSTR = ROW + kRowPad;
+  constexpr int KROW = H * 16 * 2;                // key row bytes (dk = 16)
+  constexpr int KSTR = KROW + kRowPad;
+  constexpr int STAGES = TcShape<L>::STAGES;
+  constexpr int WS = wig_size(L);
+  constexpr int NTHR = H * 32;
+  constexpr int VCH = ROW / 16, KCH = KROW / 16;  // 16-byte chunks per row
+  extern __shared__ __align__(128) unsigned char smem[];
+  unsigned char* vbuf = smem;                                        // [STAGES][16][VSTR]
+  unsigned char* kbuf = vbuf + size_t(STAGES) * kTileK * VSTR;       // [STAGES][16][KSTR]
+  float* Dq = reinterpret_cast<float*>(kbuf + size_t(STAGES) * kTileK * KSTR);   // [16][WS]
+  float* rp = Dq + kTileM * WS;                                      // [16][L+1]
+  int* tgt = reinterpret_cast<int*>(rp + kTileM * (L + 1));          // [16]
+  int* su = tgt + kTileM;                                            // [cap]
+  uint32_t* smask = reinterpret_cast<uint32_t*>(su + p.plan.cap);    // [16][cap / 32]
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int h = tid >> 5;           // this warp's head
+  const int g = lane >> 2, t = lane & 3;
+  const PlanView& pv = p.plan;
+  const int words = pv.cap / 32;
+  const char* hp_bytes = reinterpret_cast<const char*>(p.hp);
+  const char* k_bytes = reinterpret_cast<const char*>(p.k);
+
+  for (int tile = blockIdx.x; tile < pv.tiles; tile += gridDim.x) {
+    const int U = pv.ulen[tile];
+    const int nsteps = (U + kTileK - 1) / kTileK;
+    const int* __restrict__ uni = pv.uni + (long long)tile * pv.cap;
+    const uint32_t* __restrict__ mrow = pv.mask + (long long)tile * kTileM * words;
+
+    if (tid < kTileM) {
+      const long long slot = (long long)tile * kTileM + tid;
+      int tg = -1;
+      if (slot < p.n) tg = p.order ? p.order[slot] : int(slot);
+      if ((unsigned)tg >= (unsigned)p.n) tg = -1;
+      tgt[tid] = tg;
+    }
+    // the tile's union indices and membership mask into shared memory
+    const int upad = nsteps * kTileK;
+    const int uw = (upad + 31) / 32;
+    for (int e = tid; e < upad; e += NTHR) su[e] = uni[e];
+    for (int e = tid; e < kTileM * uw; e += NTHR) {
+      const int r = e / uw, w = e % uw;
+      smask[r * words + w] = mrow[r * words + w];
+    }
+    __syncthreads();   // tgt, su, smask visible
+
+    // 32 threads per staged row; each copies chunks lane, lane + 32, ... of
+    // the row's value and key bytes
+    auto issue = [&](int step) {
+      const int buf = step % STAGES;
+      unsigned char* vb = vbuf + size_t(buf) * kTileK * VSTR;
+      unsigned char* kb = kbuf + size_t(buf) * kTileK * KSTR;
+      for (int r = tid >> 5; r < kTileK; r += NTHR / 32) {
+        const long long atom = su[step * kTileK + r];
+        const char* vsrc = hp_bytes + atom * ROW;
+        const char* ksrc = k_bytes + atom * KROW;
+        for (int o = lane; o < VCH + KCH; o += 32) {
+          if (o < VCH) cp_async16(smem_u32(vb + r * VSTR + o * 16), vsrc + o * 16);
+          else cp_async16(smem_u32(kb + r * KSTR + (o - VCH) * 16), ksrc + (o - VCH) * 16);
+        }
+      }
+    };
+#pragma unroll
+    for (int s = 0; s < STAGES - 1; ++s) {
+      if (s < nsteps) issue(s);
+      cp_async_commit();
+    }
+
+    // Q fragment of this head for the tile's 16 targets
+    uint32_t qa[4];
+    {
+      const int t0 = tgt[g], t1 = tgt[g + 8];
+      const uint32_t* q32 = reinterpret_cast<const uint32_t*>(p.q);
+      qa[0] = t0 >= 0 ? __ldg(q32 + ((size_t)t0 * H * 16 + h * 16 + 2 * t) / 2) : 0u;
+      qa[1] = t1 >= 0 ? __ldg(q32 + ((size_t)t1 * H * 16 + h * 16 + 2 * t) / 2) : 0u;
+      qa[2] = t0 >= 0 ? __ldg(q32 + ((size_t)t0 * H * 16 + h * 16 + 2 * t + 8) / 2) : 0u;
+      qa[3] = t1 >= 0 ? __ldg(q32 + ((size_t)t1 * H * 16 + h * 16 + 2 * t + 8) / 2) : 0u;
+    }
+    if constexpr (FUSED) {
+      // Wigner-D matrices of the tile's targets, one warp per target
+      for (int r = h; r < kTileM; r += H) {
+        const int tg = tgt[r];
+        float Q[9];
+        float rr = 0.f;
+        if (tg >= 0) rr = alignment_rotation(p.pos[3 * tg], p.pos[3 * tg + 1], p.pos[3 * tg + 2], Q);
+        else alignment_rotation(0.f, 0.f, 0.f, Q);
+        wigner_build<L>(Q, Dq + r * WS, lane, 32, [] { __syncwarp(); });
+        if (lane == 0) {
+          float a = 1.f;
+#pragma unroll
+          for (int l = 0; l <= L; ++l) {
+            rp[r * (L + 1) + l] = a;
+            a *= rr;
+          }
+        }
+      }
+    }
+
+    float acc[D][4];
+#pragma unroll
+    for (int d = 0; d < D; ++d)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[d][e] = 0.f;
+    float mref0 = -INFINITY, mref1 = -INFINITY, z0 = 0.f, z1 = 0.f;
+    constexpr float kLazy = 8.f;
+
+    for (int s = 0; s < nsteps; ++s) {
+      cp_async_wait<STAGES - 2>();
+      __syncthreads();
+      if (s + STAGES - 1 < nsteps) issue(s + STAGES - 1);
+      cp_async_commit();
+      const int buf = s % STAGES;
+      const uint32_t vb = smem_u32(vbuf + size_t(buf) * kTileK * VSTR);
+      const uint32_t kb = smem_u32(kbuf + size_t(buf) * kTileK * KSTR);
+      const int u0 = s * kTileK;
+
+      // ---- S = Q K^T for 16 union atoms
+      uint32_t kf[4];
+      {
+        const int row = (lane & 7) + 8 * (lane >> 4);
+        const int half = (lane >> 3) & 1;
+        ldsm_x4(kf, kb + row * KSTR + h * 32 + half * 16);
+      }
+      float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+      mma_bf16(s0, qa, kf[0], kf[1]);
+      mma_bf16(s1, qa, kf[2], kf[3]);
+
+      // ---- mask, online softmax (rows g and g+8 of the tile)
+      const uint32_t w0 = smask[g * words + (u0 >> 5)] >> (u0 & 31);
+      const uint32_t w1 = smask[(g + 8) * words + (u0 >> 5)] >> (u0 & 31);
+      float v[8];   // row g: cols 2t, 2t+1, 8+2t, 9+2t ; row g+8: same
+      v[0] = ((w0 >> (2 * t)) & 1u) ? s0[0] * p.qscale : -INFINITY;
+      v[1] = ((w0 >> (2 * t + 1)) & 1u) ? s0[1] * p.qscale : -INFINITY;
+      v[2] = ((w0 >> (2 * t + 8)) & 1u) ? s1[0] * p.qscale : -INFINITY;
+      v[3] = ((w0 >> (2 * t + 9)) & 1u) ? s1[1] * p.qscale : -INFINITY;
+      v[4] = ((w1 >> (2 * t)) & 1u) ? s0[2] * p.qscale : -INFINITY;
+      v[5] = ((w1 >> (2 * t + 1)) & 1u) ? s0[3] * p.qscale : -INFINITY;
+      v[6] = ((w1 >> (2 * t + 8)) & 1u) ? s1[2] * p.qscale : -INFINITY;
+      v[7] = ((w1 >> (2 * t + 9)) & 1u) ? s1[3] * p.qscale : -INFINITY;
+      float mx0 = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
+      float mx1 = fmaxf(fmaxf(v[4], v[5]), fmaxf(v[6], v[7]));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      const bool r0 = mx0 > mref0 + kLazy, r1 = mx1 > mref1 + kLazy;
+      if (__any_sync(0xffffffffu, r0 || r1)) {
+        const float sc0 = r0 ? fast_exp2(mref0 - mx0) : 1.f;
+        const float sc1 = r1 ? fast_exp2(mref1 - mx1) : 1.f;
+        z0 *= sc0;
+        z1 *= sc1;
+#pragma unroll
+        for (int d = 0; d < D; ++d) {
+          acc[d][0] *= sc0;
+          acc[d][1] *= sc0;
+          acc[d][2] *= sc1;
+          acc[d][3] *= sc1;
+        }
+        if (r0) mref0 = mx0;
+        if (r1) mref1 = mx1;
+      }
+      float pr[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) pr[e] = v[e] == -INFINITY ? 0.f : fast_exp2(v[e] - mref0);
+#pragma unroll
+      for (int e = 4; e < 8; ++e) pr[e] = v[e] == -INFINITY ? 0.f : fast_exp2(v[e] - mref1);
+      uint32_t pa[4];
+      float q0, q1, q2, q3, q4, q5, q6, q7;
+      pa[0] = pack_bf16(pr[0], pr[1], q0, q1);   // row g,   k = 2t, 2t+1
+      pa[1] = pack_bf16(pr[4], pr[5], q4, q5);   // row g+8, k = 2t, 2t+1
+      pa[2] = pack_bf16(pr[2], pr[3], q2, q3);   // row g,   k = 2t+8, 2t+9
+      pa[3] = pack_bf16(pr[6], pr[7], q6, q7);   // row g+8, k = 2t+8, 2t+9
+      z0 += (q0 + q1) + (q2 + q3);
+      z1 += (q4 + q5) + (q6 + q7);
+
+      // ---- O += P V (one n8 tile per component of this head's 8 channels)
+      {
+        const int mj = lane >> 3;                 // matrix of this lane's row address
+        const int row = (lane & 7) + 8 * (mj & 1);
+        const uint32_t base = vb + row * VSTR + h * 16;
+#pragma unroll
+        for (int d = 0; d + 1 < D; d += 2) {
+          uint32_t vf[4];
+          ldsm_x4_t(vf, base + (d + (mj >> 1)) * (C * 2));
+          mma_bf16(acc[d], pa, vf[0], vf[1]);
+          mma_bf16(acc[d + 1], pa, vf[2], vf[3]);
+        }
+        if constexpr (D % 2) {
+          uint32_t vf[2];
+          ldsm_x2_t(vf, base + (D - 1) * (C * 2));
+          mma_bf16(acc[D - 1], pa, vf[0], vf[1]);
+        }
+      }
+    }
+    cp_async_wait<0>();
+    __syncthreads();   // Dq / rp written; all staged buffers drained
+
+    // ---- epilogue: normalise; either write m or apply the target coupling
+    z0 += __shfl_xor_sync(0xffffffffu, z0, 1);
+    z0 += __shfl_xor_sync(0xffffffffu, z0, 2);
+    z1 += __shfl_xor_sync(0xffffffffu, z1, 1);
+    z1 += __shfl_xor_sync(0xffffffffu, z1, 2);
+    const float inv0 = z0 > 0.f ? 1.f / z0 : 0.f;
+    const float inv1 = z1 > 0.f ? 1.f / z1 : 0.f;
+    const int ch = h * 8 + 2 * t;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int r = g + 8 * half;
+      const int tg = tgt[r];
+      if (tg < 0) continue;
+      const float inv = half ? inv1 : inv0;
+      float* o = p.out + (size_t)tg * D * C + ch;
+      if constexpr (!FUSED) {
+#pragma unroll
+        for (int d = 0; d < D; ++d)
+          *reinterpret_cast<float2*>(o + d * C) =
+              make_float2(acc[d][2 * half] * inv, acc[d][2 * half + 1] * inv);
+      } else if constexpr (L >= 3) {
+        // register budget: one channel at a time, scalar stores
+        float rpow[L + 1];
+#pragma unroll
+        for (int l = 0; l <= L; ++l) rpow[l] = rp[r * (L + 1) + l];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float x[D];
+#pragma unroll
+          for (int d = 0; d < D; ++d) x[d] = acc[d][2 * half + e] * inv;
+          eaas_channel<L>(x, Dq + r * WS, rpow, p.tab,
+                          [&](int pp) { return __ldg(p.w2 + pp * C + ch + e); },
+                          [&](int d, float val) { o[d * C + e] = val; });
+        }
+      } else {
+        float rpow[L + 1];
+#pragma unroll
+        for (int l = 0; l <= L; ++l) rpow[l] = rp[r * (L + 1) + l];
+        float y0[D], y1[D];
+        {
+          float x[D];
+#pragma unroll
+          for (int d = 0; d < D; ++d) x[d] = acc[d][2 * half] * inv;
+          eaas_channel<L>(x, Dq + r * WS, rpow, p.tab,
+                          [&](int pp) { return __ldg(p.w2 + pp * C + ch); },
+                          [&](int d, float val) { y0[d] = val; });
+        }
+        {
+          float x[D];
+#pragma unroll
+          for (int d = 0; d < D; ++d) x[d] = acc[d][2 * half + 1] * inv;
+          eaas_channel<L>(x, Dq + r * WS, rpow, p.tab,
+                          [&](int pp) { return __ldg(p.w2 + pp * C + ch + 1); },
+                          [&](int d, float val) { y1[d] = val; });
+        }
+#pragma unroll
+        for (int d = 0; d < D; ++d) *reinterpret_cast<float2*>(o + d * C) = make_float2(y0[d], y1[d]);
+      }
+    }
+    __syncthreads();   // tgt / Dq / rp are rewritten by the next tile
+  }
+}
+
+template <int L, int H, bool FUSED>
+int launch_tc_t(const TcParams& p, int tiles, cudaStream_t st) {
+  const size_t shmem = tc_smem_fixed<L, H>() + tc_smem_plan(p.plan.cap);
+  if (shmem > 227 * 1024) return EGAT_ERR_UNSUPPORTED;
+  auto kern = otf_attention_tc_kernel<L, H, FUSED>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(shmem)) !=
+      cudaSuccess)
+    return EGAT_ERR_CUDA;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = tiles < sms ? tiles : sms;
+  kern<<<grid, H * 32, shmem, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
+}
+
+}  // namespace
+
+bool tc_attention_supported(const egat_shape& s) {
+  if (!(s.dtype == EGAT_BF16 && s.graph_mode == EGAT_GRAPH_PADDED && s.dk == 16 && s.H == 16 &&
+        s.C == 128 && s.lmax >= 1 && s.lmax <= 3))
+    return false;
+  if (plan_smem_bytes(s.n, s.K) > kPlanSmemLimit) return false;
+  const size_t fixed = s.lmax == 1 ? tc_smem_fixed<1, 16>()
+                     : s.lmax == 2 ? tc_smem_fixed<2, 16>() : tc_smem_fixed<3, 16>();
+  return fixed + tc_smem_plan(plan_capacity(s.K)) <= 227 * 1024;
+}
+
+int launch_attention_tc(const egat_shape& s, bool fused, const void* d_q, const void* d_k,
+                        const void* d_hp, const void* d_plan, const int32_t* d_order,
+                        const float* d_pos, const float* d_w2, float* d_out, cudaStream_t st) {
+  if (!tc_attention_supported(s)) return EGAT_ERR_UNSUPPORTED;
+  TcParams p;
+  p.q = static_cast<const __nv_bfloat16*>(d_q);
+  p.k = static_cast<const __nv_bfloat16*>(d_k);
+  p.hp = static_cast<const __nv_bfloat16*>(d_hp);
+  p.plan = plan_view(const_cast<void*>(d_plan), s.n, s.K);
+  p.order = d_order;
+  p.out = d_out;
+  p.pos = d_pos;
+  p.w2 = d_w2;
+  p.n = s.n;
+  p.qscale = float(1.4426950408889634 / std::sqrt(double(s.dk)));
+  if (fused) p.tab = eaas_table(s.lmax);
+  else memset(&p.tab, 0, sizeof(p.tab));
+  const int tiles = p.plan.tiles;
+  switch (s.lmax) {
+    case 1: return fused ? launch_tc_t<1, 16, true>(p, tiles, st) : launch_tc_t<1, 16, false>(p, tiles, st);
+    case 2: return fused ? launch_tc_t<2, 16, true>(p, tiles, st) : launch_tc_t<2, 16, false>(p, tiles, st);
+    case 3: return fused ? launch_tc_t<3, 16, true>(p, tiles, st) : launch_tc_t<3, 16, false>(p, tiles, st);
+    default: return EGAT_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace egat

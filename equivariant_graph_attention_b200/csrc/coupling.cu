@@ -6,11 +6,11 @@
 // Memory" §2.1 (Lemma 4.1: only m = 0 of the solid harmonic survives in the
 // aligned frame; Eq. 13: the re-index rule).
 //
-// Kernel layout: one thread per (atom, channel); a warp covers 32 channels of
-// one atom (or all 16 channels of two atoms).  The warp builds the atom's
-// Wigner-D matrices (degree 1 from the alignment rotation, higher degrees by
-// the Ivanic–Ruedenberg recursion, entries in parallel) in shared memory;
-// each lane then rotates its channel's components into the aligned frame,
+// Kernel layout: a group of C/CPL lanes per atom, each lane owning CPL
+// consecutive channels.  The group builds the atom's Wigner-D matrices
+// (degree 1 from the alignment rotation, higher degrees by the
+// Ivanic–Ruedenberg recursion, entries in parallel) in shared memory once;
+// each lane then rotates its channels' components into the aligned frame,
 // applies the sparse re-index with the path weights, and rotates back.
 // Memory traffic is one read of h and one write of h' (streaming, HBM-bound).
 #include <cmath>
@@ -104,94 +104,130 @@ struct EaasParams {
   EaasTable tab;
 };
 
-// One warp owns a block of G = min(C, 32) channels of 32/G atoms at a time
-// (lane = channel, so every load and store of a component row is coalesced).
-// The warp's channel block is fixed, so the path weights of its lane's channel
-// stay in registers.  Each warp builds the Wigner-D matrices of its atoms in
-// its own shared-memory slot with warp-level synchronisation only, and the
-// next atom's position and features are fetched before the current atom is
-// coupled.
+// CPL consecutive channels of one component row (vector load / store).
+template <typename T, int CPL>
+struct ChanVec;
+template <>
+struct ChanVec<__nv_bfloat16, 4> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[4]) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    v[0] = __uint_as_float(u.x << 16); v[1] = __uint_as_float(u.x & 0xffff0000u);
+    v[2] = __uint_as_float(u.y << 16); v[3] = __uint_as_float(u.y & 0xffff0000u);
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[4]) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&a);
+    u.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = u;
+  }
+};
+template <>
+struct ChanVec<__nv_bfloat16, 2> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[2]) {
+    const uint32_t u = __ldg(reinterpret_cast<const unsigned int*>(p));
+    v[0] = __uint_as_float(u << 16); v[1] = __uint_as_float(u & 0xffff0000u);
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[2]) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
+    *reinterpret_cast<__nv_bfloat162*>(p) = a;
+  }
+};
+template <>
+struct ChanVec<float, 4> {
+  static __device__ __forceinline__ void load(const float* p, float (&v)[4]) {
+    const float4 u = __ldg(reinterpret_cast<const float4*>(p));
+    v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+  }
+  static __device__ __forceinline__ void store(float* p, const float (&v)[4]) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+};
+template <>
+struct ChanVec<float, 2> {
+  static __device__ __forceinline__ void load(const float* p, float (&v)[2]) {
+    const float2 u = __ldg(reinterpret_cast<const float2*>(p));
+    v[0] = u.x; v[1] = u.y;
+  }
+  static __device__ __forceinline__ void store(float* p, const float (&v)[2]) {
+    *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+  }
+};
+
+// A group of G = C/CPL lanes owns one atom; each lane owns CPL consecutive
+// channels (CPL = 4 up to lmax 2, 2 at lmax 3 for the register budget), so
+// component rows move in 8-16 byte vectors.  The group builds the atom's
+// Wigner-D matrices once in shared memory (groups of up to 32 lanes inside a
+// warp; a 64-lane group spans two warps, each building its own copy), then
+// every lane couples its channels with the matrices held in registers.
 template <int L, typename T>
 __global__ void __launch_bounds__(kEaasWarps * 32, (L >= 3 ? 1 : 2))
 eaas_source_kernel(const __grid_constant__ EaasParams p) {
   constexpr int D = (L + 1) * (L + 1);
-  constexpr int NP = num_paths(L);
   constexpr int WS = wig_size(L);
-  __shared__ float Dsm[kEaasWarps][2][WS];   // up to 2 atoms per warp (C = 16)
+  constexpr int CPL = L >= 3 ? 2 : 4;
+  constexpr int kMaxSlots = 32 / 4;              // C >= 16 -> G >= 4 lanes
+  __shared__ float Dsm[kEaasWarps][kMaxSlots][WS];
 
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
   const int C = p.C;
-  const int G = C < 32 ? C : 32;          // lanes per atom
-  const int AW = 32 / G;                  // atoms per warp (1 or 2)
-  const int slot = lane / G;              // which of the warp's atoms
-  const int g = lane % G;
-  const int nblk = C / G;                 // channel blocks per atom
+  const int G = C / CPL;                        // lanes per atom
+  const int WPA = G > 32 ? G / 32 : 1;          // warps per atom
+  const int GW = G > 32 ? 32 : G;               // lanes of this warp in the group
+  const int AW = 32 / GW;                       // atoms per warp
+  const int slot = lane / GW;
+  const int gl = lane % GW;                     // lane within the warp's part of the group
   const long long gwarp = (long long)blockIdx.x * kEaasWarps + wib;
   const long long nwarps = (long long)gridDim.x * kEaasWarps;
-  const int cb = int(gwarp % nblk);
-  const int c = cb * G + g;               // this lane's channel
+  const int part = int(gwarp % WPA);            // which warp of the atom's group
+  const int c0 = (part * 32 + gl) * CPL;         // first channel of this lane
   const long long ngroups = ((long long)p.n + AW - 1) / AW;
   const T* __restrict__ x = static_cast<const T*>(p.x);
   T* __restrict__ y = static_cast<T*>(p.y);
-
-  // weights of this lane's channel: registers up to lmax 2, L1-cached loads above
-  constexpr bool kRegW = NP <= 15;
-  float wreg[kRegW ? NP : 1];
-#pragma unroll
-  for (int q = 0; q < (kRegW ? NP : 0); ++q) wreg[q] = __ldg(p.w + q * C + c);
-  const float* __restrict__ wcol = p.w + c;
-
   float* Dme = Dsm[wib][slot];
-  long long grp = gwarp / nblk;
-  const long long gstride = nwarps / nblk;   // launch keeps nwarps a multiple of nblk
 
-  // prefetch the first atom
-  float px = 0.f, py = 0.f, pz = 0.f, xin[D];
-  auto fetch = [&](long long gr, float& fx, float& fy, float& fz, float (&xv)[D]) {
-    const long long at = gr * AW + slot;
-    if (gr < ngroups && at < p.n) {
-      fx = __ldg(p.pos + 3 * at);
-      fy = __ldg(p.pos + 3 * at + 1);
-      fz = __ldg(p.pos + 3 * at + 2);
-      const T* xr = x + (size_t)at * D * C + c;
-#pragma unroll
-      for (int d = 0; d < D; ++d) xv[d] = load_one<T>(xr + d * C);
-    }
-  };
-  fetch(grp, px, py, pz, xin);
-  // lmax 3 keeps no second feature row in flight (register budget)
-  constexpr bool kPrefetch = L <= 2;
-  for (; grp < ngroups; grp += gstride) {
+  for (long long grp = gwarp / WPA; grp < ngroups; grp += nwarps / WPA) {
     const long long at = grp * AW + slot;
-    float nx = 0.f, ny = 0.f, nz = 0.f, xnext[kPrefetch ? D : 1];
-    if constexpr (kPrefetch) fetch(grp + gstride, nx, ny, nz, xnext);
+    const bool live = at < p.n;
     float Q[9];
-    const float r = alignment_rotation(px, py, pz, Q);
+    float r = 0.f;
+    if (live) r = alignment_rotation(__ldg(p.pos + 3 * at), __ldg(p.pos + 3 * at + 1),
+                                     __ldg(p.pos + 3 * at + 2), Q);
+    else alignment_rotation(0.f, 0.f, 0.f, Q);
+    float xv[CPL][D];
+    if (live) {
+      const T* xr = x + (size_t)at * D * C + c0;
+#pragma unroll
+      for (int d = 0; d < D; ++d) {
+        float v[CPL];
+        ChanVec<T, CPL>::load(xr + d * C, v);
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) xv[k][d] = v[k];
+      }
+    }
     float rpow[L + 1];
     rpow[0] = 1.f;
 #pragma unroll
     for (int l = 1; l <= L; ++l) rpow[l] = rpow[l - 1] * r;
     __syncwarp();                             // previous atom's readers are done
-    wigner_build<L>(Q, Dme, g, G, [] { __syncwarp(); });
-    if (at < p.n) {
-      T* yr = y + (size_t)at * D * C + c;
-      eaas_channel<L>(
-          xin, Dme, rpow, p.tab,
-          [&](int q) {
-            if constexpr (kRegW) return wreg[q];
-            else return __ldg(wcol + q * C);
-          },
-          [&](int d, float v) { store_one<T>(yr + d * C, v); });
-    }
-    if constexpr (kPrefetch) {
-      px = nx;
-      py = ny;
-      pz = nz;
+    wigner_build<L>(Q, Dme, gl, GW, [] { __syncwarp(); });
+    if (live) {
+      float yv[CPL][D];
 #pragma unroll
-      for (int d = 0; d < D; ++d) xin[d] = xnext[d];
-    } else {
-      fetch(grp + gstride, px, py, pz, xin);
+      for (int k = 0; k < CPL; ++k) {
+        const float* __restrict__ wcol = p.w + c0 + k;
+        eaas_channel<L>(xv[k], Dme, rpow, p.tab, [&](int q) { return __ldg(wcol + q * C); },
+                        [&](int d, float v) { yv[k][d] = v; });
+      }
+      T* yr = y + (size_t)at * D * C + c0;
+#pragma unroll
+      for (int d = 0; d < D; ++d) {
+        float v[CPL];
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) v[k] = yv[k][d];
+        ChanVec<T, CPL>::store(yr + d * C, v);
+      }
     }
   }
 }
@@ -207,17 +243,16 @@ int launch_eaas_t(const egat_shape& s, const void* d_x, const float* d_pos, cons
   p.n = s.n;
   p.C = s.C;
   p.tab = eaas_table(L);
-  const int G = s.C < 32 ? s.C : 32;
-  const int nblk = s.C / G;
-  const long long groups = ((long long)s.n + (32 / G) - 1) / (32 / G);
+  constexpr int CPL = L >= 3 ? 2 : 4;
+  const int G = s.C / CPL;
+  const int WPA = G > 32 ? G / 32 : 1;
+  const int AW = 32 / (G > 32 ? 32 : G);
+  const long long groups = ((long long)s.n + AW - 1) / AW;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // warps needed: one per (atom group, channel block); cap at 8 resident blocks per SM
-  const long long want = (groups * nblk + kEaasWarps - 1) / kEaasWarps;
-  int grid = int(std::max<long long>(1, std::min<long long>(want, (long long)sms * 8)));
-  // keep the total warp count a multiple of the channel-block count
-  while ((long long)grid * kEaasWarps % nblk) ++grid;
+  const long long want = (groups * WPA + kEaasWarps - 1) / kEaasWarps;
+  const int grid = int(std::max<long long>(1, std::min<long long>(want, (long long)sms * 8)));
   eaas_source_kernel<L, T><<<grid, kEaasWarps * 32, 0, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
 }

@@ -32,6 +32,7 @@ struct GraphWs {
   int* bucket_start;   // [M + 1]
   int* cursor;         // [M]
   int* deg;            // [n] untruncated degree
+  int* trunc;          // [1 + n]: count, then sorted slots of rows with > K neighbours
   int* partial;        // scan partials
   size_t bytes;
 };
@@ -67,6 +68,7 @@ GraphWs carve(void* base, int n) {
   w.bucket_start = static_cast<int*>(take(sizeof(int) * (M + 1)));
   w.cursor = static_cast<int*>(take(sizeof(int) * M));
   w.deg = static_cast<int*>(take(sizeof(int) * size_t(n)));
+  w.trunc = static_cast<int*>(take(sizeof(int) * (size_t(n) + 1)));
   w.partial = static_cast<int*>(take(sizeof(int) * (nparts + 1)));
   w.bytes = off;
   return w;
@@ -347,19 +349,15 @@ __device__ __forceinline__ void warp_bitonic_sort(unsigned long long* keys, int 
 }
 
 // Padded list, one warp per atom (atoms taken in cell order).  One sweep
-// writes the first K neighbours and counts all of them.  A row with more than
-// K neighbours finds the key (d^2 << shift | j) of its K-th nearest — by a
-// shared-memory sort of all its keys when they fit, by bisection otherwise —
-// and is rewritten with exactly the keys up to it (ties to smaller j).  Row
-// order is the sweep order: the 125 cells in a fixed order, atoms of a cell
-// by index — deterministic, independent of thread scheduling.
-__global__ void __launch_bounds__(kFillWarps * 32)
+// writes the first K neighbours and counts all of them; an atom with more
+// than K is appended to the truncation list for fix_truncated.  Row order is
+// the sweep order: the 125 cells in a fixed order, atoms of a cell by index —
+// deterministic, independent of thread scheduling.
+__global__ void __launch_bounds__(kFillWarps * 32, 12)
 fill_padded(Search s, int n, int K, int32_t* __restrict__ nbr, int32_t* __restrict__ cnt,
-            int* __restrict__ overflow) {
-  __shared__ unsigned long long keys_all[kFillWarps][kSelectCap];
+            int* __restrict__ trunc) {
   const int lane = threadIdx.x & 31;
-  const int wib = threadIdx.x >> 5;
-  const int w = blockIdx.x * kFillWarps + wib;
+  const int w = blockIdx.x * kFillWarps + (threadIdx.x >> 5);
   if (w >= n) return;
   const int4 p = s.spos[w];
   const int4 c = s.scell[w];
@@ -371,28 +369,52 @@ fill_padded(Search s, int n, int K, int32_t* __restrict__ nbr, int32_t* __restri
     if (hit && pos < K) row[pos] = j;
     total += __popc(m);
   });
-  if (total > K) {
+  const int take = total < K ? total : K;
+  for (int t = take + lane; t < K; t += 32) row[t] = -1;
+  if (lane == 0) {
+    cnt[p.w] = take;
+    if (total > K) trunc[1 + atomicAdd(&trunc[0], 1)] = w;
+  }
+}
+
+// Rows with more than K neighbours, one warp per listed atom (persistent
+// warps; the loop is bounded by the device-side count).  The key
+// (d^2 << shift | j) of the K-th nearest comes from a shared-memory sort of
+// all the atom's keys when they fit, by bisection otherwise; the row is then
+// rewritten, in sweep order, with exactly the keys up to it (ties to smaller j).
+__global__ void __launch_bounds__(kFillWarps * 32)
+fix_truncated(Search s, int K, int32_t* __restrict__ nbr, const int* __restrict__ trunc,
+              int* __restrict__ overflow) {
+  __shared__ unsigned long long keys_all[kFillWarps][kSelectCap];
+  const int lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
+  const int ntr = trunc[0];
+  for (int t = blockIdx.x * kFillWarps + wib; t < ntr; t += gridDim.x * kFillWarps) {
+    const int w = trunc[1 + t];
+    const int4 p = s.spos[w];
+    const int4 c = s.scell[w];
+    int32_t* row = nbr + (long long)p.w * K;
+    unsigned long long* keys = keys_all[wib];
+    int total = 0;
+    for_each_neighbour(s, p, c, [&](bool hit, int j, long long d2) {
+      const unsigned m = __ballot_sync(0xffffffffu, hit);
+      const int pos = total + __popc(m & ((1u << lane) - 1u));
+      if (hit && pos < kSelectCap)
+        keys[pos] = (((unsigned long long)d2) << s.key_shift) | (unsigned long long)j;
+      total += __popc(m);
+    });
     unsigned long long thresh;
     if (total <= kSelectCap) {
-      unsigned long long* keys = keys_all[wib];
-      int filled = 0;
-      for_each_neighbour(s, p, c, [&](bool hit, int j, long long d2) {
-        const unsigned m = __ballot_sync(0xffffffffu, hit);
-        const int pos = filled + __popc(m & ((1u << lane) - 1u));
-        if (hit && pos < kSelectCap)
-          keys[pos] = (((unsigned long long)d2) << s.key_shift) | (unsigned long long)j;
-        filled += __popc(m);
-      });
       int size = 1;
       while (size < total) size <<= 1;
-      for (int t = total + lane; t < size; t += 32) keys[t] = ~0ull;
+      for (int q = total + lane; q < size; q += 32) keys[q] = ~0ull;
       __syncwarp();
       warp_bitonic_sort(keys, size);
       thresh = keys[K - 1];
-      __syncwarp();
     } else {
       thresh = kth_key(s, p, c, K);
     }
+    __syncwarp();
     int written = 0;
     for_each_neighbour(s, p, c, [&](bool hit, int j, long long d2) {
       const bool keep = hit && ((((unsigned long long)d2) << s.key_shift) |
@@ -402,12 +424,7 @@ fill_padded(Search s, int n, int K, int32_t* __restrict__ nbr, int32_t* __restri
       if (keep && pos < K) row[pos] = j;
       written += __popc(m);
     });
-  }
-  const int take = total < K ? total : K;
-  for (int t = take + lane; t < K; t += 32) row[t] = -1;
-  if (lane == 0) {
-    cnt[p.w] = take;
-    if (total > K) atomicAdd(overflow, total - K);
+    if (lane == 0) atomicAdd(overflow, total - K);
   }
 }
 
@@ -461,7 +478,12 @@ int build_graph(const int32_t* d_pos_q, int n, int cutoff_q, int K, int mode,
   Search s{w.spos, w.scell, w.bucket_start, bits, (long long)cutoff_q * cutoff_q, key_shift};
   const unsigned nfill = unsigned((n + kFillWarps - 1) / kFillWarps);
   if (mode == EGAT_GRAPH_PADDED) {
-    fill_padded<<<nfill, kFillWarps * 32, 0, st>>>(s, n, K, d_a, d_b, d_overflow);
+    if (cudaMemsetAsync(w.trunc, 0, sizeof(int), st) != cudaSuccess) return EGAT_ERR_CUDA;
+    fill_padded<<<nfill, kFillWarps * 32, 0, st>>>(s, n, K, d_a, d_b, w.trunc);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    fix_truncated<<<sms * 2, kFillWarps * 32, 0, st>>>(s, K, d_a, w.trunc, d_overflow);
   } else {
     const long long nthreads = (long long)n * 32;
     count_neighbours<<<unsigned((nthreads + tb - 1) / tb), tb, 0, st>>>(s, n, w.deg);

@@ -1,0 +1,209 @@
+// Attention plan for the tensor-core attention path: targets in tiles of
+// kTileM consecutive atoms of the traversal order, and per tile the sorted
+// union of their neighbour lists with a (target x union) membership bitmask.
+//
+// The streaming attention of "E2Former-V2：突破等变图神经网络计算瓶颈的创新架构"
+// §3.2 processes each target independently; grouping spatially adjacent
+// targets (the cell order of the graph builder) lets one tile read each
+// neighbour row once for all of its targets, and the membership mask keeps
+// the softmax exactly over each target's own neighbour list.
+//
+// One 256-thread CTA per tile builds the union from a shared-memory bitmap
+// over atom indices (ascending atom index: a deterministic order) and sets one
+// mask bit per (target, neighbour) at the position given by the bitmap's
+// prefix counts.
+#include "egat_device.cuh"
+#include "egat_host.h"
+
+namespace egat {
+namespace {
+
+constexpr int kPlanThreads = 256;
+
+struct PlanParams {
+  const int32_t* nbr;    // [n][K]
+  const int32_t* cnt;    // [n] or null (then every slot is scanned, -1 skipped)
+  const int32_t* order;  // [n] or null
+  PlanView plan;
+  int n, K;
+};
+
+// One CTA per tile.  Shared memory holds a bitmap over all atom indices
+// (bit j set when atom j is a neighbour of some target of the tile), the
+// per-word prefix counts of that bitmap, and the tile's membership mask.
+//  1. set the bits of every neighbour of the tile's targets;
+//  2. prefix-count the bitmap's words: the union, in ascending atom index, is
+//     read straight off the bitmap, and the union position of atom j is
+//     prefix[j / 32] + popcount(bits of word j / 32 below j);
+//  3. one membership bit per (target, neighbour) at that position.
+// Cost per tile is O(n / 32) words plus O(16 K) entries; deterministic.
+__global__ void __launch_bounds__(kPlanThreads) build_plan_kernel(const __grid_constant__ PlanParams p) {
+  extern __shared__ uint32_t sm[];
+  const PlanView& pv = p.plan;
+  const int cap = pv.cap;                         // >= kTileM * K, power of two
+  const int words = cap / 32;                     // mask words per target row
+  const int nw = (p.n + 31) / 32;                 // bitmap words
+  uint32_t* bitmap = sm;                          // [nw]
+  uint32_t* prefix = sm + nw;                     // [nw]
+  uint32_t* mask = sm + 2 * nw;                   // [kTileM][words]
+  __shared__ int tgt[kTileM], off[kTileM + 1];
+  __shared__ int warp_sum[kPlanThreads / 32];
+  __shared__ int s_unique;
+  const int tile = blockIdx.x;
+
+  if (threadIdx.x < kTileM) {
+    const long long slot = (long long)tile * kTileM + threadIdx.x;
+    int t = -1;
+    if (slot < p.n) t = p.order ? p.order[slot] : int(slot);
+    if ((unsigned)t >= (unsigned)p.n) t = -1;
+    tgt[threadIdx.x] = t;
+  }
+  for (int i = threadIdx.x; i < nw; i += blockDim.x) bitmap[i] = 0u;
+  for (int i = threadIdx.x; i < kTileM * words; i += blockDim.x) mask[i] = 0u;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int sum = 0;
+    for (int r = 0; r < kTileM; ++r) {
+      off[r] = sum;
+      int c = 0;
+      if (tgt[r] >= 0) {
+        c = p.cnt ? p.cnt[tgt[r]] : p.K;
+        c = c < 0 ? 0 : (c > p.K ? p.K : c);
+      }
+      sum += c;
+    }
+    off[kTileM] = sum;
+  }
+  __syncthreads();
+  const int total = off[kTileM];
+  auto entry = [&](int e, int& r) {
+    r = 0;
+    while (r + 1 < kTileM && off[r + 1] <= e) ++r;
+    return p.nbr[(long long)tgt[r] * p.K + (e - off[r])];
+  };
+  // 1. bitmap of the union
+  for (int e = threadIdx.x; e < total; e += blockDim.x) {
+    int r;
+    const int j = entry(e, r);
+    if ((unsigned)j < (unsigned)p.n) atomicOr(&bitmap[j >> 5], 1u << (j & 31));
+  }
+  __syncthreads();
+  // 2. per-word exclusive prefix counts (contiguous chunk per thread + block scan)
+  const int per = (nw + kPlanThreads - 1) / kPlanThreads;
+  const int w0 = threadIdx.x * per;
+  const int w1 = min(w0 + per, nw);
+  int mine = 0;
+  for (int w = w0; w < w1; ++w) mine += __popc(bitmap[w]);
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_sum[wid] = incl;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int w = 0; w < kPlanThreads / 32; ++w) {
+      const int v = warp_sum[w];
+      warp_sum[w] = acc;
+      acc += v;
+    }
+    s_unique = acc;
+  }
+  __syncthreads();
+  const int U = s_unique;
+  int* uni = pv.uni + (long long)tile * cap;
+  {
+    int pos = warp_sum[wid] + incl - mine;
+    for (int w = w0; w < w1; ++w) {
+      prefix[w] = uint32_t(pos);
+      uint32_t b = bitmap[w];
+      while (b) {
+        const int bit = __ffs(b) - 1;
+        uni[pos++] = w * 32 + bit;
+        b &= b - 1;
+      }
+    }
+  }
+  __syncthreads();
+  // pad the union to a multiple of the k-step with a valid index (masked out)
+  const int upad = (U + kTileK - 1) / kTileK * kTileK;
+  const int filler = U > 0 ? uni[0] : 0;
+  for (int e = U + threadIdx.x; e < upad; e += blockDim.x) uni[e] = filler;
+  if (threadIdx.x == 0) pv.ulen[tile] = U;
+  // 3. membership bits
+  for (int e = threadIdx.x; e < total; e += blockDim.x) {
+    int r;
+    const int j = entry(e, r);
+    if ((unsigned)j >= (unsigned)p.n) continue;
+    const int pos = int(prefix[j >> 5]) + __popc(bitmap[j >> 5] & ((1u << (j & 31)) - 1u));
+    atomicOr(&mask[r * words + (pos >> 5)], 1u << (pos & 31));
+  }
+  __syncthreads();
+  uint32_t* gmask = pv.mask + (long long)tile * kTileM * words;
+  const int uw = (upad + 31) / 32;
+  for (int i = threadIdx.x; i < kTileM * uw; i += blockDim.x) {
+    const int r = i / uw, w = i % uw;
+    gmask[r * words + w] = mask[r * words + w];
+  }
+}
+
+}  // namespace
+
+size_t plan_smem_bytes(int n, int K) {
+  const size_t nw = (size_t(n) + 31) / 32;
+  return 2 * nw * sizeof(uint32_t) + size_t(kTileM) * (plan_capacity(K) / 32) * sizeof(uint32_t);
+}
+
+int plan_capacity(int K) {
+  int cap = 32;
+  while (cap < kTileM * K) cap <<= 1;
+  return cap;
+}
+
+size_t plan_bytes(int n, int K) {
+  const size_t tiles = (size_t(n) + kTileM - 1) / kTileM;
+  const size_t cap = size_t(plan_capacity(K));
+  auto a256 = [](size_t x) { return (x + 255) & ~size_t(255); };
+  return a256(tiles * sizeof(int)) + a256(tiles * cap * sizeof(int)) +
+         a256(tiles * kTileM * (cap / 32) * sizeof(uint32_t));
+}
+
+PlanView plan_view(void* base, int n, int K) {
+  const size_t tiles = (size_t(n) + kTileM - 1) / kTileM;
+  const int cap = plan_capacity(K);
+  auto a256 = [](size_t x) { return (x + 255) & ~size_t(255); };
+  PlanView v;
+  char* b = static_cast<char*>(base);
+  v.ulen = reinterpret_cast<int*>(b);
+  b += a256(tiles * sizeof(int));
+  v.uni = reinterpret_cast<int*>(b);
+  b += a256(tiles * size_t(cap) * sizeof(int));
+  v.mask = reinterpret_cast<uint32_t*>(b);
+  v.cap = cap;
+  v.tiles = int(tiles);
+  return v;
+}
+
+int launch_build_plan(int n, int K, const int32_t* d_nbr, const int32_t* d_cnt,
+                      const int32_t* d_order, void* d_plan, cudaStream_t st) {
+  PlanParams p;
+  p.nbr = d_nbr;
+  p.cnt = d_cnt;
+  p.order = d_order;
+  p.plan = plan_view(d_plan, n, K);
+  p.n = n;
+  p.K = K;
+  const size_t shmem = plan_smem_bytes(n, K);
+  if (shmem > 48 * 1024) {
+    if (cudaFuncSetAttribute(build_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(shmem)) != cudaSuccess)
+      return EGAT_ERR_CUDA;
+  }
+  build_plan_kernel<<<p.plan.tiles, kPlanThreads, shmem, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
+}
+
+}  // namespace egat

@@ -37,7 +37,8 @@ EGAT_GRAPH_CSR = 1
 EXPORTS = ["egat_version", "egat_strerror", "egat_num_paths", "egat_graph_workspace_bytes",
            "egat_build_graph", "egat_eaas_couple", "egat_otf_attention",
            "egat_otf_attention_coupled",
-           "egat_forward_workspace_bytes", "egat_forward", "egat_forward_noalloc"]
+           "egat_forward_workspace_bytes", "egat_forward", "egat_forward_noalloc",
+           "egat_attention_plan_bytes", "egat_build_attention_plan", "egat_otf_attention_tiled"]
 
 
 class EgatError(RuntimeError):
@@ -88,6 +89,12 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.egat_forward_workspace_bytes.argtypes = [sp, ctypes.POINTER(sz)]
     lib.egat_forward.restype = ctypes.c_int
     lib.egat_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
+    lib.egat_attention_plan_bytes.restype = ctypes.c_int
+    lib.egat_attention_plan_bytes.argtypes = [sp, ctypes.POINTER(sz)]
+    lib.egat_build_attention_plan.restype = ctypes.c_int
+    lib.egat_build_attention_plan.argtypes = [sp, vp, vp, vp, vp, sz, vp]
+    lib.egat_otf_attention_tiled.restype = ctypes.c_int
+    lib.egat_otf_attention_tiled.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp]
     lib.egat_forward_noalloc.restype = ctypes.c_int
     lib.egat_forward_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     if path is None:
@@ -245,6 +252,45 @@ def egat_otf_attention_coupled(shape: Shape, q: torch.Tensor, k: torch.Tensor, h
         ctypes.byref(cs), _ptr(q), _ptr(k), _ptr(hp), _ptr(nbr_or_rowptr), _ptr(cnt_or_col),
         _ptr(order), _ptr(pos), _ptr(w2), _ptr(out), _stream(stream))
     _check("egat_otf_attention_coupled", rc)
+    return out
+
+
+def egat_attention_plan_bytes(shape: Shape) -> int:
+    out = ctypes.c_size_t(0)
+    cs = shape.c()
+    _check("egat_attention_plan_bytes",
+           load_library().egat_attention_plan_bytes(ctypes.byref(cs), ctypes.byref(out)))
+    return out.value
+
+
+def egat_build_attention_plan(shape: Shape, nbr: torch.Tensor, cnt: Optional[torch.Tensor],
+                              order: Optional[torch.Tensor] = None,
+                              plan: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Per-tile neighbour unions and membership masks for egat_otf_attention_tiled."""
+    nb = egat_attention_plan_bytes(shape)
+    if plan is None:
+        plan = torch.empty(max(nb, 16), dtype=torch.uint8, device=nbr.device)
+    cs = shape.c()
+    rc = load_library().egat_build_attention_plan(ctypes.byref(cs), _ptr(nbr), _ptr(cnt),
+                                                  _ptr(order), _ptr(plan), plan.numel(),
+                                                  _stream(stream))
+    _check("egat_build_attention_plan", rc)
+    return plan
+
+
+def egat_otf_attention_tiled(shape: Shape, q: torch.Tensor, k: torch.Tensor, hp: torch.Tensor,
+                             plan: torch.Tensor, order: Optional[torch.Tensor] = None,
+                             pos: Optional[torch.Tensor] = None, w2: Optional[torch.Tensor] = None,
+                             fused: bool = True, out: Optional[torch.Tensor] = None,
+                             stream=None) -> torch.Tensor:
+    """Tensor-core attention over a plan: ^h (fused) or m, float32 [n, D, C]."""
+    if out is None:
+        out = torch.empty((shape.n, shape.D, shape.C), dtype=torch.float32, device=hp.device)
+    cs = shape.c()
+    rc = load_library().egat_otf_attention_tiled(
+        ctypes.byref(cs), _ptr(q), _ptr(k), _ptr(hp), _ptr(plan), _ptr(order), _ptr(pos),
+        _ptr(w2), _ptr(out), 1 if fused else 0, _stream(stream))
+    _check("egat_otf_attention_tiled", rc)
     return out
 
 

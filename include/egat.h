@@ -183,10 +183,45 @@ EGAT_API int egat_otf_attention_coupled(const egat_shape* s, const void* d_q, co
                                         void* stream);
 
 /*
+ * Tensor-core attention (steps 3 and 3+4 for bf16 storage, padded graphs,
+ * C = 128, H = 16, dk = 16; other shapes return EGAT_ERR_UNSUPPORTED and use
+ * egat_otf_attention / egat_otf_attention_coupled).  Targets are taken in
+ * tiles of 16 consecutive entries of d_order (identity when NULL); one tile
+ * streams the union of its targets' neighbour lists once through shared
+ * memory and computes, per head, S = Q K^T and O += P V with bf16 mma.sync
+ * (fp32 accumulation), the softmax restricted to each target's own
+ * neighbours by a membership mask.  Same result as the per-target kernel up
+ * to rounding: the softmax weights enter the P V product as bf16.
+ *
+ * egat_attention_plan_bytes / egat_build_attention_plan: per tile, the
+ * union of the 16 targets' neighbour lists in ascending atom index and a
+ * (16 x union) membership bitmask, built from the padded list (d_nbr, d_cnt —
+ * d_cnt may be NULL) and d_order into caller memory d_plan of at least the
+ * queried size.  The builder keeps a bitmap over all n atoms per tile in
+ * shared memory, so it supports n up to about 800,000 atoms (2 * n / 8 bytes
+ * plus the tile mask within 200 KiB; larger n returns EGAT_ERR_UNSUPPORTED
+ * and egat_forward falls back to the per-target kernel).  The plan depends
+ * only on the graph; it is reused by every attention call on it.
+ * egat_otf_attention_tiled: fused = 1 writes ^h (d_pos, d_w2 required),
+ * fused = 0 writes m; d_order must be the array the plan was built with.
+ */
+EGAT_API int egat_attention_plan_bytes(const egat_shape* s, size_t* bytes);
+EGAT_API int egat_build_attention_plan(const egat_shape* s, const int32_t* d_nbr,
+                                       const int32_t* d_cnt, const int32_t* d_order,
+                                       void* d_plan, size_t plan_bytes, void* stream);
+EGAT_API int egat_otf_attention_tiled(const egat_shape* s, const void* d_q, const void* d_k,
+                                      const void* d_hp, const void* d_plan,
+                                      const int32_t* d_order, const float* d_pos,
+                                      const float* d_w2, float* d_out, int32_t fused,
+                                      void* stream);
+
+/*
  * Steps 2-4 — the fused forward pass ([EX] §3.1):
- *   h' = EAAS(h, r, w1) into workspace;  then one kernel per target streams
- *   its neighbours (step 3) and applies ^h_i = EAAS(m_i, r_i, w2) to the
- *   on-chip m_i before writing ^h_i.
+ *   h' = EAAS(h, r, w1) into workspace;  then the attention kernel streams
+ *   each target's neighbours (step 3) and applies ^h_i = EAAS(m_i, r_i, w2) to
+ *   the on-chip m_i before writing ^h_i.  Shapes the tensor-core path
+ *   supports build the attention plan into the workspace and use
+ *   egat_otf_attention_tiled; the others use the per-target kernel.
  *  d_out  float32 [n][D][C];  d_ws at least egat_forward_workspace_bytes(s).
  */
 EGAT_API int egat_forward_workspace_bytes(const egat_shape* s, size_t* bytes);
