@@ -20,7 +20,9 @@
 //    fragments by one ldmatrix.x4;
 //  * the plan's membership bits mask S to each target's own neighbours; the
 //    online softmax keeps a per-row reference maximum raised lazily (only by
-//    more than 2^8), so z and the accumulators share one reference;
+//    more than 2^8), so z and the accumulators share one reference; z is the
+//    mma of P with an all-ones fragment — the row sums of exactly the bf16
+//    weights that enter P V;
 //  * the probabilities become the bf16 A fragment directly (the S fragment
 //    layout of two n8 tiles is the A layout of one k16 step) and P V_h runs
 //    as one mma.sync per component of the head's 8 channels, the value
@@ -87,20 +89,15 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-// two floats -> bf16x2 (lo in the low half), round to nearest even; also
-// returns the rounded values so the normaliser sums exactly what the mma uses
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi, float& rlo, float& rhi) {
-  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  const uint32_t u = *reinterpret_cast<const uint32_t*>(&v);
-  rlo = __uint_as_float(u << 16);
-  rhi = __uint_as_float(u & 0xffff0000u);
-  return u;
-}
 
+// A pipeline stage holds KS k-steps (KS * kTileK union rows): one barrier per
+// stage; STAGES stages are in flight.
 template <int L>
 struct TcShape {
   static constexpr int D = (L + 1) * (L + 1);
-  static constexpr int STAGES = L >= 3 ? 2 : 3;
+  static constexpr int KS = L >= 3 ? 1 : 2;
+  static constexpr int STAGES = L >= 3 ? 2 : (L == 2 ? 2 : 3);
+  static constexpr int RS = KS * kTileK;   // rows per stage
 };
 
 // staging buffers, then the tile's Wigner-D / |r|^l / targets, then the tile's
@@ -111,11 +108,12 @@ constexpr size_t tc_smem_fixed() {
   constexpr int C = 8 * H;
   constexpr int VSTR = D * C * 2 + kRowPad;
   constexpr int KSTR = H * 16 * 2 + kRowPad;
-  return size_t(TcShape<L>::STAGES) * kTileK * (VSTR + KSTR) +
+  return size_t(TcShape<L>::STAGES) * TcShape<L>::RS * (VSTR + KSTR) +
          size_t(kTileM) * (wig_size(L) + L + 1) * sizeof(float) + kTileM * sizeof(int);
 }
+// mask rows are padded by one word so the 8 rows a warp reads sit in distinct banks
 inline size_t tc_smem_plan(int cap) {
-  return size_t(cap) * sizeof(int) + size_t(kTileM) * (cap / 32) * sizeof(uint32_t);
+  return size_t(cap) * sizeof(int) + size_t(kTileM) * (cap / 32 + 1) * sizeof(uint32_t);
 }
 
 template <int L, int H, bool FUSED>
@@ -128,17 +126,19 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
   constexpr int KROW = H * 16 * 2;                // key row bytes (dk = 16)
   constexpr int KSTR = KROW + kRowPad;
   constexpr int STAGES = TcShape<L>::STAGES;
+  constexpr int KS = TcShape<L>::KS;
+  constexpr int RS = TcShape<L>::RS;
   constexpr int WS = wig_size(L);
   constexpr int NTHR = H * 32;
   constexpr int VCH = ROW / 16, KCH = KROW / 16;  // 16-byte chunks per row
   extern __shared__ __align__(128) unsigned char smem[];
-  unsigned char* vbuf = smem;                                        // [STAGES][16][VSTR]
-  unsigned char* kbuf = vbuf + size_t(STAGES) * kTileK * VSTR;       // [STAGES][16][KSTR]
-  float* Dq = reinterpret_cast<float*>(kbuf + size_t(STAGES) * kTileK * KSTR);   // [16][WS]
+  unsigned char* vbuf = smem;                                        // [STAGES][RS][VSTR]
+  unsigned char* kbuf = vbuf + size_t(STAGES) * RS * VSTR;           // [STAGES][RS][KSTR]
+  float* Dq = reinterpret_cast<float*>(kbuf + size_t(STAGES) * RS * KSTR);   // [16][WS]
   float* rp = Dq + kTileM * WS;                                      // [16][L+1]
   int* tgt = reinterpret_cast<int*>(rp + kTileM * (L + 1));          // [16]
   int* su = tgt + kTileM;                                            // [cap]
-  uint32_t* smask = reinterpret_cast<uint32_t*>(su + p.plan.cap);    // [16][cap / 32]
+  uint32_t* smask = reinterpret_cast<uint32_t*>(su + p.plan.cap);    // [16][cap / 32 + 1]
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -146,12 +146,14 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
   const int g = lane >> 2, t = lane & 3;
   const PlanView& pv = p.plan;
   const int words = pv.cap / 32;
+  const int swords = words + 1;     // padded shared-memory mask row
   const char* hp_bytes = reinterpret_cast<const char*>(p.hp);
   const char* k_bytes = reinterpret_cast<const char*>(p.k);
 
   for (int tile = blockIdx.x; tile < pv.tiles; tile += gridDim.x) {
     const int U = pv.ulen[tile];
-    const int nsteps = (U + kTileK - 1) / kTileK;
+    const int nsteps = (U + kTileK - 1) / kTileK;         // k-steps of 16 union rows
+    const int nstages = (nsteps + KS - 1) / KS;
     const int* __restrict__ uni = pv.uni + (long long)tile * pv.cap;
     const uint32_t* __restrict__ mrow = pv.mask + (long long)tile * kTileM * words;
 
@@ -168,18 +170,20 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
     for (int e = tid; e < upad; e += NTHR) su[e] = uni[e];
     for (int e = tid; e < kTileM * uw; e += NTHR) {
       const int r = e / uw, w = e % uw;
-      smask[r * words + w] = mrow[r * words + w];
+      smask[r * swords + w] = mrow[r * words + w];
     }
     __syncthreads();   // tgt, su, smask visible
 
     // 32 threads per staged row; each copies chunks lane, lane + 32, ... of
-    // the row's value and key bytes
-    auto issue = [&](int step) {
-      const int buf = step % STAGES;
-      unsigned char* vb = vbuf + size_t(buf) * kTileK * VSTR;
-      unsigned char* kb = kbuf + size_t(buf) * kTileK * KSTR;
-      for (int r = tid >> 5; r < kTileK; r += NTHR / 32) {
-        const long long atom = su[step * kTileK + r];
+    // the row's value and key bytes (rows past the padded union are skipped)
+    auto issue = [&](int stage) {
+      const int buf = stage % STAGES;
+      unsigned char* vb = vbuf + size_t(buf) * RS * VSTR;
+      unsigned char* kb = kbuf + size_t(buf) * RS * KSTR;
+      for (int r = tid >> 5; r < RS; r += NTHR / 32) {
+        const int u = stage * RS + r;
+        if (u >= upad) break;
+        const long long atom = su[u];
         const char* vsrc = hp_bytes + atom * ROW;
         const char* ksrc = k_bytes + atom * KROW;
         for (int o = lane; o < VCH + KCH; o += 32) {
@@ -190,7 +194,7 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
     };
 #pragma unroll
     for (int s = 0; s < STAGES - 1; ++s) {
-      if (s < nsteps) issue(s);
+      if (s < nstages) issue(s);
       cp_async_commit();
     }
 
@@ -229,17 +233,29 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
     for (int d = 0; d < D; ++d)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[d][e] = 0.f;
-    float mref0 = -INFINITY, mref1 = -INFINITY, z0 = 0.f, z1 = 0.f;
+    // zacc: P times an all-ones B fragment, i.e. the row sums of exactly the
+    // bf16 weights the P V product uses (zacc[0] row g, zacc[2] row g+8)
+    float zacc[4] = {0.f, 0.f, 0.f, 0.f};
+    constexpr uint32_t kOnes = 0x3f803f80u;   // bf16x2 (1, 1)
+    // reference maxima (log2 domain): a finite sentinel, so that a masked
+    // entry (-inf) gives exp2(-inf) = 0 without a select
+    constexpr float kNone = -1e30f;
+    float mref0 = kNone, mref1 = kNone;
     constexpr float kLazy = 8.f;
+    const float qs = p.qscale;
 
-    for (int s = 0; s < nsteps; ++s) {
+    for (int st = 0; st < nstages; ++st) {
       cp_async_wait<STAGES - 2>();
       __syncthreads();
-      if (s + STAGES - 1 < nsteps) issue(s + STAGES - 1);
+      if (st + STAGES - 1 < nstages) issue(st + STAGES - 1);
       cp_async_commit();
-      const int buf = s % STAGES;
-      const uint32_t vb = smem_u32(vbuf + size_t(buf) * kTileK * VSTR);
-      const uint32_t kb = smem_u32(kbuf + size_t(buf) * kTileK * KSTR);
+      const int buf = st % STAGES;
+#pragma unroll
+      for (int j = 0; j < KS; ++j) {
+      const int s = st * KS + j;       // k-step
+      if (s >= nsteps) break;
+      const uint32_t vb = smem_u32(vbuf + (size_t(buf) * RS + j * kTileK) * VSTR);
+      const uint32_t kb = smem_u32(kbuf + (size_t(buf) * RS + j * kTileK) * KSTR);
       const int u0 = s * kTileK;
 
       // ---- S = Q K^T for 16 union atoms
@@ -253,30 +269,35 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
       mma_bf16(s0, qa, kf[0], kf[1]);
       mma_bf16(s1, qa, kf[2], kf[3]);
 
-      // ---- mask, online softmax (rows g and g+8 of the tile)
-      const uint32_t w0 = smask[g * words + (u0 >> 5)] >> (u0 & 31);
-      const uint32_t w1 = smask[(g + 8) * words + (u0 >> 5)] >> (u0 & 31);
-      float v[8];   // row g: cols 2t, 2t+1, 8+2t, 9+2t ; row g+8: same
-      v[0] = ((w0 >> (2 * t)) & 1u) ? s0[0] * p.qscale : -INFINITY;
-      v[1] = ((w0 >> (2 * t + 1)) & 1u) ? s0[1] * p.qscale : -INFINITY;
-      v[2] = ((w0 >> (2 * t + 8)) & 1u) ? s1[0] * p.qscale : -INFINITY;
-      v[3] = ((w0 >> (2 * t + 9)) & 1u) ? s1[1] * p.qscale : -INFINITY;
-      v[4] = ((w1 >> (2 * t)) & 1u) ? s0[2] * p.qscale : -INFINITY;
-      v[5] = ((w1 >> (2 * t + 1)) & 1u) ? s0[3] * p.qscale : -INFINITY;
-      v[6] = ((w1 >> (2 * t + 8)) & 1u) ? s1[2] * p.qscale : -INFINITY;
-      v[7] = ((w1 >> (2 * t + 9)) & 1u) ? s1[3] * p.qscale : -INFINITY;
+      // ---- mask (rows g and g+8 of the tile; bit k <-> union atom u0 + k)
+      const uint32_t w0 = smask[g * swords + (u0 >> 5)] >> ((u0 & 31) + 2 * t);
+      const uint32_t w1 = smask[(g + 8) * swords + (u0 >> 5)] >> ((u0 & 31) + 2 * t);
+      float v[8];   // raw logits; row g: cols 2t, 2t+1, 8+2t, 9+2t ; row g+8: same
+      v[0] = (w0 & 1u) ? s0[0] : -INFINITY;
+      v[1] = (w0 & 2u) ? s0[1] : -INFINITY;
+      v[2] = (w0 & 0x100u) ? s1[0] : -INFINITY;
+      v[3] = (w0 & 0x200u) ? s1[1] : -INFINITY;
+      v[4] = (w1 & 1u) ? s0[2] : -INFINITY;
+      v[5] = (w1 & 2u) ? s0[3] : -INFINITY;
+      v[6] = (w1 & 0x100u) ? s1[2] : -INFINITY;
+      v[7] = (w1 & 0x200u) ? s1[3] : -INFINITY;
+      // ---- online softmax: row maxima of the raw logits, scaled once
       float mx0 = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
       float mx1 = fmaxf(fmaxf(v[4], v[5]), fmaxf(v[6], v[7]));
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      mx0 *= qs;
+      mx1 *= qs;
       const bool r0 = mx0 > mref0 + kLazy, r1 = mx1 > mref1 + kLazy;
       if (__any_sync(0xffffffffu, r0 || r1)) {
         const float sc0 = r0 ? fast_exp2(mref0 - mx0) : 1.f;
         const float sc1 = r1 ? fast_exp2(mref1 - mx1) : 1.f;
-        z0 *= sc0;
-        z1 *= sc1;
+        zacc[0] *= sc0;
+        zacc[1] *= sc0;
+        zacc[2] *= sc1;
+        zacc[3] *= sc1;
 #pragma unroll
         for (int d = 0; d < D; ++d) {
           acc[d][0] *= sc0;
@@ -289,17 +310,18 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
       }
       float pr[8];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) pr[e] = v[e] == -INFINITY ? 0.f : fast_exp2(v[e] - mref0);
+      for (int e = 0; e < 4; ++e) pr[e] = fast_exp2(fmaf(v[e], qs, -mref0));
 #pragma unroll
-      for (int e = 4; e < 8; ++e) pr[e] = v[e] == -INFINITY ? 0.f : fast_exp2(v[e] - mref1);
+      for (int e = 4; e < 8; ++e) pr[e] = fast_exp2(fmaf(v[e], qs, -mref1));
       uint32_t pa[4];
-      float q0, q1, q2, q3, q4, q5, q6, q7;
-      pa[0] = pack_bf16(pr[0], pr[1], q0, q1);   // row g,   k = 2t, 2t+1
-      pa[1] = pack_bf16(pr[4], pr[5], q4, q5);   // row g+8, k = 2t, 2t+1
-      pa[2] = pack_bf16(pr[2], pr[3], q2, q3);   // row g,   k = 2t+8, 2t+9
-      pa[3] = pack_bf16(pr[6], pr[7], q6, q7);   // row g+8, k = 2t+8, 2t+9
-      z0 += (q0 + q1) + (q2 + q3);
-      z1 += (q4 + q5) + (q6 + q7);
+      {
+        __nv_bfloat162 b;
+        b = __floats2bfloat162_rn(pr[0], pr[1]); pa[0] = *reinterpret_cast<uint32_t*>(&b);  // row g,   k 2t
+        b = __floats2bfloat162_rn(pr[4], pr[5]); pa[1] = *reinterpret_cast<uint32_t*>(&b);  // row g+8, k 2t
+        b = __floats2bfloat162_rn(pr[2], pr[3]); pa[2] = *reinterpret_cast<uint32_t*>(&b);  // row g,   k 2t+8
+        b = __floats2bfloat162_rn(pr[6], pr[7]); pa[3] = *reinterpret_cast<uint32_t*>(&b);  // row g+8, k 2t+8
+      }
+      mma_bf16(zacc, pa, kOnes, kOnes);
 
       // ---- O += P V (one n8 tile per component of this head's 8 channels)
       {
@@ -319,18 +341,45 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
           mma_bf16(acc[D - 1], pa, vf[0], vf[1]);
         }
       }
+      }   // k-steps of the stage
     }
     cp_async_wait<0>();
     __syncthreads();   // Dq / rp written; all staged buffers drained
 
     // ---- epilogue: normalise; either write m or apply the target coupling
-    z0 += __shfl_xor_sync(0xffffffffu, z0, 1);
-    z0 += __shfl_xor_sync(0xffffffffu, z0, 2);
-    z1 += __shfl_xor_sync(0xffffffffu, z1, 1);
-    z1 += __shfl_xor_sync(0xffffffffu, z1, 2);
-    const float inv0 = z0 > 0.f ? 1.f / z0 : 0.f;
-    const float inv1 = z1 > 0.f ? 1.f / z1 : 0.f;
+    const float inv0 = zacc[0] > 0.f ? 1.f / zacc[0] : 0.f;
+    const float inv1 = zacc[2] > 0.f ? 1.f / zacc[2] : 0.f;
     const int ch = h * 8 + 2 * t;
+    if constexpr (FUSED && L >= 3) {
+      // register budget: m of both rows goes through this warp's slice of the
+      // drained staging buffers (8 KB per warp) so the accumulators are free
+      // before the coupling; one channel at a time, scalar stores
+      float* mw = reinterpret_cast<float*>(vbuf) + h * (kTileM * D * 8);
+#pragma unroll
+      for (int d = 0; d < D; ++d) {
+        *reinterpret_cast<float2*>(mw + (g * D + d) * 8 + 2 * t) =
+            make_float2(acc[d][0] * inv0, acc[d][1] * inv0);
+        *reinterpret_cast<float2*>(mw + ((g + 8) * D + d) * 8 + 2 * t) =
+            make_float2(acc[d][2] * inv1, acc[d][3] * inv1);
+      }
+      __syncwarp();
+#pragma unroll 1
+      for (int pr = 0; pr < 4; ++pr) {
+        const int r = g + 8 * (pr >> 1), e = pr & 1;
+        const int tg = tgt[r];
+        if (tg < 0) continue;
+        float rpow[L + 1];
+#pragma unroll
+        for (int l = 0; l <= L; ++l) rpow[l] = rp[r * (L + 1) + l];
+        float x[D];
+#pragma unroll
+        for (int d = 0; d < D; ++d) x[d] = mw[(r * D + d) * 8 + 2 * t + e];
+        float* o = p.out + (size_t)tg * D * C + ch + e;
+        eaas_channel<L>(x, Dq + r * WS, rpow, p.tab,
+                        [&](int pp) { return __ldg(p.w2 + pp * C + ch + e); },
+                        [&](int d, float val) { o[d * C] = val; });
+      }
+    } else
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       const int r = g + 8 * half;
@@ -343,20 +392,6 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
         for (int d = 0; d < D; ++d)
           *reinterpret_cast<float2*>(o + d * C) =
               make_float2(acc[d][2 * half] * inv, acc[d][2 * half + 1] * inv);
-      } else if constexpr (L >= 3) {
-        // register budget: one channel at a time, scalar stores
-        float rpow[L + 1];
-#pragma unroll
-        for (int l = 0; l <= L; ++l) rpow[l] = rp[r * (L + 1) + l];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          float x[D];
-#pragma unroll
-          for (int d = 0; d < D; ++d) x[d] = acc[d][2 * half + e] * inv;
-          eaas_channel<L>(x, Dq + r * WS, rpow, p.tab,
-                          [&](int pp) { return __ldg(p.w2 + pp * C + ch + e); },
-                          [&](int d, float val) { o[d * C + e] = val; });
-        }
       } else {
         float rpow[L + 1];
 #pragma unroll
