@@ -242,9 +242,10 @@ constexpr int kBlockCells = kWidth * kWidth * kWidth;
 // and the warp walks that flat candidate list 32 at a time, each lane finding
 // its candidate's cell by a binary search over the scanned offsets.
 template <typename F>
-__device__ __forceinline__ void for_each_neighbour(const Search& s, int4 p, int4 c, F&& f) {
+__device__ __forceinline__ void for_each_neighbour_rounds(const Search& s, int4 p, int4 c,
+                                                          int round0, int round_step, F&& f) {
   const int lane = threadIdx.x & 31;
-  for (int r0 = 0; r0 < kBlockCells; r0 += 32) {
+  for (int r0 = round0 * 32; r0 < kBlockCells; r0 += round_step * 32) {
     const int l = r0 + lane;
     int beg = 0, len = 0, cx = 0, cy = 0, cz = 0;
     if (l < kBlockCells) {
@@ -295,6 +296,11 @@ __device__ __forceinline__ void for_each_neighbour(const Search& s, int4 p, int4
       f(hit, j, d2);
     }
   }
+}
+
+template <typename F>
+__device__ __forceinline__ void for_each_neighbour(const Search& s, int4 p, int4 c, F&& f) {
+  for_each_neighbour_rounds(s, p, c, 0, 1, f);
 }
 
 __global__ void count_neighbours(Search s, int n, int* __restrict__ deg) {
@@ -377,54 +383,77 @@ fill_padded(Search s, int n, int K, int32_t* __restrict__ nbr, int32_t* __restri
   }
 }
 
-// Rows with more than K neighbours, one warp per listed atom (persistent
-// warps; the loop is bounded by the device-side count).  The key
-// (d^2 << shift | j) of the K-th nearest comes from a shared-memory sort of
-// all the atom's keys when they fit, by bisection otherwise; the row is then
-// rewritten, in sweep order, with exactly the keys up to it (ties to smaller j).
-__global__ void __launch_bounds__(kFillWarps * 32)
+// Rows with more than K neighbours: one CTA of kFixWarps warps per listed atom
+// (persistent CTAs; the loop is bounded by the device-side count).  The warps
+// split the 125-cell sweep by rounds and gather every neighbour's key
+// (d^2 << shift | j) into shared memory; a block-wide bitonic sort orders them
+// and the row is rewritten with the K smallest keys, nearest first (ties to
+// the smaller index).  Rows with more keys than fit use bisection for the K-th
+// key and one warp rewrites them in sweep order.
+constexpr int kFixWarps = 4;
+
+__global__ void __launch_bounds__(kFixWarps * 32)
 fix_truncated(Search s, int K, int32_t* __restrict__ nbr, const int* __restrict__ trunc,
               int* __restrict__ overflow) {
-  __shared__ unsigned long long keys_all[kFillWarps][kSelectCap];
+  __shared__ unsigned long long keys[kSelectCap];
+  __shared__ int s_total;
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
   const int ntr = trunc[0];
-  for (int t = blockIdx.x * kFillWarps + wib; t < ntr; t += gridDim.x * kFillWarps) {
+  const unsigned long long jmask = (1ull << s.key_shift) - 1ull;
+  for (int t = blockIdx.x; t < ntr; t += gridDim.x) {
     const int w = trunc[1 + t];
     const int4 p = s.spos[w];
     const int4 c = s.scell[w];
     int32_t* row = nbr + (long long)p.w * K;
-    unsigned long long* keys = keys_all[wib];
-    int total = 0;
-    for_each_neighbour(s, p, c, [&](bool hit, int j, long long d2) {
+    if (threadIdx.x == 0) s_total = 0;
+    __syncthreads();
+    for_each_neighbour_rounds(s, p, c, wib, kFixWarps, [&](bool hit, int j, long long d2) {
       const unsigned m = __ballot_sync(0xffffffffu, hit);
-      const int pos = total + __popc(m & ((1u << lane) - 1u));
+      int base = 0;
+      if (lane == 0 && m) base = atomicAdd(&s_total, __popc(m));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      const int pos = base + __popc(m & ((1u << lane) - 1u));
       if (hit && pos < kSelectCap)
         keys[pos] = (((unsigned long long)d2) << s.key_shift) | (unsigned long long)j;
-      total += __popc(m);
     });
-    unsigned long long thresh;
+    __syncthreads();
+    const int total = s_total;
     if (total <= kSelectCap) {
-      int size = 1;
+      int size = 32;
       while (size < total) size <<= 1;
-      for (int q = total + lane; q < size; q += 32) keys[q] = ~0ull;
-      __syncwarp();
-      warp_bitonic_sort(keys, size);
-      thresh = keys[K - 1];
-    } else {
-      thresh = kth_key(s, p, c, K);
+      for (int q = total + threadIdx.x; q < size; q += blockDim.x) keys[q] = ~0ull;
+      __syncthreads();
+      for (int k = 2; k <= size; k <<= 1) {
+        for (int jj = k >> 1; jj > 0; jj >>= 1) {
+          for (int i = threadIdx.x; i < size; i += blockDim.x) {
+            const int ixj = i ^ jj;
+            if (ixj > i) {
+              const unsigned long long a = keys[i], b = keys[ixj];
+              if ((a > b) == ((i & k) == 0)) {
+                keys[i] = b;
+                keys[ixj] = a;
+              }
+            }
+          }
+          __syncthreads();
+        }
+      }
+      for (int q = threadIdx.x; q < K; q += blockDim.x) row[q] = int32_t(keys[q] & jmask);
+    } else if (wib == 0) {
+      const unsigned long long thresh = kth_key(s, p, c, K);
+      int written = 0;
+      for_each_neighbour(s, p, c, [&](bool hit, int j, long long d2) {
+        const bool keep = hit && ((((unsigned long long)d2) << s.key_shift) |
+                                  (unsigned long long)j) <= thresh;
+        const unsigned m = __ballot_sync(0xffffffffu, keep);
+        const int pos = written + __popc(m & ((1u << lane) - 1u));
+        if (keep && pos < K) row[pos] = j;
+        written += __popc(m);
+      });
     }
-    __syncwarp();
-    int written = 0;
-    for_each_neighbour(s, p, c, [&](bool hit, int j, long long d2) {
-      const bool keep = hit && ((((unsigned long long)d2) << s.key_shift) |
-                                (unsigned long long)j) <= thresh;
-      const unsigned m = __ballot_sync(0xffffffffu, keep);
-      const int pos = written + __popc(m & ((1u << lane) - 1u));
-      if (keep && pos < K) row[pos] = j;
-      written += __popc(m);
-    });
-    if (lane == 0) atomicAdd(overflow, total - K);
+    if (threadIdx.x == 0) atomicAdd(overflow, total - K);
+    __syncthreads();
   }
 }
 
@@ -483,7 +512,7 @@ int build_graph(const int32_t* d_pos_q, int n, int cutoff_q, int K, int mode,
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    fix_truncated<<<sms * 2, kFillWarps * 32, 0, st>>>(s, K, d_a, w.trunc, d_overflow);
+    fix_truncated<<<sms * 4, kFixWarps * 32, 0, st>>>(s, K, d_a, w.trunc, d_overflow);
   } else {
     const long long nthreads = (long long)n * 32;
     count_neighbours<<<unsigned((nthreads + tb - 1) / tb), tb, 0, st>>>(s, n, w.deg);

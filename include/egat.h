@@ -120,8 +120,10 @@ EGAT_API int egat_num_paths(int lmax);
  *                  col_capacity are not written and *d_overflow = their
  *                  number.
  *                Row order, both modes: the 5 x 5 x 5 cells around the
- *                atom's cell in a fixed sweep, atoms of one cell by index — a
- *                deterministic order (the same arrays on every call).
+ *                atom's cell in a fixed sweep, atoms of one cell by index; a
+ *                truncated padded row lists its K nearest by (squared
+ *                distance, index) instead.  Deterministic either way (the
+ *                same arrays on every call).
  *  d_order       optional int32 [n]: atoms listed cell by cell (Morton
  *                order of cells) — a traversal order with spatial locality
  *                for egat_otf_attention / egat_forward.  May be NULL.
