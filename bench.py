@@ -199,6 +199,9 @@ def main():
     ap.add_argument("--cpu-targets", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--attention", default="auto", choices=["auto", "tiled", "per-target"],
+                    help="steps 3+4 kernel: tensor-core tiles when the shape allows (auto), or "
+                         "the per-target kernel")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -257,7 +260,10 @@ def main():
 
     plan_sz = ctypes.c_size_t(0)
     tiled = (lib.egat_attention_plan_bytes(ctypes.byref(cshape), ctypes.byref(plan_sz)) == 0
-             and wl.dtype == "bf16" and wl.C == 128 and wl.H == 16 and wl.dk == 16)
+             and wl.dtype == "bf16" and wl.C == 128 and wl.H == 16 and wl.dk == 16
+             and args.attention != "per-target")
+    if args.attention == "tiled" and not tiled:
+        raise SystemExit("the tensor-core attention path does not support this workload")
     plan = torch.empty(max(plan_sz.value, 16), dtype=torch.uint8, device=dev)
 
     def build_plan():
