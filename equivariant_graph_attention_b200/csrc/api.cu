@@ -83,6 +83,9 @@ int egat_build_graph(const int32_t* d_pos_q, int32_t n, int32_t cutoff_q, int32_
                      int32_t* d_order, int32_t* d_overflow, void* d_ws, size_t ws_bytes,
                      void* stream) {
   if (n < 0 || cutoff_q <= 0 || !d_overflow) return EGAT_ERR_ARG;
+  // candidate cells span at most 20 cells of edge ceil(cutoff_q / 2) per axis;
+  // this keeps every coordinate difference the kernels form within 32 bits
+  if (cutoff_q > (1 << 26)) return EGAT_ERR_UNSUPPORTED;
   if (mode == EGAT_GRAPH_PADDED) {
     if (K < 1 || K > 1024) return EGAT_ERR_ARG;
   } else if (mode == EGAT_GRAPH_CSR) {

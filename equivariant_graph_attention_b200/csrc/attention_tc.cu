@@ -112,6 +112,11 @@ constexpr size_t tc_smem_fixed() {
          size_t(kTileM) * (wig_size(L) + L + 1) * sizeof(float) + kTileM * sizeof(int);
 }
 // mask rows are padded by one word so the 8 rows a warp reads sit in distinct banks
+// fused kernels keep the target-coupling weights [P][C] in shared memory
+template <int L, int H>
+constexpr size_t tc_smem_w2() {
+  return size_t(num_paths(L)) * 8 * H * sizeof(float);
+}
 inline size_t tc_smem_plan(int cap) {
   return size_t(cap) * sizeof(int) + size_t(kTileM) * (cap / 32 + 1) * sizeof(uint32_t);
 }
@@ -139,6 +144,10 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
   int* tgt = reinterpret_cast<int*>(rp + kTileM * (L + 1));          // [16]
   int* su = tgt + kTileM;                                            // [cap]
   uint32_t* smask = reinterpret_cast<uint32_t*>(su + p.plan.cap);    // [16][cap / 32 + 1]
+  float* sw2 = reinterpret_cast<float*>(smask + kTileM * (p.plan.cap / 32 + 1));   // [P][C]
+  if constexpr (FUSED) {
+    for (int e = threadIdx.x; e < num_paths(L) * C; e += H * 32) sw2[e] = __ldg(p.w2 + e);
+  }
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -250,24 +259,31 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
       if (st + STAGES - 1 < nstages) issue(st + STAGES - 1);
       cp_async_commit();
       const int buf = st % STAGES;
+      // ---- S = Q K^T for every k-step of the stage first, so the tensor
+      // core works on one step's P V while the next step's softmax runs
+      float sf[KS][2][4];
+#pragma unroll
+      for (int j = 0; j < KS; ++j) {
+        if (st * KS + j < nsteps) {
+          const uint32_t kb = smem_u32(kbuf + (size_t(buf) * RS + j * kTileK) * KSTR);
+          uint32_t kf[4];
+          const int row = (lane & 7) + 8 * (lane >> 4);
+          const int half = (lane >> 3) & 1;
+          ldsm_x4(kf, kb + row * KSTR + h * 32 + half * 16);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sf[j][0][e] = sf[j][1][e] = 0.f;
+          mma_bf16(sf[j][0], qa, kf[0], kf[1]);
+          mma_bf16(sf[j][1], qa, kf[2], kf[3]);
+        }
+      }
 #pragma unroll
       for (int j = 0; j < KS; ++j) {
       const int s = st * KS + j;       // k-step
       if (s >= nsteps) break;
       const uint32_t vb = smem_u32(vbuf + (size_t(buf) * RS + j * kTileK) * VSTR);
-      const uint32_t kb = smem_u32(kbuf + (size_t(buf) * RS + j * kTileK) * KSTR);
       const int u0 = s * kTileK;
-
-      // ---- S = Q K^T for 16 union atoms
-      uint32_t kf[4];
-      {
-        const int row = (lane & 7) + 8 * (lane >> 4);
-        const int half = (lane >> 3) & 1;
-        ldsm_x4(kf, kb + row * KSTR + h * 32 + half * 16);
-      }
-      float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-      mma_bf16(s0, qa, kf[0], kf[1]);
-      mma_bf16(s1, qa, kf[2], kf[3]);
+      const float* s0 = sf[j][0];
+      const float* s1 = sf[j][1];
 
       // ---- mask (rows g and g+8 of the tile; bit k <-> union atom u0 + k)
       const uint32_t w0 = smask[g * swords + (u0 >> 5)] >> ((u0 & 31) + 2 * t);
@@ -376,7 +392,7 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
         for (int d = 0; d < D; ++d) x[d] = mw[(r * D + d) * 8 + 2 * t + e];
         float* o = p.out + (size_t)tg * D * C + ch + e;
         eaas_channel<L>(x, Dq + r * WS, rpow, p.tab,
-                        [&](int pp) { return __ldg(p.w2 + pp * C + ch + e); },
+                        [&](int pp) { return sw2[pp * C + ch + e]; },
                         [&](int d, float val) { o[d * C] = val; });
       }
     } else
@@ -402,7 +418,7 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
 #pragma unroll
           for (int d = 0; d < D; ++d) x[d] = acc[d][2 * half] * inv;
           eaas_channel<L>(x, Dq + r * WS, rpow, p.tab,
-                          [&](int pp) { return __ldg(p.w2 + pp * C + ch); },
+                          [&](int pp) { return sw2[pp * C + ch]; },
                           [&](int d, float val) { y0[d] = val; });
         }
         {
@@ -410,7 +426,7 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
 #pragma unroll
           for (int d = 0; d < D; ++d) x[d] = acc[d][2 * half + 1] * inv;
           eaas_channel<L>(x, Dq + r * WS, rpow, p.tab,
-                          [&](int pp) { return __ldg(p.w2 + pp * C + ch + 1); },
+                          [&](int pp) { return sw2[pp * C + ch + 1]; },
                           [&](int d, float val) { y1[d] = val; });
         }
 #pragma unroll
@@ -423,7 +439,8 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
 
 template <int L, int H, bool FUSED>
 int launch_tc_t(const TcParams& p, int tiles, cudaStream_t st) {
-  const size_t shmem = tc_smem_fixed<L, H>() + tc_smem_plan(p.plan.cap);
+  const size_t shmem = tc_smem_fixed<L, H>() + tc_smem_plan(p.plan.cap) +
+                       (FUSED ? tc_smem_w2<L, H>() : 0);
   if (shmem > 227 * 1024) return EGAT_ERR_UNSUPPORTED;
   auto kern = otf_attention_tc_kernel<L, H, FUSED>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(shmem)) !=
@@ -446,7 +463,9 @@ bool tc_attention_supported(const egat_shape& s) {
   if (plan_smem_bytes(s.n, s.K) > kPlanSmemLimit) return false;
   const size_t fixed = s.lmax == 1 ? tc_smem_fixed<1, 16>()
                      : s.lmax == 2 ? tc_smem_fixed<2, 16>() : tc_smem_fixed<3, 16>();
-  return fixed + tc_smem_plan(plan_capacity(s.K)) <= 227 * 1024;
+  const size_t w2 = s.lmax == 1 ? tc_smem_w2<1, 16>()
+                  : s.lmax == 2 ? tc_smem_w2<2, 16>() : tc_smem_w2<3, 16>();
+  return fixed + tc_smem_plan(plan_capacity(s.K)) + w2 <= 227 * 1024;
 }
 
 int launch_attention_tc(const egat_shape& s, bool fused, const void* d_q, const void* d_k,

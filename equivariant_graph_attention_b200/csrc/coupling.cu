@@ -167,7 +167,9 @@ eaas_source_kernel(const __grid_constant__ EaasParams p) {
   constexpr int WS = wig_size(L);
   constexpr int CPL = L >= 3 ? 2 : 4;
   constexpr int kMaxSlots = 32 / 4;              // C >= 16 -> G >= 4 lanes
+  constexpr int NP = num_paths(L);
   __shared__ float Dsm[kEaasWarps][kMaxSlots][WS];
+  extern __shared__ float sw[];                   // path weights [P][C]
 
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
@@ -186,6 +188,8 @@ eaas_source_kernel(const __grid_constant__ EaasParams p) {
   const T* __restrict__ x = static_cast<const T*>(p.x);
   T* __restrict__ y = static_cast<T*>(p.y);
   float* Dme = Dsm[wib][slot];
+  for (int e = threadIdx.x; e < NP * C; e += blockDim.x) sw[e] = __ldg(p.w + e);
+  __syncthreads();
 
   for (long long grp = gwarp / WPA; grp < ngroups; grp += nwarps / WPA) {
     const long long at = grp * AW + slot;
@@ -213,21 +217,10 @@ eaas_source_kernel(const __grid_constant__ EaasParams p) {
     __syncwarp();                             // previous atom's readers are done
     wigner_build<L>(Q, Dme, gl, GW, [] { __syncwarp(); });
     if (live) {
-      float yv[CPL][D];
-#pragma unroll
-      for (int k = 0; k < CPL; ++k) {
-        const float* __restrict__ wcol = p.w + c0 + k;
-        eaas_channel<L>(xv[k], Dme, rpow, p.tab, [&](int q) { return __ldg(wcol + q * C); },
-                        [&](int d, float v) { yv[k][d] = v; });
-      }
       T* yr = y + (size_t)at * D * C + c0;
-#pragma unroll
-      for (int d = 0; d < D; ++d) {
-        float v[CPL];
-#pragma unroll
-        for (int k = 0; k < CPL; ++k) v[k] = yv[k][d];
-        ChanVec<T, CPL>::store(yr + d * C, v);
-      }
+      const float* swc = sw + c0;
+      eaas_multi<L, CPL>(xv, Dme, rpow, p.tab, [&](int q, int k) { return swc[q * C + k]; },
+                         [&](int d, const float (&v)[CPL]) { ChanVec<T, CPL>::store(yr + d * C, v); });
     }
   }
 }
@@ -253,7 +246,8 @@ int launch_eaas_t(const egat_shape& s, const void* d_x, const float* d_pos, cons
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long want = (groups * WPA + kEaasWarps - 1) / kEaasWarps;
   const int grid = int(std::max<long long>(1, std::min<long long>(want, (long long)sms * 8)));
-  eaas_source_kernel<L, T><<<grid, kEaasWarps * 32, 0, st>>>(p);
+  const size_t shmem = size_t(num_paths(L)) * s.C * sizeof(float);
+  eaas_source_kernel<L, T><<<grid, kEaasWarps * 32, shmem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
 }
 

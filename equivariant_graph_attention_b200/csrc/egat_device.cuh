@@ -342,4 +342,87 @@ __device__ __forceinline__ void eaas_channel(float (&x)[(L + 1) * (L + 1)],
   });
 }
 
+// The same operator on NCH channels at once (channels of one atom share the
+// Wigner-D matrices): each matrix entry is read once and applied to every
+// channel.  x[k][d] is overwritten; wgt(p, k) returns w[p] of channel k;
+// out(d, y) receives component d of all NCH channels.
+template <int L, int NCH, typename WFn, typename OutFn>
+__device__ __forceinline__ void eaas_multi(float (&x)[NCH][(L + 1) * (L + 1)],
+                                           const float* __restrict__ Dsm,
+                                           const float (&rpow)[L + 1], const EaasTable& tab,
+                                           WFn wgt, OutFn out) {
+  constexpr int D = (L + 1) * (L + 1);
+  float t[NCH][D];
+#pragma unroll
+  for (int k = 0; k < NCH; ++k)
+#pragma unroll
+    for (int i = 0; i < D; ++i) t[k][i] = 0.f;
+  static_for<1, L + 1>([&](auto lc) {
+    constexpr int l = decltype(lc)::value;
+    constexpr int w = 2 * l + 1;
+    const float* Dl = Dsm + wig_off(l);
+    float tmp[NCH][w];
+#pragma unroll
+    for (int a = 0; a < w; ++a) {
+#pragma unroll
+      for (int k = 0; k < NCH; ++k) tmp[k][a] = 0.f;
+#pragma unroll
+      for (int b = 0; b < w; ++b) {
+        const float dv = Dl[b * w + a];
+#pragma unroll
+        for (int k = 0; k < NCH; ++k) tmp[k][a] = fmaf(dv, x[k][l * l + b], tmp[k][a]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < NCH; ++k)
+#pragma unroll
+      for (int a = 0; a < w; ++a) x[k][l * l + a] = tmp[k][a];
+  });
+  static_for<0, num_paths(L)>([&](auto pc) {
+    constexpr int p = decltype(pc)::value;
+    constexpr int li = path_info(L, p, 0);
+    constexpr int lf = path_info(L, p, 1);
+    constexpr int lo = path_info(L, p, 2);
+    constexpr bool even = ((li + lf + lo) % 2) == 0;
+    float wp[NCH];
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) wp[k] = wgt(p, k) * rpow[lf];
+#pragma unroll
+    for (int mo = -lo; mo <= lo; ++mo) {
+      const int src = even ? mo : -mo;
+      const bool live = (iabs(mo) <= li) && (even || mo != 0);
+      if (live) {
+        const float f = tab.f[p][mo + lo];
+#pragma unroll
+        for (int k = 0; k < NCH; ++k)
+          t[k][lo * lo + lo + mo] = fmaf(wp[k] * f, x[k][li * li + li + src], t[k][lo * lo + lo + mo]);
+      }
+    }
+  });
+  {
+    float y[NCH];
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) y[k] = t[k][0];
+    out(0, y);
+  }
+  static_for<1, L + 1>([&](auto lc) {
+    constexpr int l = decltype(lc)::value;
+    constexpr int w = 2 * l + 1;
+    const float* Dl = Dsm + wig_off(l);
+#pragma unroll
+    for (int a = 0; a < w; ++a) {
+      float y[NCH];
+#pragma unroll
+      for (int k = 0; k < NCH; ++k) y[k] = 0.f;
+#pragma unroll
+      for (int b = 0; b < w; ++b) {
+        const float dv = Dl[a * w + b];
+#pragma unroll
+        for (int k = 0; k < NCH; ++k) y[k] = fmaf(dv, t[k][l * l + b], y[k]);
+      }
+      out(l * l + a, y);
+    }
+  });
+}
+
 }  // namespace egat

@@ -220,6 +220,14 @@ __global__ void rank_in_bucket(int n, const int4* __restrict__ cell,
   if (order) order[dst] = me.w;
 }
 
+// Exact squared distance of two grid points in the same 2-cell neighbourhood:
+// the coordinate differences fit in 32 bits (the host bounds the cutoff), so
+// each square is one widening 32 x 32 -> 64-bit multiply.
+__device__ __forceinline__ long long sq_dist(int4 a, int4 b) {
+  const int dx = a.x - b.x, dy = a.y - b.y, dz = a.z - b.z;
+  return (long long)dx * dx + (long long)dy * dy + (long long)dz * dz;
+}
+
 struct Search {
   const int4* spos;
   const int4* scell;
@@ -287,9 +295,7 @@ __device__ __forceinline__ void for_each_neighbour_rounds(const Search& s, int4 
         const int4 q = s.spos[slot];
         if (cc.x == ocx && cc.y == ocy && cc.z == ocz) {
           j = q.w;
-          const long long ddx = (long long)q.x - p.x, ddy = (long long)q.y - p.y,
-                          ddz = (long long)q.z - p.z;
-          d2 = ddx * ddx + ddy * ddy + ddz * ddz;
+          d2 = sq_dist(q, p);
           hit = (j != p.w) && (d2 <= s.rc2);
         }
       }

@@ -119,17 +119,17 @@ EGAT_API int egat_num_paths(int lmax);
  *                  d_cnt_or_col = col int32 [col_capacity]; entries past
  *                  col_capacity are not written and *d_overflow = their
  *                  number.
- *                Row order, both modes: the 5 x 5 x 5 cells around the
- *                atom's cell in a fixed sweep, atoms of one cell by index; a
- *                truncated padded row lists its K nearest by (squared
- *                distance, index) instead.  Deterministic either way (the
- *                same arrays on every call).
+ *                Row order: cell order of the neighbourhood (atoms of one
+ *                cell by index); a truncated padded row lists its K nearest
+ *                by (squared distance, index).  Deterministic: the same
+ *                arrays on every call.
  *  d_order       optional int32 [n]: atoms listed cell by cell (Morton
  *                order of cells) — a traversal order with spatial locality
  *                for egat_otf_attention / egat_forward.  May be NULL.
  *  d_overflow    int32 [1], zeroed and then set by this call.
  *  d_ws, ws_bytes  scratch of at least egat_graph_workspace_bytes(n).
- * Returns EGAT_ERR_UNSUPPORTED when cutoff_q^2 * 2^ceil(log2 n) >= 2^64.
+ * Returns EGAT_ERR_UNSUPPORTED when cutoff_q > 2^26 (1,024 Å on a 2^-16 Å
+ * grid) or cutoff_q^2 * 2^ceil(log2 n) >= 2^64.
  */
 EGAT_API int egat_graph_workspace_bytes(int32_t n, size_t* bytes);
 EGAT_API int egat_build_graph(const int32_t* d_pos_q, int32_t n, int32_t cutoff_q, int32_t K,

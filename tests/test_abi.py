@@ -102,3 +102,4 @@ def test_pointer_and_size_validation(lib):
     assert g(10, 100, 8, 5, ok) == egat.EGAT_ERR_ARG
     assert g(10, 100, 8, 0, None) == egat.EGAT_ERR_ARG
     assert g(1 << 30, 2 ** 31 - 1, 8, 0, ok) == egat.EGAT_ERR_UNSUPPORTED
+    assert g(10, (1 << 26) + 1, 8, 0, ok) == egat.EGAT_ERR_UNSUPPORTED
