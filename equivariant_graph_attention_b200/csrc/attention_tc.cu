@@ -252,6 +252,9 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
     float mref0 = kNone, mref1 = kNone;
     constexpr float kLazy = 8.f;
     const float qs = p.qscale;
+    const float inv_qs = 1.f / qs;
+    // raw-logit thresholds that trigger a raise; start below any finite logit
+    float thr0 = -INFINITY, thr1 = -INFINITY;
 
     for (int st = 0; st < nstages; ++st) {
       cp_async_wait<STAGES - 2>();
@@ -297,17 +300,22 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
       v[5] = (w1 & 2u) ? s0[3] : -INFINITY;
       v[6] = (w1 & 0x100u) ? s1[2] : -INFINITY;
       v[7] = (w1 & 0x200u) ? s1[3] : -INFINITY;
-      // ---- online softmax: row maxima of the raw logits, scaled once
-      float mx0 = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
-      float mx1 = fmaxf(fmaxf(v[4], v[5]), fmaxf(v[6], v[7]));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      mx0 *= qs;
-      mx1 *= qs;
-      const bool r0 = mx0 > mref0 + kLazy, r1 = mx1 > mref1 + kLazy;
-      if (__any_sync(0xffffffffu, r0 || r1)) {
+      // ---- online softmax.  Common case: no logit of the warp's rows exceeds
+      // its row's raw threshold (mref + kLazy) / qs, tested per entry with no
+      // cross-lane traffic.  Otherwise the row maxima are formed exactly and
+      // the rows that need it are rescaled.
+      const bool over = (v[0] > thr0) | (v[1] > thr0) | (v[2] > thr0) | (v[3] > thr0) |
+                        (v[4] > thr1) | (v[5] > thr1) | (v[6] > thr1) | (v[7] > thr1);
+      if (__any_sync(0xffffffffu, over)) {
+        float mx0 = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
+        float mx1 = fmaxf(fmaxf(v[4], v[5]), fmaxf(v[6], v[7]));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+        mx0 *= qs;
+        mx1 *= qs;
+        const bool r0 = mx0 > mref0 + kLazy, r1 = mx1 > mref1 + kLazy;
         const float sc0 = r0 ? fast_exp2(mref0 - mx0) : 1.f;
         const float sc1 = r1 ? fast_exp2(mref1 - mx1) : 1.f;
         zacc[0] *= sc0;
@@ -321,8 +329,14 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
           acc[d][2] *= sc1;
           acc[d][3] *= sc1;
         }
-        if (r0) mref0 = mx0;
-        if (r1) mref1 = mx1;
+        if (r0) {
+          mref0 = mx0;
+          thr0 = (mref0 + kLazy) * inv_qs;
+        }
+        if (r1) {
+          mref1 = mx1;
+          thr1 = (mref1 + kLazy) * inv_qs;
+        }
       }
       float pr[8];
 #pragma unroll
