@@ -193,11 +193,19 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
         const int u = stage * RS + r;
         if (u >= upad) break;
         const long long atom = su[u];
-        const char* vsrc = hp_bytes + atom * ROW;
-        const char* ksrc = k_bytes + atom * KROW;
-        for (int o = lane; o < VCH + KCH; o += 32) {
-          if (o < VCH) cp_async16(smem_u32(vb + r * VSTR + o * 16), vsrc + o * 16);
-          else cp_async16(smem_u32(kb + r * KSTR + (o - VCH) * 16), ksrc + (o - VCH) * 16);
+        const char* vsrc = hp_bytes + atom * ROW + lane * 16;
+        const char* ksrc = k_bytes + atom * KROW + lane * 16;
+        const uint32_t vdst = smem_u32(vb + r * VSTR + lane * 16);
+        const uint32_t kdst = smem_u32(kb + r * KSTR + lane * 16);
+#pragma unroll
+        for (int i = 0; i < VCH / 32; ++i) cp_async16(vdst + i * 512, vsrc + i * 512);
+        if constexpr (VCH % 32) {
+          if (lane < VCH % 32) cp_async16(vdst + (VCH / 32) * 512, vsrc + (VCH / 32) * 512);
+        }
+#pragma unroll
+        for (int i = 0; i < KCH / 32; ++i) cp_async16(kdst + i * 512, ksrc + i * 512);
+        if constexpr (KCH % 32) {
+          if (lane < KCH % 32) cp_async16(kdst + (KCH / 32) * 512, ksrc + (KCH / 32) * 512);
         }
       }
     };
@@ -426,25 +434,18 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
         float rpow[L + 1];
 #pragma unroll
         for (int l = 0; l <= L; ++l) rpow[l] = rp[r * (L + 1) + l];
-        float y0[D], y1[D];
-        {
-          float x[D];
+        // channels 2t and 2t+1 of one target share its Wigner-D matrices
+        float x[2][D];
 #pragma unroll
-          for (int d = 0; d < D; ++d) x[d] = acc[d][2 * half] * inv;
-          eaas_channel<L>(x, Dq + r * WS, rpow, p.tab,
-                          [&](int pp) { return sw2[pp * C + ch]; },
-                          [&](int d, float val) { y0[d] = val; });
+        for (int d = 0; d < D; ++d) {
+          x[0][d] = acc[d][2 * half] * inv;
+          x[1][d] = acc[d][2 * half + 1] * inv;
         }
-        {
-          float x[D];
-#pragma unroll
-          for (int d = 0; d < D; ++d) x[d] = acc[d][2 * half + 1] * inv;
-          eaas_channel<L>(x, Dq + r * WS, rpow, p.tab,
-                          [&](int pp) { return sw2[pp * C + ch + 1]; },
-                          [&](int d, float val) { y1[d] = val; });
-        }
-#pragma unroll
-        for (int d = 0; d < D; ++d) *reinterpret_cast<float2*>(o + d * C) = make_float2(y0[d], y1[d]);
+        eaas_multi<L, 2>(x, Dq + r * WS, rpow, p.tab,
+                         [&](int pp, int k) { return sw2[pp * C + ch + k]; },
+                         [&](int d, const float (&y)[2]) {
+                           *reinterpret_cast<float2*>(o + d * C) = make_float2(y[0], y[1]);
+                         });
       }
     }
     __syncthreads();   // tgt / Dq / rp are rewritten by the next tile
