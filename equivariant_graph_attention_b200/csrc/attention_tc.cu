@@ -163,6 +163,9 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
     const int U = pv.ulen[tile];
     const int nsteps = (U + kTileK - 1) / kTileK;         // k-steps of 16 union rows
     const int nstages = (nsteps + KS - 1) / KS;
+    // the plan pads the union to whole k-steps; here it is padded further to
+    // whole stages with its first atom, whose mask bits there are zero
+    const int ustep = nsteps * kTileK;
     const int* __restrict__ uni = pv.uni + (long long)tile * pv.cap;
     const uint32_t* __restrict__ mrow = pv.mask + (long long)tile * kTileM * words;
 
@@ -174,13 +177,14 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
       tgt[tid] = tg;
     }
     // the tile's union indices and membership mask into shared memory
-    const int upad = nsteps * kTileK;
-    const int uw = (upad + 31) / 32;
-    for (int e = tid; e < upad; e += NTHR) su[e] = uni[e];
+    const int upad = nstages * RS;
+    const int uw = (ustep + 31) / 32;   // mask words the plan wrote
+    for (int e = tid; e < upad; e += NTHR) su[e] = uni[e < ustep ? e : 0];
     for (int e = tid; e < kTileM * uw; e += NTHR) {
       const int r = e / uw, w = e % uw;
       smask[r * swords + w] = mrow[r * words + w];
     }
+    if (upad > 32 * uw && tid < kTileM) smask[tid * swords + uw] = 0u;
     __syncthreads();   // tgt, su, smask visible
 
     // 32 threads per staged row; each copies chunks lane, lane + 32, ... of
@@ -270,53 +274,54 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
       if (st + STAGES - 1 < nstages) issue(st + STAGES - 1);
       cp_async_commit();
       const int buf = st % STAGES;
-      // ---- S = Q K^T for every k-step of the stage first, so the tensor
-      // core works on one step's P V while the next step's softmax runs
+      // ---- S = Q K^T for every k-step of the stage (stages are whole:
+      // the union is padded to a multiple of RS rows)
       float sf[KS][2][4];
 #pragma unroll
       for (int j = 0; j < KS; ++j) {
-        if (st * KS + j < nsteps) {
-          const uint32_t kb = smem_u32(kbuf + (size_t(buf) * RS + j * kTileK) * KSTR);
-          uint32_t kf[4];
-          const int row = (lane & 7) + 8 * (lane >> 4);
-          const int half = (lane >> 3) & 1;
-          ldsm_x4(kf, kb + row * KSTR + h * 32 + half * 16);
+        const uint32_t kb = smem_u32(kbuf + (size_t(buf) * RS + j * kTileK) * KSTR);
+        uint32_t kf[4];
+        const int row = (lane & 7) + 8 * (lane >> 4);
+        const int half = (lane >> 3) & 1;
+        ldsm_x4(kf, kb + row * KSTR + h * 32 + half * 16);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) sf[j][0][e] = sf[j][1][e] = 0.f;
-          mma_bf16(sf[j][0], qa, kf[0], kf[1]);
-          mma_bf16(sf[j][1], qa, kf[2], kf[3]);
-        }
+        for (int e = 0; e < 4; ++e) sf[j][0][e] = sf[j][1][e] = 0.f;
+        mma_bf16(sf[j][0], qa, kf[0], kf[1]);
+        mma_bf16(sf[j][1], qa, kf[2], kf[3]);
       }
+      // ---- mask (rows g and g+8 of the tile; bit k <-> union atom ub + k);
+      // the stage's RS <= 32 bits sit in one mask word
+      const int ub = st * RS;
+      const uint32_t m0 = smask[g * swords + (ub >> 5)] >> ((ub & 31) + 2 * t);
+      const uint32_t m1 = smask[(g + 8) * swords + (ub >> 5)] >> ((ub & 31) + 2 * t);
+      float v[KS][8];   // raw logits; row g: cols 2t, 2t+1, 8+2t, 9+2t ; row g+8: same
+      bool over = false;
 #pragma unroll
       for (int j = 0; j < KS; ++j) {
-      const int s = st * KS + j;       // k-step
-      if (s >= nsteps) break;
-      const uint32_t vb = smem_u32(vbuf + (size_t(buf) * RS + j * kTileK) * VSTR);
-      const int u0 = s * kTileK;
-      const float* s0 = sf[j][0];
-      const float* s1 = sf[j][1];
-
-      // ---- mask (rows g and g+8 of the tile; bit k <-> union atom u0 + k)
-      const uint32_t w0 = smask[g * swords + (u0 >> 5)] >> ((u0 & 31) + 2 * t);
-      const uint32_t w1 = smask[(g + 8) * swords + (u0 >> 5)] >> ((u0 & 31) + 2 * t);
-      float v[8];   // raw logits; row g: cols 2t, 2t+1, 8+2t, 9+2t ; row g+8: same
-      v[0] = (w0 & 1u) ? s0[0] : -INFINITY;
-      v[1] = (w0 & 2u) ? s0[1] : -INFINITY;
-      v[2] = (w0 & 0x100u) ? s1[0] : -INFINITY;
-      v[3] = (w0 & 0x200u) ? s1[1] : -INFINITY;
-      v[4] = (w1 & 1u) ? s0[2] : -INFINITY;
-      v[5] = (w1 & 2u) ? s0[3] : -INFINITY;
-      v[6] = (w1 & 0x100u) ? s1[2] : -INFINITY;
-      v[7] = (w1 & 0x200u) ? s1[3] : -INFINITY;
-      // ---- online softmax.  Common case: no logit of the warp's rows exceeds
-      // its row's raw threshold (mref + kLazy) / qs, tested per entry with no
-      // cross-lane traffic.  Otherwise the row maxima are formed exactly and
-      // the rows that need it are rescaled.
-      const bool over = (v[0] > thr0) | (v[1] > thr0) | (v[2] > thr0) | (v[3] > thr0) |
-                        (v[4] > thr1) | (v[5] > thr1) | (v[6] > thr1) | (v[7] > thr1);
+        const uint32_t w0 = m0 >> (16 * j), w1 = m1 >> (16 * j);
+        v[j][0] = (w0 & 1u) ? sf[j][0][0] : -INFINITY;
+        v[j][1] = (w0 & 2u) ? sf[j][0][1] : -INFINITY;
+        v[j][2] = (w0 & 0x100u) ? sf[j][1][0] : -INFINITY;
+        v[j][3] = (w0 & 0x200u) ? sf[j][1][1] : -INFINITY;
+        v[j][4] = (w1 & 1u) ? sf[j][0][2] : -INFINITY;
+        v[j][5] = (w1 & 2u) ? sf[j][0][3] : -INFINITY;
+        v[j][6] = (w1 & 0x100u) ? sf[j][1][2] : -INFINITY;
+        v[j][7] = (w1 & 0x200u) ? sf[j][1][3] : -INFINITY;
+        over |= (v[j][0] > thr0) | (v[j][1] > thr0) | (v[j][2] > thr0) | (v[j][3] > thr0) |
+                (v[j][4] > thr1) | (v[j][5] > thr1) | (v[j][6] > thr1) | (v[j][7] > thr1);
+      }
+      // ---- online softmax, one test per stage.  Common case: no logit of
+      // the warp's rows exceeds its row's raw threshold (mref + kLazy) / qs,
+      // tested per entry with no cross-lane traffic.  Otherwise the row
+      // maxima over the stage are formed exactly and the rows that need it
+      // are rescaled.
       if (__any_sync(0xffffffffu, over)) {
-        float mx0 = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
-        float mx1 = fmaxf(fmaxf(v[4], v[5]), fmaxf(v[6], v[7]));
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < KS; ++j) {
+          mx0 = fmaxf(mx0, fmaxf(fmaxf(v[j][0], v[j][1]), fmaxf(v[j][2], v[j][3])));
+          mx1 = fmaxf(mx1, fmaxf(fmaxf(v[j][4], v[j][5]), fmaxf(v[j][6], v[j][7])));
+        }
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
@@ -346,23 +351,25 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
           thr1 = (mref1 + kLazy) * inv_qs;
         }
       }
-      float pr[8];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) pr[e] = fast_exp2(fmaf(v[e], qs, -mref0));
+      for (int j = 0; j < KS; ++j) {
+        float pr[8];
 #pragma unroll
-      for (int e = 4; e < 8; ++e) pr[e] = fast_exp2(fmaf(v[e], qs, -mref1));
-      uint32_t pa[4];
-      {
-        __nv_bfloat162 b;
-        b = __floats2bfloat162_rn(pr[0], pr[1]); pa[0] = *reinterpret_cast<uint32_t*>(&b);  // row g,   k 2t
-        b = __floats2bfloat162_rn(pr[4], pr[5]); pa[1] = *reinterpret_cast<uint32_t*>(&b);  // row g+8, k 2t
-        b = __floats2bfloat162_rn(pr[2], pr[3]); pa[2] = *reinterpret_cast<uint32_t*>(&b);  // row g,   k 2t+8
-        b = __floats2bfloat162_rn(pr[6], pr[7]); pa[3] = *reinterpret_cast<uint32_t*>(&b);  // row g+8, k 2t+8
-      }
-      mma_bf16(zacc, pa, kOnes, kOnes);
+        for (int e = 0; e < 4; ++e) pr[e] = fast_exp2(fmaf(v[j][e], qs, -mref0));
+#pragma unroll
+        for (int e = 4; e < 8; ++e) pr[e] = fast_exp2(fmaf(v[j][e], qs, -mref1));
+        uint32_t pa[4];
+        {
+          __nv_bfloat162 b;
+          b = __floats2bfloat162_rn(pr[0], pr[1]); pa[0] = *reinterpret_cast<uint32_t*>(&b);  // row g,   k 2t
+          b = __floats2bfloat162_rn(pr[4], pr[5]); pa[1] = *reinterpret_cast<uint32_t*>(&b);  // row g+8, k 2t
+          b = __floats2bfloat162_rn(pr[2], pr[3]); pa[2] = *reinterpret_cast<uint32_t*>(&b);  // row g,   k 2t+8
+          b = __floats2bfloat162_rn(pr[6], pr[7]); pa[3] = *reinterpret_cast<uint32_t*>(&b);  // row g+8, k 2t+8
+        }
+        mma_bf16(zacc, pa, kOnes, kOnes);
 
-      // ---- O += P V (one n8 tile per component of this head's 8 channels)
-      {
+        // ---- O += P V (one n8 tile per component of this head's 8 channels)
+        const uint32_t vb = smem_u32(vbuf + (size_t(buf) * RS + j * kTileK) * VSTR);
         const int mj = lane >> 3;                 // matrix of this lane's row address
         const int row = (lane & 7) + 8 * (mj & 1);
         const uint32_t base = vb + row * VSTR + h * 16;
@@ -378,7 +385,6 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
           ldsm_x2_t(vf, base + (D - 1) * (C * 2));
           mma_bf16(acc[D - 1], pa, vf[0], vf[1]);
         }
-      }
       }   // k-steps of the stage
     }
     cp_async_wait<0>();
