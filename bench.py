@@ -4,7 +4,8 @@
 
 One step = one pass of the whole hot path over one synthetic system:
 radius graph (egat_build_graph) -> attention plan (egat_build_attention_plan,
-tensor-core shapes) -> EAAS source coupling (egat_eaas_couple) -> on-the-fly
+tensor-core shapes) -> EAAS source coupling (egat_eaas_couple_planned with the
+plan's rotations on tensor-core shapes, egat_eaas_couple otherwise) -> on-the-fly
 attention with the target coupling fused (egat_otf_attention_tiled on
 tensor-core shapes, egat_otf_attention_coupled otherwise).
 The default workload is the 32,768-atom, K = 256, ℓmax = 2, bf16-storage
@@ -42,12 +43,14 @@ METRIC = "atoms/s & edges/s, fused EAAS+on-the-fly attention; % of HBM roofline"
 DEFAULT_WORKLOAD = "uniform32768_K256_l2_bf16"
 FLUSH_BYTES = 256 << 20
 #: kernels this library launches per step: graph (assign, scan x3, scatter,
-#: rank, fill, truncated-row fix) + attention plan (tensor-core shapes) +
-#: source coupling + fused attention
+#: rank, fill, truncated-row fix) + attention plan (tensor-core shapes: unions
+#: and masks, tile records) + source coupling + fused attention
 LAUNCHES_GRAPH = 8
+LAUNCHES_PLAN = 2
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attention_traffic.json")
 KERNEL_SOURCES = ["equivariant_graph_attention_b200/csrc/attention.cu",
                   "equivariant_graph_attention_b200/csrc/attention_tc.cu",
+                  "equivariant_graph_attention_b200/csrc/plan.cu",
                   "equivariant_graph_attention_b200/csrc/egat_device.cuh"]
 
 
@@ -253,10 +256,6 @@ def main():
                                   gws.data_ptr(), gws.numel(), sp)
         egat._check("egat_build_graph", rc)
 
-    def couple():
-        rc = lib.egat_eaas_couple(ctypes.byref(cshape), h.data_ptr(), pos.data_ptr(),
-                                  w1.data_ptr(), hp.data_ptr(), sp)
-        egat._check("egat_eaas_couple", rc)
 
     plan_sz = ctypes.c_size_t(0)
     tiled = (lib.egat_attention_plan_bytes(ctypes.byref(cshape), ctypes.byref(plan_sz)) == 0
@@ -269,15 +268,25 @@ def main():
     def build_plan():
         if tiled:
             rc = lib.egat_build_attention_plan(ctypes.byref(cshape), nbr.data_ptr(),
-                                               cnt.data_ptr(), order.data_ptr(), plan.data_ptr(),
-                                               plan.numel(), sp)
+                                               cnt.data_ptr(), order.data_ptr(), pos.data_ptr(),
+                                               plan.data_ptr(), plan.numel(), sp)
             egat._check("egat_build_attention_plan", rc)
+
+    def couple():
+        if tiled:   # rotations from the plan's tile records
+            rc = lib.egat_eaas_couple_planned(ctypes.byref(cshape), h.data_ptr(), plan.data_ptr(),
+                                              w1.data_ptr(), hp.data_ptr(), sp)
+            egat._check("egat_eaas_couple_planned", rc)
+        else:
+            rc = lib.egat_eaas_couple(ctypes.byref(cshape), h.data_ptr(), pos.data_ptr(),
+                                      w1.data_ptr(), hp.data_ptr(), sp)
+            egat._check("egat_eaas_couple", rc)
 
     def attend():
         if tiled:
             rc = lib.egat_otf_attention_tiled(ctypes.byref(cshape), q.data_ptr(), k.data_ptr(),
-                                              hp.data_ptr(), plan.data_ptr(), order.data_ptr(),
-                                              pos.data_ptr(), w2.data_ptr(), out.data_ptr(), 1, sp)
+                                              hp.data_ptr(), plan.data_ptr(), w2.data_ptr(),
+                                              out.data_ptr(), 1, sp)
             egat._check("egat_otf_attention_tiled", rc)
         else:
             rc = lib.egat_otf_attention_coupled(ctypes.byref(cshape), q.data_ptr(), k.data_ptr(),
@@ -286,7 +295,7 @@ def main():
                                                 out.data_ptr(), sp)
             egat._check("egat_otf_attention_coupled", rc)
     attn_name = "otf_attention_tiled" if tiled else "otf_attention_coupled"
-    launches_per_step = LAUNCHES_GRAPH + (1 if tiled else 0) + 2
+    launches_per_step = LAUNCHES_GRAPH + (LAUNCHES_PLAN if tiled else 0) + 2
 
     for _ in range(args.warmup):
         flush.fill_(1)
@@ -408,6 +417,10 @@ def main():
         e2e_ms = float(tt.item())
     e2e_value = wl.n * ws * args.e2e_steps / (e2e_ms / 1000.0)
     e2e_ok = bool(torch.equal(host_out[0].to(dev), out))   # pipelined result == device-timed result
+    # no bounded device wait may have given up in any of the runs above
+    status = lib.egat_take_device_status(torch.cuda.current_stream(dev).cuda_stream)
+    if status != egat.EGAT_OK:
+        raise RuntimeError(f"device status after the runs: {lib.egat_strerror(status).decode()}")
 
     # ------------------------------------------------------------------ roofline
     peaks = measured_peaks()

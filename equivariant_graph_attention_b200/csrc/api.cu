@@ -44,7 +44,7 @@ size_t hp_bytes(const egat_shape& s) {
 // forward workspace: h', then (tensor-core shapes) the attention plan
 size_t forward_ws_bytes(const egat_shape& s) {
   size_t b = hp_bytes(s);
-  if (tc_attention_supported(s) && s.n > 0) b += plan_bytes(s.n, s.K);
+  if (tc_attention_supported(s) && s.n > 0) b += plan_bytes(s.n, s.K, s.lmax);
   return b;
 }
 
@@ -63,6 +63,7 @@ const char* egat_strerror(int code) {
     case EGAT_ERR_WORKSPACE: return "workspace too small";
     case EGAT_ERR_SCRATCH_LIMIT:
       return "problem needs more scratch than egat_forward_noalloc's fixed array holds";
+    case EGAT_ERR_TIMEOUT: return "a bounded device wait gave up (results of that launch are invalid)";
     default: return "unknown egat status";
   }
 }
@@ -167,40 +168,52 @@ int egat_attention_plan_bytes(const egat_shape* s, size_t* bytes) {
   if (rc != EGAT_OK) return rc;
   if (s->graph_mode != EGAT_GRAPH_PADDED) return EGAT_ERR_UNSUPPORTED;
   if (plan_smem_bytes(s->n, s->K) > kPlanSmemLimit) return EGAT_ERR_UNSUPPORTED;
-  *bytes = s->n > 0 ? plan_bytes(s->n, s->K) : 0;
+  *bytes = s->n > 0 ? plan_bytes(s->n, s->K, s->lmax) : 0;
   return EGAT_OK;
 }
 
 int egat_build_attention_plan(const egat_shape* s, const int32_t* d_nbr, const int32_t* d_cnt,
-                              const int32_t* d_order, void* d_plan, size_t plan_bytes_given,
-                              void* stream) {
+                              const int32_t* d_order, const float* d_pos, void* d_plan,
+                              size_t plan_bytes_given, void* stream) {
   const int rc = check_shape(s, true);
   if (rc != EGAT_OK) return rc;
   if (s->graph_mode != EGAT_GRAPH_PADDED) return EGAT_ERR_UNSUPPORTED;
   if (plan_smem_bytes(s->n, s->K) > kPlanSmemLimit) return EGAT_ERR_UNSUPPORTED;
   if (s->n == 0) return EGAT_OK;
-  if (!d_nbr || !d_plan) return EGAT_ERR_ARG;
-  if (!aligned16(d_plan) || !aligned4(d_nbr)) return EGAT_ERR_ARG;
-  if (plan_bytes_given < plan_bytes(s->n, s->K)) return EGAT_ERR_WORKSPACE;
-  return launch_build_plan(s->n, s->K, d_nbr, d_cnt, d_order, d_plan,
+  if (!d_nbr || !d_pos || !d_plan) return EGAT_ERR_ARG;
+  if (!aligned16(d_plan) || !aligned4(d_nbr) || !aligned4(d_pos)) return EGAT_ERR_ARG;
+  if (plan_bytes_given < plan_bytes(s->n, s->K, s->lmax)) return EGAT_ERR_WORKSPACE;
+  return launch_build_plan(s->n, s->K, s->lmax, d_nbr, d_cnt, d_order, d_pos, d_plan,
                            static_cast<cudaStream_t>(stream));
 }
 
+int egat_eaas_couple_planned(const egat_shape* s, const void* d_h, const void* d_plan,
+                             const float* d_w1, void* d_hout, void* stream) {
+  const int rc = check_shape(s, true);
+  if (rc != EGAT_OK) return rc;
+  if (s->graph_mode != EGAT_GRAPH_PADDED) return EGAT_ERR_UNSUPPORTED;
+  if (plan_smem_bytes(s->n, s->K) > kPlanSmemLimit) return EGAT_ERR_UNSUPPORTED;
+  if (s->n == 0) return EGAT_OK;
+  if (!d_h || !d_plan || !d_w1 || !d_hout) return EGAT_ERR_ARG;
+  if (!aligned16(d_h) || !aligned16(d_plan) || !aligned16(d_hout) || !aligned4(d_w1))
+    return EGAT_ERR_ARG;
+  return launch_eaas_planned(*s, d_h, d_plan, d_w1, d_hout, static_cast<cudaStream_t>(stream));
+}
+
 int egat_otf_attention_tiled(const egat_shape* s, const void* d_q, const void* d_k,
-                             const void* d_hp, const void* d_plan, const int32_t* d_order,
-                             const float* d_pos, const float* d_w2, float* d_out, int32_t fused,
-                             void* stream) {
+                             const void* d_hp, const void* d_plan, const float* d_w2,
+                             float* d_out, int32_t fused, void* stream) {
   const int rc = check_shape(s, true);
   if (rc != EGAT_OK) return rc;
   if (!tc_attention_supported(*s)) return EGAT_ERR_UNSUPPORTED;
   if (s->n == 0) return EGAT_OK;
   if (!d_q || !d_k || !d_hp || !d_plan || !d_out) return EGAT_ERR_ARG;
-  if (fused && (!d_pos || !d_w2)) return EGAT_ERR_ARG;
+  if (fused && !d_w2) return EGAT_ERR_ARG;
   if (!aligned16(d_q) || !aligned16(d_k) || !aligned16(d_hp) || !aligned16(d_plan) ||
       !aligned16(d_out))
     return EGAT_ERR_ARG;
-  if (fused && (!aligned4(d_pos) || !aligned4(d_w2))) return EGAT_ERR_ARG;
-  return launch_attention_tc(*s, fused != 0, d_q, d_k, d_hp, d_plan, d_order, d_pos, d_w2, d_out,
+  if (fused && !aligned4(d_w2)) return EGAT_ERR_ARG;
+  return launch_attention_tc(*s, fused != 0, d_q, d_k, d_hp, d_plan, d_w2, d_out,
                              static_cast<cudaStream_t>(stream));
 }
 
@@ -221,11 +234,12 @@ int egat_forward(const egat_shape* s, const void* d_h, const float* d_pos, const
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (tc_attention_supported(*s)) {
     void* plan = static_cast<char*>(d_ws) + hp_bytes(*s);
-    int e = launch_build_plan(s->n, s->K, d_nbr_or_rowptr, d_cnt_or_col, d_order, plan, st);
+    int e = launch_build_plan(s->n, s->K, s->lmax, d_nbr_or_rowptr, d_cnt_or_col, d_order, d_pos,
+                              plan, st);
     if (e != EGAT_OK) return e;
-    e = launch_eaas_source(*s, d_h, d_pos, d_w1, d_ws, st);
+    e = launch_eaas_planned(*s, d_h, plan, d_w1, d_ws, st);
     if (e != EGAT_OK) return e;
-    return launch_attention_tc(*s, true, d_q, d_k, d_ws, plan, d_order, d_pos, d_w2, d_out, st);
+    return launch_attention_tc(*s, true, d_q, d_k, d_ws, plan, d_w2, d_out, st);
   }
   int e = launch_eaas_source(*s, d_h, d_pos, d_w1, d_ws, st);
   if (e != EGAT_OK) return e;
@@ -234,3 +248,15 @@ int egat_forward(const egat_shape* s, const void* d_h, const float* d_pos, const
 }
 
 }  // extern "C"
+
+int egat_take_device_status(void* stream) {
+  unsigned int n = 0;
+  const int rc = take_wait_timeouts(static_cast<cudaStream_t>(stream), &n);
+  if (rc != EGAT_OK) return rc;
+  return n ? EGAT_ERR_TIMEOUT : EGAT_OK;
+}
+
+int egat_selftest_wait_timeout(int32_t polls, void* stream) {
+  if (polls < 1 || polls > (1 << 20)) return EGAT_ERR_ARG;
+  return launch_wait_timeout_selftest(polls, static_cast<cudaStream_t>(stream));
+}

@@ -11,18 +11,26 @@
 //
 // How it maps to B200: a tile of 16 spatially adjacent targets (consecutive
 // in the cell order) reads each row of the union of their neighbour lists
-// once.  One warp per head; per k-step of 16 union atoms:
-//  * the tile's union indices and membership mask are copied to shared
-//    memory once; the 16 key rows and 16 value rows of a step are staged in
-//    shared memory with cp.async (32 threads per row; rows padded by 16 bytes
-//    so ldmatrix phases hit distinct banks), kept `STAGES` steps ahead;
-//  * S = Q_h K_h^T with two mma.sync m16n8k16 (bf16 in, f32 out), the key
-//    fragments by one ldmatrix.x4;
+// once.  A persistent CTA per SM, one warp per head; per tile:
+//  * the tile's union indices and membership mask (from the plan) go to
+//    shared memory, and so does its record: the 16 target ids, |r|^l and the
+//    Wigner-D matrices of their alignment rotations, built once per atom by
+//    the plan, so nothing is rebuilt here;
+//  * the union streams through shared memory in stages of RS rows, STAGES
+//    stages in flight: one thread per row issues its value row and key row as
+//    two bulk copies (cp.async.bulk, the TMA engine's 1-D form, no multicast)
+//    that complete the stage buffer's mbarrier by their byte count; rows are
+//    padded by 16 bytes so ldmatrix phases hit distinct banks.  Every wait on
+//    an mbarrier is bounded (bounded_wait): a wait that gives up is counted
+//    for egat_take_device_status and the CTA stops waiting, so no launch can
+//    hang;
+//  * per 16 union atoms and head, S = Q_h K_h^T with two mma.sync m16n8k16
+//    (bf16 in, f32 out), the key fragments by one ldmatrix.x4;
 //  * the plan's membership bits mask S to each target's own neighbours; the
 //    online softmax keeps a per-row reference maximum raised lazily (only by
-//    more than 2^8), so z and the accumulators share one reference; z is the
-//    mma of P with an all-ones fragment — the row sums of exactly the bf16
-//    weights that enter P V;
+//    more than 2^8), tested once per stage, so z and the accumulators share
+//    one reference; z is the mma of P with an all-ones fragment — the row
+//    sums of exactly the bf16 weights that enter P V;
 //  * the probabilities become the bf16 A fragment directly (the S fragment
 //    layout of two n8 tiles is the A layout of one k16 step) and P V_h runs
 //    as one mma.sync per component of the head's 8 channels, the value
@@ -39,6 +47,8 @@ namespace egat {
 namespace {
 
 constexpr int kRowPad = 16;   // bytes of padding per staged row
+// stage mbarriers (up to 3) and the abort flag, after 16-byte alignment
+constexpr size_t kBarBytes = 16 + 8 * 3 + 8;
 
 struct TcParams {
   const __nv_bfloat16* q;
@@ -57,13 +67,59 @@ struct TcParams {
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src));
+// mbarrier and bulk-copy (TMA engine, no multicast) helpers
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count));
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+
+// Waits that gave up since the last egat_take_device_status (all launches on
+// this device).
+__device__ unsigned int g_wait_timeouts;
+// Polls before a wait gives up.  try_wait suspends the thread for at most a
+// hardware-defined interval per poll, so this bounds a wait to about a
+// second; a stage's copies normally land within microseconds.
+constexpr int kWaitPolls = 1 << 20;
+constexpr int kDrainPolls = 1 << 14;
+
+// Wait until the phase of parity `parity` of the mbarrier at `bar` has
+// completed, polling at most `polls` times.  On giving up: count it, set the
+// CTA's abort flag and return false; once the flag is set, waits return at
+// once, so a CTA whose copies never land finishes its loop (with meaningless
+// results, reported by egat_take_device_status) instead of hanging.
+__device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, int polls,
+                                             volatile int* abort_flag) {
+  if (*abort_flag) return false;
+  for (int i = 0; i < polls; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  atomicAdd(&g_wait_timeouts, 1u);
+  *abort_flag = 1;
+  return false;
 }
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
@@ -145,6 +201,15 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
   int* su = tgt + kTileM;                                            // [cap]
   uint32_t* smask = reinterpret_cast<uint32_t*>(su + p.plan.cap);    // [16][cap / 32 + 1]
   float* sw2 = reinterpret_cast<float*>(smask + kTileM * (p.plan.cap / 32 + 1));   // [P][C]
+  uint64_t* fullbar = reinterpret_cast<uint64_t*>(
+      (reinterpret_cast<uintptr_t>(sw2 + (FUSED ? num_paths(L) * C : 0)) + 15) & ~uintptr_t(15));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(fullbar + STAGES);
+  if (threadIdx.x == 0) {
+    // one arrival per staged row of a stage; its bulk copies add the bytes
+    for (int b = 0; b < STAGES; ++b) mbar_init(smem_u32(fullbar + b), RS);
+    mbar_fence_init();
+    *abort_flag = 0;
+  }
   if constexpr (FUSED) {
     for (int e = threadIdx.x; e < num_paths(L) * C; e += H * 32) sw2[e] = __ldg(p.w2 + e);
   }
@@ -159,6 +224,7 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
   const char* hp_bytes = reinterpret_cast<const char*>(p.hp);
   const char* k_bytes = reinterpret_cast<const char*>(p.k);
 
+  int gbase = 0;   // stages staged by this CTA before the current tile
   for (int tile = blockIdx.x; tile < pv.tiles; tile += gridDim.x) {
     const int U = pv.ulen[tile];
     const int nsteps = (U + kTileK - 1) / kTileK;         // k-steps of 16 union rows
@@ -167,14 +233,16 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
     // whole stages with its first atom, whose mask bits there are zero
     const int ustep = nsteps * kTileK;
     const int* __restrict__ uni = pv.uni + (long long)tile * pv.cap;
-    const uint32_t* __restrict__ mrow = pv.mask + (long long)tile * kTileM * words;
+    const uint32_t* __restrict__ mrow = pv.mask + (long long)tile * words * kTileM;
 
-    if (tid < kTileM) {
-      const long long slot = (long long)tile * kTileM + tid;
-      int tg = -1;
-      if (slot < p.n) tg = p.order ? p.order[slot] : int(slot);
-      if ((unsigned)tg >= (unsigned)p.n) tg = -1;
-      tgt[tid] = tg;
+    {
+      constexpr int RW = kTileM * (1 + (L + 1) + WS);
+      const float* R = pv.rec + (long long)tile * RW;
+      if (tid < kTileM) tgt[tid] = reinterpret_cast<const int*>(R)[tid];
+      if constexpr (FUSED) {
+        for (int e = tid; e < kTileM * (L + 1); e += NTHR) rp[e] = R[kTileM + e];
+        for (int e = tid; e < kTileM * WS; e += NTHR) Dq[e] = R[kTileM * (2 + L) + e];
+      }
     }
     // the tile's union indices and membership mask into shared memory
     const int upad = nstages * RS;
@@ -182,42 +250,31 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
     for (int e = tid; e < upad; e += NTHR) su[e] = uni[e < ustep ? e : 0];
     for (int e = tid; e < kTileM * uw; e += NTHR) {
       const int r = e / uw, w = e % uw;
-      smask[r * swords + w] = mrow[r * words + w];
+      smask[r * swords + w] = mrow[w * kTileM + r];
     }
     if (upad > 32 * uw && tid < kTileM) smask[tid * swords + uw] = 0u;
     __syncthreads();   // tgt, su, smask visible
 
     // 32 threads per staged row; each copies chunks lane, lane + 32, ... of
     // the row's value and key bytes (rows past the padded union are skipped)
+    // one thread per staged row: its value row and key row as two bulk copies
+    // whose bytes complete the stage buffer's mbarrier phase
     auto issue = [&](int stage) {
-      const int buf = stage % STAGES;
-      unsigned char* vb = vbuf + size_t(buf) * RS * VSTR;
-      unsigned char* kb = kbuf + size_t(buf) * RS * KSTR;
-      for (int r = tid >> 5; r < RS; r += NTHR / 32) {
-        const int u = stage * RS + r;
-        if (u >= upad) break;
-        const long long atom = su[u];
-        const char* vsrc = hp_bytes + atom * ROW + lane * 16;
-        const char* ksrc = k_bytes + atom * KROW + lane * 16;
-        const uint32_t vdst = smem_u32(vb + r * VSTR + lane * 16);
-        const uint32_t kdst = smem_u32(kb + r * KSTR + lane * 16);
-#pragma unroll
-        for (int i = 0; i < VCH / 32; ++i) cp_async16(vdst + i * 512, vsrc + i * 512);
-        if constexpr (VCH % 32) {
-          if (lane < VCH % 32) cp_async16(vdst + (VCH / 32) * 512, vsrc + (VCH / 32) * 512);
-        }
-#pragma unroll
-        for (int i = 0; i < KCH / 32; ++i) cp_async16(kdst + i * 512, ksrc + i * 512);
-        if constexpr (KCH % 32) {
-          if (lane < KCH % 32) cp_async16(kdst + (KCH / 32) * 512, ksrc + (KCH / 32) * 512);
-        }
+      const int gs = gbase + stage;
+      const int buf = gs % STAGES;
+      constexpr int RSTRIDE = NTHR / RS;
+      if (tid % RSTRIDE == 0) {
+        const int r = tid / RSTRIDE;
+        const long long atom = su[stage * RS + r];
+        const uint32_t bar = smem_u32(fullbar + buf);
+        mbar_arrive_expect_tx(bar, ROW + KROW);
+        bulk_g2s(smem_u32(vbuf + (size_t(buf) * RS + r) * VSTR), hp_bytes + atom * ROW, ROW, bar);
+        bulk_g2s(smem_u32(kbuf + (size_t(buf) * RS + r) * KSTR), k_bytes + atom * KROW, KROW, bar);
       }
     };
 #pragma unroll
-    for (int s = 0; s < STAGES - 1; ++s) {
+    for (int s = 0; s < STAGES - 1; ++s)
       if (s < nstages) issue(s);
-      cp_async_commit();
-    }
 
     // Q fragment of this head for the tile's 16 targets
     uint32_t qa[4];
@@ -229,26 +286,6 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
       qa[2] = t0 >= 0 ? __ldg(q32 + ((size_t)t0 * H * 16 + h * 16 + 2 * t + 8) / 2) : 0u;
       qa[3] = t1 >= 0 ? __ldg(q32 + ((size_t)t1 * H * 16 + h * 16 + 2 * t + 8) / 2) : 0u;
     }
-    if constexpr (FUSED) {
-      // Wigner-D matrices of the tile's targets, one warp per target
-      for (int r = h; r < kTileM; r += H) {
-        const int tg = tgt[r];
-        float Q[9];
-        float rr = 0.f;
-        if (tg >= 0) rr = alignment_rotation(p.pos[3 * tg], p.pos[3 * tg + 1], p.pos[3 * tg + 2], Q);
-        else alignment_rotation(0.f, 0.f, 0.f, Q);
-        wigner_build<L>(Q, Dq + r * WS, lane, 32, [] { __syncwarp(); });
-        if (lane == 0) {
-          float a = 1.f;
-#pragma unroll
-          for (int l = 0; l <= L; ++l) {
-            rp[r * (L + 1) + l] = a;
-            a *= rr;
-          }
-        }
-      }
-    }
-
     float acc[D][4];
 #pragma unroll
     for (int d = 0; d < D; ++d)
@@ -269,11 +306,11 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
     float thr0 = -INFINITY, thr1 = -INFINITY;
 
     for (int st = 0; st < nstages; ++st) {
-      cp_async_wait<STAGES - 2>();
-      __syncthreads();
+      __syncthreads();   // every warp is done with the buffer about to be refilled
       if (st + STAGES - 1 < nstages) issue(st + STAGES - 1);
-      cp_async_commit();
-      const int buf = st % STAGES;
+      const int buf = (gbase + st) % STAGES;
+      bounded_wait(smem_u32(fullbar + buf), uint32_t((gbase + st) / STAGES) & 1u, kWaitPolls,
+                   abort_flag);
       // ---- S = Q K^T for every k-step of the stage (stages are whole:
       // the union is padded to a multiple of RS rows)
       float sf[KS][2][4];
@@ -387,8 +424,8 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
         }
       }   // k-steps of the stage
     }
-    cp_async_wait<0>();
-    __syncthreads();   // Dq / rp written; all staged buffers drained
+    __syncthreads();   // all staged buffers consumed
+    gbase += nstages;
 
     // ---- epilogue: normalise; either write m or apply the target coupling
     const float inv0 = zacc[0] > 0.f ? 1.f / zacc[0] : 0.f;
@@ -454,14 +491,37 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
                          });
       }
     }
+    if constexpr (FUSED && L >= 3) fence_proxy_async_smem();   // scratch before bulk copies
     __syncthreads();   // tgt / Dq / rp are rewritten by the next tile
+  }
+  if (*abort_flag && threadIdx.x == 0) {
+    // a wait gave up: give each buffer's last fill a short, bounded chance to
+    // land before the CTA's shared memory is released
+    volatile int none = 0;
+    for (int b = 0; b < STAGES && b < gbase; ++b)
+      bounded_wait(smem_u32(fullbar + b), uint32_t((gbase - 1 - b) / STAGES) & 1u, kDrainPolls, &none);
+  }
+}
+
+// A wait that cannot succeed: one arrival announces 16 bytes that no copy
+// will deliver, so the phase never completes and bounded_wait must give up
+// after `polls` polls — exercises the timeout report without any fault.
+__global__ void wait_timeout_selftest_kernel(int polls) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    mbar_fence_init();
+    mbar_arrive_expect_tx(smem_u32(&bar), 16);
+    bounded_wait(smem_u32(&bar), 0u, polls, &abort_flag);
   }
 }
 
 template <int L, int H, bool FUSED>
 int launch_tc_t(const TcParams& p, int tiles, cudaStream_t st) {
   const size_t shmem = tc_smem_fixed<L, H>() + tc_smem_plan(p.plan.cap) +
-                       (FUSED ? tc_smem_w2<L, H>() : 0);
+                       (FUSED ? tc_smem_w2<L, H>() : 0) + kBarBytes;
   if (shmem > 227 * 1024) return EGAT_ERR_UNSUPPORTED;
   auto kern = otf_attention_tc_kernel<L, H, FUSED>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(shmem)) !=
@@ -486,21 +546,21 @@ bool tc_attention_supported(const egat_shape& s) {
                      : s.lmax == 2 ? tc_smem_fixed<2, 16>() : tc_smem_fixed<3, 16>();
   const size_t w2 = s.lmax == 1 ? tc_smem_w2<1, 16>()
                   : s.lmax == 2 ? tc_smem_w2<2, 16>() : tc_smem_w2<3, 16>();
-  return fixed + tc_smem_plan(plan_capacity(s.K)) + w2 <= 227 * 1024;
+  return fixed + tc_smem_plan(plan_capacity(s.K)) + w2 + kBarBytes <= 227 * 1024;
 }
 
 int launch_attention_tc(const egat_shape& s, bool fused, const void* d_q, const void* d_k,
-                        const void* d_hp, const void* d_plan, const int32_t* d_order,
-                        const float* d_pos, const float* d_w2, float* d_out, cudaStream_t st) {
+                        const void* d_hp, const void* d_plan, const float* d_w2, float* d_out,
+                        cudaStream_t st) {
   if (!tc_attention_supported(s)) return EGAT_ERR_UNSUPPORTED;
   TcParams p;
   p.q = static_cast<const __nv_bfloat16*>(d_q);
   p.k = static_cast<const __nv_bfloat16*>(d_k);
   p.hp = static_cast<const __nv_bfloat16*>(d_hp);
-  p.plan = plan_view(const_cast<void*>(d_plan), s.n, s.K);
-  p.order = d_order;
+  p.plan = plan_view(const_cast<void*>(d_plan), s.n, s.K, s.lmax);
+  p.order = nullptr;
   p.out = d_out;
-  p.pos = d_pos;
+  p.pos = nullptr;
   p.w2 = d_w2;
   p.n = s.n;
   p.qscale = float(1.4426950408889634 / std::sqrt(double(s.dk)));
@@ -513,6 +573,22 @@ int launch_attention_tc(const egat_shape& s, bool fused, const void* d_q, const 
     case 3: return fused ? launch_tc_t<3, 16, true>(p, tiles, st) : launch_tc_t<3, 16, false>(p, tiles, st);
     default: return EGAT_ERR_UNSUPPORTED;
   }
+}
+
+int take_wait_timeouts(cudaStream_t st, unsigned int* count) {
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_wait_timeouts) != cudaSuccess) return EGAT_ERR_CUDA;
+  unsigned int h = 0;
+  if (cudaMemcpyAsync(&h, addr, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemsetAsync(addr, 0, sizeof(h), st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
+    return EGAT_ERR_CUDA;
+  *count = h;
+  return EGAT_OK;
+}
+
+int launch_wait_timeout_selftest(int polls, cudaStream_t st) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, st>>>(polls);
+  return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
 }
 
 }  // namespace egat

@@ -101,6 +101,8 @@ struct EaasParams {
   void* y;
   int n;
   int C;
+  const float* rec;   // planned form: the attention plan's tile records
+  long long items;    // atoms, or target slots of the plan (tiles * kTileM)
   EaasTable tab;
 };
 
@@ -160,7 +162,10 @@ struct ChanVec<float, 2> {
 // Wigner-D matrices once in shared memory (groups of up to 32 lanes inside a
 // warp; a 64-lane group spans two warps, each building its own copy), then
 // every lane couples its channels with the matrices held in registers.
-template <int L, typename T>
+// PLANNED: the items are the target slots of an attention plan, whose tile
+// records already hold each atom's index, |r|^l and Wigner-D matrices; the
+// group copies them instead of building them.
+template <int L, typename T, bool PLANNED>
 __global__ void __launch_bounds__(kEaasWarps * 32, (L >= 3 ? 1 : 2))
 eaas_source_kernel(const __grid_constant__ EaasParams p) {
   constexpr int D = (L + 1) * (L + 1);
@@ -184,7 +189,8 @@ eaas_source_kernel(const __grid_constant__ EaasParams p) {
   const long long nwarps = (long long)gridDim.x * kEaasWarps;
   const int part = int(gwarp % WPA);            // which warp of the atom's group
   const int c0 = (part * 32 + gl) * CPL;         // first channel of this lane
-  const long long ngroups = ((long long)p.n + AW - 1) / AW;
+  const long long ngroups = (p.items + AW - 1) / AW;
+  constexpr int REC = kTileM * (1 + (L + 1) + WS);
   const T* __restrict__ x = static_cast<const T*>(p.x);
   T* __restrict__ y = static_cast<T*>(p.y);
   float* Dme = Dsm[wib][slot];
@@ -192,13 +198,26 @@ eaas_source_kernel(const __grid_constant__ EaasParams p) {
   __syncthreads();
 
   for (long long grp = gwarp / WPA; grp < ngroups; grp += nwarps / WPA) {
-    const long long at = grp * AW + slot;
-    const bool live = at < p.n;
+    const long long item = grp * AW + slot;
+    long long at = item;
+    bool live = item < p.items;
+    const float* R = nullptr;
+    int rs = 0;
+    if constexpr (PLANNED) {
+      if (live) {
+        R = p.rec + (item / kTileM) * REC;
+        rs = int(item % kTileM);
+        at = reinterpret_cast<const int*>(R)[rs];
+        live = (unsigned long long)at < (unsigned long long)p.n;
+      }
+    }
     float Q[9];
     float r = 0.f;
-    if (live) r = alignment_rotation(__ldg(p.pos + 3 * at), __ldg(p.pos + 3 * at + 1),
-                                     __ldg(p.pos + 3 * at + 2), Q);
-    else alignment_rotation(0.f, 0.f, 0.f, Q);
+    if constexpr (!PLANNED) {
+      if (live) r = alignment_rotation(__ldg(p.pos + 3 * at), __ldg(p.pos + 3 * at + 1),
+                                       __ldg(p.pos + 3 * at + 2), Q);
+      else alignment_rotation(0.f, 0.f, 0.f, Q);
+    }
     float xv[CPL][D];
     if (live) {
       const T* xr = x + (size_t)at * D * C + c0;
@@ -211,11 +230,20 @@ eaas_source_kernel(const __grid_constant__ EaasParams p) {
       }
     }
     float rpow[L + 1];
-    rpow[0] = 1.f;
+    if constexpr (PLANNED) {
 #pragma unroll
-    for (int l = 1; l <= L; ++l) rpow[l] = rpow[l - 1] * r;
-    __syncwarp();                             // previous atom's readers are done
-    wigner_build<L>(Q, Dme, gl, GW, [] { __syncwarp(); });
+      for (int l = 0; l <= L; ++l) rpow[l] = live ? __ldg(R + kTileM + rs * (L + 1) + l) : 0.f;
+      __syncwarp();                           // previous atom's readers are done
+      if (live)
+        for (int e = gl; e < WS; e += GW) Dme[e] = __ldg(R + kTileM * (2 + L) + rs * WS + e);
+      __syncwarp();
+    } else {
+      rpow[0] = 1.f;
+#pragma unroll
+      for (int l = 1; l <= L; ++l) rpow[l] = rpow[l - 1] * r;
+      __syncwarp();                           // previous atom's readers are done
+      wigner_build<L>(Q, Dme, gl, GW, [] { __syncwarp(); });
+    }
     if (live) {
       T* yr = y + (size_t)at * D * C + c0;
       const float* swc = sw + c0;
@@ -224,10 +252,9 @@ eaas_source_kernel(const __grid_constant__ EaasParams p) {
     }
   }
 }
-
-template <int L, typename T>
-int launch_eaas_t(const egat_shape& s, const void* d_x, const float* d_pos, const float* d_w,
-                  void* d_y, cudaStream_t st) {
+template <int L, typename T, bool PLANNED>
+int launch_eaas_t(const egat_shape& s, const void* d_x, const float* d_pos, const float* rec,
+                  long long items, const float* d_w, void* d_y, cudaStream_t st) {
   EaasParams p;
   p.x = d_x;
   p.pos = d_pos;
@@ -235,19 +262,21 @@ int launch_eaas_t(const egat_shape& s, const void* d_x, const float* d_pos, cons
   p.y = d_y;
   p.n = s.n;
   p.C = s.C;
+  p.rec = rec;
+  p.items = items;
   p.tab = eaas_table(L);
   constexpr int CPL = L >= 3 ? 2 : 4;
   const int G = s.C / CPL;
   const int WPA = G > 32 ? G / 32 : 1;
   const int AW = 32 / (G > 32 ? 32 : G);
-  const long long groups = ((long long)s.n + AW - 1) / AW;
+  const long long groups = (items + AW - 1) / AW;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long want = (groups * WPA + kEaasWarps - 1) / kEaasWarps;
   const int grid = int(std::max<long long>(1, std::min<long long>(want, (long long)sms * 8)));
   const size_t shmem = size_t(num_paths(L)) * s.C * sizeof(float);
-  eaas_source_kernel<L, T><<<grid, kEaasWarps * 32, shmem, st>>>(p);
+  eaas_source_kernel<L, T, PLANNED><<<grid, kEaasWarps * 32, shmem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
 }
 
@@ -256,13 +285,30 @@ int launch_eaas_t(const egat_shape& s, const void* d_x, const float* d_pos, cons
 int launch_eaas_source(const egat_shape& s, const void* d_x, const float* d_pos,
                        const float* d_w, void* d_y, cudaStream_t st) {
   const bool bf = s.dtype == EGAT_BF16;
+  const long long n = s.n;
   switch (s.lmax) {
-    case 1: return bf ? launch_eaas_t<1, __nv_bfloat16>(s, d_x, d_pos, d_w, d_y, st)
-                      : launch_eaas_t<1, float>(s, d_x, d_pos, d_w, d_y, st);
-    case 2: return bf ? launch_eaas_t<2, __nv_bfloat16>(s, d_x, d_pos, d_w, d_y, st)
-                      : launch_eaas_t<2, float>(s, d_x, d_pos, d_w, d_y, st);
-    case 3: return bf ? launch_eaas_t<3, __nv_bfloat16>(s, d_x, d_pos, d_w, d_y, st)
-                      : launch_eaas_t<3, float>(s, d_x, d_pos, d_w, d_y, st);
+    case 1: return bf ? launch_eaas_t<1, __nv_bfloat16, false>(s, d_x, d_pos, nullptr, n, d_w, d_y, st)
+                      : launch_eaas_t<1, float, false>(s, d_x, d_pos, nullptr, n, d_w, d_y, st);
+    case 2: return bf ? launch_eaas_t<2, __nv_bfloat16, false>(s, d_x, d_pos, nullptr, n, d_w, d_y, st)
+                      : launch_eaas_t<2, float, false>(s, d_x, d_pos, nullptr, n, d_w, d_y, st);
+    case 3: return bf ? launch_eaas_t<3, __nv_bfloat16, false>(s, d_x, d_pos, nullptr, n, d_w, d_y, st)
+                      : launch_eaas_t<3, float, false>(s, d_x, d_pos, nullptr, n, d_w, d_y, st);
+    default: return EGAT_ERR_UNSUPPORTED;
+  }
+}
+
+int launch_eaas_planned(const egat_shape& s, const void* d_x, const void* d_plan, const float* d_w,
+                        void* d_y, cudaStream_t st) {
+  const bool bf = s.dtype == EGAT_BF16;
+  const PlanView pv = plan_view(const_cast<void*>(d_plan), s.n, s.K, s.lmax);
+  const long long items = (long long)pv.tiles * kTileM;
+  switch (s.lmax) {
+    case 1: return bf ? launch_eaas_t<1, __nv_bfloat16, true>(s, d_x, nullptr, pv.rec, items, d_w, d_y, st)
+                      : launch_eaas_t<1, float, true>(s, d_x, nullptr, pv.rec, items, d_w, d_y, st);
+    case 2: return bf ? launch_eaas_t<2, __nv_bfloat16, true>(s, d_x, nullptr, pv.rec, items, d_w, d_y, st)
+                      : launch_eaas_t<2, float, true>(s, d_x, nullptr, pv.rec, items, d_w, d_y, st);
+    case 3: return bf ? launch_eaas_t<3, __nv_bfloat16, true>(s, d_x, nullptr, pv.rec, items, d_w, d_y, st)
+                      : launch_eaas_t<3, float, true>(s, d_x, nullptr, pv.rec, items, d_w, d_y, st);
     default: return EGAT_ERR_UNSUPPORTED;
   }
 }

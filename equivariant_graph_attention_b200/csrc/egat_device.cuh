@@ -255,6 +255,79 @@ __device__ __forceinline__ float ir_entry(int l, int m, int mp, const float* D1,
   return val;
 }
 
+// The same recursion with every index and coefficient fixed at compile time:
+// one thread builds all of D^0..D^L in registers, straight-line, with no
+// branches, runtime square roots or shared memory.  D is the concatenated
+// block (wig_off); D^1 and D^{l-1} are read from it while D^l is written.
+__host__ __device__ constexpr double ct_sqrt(double x) {
+  if (x <= 0.0) return 0.0;
+  double r = x < 1.0 ? 1.0 : x;
+  for (int i = 0; i < 200; ++i) r = 0.5 * (r + x / r);   // Newton; converged long before
+  return r;
+}
+template <int l, int i, int a, int b, int N>
+__device__ __forceinline__ float ir_P(const float (&D)[N]) {
+  constexpr int o1 = wig_off(1), op = wig_off(l - 1), wp = 2 * l - 1;
+  constexpr int row = op + (a + l - 1) * wp;
+  if constexpr (b == l)
+    return D[o1 + (i + 1) * 3 + 2] * D[row + 2 * l - 2] - D[o1 + (i + 1) * 3 + 0] * D[row];
+  else if constexpr (b == -l)
+    return D[o1 + (i + 1) * 3 + 2] * D[row] + D[o1 + (i + 1) * 3 + 0] * D[row + 2 * l - 2];
+  else
+    return D[o1 + (i + 1) * 3 + 1] * D[row + b + l - 1];
+}
+template <int l, int m, int mp, int N>
+__device__ __forceinline__ float ir_entry_ct(const float (&D)[N]) {
+  constexpr double d = (iabs(mp) == l) ? double((2 * l) * (2 * l - 1)) : double((l + mp) * (l - mp));
+  constexpr int am = iabs(m);
+  float val = 0.f;
+  if constexpr (am < l) {
+    constexpr float u = float(ct_sqrt(double((l + m) * (l - m)) / d));
+    val += u * ir_P<l, 0, m, mp>(D);
+  }
+  {
+    constexpr float v = float(0.5 * ct_sqrt(double((m == 0 ? 2 : 1) * (l + am - 1) * (l + am)) / d) *
+                              (m == 0 ? -1.0 : 1.0));
+    float V;
+    if constexpr (m == 0) {
+      V = ir_P<l, 1, 1, mp>(D) + ir_P<l, -1, -1, mp>(D);
+    } else if constexpr (m == 1) {
+      V = ir_P<l, 1, 0, mp>(D) * 1.41421356237309515f;
+    } else if constexpr (m > 1) {
+      V = ir_P<l, 1, m - 1, mp>(D) - ir_P<l, -1, -m + 1, mp>(D);
+    } else if constexpr (m == -1) {
+      V = ir_P<l, -1, 0, mp>(D) * 1.41421356237309515f;
+    } else {
+      V = ir_P<l, 1, m + 1, mp>(D) + ir_P<l, -1, -m - 1, mp>(D);
+    }
+    val += v * V;
+  }
+  if constexpr (m != 0 && am < l - 1) {
+    constexpr float w = float(-0.5 * ct_sqrt(double((l - am - 1) * (l - am)) / d));
+    float W;
+    if constexpr (m > 0) W = ir_P<l, 1, m + 1, mp>(D) + ir_P<l, -1, -m - 1, mp>(D);
+    else W = ir_P<l, 1, m - 1, mp>(D) - ir_P<l, -1, -m + 1, mp>(D);
+    val += w * W;
+  }
+  return val;
+}
+template <int L>
+__device__ __forceinline__ void wigner_regs(const float (&Q)[9], float (&D)[wig_size(L)]) {
+  D[0] = 1.f;
+  static_for<0, 9>([&](auto ec) {
+    constexpr int e = decltype(ec)::value;
+    D[wig_off(1) + e] = Q[wig1_src(e)];
+  });
+  static_for<2, L + 1>([&](auto lc) {
+    constexpr int l = decltype(lc)::value;
+    constexpr int w = 2 * l + 1;
+    static_for<0, w * w>([&](auto ec) {
+      constexpr int e = decltype(ec)::value;
+      D[wig_off(l) + e] = ir_entry_ct<l, e / w - l, e % w - l>(D);
+    });
+  });
+}
+
 // Build D^0..D^L for one rotation into Dsm (wig_size(L) floats) using
 // `nthreads` cooperating threads (thread index `tid`); `sync` is called
 // between degrees.  Dsm must be visible to all cooperating threads.

@@ -42,28 +42,48 @@ inline size_t storage_bytes(int dtype) { return dtype == EGAT_BF16 ? 2 : 4; }
 constexpr int kTileM = 16;
 constexpr int kTileK = 16;
 
-// Per-tile neighbour union and membership bitmask (device memory views).
+// Per-tile neighbour union, membership bitmask and target record (device
+// memory views).  Unions are padded to whole multiples of kPlanPad entries
+// (at least one, also for an empty union) with a valid atom index whose mask
+// bits are zero, so that a consumer may stream them in chunks of kPlanPad.
+constexpr int kPlanPad = 32;
 struct PlanView {
   int* ulen;        // [tiles] union length
-  int* uni;         // [tiles][cap] union atom indices (ascending), padded to kTileK
-  uint32_t* mask;   // [tiles][kTileM][cap / 32] bit u of row r: union atom u is a neighbour
+  int* uni;         // [tiles][cap] union atom indices (ascending), padded to kPlanPad
+  uint32_t* mask;   // [tiles][cap / 32][kTileM] word w of row r: bits of union atoms 32w..32w+31
+  float* rec;       // [tiles][plan_record_words(lmax)] target ids, |r|^l, Wigner-D (see below)
   int cap;          // union capacity per tile (power of two >= kTileM * K)
   int tiles;
 };
+// Tile record: int32 target[kTileM] (-1 past n), float rpow[kTileM][lmax+1]
+// (|r|^0..|r|^lmax), float D[kTileM][wig_size(lmax)] (real Wigner-D of the
+// alignment rotation, degrees 0..lmax) — everything the attention epilogue
+// needs per target, so the attention kernel builds nothing per tile.
+inline int plan_record_words(int lmax) {
+  const int ws = (lmax + 1) * (2 * lmax + 1) * (2 * lmax + 3) / 3;   // sum of (2l+1)^2
+  return kTileM * (1 + (lmax + 1) + ws);
+}
 int plan_capacity(int K);
 // shared memory of the plan kernel: two bitmap-sized arrays over all atoms and
 // one tile mask; the tensor-core path is used while this fits a CTA
 size_t plan_smem_bytes(int n, int K);
 constexpr size_t kPlanSmemLimit = 200 * 1024;
-size_t plan_bytes(int n, int K);
-PlanView plan_view(void* base, int n, int K);
-int launch_build_plan(int n, int K, const int32_t* d_nbr, const int32_t* d_cnt,
-                      const int32_t* d_order, void* d_plan, cudaStream_t st);
+size_t plan_bytes(int n, int K, int lmax);
+PlanView plan_view(void* base, int n, int K, int lmax);
+int launch_build_plan(int n, int K, int lmax, const int32_t* d_nbr, const int32_t* d_cnt,
+                      const int32_t* d_order, const float* d_pos, void* d_plan, cudaStream_t st);
+// Step 2 for every atom listed in a plan's tile records, rotations from them.
+int launch_eaas_planned(const egat_shape& s, const void* d_x, const void* d_plan, const float* d_w,
+                        void* d_y, cudaStream_t st);
 // Tiled tensor-core attention (bf16 storage, C/H = 8, dk = 16): fused = true
 // applies the target coupling and writes ^h; false writes m.
 bool tc_attention_supported(const egat_shape& s);
+// Bounded-wait report of the tensor-core kernel: read and clear the count of
+// waits that gave up (synchronises st); the self-test launch.
+int take_wait_timeouts(cudaStream_t st, unsigned int* count);
+int launch_wait_timeout_selftest(int polls, cudaStream_t st);
 int launch_attention_tc(const egat_shape& s, bool fused, const void* d_q, const void* d_k,
-                        const void* d_hp, const void* d_plan, const int32_t* d_order,
-                        const float* d_pos, const float* d_w2, float* d_out, cudaStream_t st);
+                        const void* d_hp, const void* d_plan, const float* d_w2, float* d_out,
+                        cudaStream_t st);
 
 }  // namespace egat

@@ -11,7 +11,10 @@
 // One 256-thread CTA per tile builds the union from a shared-memory bitmap
 // over atom indices (ascending atom index: a deterministic order) and sets one
 // mask bit per (target, neighbour) at the position given by the bitmap's
-// prefix counts.
+// prefix counts.  A second kernel writes each tile's target record: target
+// ids, |r|^l and the real Wigner-D matrices of the targets' alignment
+// rotations ([EX] §2.1), which the target coupling of the attention epilogue
+// applies.
 #include "egat_device.cuh"
 #include "egat_host.h"
 
@@ -128,8 +131,9 @@ __global__ void __launch_bounds__(kPlanThreads) build_plan_kernel(const __grid_c
     }
   }
   __syncthreads();
-  // pad the union to a multiple of the k-step with a valid index (masked out)
-  const int upad = (U + kTileK - 1) / kTileK * kTileK;
+  // pad the union to whole chunks of kPlanPad (at least one) with a valid
+  // index whose mask bits stay zero
+  const int upad = U > 0 ? (U + kPlanPad - 1) / kPlanPad * kPlanPad : kPlanPad;
   const int filler = U > 0 ? uni[0] : 0;
   for (int e = U + threadIdx.x; e < upad; e += blockDim.x) uni[e] = filler;
   if (threadIdx.x == 0) pv.ulen[tile] = U;
@@ -142,11 +146,46 @@ __global__ void __launch_bounds__(kPlanThreads) build_plan_kernel(const __grid_c
     atomicOr(&mask[r * words + (pos >> 5)], 1u << (pos & 31));
   }
   __syncthreads();
-  uint32_t* gmask = pv.mask + (long long)tile * kTileM * words;
-  const int uw = (upad + 31) / 32;
+  // word-major in memory: the kTileM words of one 32-atom chunk are contiguous
+  uint32_t* gmask = pv.mask + (long long)tile * words * kTileM;
+  const int uw = upad / 32;
   for (int i = threadIdx.x; i < kTileM * uw; i += blockDim.x) {
-    const int r = i / uw, w = i % uw;
-    gmask[r * words + w] = mask[r * words + w];
+    const int w = i / kTileM, r = i % kTileM;
+    gmask[i] = mask[r * words + w];
+  }
+}
+
+// One thread per target slot (tile * kTileM + r): the slot's atom, |r|^l and
+// the Wigner-D matrices of its alignment rotation (identity for an empty slot
+// or an atom at the origin), built in registers, into the tile record.
+constexpr int kRecThreads = 128;
+template <int L>
+__global__ void __launch_bounds__(kRecThreads)
+tile_records_kernel(const int32_t* __restrict__ order, const float* __restrict__ pos, int n,
+                    int tiles, float* __restrict__ rec) {
+  constexpr int WS = wig_size(L);
+  constexpr int REC = kTileM * (1 + (L + 1) + WS);
+  const long long slot = (long long)blockIdx.x * kRecThreads + threadIdx.x;
+  if (slot >= (long long)tiles * kTileM) return;
+  const int tile = int(slot / kTileM), r = int(slot % kTileM);
+  int tg = -1;
+  if (slot < n) tg = order ? order[slot] : int(slot);
+  if ((unsigned)tg >= (unsigned)n) tg = -1;
+  float Q[9];
+  float rr = 0.f;
+  if (tg >= 0) rr = alignment_rotation(pos[3 * tg], pos[3 * tg + 1], pos[3 * tg + 2], Q);
+  else alignment_rotation(0.f, 0.f, 0.f, Q);
+  float D[WS];
+  wigner_regs<L>(Q, D);
+  float* R = rec + (long long)tile * REC;
+#pragma unroll
+  for (int e = 0; e < WS; ++e) R[kTileM * (2 + L) + r * WS + e] = D[e];
+  reinterpret_cast<int*>(R)[r] = tg;
+  float a = 1.f;
+#pragma unroll
+  for (int l = 0; l <= L; ++l) {
+    R[kTileM + r * (L + 1) + l] = a;
+    a *= rr;
   }
 }
 
@@ -163,15 +202,16 @@ int plan_capacity(int K) {
   return cap;
 }
 
-size_t plan_bytes(int n, int K) {
+size_t plan_bytes(int n, int K, int lmax) {
   const size_t tiles = (size_t(n) + kTileM - 1) / kTileM;
   const size_t cap = size_t(plan_capacity(K));
   auto a256 = [](size_t x) { return (x + 255) & ~size_t(255); };
   return a256(tiles * sizeof(int)) + a256(tiles * cap * sizeof(int)) +
-         a256(tiles * kTileM * (cap / 32) * sizeof(uint32_t));
+         a256(tiles * kTileM * (cap / 32) * sizeof(uint32_t)) +
+         a256(tiles * size_t(plan_record_words(lmax)) * sizeof(float));
 }
 
-PlanView plan_view(void* base, int n, int K) {
+PlanView plan_view(void* base, int n, int K, int lmax) {
   const size_t tiles = (size_t(n) + kTileM - 1) / kTileM;
   const int cap = plan_capacity(K);
   auto a256 = [](size_t x) { return (x + 255) & ~size_t(255); };
@@ -182,18 +222,21 @@ PlanView plan_view(void* base, int n, int K) {
   v.uni = reinterpret_cast<int*>(b);
   b += a256(tiles * size_t(cap) * sizeof(int));
   v.mask = reinterpret_cast<uint32_t*>(b);
+  b += a256(tiles * kTileM * (size_t(cap) / 32) * sizeof(uint32_t));
+  v.rec = reinterpret_cast<float*>(b);
+  (void)lmax;
   v.cap = cap;
   v.tiles = int(tiles);
   return v;
 }
 
-int launch_build_plan(int n, int K, const int32_t* d_nbr, const int32_t* d_cnt,
-                      const int32_t* d_order, void* d_plan, cudaStream_t st) {
+int launch_build_plan(int n, int K, int lmax, const int32_t* d_nbr, const int32_t* d_cnt,
+                      const int32_t* d_order, const float* d_pos, void* d_plan, cudaStream_t st) {
   PlanParams p;
   p.nbr = d_nbr;
   p.cnt = d_cnt;
   p.order = d_order;
-  p.plan = plan_view(d_plan, n, K);
+  p.plan = plan_view(d_plan, n, K, lmax);
   p.n = n;
   p.K = K;
   const size_t shmem = plan_smem_bytes(n, K);
@@ -203,6 +246,15 @@ int launch_build_plan(int n, int K, const int32_t* d_nbr, const int32_t* d_cnt,
       return EGAT_ERR_CUDA;
   }
   build_plan_kernel<<<p.plan.tiles, kPlanThreads, shmem, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return EGAT_ERR_CUDA;
+  const int tiles = p.plan.tiles;
+  const int blocks = (tiles * kTileM + kRecThreads - 1) / kRecThreads;
+  switch (lmax) {
+    case 1: tile_records_kernel<1><<<blocks, kRecThreads, 0, st>>>(d_order, d_pos, n, tiles, p.plan.rec); break;
+    case 2: tile_records_kernel<2><<<blocks, kRecThreads, 0, st>>>(d_order, d_pos, n, tiles, p.plan.rec); break;
+    case 3: tile_records_kernel<3><<<blocks, kRecThreads, 0, st>>>(d_order, d_pos, n, tiles, p.plan.rec); break;
+    default: return EGAT_ERR_UNSUPPORTED;
+  }
   return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
 }
 

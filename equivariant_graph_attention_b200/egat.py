@@ -26,6 +26,7 @@ EGAT_ERR_UNSUPPORTED = -2
 EGAT_ERR_CUDA = -3
 EGAT_ERR_WORKSPACE = -4
 EGAT_ERR_SCRATCH_LIMIT = -5
+EGAT_ERR_TIMEOUT = -6
 #: size of the fixed scratch array behind egat_forward_noalloc
 NOALLOC_SCRATCH_BYTES = 32 << 20
 EGAT_F32 = 0
@@ -38,7 +39,8 @@ EXPORTS = ["egat_version", "egat_strerror", "egat_num_paths", "egat_graph_worksp
            "egat_build_graph", "egat_eaas_couple", "egat_otf_attention",
            "egat_otf_attention_coupled",
            "egat_forward_workspace_bytes", "egat_forward", "egat_forward_noalloc",
-           "egat_attention_plan_bytes", "egat_build_attention_plan", "egat_otf_attention_tiled"]
+           "egat_attention_plan_bytes", "egat_build_attention_plan", "egat_otf_attention_tiled",
+           "egat_eaas_couple_planned", "egat_take_device_status", "egat_selftest_wait_timeout"]
 
 
 class EgatError(RuntimeError):
@@ -92,9 +94,15 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.egat_attention_plan_bytes.restype = ctypes.c_int
     lib.egat_attention_plan_bytes.argtypes = [sp, ctypes.POINTER(sz)]
     lib.egat_build_attention_plan.restype = ctypes.c_int
-    lib.egat_build_attention_plan.argtypes = [sp, vp, vp, vp, vp, sz, vp]
+    lib.egat_build_attention_plan.argtypes = [sp, vp, vp, vp, vp, vp, sz, vp]
+    lib.egat_take_device_status.restype = ctypes.c_int
+    lib.egat_take_device_status.argtypes = [vp]
+    lib.egat_selftest_wait_timeout.restype = ctypes.c_int
+    lib.egat_selftest_wait_timeout.argtypes = [i32, vp]
+    lib.egat_eaas_couple_planned.restype = ctypes.c_int
+    lib.egat_eaas_couple_planned.argtypes = [sp, vp, vp, vp, vp, vp]
     lib.egat_otf_attention_tiled.restype = ctypes.c_int
-    lib.egat_otf_attention_tiled.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp]
+    lib.egat_otf_attention_tiled.argtypes = [sp, vp, vp, vp, vp, vp, vp, i32, vp]
     lib.egat_forward_noalloc.restype = ctypes.c_int
     lib.egat_forward_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     if path is None:
@@ -265,31 +273,57 @@ def egat_attention_plan_bytes(shape: Shape) -> int:
 
 def egat_build_attention_plan(shape: Shape, nbr: torch.Tensor, cnt: Optional[torch.Tensor],
                               order: Optional[torch.Tensor] = None,
+                              pos: Optional[torch.Tensor] = None,
                               plan: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """Per-tile neighbour unions and membership masks for egat_otf_attention_tiled."""
+    """Per-tile neighbour unions, membership masks and target records (atom ids,
+    |r|^l, Wigner-D of the alignment rotations) for egat_otf_attention_tiled.
+    `pos` (float32 [n, 3]) is required."""
     nb = egat_attention_plan_bytes(shape)
     if plan is None:
         plan = torch.empty(max(nb, 16), dtype=torch.uint8, device=nbr.device)
     cs = shape.c()
     rc = load_library().egat_build_attention_plan(ctypes.byref(cs), _ptr(nbr), _ptr(cnt),
-                                                  _ptr(order), _ptr(plan), plan.numel(),
-                                                  _stream(stream))
+                                                  _ptr(order), _ptr(pos), _ptr(plan),
+                                                  plan.numel(), _stream(stream))
     _check("egat_build_attention_plan", rc)
     return plan
 
 
+def egat_take_device_status(stream=None) -> int:
+    """Synchronise the stream; EGAT_ERR_TIMEOUT if a bounded device wait gave up
+    since the last call (the count is cleared), EGAT_OK otherwise."""
+    return load_library().egat_take_device_status(_stream(stream))
+
+
+def egat_selftest_wait_timeout(polls: int = 1000, stream=None) -> None:
+    """Launch the wait that cannot succeed (see include/egat.h)."""
+    _check("egat_selftest_wait_timeout",
+           load_library().egat_selftest_wait_timeout(int(polls), _stream(stream)))
+
+
+def egat_eaas_couple_planned(shape: Shape, h: torch.Tensor, plan: torch.Tensor, w: torch.Tensor,
+                             out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Step 2 for the atoms of an attention plan, rotations from its tile records."""
+    if out is None:
+        out = torch.empty_like(h)
+    cs = shape.c()
+    rc = load_library().egat_eaas_couple_planned(ctypes.byref(cs), _ptr(h), _ptr(plan), _ptr(w),
+                                                 _ptr(out), _stream(stream))
+    _check("egat_eaas_couple_planned", rc)
+    return out
+
+
 def egat_otf_attention_tiled(shape: Shape, q: torch.Tensor, k: torch.Tensor, hp: torch.Tensor,
-                             plan: torch.Tensor, order: Optional[torch.Tensor] = None,
-                             pos: Optional[torch.Tensor] = None, w2: Optional[torch.Tensor] = None,
+                             plan: torch.Tensor, w2: Optional[torch.Tensor] = None,
                              fused: bool = True, out: Optional[torch.Tensor] = None,
                              stream=None) -> torch.Tensor:
-    """Tensor-core attention over a plan: ^h (fused) or m, float32 [n, D, C]."""
+    """Tensor-core attention over a plan: ^h (fused, w2 required) or m, float32 [n, D, C]."""
     if out is None:
         out = torch.empty((shape.n, shape.D, shape.C), dtype=torch.float32, device=hp.device)
     cs = shape.c()
     rc = load_library().egat_otf_attention_tiled(
-        ctypes.byref(cs), _ptr(q), _ptr(k), _ptr(hp), _ptr(plan), _ptr(order), _ptr(pos),
-        _ptr(w2), _ptr(out), 1 if fused else 0, _stream(stream))
+        ctypes.byref(cs), _ptr(q), _ptr(k), _ptr(hp), _ptr(plan), _ptr(w2), _ptr(out),
+        1 if fused else 0, _stream(stream))
     _check("egat_otf_attention_tiled", rc)
     return out
 

@@ -66,7 +66,8 @@ enum {
   EGAT_ERR_UNSUPPORTED = -2,  /* shape outside the supported set above */
   EGAT_ERR_CUDA = -3,         /* a CUDA launch or runtime call failed */
   EGAT_ERR_WORKSPACE = -4,    /* workspace smaller than the query returned */
-  EGAT_ERR_SCRATCH_LIMIT = -5 /* egat_forward_noalloc: problem larger than its fixed scratch */
+  EGAT_ERR_SCRATCH_LIMIT = -5, /* egat_forward_noalloc: problem larger than its fixed scratch */
+  EGAT_ERR_TIMEOUT = -6        /* egat_take_device_status: a bounded device wait gave up */
 };
 
 /* storage type of h, q, k and h' (accumulation and outputs are float32) */
@@ -196,26 +197,40 @@ EGAT_API int egat_otf_attention_coupled(const egat_shape* s, const void* d_q, co
  * to rounding: the softmax weights enter the P V product as bf16.
  *
  * egat_attention_plan_bytes / egat_build_attention_plan: per tile, the
- * union of the 16 targets' neighbour lists in ascending atom index and a
- * (16 x union) membership bitmask, built from the padded list (d_nbr, d_cnt —
- * d_cnt may be NULL) and d_order into caller memory d_plan of at least the
- * queried size.  The builder keeps a bitmap over all n atoms per tile in
- * shared memory, so it supports n up to about 800,000 atoms (2 * n / 8 bytes
- * plus the tile mask within 200 KiB; larger n returns EGAT_ERR_UNSUPPORTED
- * and egat_forward falls back to the per-target kernel).  The plan depends
- * only on the graph; it is reused by every attention call on it.
- * egat_otf_attention_tiled: fused = 1 writes ^h (d_pos, d_w2 required),
- * fused = 0 writes m; d_order must be the array the plan was built with.
+ * union of the 16 targets' neighbour lists in ascending atom index, a
+ * (16 x union) membership bitmask, and a target record (the 16 atom ids,
+ * |r|^l and the real Wigner-D matrices of their alignment rotations for the
+ * target coupling), built from the padded list (d_nbr, d_cnt — d_cnt may be
+ * NULL), d_order and d_pos (float32 [n][3], required) into caller memory
+ * d_plan of at least the queried size.  The builder keeps a bitmap over all n
+ * atoms per tile in shared memory, so it supports n up to about 800,000
+ * atoms (2 * n / 8 bytes plus the tile mask within 200 KiB; larger n returns
+ * EGAT_ERR_UNSUPPORTED and egat_forward falls back to the per-target kernel).
+ * The plan depends only on the graph and the positions; it is reused by
+ * every attention call on them.
+ * egat_otf_attention_tiled: fused = 1 writes ^h (d_w2 required), fused = 0
+ * writes m (d_w2 unused); target order and rotations come from the plan.
  */
 EGAT_API int egat_attention_plan_bytes(const egat_shape* s, size_t* bytes);
 EGAT_API int egat_build_attention_plan(const egat_shape* s, const int32_t* d_nbr,
                                        const int32_t* d_cnt, const int32_t* d_order,
-                                       void* d_plan, size_t plan_bytes, void* stream);
+                                       const float* d_pos, void* d_plan, size_t plan_bytes,
+                                       void* stream);
+/*
+ * Step 2 on an attention plan — the source coupling of egat_eaas_couple for
+ * every atom the plan lists, with each atom's |r|^l and Wigner-D matrices
+ * read from the plan's tile records instead of being built again (the plan
+ * builds them once per atom for the target coupling).  Same result as
+ * egat_eaas_couple up to the rounding of the Wigner-D construction.
+ *  d_plan  built by egat_build_attention_plan for the same shape and d_pos
+ *  d_h, d_w1, d_hout  as egat_eaas_couple
+ * Returns EGAT_ERR_UNSUPPORTED where egat_build_attention_plan would.
+ */
+EGAT_API int egat_eaas_couple_planned(const egat_shape* s, const void* d_h, const void* d_plan,
+                                      const float* d_w1, void* d_hout, void* stream);
 EGAT_API int egat_otf_attention_tiled(const egat_shape* s, const void* d_q, const void* d_k,
-                                      const void* d_hp, const void* d_plan,
-                                      const int32_t* d_order, const float* d_pos,
-                                      const float* d_w2, float* d_out, int32_t fused,
-                                      void* stream);
+                                      const void* d_hp, const void* d_plan, const float* d_w2,
+                                      float* d_out, int32_t fused, void* stream);
 
 /*
  * Steps 2-4 — the fused forward pass ([EX] §3.1):
@@ -242,8 +257,9 @@ EGAT_API int egat_forward(const egat_shape* s, const void* d_h, const float* d_p
  * array of EGAT_NOALLOC_SCRATCH_BYTES bytes that every GPU loading the library
  * holds until the process exits.  It performs no allocation.
  *  - Limit: egat_forward_workspace_bytes(s) <= EGAT_NOALLOC_SCRATCH_BYTES,
- *    i.e. n * (lmax+1)^2 * C * (2 for bf16, 4 for f32) bytes rounded up to
- *    256; larger problems return EGAT_ERR_SCRATCH_LIMIT without launching.
+ *    i.e. h' (n * (lmax+1)^2 * C * (2 for bf16, 4 for f32) bytes, rounded up
+ *    to 256) plus, for shapes on the tensor-core path, the attention plan;
+ *    larger problems return EGAT_ERR_SCRATCH_LIMIT without launching.
  *  - The first call on a device, made with that device current, looks up the
  *    array's device address once (cudaGetSymbolAddress); make that first call
  *    before any stream capture.
@@ -257,6 +273,28 @@ EGAT_API int egat_forward_noalloc(const egat_shape* s, const void* d_h, const fl
                                   const int32_t* d_nbr_or_rowptr, const int32_t* d_cnt_or_col,
                                   const int32_t* d_order, const float* d_w1, const float* d_w2,
                                   float* d_out, void* stream);
+
+/*
+ * Device status.  The tensor-core attention kernel waits on mbarriers for its
+ * bulk copies; every such wait is bounded (about a second).  A wait that
+ * gives up is counted on the device, the kernel stops waiting and finishes
+ * with meaningless output instead of hanging.  The pages have no
+ * counterpart: this is the library's failure report.
+ *
+ * egat_take_device_status: synchronises `stream`, then returns
+ * EGAT_ERR_TIMEOUT if any wait gave up on the current device since the last
+ * call (and clears the count), EGAT_OK otherwise, EGAT_ERR_CUDA if the
+ * synchronisation or the read failed.  Call it after the work whose result
+ * matters; it is not meant for a timed region.
+ *
+ * egat_selftest_wait_timeout: launches a one-warp kernel whose wait cannot
+ * succeed (an mbarrier expecting bytes no copy delivers) and gives up after
+ * `polls` polls (1 .. 1048576), so that egat_take_device_status reports
+ * EGAT_ERR_TIMEOUT — a test of the failure path that faults nothing.
+ * Asynchronous on `stream`; EGAT_ERR_ARG for polls out of range.
+ */
+EGAT_API int egat_take_device_status(void* stream);
+EGAT_API int egat_selftest_wait_timeout(int32_t polls, void* stream);
 
 #ifdef __cplusplus
 }

@@ -49,9 +49,10 @@ def test_host_only_queries(lib):
     assert egat.egat_graph_workspace_bytes(1000) > 0
     s = egat.Shape(n=32768, lmax=2, C=128, H=16, dk=16, K=256, dtype="bf16")
     # h' plus, for tensor-core shapes, the attention plan (2048 tiles: union
-    # capacity 4096 ints and a 16 x 128-word mask each, plus lengths)
+    # capacity 4096 ints, a 16 x 128-word mask and a target record of
+    # 16 x (1 id + 3 powers |r|^l + 35 Wigner-D entries) words each, plus lengths)
     plan = egat.egat_attention_plan_bytes(s)
-    assert plan == 2048 * 4 + 2048 * 4096 * 4 + 2048 * 16 * 128 * 4
+    assert plan == 2048 * 4 + 2048 * 4096 * 4 + 2048 * 16 * 128 * 4 + 2048 * 16 * 39 * 4
     assert egat.egat_forward_workspace_bytes(s) == 32768 * 9 * 128 * 2 + plan
     f32 = egat.Shape(n=648, lmax=2, C=128, H=16, dk=16, K=64, dtype="f32")
     assert egat.egat_forward_workspace_bytes(f32) == 648 * 9 * 128 * 4
@@ -103,3 +104,35 @@ def test_pointer_and_size_validation(lib):
     assert g(10, 100, 8, 0, None) == egat.EGAT_ERR_ARG
     assert g(1 << 30, 2 ** 31 - 1, 8, 0, ok) == egat.EGAT_ERR_UNSUPPORTED
     assert g(10, (1 << 26) + 1, 8, 0, ok) == egat.EGAT_ERR_UNSUPPORTED
+
+
+def test_plan_and_status_entry_validation(lib):
+    """Host-side checks of the plan, planned-coupling, tiled-attention and
+    self-test entry points (no launch happens on these paths)."""
+    cs = egat.Shape(n=10, lmax=2, C=128, H=16, dk=16, K=64, dtype="bf16").c()
+    ok = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)
+    # plan: positions are required; the plan buffer must be 16-byte aligned and large enough
+    assert lib.egat_build_attention_plan(ctypes.byref(cs), ok, ok, None, None, ok, 1 << 30,
+                                         None) == egat.EGAT_ERR_ARG
+    assert lib.egat_build_attention_plan(ctypes.byref(cs), ok, ok, None, ok, odd, 1 << 30,
+                                         None) == egat.EGAT_ERR_ARG
+    assert lib.egat_build_attention_plan(ctypes.byref(cs), ok, ok, None, ok, ok, 16,
+                                         None) == egat.EGAT_ERR_WORKSPACE
+    csr = egat.Shape(n=10, lmax=2, C=128, H=16, dk=16, K=64, dtype="bf16", graph_mode="csr",
+                     n_edges=10).c()
+    assert lib.egat_build_attention_plan(ctypes.byref(csr), ok, ok, None, ok, ok, 1 << 30,
+                                         None) == egat.EGAT_ERR_UNSUPPORTED
+    # planned coupling: every pointer required, storage 16-byte aligned
+    assert lib.egat_eaas_couple_planned(ctypes.byref(cs), None, ok, ok, ok, None) == egat.EGAT_ERR_ARG
+    assert lib.egat_eaas_couple_planned(ctypes.byref(cs), odd, ok, ok, ok, None) == egat.EGAT_ERR_ARG
+    # tiled attention: w2 required when fused, not otherwise checked
+    assert lib.egat_otf_attention_tiled(ctypes.byref(cs), ok, ok, ok, ok, None, ok, 1,
+                                        None) == egat.EGAT_ERR_ARG
+    f32 = egat.Shape(n=10, lmax=2, C=128, H=16, dk=16, K=64, dtype="f32").c()
+    assert lib.egat_otf_attention_tiled(ctypes.byref(f32), ok, ok, ok, ok, ok, ok, 1,
+                                        None) == egat.EGAT_ERR_UNSUPPORTED
+    # self-test: poll count range
+    assert lib.egat_selftest_wait_timeout(0, None) == egat.EGAT_ERR_ARG
+    assert lib.egat_selftest_wait_timeout((1 << 20) + 1, None) == egat.EGAT_ERR_ARG
+    assert lib.egat_strerror(egat.EGAT_ERR_TIMEOUT).startswith(b"a bounded device wait")

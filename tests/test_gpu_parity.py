@@ -112,6 +112,26 @@ def test_graph_full_size_sampled_rows(name):
 
 # --------------------------------------------------------------------------- steps 2, 3
 @pytest.mark.parametrize("name", SMALL + LARGE)
+def test_eaas_couple_planned_parity(name):
+    """Step 2 with the rotations taken from the attention plan's tile records
+    (egat_eaas_couple_planned), against the oracle on every atom the sample
+    covers; every atom of the system is written exactly once."""
+    egat = _egat()
+    wl, d = _data(name)
+    dev = device_inputs(wl, d)
+    shape = shape_of(wl)
+    g = egat.egat_build_graph(dev["pos_q"], wl.cutoff_q, K=wl.K)
+    plan = egat.egat_build_attention_plan(shape, g["nbr"], g["cnt"], g["order"], dev["pos"])
+    hp = torch.full_like(dev["h"], float("nan"))
+    egat.egat_eaas_couple_planned(shape, dev["h"], plan, dev["w1"], out=hp)
+    assert not torch.isnan(hp.float()).any()
+    rows = np.arange(wl.n) if wl.n <= 4096 else np.array(sample_targets(wl, _full_degree(name), 300))
+    ref = source_coupling(d["h"][rows], d["pos"][rows], d["w1"], wl.lmax)
+    got = hp[torch.from_numpy(rows).cuda()].float().cpu().numpy()
+    assert block_rel_error(got, ref, wl.lmax) < TOL[wl.dtype]
+
+
+@pytest.mark.parametrize("name", SMALL + LARGE)
 def test_eaas_couple_parity(name):
     egat = _egat()
     wl, d = _data(name)

@@ -17,6 +17,7 @@ import pytest
 import torch
 
 from oracle.attention import aggregate, forward as oracle_forward
+from oracle import so3
 from oracle.graph import radius_graph
 from equivariant_graph_attention_b200 import synth
 from tests.parity_util import TOL, block_rel_error, device_inputs, sample_targets, shape_of
@@ -38,7 +39,7 @@ def _data(name):
     return wl, synth.make(wl)
 
 
-def _plan_views(plan: torch.Tensor, n: int, K: int):
+def _plan_views(plan: torch.Tensor, n: int, K: int, lmax: int):
     tiles = (n + TILE - 1) // TILE
     cap = 32
     while cap < TILE * K:
@@ -49,21 +50,30 @@ def _plan_views(plan: torch.Tensor, n: int, K: int):
     o = a256(tiles * 4)
     uni = raw[o:o + tiles * cap * 4].view(np.int32).reshape(tiles, cap)
     o += a256(tiles * cap * 4)
-    mask = raw[o:o + tiles * TILE * (cap // 32) * 4].view(np.uint32).reshape(tiles, TILE, cap // 32)
-    return ulen, uni, mask
+    mask = raw[o:o + tiles * TILE * (cap // 32) * 4].view(np.uint32).reshape(tiles, cap // 32, TILE)
+    o += a256(tiles * TILE * (cap // 32) * 4)
+    ws = sum((2 * l + 1) ** 2 for l in range(lmax + 1))
+    rw = TILE * (1 + (lmax + 1) + ws)
+    rec = raw[o:o + tiles * rw * 4].view(np.float32).reshape(tiles, rw)
+    return ulen, uni, mask, rec
 
 
 @pytest.mark.parametrize("name", ["uniform4096_l2_bf16", "uniform32768_K256_l2_bf16"])
 def test_plan_matches_numpy(name):
+    """Union, padding and membership bits rebuilt with numpy (bit for bit), and
+    the tile records: target ids exactly, |r|^l and the Wigner-D blocks of the
+    targets' alignment rotations against the oracle's (least-squares) D."""
     egat = _egat()
     wl, d = _data(name)
     dev = device_inputs(wl, d)
     g = egat.egat_build_graph(dev["pos_q"], wl.cutoff_q, K=wl.K)
     shape = shape_of(wl)
-    plan = egat.egat_build_attention_plan(shape, g["nbr"], g["cnt"], g["order"])
-    ulen, uni, mask = _plan_views(plan, wl.n, wl.K)
+    plan = egat.egat_build_attention_plan(shape, g["nbr"], g["cnt"], g["order"], dev["pos"])
+    ulen, uni, mask, rec = _plan_views(plan, wl.n, wl.K, wl.lmax)
     nbr, cnt, order = g["nbr"].cpu().numpy(), g["cnt"].cpu().numpy(), g["order"].cpu().numpy()
+    pos = dev["pos"].cpu().numpy().astype(np.float64)
     tiles = (wl.n + TILE - 1) // TILE
+    ws = sum((2 * l + 1) ** 2 for l in range(wl.lmax + 1))
     pick = range(tiles) if tiles <= 256 else np.random.default_rng(3).choice(tiles, 64, replace=False)
     for t in pick:
         rows = order[t * TILE:(t + 1) * TILE]
@@ -72,14 +82,31 @@ def test_plan_matches_numpy(name):
         U = int(ulen[t])
         assert U == len(ref)
         assert np.array_equal(uni[t, :U], ref)
-        upad = (U + 15) // 16 * 16
+        upad = max(32, (U + 31) // 32 * 32)
         assert np.all(uni[t, U:upad] == (ref[0] if U else 0))
         for r, js in enumerate(lists):
             bits = np.zeros(upad, dtype=bool)
             bits[np.searchsorted(ref, js)] = True
             u = np.arange(upad)
-            got = ((mask[t, r, u // 32] >> (u % 32).astype(np.uint32)) & 1).astype(bool)
+            got = ((mask[t, u // 32, r] >> (u % 32).astype(np.uint32)) & 1).astype(bool)
             assert np.array_equal(got, bits), (t, r)
+        # tile record
+        ids = rec[t, :TILE].view(np.int32)
+        want = np.full(TILE, -1, np.int32)
+        want[:len(rows)] = rows
+        assert np.array_equal(ids, want)
+        rp = rec[t, TILE:TILE * (wl.lmax + 2)].reshape(TILE, wl.lmax + 1)
+        Dr = rec[t, TILE * (wl.lmax + 2):].reshape(TILE, ws)
+        for r, a in enumerate(rows[:4]):
+            rr = float(np.linalg.norm(pos[a]))
+            assert np.allclose(rp[r], [rr ** l for l in range(wl.lmax + 1)], rtol=1e-5, atol=0)
+            Q = so3.alignment_rotation(pos[a])
+            off = 0
+            for l in range(wl.lmax + 1):
+                w = 2 * l + 1
+                got = Dr[r, off:off + w * w].reshape(w, w)
+                assert np.allclose(got, so3.wigner_D(l, Q), atol=2e-5), (t, r, l)
+                off += w * w
 
 
 @pytest.mark.parametrize("name", BF16)
@@ -92,9 +119,8 @@ def test_tiled_attention_parity(name):
     hp = torch.from_numpy(vals).to("cuda", dtype=torch.bfloat16)
     g = egat.egat_build_graph(dev["pos_q"], wl.cutoff_q, K=wl.K)
     shape = shape_of(wl)
-    plan = egat.egat_build_attention_plan(shape, g["nbr"], g["cnt"], g["order"])
-    m = egat.egat_otf_attention_tiled(shape, dev["q"], dev["k"], hp, plan, order=g["order"],
-                                      fused=False)
+    plan = egat.egat_build_attention_plan(shape, g["nbr"], g["cnt"], g["order"], dev["pos"])
+    m = egat.egat_otf_attention_tiled(shape, dev["q"], dev["k"], hp, plan, fused=False)
     rows = list(range(wl.n)) if wl.n <= 4096 else sample_targets(
         wl, np.minimum(g["cnt"].cpu().numpy(), wl.K))
     lists, _ = radius_graph(d["pos_q"], wl.cutoff_q, K=wl.K, rows=rows)
@@ -114,9 +140,8 @@ def test_tiled_fused_matches_per_target_kernel(name):
     g = egat.egat_build_graph(dev["pos_q"], wl.cutoff_q, K=wl.K)
     shape = shape_of(wl)
     hp = egat.egat_eaas_couple(shape, dev["h"], dev["pos"], dev["w1"])
-    plan = egat.egat_build_attention_plan(shape, g["nbr"], g["cnt"], g["order"])
-    a = egat.egat_otf_attention_tiled(shape, dev["q"], dev["k"], hp, plan, order=g["order"],
-                                      pos=dev["pos"], w2=dev["w2"], fused=True)
+    plan = egat.egat_build_attention_plan(shape, g["nbr"], g["cnt"], g["order"], dev["pos"])
+    a = egat.egat_otf_attention_tiled(shape, dev["q"], dev["k"], hp, plan, w2=dev["w2"], fused=True)
     b = egat.egat_otf_attention_coupled(shape, dev["q"], dev["k"], hp, g["nbr"], g["cnt"],
                                         dev["pos"], dev["w2"], order=g["order"])
     err = block_rel_error(a.cpu().numpy(), b.cpu().numpy(), wl.lmax)
