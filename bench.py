@@ -162,6 +162,34 @@ def dist_env():
     return ws, rank, local
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The largest `value` over all ranks (the job's time is its slowest rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, device) -> float:
+    """`value` summed over all ranks (units processed by the whole job)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def job_rate(local_units: float, local_ms: float, device) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest
+    rank's time."""
+    return sum_over_ranks(local_units, device) / (max_over_ranks(local_ms, device) / 1000.0)
+
+
 def run_reference(args, wl: synth.Workload):
     ws, rank, _ = dist_env()
     if rank != 0:
@@ -202,6 +230,8 @@ def main():
     ap.add_argument("--cpu-targets", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--backward-steps", type=int, default=5,
+                    help="timed calls of egat_backward reported beside the forward (0: skip)")
     ap.add_argument("--attention", default="auto", choices=["auto", "tiled", "per-target"],
                     help="steps 3+4 kernel: tensor-core tiles when the shape allows (auto), or "
                          "the per-target kernel")
@@ -336,13 +366,11 @@ def main():
     t_attn = sum(e[3].elapsed_time(e[4]) for e in ev) / args.steps
     t_step = sum(e[0].elapsed_time(e[4]) for e in ev) / args.steps      # ms
     total_ms = t_step * args.steps
-    if ws > 1:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
-    atoms_total = wl.n * ws * args.steps
-    value = atoms_total / (total_ms / 1000.0)
-    edges_per_s = alg["edges"] * ws * args.steps / (total_ms / 1000.0)
+    # every rank ran its own system: atoms and edges add up over ranks, the
+    # job's time is the slowest rank's
+    value = job_rate(wl.n * args.steps, total_ms, dev)
+    edges_per_s = job_rate(alg["edges"] * args.steps, total_ms, dev)
+    t_step = max_over_ranks(total_ms, dev) / args.steps
 
     # ------------------------------------------------------------------ e2e
     # the same step through the public C ABI (egat_build_graph + egat_forward)
@@ -411,12 +439,48 @@ def main():
     eb.record(s_out)
     torch.cuda.synchronize(dev)
     e2e_ms = ea.elapsed_time(eb)
-    if ws > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    e2e_value = wl.n * ws * args.e2e_steps / (e2e_ms / 1000.0)
+    e2e_value = job_rate(wl.n * args.e2e_steps, e2e_ms, dev)
+    e2e_ms = max_over_ranks(e2e_ms, dev)
     e2e_ok = bool(torch.equal(host_out[0].to(dev), out))   # pipelined result == device-timed result
+    # ------------------------------------------------------------------ backward
+    # gradients of <G, ^h> for a seeded upstream gradient G (egat_backward:
+    # dL/dh, dL/dq, dL/dk; the attention is recomputed, in-lists built inside),
+    # each call after an L2 flush, timed with events on the launching stream
+    bwd = None
+    if args.backward_steps > 0:
+        gen = torch.Generator(device="cpu").manual_seed(1234 + rank)
+        G = torch.randn((wl.n, wl.D, wl.C), generator=gen, dtype=torch.float32).to(dev)
+        bws_t = torch.empty(max(egat.egat_backward_workspace_bytes(shape), 16), dtype=torch.uint8,
+                            device=dev)
+        dh_t = torch.empty((wl.n, wl.D, wl.C), dtype=torch.float32, device=dev)
+        dq_t = torch.empty((wl.n, wl.H, wl.dk), dtype=torch.float32, device=dev)
+        dk_t = torch.empty((wl.n, wl.H, wl.dk), dtype=torch.float32, device=dev)
+
+        def backward_call():
+            rc = lib.egat_backward(ctypes.byref(cshape), h.data_ptr(), pos.data_ptr(), q.data_ptr(),
+                                   k.data_ptr(), nbr.data_ptr(), cnt.data_ptr(), w1.data_ptr(),
+                                   w2.data_ptr(), G.data_ptr(), bws_t.data_ptr(), bws_t.numel(),
+                                   dh_t.data_ptr(), dq_t.data_ptr(), dk_t.data_ptr(), sp)
+            egat._check("egat_backward", rc)
+
+        graph()                                           # this system's neighbour lists
+        backward_call()                                   # warm-up
+        torch.cuda.synchronize(dev)
+        bms = []
+        for _ in range(args.backward_steps):
+            flush.fill_(3)
+            ba, bb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ba.record(torch.cuda.current_stream(dev))
+            backward_call()
+            bb.record(torch.cuda.current_stream(dev))
+            torch.cuda.synchronize(dev)
+            bms.append(ba.elapsed_time(bb))
+        t_bwd = sum(bms) / len(bms)
+        bwd = {"ms": max_over_ranks(t_bwd, dev),
+               "atoms_per_s": job_rate(wl.n, t_bwd, dev),
+               "edges_per_s": job_rate(alg["edges"], t_bwd, dev),
+               "what": "dL/dh, dL/dq, dL/dk of <G, ^h> (egat_backward), L2 flushed before each call"}
+
     # no bounded device wait may have given up in any of the runs above
     status = lib.egat_take_device_status(torch.cuda.current_stream(dev).cuda_stream)
     if status != egat.EGAT_OK:
@@ -466,6 +530,7 @@ def main():
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.e2e_steps,
                     "pipelined": "copy-in / compute / copy-out streams, 2 buffers",
                     "matches_device_result": e2e_ok},
+            "backward": bwd,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
         }

@@ -40,6 +40,7 @@
 // per-channel EAAS epilogue needs, so the target coupling runs from registers.
 #include <cfloat>
 
+#include "egat_async.cuh"
 #include "egat_device.cuh"
 #include "egat_host.h"
 
@@ -47,8 +48,6 @@ namespace egat {
 namespace {
 
 constexpr int kRowPad = 16;   // bytes of padding per staged row
-// stage mbarriers (up to 3) and the abort flag, after 16-byte alignment
-constexpr size_t kBarBytes = 16 + 8 * 3 + 8;
 
 struct TcParams {
   const __nv_bfloat16* q;
@@ -64,63 +63,6 @@ struct TcParams {
   EaasTable tab;
 };
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-// mbarrier and bulk-copy (TMA engine, no multicast) helpers
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_fence_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
-      "l"(src), "r"(bytes), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-}
-
-// Waits that gave up since the last egat_take_device_status (all launches on
-// this device).
-__device__ unsigned int g_wait_timeouts;
-// Polls before a wait gives up.  try_wait suspends the thread for at most a
-// hardware-defined interval per poll, so this bounds a wait to about a
-// second; a stage's copies normally land within microseconds.
-constexpr int kWaitPolls = 1 << 20;
-constexpr int kDrainPolls = 1 << 14;
-
-// Wait until the phase of parity `parity` of the mbarrier at `bar` has
-// completed, polling at most `polls` times.  On giving up: count it, set the
-// CTA's abort flag and return false; once the flag is set, waits return at
-// once, so a CTA whose copies never land finishes its loop (with meaningless
-// results, reported by egat_take_device_status) instead of hanging.
-__device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, int polls,
-                                             volatile int* abort_flag) {
-  if (*abort_flag) return false;
-  for (int i = 0; i < polls; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  atomicAdd(&g_wait_timeouts, 1u);
-  *abort_flag = 1;
-  return false;
-}
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -156,63 +98,71 @@ struct TcShape {
   static constexpr int RS = KS * kTileK;   // rows per stage
 };
 
-// staging buffers, then the tile's Wigner-D / |r|^l / targets, then the tile's
-// union indices [cap] and membership mask [kTileM][cap / 32]
+// Shared-memory layout (byte offsets; every region 16-byte aligned): staged
+// value and key rows, the tile's query rows, two tile records (current and
+// next), the target-coupling weights [P][C] (fused), the mbarriers and the
+// abort flag, then the tile's union indices [cap] and word-major membership
+// mask [cap / 32][16] (6 cap bytes, sized at launch).
+template <int L, int H, bool FUSED>
+struct TcSmem {
+  using Sh = TcShape<L>;
+  static constexpr int D = Sh::D, C = 8 * H;
+  static constexpr int VSTR = D * C * 2 + kRowPad;   // staged value row
+  static constexpr int KSTR = H * 32 + kRowPad;      // staged key row (dk = 16)
+  static constexpr int QSTR = KSTR;                  // staged query row
+  static constexpr int REC = plan_record_words(L);
+  static_assert(REC % 4 == 0, "records move in 16-byte units");
+  static constexpr int NBARS = Sh::STAGES + 4;       // rows [STAGES], record [2], indices, mask
+  static constexpr size_t vbuf = 0;
+  static constexpr size_t kbuf = vbuf + size_t(Sh::STAGES) * Sh::RS * VSTR;
+  static constexpr size_t sq = kbuf + size_t(Sh::STAGES) * Sh::RS * KSTR;
+  static constexpr size_t rec = sq + size_t(kTileM) * QSTR;
+  static constexpr size_t sw2 = rec + 2 * size_t(REC) * 4;
+  static constexpr size_t bars = sw2 + (FUSED ? size_t(num_paths(L)) * C * 4 : 0);
+  static constexpr size_t su = bars + (size_t(NBARS) * 8 + 4 + 15) / 16 * 16;
+  static size_t total(int cap) { return su + size_t(cap) * 4 + size_t(cap / 32) * kTileM * 4; }
+};
+// the fused epilogue at lmax >= 3 keeps m of the tile in the stage buffers
 template <int L, int H>
-constexpr size_t tc_smem_fixed() {
-  constexpr int D = (L + 1) * (L + 1);
-  constexpr int C = 8 * H;
-  constexpr int VSTR = D * C * 2 + kRowPad;
-  constexpr int KSTR = H * 16 * 2 + kRowPad;
-  return size_t(TcShape<L>::STAGES) * TcShape<L>::RS * (VSTR + KSTR) +
-         size_t(kTileM) * (wig_size(L) + L + 1) * sizeof(float) + kTileM * sizeof(int);
+constexpr bool tc_scratch_fits() {
+  return size_t(H) * kTileM * TcShape<L>::D * 8 * 4 <=
+         size_t(TcShape<L>::STAGES) * TcShape<L>::RS * TcSmem<L, H, true>::VSTR;
 }
-// mask rows are padded by one word so the 8 rows a warp reads sit in distinct banks
-// fused kernels keep the target-coupling weights [P][C] in shared memory
-template <int L, int H>
-constexpr size_t tc_smem_w2() {
-  return size_t(num_paths(L)) * 8 * H * sizeof(float);
-}
-inline size_t tc_smem_plan(int cap) {
-  return size_t(cap) * sizeof(int) + size_t(kTileM) * (cap / 32 + 1) * sizeof(uint32_t);
-}
+static_assert(tc_scratch_fits<3, 16>(), "lmax 3 epilogue scratch");
 
 template <int L, int H, bool FUSED>
 __global__ void __launch_bounds__(H * 32, 1)
 otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
+  using Sm = TcSmem<L, H, FUSED>;
   constexpr int D = (L + 1) * (L + 1);
   constexpr int C = 8 * H;
   constexpr int ROW = D * C * 2;                  // value row bytes
-  constexpr int VSTR = ROW + kRowPad;
-  constexpr int KROW = H * 16 * 2;                // key row bytes (dk = 16)
-  constexpr int KSTR = KROW + kRowPad;
+  constexpr int VSTR = Sm::VSTR;
+  constexpr int KROW = H * 16 * 2;                // key / query row bytes (dk = 16)
+  constexpr int KSTR = Sm::KSTR;
+  constexpr int QSTR = Sm::QSTR;
   constexpr int STAGES = TcShape<L>::STAGES;
   constexpr int KS = TcShape<L>::KS;
   constexpr int RS = TcShape<L>::RS;
+  constexpr int REC = Sm::REC;
   constexpr int WS = wig_size(L);
   constexpr int NTHR = H * 32;
-  constexpr int VCH = ROW / 16, KCH = KROW / 16;  // 16-byte chunks per row
+  // the fused lmax 3 epilogue uses the stage buffers as scratch, so there the
+  // next tile's first rows are staged after it
+  constexpr bool kEarlyRows = !(FUSED && L >= 3);
   extern __shared__ __align__(128) unsigned char smem[];
-  unsigned char* vbuf = smem;                                        // [STAGES][RS][VSTR]
-  unsigned char* kbuf = vbuf + size_t(STAGES) * RS * VSTR;           // [STAGES][RS][KSTR]
-  float* Dq = reinterpret_cast<float*>(kbuf + size_t(STAGES) * RS * KSTR);   // [16][WS]
-  float* rp = Dq + kTileM * WS;                                      // [16][L+1]
-  int* tgt = reinterpret_cast<int*>(rp + kTileM * (L + 1));          // [16]
-  int* su = tgt + kTileM;                                            // [cap]
-  uint32_t* smask = reinterpret_cast<uint32_t*>(su + p.plan.cap);    // [16][cap / 32 + 1]
-  float* sw2 = reinterpret_cast<float*>(smask + kTileM * (p.plan.cap / 32 + 1));   // [P][C]
-  uint64_t* fullbar = reinterpret_cast<uint64_t*>(
-      (reinterpret_cast<uintptr_t>(sw2 + (FUSED ? num_paths(L) * C : 0)) + 15) & ~uintptr_t(15));
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(fullbar + STAGES);
-  if (threadIdx.x == 0) {
-    // one arrival per staged row of a stage; its bulk copies add the bytes
-    for (int b = 0; b < STAGES; ++b) mbar_init(smem_u32(fullbar + b), RS);
-    mbar_fence_init();
-    *abort_flag = 0;
-  }
-  if constexpr (FUSED) {
-    for (int e = threadIdx.x; e < num_paths(L) * C; e += H * 32) sw2[e] = __ldg(p.w2 + e);
-  }
+  unsigned char* vbuf = smem + Sm::vbuf;                                 // [STAGES][RS][VSTR]
+  unsigned char* kbuf = smem + Sm::kbuf;                                 // [STAGES][RS][KSTR]
+  unsigned char* sq = smem + Sm::sq;                                     // [16][QSTR]
+  float* recbuf = reinterpret_cast<float*>(smem + Sm::rec);              // [2][REC]
+  float* sw2 = reinterpret_cast<float*>(smem + Sm::sw2);                 // [P][C]
+  uint64_t* fullbar = reinterpret_cast<uint64_t*>(smem + Sm::bars);      // [STAGES] a stage's rows
+  uint64_t* recbar = fullbar + STAGES;                                   // [2] a tile record
+  uint64_t* idxbar = recbar + 2;                                         // a tile's indices + queries
+  uint64_t* mskbar = idxbar + 1;                                         // a tile's mask
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(mskbar + 1);
+  int* su = reinterpret_cast<int*>(smem + Sm::su);                       // [cap]
+  uint32_t* smask = reinterpret_cast<uint32_t*>(su + p.plan.cap);        // [cap / 32][16]
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -220,71 +170,112 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
   const int g = lane >> 2, t = lane & 3;
   const PlanView& pv = p.plan;
   const int words = pv.cap / 32;
-  const int swords = words + 1;     // padded shared-memory mask row
+  const int grid = gridDim.x;
   const char* hp_bytes = reinterpret_cast<const char*>(p.hp);
   const char* k_bytes = reinterpret_cast<const char*>(p.k);
+  const char* q_bytes = reinterpret_cast<const char*>(p.q);
+  if (blockIdx.x >= pv.tiles) return;   // whole CTA
 
+  if (tid == 0) {
+    // a stage buffer: one arrival per staged row, whose bulk copies add the
+    // bytes; records, indices and masks: one arrival by the issuing thread
+    for (int b = 0; b < STAGES; ++b) mbar_init(smem_u32(fullbar + b), RS);
+    for (int b = 0; b < 4; ++b) mbar_init(smem_u32(recbar + b), 1);
+    mbar_fence_init();
+    *abort_flag = 0;
+  }
+  if constexpr (FUSED) {
+    for (int e = tid; e < num_paths(L) * C; e += NTHR) sw2[e] = __ldg(p.w2 + e);
+  }
+  __syncthreads();
+
+  // union length of a tile record, clamped so that a record that never
+  // arrived (after a wait gave up) still gives bounded, in-range copies
+  auto rec_ulen = [&](const float* rec) {
+    const int U = reinterpret_cast<const int*>(rec)[0];
+    return U < 0 ? 0 : (U > pv.cap ? pv.cap : U);
+  };
+  auto stages_of = [&](const float* rec) { return (rec_ulen(rec) + RS - 1) / RS; };
+  // thread 0: a tile's record into recbuf[b]
+  auto issue_record = [&](int tl, int b) {
+    const uint32_t bar = smem_u32(recbar + b);
+    mbar_arrive_expect_tx(bar, REC * 4);
+    bulk_g2s(smem_u32(recbuf + b * REC), pv.rec + (long long)tl * REC, REC * 4, bar);
+  };
+  // thread 0: a tile's union indices (as the plan padded them) and the query
+  // rows of its targets (atom 0's row for an empty slot; unused)
+  auto issue_index = [&](int tl, const float* rec) {
+    const int U = rec_ulen(rec);
+    const int upad = U > 0 ? (U + kPlanPad - 1) / kPlanPad * kPlanPad : kPlanPad;
+    const uint32_t bar = smem_u32(idxbar);
+    mbar_arrive_expect_tx(bar, upad * 4 + kTileM * KROW);
+    bulk_g2s(smem_u32(su), pv.uni + (long long)tl * pv.cap, upad * 4, bar);
+    const int* tg = reinterpret_cast<const int*>(rec) + kRecTgt;
+    for (int r = 0; r < kTileM; ++r) {
+      const long long a = (unsigned)tg[r] < (unsigned)p.n ? tg[r] : 0;
+      bulk_g2s(smem_u32(sq + r * QSTR), q_bytes + a * KROW, KROW, bar);
+    }
+  };
+  // thread 0: a tile's membership mask (the words the plan wrote)
+  auto issue_mask = [&](int tl, const float* rec) {
+    const int U = rec_ulen(rec);
+    const int uw = U > 0 ? (U + 31) / 32 : 1;
+    const uint32_t bar = smem_u32(mskbar);
+    mbar_arrive_expect_tx(bar, uw * kTileM * 4);
+    bulk_g2s(smem_u32(smask), pv.mask + (long long)tl * words * kTileM, uw * kTileM * 4, bar);
+  };
+  // one thread per staged row: rows of tile-local stage s (global stage gs) as
+  // two bulk copies whose bytes complete the stage buffer's mbarrier phase
+  auto issue_rows = [&](int s, int gs) {
+    const int buf = gs % STAGES;
+    constexpr int RSTRIDE = NTHR / RS;
+    if (tid % RSTRIDE == 0) {
+      const int r = tid / RSTRIDE;
+      long long atom = su[s * RS + r];
+      if ((unsigned long long)atom >= (unsigned long long)p.n) atom = 0;
+      const uint32_t bar = smem_u32(fullbar + buf);
+      mbar_arrive_expect_tx(bar, ROW + KROW);
+      bulk_g2s(smem_u32(vbuf + (size_t(buf) * RS + r) * VSTR), hp_bytes + atom * ROW, ROW, bar);
+      bulk_g2s(smem_u32(kbuf + (size_t(buf) * RS + r) * KSTR), k_bytes + atom * KROW, KROW, bar);
+    }
+  };
+
+  // first tile: record, then its indices, queries and mask, then its first rows
+  int tile = blockIdx.x;
   int gbase = 0;   // stages staged by this CTA before the current tile
-  for (int tile = blockIdx.x; tile < pv.tiles; tile += gridDim.x) {
-    const int U = pv.ulen[tile];
-    const int nsteps = (U + kTileK - 1) / kTileK;         // k-steps of 16 union rows
-    const int nstages = (nsteps + KS - 1) / KS;
-    // the plan pads the union to whole k-steps; here it is padded further to
-    // whole stages with its first atom, whose mask bits there are zero
-    const int ustep = nsteps * kTileK;
-    const int* __restrict__ uni = pv.uni + (long long)tile * pv.cap;
-    const uint32_t* __restrict__ mrow = pv.mask + (long long)tile * words * kTileM;
+  if (tid == 0) issue_record(tile, 0);
+  bounded_wait(smem_u32(recbar), 0u, kWaitPolls, abort_flag);
+  if (tid == 0) {
+    issue_index(tile, recbuf);
+    issue_mask(tile, recbuf);
+  }
+  bounded_wait(smem_u32(idxbar), 0u, kWaitPolls, abort_flag);
+  {
+    const int ns = stages_of(recbuf);
+    for (int s = 0; s < STAGES - 1 && s < ns; ++s) issue_rows(s, s);
+  }
 
-    {
-      constexpr int RW = kTileM * (1 + (L + 1) + WS);
-      const float* R = pv.rec + (long long)tile * RW;
-      if (tid < kTileM) tgt[tid] = reinterpret_cast<const int*>(R)[tid];
-      if constexpr (FUSED) {
-        for (int e = tid; e < kTileM * (L + 1); e += NTHR) rp[e] = R[kTileM + e];
-        for (int e = tid; e < kTileM * WS; e += NTHR) Dq[e] = R[kTileM * (2 + L) + e];
-      }
-    }
-    // the tile's union indices and membership mask into shared memory
-    const int upad = nstages * RS;
-    const int uw = (ustep + 31) / 32;   // mask words the plan wrote
-    for (int e = tid; e < upad; e += NTHR) su[e] = uni[e < ustep ? e : 0];
-    for (int e = tid; e < kTileM * uw; e += NTHR) {
-      const int r = e / uw, w = e % uw;
-      smask[r * swords + w] = mrow[w * kTileM + r];
-    }
-    if (upad > 32 * uw && tid < kTileM) smask[tid * swords + uw] = 0u;
-    __syncthreads();   // tgt, su, smask visible
-
-    // 32 threads per staged row; each copies chunks lane, lane + 32, ... of
-    // the row's value and key bytes (rows past the padded union are skipped)
-    // one thread per staged row: its value row and key row as two bulk copies
-    // whose bytes complete the stage buffer's mbarrier phase
-    auto issue = [&](int stage) {
-      const int gs = gbase + stage;
-      const int buf = gs % STAGES;
-      constexpr int RSTRIDE = NTHR / RS;
-      if (tid % RSTRIDE == 0) {
-        const int r = tid / RSTRIDE;
-        const long long atom = su[stage * RS + r];
-        const uint32_t bar = smem_u32(fullbar + buf);
-        mbar_arrive_expect_tx(bar, ROW + KROW);
-        bulk_g2s(smem_u32(vbuf + (size_t(buf) * RS + r) * VSTR), hp_bytes + atom * ROW, ROW, bar);
-        bulk_g2s(smem_u32(kbuf + (size_t(buf) * RS + r) * KSTR), k_bytes + atom * KROW, KROW, bar);
-      }
-    };
-#pragma unroll
-    for (int s = 0; s < STAGES - 1; ++s)
-      if (s < nstages) issue(s);
+  int k = 0;   // this CTA's tile sequence number
+  for (; tile < pv.tiles; ++k, tile += grid) {
+    const float* rec = recbuf + (k & 1) * REC;
+    const float* nrec = recbuf + ((k + 1) & 1) * REC;
+    const int next = tile + grid;
+    const bool has_next = next < pv.tiles;
+    // this tile's record, indices, queries and mask (all issued during the
+    // previous tile, or above)
+    bounded_wait(smem_u32(recbar + (k & 1)), uint32_t(k >> 1) & 1u, kWaitPolls, abort_flag);
+    bounded_wait(smem_u32(idxbar), uint32_t(k) & 1u, kWaitPolls, abort_flag);
+    bounded_wait(smem_u32(mskbar), uint32_t(k) & 1u, kWaitPolls, abort_flag);
+    // the next tile's record into the other buffer (its last reader, the
+    // previous tile's epilogue, finished before that tile's last barrier)
+    if (tid == 0 && has_next) issue_record(next, (k + 1) & 1);
+    const int nstages = stages_of(rec);
 
     // Q fragment of this head for the tile's 16 targets
     uint32_t qa[4];
     {
-      const int t0 = tgt[g], t1 = tgt[g + 8];
-      const uint32_t* q32 = reinterpret_cast<const uint32_t*>(p.q);
-      qa[0] = t0 >= 0 ? __ldg(q32 + ((size_t)t0 * H * 16 + h * 16 + 2 * t) / 2) : 0u;
-      qa[1] = t1 >= 0 ? __ldg(q32 + ((size_t)t1 * H * 16 + h * 16 + 2 * t) / 2) : 0u;
-      qa[2] = t0 >= 0 ? __ldg(q32 + ((size_t)t0 * H * 16 + h * 16 + 2 * t + 8) / 2) : 0u;
-      qa[3] = t1 >= 0 ? __ldg(q32 + ((size_t)t1 * H * 16 + h * 16 + 2 * t + 8) / 2) : 0u;
+      const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
+      ldsm_x4(qa, smem_u32(sq + row * QSTR + h * 32 + (lane >> 4) * 16));
     }
     float acc[D][4];
 #pragma unroll
@@ -305,9 +296,17 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
     // raw-logit thresholds that trigger a raise; start below any finite logit
     float thr0 = -INFINITY, thr1 = -INFINITY;
 
+    // the stage after which the indices and query rows are free for the next
+    // tile: its barrier follows the last issue that reads them
+    const int trig = nstages - STAGES + 1 > 0 ? nstages - STAGES + 1 : 0;
     for (int st = 0; st < nstages; ++st) {
       __syncthreads();   // every warp is done with the buffer about to be refilled
-      if (st + STAGES - 1 < nstages) issue(st + STAGES - 1);
+      if (st + STAGES - 1 < nstages) issue_rows(st + STAGES - 1, gbase + st + STAGES - 1);
+      if (st == trig && tid == 0 && has_next) {
+        bounded_wait(smem_u32(recbar + ((k + 1) & 1)), uint32_t((k + 1) >> 1) & 1u, kWaitPolls,
+                     abort_flag);
+        issue_index(next, nrec);
+      }
       const int buf = (gbase + st) % STAGES;
       bounded_wait(smem_u32(fullbar + buf), uint32_t((gbase + st) / STAGES) & 1u, kWaitPolls,
                    abort_flag);
@@ -329,8 +328,8 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
       // ---- mask (rows g and g+8 of the tile; bit k <-> union atom ub + k);
       // the stage's RS <= 32 bits sit in one mask word
       const int ub = st * RS;
-      const uint32_t m0 = smask[g * swords + (ub >> 5)] >> ((ub & 31) + 2 * t);
-      const uint32_t m1 = smask[(g + 8) * swords + (ub >> 5)] >> ((ub & 31) + 2 * t);
+      const uint32_t m0 = smask[(ub >> 5) * kTileM + g] >> ((ub & 31) + 2 * t);
+      const uint32_t m1 = smask[(ub >> 5) * kTileM + g + 8] >> ((ub & 31) + 2 * t);
       float v[KS][8];   // raw logits; row g: cols 2t, 2t+1, 8+2t, 9+2t ; row g+8: same
       bool over = false;
 #pragma unroll
@@ -424,10 +423,32 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
         }
       }   // k-steps of the stage
     }
-    __syncthreads();   // all staged buffers consumed
+    __syncthreads();   // every warp is done with the stage buffers and the mask
     gbase += nstages;
+    if (tid == 0 && has_next) {
+      if (nstages == 0) {
+        bounded_wait(smem_u32(recbar + ((k + 1) & 1)), uint32_t((k + 1) >> 1) & 1u, kWaitPolls,
+                     abort_flag);
+        issue_index(next, nrec);
+      }
+      issue_mask(next, nrec);
+    }
+    // the next tile's first rows (needs its record and indices)
+    auto stage_next = [&]() {
+      bounded_wait(smem_u32(recbar + ((k + 1) & 1)), uint32_t((k + 1) >> 1) & 1u, kWaitPolls,
+                   abort_flag);
+      bounded_wait(smem_u32(idxbar), uint32_t(k + 1) & 1u, kWaitPolls, abort_flag);
+      const int ns = stages_of(nrec);
+      for (int s = 0; s < STAGES - 1 && s < ns; ++s) issue_rows(s, gbase + s);
+    };
+    if (kEarlyRows && has_next) stage_next();
 
-    // ---- epilogue: normalise; either write m or apply the target coupling
+    // ---- epilogue of the tile: normalise; either write m or apply the target
+    // coupling (the next tile's first rows are already in flight, except at
+    // fused lmax 3)
+    const int* tgt = reinterpret_cast<const int*>(rec) + kRecTgt;
+    const float* rp = rec + kRecRp;             // [16][L+1]
+    const float* Dq = rec + rec_off_D(L);       // [16][WS]
     const float inv0 = zacc[0] > 0.f ? 1.f / zacc[0] : 0.f;
     const float inv1 = zacc[2] > 0.f ? 1.f / zacc[2] : 0.f;
     const int ch = h * 8 + 2 * t;
@@ -491,15 +512,25 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
                          });
       }
     }
-    if constexpr (FUSED && L >= 3) fence_proxy_async_smem();   // scratch before bulk copies
-    __syncthreads();   // tgt / Dq / rp are rewritten by the next tile
+    if constexpr (!kEarlyRows) fence_proxy_async_smem();   // scratch before bulk copies
+    __syncthreads();   // the record buffer and the stage buffers are refilled next
+    if (!kEarlyRows && has_next) stage_next();
   }
-  if (*abort_flag && threadIdx.x == 0) {
-    // a wait gave up: give each buffer's last fill a short, bounded chance to
-    // land before the CTA's shared memory is released
+  if (*abort_flag && tid == 0) {
+    // a wait gave up: give every barrier's last phase a short, bounded chance
+    // to complete before the CTA's shared memory is released
     volatile int none = 0;
     for (int b = 0; b < STAGES && b < gbase; ++b)
-      bounded_wait(smem_u32(fullbar + b), uint32_t((gbase - 1 - b) / STAGES) & 1u, kDrainPolls, &none);
+      bounded_wait(smem_u32(fullbar + b), uint32_t((gbase - 1 - b) / STAGES) & 1u, kDrainPolls,
+                   &none);
+    for (int b = 0; b < 2; ++b) {
+      const int last = k - 1 - ((k - 1 - b) & 1);   // last tile sequence number of parity b
+      if (last >= 0) bounded_wait(smem_u32(recbar + b), uint32_t(last >> 1) & 1u, kDrainPolls, &none);
+    }
+    if (k > 0) {
+      bounded_wait(smem_u32(idxbar), uint32_t(k - 1) & 1u, kDrainPolls, &none);
+      bounded_wait(smem_u32(mskbar), uint32_t(k - 1) & 1u, kDrainPolls, &none);
+    }
   }
 }
 
@@ -520,8 +551,7 @@ __global__ void wait_timeout_selftest_kernel(int polls) {
 
 template <int L, int H, bool FUSED>
 int launch_tc_t(const TcParams& p, int tiles, cudaStream_t st) {
-  const size_t shmem = tc_smem_fixed<L, H>() + tc_smem_plan(p.plan.cap) +
-                       (FUSED ? tc_smem_w2<L, H>() : 0) + kBarBytes;
+  const size_t shmem = TcSmem<L, H, FUSED>::total(p.plan.cap);
   if (shmem > 227 * 1024) return EGAT_ERR_UNSUPPORTED;
   auto kern = otf_attention_tc_kernel<L, H, FUSED>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(shmem)) !=
@@ -542,11 +572,10 @@ bool tc_attention_supported(const egat_shape& s) {
         s.C == 128 && s.lmax >= 1 && s.lmax <= 3))
     return false;
   if (plan_smem_bytes(s.n, s.K) > kPlanSmemLimit) return false;
-  const size_t fixed = s.lmax == 1 ? tc_smem_fixed<1, 16>()
-                     : s.lmax == 2 ? tc_smem_fixed<2, 16>() : tc_smem_fixed<3, 16>();
-  const size_t w2 = s.lmax == 1 ? tc_smem_w2<1, 16>()
-                  : s.lmax == 2 ? tc_smem_w2<2, 16>() : tc_smem_w2<3, 16>();
-  return fixed + tc_smem_plan(plan_capacity(s.K)) + w2 + kBarBytes <= 227 * 1024;
+  const int cap = plan_capacity(s.K);
+  const size_t smem = s.lmax == 1 ? TcSmem<1, 16, true>::total(cap)
+                    : s.lmax == 2 ? TcSmem<2, 16, true>::total(cap) : TcSmem<3, 16, true>::total(cap);
+  return smem <= 227 * 1024;
 }
 
 int launch_attention_tc(const egat_shape& s, bool fused, const void* d_q, const void* d_k,
@@ -575,15 +604,8 @@ int launch_attention_tc(const egat_shape& s, bool fused, const void* d_q, const 
   }
 }
 
-int take_wait_timeouts(cudaStream_t st, unsigned int* count) {
-  void* addr = nullptr;
-  if (cudaGetSymbolAddress(&addr, g_wait_timeouts) != cudaSuccess) return EGAT_ERR_CUDA;
-  unsigned int h = 0;
-  if (cudaMemcpyAsync(&h, addr, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-      cudaMemsetAsync(addr, 0, sizeof(h), st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
-    return EGAT_ERR_CUDA;
-  *count = h;
-  return EGAT_OK;
+int take_wait_timeouts_attention(cudaStream_t st, unsigned int* count) {
+  return take_unit_wait_timeouts(st, count) == 0 ? EGAT_OK : EGAT_ERR_CUDA;
 }
 
 int launch_wait_timeout_selftest(int polls, cudaStream_t st) {

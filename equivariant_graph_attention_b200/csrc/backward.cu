@@ -1,0 +1,589 @@
+// Backward pass of steps 2-4: the gradients of L = sum_i <G_i, ^h_i> with
+// respect to the features h, the queries q and the keys k, for an upstream
+// gradient G = dL/d^h.
+//
+// The pages name the backward pass as the step after the forward (forces as
+// energy gradients in the Conservative mode) and keep the attention weights
+// off HBM ("E2Former-V2：突破等变图神经网络计算瓶颈的创新架构" §3.2, linear
+// activation memory; "E2Former-V2: On-the-Fly Equivariant Attention with
+// Linear Activation Memory" §2.2).  Here too no per-edge quantity is stored:
+// every weight is recomputed from q, k and one log-sum-exp per (target,
+// head).  Steps, each the adjoint of a forward step:
+//  1. dm = T*(G; r, w2): the target coupling is linear in m, so its adjoint
+//     is the same rotate / re-index / rotate-back operator with the re-index
+//     read backwards (eaas_channel_adjoint).  h' and dm are held in float32
+//     whatever the storage type: the softmax backward subtracts nearly equal
+//     quantities (dalpha - Delta), and bf16 intermediates there cost up to 3e-2
+//     relative error on single (atom, head) rows of dq and dk;
+//  2. the neighbour lists are transposed (in-lists: the targets each atom
+//     serves), sorted so every sum runs in a fixed order;
+//  3. per target i (one warp): the forward recomputed gives m_i and the
+//     per-head log-sum-exp; Delta_i = <dm_i, m_i> per head; a second sweep
+//     gives ds_ij = alpha_ij (<dm_i, h'_j>_head - Delta_i) and
+//     dq_i = sum_j ds_ij k_j / sqrt(dk);
+//  4. per source j (one warp) over its in-list: alpha_ij from q_i, k_j and
+//     the target's log-sum-exp, dh'_j = sum_i alpha_ij dm_i,
+//     dk_j = sum_i ds_ij q_i / sqrt(dk); the epilogue applies the adjoint of
+//     the source coupling, dh_j = T*(dh'_j; r_j, w1).
+// Step 2's in-lists make every gradient a gather: no atomics touch a result.
+#include <cfloat>
+#include <climits>
+
+#include "egat_device.cuh"
+#include "egat_host.h"
+
+namespace egat {
+namespace {
+
+constexpr int kBwdWarps = 4;
+constexpr int kSortCap = 4096;   // in-list length sorted in shared memory
+
+// ---------------------------------------------------------------- step 1
+template <int L, typename T>
+__global__ void __launch_bounds__(kBwdWarps * 32)
+adjoint_coupling_kernel(const float* __restrict__ g, const float* __restrict__ pos,
+                        const float* __restrict__ w, T* __restrict__ out, int n, int C,
+                        const __grid_constant__ EaasTable tab) {
+  constexpr int D = (L + 1) * (L + 1);
+  constexpr int WS = wig_size(L);
+  __shared__ float Dsm[kBwdWarps][WS];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int a = blockIdx.x * kBwdWarps + wib;
+  if (a >= n) return;   // whole warp
+  float Q[9];
+  const float r = alignment_rotation(pos[3 * a], pos[3 * a + 1], pos[3 * a + 2], Q);
+  float rpow[L + 1];
+  rpow[0] = 1.f;
+#pragma unroll
+  for (int l = 1; l <= L; ++l) rpow[l] = rpow[l - 1] * r;
+  wigner_build<L>(Q, Dsm[wib], lane, 32, [] { __syncwarp(); });
+  __syncwarp();
+  for (int c = lane; c < C; c += 32) {
+    float x[D];
+#pragma unroll
+    for (int d = 0; d < D; ++d) x[d] = g[((size_t)a * D + d) * C + c];
+    eaas_channel_adjoint<L>(x, Dsm[wib], rpow, tab, [&](int pp) { return __ldg(w + pp * C + c); },
+                            [&](int d, float v) { store_one<T>(out + ((size_t)a * D + d) * C + c, v); });
+  }
+}
+
+// ---------------------------------------------------------------- step 2
+__device__ __forceinline__ int row_count(const int32_t* cnt, int i, int K) {
+  int c = cnt ? cnt[i] : K;
+  return c < 0 ? 0 : (c > K ? K : c);
+}
+
+__global__ void in_degree_kernel(const int32_t* __restrict__ nbr, const int32_t* __restrict__ cnt,
+                                 int n, int K, int* __restrict__ deg) {
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (long long)n * K) return;
+  const int i = int(e / K), s = int(e % K);
+  if (s >= row_count(cnt, i, K)) return;
+  const int j = nbr[e];
+  if ((unsigned)j < (unsigned)n) atomicAdd(&deg[j], 1);
+}
+
+// exclusive scan of deg[0..n) into ptr[0..n] by one CTA (chunk per thread)
+__global__ void __launch_bounds__(1024) scan_one_cta_kernel(const int* __restrict__ deg, int n,
+                                                           int* __restrict__ ptr) {
+  __shared__ int part[1024];
+  const int t = threadIdx.x;
+  const int per = (n + 1023) / 1024;
+  const int b0 = min(t * per, n), b1 = min(b0 + per, n);
+  int sum = 0;
+  for (int k = b0; k < b1; ++k) sum += deg[k];
+  part[t] = sum;
+  __syncthreads();
+  for (int o = 1; o < 1024; o <<= 1) {
+    const int v = t >= o ? part[t - o] : 0;
+    __syncthreads();
+    part[t] += v;
+    __syncthreads();
+  }
+  int run = t ? part[t - 1] : 0;
+  for (int k = b0; k < b1; ++k) {
+    ptr[k] = run;
+    run += deg[k];
+  }
+  if (t == 1023) ptr[n] = part[1023];
+}
+
+__global__ void in_fill_kernel(const int32_t* __restrict__ nbr, const int32_t* __restrict__ cnt,
+                               int n, int K, const int* __restrict__ ptr, int* __restrict__ cursor,
+                               int* __restrict__ in) {
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (long long)n * K) return;
+  const int i = int(e / K), s = int(e % K);
+  if (s >= row_count(cnt, i, K)) return;
+  const int j = nbr[e];
+  if ((unsigned)j >= (unsigned)n) return;
+  in[ptr[j] + atomicAdd(&cursor[j], 1)] = i;
+}
+
+// Sort every in-list ascending: a block-wide bitonic sort in shared memory
+// up to kSortCap entries; a longer list (only for very dense systems) is
+// ranked element by element through `scratch` (its entries are distinct).
+__global__ void __launch_bounds__(256) in_sort_kernel(const int* __restrict__ ptr,
+                                                      int* __restrict__ in,
+                                                      int* __restrict__ scratch) {
+  __shared__ int key[kSortCap];
+  const int j = blockIdx.x;
+  const int beg = ptr[j], len = ptr[j + 1] - beg;
+  if (len <= 1) return;
+  if (len <= kSortCap) {
+    int m = 1;
+    while (m < len) m <<= 1;
+    for (int t = threadIdx.x; t < m; t += blockDim.x) key[t] = t < len ? in[beg + t] : INT_MAX;
+    __syncthreads();
+    for (int size = 2; size <= m; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        for (int t = threadIdx.x; t < m; t += blockDim.x) {
+          const int u = t ^ stride;
+          if (u > t) {
+            const bool up = (t & size) == 0;
+            const int a = key[t], b = key[u];
+            if ((a > b) == up) {
+              key[t] = b;
+              key[u] = a;
+            }
+          }
+        }
+        __syncthreads();
+      }
+    }
+    for (int t = threadIdx.x; t < len; t += blockDim.x) in[beg + t] = key[t];
+  } else {
+    for (int t = threadIdx.x; t < len; t += blockDim.x) {
+      const int v = in[beg + t];
+      int rank = 0;
+      for (int u = 0; u < len; ++u) rank += in[beg + u] < v;
+      scratch[beg + rank] = v;
+    }
+    __syncthreads();
+    for (int t = threadIdx.x; t < len; t += blockDim.x) in[beg + t] = scratch[beg + t];
+  }
+}
+
+// ---------------------------------------------------------------- steps 3, 4
+struct BwdParams {
+  const void* q;
+  const void* k;
+  const void* hp;
+  const void* dm;
+  const int32_t* nbr;    // [n][K]
+  const int32_t* cnt;    // [n] or null
+  const int* in_ptr;     // [n+1]
+  const int* in;         // in-lists
+  float* lse;            // [n][H]  log2-domain log-sum-exp of the logits
+  float* delta;          // [n][H]
+  float* dq;             // [n][H][dk]
+  float* dk;             // [n][H][dk]
+  float* dh;             // [n][D][C]
+  const float* pos;
+  const float* w1;
+  int n, H, dk_, K, cph;
+  float qscale;          // log2(e) / sqrt(dk)
+  float kscale;          // 1 / sqrt(dk)
+  EaasTable tab;
+};
+
+// sum over the lanes whose value chunks belong to the same head: the bits of
+// the lane index inside a head's chunks (below cph) and the component bits
+// (CPW and above)
+template <int CPW>
+__device__ __forceinline__ float head_sum(float v, int cph) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1)
+    if (o < cph || o >= CPW) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <int L, int C, typename T>
+struct BwdLayout {
+  static constexpr int D = (L + 1) * (L + 1);
+  static constexpr int NCH = D * C / 8;          // 8-element chunks per row
+  static constexpr int TPL = (NCH + 31) / 32;    // chunks per lane
+  static constexpr int CPW = C / 8;              // chunks per component
+  static_assert(32 % CPW == 0, "C/8 must divide 32");
+};
+
+// per-lane partial dot product of two rows held as chunks
+template <int TPL, int NCH>
+__device__ __forceinline__ float chunk_dot(const float (&a)[TPL][8], const float (&b)[TPL][8],
+                                           int lane) {
+  float s = 0.f;
+#pragma unroll
+  for (int t = 0; t < TPL; ++t)
+    if (lane + 32 * t < NCH)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s = fmaf(a[t][e], b[t][e], s);
+  return s;
+}
+
+template <int TPL, int NCH, typename T>
+__device__ __forceinline__ void load_row(const T* __restrict__ row, float (&v)[TPL][8], int lane) {
+#pragma unroll
+  for (int t = 0; t < TPL; ++t) {
+    const int q = lane + 32 * t;
+    Chunk8<T> c;
+    if (q < NCH) c.load(row + 8 * q);
+    else c.zero();
+    c.to_f32(v[t]);
+  }
+}
+
+// Step 3: one warp per target.
+template <int L, int C, typename T>
+__global__ void __launch_bounds__(kBwdWarps * 32)
+attn_bwd_target_kernel(const __grid_constant__ BwdParams p) {
+  using Ly = BwdLayout<L, C, T>;
+  constexpr int D = Ly::D, NCH = Ly::NCH, TPL = Ly::TPL, CPW = Ly::CPW;
+  const int lane = threadIdx.x & 31;
+  const int i = blockIdx.x * kBwdWarps + (threadIdx.x >> 5);
+  if (i >= p.n) return;   // whole warp
+  const T* __restrict__ qp = static_cast<const T*>(p.q);
+  const T* __restrict__ kp = static_cast<const T*>(p.k);
+  const float* __restrict__ hp = static_cast<const float*>(p.hp);
+  const float* __restrict__ dmp = static_cast<const float*>(p.dm);
+  const int hdk = p.H * p.dk_;
+  const int kch = hdk >> 3;
+  const int G = p.dk_ >> 3;
+  const int head = ((lane % CPW) * 8 * p.H) / C;
+
+  float qv[8];
+  {
+    Chunk8<T> qc;
+    if (lane < kch) qc.load(qp + (size_t)i * hdk + 8 * lane);
+    else qc.zero();
+    qc.to_f32(qv);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) qv[e] *= p.qscale;
+  }
+  auto logit = [&](int j) {   // log2-domain logit of this lane's head
+    float kf[8];
+    Chunk8<T> kc;
+    if (lane < kch) kc.load(kp + (size_t)j * hdk + 8 * lane);
+    else kc.zero();
+    kc.to_f32(kf);
+    float sp = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sp = fmaf(qv[e], kf[e], sp);
+    for (int o = 1; o < G; o <<= 1) sp += __shfl_xor_sync(0xffffffffu, sp, o);
+    return __shfl_sync(0xffffffffu, sp, head * G);
+  };
+  const long long beg = (long long)i * p.K;
+  const long long end = beg + row_count(p.cnt, i, p.K);
+
+  // pass 1: the forward recomputed (two-pass softmax: maximum, then sums)
+  float mx = -INFINITY;
+  for (long long s = beg; s < end; ++s) {
+    const int j = p.nbr[s];
+    if ((unsigned)j >= (unsigned)p.n) continue;
+    mx = fmaxf(mx, logit(j));
+  }
+  float z = 0.f;
+  float acc[TPL][8];
+#pragma unroll
+  for (int t = 0; t < TPL; ++t)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[t][e] = 0.f;
+  for (long long s = beg; s < end; ++s) {
+    const int j = p.nbr[s];
+    if ((unsigned)j >= (unsigned)p.n) continue;
+    const float pw = exp2f(logit(j) - mx);
+    z += pw;
+    float hv[TPL][8];
+    load_row<TPL, NCH>(hp + (size_t)j * D * C, hv, lane);
+#pragma unroll
+    for (int t = 0; t < TPL; ++t)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[t][e] = fmaf(pw, hv[t][e], acc[t][e]);
+  }
+  const float lse = z > 0.f ? mx + log2f(z) : -INFINITY;
+  const float inv = z > 0.f ? 1.f / z : 0.f;
+  float dmv[TPL][8];
+  load_row<TPL, NCH>(dmp + (size_t)i * D * C, dmv, lane);
+#pragma unroll
+  for (int t = 0; t < TPL; ++t)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[t][e] *= inv;   // m_i
+  const float delta = head_sum<CPW>(chunk_dot<TPL, NCH>(dmv, acc, lane), p.cph);
+  if (lane < CPW && lane % p.cph == 0) {
+    p.lse[(size_t)i * p.H + head] = lse;
+    p.delta[(size_t)i * p.H + head] = delta;
+  }
+
+  // pass 2: ds_ij and dq_i
+  float dqv[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) dqv[e] = 0.f;
+  const int khead = lane < kch ? lane / G : 0;   // head of this lane's key chunk
+  for (long long s = beg; s < end; ++s) {
+    const int j = p.nbr[s];
+    if ((unsigned)j >= (unsigned)p.n) continue;
+    const float a = exp2f(logit(j) - lse);
+    float hv[TPL][8];
+    load_row<TPL, NCH>(hp + (size_t)j * D * C, hv, lane);
+    const float da = head_sum<CPW>(chunk_dot<TPL, NCH>(dmv, hv, lane), p.cph);
+    const float ds = a * (da - delta);
+    const float dsk = __shfl_sync(0xffffffffu, ds, khead * p.cph);
+    if (lane < kch) {
+      float kf[8];
+      Chunk8<T> kc;
+      kc.load(kp + (size_t)j * hdk + 8 * lane);
+      kc.to_f32(kf);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) dqv[e] = fmaf(dsk, kf[e], dqv[e]);
+    }
+  }
+  if (lane < kch) {
+    float* o = p.dq + (size_t)i * hdk + 8 * lane;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[e] = dqv[e] * p.kscale;
+  }
+}
+
+// Step 4: one warp per source atom over its in-list, then the adjoint of the
+// source coupling in the epilogue.
+template <int L, int C, typename T>
+__global__ void __launch_bounds__(kBwdWarps * 32)
+attn_bwd_source_kernel(const __grid_constant__ BwdParams p) {
+  using Ly = BwdLayout<L, C, T>;
+  constexpr int D = Ly::D, NCH = Ly::NCH, TPL = Ly::TPL, CPW = Ly::CPW;
+  constexpr int WS = wig_size(L);
+  extern __shared__ float smem[];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int j = blockIdx.x * kBwdWarps + wib;
+  if (j >= p.n) return;   // whole warp
+  const T* __restrict__ qp = static_cast<const T*>(p.q);
+  const T* __restrict__ kp = static_cast<const T*>(p.k);
+  const float* __restrict__ hp = static_cast<const float*>(p.hp);
+  const float* __restrict__ dmp = static_cast<const float*>(p.dm);
+  const int hdk = p.H * p.dk_;
+  const int kch = hdk >> 3;
+  const int G = p.dk_ >> 3;
+  const int head = ((lane % CPW) * 8 * p.H) / C;
+  const int khead = lane < kch ? lane / G : 0;
+
+  float kv[8];
+  {
+    Chunk8<T> kc;
+    if (lane < kch) kc.load(kp + (size_t)j * hdk + 8 * lane);
+    else kc.zero();
+    kc.to_f32(kv);
+  }
+  float hv[TPL][8];
+  load_row<TPL, NCH>(hp + (size_t)j * D * C, hv, lane);
+  float dhp[TPL][8];
+#pragma unroll
+  for (int t = 0; t < TPL; ++t)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) dhp[t][e] = 0.f;
+  float dkv[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) dkv[e] = 0.f;
+
+  const int b = p.in_ptr[j], e_ = p.in_ptr[j + 1];
+  for (int s = b; s < e_; ++s) {
+    const int i = p.in[s];
+    if ((unsigned)i >= (unsigned)p.n) continue;
+    float qf[8];
+    {
+      Chunk8<T> qc;
+      if (lane < kch) qc.load(qp + (size_t)i * hdk + 8 * lane);
+      else qc.zero();
+      qc.to_f32(qf);
+    }
+    float sp = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sp = fmaf(qf[e] * p.qscale, kv[e], sp);
+    for (int o = 1; o < G; o <<= 1) sp += __shfl_xor_sync(0xffffffffu, sp, o);
+    const float sl = __shfl_sync(0xffffffffu, sp, head * G);
+    const float a = exp2f(sl - __ldg(p.lse + (size_t)i * p.H + head));
+    float dmv[TPL][8];
+    load_row<TPL, NCH>(dmp + (size_t)i * D * C, dmv, lane);
+    const float da = head_sum<CPW>(chunk_dot<TPL, NCH>(dmv, hv, lane), p.cph);
+    const float ds = a * (da - __ldg(p.delta + (size_t)i * p.H + head));
+#pragma unroll
+    for (int t = 0; t < TPL; ++t)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) dhp[t][e] = fmaf(a, dmv[t][e], dhp[t][e]);
+    const float dsk = __shfl_sync(0xffffffffu, ds, khead * p.cph);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) dkv[e] = fmaf(dsk, qf[e], dkv[e]);
+  }
+  if (lane < kch) {
+    float* o = p.dk + (size_t)j * hdk + 8 * lane;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[e] = dkv[e] * p.kscale;
+  }
+
+  // epilogue: dh_j = T*(dh'_j; r_j, w1), one channel per lane at a time
+  float* gbuf = smem + wib * (D * C + WS);
+  float* Dsm = gbuf + D * C;
+#pragma unroll
+  for (int t = 0; t < TPL; ++t) {
+    const int q = lane + 32 * t;
+    if (q < NCH)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) gbuf[8 * q + e] = dhp[t][e];
+  }
+  float Q[9];
+  const float r = alignment_rotation(p.pos[3 * j], p.pos[3 * j + 1], p.pos[3 * j + 2], Q);
+  float rpow[L + 1];
+  rpow[0] = 1.f;
+#pragma unroll
+  for (int l = 1; l <= L; ++l) rpow[l] = rpow[l - 1] * r;
+  wigner_build<L>(Q, Dsm, lane, 32, [] { __syncwarp(); });
+  __syncwarp();
+  float* o = p.dh + (size_t)j * D * C;
+  for (int c = lane; c < C; c += 32) {
+    float x[D];
+#pragma unroll
+    for (int d = 0; d < D; ++d) x[d] = gbuf[d * C + c];
+    eaas_channel_adjoint<L>(x, Dsm, rpow, p.tab, [&](int pp) { return __ldg(p.w1 + pp * C + c); },
+                            [&](int d, float v) { o[d * C + c] = v; });
+  }
+}
+
+template <int L, int C, typename T>
+int launch_attn_bwd(const BwdParams& p, cudaStream_t st) {
+  constexpr int D = (L + 1) * (L + 1);
+  const int grid = (p.n + kBwdWarps - 1) / kBwdWarps;
+  attn_bwd_target_kernel<L, C, T><<<grid, kBwdWarps * 32, 0, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return EGAT_ERR_CUDA;
+  const size_t shmem = size_t(kBwdWarps) * (D * C + wig_size(L)) * sizeof(float);
+  auto kern = attn_bwd_source_kernel<L, C, T>;
+  if (shmem > 48 * 1024 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(shmem)) != cudaSuccess)
+    return EGAT_ERR_CUDA;
+  kern<<<grid, kBwdWarps * 32, shmem, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
+}
+
+template <int L, typename T>
+int dispatch_c(const BwdParams& p, int C, cudaStream_t st) {
+  switch (C) {
+    case 16: return launch_attn_bwd<L, 16, T>(p, st);
+    case 32: return launch_attn_bwd<L, 32, T>(p, st);
+    case 64: return launch_attn_bwd<L, 64, T>(p, st);
+    case 128: return launch_attn_bwd<L, 128, T>(p, st);
+    default: return EGAT_ERR_UNSUPPORTED;
+  }
+}
+
+template <int L, typename T>
+int launch_adjoint(const egat_shape& s, const float* g, const float* pos, const float* w, void* out,
+                   cudaStream_t st) {
+  const int grid = (s.n + kBwdWarps - 1) / kBwdWarps;
+  adjoint_coupling_kernel<L, T><<<grid, kBwdWarps * 32, 0, st>>>(g, pos, w, static_cast<T*>(out), s.n,
+                                                                s.C, eaas_table(L));
+  return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
+}
+
+size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct BwdWs {
+  void* hp;
+  void* dm;
+  int* deg;
+  int* ptr;
+  int* cursor;
+  int* in;
+  int* scratch;
+  float* lse;
+  float* delta;
+  size_t bytes;
+};
+
+BwdWs bwd_ws(const egat_shape& s, void* base) {
+  const size_t D = size_t(s.lmax + 1) * (s.lmax + 1);
+  const size_t row = D * s.C * sizeof(float);   // h' and dm in float32
+  const size_t n = size_t(s.n), E = size_t(s.n) * s.K;
+  BwdWs w;
+  char* b = static_cast<char*>(base);
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    void* ptr = b ? b + o : nullptr;
+    o += a256(bytes);
+    return ptr;
+  };
+  w.hp = take(n * row);
+  w.dm = take(n * row);
+  w.deg = static_cast<int*>(take(n * 4));
+  w.ptr = static_cast<int*>(take((n + 1) * 4));
+  w.cursor = static_cast<int*>(take(n * 4));
+  w.in = static_cast<int*>(take(E * 4));
+  w.scratch = static_cast<int*>(take(E * 4));
+  w.lse = static_cast<float*>(take(n * s.H * 4));
+  w.delta = static_cast<float*>(take(n * s.H * 4));
+  w.bytes = o;
+  return w;
+}
+
+}  // namespace
+
+size_t backward_ws_bytes(const egat_shape& s) { return bwd_ws(s, nullptr).bytes; }
+
+int launch_backward(const egat_shape& s, const void* d_h, const float* d_pos, const void* d_q,
+                    const void* d_k, const int32_t* d_nbr, const int32_t* d_cnt, const float* d_w1,
+                    const float* d_w2, const float* d_g, void* d_ws, float* d_dh, float* d_dq,
+                    float* d_dk, cudaStream_t st) {
+  const BwdWs w = bwd_ws(s, d_ws);
+  const bool bf = s.dtype == EGAT_BF16;
+  // h' = source coupling (forward step 2), in float32
+  int e = launch_eaas_source_f32out(s, d_h, d_pos, d_w1, static_cast<float*>(w.hp), st);
+  if (e != EGAT_OK) return e;
+  // step 1: dm = T*(G; r, w2)
+  switch (s.lmax) {
+    case 1: e = launch_adjoint<1, float>(s, d_g, d_pos, d_w2, w.dm, st); break;
+    case 2: e = launch_adjoint<2, float>(s, d_g, d_pos, d_w2, w.dm, st); break;
+    case 3: e = launch_adjoint<3, float>(s, d_g, d_pos, d_w2, w.dm, st); break;
+    default: return EGAT_ERR_UNSUPPORTED;
+  }
+  if (e != EGAT_OK) return e;
+  // step 2: in-lists
+  if (cudaMemsetAsync(w.deg, 0, size_t(s.n) * 4, st) != cudaSuccess ||
+      cudaMemsetAsync(w.cursor, 0, size_t(s.n) * 4, st) != cudaSuccess)
+    return EGAT_ERR_CUDA;
+  const long long E = (long long)s.n * s.K;
+  const int eb = int((E + 255) / 256);
+  in_degree_kernel<<<eb, 256, 0, st>>>(d_nbr, d_cnt, s.n, s.K, w.deg);
+  scan_one_cta_kernel<<<1, 1024, 0, st>>>(w.deg, s.n, w.ptr);
+  in_fill_kernel<<<eb, 256, 0, st>>>(d_nbr, d_cnt, s.n, s.K, w.ptr, w.cursor, w.in);
+  in_sort_kernel<<<s.n, 256, 0, st>>>(w.ptr, w.in, w.scratch);
+  if (cudaGetLastError() != cudaSuccess) return EGAT_ERR_CUDA;
+  // steps 3, 4
+  BwdParams p;
+  p.q = d_q;
+  p.k = d_k;
+  p.hp = w.hp;
+  p.dm = w.dm;
+  p.nbr = d_nbr;
+  p.cnt = d_cnt;
+  p.in_ptr = w.ptr;
+  p.in = w.in;
+  p.lse = w.lse;
+  p.delta = w.delta;
+  p.dq = d_dq;
+  p.dk = d_dk;
+  p.dh = d_dh;
+  p.pos = d_pos;
+  p.w1 = d_w1;
+  p.n = s.n;
+  p.H = s.H;
+  p.dk_ = s.dk;
+  p.K = s.K;
+  p.cph = s.C / (8 * s.H);
+  p.qscale = float(1.4426950408889634 / std::sqrt(double(s.dk)));
+  p.kscale = float(1.0 / std::sqrt(double(s.dk)));
+  p.tab = eaas_table(s.lmax);
+  switch (s.lmax) {
+    case 1: return bf ? dispatch_c<1, __nv_bfloat16>(p, s.C, st) : dispatch_c<1, float>(p, s.C, st);
+    case 2: return bf ? dispatch_c<2, __nv_bfloat16>(p, s.C, st) : dispatch_c<2, float>(p, s.C, st);
+    case 3: return bf ? dispatch_c<3, __nv_bfloat16>(p, s.C, st) : dispatch_c<3, float>(p, s.C, st);
+    default: return EGAT_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace egat

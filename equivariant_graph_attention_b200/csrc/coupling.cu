@@ -16,6 +16,7 @@
 #include <cmath>
 #include <mutex>
 
+#include "egat_async.cuh"
 #include "egat_device.cuh"
 #include "egat_host.h"
 
@@ -112,7 +113,12 @@ struct ChanVec;
 template <>
 struct ChanVec<__nv_bfloat16, 4> {
   static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[4]) {
-    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    unpack(__ldg(reinterpret_cast<const uint2*>(p)), v);
+  }
+  static __device__ __forceinline__ void load_shared(const __nv_bfloat16* p, float (&v)[4]) {
+    unpack(*reinterpret_cast<const uint2*>(p), v);
+  }
+  static __device__ __forceinline__ void unpack(const uint2 u, float (&v)[4]) {
     v[0] = __uint_as_float(u.x << 16); v[1] = __uint_as_float(u.x & 0xffff0000u);
     v[2] = __uint_as_float(u.y << 16); v[3] = __uint_as_float(u.y & 0xffff0000u);
   }
@@ -130,6 +136,10 @@ struct ChanVec<__nv_bfloat16, 2> {
     const uint32_t u = __ldg(reinterpret_cast<const unsigned int*>(p));
     v[0] = __uint_as_float(u << 16); v[1] = __uint_as_float(u & 0xffff0000u);
   }
+  static __device__ __forceinline__ void load_shared(const __nv_bfloat16* p, float (&v)[2]) {
+    const uint32_t u = *reinterpret_cast<const unsigned int*>(p);
+    v[0] = __uint_as_float(u << 16); v[1] = __uint_as_float(u & 0xffff0000u);
+  }
   static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[2]) {
     __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
     *reinterpret_cast<__nv_bfloat162*>(p) = a;
@@ -141,6 +151,10 @@ struct ChanVec<float, 4> {
     const float4 u = __ldg(reinterpret_cast<const float4*>(p));
     v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
   }
+  static __device__ __forceinline__ void load_shared(const float* p, float (&v)[4]) {
+    const float4 u = *reinterpret_cast<const float4*>(p);
+    v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+  }
   static __device__ __forceinline__ void store(float* p, const float (&v)[4]) {
     *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
   }
@@ -149,6 +163,10 @@ template <>
 struct ChanVec<float, 2> {
   static __device__ __forceinline__ void load(const float* p, float (&v)[2]) {
     const float2 u = __ldg(reinterpret_cast<const float2*>(p));
+    v[0] = u.x; v[1] = u.y;
+  }
+  static __device__ __forceinline__ void load_shared(const float* p, float (&v)[2]) {
+    const float2 u = *reinterpret_cast<const float2*>(p);
     v[0] = u.x; v[1] = u.y;
   }
   static __device__ __forceinline__ void store(float* p, const float (&v)[2]) {
@@ -165,7 +183,7 @@ struct ChanVec<float, 2> {
 // PLANNED: the items are the target slots of an attention plan, whose tile
 // records already hold each atom's index, |r|^l and Wigner-D matrices; the
 // group copies them instead of building them.
-template <int L, typename T, bool PLANNED>
+template <int L, typename T, bool PLANNED, typename TO = T>
 __global__ void __launch_bounds__(kEaasWarps * 32, (L >= 3 ? 1 : 2))
 eaas_source_kernel(const __grid_constant__ EaasParams p) {
   constexpr int D = (L + 1) * (L + 1);
@@ -190,9 +208,9 @@ eaas_source_kernel(const __grid_constant__ EaasParams p) {
   const int part = int(gwarp % WPA);            // which warp of the atom's group
   const int c0 = (part * 32 + gl) * CPL;         // first channel of this lane
   const long long ngroups = (p.items + AW - 1) / AW;
-  constexpr int REC = kTileM * (1 + (L + 1) + WS);
+  constexpr int REC = plan_record_words(L);
   const T* __restrict__ x = static_cast<const T*>(p.x);
-  T* __restrict__ y = static_cast<T*>(p.y);
+  TO* __restrict__ y = static_cast<TO*>(p.y);
   float* Dme = Dsm[wib][slot];
   for (int e = threadIdx.x; e < NP * C; e += blockDim.x) sw[e] = __ldg(p.w + e);
   __syncthreads();
@@ -207,7 +225,7 @@ eaas_source_kernel(const __grid_constant__ EaasParams p) {
       if (live) {
         R = p.rec + (item / kTileM) * REC;
         rs = int(item % kTileM);
-        at = reinterpret_cast<const int*>(R)[rs];
+        at = reinterpret_cast<const int*>(R)[kRecTgt + rs];
         live = (unsigned long long)at < (unsigned long long)p.n;
       }
     }
@@ -232,10 +250,10 @@ eaas_source_kernel(const __grid_constant__ EaasParams p) {
     float rpow[L + 1];
     if constexpr (PLANNED) {
 #pragma unroll
-      for (int l = 0; l <= L; ++l) rpow[l] = live ? __ldg(R + kTileM + rs * (L + 1) + l) : 0.f;
+      for (int l = 0; l <= L; ++l) rpow[l] = live ? __ldg(R + kRecRp + rs * (L + 1) + l) : 0.f;
       __syncwarp();                           // previous atom's readers are done
       if (live)
-        for (int e = gl; e < WS; e += GW) Dme[e] = __ldg(R + kTileM * (2 + L) + rs * WS + e);
+        for (int e = gl; e < WS; e += GW) Dme[e] = __ldg(R + rec_off_D(L) + rs * WS + e);
       __syncwarp();
     } else {
       rpow[0] = 1.f;
@@ -245,14 +263,145 @@ eaas_source_kernel(const __grid_constant__ EaasParams p) {
       wigner_build<L>(Q, Dme, gl, GW, [] { __syncwarp(); });
     }
     if (live) {
-      T* yr = y + (size_t)at * D * C + c0;
+      TO* yr = y + (size_t)at * D * C + c0;
       const float* swc = sw + c0;
       eaas_multi<L, CPL>(xv, Dme, rpow, p.tab, [&](int q, int k) { return swc[q * C + k]; },
-                         [&](int d, const float (&v)[CPL]) { ChanVec<T, CPL>::store(yr + d * C, v); });
+                         [&](int d, const float (&v)[CPL]) { ChanVec<TO, CPL>::store(yr + d * C, v); });
     }
   }
 }
-template <int L, typename T, bool PLANNED>
+// Planned source coupling staged by tiles, for shapes with one warp per atom
+// (C = 128 up to lmax 2).  A persistent CTA of kTileM warps takes the plan's tiles in
+// turn.  The tile record arrives by one bulk copy two tiles ahead and the
+// tile's 16 feature rows by 16 bulk copies one tile ahead (double-buffered),
+// so the loads stream while the previous tile is coupled; warp r couples
+// target slot r from shared memory (rotation and |r|^l from the record) and
+// writes its h' row straight to global memory.  Every wait is bounded.
+template <int L, typename T>
+struct TileSmem {
+  static constexpr int D = (L + 1) * (L + 1);
+  static constexpr int CPL = L >= 3 ? 2 : 4;
+  static constexpr int C = 32 * CPL;
+  static constexpr int ROWB = D * C * int(sizeof(T));
+  static constexpr int REC = plan_record_words(L);
+  static constexpr size_t rows = 0;                                       // [2][16][ROWB]
+  static constexpr size_t recs = rows + size_t(2) * kTileM * ROWB;        // [3][REC]
+  static constexpr size_t sw = recs + size_t(3) * REC * 4;                // [P][C]
+  static constexpr size_t bars = sw + size_t(num_paths(L)) * C * 4;       // rows [2], records [3]
+  static constexpr size_t total = bars + 5 * 8 + 16;
+  static_assert(ROWB % 16 == 0 && REC % 4 == 0 && bars % 8 == 0, "bulk-copy alignment");
+};
+
+template <int L, typename T>
+__global__ void __launch_bounds__(kTileM * 32, 1)
+eaas_tile_kernel(const __grid_constant__ EaasParams p) {
+  using Sm = TileSmem<L, T>;
+  constexpr int D = Sm::D, CPL = Sm::CPL, C = Sm::C, ROWB = Sm::ROWB, REC = Sm::REC;
+  constexpr int WS = wig_size(L);
+  constexpr int NP = num_paths(L);
+  extern __shared__ __align__(128) unsigned char smem[];
+  unsigned char* rows = smem + Sm::rows;
+  float* recs = reinterpret_cast<float*>(smem + Sm::recs);
+  float* sw = reinterpret_cast<float*>(smem + Sm::sw);
+  uint64_t* rowbar = reinterpret_cast<uint64_t*>(smem + Sm::bars);   // [2] a tile's rows
+  uint64_t* recbar = rowbar + 2;                                     // [3] a tile record
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(recbar + 3);
+
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int tiles = int(p.items / kTileM);
+  const int grid = gridDim.x;
+  if (blockIdx.x >= tiles) return;   // whole CTA
+  if (tid == 0) {
+    for (int b = 0; b < 5; ++b) mbar_init(smem_u32(rowbar + b), 1);
+    mbar_fence_init();
+    *abort_flag = 0;
+  }
+  for (int e = tid; e < NP * C; e += blockDim.x) sw[e] = __ldg(p.w + e);
+  __syncthreads();
+
+  const char* xb = static_cast<const char*>(p.x);
+  T* __restrict__ y = static_cast<T*>(p.y);
+  // thread 0: a tile's record into recs[b]
+  auto issue_rec = [&](int tl, int b) {
+    const uint32_t bar = smem_u32(recbar + b);
+    mbar_arrive_expect_tx(bar, REC * 4);
+    bulk_g2s(smem_u32(recs + b * REC), p.rec + (long long)tl * REC, REC * 4, bar);
+  };
+  // thread 0: the feature rows of a tile's targets into rows[b] (empty slots
+  // are not copied)
+  auto issue_rows = [&](const float* rec, int b) {
+    const int* tg = reinterpret_cast<const int*>(rec) + kRecTgt;
+    int valid = 0;
+    for (int r = 0; r < kTileM; ++r) valid += (unsigned)tg[r] < (unsigned)p.n;
+    const uint32_t bar = smem_u32(rowbar + b);
+    mbar_arrive_expect_tx(bar, uint32_t(valid) * ROWB);
+    for (int r = 0; r < kTileM; ++r)
+      if ((unsigned)tg[r] < (unsigned)p.n)
+        bulk_g2s(smem_u32(rows + (size_t(b) * kTileM + r) * ROWB), xb + (size_t)tg[r] * ROWB, ROWB,
+                 bar);
+  };
+
+  int tile = blockIdx.x;
+  if (tid == 0) {
+    issue_rec(tile, 0);
+    bounded_wait(smem_u32(recbar), 0u, kWaitPolls, abort_flag);
+    issue_rows(recs, 0);
+    if (tile + grid < tiles) issue_rec(tile + grid, 1);
+  }
+  int j = 0;   // this CTA's tile sequence number
+  for (; tile < tiles; ++j, tile += grid) {
+    const int rb = j % 3, wb = j & 1;
+    bounded_wait(smem_u32(recbar + rb), uint32_t(j / 3) & 1u, kWaitPolls, abort_flag);
+    bounded_wait(smem_u32(rowbar + wb), uint32_t(j >> 1) & 1u, kWaitPolls, abort_flag);
+    if (tid == 0 && tile + grid < tiles) {
+      // the next tile's rows (its record arrived a tile ago) and the record
+      // after it; both buffers were last read by tile j - 1, before the
+      // barrier that ended it
+      const int nb = (j + 1) % 3;
+      bounded_wait(smem_u32(recbar + nb), uint32_t((j + 1) / 3) & 1u, kWaitPolls, abort_flag);
+      issue_rows(recs + nb * REC, (j + 1) & 1);
+      if (tile + 2 * grid < tiles) issue_rec(tile + 2 * grid, (j + 2) % 3);
+    }
+    const float* rec = recs + rb * REC;
+    const int at = reinterpret_cast<const int*>(rec)[kRecTgt + w];
+    if ((unsigned)at < (unsigned)p.n) {
+      const T* xr = reinterpret_cast<const T*>(rows + (size_t(wb) * kTileM + w) * ROWB) + lane * CPL;
+      float xv[CPL][D];
+#pragma unroll
+      for (int d = 0; d < D; ++d) {
+        float v[CPL];
+        ChanVec<T, CPL>::load_shared(xr + d * C, v);
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) xv[k][d] = v[k];
+      }
+      float rpow[L + 1];
+#pragma unroll
+      for (int l = 0; l <= L; ++l) rpow[l] = rec[kRecRp + w * (L + 1) + l];
+      T* yr = y + (size_t)at * D * C + lane * CPL;
+      const float* swc = sw + lane * CPL;
+      eaas_multi<L, CPL>(xv, rec + rec_off_D(L) + w * WS, rpow, p.tab,
+                         [&](int q, int k) { return swc[q * C + k]; },
+                         [&](int d, const float (&v)[CPL]) { ChanVec<T, CPL>::store(yr + d * C, v); });
+    }
+    __syncthreads();   // rows[wb] and recs[rb] are refilled one and two tiles ahead
+  }
+  if (*abort_flag && tid == 0) {
+    // a wait gave up: give every barrier's last phase a short, bounded chance
+    // to complete before the CTA's shared memory is released
+    volatile int none = 0;
+    for (int b = 0; b < 2; ++b) {
+      const int last = j - 1 - ((j - 1 - b) & 1);   // last tile sequence number with j % 2 == b
+      if (last >= 0) bounded_wait(smem_u32(rowbar + b), uint32_t(last >> 1) & 1u, kDrainPolls, &none);
+    }
+    for (int b = 0; b < 3; ++b) {
+      int last = j - 1;
+      while (last >= 0 && last % 3 != b) --last;
+      if (last >= 0) bounded_wait(smem_u32(recbar + b), uint32_t(last / 3) & 1u, kDrainPolls, &none);
+    }
+  }
+}
+
+template <int L, typename T, bool PLANNED, typename TO = T>
 int launch_eaas_t(const egat_shape& s, const void* d_x, const float* d_pos, const float* rec,
                   long long items, const float* d_w, void* d_y, cudaStream_t st) {
   EaasParams p;
@@ -276,7 +425,7 @@ int launch_eaas_t(const egat_shape& s, const void* d_x, const float* d_pos, cons
   const long long want = (groups * WPA + kEaasWarps - 1) / kEaasWarps;
   const int grid = int(std::max<long long>(1, std::min<long long>(want, (long long)sms * 8)));
   const size_t shmem = size_t(num_paths(L)) * s.C * sizeof(float);
-  eaas_source_kernel<L, T, PLANNED><<<grid, kEaasWarps * 32, shmem, st>>>(p);
+  eaas_source_kernel<L, T, PLANNED, TO><<<grid, kEaasWarps * 32, shmem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
 }
 
@@ -297,11 +446,60 @@ int launch_eaas_source(const egat_shape& s, const void* d_x, const float* d_pos,
   }
 }
 
+template <int L, typename T>
+int launch_eaas_tile(const egat_shape& s, const void* d_x, const float* rec, long long items,
+                     const float* d_w, void* d_y, cudaStream_t st) {
+  EaasParams p;
+  p.x = d_x;
+  p.pos = nullptr;
+  p.w = d_w;
+  p.y = d_y;
+  p.n = s.n;
+  p.C = s.C;
+  p.rec = rec;
+  p.items = items;
+  p.tab = eaas_table(L);
+  constexpr size_t shmem = TileSmem<L, T>::total;
+  auto kern = eaas_tile_kernel<L, T>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(shmem)) !=
+      cudaSuccess)
+    return EGAT_ERR_CUDA;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int tiles = int(items / kTileM);
+  const int grid = tiles < sms ? tiles : sms;
+  kern<<<grid, kTileM * 32, shmem, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
+}
+
+int launch_eaas_source_f32out(const egat_shape& s, const void* d_x, const float* d_pos,
+                              const float* d_w, float* d_y, cudaStream_t st) {
+  const bool bf = s.dtype == EGAT_BF16;
+  const long long n = s.n;
+  switch (s.lmax) {
+    case 1: return bf ? launch_eaas_t<1, __nv_bfloat16, false, float>(s, d_x, d_pos, nullptr, n, d_w, d_y, st)
+                      : launch_eaas_t<1, float, false>(s, d_x, d_pos, nullptr, n, d_w, d_y, st);
+    case 2: return bf ? launch_eaas_t<2, __nv_bfloat16, false, float>(s, d_x, d_pos, nullptr, n, d_w, d_y, st)
+                      : launch_eaas_t<2, float, false>(s, d_x, d_pos, nullptr, n, d_w, d_y, st);
+    case 3: return bf ? launch_eaas_t<3, __nv_bfloat16, false, float>(s, d_x, d_pos, nullptr, n, d_w, d_y, st)
+                      : launch_eaas_t<3, float, false>(s, d_x, d_pos, nullptr, n, d_w, d_y, st);
+    default: return EGAT_ERR_UNSUPPORTED;
+  }
+}
+
 int launch_eaas_planned(const egat_shape& s, const void* d_x, const void* d_plan, const float* d_w,
                         void* d_y, cudaStream_t st) {
   const bool bf = s.dtype == EGAT_BF16;
   const PlanView pv = plan_view(const_cast<void*>(d_plan), s.n, s.K, s.lmax);
   const long long items = (long long)pv.tiles * kTileM;
+  // one warp per atom: the tile-staged kernel
+  if (s.lmax <= 2 && s.C == 128) {
+    if (s.lmax == 1) return bf ? launch_eaas_tile<1, __nv_bfloat16>(s, d_x, pv.rec, items, d_w, d_y, st)
+                               : launch_eaas_tile<1, float>(s, d_x, pv.rec, items, d_w, d_y, st);
+    return bf ? launch_eaas_tile<2, __nv_bfloat16>(s, d_x, pv.rec, items, d_w, d_y, st)
+              : launch_eaas_tile<2, float>(s, d_x, pv.rec, items, d_w, d_y, st);
+  }
   switch (s.lmax) {
     case 1: return bf ? launch_eaas_t<1, __nv_bfloat16, true>(s, d_x, nullptr, pv.rec, items, d_w, d_y, st)
                       : launch_eaas_t<1, float, true>(s, d_x, nullptr, pv.rec, items, d_w, d_y, st);
@@ -311,6 +509,10 @@ int launch_eaas_planned(const egat_shape& s, const void* d_x, const void* d_plan
                       : launch_eaas_t<3, float, true>(s, d_x, nullptr, pv.rec, items, d_w, d_y, st);
     default: return EGAT_ERR_UNSUPPORTED;
   }
+}
+
+int take_wait_timeouts_coupling(cudaStream_t st, unsigned int* count) {
+  return take_unit_wait_timeouts(st, count) == 0 ? EGAT_OK : EGAT_ERR_CUDA;
 }
 
 }  // namespace egat

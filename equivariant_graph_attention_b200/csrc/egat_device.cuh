@@ -415,6 +415,65 @@ __device__ __forceinline__ void eaas_channel(float (&x)[(L + 1) * (L + 1)],
   });
 }
 
+// The transpose of eaas_channel for fixed r and weights (the adjoint used by
+// the backward pass): the coupling is y = D Rw D^T x with Rw the weighted
+// axis-frame re-index, so its transpose is D Rw^T D^T g — the same rotations
+// around the re-index read backwards (output degree lo -> input degree li).
+// g is overwritten; out(d, v) receives component d of the result.
+template <int L, typename WFn, typename OutFn>
+__device__ __forceinline__ void eaas_channel_adjoint(float (&g)[(L + 1) * (L + 1)],
+                                                     const float* __restrict__ Dsm,
+                                                     const float (&rpow)[L + 1],
+                                                     const EaasTable& tab, WFn wgt, OutFn out) {
+  constexpr int D = (L + 1) * (L + 1);
+  float t[D];
+#pragma unroll
+  for (int i = 0; i < D; ++i) t[i] = 0.f;
+  static_for<1, L + 1>([&](auto lc) {
+    constexpr int l = decltype(lc)::value;
+    constexpr int w = 2 * l + 1;
+    const float* Dl = Dsm + wig_off(l);
+    float tmp[w];
+#pragma unroll
+    for (int a = 0; a < w; ++a) {
+      float s = 0.f;
+#pragma unroll
+      for (int b = 0; b < w; ++b) s = fmaf(Dl[b * w + a], g[l * l + b], s);
+      tmp[a] = s;
+    }
+#pragma unroll
+    for (int a = 0; a < w; ++a) g[l * l + a] = tmp[a];
+  });
+  static_for<0, num_paths(L)>([&](auto pc) {
+    constexpr int p = decltype(pc)::value;
+    constexpr int li = path_info(L, p, 0);
+    constexpr int lf = path_info(L, p, 1);
+    constexpr int lo = path_info(L, p, 2);
+    constexpr bool even = ((li + lf + lo) % 2) == 0;
+    const float wp = wgt(p) * rpow[lf];
+#pragma unroll
+    for (int mo = -lo; mo <= lo; ++mo) {
+      const int src = even ? mo : -mo;
+      const bool live = (iabs(mo) <= li) && (even || mo != 0);
+      if (live) t[li * li + li + src] = fmaf(wp * tab.f[p][mo + lo], g[lo * lo + lo + mo],
+                                             t[li * li + li + src]);
+    }
+  });
+  out(0, t[0]);
+  static_for<1, L + 1>([&](auto lc) {
+    constexpr int l = decltype(lc)::value;
+    constexpr int w = 2 * l + 1;
+    const float* Dl = Dsm + wig_off(l);
+#pragma unroll
+    for (int a = 0; a < w; ++a) {
+      float s = 0.f;
+#pragma unroll
+      for (int b = 0; b < w; ++b) s = fmaf(Dl[a * w + b], t[l * l + b], s);
+      out(l * l + a, s);
+    }
+  });
+}
+
 // The same operator on NCH channels at once (channels of one atom share the
 // Wigner-D matrices): each matrix entry is read once and applied to every
 // channel.  x[k][d] is overwritten; wgt(p, k) returns w[p] of channel k;

@@ -55,14 +55,17 @@ struct PlanView {
   int cap;          // union capacity per tile (power of two >= kTileM * K)
   int tiles;
 };
-// Tile record: int32 target[kTileM] (-1 past n), float rpow[kTileM][lmax+1]
-// (|r|^0..|r|^lmax), float D[kTileM][wig_size(lmax)] (real Wigner-D of the
-// alignment rotation, degrees 0..lmax) — everything the attention epilogue
-// needs per target, so the attention kernel builds nothing per tile.
-inline int plan_record_words(int lmax) {
-  const int ws = (lmax + 1) * (2 * lmax + 1) * (2 * lmax + 3) / 3;   // sum of (2l+1)^2
-  return kTileM * (1 + (lmax + 1) + ws);
-}
+// Tile record (words): a header (union length, three zeros), int32
+// target[kTileM] (-1 past n), float rpow[kTileM][lmax+1] (|r|^0..|r|^lmax),
+// float D[kTileM][wig] (real Wigner-D of the alignment rotation, degrees
+// 0..lmax, wig = sum of (2l+1)^2) — everything the attention kernel needs per
+// tile besides the union itself, so it builds nothing per tile.
+constexpr int kRecHdr = 4;
+constexpr int rec_wig_size(int lmax) { return (lmax + 1) * (2 * lmax + 1) * (2 * lmax + 3) / 3; }
+constexpr int kRecTgt = kRecHdr;
+constexpr int kRecRp = kRecHdr + kTileM;
+constexpr int rec_off_D(int lmax) { return kRecHdr + kTileM * (2 + lmax); }
+constexpr int plan_record_words(int lmax) { return rec_off_D(lmax) + kTileM * rec_wig_size(lmax); }
 int plan_capacity(int K);
 // shared memory of the plan kernel: two bitmap-sized arrays over all atoms and
 // one tile mask; the tensor-core path is used while this fits a CTA
@@ -72,15 +75,27 @@ size_t plan_bytes(int n, int K, int lmax);
 PlanView plan_view(void* base, int n, int K, int lmax);
 int launch_build_plan(int n, int K, int lmax, const int32_t* d_nbr, const int32_t* d_cnt,
                       const int32_t* d_order, const float* d_pos, void* d_plan, cudaStream_t st);
+// Step 2 with a float32 result whatever the storage type (the backward pass
+// keeps its intermediates in float32).
+int launch_eaas_source_f32out(const egat_shape& s, const void* d_x, const float* d_pos,
+                              const float* d_w, float* d_y, cudaStream_t st);
 // Step 2 for every atom listed in a plan's tile records, rotations from them.
 int launch_eaas_planned(const egat_shape& s, const void* d_x, const void* d_plan, const float* d_w,
                         void* d_y, cudaStream_t st);
 // Tiled tensor-core attention (bf16 storage, C/H = 8, dk = 16): fused = true
 // applies the target coupling and writes ^h; false writes m.
 bool tc_attention_supported(const egat_shape& s);
-// Bounded-wait report of the tensor-core kernel: read and clear the count of
-// waits that gave up (synchronises st); the self-test launch.
-int take_wait_timeouts(cudaStream_t st, unsigned int* count);
+// Backward pass (gradients of <G, ^h> with respect to h, q, k): workspace and launch.
+size_t backward_ws_bytes(const egat_shape& s);
+int launch_backward(const egat_shape& s, const void* d_h, const float* d_pos, const void* d_q,
+                    const void* d_k, const int32_t* d_nbr, const int32_t* d_cnt, const float* d_w1,
+                    const float* d_w2, const float* d_g, void* d_ws, float* d_dh, float* d_dq,
+                    float* d_dk, cudaStream_t st);
+// Bounded-wait reports (one per compilation unit with mbarrier waits): read
+// and clear the count of waits that gave up (synchronises st); the self-test
+// launch.
+int take_wait_timeouts_attention(cudaStream_t st, unsigned int* count);
+int take_wait_timeouts_coupling(cudaStream_t st, unsigned int* count);
 int launch_wait_timeout_selftest(int polls, cudaStream_t st);
 int launch_attention_tc(const egat_shape& s, bool fused, const void* d_q, const void* d_k,
                         const void* d_hp, const void* d_plan, const float* d_w2, float* d_out,

@@ -235,7 +235,15 @@ struct Search {
   int bits;
   long long rc2;
   int key_shift;
+  int cq;          // cell edge (grid units)
 };
+
+// Distance along one axis from coordinate v to the cell c of edge cq, whose
+// points have coordinates c*cq .. c*cq + cq - 1 (0 when v lies in it).
+__device__ __forceinline__ long long axis_gap(int v, int c, int cq) {
+  const long long lo = (long long)c * cq, hi = lo + cq - 1;
+  return v < lo ? lo - v : (v > hi ? v - hi : 0);
+}
 
 // Cells have edge ceil(r_c / 2), so every neighbour lies in the 5 x 5 x 5
 // block of cells around the atom's cell.
@@ -260,9 +268,14 @@ __device__ __forceinline__ void for_each_neighbour_rounds(const Search& s, int4 
       cx = c.x + l % kWidth - kSpan;
       cy = c.y + (l / kWidth) % kWidth - kSpan;
       cz = c.z + l / (kWidth * kWidth) - kSpan;
-      const int b = bucket_of(cx, cy, cz, s.bits);
-      beg = s.bucket_start[b];
-      len = s.bucket_start[b + 1] - beg;
+      // a cell whose box lies beyond the cutoff from p holds no neighbour
+      const long long gx = axis_gap(p.x, cx, s.cq), gy = axis_gap(p.y, cy, s.cq),
+                      gz = axis_gap(p.z, cz, s.cq);
+      if (gx * gx + gy * gy + gz * gz <= s.rc2) {
+        const int b = bucket_of(cx, cy, cz, s.bits);
+        beg = s.bucket_start[b];
+        len = s.bucket_start[b + 1] - beg;
+      }
     }
     int inc = len;
 #pragma unroll
@@ -510,7 +523,7 @@ int build_graph(const int32_t* d_pos_q, int n, int cutoff_q, int K, int mode,
   if (launch_scan(w.bucket_cnt, M, w.partial, w.bucket_start, st) != EGAT_OK) return EGAT_ERR_CUDA;
   scatter_atoms<<<nb, tb, 0, st>>>(d_pos_q, n, w.cell, w.bucket_start, w.cursor, w.tpos);
   rank_in_bucket<<<nb, tb, 0, st>>>(n, w.cell, w.bucket_start, w.tpos, w.spos, w.scell, d_order);
-  Search s{w.spos, w.scell, w.bucket_start, bits, (long long)cutoff_q * cutoff_q, key_shift};
+  Search s{w.spos, w.scell, w.bucket_start, bits, (long long)cutoff_q * cutoff_q, key_shift, cell_q};
   const unsigned nfill = unsigned((n + kFillWarps - 1) / kFillWarps);
   if (mode == EGAT_GRAPH_PADDED) {
     if (cudaMemsetAsync(w.trunc, 0, sizeof(int), st) != cudaSuccess) return EGAT_ERR_CUDA;

@@ -49,47 +49,41 @@ __global__ void __launch_bounds__(kPlanThreads) build_plan_kernel(const __grid_c
   uint32_t* bitmap = sm;                          // [nw]
   uint32_t* prefix = sm + nw;                     // [nw]
   uint32_t* mask = sm + 2 * nw;                   // [kTileM][words]
-  __shared__ int tgt[kTileM], off[kTileM + 1];
+  __shared__ int tgt[kTileM], rowcnt[kTileM];
   __shared__ int warp_sum[kPlanThreads / 32];
   __shared__ int s_unique;
   const int tile = blockIdx.x;
 
+  // the tile's targets and their neighbour counts (0 for an empty slot)
   if (threadIdx.x < kTileM) {
     const long long slot = (long long)tile * kTileM + threadIdx.x;
     int t = -1;
     if (slot < p.n) t = p.order ? p.order[slot] : int(slot);
     if ((unsigned)t >= (unsigned)p.n) t = -1;
+    int c = 0;
+    if (t >= 0) {
+      c = p.cnt ? p.cnt[t] : p.K;
+      c = c < 0 ? 0 : (c > p.K ? p.K : c);
+    }
     tgt[threadIdx.x] = t;
+    rowcnt[threadIdx.x] = c;
   }
   for (int i = threadIdx.x; i < nw; i += blockDim.x) bitmap[i] = 0u;
   for (int i = threadIdx.x; i < kTileM * words; i += blockDim.x) mask[i] = 0u;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int sum = 0;
+  // visit every (target row, neighbour) entry of the tile: rows in turn,
+  // the row's entries spread over the threads (coalesced loads of nbr)
+  auto for_each_entry = [&](auto&& f) {
     for (int r = 0; r < kTileM; ++r) {
-      off[r] = sum;
-      int c = 0;
-      if (tgt[r] >= 0) {
-        c = p.cnt ? p.cnt[tgt[r]] : p.K;
-        c = c < 0 ? 0 : (c > p.K ? p.K : c);
-      }
-      sum += c;
+      const int c = rowcnt[r];
+      const int32_t* row = p.nbr + (long long)(tgt[r] < 0 ? 0 : tgt[r]) * p.K;
+      for (int e = threadIdx.x; e < c; e += blockDim.x) f(r, row[e]);
     }
-    off[kTileM] = sum;
-  }
-  __syncthreads();
-  const int total = off[kTileM];
-  auto entry = [&](int e, int& r) {
-    r = 0;
-    while (r + 1 < kTileM && off[r + 1] <= e) ++r;
-    return p.nbr[(long long)tgt[r] * p.K + (e - off[r])];
   };
   // 1. bitmap of the union
-  for (int e = threadIdx.x; e < total; e += blockDim.x) {
-    int r;
-    const int j = entry(e, r);
+  for_each_entry([&](int, int j) {
     if ((unsigned)j < (unsigned)p.n) atomicOr(&bitmap[j >> 5], 1u << (j & 31));
-  }
+  });
   __syncthreads();
   // 2. per-word exclusive prefix counts (contiguous chunk per thread + block scan)
   const int per = (nw + kPlanThreads - 1) / kPlanThreads;
@@ -138,13 +132,11 @@ __global__ void __launch_bounds__(kPlanThreads) build_plan_kernel(const __grid_c
   for (int e = U + threadIdx.x; e < upad; e += blockDim.x) uni[e] = filler;
   if (threadIdx.x == 0) pv.ulen[tile] = U;
   // 3. membership bits
-  for (int e = threadIdx.x; e < total; e += blockDim.x) {
-    int r;
-    const int j = entry(e, r);
-    if ((unsigned)j >= (unsigned)p.n) continue;
+  for_each_entry([&](int r, int j) {
+    if ((unsigned)j >= (unsigned)p.n) return;
     const int pos = int(prefix[j >> 5]) + __popc(bitmap[j >> 5] & ((1u << (j & 31)) - 1u));
     atomicOr(&mask[r * words + (pos >> 5)], 1u << (pos & 31));
-  }
+  });
   __syncthreads();
   // word-major in memory: the kTileM words of one 32-atom chunk are contiguous
   uint32_t* gmask = pv.mask + (long long)tile * words * kTileM;
@@ -161,10 +153,11 @@ __global__ void __launch_bounds__(kPlanThreads) build_plan_kernel(const __grid_c
 constexpr int kRecThreads = 128;
 template <int L>
 __global__ void __launch_bounds__(kRecThreads)
-tile_records_kernel(const int32_t* __restrict__ order, const float* __restrict__ pos, int n,
-                    int tiles, float* __restrict__ rec) {
+tile_records_kernel(const int32_t* __restrict__ order, const float* __restrict__ pos,
+                    const int* __restrict__ ulen, int n, int tiles, float* __restrict__ rec) {
   constexpr int WS = wig_size(L);
-  constexpr int REC = kTileM * (1 + (L + 1) + WS);
+  constexpr int REC = plan_record_words(L);
+  static_assert(WS == rec_wig_size(L) && REC % 4 == 0, "record layout");
   const long long slot = (long long)blockIdx.x * kRecThreads + threadIdx.x;
   if (slot >= (long long)tiles * kTileM) return;
   const int tile = int(slot / kTileM), r = int(slot % kTileM);
@@ -179,14 +172,15 @@ tile_records_kernel(const int32_t* __restrict__ order, const float* __restrict__
   wigner_regs<L>(Q, D);
   float* R = rec + (long long)tile * REC;
 #pragma unroll
-  for (int e = 0; e < WS; ++e) R[kTileM * (2 + L) + r * WS + e] = D[e];
-  reinterpret_cast<int*>(R)[r] = tg;
+  for (int e = 0; e < WS; ++e) R[rec_off_D(L) + r * WS + e] = D[e];
+  reinterpret_cast<int*>(R)[kRecTgt + r] = tg;
   float a = 1.f;
 #pragma unroll
   for (int l = 0; l <= L; ++l) {
-    R[kTileM + r * (L + 1) + l] = a;
+    R[kRecRp + r * (L + 1) + l] = a;
     a *= rr;
   }
+  if (r < kRecHdr) reinterpret_cast<int*>(R)[r] = r == 0 ? ulen[tile] : 0;
 }
 
 }  // namespace
@@ -250,9 +244,9 @@ int launch_build_plan(int n, int K, int lmax, const int32_t* d_nbr, const int32_
   const int tiles = p.plan.tiles;
   const int blocks = (tiles * kTileM + kRecThreads - 1) / kRecThreads;
   switch (lmax) {
-    case 1: tile_records_kernel<1><<<blocks, kRecThreads, 0, st>>>(d_order, d_pos, n, tiles, p.plan.rec); break;
-    case 2: tile_records_kernel<2><<<blocks, kRecThreads, 0, st>>>(d_order, d_pos, n, tiles, p.plan.rec); break;
-    case 3: tile_records_kernel<3><<<blocks, kRecThreads, 0, st>>>(d_order, d_pos, n, tiles, p.plan.rec); break;
+    case 1: tile_records_kernel<1><<<blocks, kRecThreads, 0, st>>>(d_order, d_pos, p.plan.ulen, n, tiles, p.plan.rec); break;
+    case 2: tile_records_kernel<2><<<blocks, kRecThreads, 0, st>>>(d_order, d_pos, p.plan.ulen, n, tiles, p.plan.rec); break;
+    case 3: tile_records_kernel<3><<<blocks, kRecThreads, 0, st>>>(d_order, d_pos, p.plan.ulen, n, tiles, p.plan.rec); break;
     default: return EGAT_ERR_UNSUPPORTED;
   }
   return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;

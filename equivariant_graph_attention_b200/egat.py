@@ -40,7 +40,8 @@ EXPORTS = ["egat_version", "egat_strerror", "egat_num_paths", "egat_graph_worksp
            "egat_otf_attention_coupled",
            "egat_forward_workspace_bytes", "egat_forward", "egat_forward_noalloc",
            "egat_attention_plan_bytes", "egat_build_attention_plan", "egat_otf_attention_tiled",
-           "egat_eaas_couple_planned", "egat_take_device_status", "egat_selftest_wait_timeout"]
+           "egat_eaas_couple_planned", "egat_take_device_status", "egat_selftest_wait_timeout",
+           "egat_backward_workspace_bytes", "egat_backward"]
 
 
 class EgatError(RuntimeError):
@@ -95,6 +96,10 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.egat_attention_plan_bytes.argtypes = [sp, ctypes.POINTER(sz)]
     lib.egat_build_attention_plan.restype = ctypes.c_int
     lib.egat_build_attention_plan.argtypes = [sp, vp, vp, vp, vp, vp, sz, vp]
+    lib.egat_backward_workspace_bytes.restype = ctypes.c_int
+    lib.egat_backward_workspace_bytes.argtypes = [sp, ctypes.POINTER(sz)]
+    lib.egat_backward.restype = ctypes.c_int
+    lib.egat_backward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp, vp, vp]
     lib.egat_take_device_status.restype = ctypes.c_int
     lib.egat_take_device_status.argtypes = [vp]
     lib.egat_selftest_wait_timeout.restype = ctypes.c_int
@@ -287,6 +292,35 @@ def egat_build_attention_plan(shape: Shape, nbr: torch.Tensor, cnt: Optional[tor
                                                   plan.numel(), _stream(stream))
     _check("egat_build_attention_plan", rc)
     return plan
+
+
+def egat_backward_workspace_bytes(shape: Shape) -> int:
+    out = ctypes.c_size_t(0)
+    cs = shape.c()
+    _check("egat_backward_workspace_bytes",
+           load_library().egat_backward_workspace_bytes(ctypes.byref(cs), ctypes.byref(out)))
+    return out.value
+
+
+def egat_backward(shape: Shape, h: torch.Tensor, pos: torch.Tensor, q: torch.Tensor,
+                  k: torch.Tensor, nbr: torch.Tensor, cnt: Optional[torch.Tensor],
+                  w1: torch.Tensor, w2: torch.Tensor, grad_out: torch.Tensor,
+                  workspace: Optional[torch.Tensor] = None, stream=None):
+    """(dL/dh, dL/dq, dL/dk) float32 for the upstream gradient grad_out = dL/d^h."""
+    nb = egat_backward_workspace_bytes(shape)
+    if workspace is None:
+        workspace = torch.empty(max(nb, 16), dtype=torch.uint8, device=h.device)
+    dev = h.device
+    dh = torch.empty((shape.n, shape.D, shape.C), dtype=torch.float32, device=dev)
+    dq = torch.empty((shape.n, shape.H, shape.dk), dtype=torch.float32, device=dev)
+    dk = torch.empty((shape.n, shape.H, shape.dk), dtype=torch.float32, device=dev)
+    cs = shape.c()
+    rc = load_library().egat_backward(
+        ctypes.byref(cs), _ptr(h), _ptr(pos), _ptr(q), _ptr(k), _ptr(nbr), _ptr(cnt), _ptr(w1),
+        _ptr(w2), _ptr(grad_out), _ptr(workspace), workspace.numel(), _ptr(dh), _ptr(dq), _ptr(dk),
+        _stream(stream))
+    _check("egat_backward", rc)
+    return dh, dq, dk
 
 
 def egat_take_device_status(stream=None) -> int:

@@ -275,6 +275,30 @@ EGAT_API int egat_forward_noalloc(const egat_shape* s, const void* d_h, const fl
                                   float* d_out, void* stream);
 
 /*
+ * Backward pass of steps 2-4 (the step after the forward: forces and training
+ * need gradients; [EX] §3.2 keeps per-edge quantities off HBM, and so does
+ * this pass: every attention weight is recomputed from q, k and one
+ * log-sum-exp per target and head).  For an upstream gradient
+ * G = dL/d^h (float32 [n][D][C]) of the forward egat_forward computes on the
+ * padded graph (d_nbr, d_cnt; d_cnt may be NULL), writes
+ *  d_dh  float32 [n][D][C]   dL/dh
+ *  d_dq  float32 [n][H][dk]  dL/dq
+ *  d_dk  float32 [n][H][dk]  dL/dk
+ * (gradients with respect to positions and weights are not computed).  The
+ * in-lists (targets served by each atom) are built and sorted inside, so
+ * every gradient is a gather in a fixed order: deterministic, no atomics on
+ * results.  Padded graphs only (CSR returns EGAT_ERR_UNSUPPORTED), n * K below
+ * 2^31; d_ws at least egat_backward_workspace_bytes(s) (h', dL/dm in the
+ * storage type, in-lists, per-target statistics).
+ */
+EGAT_API int egat_backward_workspace_bytes(const egat_shape* s, size_t* bytes);
+EGAT_API int egat_backward(const egat_shape* s, const void* d_h, const float* d_pos, const void* d_q,
+                           const void* d_k, const int32_t* d_nbr, const int32_t* d_cnt,
+                           const float* d_w1, const float* d_w2, const float* d_grad_out,
+                           void* d_ws, size_t ws_bytes, float* d_dh, float* d_dq, float* d_dk,
+                           void* stream);
+
+/*
  * Device status.  The tensor-core attention kernel waits on mbarriers for its
  * bulk copies; every such wait is bounded (about a second).  A wait that
  * gives up is counted on the device, the kernel stops waiting and finishes

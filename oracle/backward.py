@@ -1,0 +1,95 @@
+"""Backward pass of the oracle's forward (``attention.forward``).  Test
+infrastructure only.
+
+The pages name the backward pass as the step after the forward: the
+Conservative mode takes forces as gradients of the energy, and the streaming
+attention is recomputed rather than storing the attention weights
+([EX] §3.2 on linear activation memory; [TS] §2.2).  This module writes out
+the gradients of a scalar loss L = sum_i <G_i, ^h_i> (G the upstream
+gradient) with respect to the features h, queries q and keys k, each step as
+the plain adjoint of the corresponding forward step:
+
+1. target coupling  ^h_i = T(m_i; r_i, w2) is linear in m_i, so
+   dL/dm_i = T^*(G_i; r_i, w2), the transpose of the same dense contraction;
+2. aggregation m_i = sum_j alpha_ij h'_j over the head of each channel:
+   dL/dh'_j   += alpha_ij dL/dm_i                (over the targets i of j),
+   dalpha_ij  = sum over the head's channels and components of
+                dL/dm_i * h'_j,
+   ds_ij      = alpha_ij (dalpha_ij - sum_j' alpha_ij' dalpha_ij')
+                (softmax Jacobian),
+   dL/dq_i    = sum_j ds_ij k_j / sqrt(d_k),
+   dL/dk_j   += ds_ij q_i / sqrt(d_k);
+3. source coupling h'_j = T(h_j; r_j, w1): dL/dh_j = T^*(dL/dh'_j; r_j, w1).
+
+Gradients with respect to positions and weights are not computed here.
+Layouts as in ``attention``; every atom is a target (nbrs[i] = N(i)).
+"""
+from __future__ import annotations
+
+from typing import Sequence, Tuple
+
+import numpy as np
+
+from . import so3
+from .attention import _block, head_of_channel, logits, softmax_two_pass, source_coupling
+
+
+def tensor_product_adjoint(g: np.ndarray, pos: np.ndarray, w: np.ndarray, lmax: int) -> np.ndarray:
+    """The transpose of ``attention.tensor_product`` as a linear map x -> y for
+    fixed positions and weights:
+
+        x^{li}[mi][c] = sum_{p=(li,lf,lo)} w[p][c] sum_{m,mf} T_p[m,mi,mf] g^{lo}[m][c] R^{lf}_{mf}(r).
+
+    g [N, D, C]; pos [N, 3]; w [P, C].  Returns [N, D, C] float64.
+    """
+    g = np.asarray(g, dtype=np.float64)
+    pos = np.asarray(pos, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    plist = so3.paths(lmax)
+    assert w.shape[0] == len(plist)
+    R = [so3.solid_harmonics(l, pos) for l in range(lmax + 1)]
+    x = np.zeros_like(g)
+    for p, (li, lf, lo) in enumerate(plist):
+        T = so3.real_cg(li, lf, lo)
+        contrib = np.einsum("oif,noc,nf->nic", T, _block(g, lo), R[lf])
+        x[:, li * li:(li + 1) * (li + 1), :] += contrib * w[p][None, None, :]
+    return x
+
+
+def attention_backward(q, k, hp, dm, nbrs: Sequence[np.ndarray]) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Step 2's adjoint: given dL/dm for every target, returns (dL/dh', dL/dq, dL/dk)."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    hp = np.asarray(hp, dtype=np.float64)
+    dm = np.asarray(dm, dtype=np.float64)
+    N, D, C = hp.shape
+    H, dk_ = q.shape[1], q.shape[2]
+    hc = head_of_channel(C, H)
+    member = np.zeros((C, H))
+    member[np.arange(C), hc] = 1.0                  # channel -> head
+    scale = 1.0 / np.sqrt(dk_)
+    dhp = np.zeros_like(hp)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    for i, js in enumerate(nbrs):
+        js = np.asarray(js, dtype=np.int64)
+        if js.size == 0:
+            continue
+        a = softmax_two_pass(logits(q[i], k[js]))            # [J, H]
+        da = np.einsum("dc,jdc->jc", dm[i], hp[js]) @ member   # [J, H]
+        ds = a * (da - (a * da).sum(axis=0, keepdims=True))
+        dq[i] += np.einsum("jh,jhd->hd", ds, k[js]) * scale
+        np.add.at(dk, js, np.einsum("jh,hd->jhd", ds, q[i]) * scale)
+        np.add.at(dhp, js, np.einsum("jc,dc->jdc", a[:, hc], dm[i]))
+    return dhp, dq, dk
+
+
+def backward(h, pos, q, k, w1, w2, lmax: int, nbrs: Sequence[np.ndarray],
+             G) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """(dL/dh, dL/dq, dL/dk) for L = sum_i <G_i, ^h_i>, ^h = attention.forward."""
+    pos = np.asarray(pos, dtype=np.float64)
+    hp = source_coupling(h, pos, w1, lmax)
+    dm = tensor_product_adjoint(G, pos, w2, lmax)
+    dhp, dq, dk = attention_backward(q, k, hp, dm, nbrs)
+    dh = tensor_product_adjoint(dhp, pos, w1, lmax)
+    return dh, dq, dk

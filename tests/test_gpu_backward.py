@@ -1,0 +1,104 @@
+"""GPU parity of the backward pass (egat_backward) against the oracle's
+backward (oracle/backward.py), which finite differences of the oracle forward
+pin (tests/test_oracle_backward.py).
+
+dL/dh is compared block by block (the forward's metric); dL/dq and dL/dk row
+by row over (atom, head) with the same relative-norm metric.  Bars as for the
+forward: 1e-4 for float32 storage, 2e-2 for bf16 storage (h' and dL/dm are
+held in bf16 there).  Also: tiny ragged systems with an isolated atom and an
+atom at the origin, and bitwise determinism across calls.
+"""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+from oracle.backward import backward as oracle_backward
+from oracle.graph import radius_graph
+from equivariant_graph_attention_b200 import synth
+from tests.parity_util import TOL, block_rel_error, device_inputs, shape_of
+
+pytestmark = pytest.mark.gpu
+
+SMALL = ["uniform64_l1_f32", "water216_l2_f32", "uniform4096_l2_bf16"]
+
+
+def _egat():
+    from equivariant_graph_attention_b200 import egat
+    return egat
+
+
+def row_rel_error(gpu: np.ndarray, ref: np.ndarray) -> float:
+    """max over (atom, head) rows of ||gpu - ref|| / ||ref|| (zero rows must match exactly)."""
+    g = np.asarray(gpu, dtype=np.float64).reshape(-1, gpu.shape[-1])
+    r = np.asarray(ref, dtype=np.float64).reshape(-1, ref.shape[-1])
+    nr = np.linalg.norm(r, axis=1)
+    ne = np.linalg.norm(g - r, axis=1)
+    zero = nr == 0.0
+    assert np.all(ne[zero] <= 1e-30), "nonzero gradient where the reference is exactly zero"
+    return float(np.max(ne[~zero] / nr[~zero])) if np.any(~zero) else 0.0
+
+
+@functools.lru_cache(maxsize=None)
+def _case(name):
+    wl = synth.WORKLOADS[name]
+    d = synth.make(wl)
+    G = np.random.default_rng(17).standard_normal((wl.n, wl.D, wl.C)).astype(np.float32)
+    lists, _ = radius_graph(d["pos_q"], wl.cutoff_q, K=wl.K)
+    ref = oracle_backward(d["h"], d["pos"], d["q"], d["k"], d["w1"], d["w2"], wl.lmax, lists, G)
+    return wl, d, G, ref
+
+
+def _run(wl, d, G):
+    egat = _egat()
+    dev = device_inputs(wl, d)
+    g = egat.egat_build_graph(dev["pos_q"], wl.cutoff_q, K=wl.K)
+    Gd = torch.from_numpy(G).cuda()
+    return egat.egat_backward(shape_of(wl), dev["h"], dev["pos"], dev["q"], dev["k"], g["nbr"],
+                              g["cnt"], dev["w1"], dev["w2"], Gd)
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_backward_parity(name):
+    wl, d, G, (rdh, rdq, rdk) = _case(name)
+    dh, dq, dk = (x.cpu().numpy() for x in _run(wl, d, G))
+    e_h = block_rel_error(dh, rdh, wl.lmax)
+    e_q = row_rel_error(dq, rdq)
+    e_k = row_rel_error(dk, rdk)
+    print(f"backward {name}: dh {e_h:.2e}  dq {e_q:.2e}  dk {e_k:.2e}")
+    tol = TOL[wl.dtype]
+    assert e_h < tol and e_q < tol and e_k < tol
+
+
+def test_backward_is_deterministic():
+    wl, d, G, _ = _case("uniform4096_l2_bf16")
+    a = _run(wl, d, G)
+    b = _run(wl, d, G)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+    assert _egat().egat_take_device_status() == _egat().EGAT_OK
+
+
+@pytest.mark.parametrize("lmax", [1, 2, 3])
+def test_backward_edge_cases(lmax):
+    """Ragged systems with an isolated atom (all gradients zero) and atoms at the
+    origin and on the z axis."""
+    n = 23
+    rng = np.random.default_rng(40 + lmax)
+    pts = rng.uniform(-3.0, 3.0, (n, 3))
+    pts[0] = 0.0
+    pts[1] = [0.0, 0.0, -1.3]
+    pts[2] = [60.0, 60.0, 60.0]            # isolated
+    wl = synth.small_cube(n, 6.0, 3.0, 16, lmax, 32, 4, 8, "f32")
+    feats = synth.features(wl, seed=n + lmax)
+    pq = np.rint(pts / synth.GRID_QUANTUM).astype(np.int32)
+    feats.update(pos_q=pq, pos=(pq.astype(np.float64) * synth.GRID_QUANTUM).astype(np.float32))
+    G = rng.standard_normal((n, wl.D, wl.C)).astype(np.float32)
+    dh, dq, dk = (x.cpu().numpy() for x in _run(wl, feats, G))
+    lists, _ = radius_graph(pq, wl.cutoff_q, K=wl.K)
+    rdh, rdq, rdk = oracle_backward(feats["h"], feats["pos"], feats["q"], feats["k"], feats["w1"],
+                                    feats["w2"], lmax, lists, G)
+    assert not dq[2].any() and not dk[2].any() and not dh[2].any()
+    assert block_rel_error(dh, rdh, lmax) < TOL["f32"]
+    assert row_rel_error(dq, rdq) < TOL["f32"] and row_rel_error(dk, rdk) < TOL["f32"]

@@ -53,7 +53,7 @@ def _plan_views(plan: torch.Tensor, n: int, K: int, lmax: int):
     mask = raw[o:o + tiles * TILE * (cap // 32) * 4].view(np.uint32).reshape(tiles, cap // 32, TILE)
     o += a256(tiles * TILE * (cap // 32) * 4)
     ws = sum((2 * l + 1) ** 2 for l in range(lmax + 1))
-    rw = TILE * (1 + (lmax + 1) + ws)
+    rw = 4 + TILE * (1 + (lmax + 1) + ws)
     rec = raw[o:o + tiles * rw * 4].view(np.float32).reshape(tiles, rw)
     return ulen, uni, mask, rec
 
@@ -90,13 +90,15 @@ def test_plan_matches_numpy(name):
             u = np.arange(upad)
             got = ((mask[t, u // 32, r] >> (u % 32).astype(np.uint32)) & 1).astype(bool)
             assert np.array_equal(got, bits), (t, r)
-        # tile record
-        ids = rec[t, :TILE].view(np.int32)
+        # tile record: header (union length, zeros), ids, |r|^l, Wigner-D
+        hdr = rec[t, :4].view(np.int32)
+        assert hdr[0] == U and not hdr[1:].any()
+        ids = rec[t, 4:4 + TILE].view(np.int32)
         want = np.full(TILE, -1, np.int32)
         want[:len(rows)] = rows
         assert np.array_equal(ids, want)
-        rp = rec[t, TILE:TILE * (wl.lmax + 2)].reshape(TILE, wl.lmax + 1)
-        Dr = rec[t, TILE * (wl.lmax + 2):].reshape(TILE, ws)
+        rp = rec[t, 4 + TILE:4 + TILE * (wl.lmax + 2)].reshape(TILE, wl.lmax + 1)
+        Dr = rec[t, 4 + TILE * (wl.lmax + 2):].reshape(TILE, ws)
         for r, a in enumerate(rows[:4]):
             rr = float(np.linalg.norm(pos[a]))
             assert np.allclose(rp[r], [rr ** l for l in range(wl.lmax + 1)], rtol=1e-5, atol=0)

@@ -1,0 +1,94 @@
+"""Pins of the oracle's backward pass (oracle/backward.py).
+
+* The adjoint of the dense coupling is checked against the forward coupling
+  through the defining identity <T x, g> = <x, T* g> on random x, g (no
+  formula retyped: the forward is called as is).
+* The whole backward (dL/dh, dL/dq, dL/dk) is checked against central finite
+  differences of the oracle forward on a tiny system, where fp64 differences
+  are accurate to about 1e-8.
+* Two special cases: a zero upstream gradient gives zero gradients, and a
+  target with a single neighbour (alpha = 1 identically) passes dL/dm straight
+  to that neighbour's h' with no logit gradient.
+"""
+import numpy as np
+import pytest
+
+from oracle import so3
+from oracle.attention import forward, tensor_product
+from oracle.backward import attention_backward, backward, tensor_product_adjoint
+from oracle.graph import radius_graph
+
+
+def _system(seed, n=10, lmax=2, C=8, H=2, dk=4):
+    rng = np.random.default_rng(seed)
+    D = (lmax + 1) ** 2
+    P = len(so3.paths(lmax))
+    pos_q = rng.integers(-3 << 16, 3 << 16, size=(n, 3), dtype=np.int64)
+    pos = pos_q * 2.0 ** -16
+    h = rng.standard_normal((n, D, C))
+    q = rng.standard_normal((n, H, dk))
+    k = rng.standard_normal((n, H, dk))
+    w1 = rng.standard_normal((P, C)) / np.sqrt(3)
+    w2 = rng.standard_normal((P, C)) / np.sqrt(3)
+    lists, _ = radius_graph(pos_q.astype(np.int32), 4 << 16, K=6)
+    G = rng.standard_normal((n, D, C))
+    return dict(h=h, pos=pos, q=q, k=k, w1=w1, w2=w2, lmax=lmax, nbrs=lists, G=G)
+
+
+@pytest.mark.parametrize("lmax", [1, 2, 3])
+def test_adjoint_identity(lmax):
+    rng = np.random.default_rng(lmax)
+    D = (lmax + 1) ** 2
+    x = rng.standard_normal((5, D, 6))
+    g = rng.standard_normal((5, D, 6))
+    pos = rng.standard_normal((5, 3)) * 2
+    w = rng.standard_normal((len(so3.paths(lmax)), 6))
+    lhs = np.sum(tensor_product(x, pos, w, lmax) * g)
+    rhs = np.sum(x * tensor_product_adjoint(g, pos, w, lmax))
+    assert abs(lhs - rhs) <= 1e-10 * max(1.0, abs(lhs))
+
+
+def _loss(s, **over):
+    a = dict(s, **over)
+    out = forward(a["h"], a["pos"], a["q"], a["k"], a["w1"], a["w2"], a["lmax"], a["nbrs"])
+    return float(np.sum(out * a["G"]))
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_backward_matches_finite_differences(seed):
+    s = _system(seed)
+    dh, dq, dk = backward(s["h"], s["pos"], s["q"], s["k"], s["w1"], s["w2"], s["lmax"],
+                          s["nbrs"], s["G"])
+    rng = np.random.default_rng(100 + seed)
+    eps = 1e-5
+    for name, grad in (("h", dh), ("q", dq), ("k", dk)):
+        arr = s[name]
+        for _ in range(12):
+            idx = tuple(int(rng.integers(0, m)) for m in arr.shape)
+            up, dn = arr.copy(), arr.copy()
+            up[idx] += eps
+            dn[idx] -= eps
+            fd = (_loss(s, **{name: up}) - _loss(s, **{name: dn})) / (2 * eps)
+            assert abs(fd - grad[idx]) <= 1e-6 * (1.0 + abs(fd)), (name, idx, fd, grad[idx])
+
+
+def test_zero_upstream_gradient_gives_zero():
+    s = _system(3)
+    dh, dq, dk = backward(s["h"], s["pos"], s["q"], s["k"], s["w1"], s["w2"], s["lmax"],
+                          s["nbrs"], np.zeros_like(s["G"]))
+    assert not dh.any() and not dq.any() and not dk.any()
+
+
+def test_single_neighbour_has_no_logit_gradient():
+    """With one neighbour alpha = 1 identically, so dL/dq and dL/dk vanish and
+    dL/dh' is dL/dm of the target."""
+    rng = np.random.default_rng(5)
+    N, D, C, H, dk = 2, 4, 4, 2, 4
+    hp = rng.standard_normal((N, D, C))
+    q = rng.standard_normal((N, H, dk))
+    k = rng.standard_normal((N, H, dk))
+    dm = rng.standard_normal((N, D, C))
+    nbrs = [np.array([1]), np.array([], dtype=np.int64)]
+    dhp, dq, dk_ = attention_backward(q, k, hp, dm, nbrs)
+    assert np.allclose(dq, 0.0, atol=1e-14) and np.allclose(dk_, 0.0, atol=1e-14)
+    assert np.allclose(dhp[1], dm[0]) and not dhp[0].any()
