@@ -444,7 +444,7 @@ def main():
     e2e_ok = bool(torch.equal(host_out[0].to(dev), out))   # pipelined result == device-timed result
     # ------------------------------------------------------------------ backward
     # gradients of <G, ^h> for a seeded upstream gradient G (egat_backward:
-    # dL/dh, dL/dq, dL/dk; the attention is recomputed, in-lists built inside),
+    # dL/dh, dL/dq, dL/dk, dL/dr; the attention is recomputed, in-lists built inside),
     # each call after an L2 flush, timed with events on the launching stream
     bwd = None
     if args.backward_steps > 0:
@@ -455,12 +455,14 @@ def main():
         dh_t = torch.empty((wl.n, wl.D, wl.C), dtype=torch.float32, device=dev)
         dq_t = torch.empty((wl.n, wl.H, wl.dk), dtype=torch.float32, device=dev)
         dk_t = torch.empty((wl.n, wl.H, wl.dk), dtype=torch.float32, device=dev)
+        dr_t = torch.empty((wl.n, 3), dtype=torch.float32, device=dev)
 
         def backward_call():
             rc = lib.egat_backward(ctypes.byref(cshape), h.data_ptr(), pos.data_ptr(), q.data_ptr(),
                                    k.data_ptr(), nbr.data_ptr(), cnt.data_ptr(), w1.data_ptr(),
                                    w2.data_ptr(), G.data_ptr(), bws_t.data_ptr(), bws_t.numel(),
-                                   dh_t.data_ptr(), dq_t.data_ptr(), dk_t.data_ptr(), sp)
+                                   dh_t.data_ptr(), dq_t.data_ptr(), dk_t.data_ptr(),
+                                   dr_t.data_ptr(), sp)
             egat._check("egat_backward", rc)
 
         graph()                                           # this system's neighbour lists
@@ -479,7 +481,8 @@ def main():
         bwd = {"ms": max_over_ranks(t_bwd, dev),
                "atoms_per_s": job_rate(wl.n, t_bwd, dev),
                "edges_per_s": job_rate(alg["edges"], t_bwd, dev),
-               "what": "dL/dh, dL/dq, dL/dk of <G, ^h> (egat_backward), L2 flushed before each call"}
+               "what": "dL/dh, dL/dq, dL/dk, dL/dr of <G, ^h> (egat_backward), L2 flushed "
+                       "before each call"}
 
     # no bounded device wait may have given up in any of the runs above
     status = lib.egat_take_device_status(torch.cuda.current_stream(dev).cuda_stream)

@@ -17,17 +17,30 @@
 //     relative error on single (atom, head) rows of dq and dk;
 //  2. the neighbour lists are transposed (in-lists: the targets each atom
 //     serves), sorted so every sum runs in a fixed order;
-//  3. per target i (one warp): the forward recomputed gives m_i and the
-//     per-head log-sum-exp; Delta_i = <dm_i, m_i> per head; a second sweep
-//     gives ds_ij = alpha_ij (<dm_i, h'_j>_head - Delta_i) and
-//     dq_i = sum_j ds_ij k_j / sqrt(dk);
+//  3. per target i (one warp): a sweep over the key rows gives the per-head
+//     log-sum-exp; one sweep over key and value rows then gives the exact
+//     weights alpha_ij, m_i, Delta_i = sum_j alpha_ij dalpha_ij per head
+//     (dalpha_ij = <dm_i, h'_j>_head) and dq_i = sum_j ds_ij k_j / sqrt(dk) with
+//     ds_ij = alpha_ij (dalpha_ij - Delta_i), accumulated as
+//     sum alpha dalpha k - Delta sum alpha k;
 //  4. per source j (one warp) over its in-list: alpha_ij from q_i, k_j and
 //     the target's log-sum-exp, dh'_j = sum_i alpha_ij dm_i,
 //     dk_j = sum_i ds_ij q_i / sqrt(dk); the epilogue applies the adjoint of
 //     the source coupling, dh_j = T*(dh'_j; r_j, w1).
 // Step 2's in-lists make every gradient a gather: no atomics touch a result.
+//  5. (optional) dL/dr: positions enter only through the solid harmonics of
+//     the two couplings.  For each coupling value <g, T(x; r)> the radial
+//     derivative is the same operator with |r|^l -> l |r|^(l-1), and the
+//     angular part follows from equivariance: rotating g, x and r together
+//     leaves it unchanged, so r x grad = -(<J g, T x> + <g, T(J x)>) with J the
+//     rotation generators of the Wigner-D representation; both are evaluated
+//     in the frame aligned with r (coupling_grad_channel).
+//     The target pass adds the target coupling's part (g = G_i, x = m_i), the
+//     source pass the source coupling's (g = dh'_j, x = h_j).
 #include <cfloat>
 #include <climits>
+#include <cmath>
+#include <mutex>
 
 #include "egat_device.cuh"
 #include "egat_host.h"
@@ -35,7 +48,7 @@
 namespace egat {
 namespace {
 
-constexpr int kBwdWarps = 4;
+constexpr int kBwdWarps = 4;   // (3 CTAs per SM for the attention passes: no spills at 168 registers)
 constexpr int kSortCap = 4096;   // in-list length sorted in shared memory
 
 // ---------------------------------------------------------------- step 1
@@ -181,11 +194,93 @@ struct BwdParams {
   float* dh;             // [n][D][C]
   const float* pos;
   const float* w1;
+  const float* w2;
+  const float* g;        // upstream gradient [n][D][C]
+  const void* h;         // input features [n][D][C] (storage type)
+  float* dpos;           // dL/dr [n][3], or null
   int n, H, dk_, K, cph;
   float qscale;          // log2(e) / sqrt(dk)
   float kscale;          // 1 / sqrt(dk)
   EaasTable tab;
+  GenTable gen;
 };
+
+// dL/dr of one atom from the coupling values <g_c, T(x_c; r)> of all its
+// channels c, with g and x staged in shared memory ([D][C] each) and the
+// warp's Wigner-D scratch Dsm.  Every lane takes channels lane, lane + 32, ...;
+// the warp reduces; the result is valid in every lane.
+template <int L, int C, typename WFn>
+__device__ __forceinline__ void atom_position_grad(const float* gs, const float* xs, float* Dsm,
+                                                   const float (&r)[3], const EaasTable& tab,
+                                                   const GenTable& gen, WFn wgt, int lane,
+                                                   float (&out)[3]) {
+  constexpr int D = (L + 1) * (L + 1);
+  const float rho = sqrtf(r[0] * r[0] + r[1] * r[1] + r[2] * r[2]);
+  out[0] = out[1] = out[2] = 0.f;
+  if (rho > 0.f) {
+    float Q[9];
+    alignment_rotation(r[0], r[1], r[2], Q);
+    wigner_build<L>(Q, Dsm, lane, 32, [] { __syncwarp(); });
+    __syncwarp();
+    float rpow[L + 1], drpow[L + 1];
+    rpow[0] = 1.f;
+    drpow[0] = 0.f;
+#pragma unroll
+    for (int l = 1; l <= L; ++l) {
+      rpow[l] = rpow[l - 1] * rho;
+      drpow[l] = float(l) * rpow[l - 1];
+    }
+    float dr = 0.f, tx = 0.f, ty = 0.f;
+    for (int c = lane; c < C; c += 32) {
+      float g[D], x[D];
+#pragma unroll
+      for (int d = 0; d < D; ++d) {
+        g[d] = gs[d * C + c];
+        x[d] = xs[d * C + c];
+      }
+      coupling_grad_channel<L>(g, x, Dsm, rpow, drpow, tab, gen, [&](int pp) { return wgt(pp, c); },
+                               dr, tx, ty);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      dr += __shfl_xor_sync(0xffffffffu, dr, o);
+      tx += __shfl_xor_sync(0xffffffffu, tx, o);
+      ty += __shfl_xor_sync(0xffffffffu, ty, o);
+    }
+    // grad = Q ( -ty / rho, tx / rho, dr ): back from the aligned frame
+    const float v0 = -ty / rho, v1 = tx / rho, v2 = dr;
+#pragma unroll
+    for (int a = 0; a < 3; ++a) out[a] = Q[3 * a] * v0 + Q[3 * a + 1] * v1 + Q[3 * a + 2] * v2;
+  } else {
+    // at r = 0 only degree-1 solid harmonics have a gradient, and R^1 is
+    // linear: the derivative along axis a is the coupling at r = e_a with
+    // the degree-1 paths alone, at unit weight
+    float rpow1[L + 1];
+#pragma unroll
+    for (int l = 0; l <= L; ++l) rpow1[l] = l == 1 ? 1.f : 0.f;
+    for (int a = 0; a < 3; ++a) {
+      float Q[9];
+      alignment_rotation(a == 0 ? 1.f : 0.f, a == 1 ? 1.f : 0.f, a == 2 ? 1.f : 0.f, Q);
+      __syncwarp();
+      wigner_build<L>(Q, Dsm, lane, 32, [] { __syncwarp(); });
+      __syncwarp();
+      float s = 0.f;
+      for (int c = lane; c < C; c += 32) {
+        float g[D], t[D];
+#pragma unroll
+        for (int d = 0; d < D; ++d) {
+          g[d] = gs[d * C + c];
+          t[d] = xs[d * C + c];
+        }
+        eaas_channel<L>(t, Dsm, rpow1, tab, [&](int pp) { return wgt(pp, c); },
+                        [&](int d, float v) { s = fmaf(g[d], v, s); });
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      out[a] = s;
+    }
+  }
+}
 
 // sum over the lanes whose value chunks belong to the same head: the bits of
 // the lane index inside a head's chunks (below cph) and the component bits
@@ -234,7 +329,7 @@ __device__ __forceinline__ void load_row(const T* __restrict__ row, float (&v)[T
 
 // Step 3: one warp per target.
 template <int L, int C, typename T>
-__global__ void __launch_bounds__(kBwdWarps * 32)
+__global__ void __launch_bounds__(kBwdWarps * 32, 3)
 attn_bwd_target_kernel(const __grid_constant__ BwdParams p) {
   using Ly = BwdLayout<L, C, T>;
   constexpr int D = Ly::D, NCH = Ly::NCH, TPL = Ly::TPL, CPW = Ly::CPW;
@@ -274,49 +369,36 @@ attn_bwd_target_kernel(const __grid_constant__ BwdParams p) {
   const long long beg = (long long)i * p.K;
   const long long end = beg + row_count(p.cnt, i, p.K);
 
-  // pass 1: the forward recomputed (two-pass softmax: maximum, then sums)
-  float mx = -INFINITY;
+  // sweep 1 (key rows only): the log-sum-exp of the logits, online
+  float mx = -INFINITY, z = 0.f;
   for (long long s = beg; s < end; ++s) {
     const int j = p.nbr[s];
     if ((unsigned)j >= (unsigned)p.n) continue;
-    mx = fmaxf(mx, logit(j));
+    const float sl = logit(j);
+    if (sl > mx) {
+      z = z * exp2f(mx - sl) + 1.f;
+      mx = sl;
+    } else {
+      z += exp2f(sl - mx);
+    }
   }
-  float z = 0.f;
+  const float lse = z > 0.f ? mx + log2f(z) : -INFINITY;
+  float dmv[TPL][8];
+  load_row<TPL, NCH>(dmp + (size_t)i * D * C, dmv, lane);
+
+  // sweep 2 (key and value rows): with the exact weights alpha_ij,
+  //   m_i = sum alpha h'_j, Delta_i = sum alpha dalpha,
+  //   A = sum alpha dalpha k_j, B = sum alpha k_j, and dq_i = (A - Delta B) / sqrt(dk)
+  // (Delta is constant over the sum, so sum alpha (dalpha - Delta) k = A - Delta B)
   float acc[TPL][8];
 #pragma unroll
   for (int t = 0; t < TPL; ++t)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[t][e] = 0.f;
-  for (long long s = beg; s < end; ++s) {
-    const int j = p.nbr[s];
-    if ((unsigned)j >= (unsigned)p.n) continue;
-    const float pw = exp2f(logit(j) - mx);
-    z += pw;
-    float hv[TPL][8];
-    load_row<TPL, NCH>(hp + (size_t)j * D * C, hv, lane);
+  float delta = 0.f;
+  float qa[8], qb[8];
 #pragma unroll
-    for (int t = 0; t < TPL; ++t)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[t][e] = fmaf(pw, hv[t][e], acc[t][e]);
-  }
-  const float lse = z > 0.f ? mx + log2f(z) : -INFINITY;
-  const float inv = z > 0.f ? 1.f / z : 0.f;
-  float dmv[TPL][8];
-  load_row<TPL, NCH>(dmp + (size_t)i * D * C, dmv, lane);
-#pragma unroll
-  for (int t = 0; t < TPL; ++t)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[t][e] *= inv;   // m_i
-  const float delta = head_sum<CPW>(chunk_dot<TPL, NCH>(dmv, acc, lane), p.cph);
-  if (lane < CPW && lane % p.cph == 0) {
-    p.lse[(size_t)i * p.H + head] = lse;
-    p.delta[(size_t)i * p.H + head] = delta;
-  }
-
-  // pass 2: ds_ij and dq_i
-  float dqv[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) dqv[e] = 0.f;
+  for (int e = 0; e < 8; ++e) qa[e] = qb[e] = 0.f;
   const int khead = lane < kch ? lane / G : 0;   // head of this lane's key chunk
   for (long long s = beg; s < end; ++s) {
     const int j = p.nbr[s];
@@ -325,28 +407,70 @@ attn_bwd_target_kernel(const __grid_constant__ BwdParams p) {
     float hv[TPL][8];
     load_row<TPL, NCH>(hp + (size_t)j * D * C, hv, lane);
     const float da = head_sum<CPW>(chunk_dot<TPL, NCH>(dmv, hv, lane), p.cph);
-    const float ds = a * (da - delta);
-    const float dsk = __shfl_sync(0xffffffffu, ds, khead * p.cph);
+    delta = fmaf(a, da, delta);
+#pragma unroll
+    for (int t = 0; t < TPL; ++t)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[t][e] = fmaf(a, hv[t][e], acc[t][e]);
+    const float ak = __shfl_sync(0xffffffffu, a, khead * p.cph);
+    const float adk = __shfl_sync(0xffffffffu, a * da, khead * p.cph);
     if (lane < kch) {
       float kf[8];
       Chunk8<T> kc;
       kc.load(kp + (size_t)j * hdk + 8 * lane);
       kc.to_f32(kf);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) dqv[e] = fmaf(dsk, kf[e], dqv[e]);
+      for (int e = 0; e < 8; ++e) {
+        qa[e] = fmaf(adk, kf[e], qa[e]);
+        qb[e] = fmaf(ak, kf[e], qb[e]);
+      }
     }
   }
+  if (lane < CPW && lane % p.cph == 0) {
+    p.lse[(size_t)i * p.H + head] = lse;
+    p.delta[(size_t)i * p.H + head] = delta;
+  }
+  const float dkh = __shfl_sync(0xffffffffu, delta, khead * p.cph);
+  float dqv[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) dqv[e] = fmaf(-dkh, qb[e], qa[e]);
   if (lane < kch) {
     float* o = p.dq + (size_t)i * hdk + 8 * lane;
 #pragma unroll
     for (int e = 0; e < 8; ++e) o[e] = dqv[e] * p.kscale;
+  }
+  if (p.dpos) {
+    // the target coupling's part of dL/dr_i: g = G_i, x = m_i
+    constexpr int WS = wig_size(L);
+    extern __shared__ float smem[];
+    float* gs = smem + (threadIdx.x >> 5) * (2 * D * C + WS);
+    float* xs = gs + D * C;
+    float* Dsm = xs + D * C;
+#pragma unroll
+    for (int t = 0; t < TPL; ++t) {
+      const int q = lane + 32 * t;
+      if (q < NCH)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xs[8 * q + e] = acc[t][e];
+    }
+    for (int e = lane; e < D * C; e += 32) gs[e] = p.g[(size_t)i * D * C + e];
+    __syncwarp();
+    const float r[3] = {p.pos[3 * i], p.pos[3 * i + 1], p.pos[3 * i + 2]};
+    float gr[3];
+    atom_position_grad<L, C>(gs, xs, Dsm, r, p.tab, p.gen,
+                             [&](int pp, int c) { return __ldg(p.w2 + pp * C + c); }, lane, gr);
+    if (lane == 0) {
+      p.dpos[3 * i] = gr[0];
+      p.dpos[3 * i + 1] = gr[1];
+      p.dpos[3 * i + 2] = gr[2];
+    }
   }
 }
 
 // Step 4: one warp per source atom over its in-list, then the adjoint of the
 // source coupling in the epilogue.
 template <int L, int C, typename T>
-__global__ void __launch_bounds__(kBwdWarps * 32)
+__global__ void __launch_bounds__(kBwdWarps * 32, 3)
 attn_bwd_source_kernel(const __grid_constant__ BwdParams p) {
   using Ly = BwdLayout<L, C, T>;
   constexpr int D = Ly::D, NCH = Ly::NCH, TPL = Ly::TPL, CPW = Ly::CPW;
@@ -419,7 +543,7 @@ attn_bwd_source_kernel(const __grid_constant__ BwdParams p) {
   }
 
   // epilogue: dh_j = T*(dh'_j; r_j, w1), one channel per lane at a time
-  float* gbuf = smem + wib * (D * C + WS);
+  float* gbuf = smem + wib * (D * C + WS + (p.dpos ? D * C : 0));
   float* Dsm = gbuf + D * C;
 #pragma unroll
   for (int t = 0; t < TPL; ++t) {
@@ -444,15 +568,40 @@ attn_bwd_source_kernel(const __grid_constant__ BwdParams p) {
     eaas_channel_adjoint<L>(x, Dsm, rpow, p.tab, [&](int pp) { return __ldg(p.w1 + pp * C + c); },
                             [&](int d, float v) { o[d * C + c] = v; });
   }
+  if (p.dpos) {
+    // the source coupling's part of dL/dr_j: g = dh'_j, x = h_j, added to the
+    // target part the target pass wrote
+    float* xs = Dsm + WS;
+    const T* hr = static_cast<const T*>(p.h) + (size_t)j * D * C;
+    for (int e = lane; e < D * C; e += 32) xs[e] = load_one<T>(hr + e);
+    __syncwarp();
+    const float r[3] = {p.pos[3 * j], p.pos[3 * j + 1], p.pos[3 * j + 2]};
+    float gr[3];
+    atom_position_grad<L, C>(gbuf, xs, Dsm, r, p.tab, p.gen,
+                             [&](int pp, int c) { return __ldg(p.w1 + pp * C + c); }, lane, gr);
+    if (lane == 0) {
+      p.dpos[3 * j] += gr[0];
+      p.dpos[3 * j + 1] += gr[1];
+      p.dpos[3 * j + 2] += gr[2];
+    }
+  }
 }
 
 template <int L, int C, typename T>
 int launch_attn_bwd(const BwdParams& p, cudaStream_t st) {
   constexpr int D = (L + 1) * (L + 1);
   const int grid = (p.n + kBwdWarps - 1) / kBwdWarps;
-  attn_bwd_target_kernel<L, C, T><<<grid, kBwdWarps * 32, 0, st>>>(p);
+  // per warp: G_i, m_i and a Wigner-D scratch when dL/dr is wanted
+  const size_t tshm = p.dpos ? size_t(kBwdWarps) * (2 * D * C + wig_size(L)) * sizeof(float) : 0;
+  auto tkern = attn_bwd_target_kernel<L, C, T>;
+  if (tshm > 48 * 1024 &&
+      cudaFuncSetAttribute(tkern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(tshm)) != cudaSuccess)
+    return EGAT_ERR_CUDA;
+  tkern<<<grid, kBwdWarps * 32, tshm, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return EGAT_ERR_CUDA;
-  const size_t shmem = size_t(kBwdWarps) * (D * C + wig_size(L)) * sizeof(float);
+  // per warp: dh'_j, the Wigner-D scratch and (dL/dr) h_j
+  const size_t shmem =
+      size_t(kBwdWarps) * (D * C + wig_size(L) + (p.dpos ? D * C : 0)) * sizeof(float);
   auto kern = attn_bwd_source_kernel<L, C, T>;
   if (shmem > 48 * 1024 &&
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(shmem)) != cudaSuccess)
@@ -482,6 +631,78 @@ int launch_adjoint(const egat_shape& s, const float* g, const float* pos, const 
 }
 
 size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// host, double precision: the Ivanic–Ruedenberg recursion of wigner_build,
+// for the rotation generators below
+double ir_entry_host(int l, int m, int mp, const double* D1, const double* Dp) {
+  const int wp = 2 * l - 1;
+  auto r1 = [&](int i, int j) { return D1[(i + 1) * 3 + (j + 1)]; };
+  auto rp = [&](int a, int b) { return Dp[(a + l - 1) * wp + (b + l - 1)]; };
+  auto P = [&](int i, int a, int b) -> double {
+    if (b == l) return r1(i, 1) * rp(a, l - 1) - r1(i, -1) * rp(a, -l + 1);
+    if (b == -l) return r1(i, 1) * rp(a, -l + 1) + r1(i, -1) * rp(a, l - 1);
+    return r1(i, 0) * rp(a, b);
+  };
+  const double d = (std::abs(mp) == l) ? double((2 * l) * (2 * l - 1)) : double((l + mp) * (l - mp));
+  const int am = std::abs(m);
+  double val = 0.0;
+  if (am < l) val += std::sqrt(double((l + m) * (l - m)) / d) * P(0, m, mp);
+  {
+    const double v = 0.5 * std::sqrt(double((m == 0 ? 2 : 1) * (l + am - 1) * (l + am)) / d) *
+                     (m == 0 ? -1.0 : 1.0);
+    double V;
+    if (m == 0) V = P(1, 1, mp) + P(-1, -1, mp);
+    else if (m > 0) V = P(1, m - 1, mp) * (m == 1 ? std::sqrt(2.0) : 1.0) - (m == 1 ? 0.0 : P(-1, -m + 1, mp));
+    else V = (m == -1 ? 0.0 : P(1, m + 1, mp)) + P(-1, -m - 1, mp) * (m == -1 ? std::sqrt(2.0) : 1.0);
+    val += v * V;
+  }
+  if (m != 0 && am < l - 1) {
+    const double w = -0.5 * std::sqrt(double((l - am - 1) * (l - am)) / d);
+    const double W = (m > 0) ? (P(1, m + 1, mp) + P(-1, -m - 1, mp)) : (P(1, m - 1, mp) - P(-1, -m + 1, mp));
+    val += w * W;
+  }
+  return val;
+}
+
+void wigner_host(const double (&Q)[9], double* D) {
+  D[0] = 1.0;
+  for (int e = 0; e < 9; ++e) D[wig_off(1) + e] = Q[wig1_src(e)];
+  for (int l = 2; l <= kMaxL; ++l) {
+    const int w = 2 * l + 1;
+    for (int e = 0; e < w * w; ++e)
+      D[wig_off(l) + e] = ir_entry_host(l, e / w - l, e % w - l, D + wig_off(1), D + wig_off(l - 1));
+  }
+}
+
+// J_a = dD(R_a(t))/dt at t = 0, by central differences of the recursion in
+// double precision (step 1e-5: error ~1e-10, far below float rounding)
+GenTable make_gen_table() {
+  GenTable g;
+  const double h = 1e-5;
+  for (int a = 0; a < 3; ++a) {
+    double Dp[wig_size(kMaxL)], Dm[wig_size(kMaxL)];
+    for (int sgn = 0; sgn < 2; ++sgn) {
+      const double t = sgn == 0 ? h : -h;
+      const double c = std::cos(t), s_ = std::sin(t);
+      double Q[9] = {1, 0, 0, 0, 1, 0, 0, 0, 1};
+      const int i = (a + 1) % 3, j = (a + 2) % 3;   // the plane the rotation turns
+      Q[i * 3 + i] = c;
+      Q[i * 3 + j] = -s_;
+      Q[j * 3 + i] = s_;
+      Q[j * 3 + j] = c;
+      wigner_host(Q, sgn == 0 ? Dp : Dm);
+    }
+    for (int e = 0; e < wig_size(kMaxL); ++e) g.J[a][e] = float((Dp[e] - Dm[e]) / (2 * h));
+  }
+  return g;
+}
+
+const GenTable& gen_table() {
+  static std::once_flag once;
+  static GenTable g;
+  std::call_once(once, [] { g = make_gen_table(); });
+  return g;
+}
 
 struct BwdWs {
   void* hp;
@@ -528,7 +749,7 @@ size_t backward_ws_bytes(const egat_shape& s) { return bwd_ws(s, nullptr).bytes;
 int launch_backward(const egat_shape& s, const void* d_h, const float* d_pos, const void* d_q,
                     const void* d_k, const int32_t* d_nbr, const int32_t* d_cnt, const float* d_w1,
                     const float* d_w2, const float* d_g, void* d_ws, float* d_dh, float* d_dq,
-                    float* d_dk, cudaStream_t st) {
+                    float* d_dk, float* d_dpos, cudaStream_t st) {
   const BwdWs w = bwd_ws(s, d_ws);
   const bool bf = s.dtype == EGAT_BF16;
   // h' = source coupling (forward step 2), in float32
@@ -570,6 +791,11 @@ int launch_backward(const egat_shape& s, const void* d_h, const float* d_pos, co
   p.dh = d_dh;
   p.pos = d_pos;
   p.w1 = d_w1;
+  p.w2 = d_w2;
+  p.g = d_g;
+  p.h = d_h;
+  p.dpos = d_dpos;
+  p.gen = gen_table();
   p.n = s.n;
   p.H = s.H;
   p.dk_ = s.dk;

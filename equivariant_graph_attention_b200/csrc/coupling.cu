@@ -271,12 +271,13 @@ eaas_source_kernel(const __grid_constant__ EaasParams p) {
   }
 }
 // Planned source coupling staged by tiles, for shapes with one warp per atom
-// (C = 128 up to lmax 2).  A persistent CTA of kTileM warps takes the plan's tiles in
-// turn.  The tile record arrives by one bulk copy two tiles ahead and the
-// tile's 16 feature rows by 16 bulk copies one tile ahead (double-buffered),
-// so the loads stream while the previous tile is coupled; warp r couples
-// target slot r from shared memory (rotation and |r|^l from the record) and
-// writes its h' row straight to global memory.  Every wait is bounded.
+// (C = 128 up to lmax 2).  Persistent CTAs of kTileM / 2 warps (two per SM)
+// take the plan's tiles in turn.  The tile record arrives by one bulk copy
+// two tiles ahead and the tile's 16 feature rows by 16 bulk copies one tile
+// ahead (double-buffered), so the loads stream while the previous tile is
+// coupled; warp w couples target slots w and w + kTileM / 2 from shared
+// memory (rotation and |r|^l from the record) and writes their h' rows
+// straight to global memory.  Every wait is bounded.
 template <int L, typename T>
 struct TileSmem {
   static constexpr int D = (L + 1) * (L + 1);
@@ -292,8 +293,11 @@ struct TileSmem {
   static_assert(ROWB % 16 == 0 && REC % 4 == 0 && bars % 8 == 0, "bulk-copy alignment");
 };
 
+// half a tile's warps per CTA, two CTAs per SM: one CTA's per-tile barrier
+// overlaps the other's work
+constexpr int kHalfWarps = kTileM / 2;
 template <int L, typename T>
-__global__ void __launch_bounds__(kTileM * 32, 1)
+__global__ void __launch_bounds__(kHalfWarps * 32, 2)
 eaas_tile_kernel(const __grid_constant__ EaasParams p) {
   using Sm = TileSmem<L, T>;
   constexpr int D = Sm::D, CPL = Sm::CPL, C = Sm::C, ROWB = Sm::ROWB, REC = Sm::REC;
@@ -307,7 +311,7 @@ eaas_tile_kernel(const __grid_constant__ EaasParams p) {
   uint64_t* recbar = rowbar + 2;                                     // [3] a tile record
   volatile int* abort_flag = reinterpret_cast<volatile int*>(recbar + 3);
 
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, wfirst = tid >> 5;
   const int tiles = int(p.items / kTileM);
   const int grid = gridDim.x;
   if (blockIdx.x >= tiles) return;   // whole CTA
@@ -363,6 +367,7 @@ eaas_tile_kernel(const __grid_constant__ EaasParams p) {
       if (tile + 2 * grid < tiles) issue_rec(tile + 2 * grid, (j + 2) % 3);
     }
     const float* rec = recs + rb * REC;
+    for (int w = wfirst; w < kTileM; w += kHalfWarps) {   // two slots per warp
     const int at = reinterpret_cast<const int*>(rec)[kRecTgt + w];
     if ((unsigned)at < (unsigned)p.n) {
       const T* xr = reinterpret_cast<const T*>(rows + (size_t(wb) * kTileM + w) * ROWB) + lane * CPL;
@@ -382,6 +387,7 @@ eaas_tile_kernel(const __grid_constant__ EaasParams p) {
       eaas_multi<L, CPL>(xv, rec + rec_off_D(L) + w * WS, rpow, p.tab,
                          [&](int q, int k) { return swc[q * C + k]; },
                          [&](int d, const float (&v)[CPL]) { ChanVec<T, CPL>::store(yr + d * C, v); });
+    }
     }
     __syncthreads();   // rows[wb] and recs[rb] are refilled one and two tiles ahead
   }
@@ -468,8 +474,8 @@ int launch_eaas_tile(const egat_shape& s, const void* d_x, const float* rec, lon
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int tiles = int(items / kTileM);
-  const int grid = tiles < sms ? tiles : sms;
-  kern<<<grid, kTileM * 32, shmem, st>>>(p);
+  const int grid = tiles < 2 * sms ? tiles : 2 * sms;
+  kern<<<grid, kHalfWarps * 32, shmem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
 }
 

@@ -63,6 +63,14 @@ struct EaasTable {
   float f[kMaxPaths][2 * kMaxL + 1];
 };
 
+// Real-basis rotation generators of degrees 0..kMaxL for the three axes:
+// J[a] holds, block-diagonally at wig_off(l), the (2l+1) x (2l+1) matrix
+// dD^l(R_a(t))/dt at t = 0 (R_a(t) the rotation by t about axis a) of this
+// library's own Wigner-D construction.  Filled on the host.
+struct GenTable {
+  float J[3][(kMaxL + 1) * (2 * kMaxL + 1) * (2 * kMaxL + 3) / 3];
+};
+
 // ---------------------------------------------------------------------------
 // packed float2 arithmetic (sm_100 f32x2 FMA / MUL on a 64-bit register pair)
 // ---------------------------------------------------------------------------
@@ -472,6 +480,98 @@ __device__ __forceinline__ void eaas_channel_adjoint(float (&g)[(L + 1) * (L + 1
       out(l * l + a, s);
     }
   });
+}
+
+// Position gradient of one channel's coupling value L_c = <g, T(x; r)> (T the
+// operator of eaas_channel: T = D Rw D^T with D = D(Q), Q z = r/|r|, and Rw the
+// weighted axis-frame re-index), evaluated in the aligned frame:
+//   g~ = D^T g, x~ = D^T x;
+//   dL_c/d|r| = <g~, Rw' x~>, Rw' with |r|^l replaced by l |r|^(l-1) (drpow);
+//   rotating g, x and r together leaves L_c unchanged, so
+//   r x grad L_c = -tau with tau_a = <J_a g, T x> + <g, T(J_a x)>, and since
+//   D^T J_a D = sum_b Q_ab J_b, tau = Q tau~ with
+//   tau~_b = <J_b g~, Rw x~> + <g~, Rw J_b x~>.
+// With r = |r| Q z only tau~_x and tau~_y matter:
+//   grad L_c = Q ( -tau~_y / |r|, tau~_x / |r|, dL_c/d|r| ).
+// This accumulates dr, tx = tau~_x, ty = tau~_y for the caller.
+template <int L, typename WFn>
+__device__ __forceinline__ void coupling_grad_channel(float (&g)[(L + 1) * (L + 1)],
+                                                      float (&x)[(L + 1) * (L + 1)],
+                                                      const float* __restrict__ Dsm,
+                                                      const float (&rpow)[L + 1],
+                                                      const float (&drpow)[L + 1],
+                                                      const EaasTable& tab, const GenTable& gen,
+                                                      WFn wgt, float& dr, float& tx, float& ty) {
+  constexpr int D = (L + 1) * (L + 1);
+  // into the aligned frame (in place)
+  auto to_frame = [&](float (&v)[D]) {
+    static_for<1, L + 1>([&](auto lc) {
+      constexpr int l = decltype(lc)::value;
+      constexpr int w = 2 * l + 1;
+      const float* Dl = Dsm + wig_off(l);
+      float tmp[w];
+#pragma unroll
+      for (int a = 0; a < w; ++a) {
+        float s = 0.f;
+#pragma unroll
+        for (int c = 0; c < w; ++c) s = fmaf(Dl[c * w + a], v[l * l + c], s);
+        tmp[a] = s;
+      }
+#pragma unroll
+      for (int a = 0; a < w; ++a) v[l * l + a] = tmp[a];
+    });
+  };
+  // <u, Rw(pw) v> for the re-index with radial factors pw
+  auto reindex_dot = [&](const float (&u)[D], const float (&v)[D], const float (&pw)[L + 1]) {
+    float acc = 0.f;
+    static_for<0, num_paths(L)>([&](auto pc) {
+      constexpr int p = decltype(pc)::value;
+      constexpr int li = path_info(L, p, 0);
+      constexpr int lf = path_info(L, p, 1);
+      constexpr int lo = path_info(L, p, 2);
+      constexpr bool even = ((li + lf + lo) % 2) == 0;
+      const float wp = wgt(p) * pw[lf];
+      float part = 0.f;
+#pragma unroll
+      for (int mo = -lo; mo <= lo; ++mo) {
+        const int src = even ? mo : -mo;
+        const bool live = (iabs(mo) <= li) && (even || mo != 0);
+        if (live) part = fmaf(tab.f[p][mo + lo] * u[lo * lo + lo + mo], v[li * li + li + src], part);
+      }
+      acc = fmaf(wp, part, acc);
+    });
+    return acc;
+  };
+  // o = J_b v (block-diagonal)
+  auto gen_apply = [&](int bax, const float (&v)[D], float (&o)[D]) {
+    o[0] = 0.f;
+    static_for<1, L + 1>([&](auto lc) {
+      constexpr int l = decltype(lc)::value;
+      constexpr int w = 2 * l + 1;
+      const float* Jl = gen.J[bax] + wig_off(l);
+#pragma unroll
+      for (int m = 0; m < w; ++m) {
+        float s = 0.f;
+#pragma unroll
+        for (int c = 0; c < w; ++c) s = fmaf(Jl[m * w + c], v[l * l + c], s);
+        o[l * l + m] = s;
+      }
+    });
+  };
+  to_frame(g);
+  to_frame(x);
+  dr += reindex_dot(g, x, drpow);
+  // <J_b g~, Rw x~> = <Rw^T J_b g~, x~> = reindex_dot(J_b g~, x~); <g~, Rw J_b x~> = reindex_dot(g~, J_b x~)
+#pragma unroll 1
+  for (int bax = 0; bax < 2; ++bax) {
+    float jv[D];
+    gen_apply(bax, g, jv);
+    float s = reindex_dot(jv, x, rpow);
+    gen_apply(bax, x, jv);
+    s += reindex_dot(g, jv, rpow);
+    tx += bax == 0 ? s : 0.f;
+    ty += bax == 1 ? s : 0.f;
+  }
 }
 
 // The same operator on NCH channels at once (channels of one atom share the

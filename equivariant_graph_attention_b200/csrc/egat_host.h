@@ -90,7 +90,7 @@ size_t backward_ws_bytes(const egat_shape& s);
 int launch_backward(const egat_shape& s, const void* d_h, const float* d_pos, const void* d_q,
                     const void* d_k, const int32_t* d_nbr, const int32_t* d_cnt, const float* d_w1,
                     const float* d_w2, const float* d_g, void* d_ws, float* d_dh, float* d_dq,
-                    float* d_dk, cudaStream_t st);
+                    float* d_dk, float* d_dpos, cudaStream_t st);
 // Bounded-wait reports (one per compilation unit with mbarrier waits): read
 // and clear the count of waits that gave up (synchronises st); the self-test
 // launch.

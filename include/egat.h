@@ -281,10 +281,12 @@ EGAT_API int egat_forward_noalloc(const egat_shape* s, const void* d_h, const fl
  * log-sum-exp per target and head).  For an upstream gradient
  * G = dL/d^h (float32 [n][D][C]) of the forward egat_forward computes on the
  * padded graph (d_nbr, d_cnt; d_cnt may be NULL), writes
- *  d_dh  float32 [n][D][C]   dL/dh
- *  d_dq  float32 [n][H][dk]  dL/dq
- *  d_dk  float32 [n][H][dk]  dL/dk
- * (gradients with respect to positions and weights are not computed).  The
+ *  d_dh    float32 [n][D][C]   dL/dh
+ *  d_dq    float32 [n][H][dk]  dL/dq
+ *  d_dk    float32 [n][H][dk]  dL/dk
+ *  d_dpos  float32 [n][3]      dL/dr (forces are its negative); may be NULL
+ * (positions enter through the solid harmonics of both couplings, the
+ * neighbour lists held fixed; weight gradients are not computed).  The
  * in-lists (targets served by each atom) are built and sorted inside, so
  * every gradient is a gather in a fixed order: deterministic, no atomics on
  * results.  Padded graphs only (CSR returns EGAT_ERR_UNSUPPORTED), n * K below
@@ -296,7 +298,7 @@ EGAT_API int egat_backward(const egat_shape* s, const void* d_h, const float* d_
                            const void* d_k, const int32_t* d_nbr, const int32_t* d_cnt,
                            const float* d_w1, const float* d_w2, const float* d_grad_out,
                            void* d_ws, size_t ws_bytes, float* d_dh, float* d_dq, float* d_dk,
-                           void* stream);
+                           float* d_dpos, void* stream);
 
 /*
  * Device status.  The tensor-core attention kernel waits on mbarriers for its

@@ -21,8 +21,17 @@ the plain adjoint of the corresponding forward step:
    dL/dk_j   += ds_ij q_i / sqrt(d_k);
 3. source coupling h'_j = T(h_j; r_j, w1): dL/dh_j = T^*(dL/dh'_j; r_j, w1).
 
-Gradients with respect to positions and weights are not computed here.
-Layouts as in ``attention``; every atom is a target (nbrs[i] = N(i)).
+Positions enter only through the solid harmonics R(r) of the two couplings
+(the logits are invariant scalars and the neighbour lists are piecewise
+constant), so the position gradient is
+
+   dL/dr_a = sum_c sum_p w2[p][c] sum T_p[m,mi,mf] G_a^{lo}[m][c] m_a^{li}[mi][c] dR^{lf}_{mf}(r_a)/dr_a
+           + sum_c sum_p w1[p][c] sum T_p[m,mi,mf] dh'_a^{lo}[m][c] h_a^{li}[mi][c] dR^{lf}_{mf}(r_a)/dr_a
+
+with the exact gradient of the solid harmonics (``so3.solid_harmonics_grad``);
+forces are its negative.  Gradients with respect to the coupling weights are
+not computed here.  Layouts as in ``attention``; every atom is a target
+(nbrs[i] = N(i)).
 """
 from __future__ import annotations
 
@@ -31,7 +40,7 @@ from typing import Sequence, Tuple
 import numpy as np
 
 from . import so3
-from .attention import _block, head_of_channel, logits, softmax_two_pass, source_coupling
+from .attention import _block, aggregate, head_of_channel, logits, softmax_two_pass, source_coupling
 
 
 def tensor_product_adjoint(g: np.ndarray, pos: np.ndarray, w: np.ndarray, lmax: int) -> np.ndarray:
@@ -93,3 +102,34 @@ def backward(h, pos, q, k, w1, w2, lmax: int, nbrs: Sequence[np.ndarray],
     dhp, dq, dk = attention_backward(q, k, hp, dm, nbrs)
     dh = tensor_product_adjoint(dhp, pos, w1, lmax)
     return dh, dq, dk
+
+
+def coupling_position_grad(g, x, pos, w, lmax: int) -> np.ndarray:
+    """d<g, T(x; r, w)>/dr for each atom: [N, 3].
+
+    sum_c sum_p w[p][c] sum_{m,mi,mf} T_p[m,mi,mf] g^{lo}[m][c] x^{li}[mi][c] dR^{lf}_{mf}/dr.
+    """
+    g = np.asarray(g, dtype=np.float64)
+    x = np.asarray(x, dtype=np.float64)
+    pos = np.asarray(pos, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    dR = [so3.solid_harmonics_grad(l, pos) for l in range(lmax + 1)]    # [N, 2l+1, 3]
+    out = np.zeros((pos.shape[0], 3))
+    for p, (li, lf, lo) in enumerate(so3.paths(lmax)):
+        if lf == 0:
+            continue
+        T = so3.real_cg(li, lf, lo)
+        bil = np.einsum("oif,noc,nic,c->nf", T, _block(g, lo), _block(x, li), w[p])
+        out += np.einsum("nf,nfa->na", bil, dR[lf])
+    return out
+
+
+def position_grad(h, pos, q, k, w1, w2, lmax: int, nbrs: Sequence[np.ndarray], G) -> np.ndarray:
+    """dL/dr [N, 3] for L = sum_i <G_i, ^h_i> (forces are -dL/dr)."""
+    pos = np.asarray(pos, dtype=np.float64)
+    hp = source_coupling(h, pos, w1, lmax)
+    m = aggregate(q, k, hp, nbrs)
+    dm = tensor_product_adjoint(G, pos, w2, lmax)
+    dhp, _, _ = attention_backward(q, k, hp, dm, nbrs)
+    return (coupling_position_grad(G, m, pos, w2, lmax)
+            + coupling_position_grad(dhp, h, pos, w1, lmax))

@@ -139,6 +139,52 @@ def solid_harmonics(l: int, r: np.ndarray) -> np.ndarray:
     return out
 
 
+_MONO_CACHE = {}
+
+
+def _monomials(l: int):
+    """Exponents (a, b, c), a + b + c = l, of the homogeneous monomials x^a y^b z^c."""
+    return [(a, b, l - a - b) for a in range(l + 1) for b in range(l + 1 - a)]
+
+
+def _solid_poly(l: int) -> np.ndarray:
+    """Coefficients [2l+1, n_monomials] of R^l in the monomial basis.
+
+    R^l is a homogeneous polynomial of degree l, so its coefficients follow
+    exactly (up to rounding) from values at more points than monomials; they
+    are fitted once by least squares over fixed random points.
+    """
+    if l not in _MONO_CACHE:
+        mono = _monomials(l)
+        pts = np.random.default_rng(4321 + l).standard_normal((4 * len(mono) + 8, 3))
+        A = np.stack([pts[:, 0] ** a * pts[:, 1] ** b * pts[:, 2] ** c for a, b, c in mono], axis=1)
+        coef, *_ = np.linalg.lstsq(A, solid_harmonics(l, pts), rcond=None)
+        _MONO_CACHE[l] = coef.T
+    return _MONO_CACHE[l]
+
+
+def solid_harmonics_grad(l: int, r: np.ndarray) -> np.ndarray:
+    """Gradient of the solid harmonics: [..., 2l+1, 3], d R^l_m / d r_a.
+
+    The exact derivative of the monomial form of R^l (see _solid_poly).
+    """
+    r = np.asarray(r, dtype=np.float64)
+    out = np.zeros(r.shape[:-1] + (2 * l + 1, 3))
+    if l == 0:
+        return out
+    coef = _solid_poly(l)
+    x, y, z = r[..., 0], r[..., 1], r[..., 2]
+    pw = lambda v, e: v ** e if e > 0 else np.ones_like(v)
+    for k, (a, b, c) in enumerate(_monomials(l)):
+        if a:
+            out[..., :, 0] += coef[:, k] * (a * pw(x, a - 1) * pw(y, b) * pw(z, c))[..., None]
+        if b:
+            out[..., :, 1] += coef[:, k] * (b * pw(x, a) * pw(y, b - 1) * pw(z, c))[..., None]
+        if c:
+            out[..., :, 2] += coef[:, k] * (c * pw(x, a) * pw(y, b) * pw(z, c - 1))[..., None]
+    return out
+
+
 # --------------------------------------------------------------------------
 # Real coupling tensors
 # --------------------------------------------------------------------------

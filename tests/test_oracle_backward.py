@@ -15,7 +15,7 @@ import pytest
 
 from oracle import so3
 from oracle.attention import forward, tensor_product
-from oracle.backward import attention_backward, backward, tensor_product_adjoint
+from oracle.backward import attention_backward, backward, position_grad, tensor_product_adjoint
 from oracle.graph import radius_graph
 
 
@@ -92,3 +92,40 @@ def test_single_neighbour_has_no_logit_gradient():
     dhp, dq, dk_ = attention_backward(q, k, hp, dm, nbrs)
     assert np.allclose(dq, 0.0, atol=1e-14) and np.allclose(dk_, 0.0, atol=1e-14)
     assert np.allclose(dhp[1], dm[0]) and not dhp[0].any()
+
+
+@pytest.mark.parametrize("l", [1, 2, 3])
+def test_solid_harmonics_gradient_matches_finite_differences(l):
+    rng = np.random.default_rng(l)
+    r = rng.standard_normal((6, 3)) * 1.7
+    got = so3.solid_harmonics_grad(l, r)
+    eps = 1e-6
+    for a in range(3):
+        e = np.zeros(3)
+        e[a] = eps
+        fd = (so3.solid_harmonics(l, r + e) - so3.solid_harmonics(l, r - e)) / (2 * eps)
+        assert np.allclose(got[..., a], fd, rtol=1e-7, atol=1e-7 * (1 + np.abs(fd).max()))
+
+
+def test_solid_harmonics_gradient_closed_form_degree1():
+    """Degree 1 is linear: R^1 = (y, z, x) in the basis order, so its gradient
+    is a constant permutation matrix."""
+    g = so3.solid_harmonics_grad(1, np.array([[0.3, -1.2, 2.5]]))[0]
+    assert np.allclose(g, [[0, 1, 0], [0, 0, 1], [1, 0, 0]], atol=1e-12)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_position_gradient_matches_finite_differences(seed):
+    """dL/dr against central differences of the oracle forward in the
+    positions (neighbour lists held fixed, as the gradient assumes)."""
+    s = _system(seed)
+    grad = position_grad(s["h"], s["pos"], s["q"], s["k"], s["w1"], s["w2"], s["lmax"],
+                         s["nbrs"], s["G"])
+    eps = 1e-6
+    for a in range(s["pos"].shape[0]):
+        for c in range(3):
+            up, dn = s["pos"].copy(), s["pos"].copy()
+            up[a, c] += eps
+            dn[a, c] -= eps
+            fd = (_loss(s, pos=up) - _loss(s, pos=dn)) / (2 * eps)
+            assert abs(fd - grad[a, c]) <= 1e-5 * (1.0 + abs(fd)), (a, c, fd, grad[a, c])
