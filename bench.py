@@ -51,7 +51,8 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attention_traffic.json")
 KERNEL_SOURCES = ["equivariant_graph_attention_b200/csrc/attention.cu",
                   "equivariant_graph_attention_b200/csrc/attention_tc.cu",
                   "equivariant_graph_attention_b200/csrc/plan.cu",
-                  "equivariant_graph_attention_b200/csrc/egat_device.cuh"]
+                  "equivariant_graph_attention_b200/csrc/egat_device.cuh",
+                  "equivariant_graph_attention_b200/csrc/egat_async.cuh"]
 
 
 def kernel_source_sha() -> str:
@@ -459,8 +460,9 @@ def main():
 
         def backward_call():
             rc = lib.egat_backward(ctypes.byref(cshape), h.data_ptr(), pos.data_ptr(), q.data_ptr(),
-                                   k.data_ptr(), nbr.data_ptr(), cnt.data_ptr(), w1.data_ptr(),
-                                   w2.data_ptr(), G.data_ptr(), bws_t.data_ptr(), bws_t.numel(),
+                                   k.data_ptr(), nbr.data_ptr(), cnt.data_ptr(), order.data_ptr(),
+                                   w1.data_ptr(), w2.data_ptr(), G.data_ptr(), bws_t.data_ptr(),
+                                   bws_t.numel(),
                                    dh_t.data_ptr(), dq_t.data_ptr(), dk_t.data_ptr(),
                                    dr_t.data_ptr(), sp)
             egat._check("egat_backward", rc)

@@ -251,12 +251,14 @@ int egat_forward(const egat_shape* s, const void* d_h, const float* d_pos, const
 
 int egat_take_device_status(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  unsigned int a = 0, b = 0;
+  unsigned int a = 0, b = 0, c = 0;
   const int ra = take_wait_timeouts_attention(st, &a);
   const int rb = take_wait_timeouts_coupling(st, &b);
+  const int rc = take_wait_timeouts_backward(st, &c);
   if (ra != EGAT_OK) return ra;
   if (rb != EGAT_OK) return rb;
-  return (a | b) ? EGAT_ERR_TIMEOUT : EGAT_OK;
+  if (rc != EGAT_OK) return rc;
+  return (a | b | c) ? EGAT_ERR_TIMEOUT : EGAT_OK;
 }
 
 int egat_selftest_wait_timeout(int32_t polls, void* stream) {
@@ -275,9 +277,10 @@ int egat_backward_workspace_bytes(const egat_shape* s, size_t* bytes) {
 }
 
 int egat_backward(const egat_shape* s, const void* d_h, const float* d_pos, const void* d_q,
-                  const void* d_k, const int32_t* d_nbr, const int32_t* d_cnt, const float* d_w1,
-                  const float* d_w2, const float* d_grad_out, void* d_ws, size_t ws_bytes,
-                  float* d_dh, float* d_dq, float* d_dk, float* d_dpos, void* stream) {
+                  const void* d_k, const int32_t* d_nbr, const int32_t* d_cnt,
+                  const int32_t* d_order, const float* d_w1, const float* d_w2,
+                  const float* d_grad_out, void* d_ws, size_t ws_bytes, float* d_dh, float* d_dq,
+                  float* d_dk, float* d_dpos, void* stream) {
   const int rc = check_shape(s, true);
   if (rc != EGAT_OK) return rc;
   if (s->graph_mode != EGAT_GRAPH_PADDED) return EGAT_ERR_UNSUPPORTED;
@@ -289,9 +292,9 @@ int egat_backward(const egat_shape* s, const void* d_h, const float* d_pos, cons
   if (!aligned16(d_h) || !aligned16(d_q) || !aligned16(d_k) || !aligned16(d_ws) ||
       !aligned16(d_grad_out) || !aligned16(d_dh) || !aligned16(d_dq) || !aligned16(d_dk) ||
       !aligned4(d_pos) || !aligned4(d_nbr) || !aligned4(d_w1) || !aligned4(d_w2) ||
-      (d_dpos && !aligned4(d_dpos)))
+      (d_dpos && !aligned4(d_dpos)) || (d_order && !aligned4(d_order)))
     return EGAT_ERR_ARG;
   if (ws_bytes < backward_ws_bytes(*s)) return EGAT_ERR_WORKSPACE;
-  return launch_backward(*s, d_h, d_pos, d_q, d_k, d_nbr, d_cnt, d_w1, d_w2, d_grad_out, d_ws, d_dh,
-                         d_dq, d_dk, d_dpos, static_cast<cudaStream_t>(stream));
+  return launch_backward(*s, d_h, d_pos, d_q, d_k, d_nbr, d_cnt, d_order, d_w1, d_w2, d_grad_out,
+                         d_ws, d_dh, d_dq, d_dk, d_dpos, static_cast<cudaStream_t>(stream));
 }

@@ -587,6 +587,73 @@ attn_bwd_source_kernel(const __grid_constant__ BwdParams p) {
   }
 }
 
+// dL/dr of every atom when the attention gradients come from the tiled
+// passes: one warp per atom adds the target coupling's part (g = G_a,
+// x = m_a, weights w2) and the source coupling's part (g = dh'_a, x = h_a,
+// weights w1).
+struct PosGradParams {
+  const float* g;     // upstream gradient [n][D][C]
+  const float* m;     // m [n][D][C]
+  const float* dhp;   // dL/dh' [n][D][C]
+  const void* h;      // input features [n][D][C] (storage type)
+  const float* pos;
+  const float* w1;
+  const float* w2;
+  float* dpos;
+  int n;
+  EaasTable tab;
+  GenTable gen;
+};
+
+template <int L, int C, typename T>
+__global__ void __launch_bounds__(kBwdWarps * 32) position_grad_kernel(const __grid_constant__ PosGradParams p) {
+  constexpr int D = (L + 1) * (L + 1);
+  constexpr int WS = wig_size(L);
+  extern __shared__ float smem[];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int a = blockIdx.x * kBwdWarps + wib;
+  if (a >= p.n) return;   // whole warp
+  float* gs = smem + wib * (2 * D * C + WS);
+  float* xs = gs + D * C;
+  float* Dsm = xs + D * C;
+  const float r[3] = {p.pos[3 * a], p.pos[3 * a + 1], p.pos[3 * a + 2]};
+  for (int e = lane; e < D * C; e += 32) {
+    gs[e] = p.g[(size_t)a * D * C + e];
+    xs[e] = p.m[(size_t)a * D * C + e];
+  }
+  __syncwarp();
+  float gt[3], gsrc[3];
+  atom_position_grad<L, C>(gs, xs, Dsm, r, p.tab, p.gen,
+                           [&](int pp, int c) { return __ldg(p.w2 + pp * C + c); }, lane, gt);
+  __syncwarp();
+  const T* hr = static_cast<const T*>(p.h) + (size_t)a * D * C;
+  for (int e = lane; e < D * C; e += 32) {
+    gs[e] = p.dhp[(size_t)a * D * C + e];
+    xs[e] = load_one<T>(hr + e);
+  }
+  __syncwarp();
+  atom_position_grad<L, C>(gs, xs, Dsm, r, p.tab, p.gen,
+                           [&](int pp, int c) { return __ldg(p.w1 + pp * C + c); }, lane, gsrc);
+  if (lane == 0) {
+    p.dpos[3 * a] = gt[0] + gsrc[0];
+    p.dpos[3 * a + 1] = gt[1] + gsrc[1];
+    p.dpos[3 * a + 2] = gt[2] + gsrc[2];
+  }
+}
+
+template <int L, typename T>
+int launch_position_grad(const PosGradParams& p, cudaStream_t st) {
+  constexpr int C = 128;
+  constexpr int D = (L + 1) * (L + 1);
+  const size_t shm = size_t(kBwdWarps) * (2 * D * C + wig_size(L)) * sizeof(float);
+  auto kern = position_grad_kernel<L, C, T>;
+  if (shm > 48 * 1024 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(shm)) != cudaSuccess)
+    return EGAT_ERR_CUDA;
+  kern<<<(p.n + kBwdWarps - 1) / kBwdWarps, kBwdWarps * 32, shm, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
+}
+
 template <int L, int C, typename T>
 int launch_attn_bwd(const BwdParams& p, cudaStream_t st) {
   constexpr int D = (L + 1) * (L + 1);
@@ -705,6 +772,7 @@ const GenTable& gen_table() {
 }
 
 struct BwdWs {
+  BwdTcWs tc;   // the tiled path's part (tiled shapes only)
   void* hp;
   void* dm;
   int* deg;
@@ -738,6 +806,10 @@ BwdWs bwd_ws(const egat_shape& s, void* base) {
   w.scratch = static_cast<int*>(take(E * 4));
   w.lse = static_cast<float*>(take(n * s.H * 4));
   w.delta = static_cast<float*>(take(n * s.H * 4));
+  if (bwd_tc_supported(s)) {
+    void* t = take(bwd_tc_ws_bytes(s));
+    if (b) w.tc = bwd_tc_ws(s, t);
+  }
   w.bytes = o;
   return w;
 }
@@ -746,12 +818,72 @@ BwdWs bwd_ws(const egat_shape& s, void* base) {
 
 size_t backward_ws_bytes(const egat_shape& s) { return bwd_ws(s, nullptr).bytes; }
 
+int launch_exclusive_scan(const int* d_in, int n, int* d_out, cudaStream_t st) {
+  scan_one_cta_kernel<<<1, 1024, 0, st>>>(d_in, n, d_out);
+  return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
+}
+
+// The tiled path (bwd_tc_supported): h' and dm in float32 rounded to tf32,
+// the forward plan (target tiles), the in-lists, then the statistics, target
+// and source passes, the source coupling's adjoint and dL/dr.
+template <int L>
+int launch_backward_tiled(const egat_shape& s, const BwdWs& w, const void* d_h, const float* d_pos,
+                          const void* d_q, const void* d_k, const int32_t* d_nbr,
+                          const int32_t* d_cnt, const int32_t* d_order, const float* d_w1,
+                          const float* d_w2, const float* d_g, float* d_dh, float* d_dq,
+                          float* d_dk, float* d_dpos, cudaStream_t st) {
+  constexpr int D = (L + 1) * (L + 1);
+  const long long vals = (long long)s.n * D * s.C;
+  float* hp = static_cast<float*>(w.hp);
+  float* dm = static_cast<float*>(w.dm);
+  int e = launch_eaas_source_f32out(s, d_h, d_pos, d_w1, hp, st);
+  if (e == EGAT_OK) e = launch_round_tf32(hp, vals, st);
+  if (e == EGAT_OK) e = launch_adjoint<L, float>(s, d_g, d_pos, d_w2, dm, st);
+  if (e == EGAT_OK) e = launch_round_tf32(dm, vals, st);
+  if (e == EGAT_OK) e = launch_build_plan(s.n, s.K, s.lmax, d_nbr, d_cnt, d_order, d_pos, w.tc.plan, st);
+  if (e != EGAT_OK) return e;
+  // in-lists (unsorted: the source plan's union is ordered by its bitmap)
+  if (cudaMemsetAsync(w.deg, 0, size_t(s.n) * 4, st) != cudaSuccess ||
+      cudaMemsetAsync(w.cursor, 0, size_t(s.n) * 4, st) != cudaSuccess)
+    return EGAT_ERR_CUDA;
+  const long long E = (long long)s.n * s.K;
+  const int eb = int((E + 255) / 256);
+  in_degree_kernel<<<eb, 256, 0, st>>>(d_nbr, d_cnt, s.n, s.K, w.deg);
+  scan_one_cta_kernel<<<1, 1024, 0, st>>>(w.deg, s.n, w.ptr);
+  in_fill_kernel<<<eb, 256, 0, st>>>(d_nbr, d_cnt, s.n, s.K, w.ptr, w.cursor, w.in);
+  if (cudaGetLastError() != cudaSuccess) return EGAT_ERR_CUDA;
+  e = launch_backward_tc(s, w.tc, d_q, d_k, hp, dm, d_order, w.ptr, w.in, d_dq, d_dk, st);
+  if (e == EGAT_OK) e = launch_adjoint<L, float>(s, w.tc.dhp, d_pos, d_w1, d_dh, st);
+  if (e != EGAT_OK || !d_dpos) return e;
+  PosGradParams pg;
+  pg.g = d_g;
+  pg.m = w.tc.m;
+  pg.dhp = w.tc.dhp;
+  pg.h = d_h;
+  pg.pos = d_pos;
+  pg.w1 = d_w1;
+  pg.w2 = d_w2;
+  pg.dpos = d_dpos;
+  pg.n = s.n;
+  pg.tab = eaas_table(s.lmax);
+  pg.gen = gen_table();
+  return launch_position_grad<L, __nv_bfloat16>(pg, st);
+}
+
 int launch_backward(const egat_shape& s, const void* d_h, const float* d_pos, const void* d_q,
-                    const void* d_k, const int32_t* d_nbr, const int32_t* d_cnt, const float* d_w1,
-                    const float* d_w2, const float* d_g, void* d_ws, float* d_dh, float* d_dq,
-                    float* d_dk, float* d_dpos, cudaStream_t st) {
+                    const void* d_k, const int32_t* d_nbr, const int32_t* d_cnt,
+                    const int32_t* d_order, const float* d_w1, const float* d_w2, const float* d_g,
+                    void* d_ws, float* d_dh, float* d_dq, float* d_dk, float* d_dpos,
+                    cudaStream_t st) {
   const BwdWs w = bwd_ws(s, d_ws);
   const bool bf = s.dtype == EGAT_BF16;
+  if (bwd_tc_supported(s)) {
+    switch (s.lmax) {
+      case 1: return launch_backward_tiled<1>(s, w, d_h, d_pos, d_q, d_k, d_nbr, d_cnt, d_order, d_w1, d_w2, d_g, d_dh, d_dq, d_dk, d_dpos, st);
+      case 2: return launch_backward_tiled<2>(s, w, d_h, d_pos, d_q, d_k, d_nbr, d_cnt, d_order, d_w1, d_w2, d_g, d_dh, d_dq, d_dk, d_dpos, st);
+      default: return EGAT_ERR_UNSUPPORTED;
+    }
+  }
   // h' = source coupling (forward step 2), in float32
   int e = launch_eaas_source_f32out(s, d_h, d_pos, d_w1, static_cast<float*>(w.hp), st);
   if (e != EGAT_OK) return e;

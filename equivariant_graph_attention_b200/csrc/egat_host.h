@@ -88,9 +88,38 @@ bool tc_attention_supported(const egat_shape& s);
 // Backward pass (gradients of <G, ^h> with respect to h, q, k): workspace and launch.
 size_t backward_ws_bytes(const egat_shape& s);
 int launch_backward(const egat_shape& s, const void* d_h, const float* d_pos, const void* d_q,
-                    const void* d_k, const int32_t* d_nbr, const int32_t* d_cnt, const float* d_w1,
-                    const float* d_w2, const float* d_g, void* d_ws, float* d_dh, float* d_dq,
-                    float* d_dk, float* d_dpos, cudaStream_t st);
+                    const void* d_k, const int32_t* d_nbr, const int32_t* d_cnt,
+                    const int32_t* d_order, const float* d_w1, const float* d_w2, const float* d_g,
+                    void* d_ws, float* d_dh, float* d_dq, float* d_dk, float* d_dpos,
+                    cudaStream_t st);
+// Exclusive scan of in[0..n) into out[0..n] (out[n] = total) by one CTA.
+int launch_exclusive_scan(const int* d_in, int n, int* d_out, cudaStream_t st);
+// Tiled tensor-core backward (bf16 storage, C = 128, H = 16, dk = 16,
+// lmax <= 2): workspace views and launches.
+struct BwdTcWs {
+  float* m;        // m [n][D][C] (the statistics pass)
+  float* dhp;      // dL/dh' [n][D][C]
+  float* stats;    // [n][2][H]: log-sum-exp, Delta
+  void* plan;      // forward plan (target tiles)
+  int* capv;       // [tiles + 1] source tile capacities
+  int* toff;       // [tiles + 1] source tile offsets
+  int* ulen;       // [tiles] source tile union lengths
+  int* uni;        // source tile unions
+  uint32_t* mask;  // source tile membership words
+};
+bool bwd_tc_supported(const egat_shape& s);
+size_t bwd_tc_ws_bytes(const egat_shape& s);
+BwdTcWs bwd_tc_ws(const egat_shape& s, void* base);
+// x (float32, count values, a multiple of 4) rounded to tf32 in place.
+int launch_round_tf32(float* x, long long count, cudaStream_t st);
+// m and the log-sum-exp (statistics pass), dq and Delta (target pass), both
+// over the forward plan's tiles in w.plan; the source plan from the in-lists,
+// dk and dh' (source pass).  d_hp and d_dm float32 rounded to tf32.
+int launch_backward_tc(const egat_shape& s, const BwdTcWs& w, const void* d_q, const void* d_k,
+                       const float* d_hp, const float* d_dm, const int32_t* d_order,
+                       const int* d_in_ptr, const int* d_in, float* d_dq, float* d_dk,
+                       cudaStream_t st);
+int take_wait_timeouts_backward(cudaStream_t st, unsigned int* count);
 // Bounded-wait reports (one per compilation unit with mbarrier waits): read
 // and clear the count of waits that gave up (synchronises st); the self-test
 // launch.

@@ -99,7 +99,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.egat_backward_workspace_bytes.restype = ctypes.c_int
     lib.egat_backward_workspace_bytes.argtypes = [sp, ctypes.POINTER(sz)]
     lib.egat_backward.restype = ctypes.c_int
-    lib.egat_backward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp, vp, vp, vp]
+    lib.egat_backward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp, vp, vp, vp]
     lib.egat_take_device_status.restype = ctypes.c_int
     lib.egat_take_device_status.argtypes = [vp]
     lib.egat_selftest_wait_timeout.restype = ctypes.c_int
@@ -305,9 +305,11 @@ def egat_backward_workspace_bytes(shape: Shape) -> int:
 def egat_backward(shape: Shape, h: torch.Tensor, pos: torch.Tensor, q: torch.Tensor,
                   k: torch.Tensor, nbr: torch.Tensor, cnt: Optional[torch.Tensor],
                   w1: torch.Tensor, w2: torch.Tensor, grad_out: torch.Tensor,
-                  workspace: Optional[torch.Tensor] = None, positions: bool = True, stream=None):
+                  workspace: Optional[torch.Tensor] = None, positions: bool = True,
+                  order: Optional[torch.Tensor] = None, stream=None):
     """(dL/dh, dL/dq, dL/dk, dL/dr) float32 for the upstream gradient grad_out = dL/d^h
-    (dL/dr is None when positions=False)."""
+    (dL/dr is None when positions=False); order = the graph builder's traversal
+    order (tiles of spatially adjacent atoms), optional."""
     nb = egat_backward_workspace_bytes(shape)
     if workspace is None:
         workspace = torch.empty(max(nb, 16), dtype=torch.uint8, device=h.device)
@@ -318,9 +320,9 @@ def egat_backward(shape: Shape, h: torch.Tensor, pos: torch.Tensor, q: torch.Ten
     dpos = torch.empty((shape.n, 3), dtype=torch.float32, device=dev) if positions else None
     cs = shape.c()
     rc = load_library().egat_backward(
-        ctypes.byref(cs), _ptr(h), _ptr(pos), _ptr(q), _ptr(k), _ptr(nbr), _ptr(cnt), _ptr(w1),
-        _ptr(w2), _ptr(grad_out), _ptr(workspace), workspace.numel(), _ptr(dh), _ptr(dq), _ptr(dk),
-        _ptr(dpos), _stream(stream))
+        ctypes.byref(cs), _ptr(h), _ptr(pos), _ptr(q), _ptr(k), _ptr(nbr), _ptr(cnt), _ptr(order),
+        _ptr(w1), _ptr(w2), _ptr(grad_out), _ptr(workspace), workspace.numel(), _ptr(dh), _ptr(dq),
+        _ptr(dk), _ptr(dpos), _stream(stream))
     _check("egat_backward", rc)
     return dh, dq, dk, dpos
 

@@ -286,19 +286,30 @@ EGAT_API int egat_forward_noalloc(const egat_shape* s, const void* d_h, const fl
  *  d_dk    float32 [n][H][dk]  dL/dk
  *  d_dpos  float32 [n][3]      dL/dr (forces are its negative); may be NULL
  * (positions enter through the solid harmonics of both couplings, the
- * neighbour lists held fixed; weight gradients are not computed).  The
- * in-lists (targets served by each atom) are built and sorted inside, so
- * every gradient is a gather in a fixed order: deterministic, no atomics on
- * results.  Padded graphs only (CSR returns EGAT_ERR_UNSUPPORTED), n * K below
- * 2^31; d_ws at least egat_backward_workspace_bytes(s) (h', dL/dm in the
- * storage type, in-lists, per-target statistics).
+ * neighbour lists held fixed; weight gradients are not computed).
+ *  d_order optional int32 [n] traversal order (a permutation, as
+ *          egat_build_graph returns it; NULL = 0..n-1).  It only groups atoms
+ *          into tiles: results do not depend on it up to rounding, speed does.
+ * Shapes of the tensor-core forward path with lmax <= 2 (bf16, C = 128,
+ * H = 16, dk = 16) run tiled passes: the forward kernel unfused (m and the
+ * log-sum-exp), a pass over tiles of 16 targets (dq) and one over tiles of 16
+ * sources and the union of the targets that list them (dk, dL/dh'), with the
+ * gradient products in tf32.  Other shapes gather per target and per source
+ * over sorted in-lists in float32.  Either way every gradient is a sum in a
+ * fixed order: deterministic, no atomics on results.  Padded graphs only (CSR
+ * returns EGAT_ERR_UNSUPPORTED), n * K below 2^31; d_ws at least
+ * egat_backward_workspace_bytes(s) (h', dL/dm, in-lists, per-target
+ * statistics and, on the tiled path, the plans, m and dL/dh').  Errors:
+ * EGAT_ERR_ARG (null or misaligned pointer), EGAT_ERR_WORKSPACE,
+ * EGAT_ERR_UNSUPPORTED, EGAT_ERR_CUDA; a bounded wait that gave up is
+ * reported by egat_take_device_status.
  */
 EGAT_API int egat_backward_workspace_bytes(const egat_shape* s, size_t* bytes);
 EGAT_API int egat_backward(const egat_shape* s, const void* d_h, const float* d_pos, const void* d_q,
                            const void* d_k, const int32_t* d_nbr, const int32_t* d_cnt,
-                           const float* d_w1, const float* d_w2, const float* d_grad_out,
-                           void* d_ws, size_t ws_bytes, float* d_dh, float* d_dq, float* d_dk,
-                           float* d_dpos, void* stream);
+                           const int32_t* d_order, const float* d_w1, const float* d_w2,
+                           const float* d_grad_out, void* d_ws, size_t ws_bytes, float* d_dh,
+                           float* d_dq, float* d_dk, float* d_dpos, void* stream);
 
 /*
  * Device status.  The tensor-core attention kernel waits on mbarriers for its

@@ -93,6 +93,63 @@ def attention_backward(q, k, hp, dm, nbrs: Sequence[np.ndarray]) -> Tuple[np.nda
     return dhp, dq, dk
 
 
+def attention_backward_at(q, k, hp, dm, nbrs, atoms):
+    """``attention_backward`` evaluated at chosen atoms only, for systems too
+    large to differentiate whole.
+
+    For every a in ``atoms``: dL/dq_a (a as a target) and dL/dk_a, dL/dh'_a (a
+    as a source, summed over the targets whose lists hold it).  ``nbrs`` maps
+    an atom i to N(i) (a dict, or a sequence over all atoms) and must hold
+    every atom in ``atoms`` and every target whose list holds one of them;
+    ``hp`` and ``dm`` are read only at the atoms those lists touch.  Returns
+    (dhp [len(atoms), D, C], dq [len(atoms), H, dk], dk [len(atoms), H, dk]).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    C = hp.shape[2]
+    H, dk_ = q.shape[1], q.shape[2]
+    hc = head_of_channel(C, H)
+    member = np.zeros((C, H))
+    member[np.arange(C), hc] = 1.0
+    scale = 1.0 / np.sqrt(dk_)
+    row_cache = {}
+
+    def target_terms(i):
+        # alpha_i. and ds_i. over N(i) (the softmax backward of target i)
+        if i not in row_cache:
+            js = np.asarray(nbrs[i], dtype=np.int64)
+            if js.size == 0:
+                row_cache[i] = (js, None, None)
+            else:
+                a = softmax_two_pass(logits(q[i], k[js]))
+                da = np.einsum("dc,jdc->jc", np.asarray(dm[i], np.float64),
+                               np.asarray(hp[js], np.float64)) @ member
+                row_cache[i] = (js, a, a * (da - (a * da).sum(axis=0, keepdims=True)))
+        return row_cache[i]
+
+    holders = {}
+    keys = nbrs.keys() if isinstance(nbrs, dict) else range(len(nbrs))
+    wanted = set(int(a) for a in atoms)
+    for i in keys:
+        for j in np.asarray(nbrs[i], dtype=np.int64):
+            if int(j) in wanted:
+                holders.setdefault(int(j), []).append(int(i))
+    A = len(atoms)
+    dhp = np.zeros((A,) + hp.shape[1:])
+    dq = np.zeros((A, H, dk_))
+    dk = np.zeros((A, H, dk_))
+    for t, a_ in enumerate(atoms):
+        js, a, ds = target_terms(int(a_))
+        if js.size:
+            dq[t] = np.einsum("jh,jhd->hd", ds, k[js]) * scale
+        for i in holders.get(int(a_), []):
+            js, a, ds = target_terms(i)
+            for pos_in_row in np.nonzero(js == int(a_))[0]:
+                dk[t] += np.einsum("h,hd->hd", ds[pos_in_row], q[i]) * scale
+                dhp[t] += a[pos_in_row][hc][None, :] * np.asarray(dm[i], np.float64)
+    return dhp, dq, dk
+
+
 def backward(h, pos, q, k, w1, w2, lmax: int, nbrs: Sequence[np.ndarray],
              G) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
     """(dL/dh, dL/dq, dL/dk) for L = sum_i <G_i, ^h_i>, ^h = attention.forward."""

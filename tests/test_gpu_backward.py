@@ -4,10 +4,13 @@ pin (tests/test_oracle_backward.py).
 
 dL/dh is compared block by block (the forward's metric); dL/dq and dL/dk row
 by row over (atom, head) and dL/dr row by row over atoms with the same
-relative-norm metric.  Bars as for the
-forward: 1e-4 for float32 storage, 2e-2 for bf16 storage (h' and dL/dm are
-held in bf16 there).  Also: tiny ragged systems with an isolated atom and an
-atom at the origin, and bitwise determinism across calls.
+relative-norm metric.  Bars as for the forward: 1e-4 for float32 storage,
+2e-2 for bf16 storage.  bf16 shapes of the tensor-core forward run the tiled
+passes (tf32 gradient products); they are checked with and without the
+traversal order, on ragged systems of 1 and 37 atoms (an isolated atom, an
+atom at the origin, a ragged last tile) and at full size (32,768 atoms,
+K = 256) on sampled atoms against the oracle evaluated at those atoms.  Also:
+tiny float32 ragged systems, and bitwise determinism across calls.
 """
 import functools
 
@@ -15,7 +18,9 @@ import numpy as np
 import pytest
 import torch
 
-from oracle.backward import backward as oracle_backward, position_grad
+from oracle.attention import aggregate, source_coupling
+from oracle.backward import (attention_backward_at, backward as oracle_backward, coupling_position_grad,
+                             position_grad, tensor_product_adjoint)
 from oracle.graph import radius_graph
 from equivariant_graph_attention_b200 import synth
 from tests.parity_util import TOL, block_rel_error, device_inputs, shape_of
@@ -61,19 +66,20 @@ def _case(name):
     return wl, d, G, ref + (dr,)
 
 
-def _run(wl, d, G):
+def _run(wl, d, G, use_order=True):
     egat = _egat()
     dev = device_inputs(wl, d)
     g = egat.egat_build_graph(dev["pos_q"], wl.cutoff_q, K=wl.K)
     Gd = torch.from_numpy(G).cuda()
     return egat.egat_backward(shape_of(wl), dev["h"], dev["pos"], dev["q"], dev["k"], g["nbr"],
-                              g["cnt"], dev["w1"], dev["w2"], Gd)
+                              g["cnt"], dev["w1"], dev["w2"], Gd,
+                              order=g["order"] if use_order else None)
 
 
-@pytest.mark.parametrize("name", SMALL)
-def test_backward_parity(name):
+@pytest.mark.parametrize("name,use_order", [(n, True) for n in SMALL] + [("uniform4096_l2_bf16", False)])
+def test_backward_parity(name, use_order):
     wl, d, G, (rdh, rdq, rdk, rdr) = _case(name)
-    dh, dq, dk, dr = (x.cpu().numpy() for x in _run(wl, d, G))
+    dh, dq, dk, dr = (x.cpu().numpy() for x in _run(wl, d, G, use_order))
     e_h = block_rel_error(dh, rdh, wl.lmax)
     e_q = row_rel_error(dq, rdq)
     e_k = row_rel_error(dk, rdk)
@@ -118,3 +124,73 @@ def test_backward_edge_cases(lmax):
     assert row_rel_error(dq, rdq) < TOL["f32"] and row_rel_error(dk, rdk) < TOL["f32"]
     # atom 0 sits at the origin (the zero-radius branch of the position gradient)
     assert row_rel_error(dr, rdr) < TOL["f32"]
+
+
+@pytest.mark.parametrize("lmax", [1, 2])
+@pytest.mark.parametrize("n", [1, 37])
+def test_tiled_backward_edge_cases(lmax, n):
+    """The tiled passes on tiny bf16 systems: a single atom (empty unions), and
+    37 atoms (a ragged last tile) with an isolated atom, an atom at the origin
+    and one on the negative z axis."""
+    rng = np.random.default_rng(70 + 3 * lmax + n)
+    pts = rng.uniform(-3.0, 3.0, (n, 3))
+    pts[0] = 0.0
+    if n > 2:
+        pts[1] = [0.0, 0.0, -1.3]
+        pts[2] = [60.0, 60.0, 60.0]        # isolated
+    wl = synth.small_cube(n, 6.0, 3.0, 16, lmax, 128, 16, 16, "bf16")
+    feats = synth.features(wl, seed=n + lmax)
+    pq = np.rint(pts / synth.GRID_QUANTUM).astype(np.int32)
+    feats.update(pos_q=pq, pos=(pq.astype(np.float64) * synth.GRID_QUANTUM).astype(np.float32))
+    G = rng.standard_normal((n, wl.D, wl.C)).astype(np.float32)
+    dh, dq, dk, dr = (x.cpu().numpy() for x in _run(wl, feats, G))
+    lists, _ = radius_graph(pq, wl.cutoff_q, K=wl.K)
+    rdh, rdq, rdk = oracle_backward(feats["h"], feats["pos"], feats["q"], feats["k"], feats["w1"],
+                                    feats["w2"], lmax, lists, G)
+    rdr = position_grad(feats["h"], feats["pos"], feats["q"], feats["k"], feats["w1"],
+                        feats["w2"], lmax, lists, G)
+    if n == 1:
+        assert not dq.any() and not dk.any() and not dh.any() and not dr.any()
+        return
+    assert not dq[2].any() and not dk[2].any() and not dh[2].any() and not dr[2].any()
+    tol = TOL["bf16"]
+    assert block_rel_error(dh, rdh, lmax) < tol
+    assert row_rel_error(dq, rdq) < tol and row_rel_error(dk, rdk) < tol
+    assert row_rel_error(dr, rdr) < tol
+    assert _egat().egat_take_device_status() == _egat().EGAT_OK
+
+
+def test_tiled_backward_full_size_sampled():
+    """32,768 atoms, K = 256, lmax 2, bf16: dL/dq, dL/dk, dL/dh and dL/dr of
+    sampled atoms (random ones, the highest-degree ones, the last atom)
+    against the oracle evaluated at those atoms."""
+    from tests.test_gpu_parity import _full_degree
+    from tests.parity_util import sample_targets
+    name = "uniform32768_K256_l2_bf16"
+    wl = synth.WORKLOADS[name]
+    d = synth.make(wl)
+    G = np.random.default_rng(17).standard_normal((wl.n, wl.D, wl.C)).astype(np.float32)
+    dh, dq, dk, dr = (x.cpu().numpy() for x in _run(wl, d, G))
+    atoms = sample_targets(wl, _full_degree(name), count=12, seed=9)
+    # every target whose list may hold a sampled atom lies within the cutoff of it
+    first, _ = radius_graph(d["pos_q"], wl.cutoff_q, rows=atoms)
+    cand = sorted(set(atoms) | {int(j) for js in first for j in js})
+    rows, _ = radius_graph(d["pos_q"], wl.cutoff_q, K=wl.K, rows=cand)
+    nbrs = dict(zip(cand, rows))
+    touched = np.array(sorted(set(cand) | {int(j) for js in rows for j in js}))
+    hp = np.zeros((wl.n, wl.D, wl.C))
+    dm = np.zeros((wl.n, wl.D, wl.C))
+    hp[touched] = source_coupling(d["h"][touched], d["pos"][touched], d["w1"], wl.lmax)
+    dm[cand] = tensor_product_adjoint(G[cand], d["pos"][cand], d["w2"], wl.lmax)
+    rdhp, rdq, rdk = attention_backward_at(d["q"], d["k"], hp, dm, nbrs, atoms)
+    rdh = tensor_product_adjoint(rdhp, d["pos"][atoms], d["w1"], wl.lmax)
+    # dL/dr: the target coupling's part (G, m) plus the source coupling's (dh', h)
+    a_idx = np.array(atoms)
+    m = aggregate(d["q"], d["k"], hp, [nbrs[a] for a in atoms], targets=atoms)
+    rdr = (coupling_position_grad(G[a_idx], m, d["pos"][a_idx], d["w2"], wl.lmax)
+           + coupling_position_grad(rdhp, d["h"][a_idx], d["pos"][a_idx], d["w1"], wl.lmax))
+    tol = TOL["bf16"]
+    e = (block_rel_error(dh[a_idx], rdh, wl.lmax), row_rel_error(dq[a_idx], rdq),
+         row_rel_error(dk[a_idx], rdk), row_rel_error(dr[a_idx], rdr))
+    print(f"backward {name} sampled: dh {e[0]:.2e}  dq {e[1]:.2e}  dk {e[2]:.2e}  dr {e[3]:.2e}")
+    assert max(e) < tol

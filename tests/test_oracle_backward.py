@@ -9,13 +9,18 @@
 * Two special cases: a zero upstream gradient gives zero gradients, and a
   target with a single neighbour (alpha = 1 identically) passes dL/dm straight
   to that neighbour's h' with no logit gradient.
+* The evaluation at chosen atoms (attention_backward_at, for systems too
+  large to differentiate whole) agrees with the whole-system attention
+  backward at those atoms, whose neighbour lists are given as a dict holding
+  only what it needs.
 """
 import numpy as np
 import pytest
 
 from oracle import so3
 from oracle.attention import forward, tensor_product
-from oracle.backward import attention_backward, backward, position_grad, tensor_product_adjoint
+from oracle.backward import (attention_backward, attention_backward_at, backward, position_grad,
+                             tensor_product_adjoint)
 from oracle.graph import radius_graph
 
 
@@ -129,3 +134,23 @@ def test_position_gradient_matches_finite_differences(seed):
             dn[a, c] -= eps
             fd = (_loss(s, pos=up) - _loss(s, pos=dn)) / (2 * eps)
             assert abs(fd - grad[a, c]) <= 1e-5 * (1.0 + abs(fd)), (a, c, fd, grad[a, c])
+
+
+def test_backward_at_chosen_atoms_matches_whole_system():
+    rng = np.random.default_rng(11)
+    n, D, C, H, dk = 40, 4, 8, 2, 4
+    pos_q = rng.integers(-4 << 16, 4 << 16, size=(n, 3), dtype=np.int64).astype(np.int32)
+    lists, _ = radius_graph(pos_q, 3 << 16, K=7)
+    q = rng.standard_normal((n, H, dk))
+    k = rng.standard_normal((n, H, dk))
+    hp = rng.standard_normal((n, D, C))
+    dm = rng.standard_normal((n, D, C))
+    dhp, dq, dk_ = attention_backward(q, k, hp, dm, lists)
+    atoms = [0, 7, 19, n - 1]
+    need = set(atoms) | {i for i in range(n) if set(lists[i].tolist()) & set(atoms)}
+    sub = {i: lists[i] for i in need}
+    a_dhp, a_dq, a_dk = attention_backward_at(q, k, hp, dm, sub, atoms)
+    assert np.abs(a_dhp - dhp[atoms]).max() <= 1e-12 * max(1.0, np.abs(dhp).max())
+    assert np.abs(a_dq - dq[atoms]).max() <= 1e-12 * max(1.0, np.abs(dq).max())
+    assert np.abs(a_dk - dk_[atoms]).max() <= 1e-12 * max(1.0, np.abs(dk_).max())
+    assert np.abs(dk_[atoms]).max() > 0 and np.abs(dq[atoms]).max() > 0
