@@ -52,7 +52,15 @@ constexpr int kBwdWarps = 4;   // (3 CTAs per SM for the attention passes: no sp
 constexpr int kSortCap = 4096;   // in-list length sorted in shared memory
 
 // ---------------------------------------------------------------- step 1
-template <int L, typename T>
+// float -> the nearest tf32 value (ties away), as a float
+__device__ __forceinline__ float round_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;\n" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
+// TF32: the result rounded to tf32 (the tiled passes' operand format)
+template <int L, typename T, bool TF32 = false>
 __global__ void __launch_bounds__(kBwdWarps * 32)
 adjoint_coupling_kernel(const float* __restrict__ g, const float* __restrict__ pos,
                         const float* __restrict__ w, T* __restrict__ out, int n, int C,
@@ -76,7 +84,9 @@ adjoint_coupling_kernel(const float* __restrict__ g, const float* __restrict__ p
 #pragma unroll
     for (int d = 0; d < D; ++d) x[d] = g[((size_t)a * D + d) * C + c];
     eaas_channel_adjoint<L>(x, Dsm[wib], rpow, tab, [&](int pp) { return __ldg(w + pp * C + c); },
-                            [&](int d, float v) { store_one<T>(out + ((size_t)a * D + d) * C + c, v); });
+                            [&](int d, float v) {
+                              store_one<T>(out + ((size_t)a * D + d) * C + c, TF32 ? round_tf32(v) : v);
+                            });
   }
 }
 
@@ -96,29 +106,43 @@ __global__ void in_degree_kernel(const int32_t* __restrict__ nbr, const int32_t*
   if ((unsigned)j < (unsigned)n) atomicAdd(&deg[j], 1);
 }
 
-// exclusive scan of deg[0..n) into ptr[0..n] by one CTA (chunk per thread)
+// exclusive scan of deg[0..n) into ptr[0..n] by one CTA: tiles of 1024
+// consecutive entries (coalesced), a warp-shuffle scan per tile, the running
+// total carried between tiles; the next tile's loads are issued before the
+// current tile's scan
 __global__ void __launch_bounds__(1024) scan_one_cta_kernel(const int* __restrict__ deg, int n,
                                                            int* __restrict__ ptr) {
-  __shared__ int part[1024];
-  const int t = threadIdx.x;
-  const int per = (n + 1023) / 1024;
-  const int b0 = min(t * per, n), b1 = min(b0 + per, n);
-  int sum = 0;
-  for (int k = b0; k < b1; ++k) sum += deg[k];
-  part[t] = sum;
-  __syncthreads();
-  for (int o = 1; o < 1024; o <<= 1) {
-    const int v = t >= o ? part[t - o] : 0;
+  __shared__ int wsum[32];
+  const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
+  int carry = 0;
+  int v = t < n ? deg[t] : 0;
+  for (int base = 0; base < n; base += 1024) {
+    const int nxt = base + 1024 + t;
+    const int vn = nxt < n ? deg[nxt] : 0;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[wid] = x;
     __syncthreads();
-    part[t] += v;
+    if (wid == 0) {
+      int s = wsum[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, s, o);
+        if (lane >= o) s += y;
+      }
+      wsum[lane] = s;
+    }
     __syncthreads();
+    if (base + t < n) ptr[base + t] = carry + (wid ? wsum[wid - 1] : 0) + x - v;
+    carry += wsum[31];
+    __syncthreads();   // wsum is rewritten by the next tile
+    v = vn;
   }
-  int run = t ? part[t - 1] : 0;
-  for (int k = b0; k < b1; ++k) {
-    ptr[k] = run;
-    run += deg[k];
-  }
-  if (t == 1023) ptr[n] = part[1023];
+  if (t == 0) ptr[n] = carry;
 }
 
 __global__ void in_fill_kernel(const int32_t* __restrict__ nbr, const int32_t* __restrict__ cnt,
@@ -605,52 +629,109 @@ struct PosGradParams {
   GenTable gen;
 };
 
+constexpr int kPgWarps = 8;
+
+// One warp per atom; both parts share the atom's rotation and Wigner-D, and
+// every lane reads its channels' columns straight from global memory (lanes
+// take consecutive channels: coalesced).
 template <int L, int C, typename T>
-__global__ void __launch_bounds__(kBwdWarps * 32) position_grad_kernel(const __grid_constant__ PosGradParams p) {
+__global__ void __launch_bounds__(kPgWarps * 32) position_grad_kernel(const __grid_constant__ PosGradParams p) {
   constexpr int D = (L + 1) * (L + 1);
   constexpr int WS = wig_size(L);
-  extern __shared__ float smem[];
+  __shared__ float Dall[kPgWarps][WS];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  const int a = blockIdx.x * kBwdWarps + wib;
+  const int a = blockIdx.x * kPgWarps + wib;
   if (a >= p.n) return;   // whole warp
-  float* gs = smem + wib * (2 * D * C + WS);
-  float* xs = gs + D * C;
-  float* Dsm = xs + D * C;
-  const float r[3] = {p.pos[3 * a], p.pos[3 * a + 1], p.pos[3 * a + 2]};
-  for (int e = lane; e < D * C; e += 32) {
-    gs[e] = p.g[(size_t)a * D * C + e];
-    xs[e] = p.m[(size_t)a * D * C + e];
+  float* Dsm = Dall[wib];
+  const float* Gr = p.g + (size_t)a * D * C;
+  const float* Mr = p.m + (size_t)a * D * C;
+  const float* Sr = p.dhp + (size_t)a * D * C;
+  const T* Xr = static_cast<const T*>(p.h) + (size_t)a * D * C;
+  const float r0 = p.pos[3 * a], r1 = p.pos[3 * a + 1], r2 = p.pos[3 * a + 2];
+  const float rho = sqrtf(r0 * r0 + r1 * r1 + r2 * r2);
+  float out[3];
+  if (rho > 0.f) {
+    float Q[9];
+    alignment_rotation(r0, r1, r2, Q);
+    wigner_build<L>(Q, Dsm, lane, 32, [] { __syncwarp(); });
+    __syncwarp();
+    float rpow[L + 1], drpow[L + 1];
+    rpow[0] = 1.f;
+    drpow[0] = 0.f;
+#pragma unroll
+    for (int l = 1; l <= L; ++l) {
+      rpow[l] = rpow[l - 1] * rho;
+      drpow[l] = float(l) * rpow[l - 1];
+    }
+    float dr = 0.f, tx = 0.f, ty = 0.f;
+    for (int c = lane; c < C; c += 32) {
+      float g[D], x[D];
+      // the target coupling's part: g = G_a, x = m_a, weights w2
+#pragma unroll
+      for (int d = 0; d < D; ++d) {
+        g[d] = __ldg(Gr + d * C + c);
+        x[d] = __ldg(Mr + d * C + c);
+      }
+      coupling_grad_channel<L>(g, x, Dsm, rpow, drpow, p.tab, p.gen,
+                               [&](int pp) { return __ldg(p.w2 + pp * C + c); }, dr, tx, ty);
+      // the source coupling's part: g = dh'_a, x = h_a, weights w1
+#pragma unroll
+      for (int d = 0; d < D; ++d) {
+        g[d] = __ldg(Sr + d * C + c);
+        x[d] = load_one<T>(Xr + d * C + c);
+      }
+      coupling_grad_channel<L>(g, x, Dsm, rpow, drpow, p.tab, p.gen,
+                               [&](int pp) { return __ldg(p.w1 + pp * C + c); }, dr, tx, ty);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      dr += __shfl_xor_sync(0xffffffffu, dr, o);
+      tx += __shfl_xor_sync(0xffffffffu, tx, o);
+      ty += __shfl_xor_sync(0xffffffffu, ty, o);
+    }
+    // grad = Q ( -ty / rho, tx / rho, dr ): back from the aligned frame
+    const float v0 = -ty / rho, v1 = tx / rho, v2 = dr;
+#pragma unroll
+    for (int e = 0; e < 3; ++e) out[e] = Q[3 * e] * v0 + Q[3 * e + 1] * v1 + Q[3 * e + 2] * v2;
+  } else {
+    // at r = 0: the derivative along axis e is the coupling at r = e_e with
+    // the degree-1 paths alone (R^1 is linear), both parts
+    float rpow1[L + 1];
+#pragma unroll
+    for (int l = 0; l <= L; ++l) rpow1[l] = l == 1 ? 1.f : 0.f;
+    for (int e = 0; e < 3; ++e) {
+      float Q[9];
+      alignment_rotation(e == 0 ? 1.f : 0.f, e == 1 ? 1.f : 0.f, e == 2 ? 1.f : 0.f, Q);
+      __syncwarp();
+      wigner_build<L>(Q, Dsm, lane, 32, [] { __syncwarp(); });
+      __syncwarp();
+      float sum = 0.f;
+      for (int c = lane; c < C; c += 32) {
+        float t[D];
+#pragma unroll
+        for (int d = 0; d < D; ++d) t[d] = __ldg(Mr + d * C + c);
+        eaas_channel<L>(t, Dsm, rpow1, p.tab, [&](int pp) { return __ldg(p.w2 + pp * C + c); },
+                        [&](int d, float v) { sum = fmaf(__ldg(Gr + d * C + c), v, sum); });
+#pragma unroll
+        for (int d = 0; d < D; ++d) t[d] = load_one<T>(Xr + d * C + c);
+        eaas_channel<L>(t, Dsm, rpow1, p.tab, [&](int pp) { return __ldg(p.w1 + pp * C + c); },
+                        [&](int d, float v) { sum = fmaf(__ldg(Sr + d * C + c), v, sum); });
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      out[e] = sum;
+    }
   }
-  __syncwarp();
-  float gt[3], gsrc[3];
-  atom_position_grad<L, C>(gs, xs, Dsm, r, p.tab, p.gen,
-                           [&](int pp, int c) { return __ldg(p.w2 + pp * C + c); }, lane, gt);
-  __syncwarp();
-  const T* hr = static_cast<const T*>(p.h) + (size_t)a * D * C;
-  for (int e = lane; e < D * C; e += 32) {
-    gs[e] = p.dhp[(size_t)a * D * C + e];
-    xs[e] = load_one<T>(hr + e);
-  }
-  __syncwarp();
-  atom_position_grad<L, C>(gs, xs, Dsm, r, p.tab, p.gen,
-                           [&](int pp, int c) { return __ldg(p.w1 + pp * C + c); }, lane, gsrc);
   if (lane == 0) {
-    p.dpos[3 * a] = gt[0] + gsrc[0];
-    p.dpos[3 * a + 1] = gt[1] + gsrc[1];
-    p.dpos[3 * a + 2] = gt[2] + gsrc[2];
+    p.dpos[3 * a] = out[0];
+    p.dpos[3 * a + 1] = out[1];
+    p.dpos[3 * a + 2] = out[2];
   }
 }
 
 template <int L, typename T>
 int launch_position_grad(const PosGradParams& p, cudaStream_t st) {
-  constexpr int C = 128;
-  constexpr int D = (L + 1) * (L + 1);
-  const size_t shm = size_t(kBwdWarps) * (2 * D * C + wig_size(L)) * sizeof(float);
-  auto kern = position_grad_kernel<L, C, T>;
-  if (shm > 48 * 1024 &&
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(shm)) != cudaSuccess)
-    return EGAT_ERR_CUDA;
-  kern<<<(p.n + kBwdWarps - 1) / kBwdWarps, kBwdWarps * 32, shm, st>>>(p);
+  position_grad_kernel<L, 128, T><<<(p.n + kPgWarps - 1) / kPgWarps, kPgWarps * 32, 0, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
 }
 
@@ -688,12 +769,12 @@ int dispatch_c(const BwdParams& p, int C, cudaStream_t st) {
   }
 }
 
-template <int L, typename T>
+template <int L, typename T, bool TF32 = false>
 int launch_adjoint(const egat_shape& s, const float* g, const float* pos, const float* w, void* out,
                    cudaStream_t st) {
   const int grid = (s.n + kBwdWarps - 1) / kBwdWarps;
-  adjoint_coupling_kernel<L, T><<<grid, kBwdWarps * 32, 0, st>>>(g, pos, w, static_cast<T*>(out), s.n,
-                                                                s.C, eaas_table(L));
+  adjoint_coupling_kernel<L, T, TF32><<<grid, kBwdWarps * 32, 0, st>>>(g, pos, w, static_cast<T*>(out),
+                                                                      s.n, s.C, eaas_table(L));
   return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
 }
 
@@ -823,7 +904,8 @@ int launch_exclusive_scan(const int* d_in, int n, int* d_out, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
 }
 
-// The tiled path (bwd_tc_supported): h' and dm in float32 rounded to tf32,
+// The tiled path (bwd_tc_supported): h' and dm in float32 rounded to tf32
+// as they are stored,
 // the forward plan (target tiles), the in-lists, then the statistics, target
 // and source passes, the source coupling's adjoint and dL/dr.
 template <int L>
@@ -832,14 +914,10 @@ int launch_backward_tiled(const egat_shape& s, const BwdWs& w, const void* d_h, 
                           const int32_t* d_cnt, const int32_t* d_order, const float* d_w1,
                           const float* d_w2, const float* d_g, float* d_dh, float* d_dq,
                           float* d_dk, float* d_dpos, cudaStream_t st) {
-  constexpr int D = (L + 1) * (L + 1);
-  const long long vals = (long long)s.n * D * s.C;
   float* hp = static_cast<float*>(w.hp);
   float* dm = static_cast<float*>(w.dm);
-  int e = launch_eaas_source_f32out(s, d_h, d_pos, d_w1, hp, st);
-  if (e == EGAT_OK) e = launch_round_tf32(hp, vals, st);
-  if (e == EGAT_OK) e = launch_adjoint<L, float>(s, d_g, d_pos, d_w2, dm, st);
-  if (e == EGAT_OK) e = launch_round_tf32(dm, vals, st);
+  int e = launch_eaas_source_f32out(s, d_h, d_pos, d_w1, hp, st, true);
+  if (e == EGAT_OK) e = launch_adjoint<L, float, true>(s, d_g, d_pos, d_w2, dm, st);
   if (e == EGAT_OK) e = launch_build_plan(s.n, s.K, s.lmax, d_nbr, d_cnt, d_order, d_pos, w.tc.plan, st);
   if (e != EGAT_OK) return e;
   // in-lists (unsorted: the source plan's union is ordered by its bitmap)

@@ -479,18 +479,21 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_target_tc_kernel(const __gri
       // dalpha for the tile's 16 targets x these 8 union atoms
       float dp[4] = {0.f, 0.f, 0.f, 0.f};
       const uint32_t hb = smem_u32(fb + (8 * nt + (lane & 7)) * FSTR + h * 32 + ((lane >> 3) & 1) * 16);
+      float dp2[4] = {0.f, 0.f, 0.f, 0.f};   // odd components: a second, independent chain
 #pragma unroll
       for (int d = 0; d + 1 < D; d += 2) {
         uint32_t r[4];
         ldsm_x4(r, hb + (d + (lane >> 4)) * (kBC * 4));
         mma_tf32(dp, dma[d], r[0], r[1]);
-        mma_tf32(dp, dma[d + 1], r[2], r[3]);
+        mma_tf32(dp2, dma[d + 1], r[2], r[3]);
       }
       if constexpr (D % 2) {
         uint32_t r[2];
         ldsm_x2(r, hb + (D - 1) * (kBC * 4));
         mma_tf32(dp, dma[D - 1], r[0], r[1]);
       }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) dp[e] += dp2[e];
       float E[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) E[e] = P[e] * dp[e];
@@ -621,18 +624,21 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_source_tc_kernel(const __gri
       P[3] = (w1 & 2u) ? fast_exp2(fmaf(s[3], qs, -lsb)) : 0.f;
       float dp[4] = {0.f, 0.f, 0.f, 0.f};
       const uint32_t db = smem_u32(fb + (8 * nt + (lane & 7)) * FSTR + h * 32 + ((lane >> 3) & 1) * 16);
+      float dp2[4] = {0.f, 0.f, 0.f, 0.f};   // odd components: a second, independent chain
 #pragma unroll
       for (int d = 0; d + 1 < D; d += 2) {
         uint32_t r[4];
         ldsm_x4(r, db + (d + (lane >> 4)) * (kBC * 4));
         mma_tf32(dp, ha[d], r[0], r[1]);
-        mma_tf32(dp, ha[d + 1], r[2], r[3]);
+        mma_tf32(dp2, ha[d + 1], r[2], r[3]);
       }
       if constexpr (D % 2) {
         uint32_t r[2];
         ldsm_x2(r, db + (D - 1) * (kBC * 4));
         mma_tf32(dp, ha[D - 1], r[0], r[1]);
       }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) dp[e] += dp2[e];
       float ds[4];
       ds[0] = P[0] * (dp[0] - dla);
       ds[1] = P[1] * (dp[1] - dlb);
@@ -786,19 +792,6 @@ __global__ void __launch_bounds__(kCsrPlanThreads) build_csr_plan_kernel(const _
   });
 }
 
-// h' and dm (float32) rounded to tf32 in place: the operands of the
-// gradient products, read as tf32 bit patterns without further conversion.
-__global__ void round_tf32_kernel(float4* __restrict__ x, long long count4) {
-  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= count4) return;
-  float4 v = x[i];
-  v.x = __uint_as_float(to_tf32(v.x));
-  v.y = __uint_as_float(to_tf32(v.y));
-  v.z = __uint_as_float(to_tf32(v.z));
-  v.w = __uint_as_float(to_tf32(v.w));
-  x[i] = v;
-}
-
 enum PassKind { kStatsPass, kTargetPass, kSourcePass };
 
 template <int L>
@@ -866,14 +859,6 @@ BwdTcWs bwd_tc_ws(const egat_shape& s, void* base) {
   w.uni = static_cast<int*>(take(ucap * 4));
   w.mask = static_cast<uint32_t*>(take(ucap / 2 * 4));
   return w;
-}
-
-int launch_round_tf32(float* x, long long count, cudaStream_t st) {
-  if (count % 4) return EGAT_ERR_ARG;
-  const long long c4 = count / 4;
-  const int blocks = int((c4 + 255) / 256);
-  if (blocks > 0) round_tf32_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<float4*>(x), c4);
-  return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
 }
 
 int launch_backward_tc(const egat_shape& s, const BwdTcWs& w, const void* d_q, const void* d_k,

@@ -174,6 +174,28 @@ struct ChanVec<float, 2> {
   }
 };
 
+// float32 stores rounded to tf32 (round to nearest, ties away): the operand
+// format of the backward's tf32 products, so they read the bits unconverted.
+// One float wide, so that pointer arithmetic on it steps in floats.
+struct Tf32Out {
+  float v;
+};
+static_assert(sizeof(Tf32Out) == sizeof(float) && alignof(Tf32Out) == alignof(float), "Tf32Out is a float");
+__device__ __forceinline__ float round_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;\n" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+template <int N>
+struct ChanVec<Tf32Out, N> {
+  static __device__ __forceinline__ void store(Tf32Out* p, const float (&v)[N]) {
+    float w[N];
+#pragma unroll
+    for (int e = 0; e < N; ++e) w[e] = round_tf32(v[e]);
+    ChanVec<float, N>::store(reinterpret_cast<float*>(p), w);
+  }
+};
+
 // A group of G = C/CPL lanes owns one atom; each lane owns CPL consecutive
 // channels (CPL = 4 up to lmax 2, 2 at lmax 3 for the register budget), so
 // component rows move in 8-16 byte vectors.  The group builds the atom's
@@ -480,9 +502,19 @@ int launch_eaas_tile(const egat_shape& s, const void* d_x, const float* rec, lon
 }
 
 int launch_eaas_source_f32out(const egat_shape& s, const void* d_x, const float* d_pos,
-                              const float* d_w, float* d_y, cudaStream_t st) {
+                              const float* d_w, float* d_y, cudaStream_t st, bool tf32) {
   const bool bf = s.dtype == EGAT_BF16;
   const long long n = s.n;
+  if (tf32) {
+    Tf32Out* y = reinterpret_cast<Tf32Out*>(d_y);
+    switch (s.lmax) {
+      case 1: return bf ? launch_eaas_t<1, __nv_bfloat16, false, Tf32Out>(s, d_x, d_pos, nullptr, n, d_w, y, st)
+                        : launch_eaas_t<1, float, false, Tf32Out>(s, d_x, d_pos, nullptr, n, d_w, y, st);
+      case 2: return bf ? launch_eaas_t<2, __nv_bfloat16, false, Tf32Out>(s, d_x, d_pos, nullptr, n, d_w, y, st)
+                        : launch_eaas_t<2, float, false, Tf32Out>(s, d_x, d_pos, nullptr, n, d_w, y, st);
+      default: return EGAT_ERR_UNSUPPORTED;
+    }
+  }
   switch (s.lmax) {
     case 1: return bf ? launch_eaas_t<1, __nv_bfloat16, false, float>(s, d_x, d_pos, nullptr, n, d_w, d_y, st)
                       : launch_eaas_t<1, float, false>(s, d_x, d_pos, nullptr, n, d_w, d_y, st);

@@ -76,9 +76,10 @@ PlanView plan_view(void* base, int n, int K, int lmax);
 int launch_build_plan(int n, int K, int lmax, const int32_t* d_nbr, const int32_t* d_cnt,
                       const int32_t* d_order, const float* d_pos, void* d_plan, cudaStream_t st);
 // Step 2 with a float32 result whatever the storage type (the backward pass
-// keeps its intermediates in float32).
+// keeps its intermediates in float32); tf32 = true rounds the stored values
+// to tf32 (lmax <= 2).
 int launch_eaas_source_f32out(const egat_shape& s, const void* d_x, const float* d_pos,
-                              const float* d_w, float* d_y, cudaStream_t st);
+                              const float* d_w, float* d_y, cudaStream_t st, bool tf32 = false);
 // Step 2 for every atom listed in a plan's tile records, rotations from them.
 int launch_eaas_planned(const egat_shape& s, const void* d_x, const void* d_plan, const float* d_w,
                         void* d_y, cudaStream_t st);
@@ -110,8 +111,6 @@ struct BwdTcWs {
 bool bwd_tc_supported(const egat_shape& s);
 size_t bwd_tc_ws_bytes(const egat_shape& s);
 BwdTcWs bwd_tc_ws(const egat_shape& s, void* base);
-// x (float32, count values, a multiple of 4) rounded to tf32 in place.
-int launch_round_tf32(float* x, long long count, cudaStream_t st);
 // m and the log-sum-exp (statistics pass), dq and Delta (target pass), both
 // over the forward plan's tiles in w.plan; the source plan from the in-lists,
 // dk and dh' (source pass).  d_hp and d_dm float32 rounded to tf32.
