@@ -303,8 +303,9 @@ eaas_source_kernel(const __grid_constant__ EaasParams p) {
 template <int L, typename T>
 struct TileSmem {
   static constexpr int D = (L + 1) * (L + 1);
-  static constexpr int CPL = L >= 3 ? 2 : 4;
-  static constexpr int C = 32 * CPL;
+  static constexpr int CPL = L >= 3 ? 2 : 4;    // channels per lane in one pass over a slot
+  static constexpr int C = 128;
+  static constexpr int HALVES = C / (32 * CPL); // passes per slot (2 at lmax 3)
   static constexpr int ROWB = D * C * int(sizeof(T));
   static constexpr int REC = plan_record_words(L);
   static constexpr size_t rows = 0;                                       // [2][16][ROWB]
@@ -316,13 +317,15 @@ struct TileSmem {
 };
 
 // half a tile's warps per CTA, two CTAs per SM: one CTA's per-tile barrier
-// overlaps the other's work
+// overlaps the other's work (one CTA per SM at lmax 3, whose rows fill the
+// shared memory)
 constexpr int kHalfWarps = kTileM / 2;
 template <int L, typename T>
-__global__ void __launch_bounds__(kHalfWarps * 32, 2)
+__global__ void __launch_bounds__(kHalfWarps * 32, L >= 3 ? 1 : 2)
 eaas_tile_kernel(const __grid_constant__ EaasParams p) {
   using Sm = TileSmem<L, T>;
   constexpr int D = Sm::D, CPL = Sm::CPL, C = Sm::C, ROWB = Sm::ROWB, REC = Sm::REC;
+  constexpr int HALVES = Sm::HALVES;
   constexpr int WS = wig_size(L);
   constexpr int NP = num_paths(L);
   extern __shared__ __align__(128) unsigned char smem[];
@@ -392,23 +395,27 @@ eaas_tile_kernel(const __grid_constant__ EaasParams p) {
     for (int w = wfirst; w < kTileM; w += kHalfWarps) {   // two slots per warp
     const int at = reinterpret_cast<const int*>(rec)[kRecTgt + w];
     if ((unsigned)at < (unsigned)p.n) {
-      const T* xr = reinterpret_cast<const T*>(rows + (size_t(wb) * kTileM + w) * ROWB) + lane * CPL;
-      float xv[CPL][D];
-#pragma unroll
-      for (int d = 0; d < D; ++d) {
-        float v[CPL];
-        ChanVec<T, CPL>::load_shared(xr + d * C, v);
-#pragma unroll
-        for (int k = 0; k < CPL; ++k) xv[k][d] = v[k];
-      }
       float rpow[L + 1];
 #pragma unroll
       for (int l = 0; l <= L; ++l) rpow[l] = rec[kRecRp + w * (L + 1) + l];
-      T* yr = y + (size_t)at * D * C + lane * CPL;
-      const float* swc = sw + lane * CPL;
-      eaas_multi<L, CPL>(xv, rec + rec_off_D(L) + w * WS, rpow, p.tab,
-                         [&](int q, int k) { return swc[q * C + k]; },
-                         [&](int d, const float (&v)[CPL]) { ChanVec<T, CPL>::store(yr + d * C, v); });
+#pragma unroll 1
+      for (int hf = 0; hf < HALVES; ++hf) {
+        const int c0 = (hf * 32 + lane) * CPL;   // this lane's first channel in this pass
+        const T* xr = reinterpret_cast<const T*>(rows + (size_t(wb) * kTileM + w) * ROWB) + c0;
+        float xv[CPL][D];
+#pragma unroll
+        for (int d = 0; d < D; ++d) {
+          float v[CPL];
+          ChanVec<T, CPL>::load_shared(xr + d * C, v);
+#pragma unroll
+          for (int k = 0; k < CPL; ++k) xv[k][d] = v[k];
+        }
+        T* yr = y + (size_t)at * D * C + c0;
+        const float* swc = sw + c0;
+        eaas_multi<L, CPL>(xv, rec + rec_off_D(L) + w * WS, rpow, p.tab,
+                           [&](int q, int k) { return swc[q * C + k]; },
+                           [&](int d, const float (&v)[CPL]) { ChanVec<T, CPL>::store(yr + d * C, v); });
+      }
     }
     }
     __syncthreads();   // rows[wb] and recs[rb] are refilled one and two tiles ahead
@@ -496,7 +503,9 @@ int launch_eaas_tile(const egat_shape& s, const void* d_x, const float* rec, lon
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int tiles = int(items / kTileM);
-  const int grid = tiles < 2 * sms ? tiles : 2 * sms;
+  // two CTAs per SM while two fit in shared memory (lmax <= 2), else one
+  const int per_sm = 2 * shmem <= 227 * 1024 ? 2 : 1;
+  const int grid = tiles < per_sm * sms ? tiles : per_sm * sms;
   kern<<<grid, kHalfWarps * 32, shmem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
 }
@@ -538,6 +547,10 @@ int launch_eaas_planned(const egat_shape& s, const void* d_x, const void* d_plan
     return bf ? launch_eaas_tile<2, __nv_bfloat16>(s, d_x, pv.rec, items, d_w, d_y, st)
               : launch_eaas_tile<2, float>(s, d_x, pv.rec, items, d_w, d_y, st);
   }
+  // lmax 3, bf16: the same kernel, each slot in two channel halves (float32
+  // rows of 8 KB would not fit two tiles of 16 in shared memory)
+  if (s.lmax == 3 && bf && s.C == 128)
+    return launch_eaas_tile<3, __nv_bfloat16>(s, d_x, pv.rec, items, d_w, d_y, st);
   switch (s.lmax) {
     case 1: return bf ? launch_eaas_t<1, __nv_bfloat16, true>(s, d_x, nullptr, pv.rec, items, d_w, d_y, st)
                       : launch_eaas_t<1, float, true>(s, d_x, nullptr, pv.rec, items, d_w, d_y, st);
