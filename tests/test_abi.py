@@ -137,3 +137,45 @@ def test_plan_and_status_entry_validation(lib):
     assert lib.egat_selftest_wait_timeout(0, None) == egat.EGAT_ERR_ARG
     assert lib.egat_selftest_wait_timeout((1 << 20) + 1, None) == egat.EGAT_ERR_ARG
     assert lib.egat_strerror(egat.EGAT_ERR_TIMEOUT).startswith(b"a bounded device wait")
+
+
+def test_backward_entry_validation(lib):
+    """egat_backward's host checks and workspace query (no launch on these paths)."""
+    a256 = lambda x: (x + 255) // 256 * 256
+    n, K, H, D, C = 32768, 256, 16, 9, 128
+    s = egat.Shape(n=n, lmax=2, C=C, H=H, dk=16, K=K, dtype="bf16")
+    tiles = n // 16
+    ucap = n * K + 32 * tiles
+    per_edge = (2 * a256(n * D * C * 4) + a256(n * 4) + a256((n + 1) * 4) + a256(n * 4)
+                + 2 * a256(n * K * 4) + 2 * a256(n * H * 4))
+    tiled = (2 * a256(n * D * C * 4) + a256(n * 2 * H * 4) + egat.egat_attention_plan_bytes(s)
+             + 3 * a256((tiles + 1) * 4) + a256(ucap * 4) + a256(ucap // 2 * 4))
+    # the tensor-core shape reserves the tiled passes' buffers (m, dL/dh', statistics, the forward
+    # plan and the source plan at n*K + 32 per tile union entries) on top of the gather path's
+    assert egat.egat_backward_workspace_bytes(s) == per_edge + a256(tiled)
+    f32 = egat.Shape(n=648, lmax=2, C=C, H=H, dk=16, K=64, dtype="f32")
+    assert egat.egat_backward_workspace_bytes(f32) == (
+        2 * a256(648 * D * C * 4) + a256(648 * 4) + a256(649 * 4) + a256(648 * 4)
+        + 2 * a256(648 * 64 * 4) + 2 * a256(648 * H * 4))
+
+    cs = egat.Shape(n=10, lmax=2, C=C, H=H, dk=16, K=64, dtype="bf16").c()
+    ok = ctypes.c_void_p(0x10000)
+    odd4 = ctypes.c_void_p(0x10002)    # not 4-byte aligned
+    odd16 = ctypes.c_void_p(0x10008)   # not 16-byte aligned
+    # s, h, pos, q, k, nbr, cnt, order, w1, w2, grad_out, ws, ws_bytes, dh, dq, dk, dpos, stream
+    args = [ok, ok, ok, ok, ok, ok, None, ok, ok, ok, ok, 1 << 30, ok, ok, ok, None, None]
+    assert lib.egat_backward(ctypes.byref(cs), *args[:6], odd4, *args[7:]) == egat.EGAT_ERR_ARG
+    for slot in (0, 2, 3, 9, 10, 12):   # h, q, k, grad_out, workspace, dh: 16-byte alignment
+        a = list(args)
+        a[slot] = odd16
+        assert lib.egat_backward(ctypes.byref(cs), *a) == egat.EGAT_ERR_ARG
+    for slot in (0, 1, 2, 3, 4, 7, 8, 9, 10, 12, 13, 14):   # required pointers
+        a = list(args)
+        a[slot] = None
+        assert lib.egat_backward(ctypes.byref(cs), *a) == egat.EGAT_ERR_ARG
+    small = list(args)
+    small[11] = 64
+    assert lib.egat_backward(ctypes.byref(cs), *small) == egat.EGAT_ERR_WORKSPACE
+    csr = egat.Shape(n=10, lmax=2, C=C, H=H, dk=16, K=64, dtype="bf16", graph_mode="csr",
+                     n_edges=10).c()
+    assert lib.egat_backward(ctypes.byref(csr), *args) == egat.EGAT_ERR_UNSUPPORTED
