@@ -480,11 +480,28 @@ def main():
             torch.cuda.synchronize(dev)
             bms.append(ba.elapsed_time(bb))
         t_bwd = sum(bms) / len(bms)
+        # the same call without dL/dr (training on energies: no forces wanted)
+        nms = []
+        for _ in range(args.backward_steps):
+            flush.fill_(3)
+            ba, bb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ba.record(torch.cuda.current_stream(dev))
+            rc = lib.egat_backward(ctypes.byref(cshape), h.data_ptr(), pos.data_ptr(), q.data_ptr(),
+                                   k.data_ptr(), nbr.data_ptr(), cnt.data_ptr(), order.data_ptr(),
+                                   w1.data_ptr(), w2.data_ptr(), G.data_ptr(), bws_t.data_ptr(),
+                                   bws_t.numel(), dh_t.data_ptr(), dq_t.data_ptr(), dk_t.data_ptr(),
+                                   None, sp)
+            egat._check("egat_backward", rc)
+            bb.record(torch.cuda.current_stream(dev))
+            torch.cuda.synchronize(dev)
+            nms.append(ba.elapsed_time(bb))
+        t_nodr = sum(nms) / len(nms)
         bwd = {"ms": max_over_ranks(t_bwd, dev),
+               "ms_without_positions": max_over_ranks(t_nodr, dev),
                "atoms_per_s": job_rate(wl.n, t_bwd, dev),
                "edges_per_s": job_rate(alg["edges"], t_bwd, dev),
                "what": "dL/dh, dL/dq, dL/dk, dL/dr of <G, ^h> (egat_backward), L2 flushed "
-                       "before each call"}
+                       "before each call; ms_without_positions: the same call without dL/dr"}
 
     # no bounded device wait may have given up in any of the runs above
     status = lib.egat_take_device_status(torch.cuda.current_stream(dev).cuda_stream)

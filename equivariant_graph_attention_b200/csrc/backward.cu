@@ -930,7 +930,8 @@ int launch_backward_tiled(const egat_shape& s, const BwdWs& w, const void* d_h, 
   scan_one_cta_kernel<<<1, 1024, 0, st>>>(w.deg, s.n, w.ptr);
   in_fill_kernel<<<eb, 256, 0, st>>>(d_nbr, d_cnt, s.n, s.K, w.ptr, w.cursor, w.in);
   if (cudaGetLastError() != cudaSuccess) return EGAT_ERR_CUDA;
-  e = launch_backward_tc(s, w.tc, d_q, d_k, hp, dm, d_order, w.ptr, w.in, d_dq, d_dk, st);
+  e = launch_backward_tc(s, w.tc, d_q, d_k, hp, dm, d_order, w.ptr, w.in, d_dq, d_dk, d_dpos != nullptr,
+                         st);
   if (e == EGAT_OK) e = launch_adjoint<L, float>(s, w.tc.dhp, d_pos, d_w1, d_dh, st);
   if (e != EGAT_OK || !d_dpos) return e;
   PosGradParams pg;

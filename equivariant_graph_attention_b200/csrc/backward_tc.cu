@@ -64,14 +64,14 @@ struct BtcShape {
   static constexpr int STAGES = L >= 2 ? 2 : 4;
 };
 
-// Shared memory (byte offsets, 16-byte aligned): staged float rows, staged
-// q / k rows, staged stats rows (source pass), the stage's mask words, the
-// mbarriers and the abort flag.
-template <int L, bool SRC>
+// Shared memory (byte offsets, 16-byte aligned): staged float rows (FR),
+// staged q / k rows, staged stats rows (source pass), the stage's mask words,
+// the mbarriers and the abort flag.
+template <int L, bool SRC, bool FR = true>
 struct BtcSmem {
   using Sh = BtcShape<L>;
   static constexpr size_t fbuf = 0;
-  static constexpr size_t kbuf = fbuf + size_t(Sh::STAGES) * Sh::RS * Sh::FSTR;
+  static constexpr size_t kbuf = fbuf + (FR ? size_t(Sh::STAGES) * Sh::RS * Sh::FSTR : 0);
   static constexpr size_t sbuf = kbuf + size_t(Sh::STAGES) * Sh::RS * kKStr;
   static constexpr size_t mbuf = sbuf + (SRC ? size_t(Sh::STAGES) * Sh::RS * kSStr : 0);
   static constexpr size_t bars = mbuf + size_t(Sh::STAGES) * kTileM * 4;
@@ -168,13 +168,14 @@ __device__ __forceinline__ int slot_atom(const int32_t* order, int tile, int r, 
   return (unsigned)a < (unsigned)n ? a : -1;
 }
 
-// The per-CTA streaming machinery of both passes: the tile's union in stages
+// The per-CTA streaming machinery of the passes: the tile's union in stages
 // of RS rows; thread r < RS stages row r of each stage (its index loaded one
-// stage ahead), thread 0 also the stage's 16 mask words.
-template <int L, bool SRC>
+// stage ahead): its float row (FR), q or k row and (source pass) statistics
+// row; thread 0 also the stage's 16 mask words.
+template <int L, bool SRC, bool FR = true>
 struct Stream {
   using Sh = BtcShape<L>;
-  using Sm = BtcSmem<L, SRC>;
+  using Sm = BtcSmem<L, SRC, FR>;
   static constexpr int RS = Sh::RS, STAGES = Sh::STAGES, FROW = Sh::FROW, FSTR = Sh::FSTR;
   unsigned char* smem;
   const char* fsrc;        // float rows (h' in the target pass, dm in the source pass)
@@ -195,10 +196,11 @@ struct Stream {
   __device__ void issue(int s, int r, int a) const {
     const int buf = s % STAGES;
     const uint32_t bar = smem_u32(bars() + buf);
-    const uint32_t bytes = FROW + kKRow + (SRC ? kSRow : 0) + (r == 0 ? kTileM * 4 : 0);
+    const uint32_t bytes = (FR ? FROW : 0) + kKRow + (SRC ? kSRow : 0) + (r == 0 ? kTileM * 4 : 0);
     mbar_arrive_expect_tx(bar, bytes);
-    bulk_g2s(smem_u32(smem + Sm::fbuf + (size_t(buf) * RS + r) * FSTR), fsrc + (size_t)a * FROW, FROW,
-             bar);
+    if constexpr (FR)
+      bulk_g2s(smem_u32(smem + Sm::fbuf + (size_t(buf) * RS + r) * FSTR), fsrc + (size_t)a * FROW, FROW,
+               bar);
     bulk_g2s(smem_u32(smem + Sm::kbuf + (size_t(buf) * RS + r) * kKStr), ksrc + (size_t)a * kKRow,
              kKRow, bar);
     if constexpr (SRC)
@@ -225,11 +227,11 @@ struct Stream {
 
 // Set up a CTA's stream for tile `tile` and start its first STAGES - 1
 // stages; returns the index thread r (< RS) stages next.
-template <int L, bool SRC>
-__device__ __forceinline__ int stream_begin(Stream<L, SRC>& S, const BtcParams& p, int tile,
+template <int L, bool SRC, bool FR = true>
+__device__ __forceinline__ int stream_begin(Stream<L, SRC, FR>& S, const BtcParams& p, int tile,
                                             unsigned char* smem, int tid) {
   using Sh = BtcShape<L>;
-  using Sm = BtcSmem<L, SRC>;
+  using Sm = BtcSmem<L, SRC, FR>;
   constexpr int RS = Sh::RS, STAGES = Sh::STAGES;
   const long long base = p.toff ? (long long)p.toff[tile] : (long long)tile * p.cap;
   const int capt = p.toff ? p.toff[tile + 1] - p.toff[tile] : p.cap;
@@ -256,25 +258,26 @@ __device__ __forceinline__ int stream_begin(Stream<L, SRC>& S, const BtcParams& 
 }
 
 // ---------------------------------------------------------------- statistics pass
-// m_i = sum_j alpha_ij h'_j and lse_i per head, with the forward kernel's
-// lazy online softmax: a per-row reference maximum raised only when a logit
-// exceeds it by more than 2^8 (tested once per stage), the accumulators and
-// the weight sums rescaled then.
-template <int L>
+// m_i = sum_j alpha_ij h'_j (WITH_M: only dL/dr needs it) and lse_i per head,
+// with the forward kernel's lazy online softmax: a per-row reference maximum
+// raised only when a logit exceeds it by more than 2^8 (tested once per
+// stage), the accumulators and the weight sums rescaled then.  Without m the
+// pass streams the key rows alone.
+template <int L, bool WITH_M>
 __global__ void __launch_bounds__(kBThreads, 1) bwd_stats_tc_kernel(const __grid_constant__ BtcParams p) {
   using Sh = BtcShape<L>;
-  using Sm = BtcSmem<L, false>;
+  using Sm = BtcSmem<L, false, WITH_M>;
   constexpr int D = Sh::D, RS = Sh::RS, STAGES = Sh::STAGES, FSTR = Sh::FSTR;
   extern __shared__ __align__(128) unsigned char smem[];
   const int tid = threadIdx.x, lane = tid & 31, h = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int tile = blockIdx.x;
 
-  Stream<L, false> S;
+  Stream<L, false, WITH_M> S;
   S.fsrc = reinterpret_cast<const char*>(p.hp);
   S.ksrc = reinterpret_cast<const char*>(p.k);
   S.ssrc = nullptr;
-  int nidx = stream_begin<L, false>(S, p, tile, smem, tid);
+  int nidx = stream_begin<L, false, WITH_M>(S, p, tile, smem, tid);
 
   const int tg0 = slot_atom(p.order, tile, g, p.n), tg1 = slot_atom(p.order, tile, g + 8, p.n);
   uint32_t qa[4];
@@ -344,12 +347,14 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_stats_tc_kernel(const __grid
       const float sc1 = r1 ? fast_exp2(mref1 - mx1) : 1.f;
       z0 *= sc0;
       z1 *= sc1;
+      if constexpr (WITH_M) {
 #pragma unroll
-      for (int d = 0; d < D; ++d) {
-        acc[d][0] *= sc0;
-        acc[d][1] *= sc0;
-        acc[d][2] *= sc1;
-        acc[d][3] *= sc1;
+        for (int d = 0; d < D; ++d) {
+          acc[d][0] *= sc0;
+          acc[d][1] *= sc0;
+          acc[d][2] *= sc1;
+          acc[d][3] *= sc1;
+        }
       }
       if (r0) {
         mref0 = mx0;
@@ -369,13 +374,15 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_stats_tc_kernel(const __grid
       P[3] = fast_exp2(fmaf(v[nt][3], qs, -mref1));
       z0 += P[0] + P[1];
       z1 += P[2] + P[3];
-      uint32_t pa[4];
-      acc_as_a(pa, P);
-      // m += P H' (B rows: union atoms 8 nt + 2t, + 1; columns: the head's channels)
-      const uint32_t* h0 = reinterpret_cast<const uint32_t*>(fb + (8 * nt + 2 * t) * FSTR) + h * 8 + g;
-      const uint32_t* h1 = h0 + FSTR / 4;
+      if constexpr (WITH_M) {
+        uint32_t pa[4];
+        acc_as_a(pa, P);
+        // m += P H' (B rows: union atoms 8 nt + 2t, + 1; columns: the head's channels)
+        const uint32_t* h0 = reinterpret_cast<const uint32_t*>(fb + (8 * nt + 2 * t) * FSTR) + h * 8 + g;
+        const uint32_t* h1 = h0 + FSTR / 4;
 #pragma unroll
-      for (int d = 0; d < D; ++d) mma_tf32(acc[d], pa, h0[d * kBC], h1[d * kBC]);
+        for (int d = 0; d < D; ++d) mma_tf32(acc[d], pa, h0[d * kBC], h1[d * kBC]);
+      }
     }
   }
   S.drain(tid);
@@ -389,11 +396,14 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_stats_tc_kernel(const __grid
     const int tg = half ? tg1 : tg0;
     if (tg < 0) continue;
     const float z = half ? z1 : z0;
-    const float inv = z > 0.f ? 1.f / z : 0.f;
-    float* o = p.m + (size_t)tg * D * kBC + h * 8 + 2 * t;
+    if constexpr (WITH_M) {
+      const float inv = z > 0.f ? 1.f / z : 0.f;
+      float* o = p.m + (size_t)tg * D * kBC + h * 8 + 2 * t;
 #pragma unroll
-    for (int d = 0; d < D; ++d)
-      *reinterpret_cast<float2*>(o + d * kBC) = make_float2(acc[d][2 * half] * inv, acc[d][2 * half + 1] * inv);
+      for (int d = 0; d < D; ++d)
+        *reinterpret_cast<float2*>(o + d * kBC) =
+            make_float2(acc[d][2 * half] * inv, acc[d][2 * half + 1] * inv);
+    }
     if (t == 0)
       p.stats[(size_t)tg * (2 * kBH) + h] = z > 0.f ? (half ? mref1 : mref0) + __log2f(z) : -INFINITY;
   }
@@ -796,10 +806,14 @@ enum PassKind { kStatsPass, kTargetPass, kSourcePass };
 
 template <int L>
 int launch_pass_t(const BtcParams& p, PassKind kind, cudaStream_t st) {
-  const size_t shm = kind == kSourcePass ? BtcSmem<L, true>::total : BtcSmem<L, false>::total;
+  // the statistics pass without m (no dL/dr wanted) streams the key rows alone
+  const bool lean = kind == kStatsPass && !p.m;
+  const size_t shm = kind == kSourcePass ? BtcSmem<L, true>::total
+                     : lean ? BtcSmem<L, false, false>::total : BtcSmem<L, false>::total;
   if (shm > 227 * 1024) return EGAT_ERR_UNSUPPORTED;
   auto kern = kind == kSourcePass ? bwd_source_tc_kernel<L>
-              : kind == kTargetPass ? bwd_target_tc_kernel<L> : bwd_stats_tc_kernel<L>;
+              : kind == kTargetPass ? bwd_target_tc_kernel<L>
+              : lean ? bwd_stats_tc_kernel<L, false> : bwd_stats_tc_kernel<L, true>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(shm)) != cudaSuccess)
     return EGAT_ERR_CUDA;
   kern<<<p.tiles, kBThreads, shm, st>>>(p);
@@ -863,7 +877,7 @@ BwdTcWs bwd_tc_ws(const egat_shape& s, void* base) {
 
 int launch_backward_tc(const egat_shape& s, const BwdTcWs& w, const void* d_q, const void* d_k,
                        const float* d_hp, const float* d_dm, const int32_t* d_order,
-                       const int* d_in_ptr, const int* d_in, float* d_dq, float* d_dk,
+                       const int* d_in_ptr, const int* d_in, float* d_dq, float* d_dk, bool want_m,
                        cudaStream_t st) {
   const int tiles = (s.n + kTileM - 1) / kTileM;
   const PlanView fp = plan_view(w.plan, s.n, s.K, s.lmax);
@@ -877,7 +891,7 @@ int launch_backward_tc(const egat_shape& s, const BwdTcWs& w, const void* d_q, c
   p.dq = d_dq;
   p.dk = d_dk;
   p.dhp = w.dhp;
-  p.m = w.m;
+  p.m = want_m ? w.m : nullptr;
   p.n = s.n;
   p.qscale = float(1.4426950408889634 / std::sqrt(double(s.dk)));
   p.kscale = float(1.0 / std::sqrt(double(s.dk)));

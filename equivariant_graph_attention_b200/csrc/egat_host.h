@@ -114,9 +114,10 @@ BwdTcWs bwd_tc_ws(const egat_shape& s, void* base);
 // m and the log-sum-exp (statistics pass), dq and Delta (target pass), both
 // over the forward plan's tiles in w.plan; the source plan from the in-lists,
 // dk and dh' (source pass).  d_hp and d_dm float32 rounded to tf32.
+// want_m = false (no dL/dr wanted) skips m: the statistics pass streams key rows alone.
 int launch_backward_tc(const egat_shape& s, const BwdTcWs& w, const void* d_q, const void* d_k,
                        const float* d_hp, const float* d_dm, const int32_t* d_order,
-                       const int* d_in_ptr, const int* d_in, float* d_dq, float* d_dk,
+                       const int* d_in_ptr, const int* d_in, float* d_dq, float* d_dk, bool want_m,
                        cudaStream_t st);
 int take_wait_timeouts_backward(cudaStream_t st, unsigned int* count);
 // Bounded-wait reports (one per compilation unit with mbarrier waits): read

@@ -284,7 +284,9 @@ EGAT_API int egat_forward_noalloc(const egat_shape* s, const void* d_h, const fl
  *  d_dh    float32 [n][D][C]   dL/dh
  *  d_dq    float32 [n][H][dk]  dL/dq
  *  d_dk    float32 [n][H][dk]  dL/dk
- *  d_dpos  float32 [n][3]      dL/dr (forces are its negative); may be NULL
+ *  d_dpos  float32 [n][3]      dL/dr (forces are its negative); may be NULL, which
+ *                              also skips m (on the tiled path the first pass
+ *                              then streams key rows alone)
  * (positions enter through the solid harmonics of both couplings, the
  * neighbour lists held fixed; weight gradients are not computed).
  *  d_order optional int32 [n] traversal order (a permutation, as

@@ -216,3 +216,26 @@ def test_tiled_backward_random_order():
     assert row_rel_error(dq, rdq) < tol and row_rel_error(dk, rdk) < tol
     assert row_rel_error(dr, rdr) < tol
     assert egat.egat_take_device_status() == egat.EGAT_OK
+
+
+def test_tiled_backward_without_positions():
+    """No dL/dr buffer: the statistics pass skips m and streams key rows alone.
+    dL/dh, dL/dq and dL/dk are bitwise those of the call with dL/dr (the
+    log-sum-exp does not depend on m) and meet the bf16 bar."""
+    egat = _egat()
+    wl, d, G, (rdh, rdq, rdk, rdr) = _case("uniform4096_l2_bf16")
+    dev = device_inputs(wl, d)
+    g = egat.egat_build_graph(dev["pos_q"], wl.cutoff_q, K=wl.K)
+    Gd = torch.from_numpy(G).cuda()
+    args = (shape_of(wl), dev["h"], dev["pos"], dev["q"], dev["k"], g["nbr"], g["cnt"], dev["w1"],
+            dev["w2"], Gd)
+    full = egat.egat_backward(*args, order=g["order"])
+    lean = egat.egat_backward(*args, positions=False, order=g["order"])
+    assert lean[3] is None
+    for a, b in zip(full[:3], lean[:3]):
+        assert torch.equal(a, b)
+    tol = TOL[wl.dtype]
+    assert block_rel_error(lean[0].cpu().numpy(), rdh, wl.lmax) < tol
+    assert row_rel_error(lean[1].cpu().numpy(), rdq) < tol
+    assert row_rel_error(lean[2].cpu().numpy(), rdk) < tol
+    assert egat.egat_take_device_status() == egat.EGAT_OK
