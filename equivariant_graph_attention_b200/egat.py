@@ -308,8 +308,9 @@ def egat_backward(shape: Shape, h: torch.Tensor, pos: torch.Tensor, q: torch.Ten
                   workspace: Optional[torch.Tensor] = None, positions: bool = True,
                   order: Optional[torch.Tensor] = None, stream=None):
     """(dL/dh, dL/dq, dL/dk, dL/dr) float32 for the upstream gradient grad_out = dL/d^h
-    (dL/dr is None when positions=False); order = the graph builder's traversal
-    order (tiles of spatially adjacent atoms), optional."""
+    (dL/dr is None when positions=False, which also skips m and makes the call
+    cheaper); order = the graph builder's traversal order (tiles of spatially
+    adjacent atoms), optional: results do not depend on it up to rounding."""
     nb = egat_backward_workspace_bytes(shape)
     if workspace is None:
         workspace = torch.empty(max(nb, 16), dtype=torch.uint8, device=h.device)
