@@ -261,6 +261,16 @@ int egat_take_device_status(void* stream) {
   return (a | b | c) ? EGAT_ERR_TIMEOUT : EGAT_OK;
 }
 
+int egat_gather_rows(const void* d_src, int64_t n_src, int64_t row_bytes, const int32_t* d_idx,
+                     int64_t count, void* d_dst, void* stream) {
+  if (n_src < 0 || count < 0 || row_bytes <= 0 || row_bytes % 16) return EGAT_ERR_ARG;
+  if (count == 0) return EGAT_OK;
+  if (!d_idx || !d_dst || (n_src > 0 && !d_src)) return EGAT_ERR_ARG;
+  if (!aligned16(d_dst) || (d_src && !aligned16(d_src)) || !aligned4(d_idx)) return EGAT_ERR_ARG;
+  return launch_gather_rows(d_src, n_src, row_bytes, d_idx, count, d_dst,
+                            static_cast<cudaStream_t>(stream));
+}
+
 int egat_selftest_wait_timeout(int32_t polls, void* stream) {
   if (polls < 1 || polls > (1 << 20)) return EGAT_ERR_ARG;
   return launch_wait_timeout_selftest(polls, static_cast<cudaStream_t>(stream));

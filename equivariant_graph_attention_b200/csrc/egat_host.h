@@ -120,6 +120,10 @@ int launch_backward_tc(const egat_shape& s, const BwdTcWs& w, const void* d_q, c
                        const int* d_in_ptr, const int* d_in, float* d_dq, float* d_dk, bool want_m,
                        cudaStream_t st);
 int take_wait_timeouts_backward(cudaStream_t st, unsigned int* count);
+// dst[r] = src[idx[r]] for r < count (rows of row_bytes, a multiple of 16; an
+// index outside [0, n_src) gives a zero row).
+int launch_gather_rows(const void* d_src, long long n_src, long long row_bytes, const int32_t* d_idx,
+                       long long count, void* d_dst, cudaStream_t st);
 // Bounded-wait reports (one per compilation unit with mbarrier waits): read
 // and clear the count of waits that gave up (synchronises st); the self-test
 // launch.

@@ -41,7 +41,7 @@ EXPORTS = ["egat_version", "egat_strerror", "egat_num_paths", "egat_graph_worksp
            "egat_forward_workspace_bytes", "egat_forward", "egat_forward_noalloc",
            "egat_attention_plan_bytes", "egat_build_attention_plan", "egat_otf_attention_tiled",
            "egat_eaas_couple_planned", "egat_take_device_status", "egat_selftest_wait_timeout",
-           "egat_backward_workspace_bytes", "egat_backward"]
+           "egat_backward_workspace_bytes", "egat_backward", "egat_gather_rows"]
 
 
 class EgatError(RuntimeError):
@@ -98,6 +98,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.egat_build_attention_plan.argtypes = [sp, vp, vp, vp, vp, vp, sz, vp]
     lib.egat_backward_workspace_bytes.restype = ctypes.c_int
     lib.egat_backward_workspace_bytes.argtypes = [sp, ctypes.POINTER(sz)]
+    lib.egat_gather_rows.restype = ctypes.c_int
+    lib.egat_gather_rows.argtypes = [vp, i64, i64, vp, i64, vp, vp]
     lib.egat_backward.restype = ctypes.c_int
     lib.egat_backward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp, vp, vp, vp]
     lib.egat_take_device_status.restype = ctypes.c_int
@@ -326,6 +328,20 @@ def egat_backward(shape: Shape, h: torch.Tensor, pos: torch.Tensor, q: torch.Ten
         _ptr(dk), _ptr(dpos), _stream(stream))
     _check("egat_backward", rc)
     return dh, dq, dk, dpos
+
+
+def egat_gather_rows(src: torch.Tensor, idx: torch.Tensor, out: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """out[r] = src[idx[r]] along the first dimension (an index outside
+    [0, len(src)) gives a zero row); rows must be a multiple of 16 bytes."""
+    n = src.shape[0]
+    row_bytes = src[0].numel() * src.element_size() if n > 0 else (
+        int(torch.tensor(src.shape[1:]).prod()) * src.element_size())
+    if out is None:
+        out = torch.empty((idx.numel(),) + tuple(src.shape[1:]), dtype=src.dtype, device=src.device)
+    _check("egat_gather_rows", load_library().egat_gather_rows(
+        _ptr(src) if n > 0 else None, n, row_bytes, _ptr(idx), idx.numel(), _ptr(out), _stream(stream)))
+    return out
 
 
 def egat_take_device_status(stream=None) -> int:

@@ -1,0 +1,160 @@
+"""Spatial domain decomposition with one halo exchange per step.
+
+One GPU reaches systems of about 10^5 atoms ("E2Former-V2：突破等变图神经网络
+计算瓶颈的创新架构" §3.2).  Past that, the atoms are split into contiguous
+blocks of the graph builder's traversal order (cells in Morton order, so a
+block is spatially compact), one block per rank.  Each step, rank r
+
+1. couples its own atoms at the source (step 2) with the library;
+2. packs the h' and k rows that other ranks need (``egat_gather_rows``) and
+   exchanges them in one all-to-all per array (NCCL over NVLink between GPUs);
+3. runs steps 3+4 for its own atoms over local arrays: its own rows first,
+   then the received halo rows (halo atoms appear only as sources, with empty
+   neighbour lists, so their outputs are zero and discarded).
+
+The plan (who owns what, which rows go where) is host logic computed once per
+neighbour list from the global padded lists, which every rank can build from
+the replicated positions (12 bytes per atom).  The only data-path collective
+is the exchange of step 2; the forward needs nothing else from other ranks.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Callable, List, Optional
+
+import numpy as np
+import torch
+
+from . import egat
+
+
+@dataclass
+class HaloPlan:
+    rank: int
+    world: int
+    owned: np.ndarray          # int64 global ids of this rank's atoms, in traversal order
+    halo: np.ndarray           # int64 global ids of the halo, grouped by owning rank, ascending within
+    recv_counts: List[int]     # per rank: halo atoms owned by it (0 for this rank)
+    send: List[np.ndarray]     # per rank: local indices (into owned) of the rows it receives from us
+    local_nbr: np.ndarray      # int32 [n_owned + n_halo, K]: owned rows in local indices, halo rows -1
+    local_cnt: np.ndarray      # int32 [n_owned + n_halo]
+
+    @property
+    def n_owned(self) -> int:
+        return int(self.owned.size)
+
+    @property
+    def n_local(self) -> int:
+        return int(self.owned.size + self.halo.size)
+
+
+def owners(order: np.ndarray, world: int) -> np.ndarray:
+    """Owning rank of every atom: rank r holds slots [r n / world, (r+1) n / world) of
+    the traversal order."""
+    order = np.asarray(order, dtype=np.int64)
+    n = order.size
+    owner = np.empty(n, dtype=np.int64)
+    for r in range(world):
+        owner[order[r * n // world:(r + 1) * n // world]] = r
+    return owner
+
+
+def _needed(nbr: np.ndarray, cnt: np.ndarray, targets: np.ndarray) -> np.ndarray:
+    """Distinct neighbours (global ids) of the given targets."""
+    n, K = nbr.shape
+    rows = nbr[targets]
+    c = np.clip(cnt[targets], 0, K)
+    valid = (np.arange(K)[None, :] < c[:, None]) & (rows >= 0) & (rows < n)
+    return np.unique(rows[valid].astype(np.int64))
+
+
+def build_plan(nbr: np.ndarray, cnt: Optional[np.ndarray], order: np.ndarray, world: int,
+               rank: int) -> HaloPlan:
+    """The halo plan of `rank` from the global padded lists (nbr [n, K], cnt [n] or
+    None for full rows) and the traversal order."""
+    nbr = np.asarray(nbr)
+    n, K = nbr.shape
+    cnt = np.full(n, K, dtype=np.int64) if cnt is None else np.asarray(cnt, dtype=np.int64)
+    order = np.asarray(order, dtype=np.int64)
+    owner = owners(order, world)
+    blocks = [order[r * n // world:(r + 1) * n // world] for r in range(world)]
+    owned = blocks[rank]
+
+    def halo_of(r: int) -> np.ndarray:
+        need = _needed(nbr, cnt, blocks[r])
+        need = need[owner[need] != r]
+        return need[np.lexsort((need, owner[need]))]      # by owning rank, then id
+
+    halo = halo_of(rank)
+    local_of = np.full(n, -1, dtype=np.int64)
+    local_of[owned] = np.arange(owned.size)
+    local_of[halo] = owned.size + np.arange(halo.size)
+    rows = nbr[owned].astype(np.int64)
+    c = np.clip(cnt[owned], 0, K)
+    valid = (np.arange(K)[None, :] < c[:, None]) & (rows >= 0) & (rows < n)
+    local_nbr = np.full((owned.size + halo.size, K), -1, dtype=np.int32)
+    local_nbr[:owned.size] = np.where(valid, local_of[np.where(valid, rows, 0)], -1)
+    local_cnt = np.zeros(owned.size + halo.size, dtype=np.int32)
+    local_cnt[:owned.size] = c
+    recv_counts = [int(np.sum(owner[halo] == p)) for p in range(world)]
+    send = []
+    for p in range(world):
+        if p == rank:
+            send.append(np.zeros(0, dtype=np.int64))
+            continue
+        theirs = halo_of(p)
+        mine = theirs[owner[theirs] == rank]               # ascending id: their receive order
+        send.append(local_of[mine])
+    return HaloPlan(rank, world, owned, halo, recv_counts, send, local_nbr, local_cnt)
+
+
+def exchange(plan: HaloPlan, own_rows: torch.Tensor, group=None,
+             pack: Optional[Callable[[torch.Tensor, torch.Tensor], torch.Tensor]] = None) -> torch.Tensor:
+    """Rows of the halo atoms (in plan.halo order) from their owners, given this
+    rank's own rows [n_owned, ...]: the send buffer is packed on the device
+    (egat_gather_rows) and one all-to-all moves it.  `pack(rows, idx)` replaces
+    the device packing (tests on CPU ranks)."""
+    import torch.distributed as dist
+    dev = own_rows.device
+    send_idx = torch.from_numpy(np.concatenate(plan.send).astype(np.int32)).to(dev)
+    if pack is None:
+        if not own_rows.is_cuda:
+            raise RuntimeError("exchange packs rows on the GPU; pass `pack` for CPU tensors")
+        send_buf = egat.egat_gather_rows(own_rows.contiguous(), send_idx)
+    else:
+        send_buf = pack(own_rows, send_idx)
+    recv = torch.empty((sum(plan.recv_counts),) + tuple(own_rows.shape[1:]), dtype=own_rows.dtype,
+                       device=dev)
+    dist.all_to_all_single(recv, send_buf, output_split_sizes=list(plan.recv_counts),
+                           input_split_sizes=[int(s.size) for s in plan.send], group=group)
+    return recv
+
+
+def forward_rank(plan: HaloPlan, shape: "egat.Shape", h: torch.Tensor, pos: torch.Tensor,
+                 q: torch.Tensor, k: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor,
+                 group=None) -> torch.Tensor:
+    """^h of this rank's atoms (float32 [n_owned, D, C], in plan.owned order) for the
+    global inputs h, pos, q, k of the `shape` system (each rank reads only its own
+    rows of h, q and k, and the positions of its own and its halo atoms)."""
+    dev = h.device
+    own = torch.from_numpy(plan.owned).to(dev)
+    loc = torch.from_numpy(np.concatenate([plan.owned, plan.halo])).to(dev)
+    n_own, n_loc = plan.n_owned, plan.n_local
+    own_i32 = own.to(torch.int32)
+    h_own = egat.egat_gather_rows(h.contiguous(), own_i32)
+    q_own = egat.egat_gather_rows(q.contiguous(), own_i32)
+    k_own = egat.egat_gather_rows(k.contiguous(), own_i32)
+    pos_loc = pos.index_select(0, loc).contiguous()
+    shape_own = egat.Shape(n=n_own, lmax=shape.lmax, C=shape.C, H=shape.H, dk=shape.dk, K=shape.K,
+                           dtype=shape.dtype)
+    hp_own = egat.egat_eaas_couple(shape_own, h_own, pos_loc[:n_own].contiguous(), w1)
+    hp_loc = torch.cat([hp_own, exchange(plan, hp_own, group)])
+    k_loc = torch.cat([k_own, exchange(plan, k_own, group)])
+    q_loc = torch.cat([q_own, torch.zeros((n_loc - n_own,) + tuple(q.shape[1:]), dtype=q.dtype,
+                                          device=dev)])
+    nbr = torch.from_numpy(plan.local_nbr).to(dev)
+    cnt = torch.from_numpy(plan.local_cnt).to(dev)
+    shape_loc = egat.Shape(n=n_loc, lmax=shape.lmax, C=shape.C, H=shape.H, dk=shape.dk, K=shape.K,
+                           dtype=shape.dtype)
+    out = egat.egat_otf_attention_coupled(shape_loc, q_loc, k_loc, hp_loc, nbr, cnt, pos_loc, w2)
+    return out[:n_own]

@@ -314,8 +314,22 @@ EGAT_API int egat_backward(const egat_shape* s, const void* d_h, const float* d_
                            float* d_dq, float* d_dk, float* d_dpos, void* stream);
 
 /*
- * Device status.  The tensor-core attention kernel waits on mbarriers for its
- * bulk copies; every such wait is bounded (about a second).  A wait that
+ * Row gather, the packing step of a halo exchange (a spatial domain
+ * decomposition across GPUs: each rank couples its own atoms and needs the
+ * h' and k rows of the neighbours it does not own; one GPU reaches about
+ * 10^5 atoms, [EX] §3.2).  d_dst[r] = d_src[d_idx[r]] for r < count, rows of
+ * row_bytes bytes (a positive multiple of 16), copied in 16-byte vectors; an
+ * index outside [0, n_src) gives a zero row.  d_src and d_dst 16-byte
+ * aligned, d_idx int32.  Asynchronous on `stream`; count = 0 is a no-op.
+ * Errors: EGAT_ERR_ARG (sizes, null or misaligned pointers), EGAT_ERR_CUDA.
+ */
+EGAT_API int egat_gather_rows(const void* d_src, int64_t n_src, int64_t row_bytes,
+                              const int32_t* d_idx, int64_t count, void* d_dst, void* stream);
+
+/*
+ * Device status.  The tensor-core attention kernel, the tile-staged source
+ * coupling and the tiled backward passes wait on mbarriers for their bulk
+ * copies; every such wait is bounded (about a second).  A wait that
  * gives up is counted on the device, the kernel stops waiting and finishes
  * with meaningless output instead of hanging.  The pages have no
  * counterpart: this is the library's failure report.

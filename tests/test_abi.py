@@ -179,3 +179,19 @@ def test_backward_entry_validation(lib):
     csr = egat.Shape(n=10, lmax=2, C=C, H=H, dk=16, K=64, dtype="bf16", graph_mode="csr",
                      n_edges=10).c()
     assert lib.egat_backward(ctypes.byref(csr), *args) == egat.EGAT_ERR_UNSUPPORTED
+
+
+def test_gather_rows_validation(lib):
+    """egat_gather_rows' host checks; a zero count returns before any launch."""
+    ok = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)
+    assert lib.egat_gather_rows(ok, 10, 64, ok, 0, ok, None) == egat.EGAT_OK
+    assert lib.egat_gather_rows(ok, 10, 24, ok, 4, ok, None) == egat.EGAT_ERR_ARG     # row size
+    assert lib.egat_gather_rows(ok, 10, 0, ok, 4, ok, None) == egat.EGAT_ERR_ARG
+    assert lib.egat_gather_rows(ok, -1, 64, ok, 4, ok, None) == egat.EGAT_ERR_ARG
+    assert lib.egat_gather_rows(ok, 10, 64, ok, -4, ok, None) == egat.EGAT_ERR_ARG
+    assert lib.egat_gather_rows(ok, 10, 64, None, 4, ok, None) == egat.EGAT_ERR_ARG
+    assert lib.egat_gather_rows(ok, 10, 64, ok, 4, None, None) == egat.EGAT_ERR_ARG
+    assert lib.egat_gather_rows(ok, 10, 64, ok, 4, odd, None) == egat.EGAT_ERR_ARG
+    assert lib.egat_gather_rows(odd, 10, 64, ok, 4, ok, None) == egat.EGAT_ERR_ARG
+    assert lib.egat_gather_rows(None, 10, 64, ok, 4, ok, None) == egat.EGAT_ERR_ARG
