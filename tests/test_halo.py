@@ -130,3 +130,27 @@ def test_decomposed_forward_on_gloo_ranks(world):
         err, scale, nh, _ = results[r]
         assert nh > 0                                  # the ranks do exchange rows
         assert err <= 1e-12 * max(1.0, scale)
+
+
+def test_plan_edge_cases():
+    """More ranks than atoms (empty blocks), no count array, isolated atoms."""
+    from equivariant_graph_attention_b200 import halo
+    nbr = np.array([[1, 2, -1], [0, -1, -1], [0, -1, -1], [-1, -1, -1], [3, -1, -1]], dtype=np.int32)
+    cnt = np.array([2, 1, 1, 0, 1], dtype=np.int32)
+    order = np.array([4, 3, 0, 1, 2])
+    plans = [halo.build_plan(nbr, cnt, order, 8, r) for r in range(8)]
+    assert sorted(np.concatenate([p.owned for p in plans]).tolist()) == [0, 1, 2, 3, 4]
+    assert sum(p.n_owned == 0 for p in plans) == 3
+    for p in plans:
+        assert len(p.send) == 8 and len(p.recv_counts) == 8
+        assert p.local_nbr.shape == (p.n_local, 3)
+    # without a count array every slot is scanned and -1 entries are skipped:
+    # rank 0 of 2 owns atoms 4 and 3 (slots 0, 1); atom 4 lists atom 3 (local 1)
+    full = halo.build_plan(nbr, None, order, 2, 0)
+    assert full.owned.tolist() == [4, 3] and full.halo.size == 0
+    assert full.local_cnt.tolist() == [3, 3]
+    assert full.local_nbr.tolist() == [[1, -1, -1], [-1, -1, -1]]
+    # rank 1 owns atoms 0, 1, 2, which list only one another
+    other = halo.build_plan(nbr, None, order, 2, 1)
+    assert other.owned.tolist() == [0, 1, 2] and other.halo.size == 0
+    assert other.send[0].size == 0 and other.recv_counts == [0, 0]
