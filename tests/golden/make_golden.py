@@ -1,9 +1,11 @@
-"""Write the oracle's output for a tiny seeded system to forward_tiny.json.
+"""Write the oracle's output for a tiny seeded system to forward_tiny.json, and
+its gradients for a seeded upstream gradient to backward_tiny.json.
 
 Calls only the oracle and the seeded input generator.  The stored values lock
-the oracle against unintended change (a regression fixture, not a pin: the
-pages print no worked example of the forward pass) and give the CUDA parity
-tests one fixed case.  Run from the repository root:
+the oracle against unintended change (regression fixtures, not pins: the
+pages print no worked example of either pass; the backward's pins are finite
+differences of the forward) and give the CUDA parity tests one fixed case.
+Run from the repository root:
 
     python tests/golden/make_golden.py
 """
@@ -33,12 +35,28 @@ def build():
     return wl, d, nbrs, full, out
 
 
+def build_backward():
+    """(G, dh, dq, dk, dr) of L = <G, ^h> for the tiny system, G ~ N(0, 1) seeded."""
+    from oracle.backward import backward, position_grad
+    wl, d, nbrs, _, _ = build()
+    G = np.random.default_rng([SPEC["seed"], 99]).standard_normal((wl.n, wl.D, wl.C))
+    dh, dq, dk = backward(d["h"], d["pos"], d["q"], d["k"], d["w1"], d["w2"], wl.lmax, nbrs, G)
+    dr = position_grad(d["h"], d["pos"], d["q"], d["k"], d["w1"], d["w2"], wl.lmax, nbrs, G)
+    return G, dh, dq, dk, dr
+
+
 def main():
     wl, d, nbrs, full, out = build()
     rec = {"spec": SPEC, "cutoff_q": wl.cutoff_q,
            "neighbours": [n.tolist() for n in nbrs], "full_degree": full.tolist(),
            "out": np.round(out, 15).tolist()}
     with open(os.path.join(HERE, "forward_tiny.json"), "w") as f:
+        json.dump(rec, f)
+    G, dh, dq, dk, dr = build_backward()
+    rec = {"spec": SPEC, "upstream_seed": [SPEC["seed"], 99],
+           "dh": np.round(dh, 15).tolist(), "dq": np.round(dq, 15).tolist(),
+           "dk": np.round(dk, 15).tolist(), "dr": np.round(dr, 15).tolist()}
+    with open(os.path.join(HERE, "backward_tiny.json"), "w") as f:
         json.dump(rec, f)
 
 

@@ -2,8 +2,9 @@
 
 * ``cg_textbook_1x1.txt``: the standard printed table of Clebsch–Gordan
   coefficients for two l = 1 states, against the oracle's Racah formula.
-* ``forward_tiny.json``: the oracle's own output for a tiny seeded system,
-  written by ``make_golden.py``; a regression lock on the oracle.
+* ``forward_tiny.json``, ``backward_tiny.json``: the oracle's own output and
+  gradients for a tiny seeded system, written by ``make_golden.py``;
+  regression locks on the oracle.
 """
 import json
 import os
@@ -12,7 +13,7 @@ from fractions import Fraction
 import numpy as np
 
 from oracle import so3
-from tests.golden.make_golden import build
+from tests.golden.make_golden import build, build_backward
 
 HERE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
@@ -43,3 +44,13 @@ def test_forward_tiny_regression():
     assert [n.tolist() for n in nbrs] == rec["neighbours"]
     assert full.tolist() == rec["full_degree"]
     assert np.max(np.abs(out - np.array(rec["out"]))) < 1e-12 * np.max(np.abs(out))
+
+
+def test_backward_tiny_regression():
+    with open(os.path.join(HERE, "backward_tiny.json")) as f:
+        rec = json.load(f)
+    _, dh, dq, dk, dr = build_backward()
+    for name, got in (("dh", dh), ("dq", dq), ("dk", dk), ("dr", dr)):
+        ref = np.array(rec[name])
+        assert ref.shape == got.shape
+        assert np.max(np.abs(got - ref)) < 1e-12 * max(1.0, np.max(np.abs(ref))), name
