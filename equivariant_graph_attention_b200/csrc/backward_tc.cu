@@ -177,6 +177,7 @@ struct Stream {
   using Sh = BtcShape<L>;
   using Sm = BtcSmem<L, SRC, FR>;
   static constexpr int RS = Sh::RS, STAGES = Sh::STAGES, FROW = Sh::FROW, FSTR = Sh::FSTR;
+  static_assert(FROW % 16 == 0 && FSTR % 16 == 0, "bulk copies move 16-byte units");
   unsigned char* smem;
   const char* fsrc;        // float rows (h' in the target pass, dm in the source pass)
   const char* ksrc;        // q / k rows

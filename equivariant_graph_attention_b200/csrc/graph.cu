@@ -353,26 +353,6 @@ __device__ unsigned long long kth_key(const Search& s, int4 p, int4 c, int K) {
   return lo;
 }
 
-__device__ __forceinline__ void warp_bitonic_sort(unsigned long long* keys, int size) {
-  // ascending sort of keys[0, size), size a power of two, one warp
-  const int lane = threadIdx.x & 31;
-  for (int k = 2; k <= size; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = lane; i < size; i += 32) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const unsigned long long a = keys[i], b = keys[ixj];
-          if ((a > b) == ((i & k) == 0)) {
-            keys[i] = b;
-            keys[ixj] = a;
-          }
-        }
-      }
-      __syncwarp();
-    }
-  }
-}
-
 // Padded list, one warp per atom (atoms taken in cell order).  One sweep
 // writes the first K neighbours and counts all of them; an atom with more
 // than K is appended to the truncation list for fix_truncated.  Row order is
