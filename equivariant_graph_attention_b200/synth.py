@@ -20,7 +20,9 @@ instead places oxygens on a jittered 6^3 grid and adds two hydrogens per
 oxygen in a uniformly random orientation.
 
 Feature recipe: ``numpy.random.default_rng([seed, tag])`` with tag 1 -> h,
-2 -> q, 3 -> k, 4 -> w1, 5 -> w2.  h, q, k ~ N(0, 1); the weight of path p is
+2 -> q, 3 -> k, 4 -> w1, 5 -> w2, 6 -> wq, 7 -> wk (the invariant query/key
+projection weights, float32 [C][H*dk], N(0, 1/C)), 8 -> the SO(2) weights of
+the edge-centric comparison convolution (float32 [NW][C], N(0, 1/(lmax+1))).  h, q, k ~ N(0, 1); the weight of path p is
 N(0, 1/fan_in(ℓo(p))) with fan_in the number of paths that feed ℓo.  For the
 bf16 workloads h, q and k are rounded to bf16 (round to nearest even) and
 returned as float32 arrays that hold exactly those values.
@@ -205,6 +207,33 @@ def features(wl: Workload, seed: int = 0) -> Dict[str, np.ndarray]:
     if wl.dtype == "bf16":
         h, q, k = round_bf16(h), round_bf16(q), round_bf16(k)
     return {"h": h, "q": q, "k": k, "w1": w1.astype(np.float32), "w2": w2.astype(np.float32)}
+
+
+def projection_weights(wl: Workload, seed: int = 0) -> Dict[str, np.ndarray]:
+    """wq, wk float32 [C][H*dk] ~ N(0, 1/C): column h*dk + d of wq maps the
+    degree-0 channels of an atom's features to component d of its head-h query
+    (so q ~ N(0, 1) for h ~ N(0, 1))."""
+    def g(tag):
+        return np.random.default_rng([seed, tag])
+
+    C, HD = wl.C, wl.H * wl.dk
+    s = np.float32(1.0 / np.sqrt(C))
+    return {"wq": g(6).standard_normal((C, HD), dtype=np.float32) * s,
+            "wk": g(7).standard_normal((C, HD), dtype=np.float32) * s}
+
+
+def escn_weight_count(lmax: int, mmax: int) -> int:
+    """Rows of the SO(2) weight array: (lmax+1)^2 for order 0, then two blocks of
+    (lmax+1-m)^2 for each order 1 <= m <= mmax (the layout is an interface fact)."""
+    return (lmax + 1) ** 2 + sum(2 * (lmax + 1 - m) ** 2 for m in range(1, mmax + 1))
+
+
+def escn_weights(wl: Workload, mmax: int, seed: int = 0) -> np.ndarray:
+    """float32 [NW][C] ~ N(0, 1/(lmax+1)): each output degree mixes lmax+1 inputs."""
+    nw = escn_weight_count(wl.lmax, mmax)
+    g = np.random.default_rng([seed, 8])
+    return (g.standard_normal((nw, wl.C), dtype=np.float32)
+            * np.float32(1.0 / np.sqrt(wl.lmax + 1))).astype(np.float32)
 
 
 def make(wl: Workload, seed: int = 0) -> Dict[str, np.ndarray]:

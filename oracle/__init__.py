@@ -18,6 +18,13 @@ It computes the plain definitions, slowly and in float64:
 * ``attention``: dense tensor-product source coupling, invariant logits,
   two-pass softmax over each atom's neighbours, aggregation, dense target
   coupling, and the composed forward pass.
+* ``projection``: the invariant query/key projection (a linear map of the
+  degree-0 channels).
+* ``storage``: bfloat16 rounding, where a test models the bf16 storage the
+  workloads specify.
+* ``escn``: the edge-centric eSCN convolution (rotate each neighbour's
+  features into its edge frame, SO(2) linear layer, rotate back, sum), the
+  comparison workload.
 
 Citations name the pages by title:
 
@@ -33,4 +40,4 @@ composed forward is pinned through those component pins and its symmetry
 properties (rotation and permutation equivariance, the ℓ_max = 0 reduction to
 masked scaled-dot-product attention).
 """
-from . import so3, graph, attention  # noqa: F401
+from . import so3, graph, attention, projection, storage, escn  # noqa: F401

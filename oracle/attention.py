@@ -105,10 +105,13 @@ def aggregate(q, k, hp, nbrs: Sequence[np.ndarray], targets: Optional[Sequence[i
 
 
 def forward(h, pos, q, k, w1, w2, lmax: int, nbrs: Sequence[np.ndarray],
-            targets: Optional[Sequence[int]] = None) -> np.ndarray:
+            targets: Optional[Sequence[int]] = None, store=None) -> np.ndarray:
     """^h for each target: source coupling -> attention -> target coupling.
 
-    Only the atoms that some target needs are coupled at the source.
+    Only the atoms that some target needs are coupled at the source.  store,
+    if given, is applied to h' between the source coupling and the attention
+    (``storage.round_bf16`` models the bf16 storage of h' that the bf16
+    workloads specify); None keeps h' in float64.
     """
     N = np.asarray(h).shape[0]
     targets = list(range(N)) if targets is None else list(targets)
@@ -117,5 +120,7 @@ def forward(h, pos, q, k, w1, w2, lmax: int, nbrs: Sequence[np.ndarray],
     hp = np.zeros(np.asarray(h).shape)
     if need.size:
         hp[need] = source_coupling(np.asarray(h)[need], np.asarray(pos)[need], w1, lmax)
+        if store is not None:
+            hp[need] = store(hp[need])
     m = aggregate(q, k, hp, nbrs, targets)
     return target_coupling(m, np.asarray(pos)[targets], w2, lmax)
