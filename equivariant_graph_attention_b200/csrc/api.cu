@@ -251,14 +251,52 @@ int egat_forward(const egat_shape* s, const void* d_h, const float* d_pos, const
 
 int egat_take_device_status(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  unsigned int a = 0, b = 0, c = 0;
+  unsigned int a = 0, b = 0, c = 0, d = 0;
   const int ra = take_wait_timeouts_attention(st, &a);
   const int rb = take_wait_timeouts_coupling(st, &b);
   const int rc = take_wait_timeouts_backward(st, &c);
+  const int rd = take_wait_timeouts_projection(st, &d);
   if (ra != EGAT_OK) return ra;
   if (rb != EGAT_OK) return rb;
   if (rc != EGAT_OK) return rc;
-  return (a | b | c) ? EGAT_ERR_TIMEOUT : EGAT_OK;
+  if (rd != EGAT_OK) return rd;
+  return (a | b | c | d) ? EGAT_ERR_TIMEOUT : EGAT_OK;
+}
+
+int egat_qk_projection(const egat_shape* s, const void* d_h, const float* d_wq, const float* d_wk,
+                       void* d_q, void* d_k, void* stream) {
+  if (!s || s->n < 0) return EGAT_ERR_ARG;
+  if (s->dtype != EGAT_F32 && s->dtype != EGAT_BF16) return EGAT_ERR_ARG;
+  if (s->lmax < 0 || s->lmax > kMaxL) return EGAT_ERR_UNSUPPORTED;
+  if (s->C < 1 || s->C > 1024 || s->H < 1 || s->dk < 1 || s->H * s->dk > 1024)
+    return EGAT_ERR_UNSUPPORTED;
+  if (s->n == 0) return EGAT_OK;
+  if (!d_h || !d_wq || !d_wk || !d_q || !d_k) return EGAT_ERR_ARG;
+  if (!aligned16(d_h) || !aligned4(d_wq) || !aligned4(d_wk) || !aligned4(d_q) || !aligned4(d_k))
+    return EGAT_ERR_ARG;
+  return launch_qk_projection(*s, d_h, d_wq, d_wk, d_q, d_k, static_cast<cudaStream_t>(stream));
+}
+
+int egat_escn_num_weights(int32_t lmax, int32_t mmax) {
+  if (lmax < 1 || lmax > kMaxL || mmax < 0 || mmax > lmax) return 0;
+  return escn_num_weights_host(lmax, mmax);
+}
+
+int egat_escn_conv(const egat_shape* s, int32_t mmax, const void* d_h, const float* d_pos,
+                   const int32_t* d_nbr, const int32_t* d_cnt, const int32_t* d_order,
+                   const float* d_w, float* d_out, void* stream) {
+  const int rc = check_shape(s, false);
+  if (rc != EGAT_OK) return rc;
+  if (s->graph_mode != EGAT_GRAPH_PADDED) return EGAT_ERR_UNSUPPORTED;
+  if (s->K < 1 || s->K > 1024) return EGAT_ERR_ARG;
+  if (mmax < 0 || mmax > s->lmax) return EGAT_ERR_ARG;
+  if (s->n == 0) return EGAT_OK;
+  if (!d_h || !d_pos || !d_nbr || !d_w || !d_out) return EGAT_ERR_ARG;
+  if (!aligned16(d_h) || !aligned4(d_pos) || !aligned4(d_nbr) || !aligned4(d_w) ||
+      !aligned4(d_out) || (d_cnt && !aligned4(d_cnt)) || (d_order && !aligned4(d_order)))
+    return EGAT_ERR_ARG;
+  return launch_escn_conv(*s, mmax, d_h, d_pos, d_nbr, d_cnt, d_order, d_w, d_out,
+                          static_cast<cudaStream_t>(stream));
 }
 
 int egat_gather_rows(const void* d_src, int64_t n_src, int64_t row_bytes, const int32_t* d_idx,

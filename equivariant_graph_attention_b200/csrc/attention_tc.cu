@@ -29,12 +29,15 @@
 //  * the plan's membership bits mask S to each target's own neighbours; the
 //    online softmax keeps a per-row reference maximum raised lazily (only by
 //    more than 2^8), tested once per stage, so z and the accumulators share
-//    one reference; z is the mma of P with an all-ones fragment — the row
-//    sums of exactly the bf16 weights that enter P V;
-//  * the probabilities become the bf16 A fragment directly (the S fragment
-//    layout of two n8 tiles is the A layout of one k16 step) and P V_h runs
-//    as one mma.sync per component of the head's 8 channels, the value
-//    fragments by ldmatrix.trans from the staged rows.
+//    one reference;
+//  * the float32 weights p become two bf16 A fragments, hi = bf16(p) and
+//    lo = bf16(p - hi) (the S fragment layout of two n8 tiles is the A layout
+//    of one k16 step), so P V carries p to about 2^-17 rather than bf16's
+//    2^-9: P V_h runs as two mma.sync per component of the head's 8 channels
+//    (the lo products one component pair behind the hi ones, off the same
+//    accumulator's dependency chain), the value fragments by ldmatrix.trans
+//    from the staged rows; z is the mma of the same hi and lo fragments with
+//    an all-ones fragment, the row sums of exactly the weights of P V.
 // The accumulator fragment of a lane holds, for targets g and g+8 and
 // channels 2t, 2t+1 of its head, every component d — exactly what the
 // per-channel EAAS epilogue needs, so the target coupling runs from registers.
@@ -86,6 +89,16 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
       "{%8,%9}, {%0,%1,%2,%3};\n"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// (a, b) as bf16x2 pairs hi + lo with hi = bf16(x) and lo = bf16(x - hi),
+// both rounded to nearest even: hi + lo equals x to about 2^-17 relative
+__device__ __forceinline__ void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  const float2 hf = __bfloat1622float2(h);
+  __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+  hi = *reinterpret_cast<uint32_t*>(&h);
+  lo = *reinterpret_cast<uint32_t*>(&l);
 }
 
 // A pipeline stage holds KS k-steps (KS * kTileK union rows): one barrier per
@@ -394,32 +407,51 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
         for (int e = 0; e < 4; ++e) pr[e] = fast_exp2(fmaf(v[j][e], qs, -mref0));
 #pragma unroll
         for (int e = 4; e < 8; ++e) pr[e] = fast_exp2(fmaf(v[j][e], qs, -mref1));
-        uint32_t pa[4];
-        {
-          __nv_bfloat162 b;
-          b = __floats2bfloat162_rn(pr[0], pr[1]); pa[0] = *reinterpret_cast<uint32_t*>(&b);  // row g,   k 2t
-          b = __floats2bfloat162_rn(pr[4], pr[5]); pa[1] = *reinterpret_cast<uint32_t*>(&b);  // row g+8, k 2t
-          b = __floats2bfloat162_rn(pr[2], pr[3]); pa[2] = *reinterpret_cast<uint32_t*>(&b);  // row g,   k 2t+8
-          b = __floats2bfloat162_rn(pr[6], pr[7]); pa[3] = *reinterpret_cast<uint32_t*>(&b);  // row g+8, k 2t+8
-        }
+        // the weights as a bf16 pair hi + lo (hi = bf16(p), lo = bf16(p - hi)):
+        // 16 significant bits, so P V and the normaliser carry the float32
+        // weights to about 2^-17 instead of bf16's 2^-9
+        uint32_t pa[4], pl[4];
+        split_bf16(pr[0], pr[1], pa[0], pl[0]);   // row g,   k 2t
+        split_bf16(pr[4], pr[5], pa[1], pl[1]);   // row g+8, k 2t
+        split_bf16(pr[2], pr[3], pa[2], pl[2]);   // row g,   k 2t+8
+        split_bf16(pr[6], pr[7], pa[3], pl[3]);   // row g+8, k 2t+8
         mma_bf16(zacc, pa, kOnes, kOnes);
 
-        // ---- O += P V (one n8 tile per component of this head's 8 channels)
+        // ---- O += P V (one n8 tile per component of this head's 8 channels).
+        // The lo products run one component pair behind the hi products, so
+        // that no mma waits on the one just issued into the same accumulator.
         const uint32_t vb = smem_u32(vbuf + (size_t(buf) * RS + j * kTileK) * VSTR);
         const int mj = lane >> 3;                 // matrix of this lane's row address
         const int row = (lane & 7) + 8 * (mj & 1);
         const uint32_t base = vb + row * VSTR + h * 16;
+        uint32_t vprev[4];
 #pragma unroll
         for (int d = 0; d + 1 < D; d += 2) {
           uint32_t vf[4];
           ldsm_x4_t(vf, base + (d + (mj >> 1)) * (C * 2));
           mma_bf16(acc[d], pa, vf[0], vf[1]);
           mma_bf16(acc[d + 1], pa, vf[2], vf[3]);
+          if (d >= 2) {
+            mma_bf16(acc[d - 2], pl, vprev[0], vprev[1]);
+            mma_bf16(acc[d - 1], pl, vprev[2], vprev[3]);
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) vprev[e] = vf[e];
         }
         if constexpr (D % 2) {
           uint32_t vf[2];
           ldsm_x2_t(vf, base + (D - 1) * (C * 2));
           mma_bf16(acc[D - 1], pa, vf[0], vf[1]);
+          if constexpr (D > 1) {
+            mma_bf16(acc[D - 3], pl, vprev[0], vprev[1]);
+            mma_bf16(acc[D - 2], pl, vprev[2], vprev[3]);
+          }
+          mma_bf16(zacc, pl, kOnes, kOnes);
+          mma_bf16(acc[D - 1], pl, vf[0], vf[1]);
+        } else {
+          mma_bf16(acc[D - 2], pl, vprev[0], vprev[1]);
+          mma_bf16(acc[D - 1], pl, vprev[2], vprev[3]);
+          mma_bf16(zacc, pl, kOnes, kOnes);
         }
       }   // k-steps of the stage
     }

@@ -324,7 +324,41 @@ struct BwdLayout {
   static constexpr int TPL = (NCH + 31) / 32;    // chunks per lane
   static constexpr int CPW = C / 8;              // chunks per component
   static_assert(32 % CPW == 0, "C/8 must divide 32");
+  // Past 5 chunks per lane (lmax 3 with 128 channels) the warp's own row
+  // (dm_i in the target pass, h'_j in the source pass) waits in the warp's
+  // shared-memory slice instead of registers, and the kernel takes the whole
+  // register file (one CTA per SM): three register rows of 64 floats would
+  // spill.
+  static constexpr bool OWN_SMEM = TPL > 5;
+  static constexpr int MINB = OWN_SMEM ? 1 : 3;
 };
+
+// this lane's chunks of a row into a warp's shared-memory slice (float32)
+template <int NCH, typename T>
+__device__ __forceinline__ void stage_row(const T* __restrict__ row, float* own, int lane) {
+  for (int q = lane; q < NCH; q += 32) {
+    Chunk8<T> c;
+    c.load(row + 8 * q);
+    float v[8];
+    c.to_f32(v);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) own[8 * q + e] = v[e];
+  }
+}
+// per-lane partial dot product of a staged row and a register row
+template <int TPL, int NCH>
+__device__ __forceinline__ float chunk_dot_smem(const float* own, const float (&b)[TPL][8],
+                                                int lane) {
+  float s = 0.f;
+#pragma unroll
+  for (int t = 0; t < TPL; ++t) {
+    const int q = lane + 32 * t;
+    if (q < NCH)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s = fmaf(own[8 * q + e], b[t][e], s);
+  }
+  return s;
+}
 
 // per-lane partial dot product of two rows held as chunks
 template <int TPL, int NCH>
@@ -353,10 +387,12 @@ __device__ __forceinline__ void load_row(const T* __restrict__ row, float (&v)[T
 
 // Step 3: one warp per target.
 template <int L, int C, typename T>
-__global__ void __launch_bounds__(kBwdWarps * 32, 3)
+__global__ void __launch_bounds__(kBwdWarps * 32, BwdLayout<L, C, T>::MINB)
 attn_bwd_target_kernel(const __grid_constant__ BwdParams p) {
   using Ly = BwdLayout<L, C, T>;
   constexpr int D = Ly::D, NCH = Ly::NCH, TPL = Ly::TPL, CPW = Ly::CPW;
+  constexpr bool OWN_SMEM = Ly::OWN_SMEM;
+  extern __shared__ float smem[];
   const int lane = threadIdx.x & 31;
   const int i = blockIdx.x * kBwdWarps + (threadIdx.x >> 5);
   if (i >= p.n) return;   // whole warp
@@ -407,8 +443,15 @@ attn_bwd_target_kernel(const __grid_constant__ BwdParams p) {
     }
   }
   const float lse = z > 0.f ? mx + log2f(z) : -INFINITY;
-  float dmv[TPL][8];
-  load_row<TPL, NCH>(dmp + (size_t)i * D * C, dmv, lane);
+  // dm_i: registers, or (OWN_SMEM) the warp's slice, where the epilogue's G_i goes later
+  float* own = smem + (threadIdx.x >> 5) * (2 * D * C + wig_size(L));
+  float dmv[OWN_SMEM ? 1 : TPL][8];
+  if constexpr (OWN_SMEM) {
+    stage_row<NCH>(dmp + (size_t)i * D * C, own, lane);
+    __syncwarp();
+  } else {
+    load_row<TPL, NCH>(dmp + (size_t)i * D * C, dmv, lane);
+  }
 
   // sweep 2 (key and value rows): with the exact weights alpha_ij,
   //   m_i = sum alpha h'_j, Delta_i = sum alpha dalpha,
@@ -430,7 +473,10 @@ attn_bwd_target_kernel(const __grid_constant__ BwdParams p) {
     const float a = exp2f(logit(j) - lse);
     float hv[TPL][8];
     load_row<TPL, NCH>(hp + (size_t)j * D * C, hv, lane);
-    const float da = head_sum<CPW>(chunk_dot<TPL, NCH>(dmv, hv, lane), p.cph);
+    float dot;
+    if constexpr (OWN_SMEM) dot = chunk_dot_smem<TPL, NCH>(own, hv, lane);
+    else dot = chunk_dot<TPL, NCH>(dmv, hv, lane);
+    const float da = head_sum<CPW>(dot, p.cph);
     delta = fmaf(a, da, delta);
 #pragma unroll
     for (int t = 0; t < TPL; ++t)
@@ -466,10 +512,10 @@ attn_bwd_target_kernel(const __grid_constant__ BwdParams p) {
   if (p.dpos) {
     // the target coupling's part of dL/dr_i: g = G_i, x = m_i
     constexpr int WS = wig_size(L);
-    extern __shared__ float smem[];
-    float* gs = smem + (threadIdx.x >> 5) * (2 * D * C + WS);
+    float* gs = own;              // (OWN_SMEM: dm_i is no longer read)
     float* xs = gs + D * C;
     float* Dsm = xs + D * C;
+    __syncwarp();
 #pragma unroll
     for (int t = 0; t < TPL; ++t) {
       const int q = lane + 32 * t;
@@ -494,10 +540,11 @@ attn_bwd_target_kernel(const __grid_constant__ BwdParams p) {
 // Step 4: one warp per source atom over its in-list, then the adjoint of the
 // source coupling in the epilogue.
 template <int L, int C, typename T>
-__global__ void __launch_bounds__(kBwdWarps * 32, 3)
+__global__ void __launch_bounds__(kBwdWarps * 32, BwdLayout<L, C, T>::MINB)
 attn_bwd_source_kernel(const __grid_constant__ BwdParams p) {
   using Ly = BwdLayout<L, C, T>;
   constexpr int D = Ly::D, NCH = Ly::NCH, TPL = Ly::TPL, CPW = Ly::CPW;
+  constexpr bool OWN_SMEM = Ly::OWN_SMEM;
   constexpr int WS = wig_size(L);
   extern __shared__ float smem[];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
@@ -520,8 +567,15 @@ attn_bwd_source_kernel(const __grid_constant__ BwdParams p) {
     else kc.zero();
     kc.to_f32(kv);
   }
-  float hv[TPL][8];
-  load_row<TPL, NCH>(hp + (size_t)j * D * C, hv, lane);
+  // h'_j: registers, or (OWN_SMEM) the warp's slice, where the epilogue's dh'_j goes later
+  float* gbuf = smem + wib * (D * C + WS + (p.dpos ? D * C : 0));
+  float hv[OWN_SMEM ? 1 : TPL][8];
+  if constexpr (OWN_SMEM) {
+    stage_row<NCH>(hp + (size_t)j * D * C, gbuf, lane);
+    __syncwarp();
+  } else {
+    load_row<TPL, NCH>(hp + (size_t)j * D * C, hv, lane);
+  }
   float dhp[TPL][8];
 #pragma unroll
   for (int t = 0; t < TPL; ++t)
@@ -550,7 +604,10 @@ attn_bwd_source_kernel(const __grid_constant__ BwdParams p) {
     const float a = exp2f(sl - __ldg(p.lse + (size_t)i * p.H + head));
     float dmv[TPL][8];
     load_row<TPL, NCH>(dmp + (size_t)i * D * C, dmv, lane);
-    const float da = head_sum<CPW>(chunk_dot<TPL, NCH>(dmv, hv, lane), p.cph);
+    float dot;
+    if constexpr (OWN_SMEM) dot = chunk_dot_smem<TPL, NCH>(gbuf, dmv, lane);
+    else dot = chunk_dot<TPL, NCH>(dmv, hv, lane);
+    const float da = head_sum<CPW>(dot, p.cph);
     const float ds = a * (da - __ldg(p.delta + (size_t)i * p.H + head));
 #pragma unroll
     for (int t = 0; t < TPL; ++t)
@@ -567,8 +624,8 @@ attn_bwd_source_kernel(const __grid_constant__ BwdParams p) {
   }
 
   // epilogue: dh_j = T*(dh'_j; r_j, w1), one channel per lane at a time
-  float* gbuf = smem + wib * (D * C + WS + (p.dpos ? D * C : 0));
   float* Dsm = gbuf + D * C;
+  __syncwarp();                   // (OWN_SMEM: h'_j is no longer read)
 #pragma unroll
   for (int t = 0; t < TPL; ++t) {
     const int q = lane + 32 * t;
@@ -739,8 +796,10 @@ template <int L, int C, typename T>
 int launch_attn_bwd(const BwdParams& p, cudaStream_t st) {
   constexpr int D = (L + 1) * (L + 1);
   const int grid = (p.n + kBwdWarps - 1) / kBwdWarps;
-  // per warp: G_i, m_i and a Wigner-D scratch when dL/dr is wanted
-  const size_t tshm = p.dpos ? size_t(kBwdWarps) * (2 * D * C + wig_size(L)) * sizeof(float) : 0;
+  // per warp: G_i, m_i and a Wigner-D scratch when dL/dr is wanted (the first
+  // D * C floats also hold dm_i when the layout keeps it in shared memory)
+  const size_t tshm = (p.dpos || BwdLayout<L, C, T>::OWN_SMEM)
+                          ? size_t(kBwdWarps) * (2 * D * C + wig_size(L)) * sizeof(float) : 0;
   auto tkern = attn_bwd_target_kernel<L, C, T>;
   if (tshm > 48 * 1024 &&
       cudaFuncSetAttribute(tkern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(tshm)) != cudaSuccess)
@@ -904,8 +963,9 @@ int launch_exclusive_scan(const int* d_in, int n, int* d_out, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
 }
 
-// The tiled path (bwd_tc_supported): h' and dm in float32 rounded to tf32
-// as they are stored,
+// The tiled path (bwd_tc_supported): h' in float32 rounded to tf32 as it is
+// stored, dm in float32 (rounded to tf32 where it enters a single tf32
+// product, split into tf32 hi + lo where it forms dL/dh'),
 // the forward plan (target tiles), the in-lists, then the statistics, target
 // and source passes, the source coupling's adjoint and dL/dr.
 template <int L>
@@ -917,7 +977,7 @@ int launch_backward_tiled(const egat_shape& s, const BwdWs& w, const void* d_h, 
   float* hp = static_cast<float*>(w.hp);
   float* dm = static_cast<float*>(w.dm);
   int e = launch_eaas_source_f32out(s, d_h, d_pos, d_w1, hp, st, true);
-  if (e == EGAT_OK) e = launch_adjoint<L, float, true>(s, d_g, d_pos, d_w2, dm, st);
+  if (e == EGAT_OK) e = launch_adjoint<L, float>(s, d_g, d_pos, d_w2, dm, st);
   if (e == EGAT_OK) e = launch_build_plan(s.n, s.K, s.lmax, d_nbr, d_cnt, d_order, d_pos, w.tc.plan, st);
   if (e != EGAT_OK) return e;
   // in-lists (unsorted: the source plan's union is ordered by its bitmap)

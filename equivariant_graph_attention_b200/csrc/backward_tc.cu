@@ -35,6 +35,9 @@
 // bounded.  The softmax derivative subtracts nearly equal numbers, so its
 // operands are float32 rounded to tf32 (10-bit mantissa), not bf16: the
 // modelled error of dq on the 4,096-atom workload is 3e-3 of the row norm.
+// dh' = alpha^T dm feeds the adjoint source coupling, whose |r|^l-scaled
+// terms cancel on small channels of dL/dh; there both operands enter as tf32
+// pairs hi + lo (three products), so dh' carries float32-level accuracy.
 // Every sum runs in a fixed order (union order, then the stage's k-steps):
 // deterministic, no atomics on results.
 #include <cfloat>
@@ -82,7 +85,7 @@ struct BtcParams {
   const __nv_bfloat16* q;   // [n][H][dk]
   const __nv_bfloat16* k;   // [n][H][dk]
   const float* hp;          // h' [n][D][C], values rounded to tf32
-  const float* dm;          // dL/dm [n][D][C], values rounded to tf32
+  const float* dm;          // dL/dm [n][D][C], float32 (not rounded)
   const int32_t* order;     // tile slot -> atom (null: identity)
   const int* ulen;          // [tiles]
   const int* uni;           // union indices, tile base = toff ? toff[t] : t * cap
@@ -151,14 +154,15 @@ __device__ __forceinline__ void acc_as_a(uint32_t (&a)[4], const float (&c)[4]) 
   a[2] = to_tf32(c[1]);
   a[3] = to_tf32(c[3]);
 }
-// The same as a pair (hi, lo) with hi + lo = c to about 2^-22 relative: two
-// tf32 products then carry c at nearly float32 precision.
+// The same as a pair (hi, lo) with hi + lo = c to about 2^-21 relative (lo
+// left as float32 bits, which the product truncates to tf32): two tf32
+// products then carry c at nearly float32 precision.
 __device__ __forceinline__ void acc_as_a_split(uint32_t (&hi)[4], uint32_t (&lo)[4], const float (&c)[4]) {
   acc_as_a(hi, c);
-  lo[0] = to_tf32(c[0] - __uint_as_float(hi[0]));
-  lo[1] = to_tf32(c[2] - __uint_as_float(hi[1]));
-  lo[2] = to_tf32(c[1] - __uint_as_float(hi[2]));
-  lo[3] = to_tf32(c[3] - __uint_as_float(hi[3]));
+  lo[0] = __float_as_uint(c[0] - __uint_as_float(hi[0]));
+  lo[1] = __float_as_uint(c[2] - __uint_as_float(hi[1]));
+  lo[2] = __float_as_uint(c[1] - __uint_as_float(hi[2]));
+  lo[3] = __float_as_uint(c[3] - __uint_as_float(hi[3]));
 }
 
 __device__ __forceinline__ int slot_atom(const int32_t* order, int tile, int r, int n) {
@@ -444,10 +448,12 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_target_tc_kernel(const __gri
 #pragma unroll
     for (int d = 0; d < D; ++d) {
       const size_t o = size_t(d) * kBC + h * 8 + t;
-      dma[d][0] = tg0 >= 0 ? __ldg(d32 + (size_t)tg0 * D * kBC + o) : 0u;
-      dma[d][1] = tg1 >= 0 ? __ldg(d32 + (size_t)tg1 * D * kBC + o) : 0u;
-      dma[d][2] = tg0 >= 0 ? __ldg(d32 + (size_t)tg0 * D * kBC + o + 4) : 0u;
-      dma[d][3] = tg1 >= 0 ? __ldg(d32 + (size_t)tg1 * D * kBC + o + 4) : 0u;
+      // dm is float32 in memory (the source pass splits it into hi + lo);
+      // this pass's products take it rounded to tf32
+      dma[d][0] = tg0 >= 0 ? to_tf32(__uint_as_float(__ldg(d32 + (size_t)tg0 * D * kBC + o))) : 0u;
+      dma[d][1] = tg1 >= 0 ? to_tf32(__uint_as_float(__ldg(d32 + (size_t)tg1 * D * kBC + o))) : 0u;
+      dma[d][2] = tg0 >= 0 ? to_tf32(__uint_as_float(__ldg(d32 + (size_t)tg0 * D * kBC + o + 4))) : 0u;
+      dma[d][3] = tg1 >= 0 ? to_tf32(__uint_as_float(__ldg(d32 + (size_t)tg1 * D * kBC + o + 4))) : 0u;
     }
   }
   const float lse0 = tg0 >= 0 ? __ldg(p.stats + (size_t)tg0 * (2 * kBH) + h) : 0.f;
@@ -636,6 +642,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_source_tc_kernel(const __gri
       float dp[4] = {0.f, 0.f, 0.f, 0.f};
       const uint32_t db = smem_u32(fb + (8 * nt + (lane & 7)) * FSTR + h * 32 + ((lane >> 3) & 1) * 16);
       float dp2[4] = {0.f, 0.f, 0.f, 0.f};   // odd components: a second, independent chain
+      // dm rows are float32; the tf32 product takes their leading 19 bits
 #pragma unroll
       for (int d = 0; d + 1 < D; d += 2) {
         uint32_t r[4];
@@ -655,9 +662,9 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_source_tc_kernel(const __gri
       ds[1] = P[1] * (dp[1] - dlb);
       ds[2] = P[2] * (dp[2] - dla);
       ds[3] = P[3] * (dp[3] - dlb);
-      uint32_t dsa[4], pa[4];
+      uint32_t dsa[4], pa[4], pl[4];
       acc_as_a(dsa, ds);
-      acc_as_a(pa, P);
+      acc_as_a_split(pa, pl, P);
       // dk += ds^T Q (B rows: union targets ca, cb)
       const unsigned char* q0 = qb + (8 * nt + 2 * t) * kKStr + h * 32;
 #pragma unroll
@@ -665,10 +672,35 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_source_tc_kernel(const __gri
         mma_tf32(dka[nd], dsa, bf16_bits_f32(q0 + (8 * nd + g) * 2),
                  bf16_bits_f32(q0 + kKStr + (8 * nd + g) * 2));
       // dh' += alpha^T dm (B rows: dm of ca, cb; columns: the head's channels)
-      const uint32_t* d0 = reinterpret_cast<const uint32_t*>(fb + (8 * nt + 2 * t) * FSTR) + h * 8 + g;
-      const uint32_t* d1 = d0 + FSTR / 4;
+      // in three tf32 products of the hi/lo splits of both operands,
+      // alpha_hi dm_hi + alpha_lo dm_hi + alpha_hi dm_lo: float32-level
+      // accuracy, which the adjoint source coupling needs (its |r|^l-scaled
+      // terms cancel on small channels of dL/dh)
+      // (hi = dm rounded to tf32; lo = dm - hi, which the product truncates to
+      // tf32: its error is 2^-10 of lo, about 2^-21 of dm).  Components go in
+      // pairs, so no product waits on the one just issued into its accumulator.
+      const float* d0 = reinterpret_cast<const float*>(fb + (8 * nt + 2 * t) * FSTR) + h * 8 + g;
+      const float* d1 = d0 + FSTR / 4;
+      auto split = [](float x, uint32_t& hi, uint32_t& lo) {
+        hi = to_tf32(x);
+        lo = __float_as_uint(x - __uint_as_float(hi));
+      };
 #pragma unroll
-      for (int d = 0; d < D; ++d) mma_tf32(dha[d], pa, d0[d * kBC], d1[d * kBC]);
+      for (int d = 0; d < D; d += 2) {
+        constexpr int kLast = D - 1;
+        const int e = d + 1 <= kLast ? d + 1 : kLast;
+        uint32_t ha0, ha1, la0, la1, hb0, hb1, lb0, lb1;
+        split(d0[d * kBC], ha0, la0);
+        split(d1[d * kBC], ha1, la1);
+        split(d0[e * kBC], hb0, lb0);
+        split(d1[e * kBC], hb1, lb1);
+        mma_tf32(dha[d], pa, ha0, ha1);
+        if (e != d) mma_tf32(dha[e], pa, hb0, hb1);
+        mma_tf32(dha[d], pl, ha0, ha1);
+        if (e != d) mma_tf32(dha[e], pl, hb0, hb1);
+        mma_tf32(dha[d], pa, la0, la1);
+        if (e != d) mma_tf32(dha[e], pa, lb0, lb1);
+      }
     }
   }
   S.drain(tid);

@@ -128,6 +128,18 @@ int launch_gather_rows(const void* d_src, long long n_src, long long row_bytes, 
 // and clear the count of waits that gave up (synchronises st); the self-test
 // launch.
 int take_wait_timeouts_attention(cudaStream_t st, unsigned int* count);
+int take_wait_timeouts_projection(cudaStream_t st, unsigned int* count);
+// Edge-centric eSCN convolution (the comparison workload): weights per channel
+// and its launch.
+int escn_num_weights_host(int lmax, int mmax);
+int launch_escn_conv(const egat_shape& s, int mmax, const void* d_h, const float* d_pos,
+                     const int32_t* d_nbr, const int32_t* d_cnt, const int32_t* d_order,
+                     const float* d_w, float* d_out, cudaStream_t st);
+// Invariant query/key projection from the degree-0 channels (tensor cores for
+// bf16 storage with C = 128 and H * dk = 256, a plain kernel otherwise).
+bool projection_tc_supported(const egat_shape& s);
+int launch_qk_projection(const egat_shape& s, const void* d_h, const float* d_wq, const float* d_wk,
+                         void* d_q, void* d_k, cudaStream_t st);
 int take_wait_timeouts_coupling(cudaStream_t st, unsigned int* count);
 int launch_wait_timeout_selftest(int polls, cudaStream_t st);
 int launch_attention_tc(const egat_shape& s, bool fused, const void* d_q, const void* d_k,

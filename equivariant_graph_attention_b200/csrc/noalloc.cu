@@ -10,11 +10,15 @@
 // library holds until the process exits.
 //
 // The array's name is only a host-side stand-in in host code, not a device
-// address, so it is never handed to a kernel directly.  The first call on
-// each device (with that device current) looks up the array's device address
-// with cudaGetSymbolAddress, checks the result and caches it for that device;
-// later calls on the device reuse the cached address.  That first call should
-// therefore come before any stream capture.
+// address, so it is never handed to a kernel directly.  The first successful
+// call on each device (with that device current) looks up the array's device
+// address with cudaGetSymbolAddress, checks the result and caches it for that
+// device; later calls on the device reuse the cached address.  A lookup that
+// fails is not cached: the next call tries again.  That first call should
+// come before any stream capture.  The cached address belongs to the device's
+// context: after cudaDeviceReset (or anything else that destroys the primary
+// context) it is stale, and this entry point must not be called again in that
+// process.
 //
 // All calls share the one array and it keeps the previous call's contents.
 // Nothing in it needs to start at zero: step 2 writes every element of h'
@@ -32,20 +36,23 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
-std::once_flag g_setup_once[kMaxDevices];
-void* g_scratch_ptr[kMaxDevices];
-cudaError_t g_setup_status[kMaxDevices];
+std::mutex g_setup_mutex;
+void* g_scratch_ptr[kMaxDevices];   // null until a lookup on that device succeeded
 
-// Device address of the scratch array on the current device (set-up once per device).
+// Device address of the scratch array on the current device (looked up once
+// per device; a failed lookup is retried by the next call).
 int scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return EGAT_ERR_CUDA;
-  std::call_once(g_setup_once[dev], [dev] {
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
-    g_setup_status[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();   // clear the sticky-free error so later calls start clean
+      return EGAT_ERR_CUDA;
+    }
     g_scratch_ptr[dev] = p;
-  });
-  if (g_setup_status[dev] != cudaSuccess || g_scratch_ptr[dev] == nullptr) return EGAT_ERR_CUDA;
+  }
   *out = g_scratch_ptr[dev];
   return EGAT_OK;
 }

@@ -41,7 +41,8 @@ EXPORTS = ["egat_version", "egat_strerror", "egat_num_paths", "egat_graph_worksp
            "egat_forward_workspace_bytes", "egat_forward", "egat_forward_noalloc",
            "egat_attention_plan_bytes", "egat_build_attention_plan", "egat_otf_attention_tiled",
            "egat_eaas_couple_planned", "egat_take_device_status", "egat_selftest_wait_timeout",
-           "egat_backward_workspace_bytes", "egat_backward", "egat_gather_rows"]
+           "egat_backward_workspace_bytes", "egat_backward", "egat_gather_rows",
+           "egat_qk_projection", "egat_escn_num_weights", "egat_escn_conv"]
 
 
 class EgatError(RuntimeError):
@@ -102,6 +103,12 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.egat_gather_rows.argtypes = [vp, i64, i64, vp, i64, vp, vp]
     lib.egat_backward.restype = ctypes.c_int
     lib.egat_backward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp, vp, vp, vp]
+    lib.egat_escn_num_weights.restype = ctypes.c_int
+    lib.egat_escn_num_weights.argtypes = [i32, i32]
+    lib.egat_escn_conv.restype = ctypes.c_int
+    lib.egat_escn_conv.argtypes = [sp, i32, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.egat_qk_projection.restype = ctypes.c_int
+    lib.egat_qk_projection.argtypes = [sp, vp, vp, vp, vp, vp, vp]
     lib.egat_take_device_status.restype = ctypes.c_int
     lib.egat_take_device_status.argtypes = [vp]
     lib.egat_selftest_wait_timeout.restype = ctypes.c_int
@@ -163,6 +170,15 @@ class Shape:
                           EGAT_BF16 if self.dtype == "bf16" else EGAT_F32,
                           EGAT_GRAPH_CSR if self.graph_mode == "csr" else EGAT_GRAPH_PADDED,
                           self.n_edges)
+
+
+def tc_attention_shape(shape: Shape) -> bool:
+    """Whether the shape is one the tensor-core attention path takes (bf16
+    storage, padded graph, C = 128, H = 16, dk = 16, lmax 1-3); the library
+    also requires n below its plan builder's limit (EGAT_ERR_UNSUPPORTED past
+    it)."""
+    return (shape.dtype == "bf16" and shape.graph_mode == "padded" and shape.C == 128
+            and shape.H == 16 and shape.dk == 16 and 1 <= shape.lmax <= 3)
 
 
 def egat_version() -> int:
@@ -236,6 +252,43 @@ def egat_eaas_couple(shape: Shape, x: torch.Tensor, pos: torch.Tensor, w: torch.
     rc = load_library().egat_eaas_couple(ctypes.byref(cs), _ptr(x), _ptr(pos), _ptr(w),
                                          _ptr(out), _stream(stream))
     _check("egat_eaas_couple", rc)
+    return out
+
+
+def egat_qk_projection(shape: Shape, h: torch.Tensor, wq: torch.Tensor, wk: torch.Tensor,
+                       q: Optional[torch.Tensor] = None, k: Optional[torch.Tensor] = None,
+                       stream=None):
+    """Invariant queries and keys from the degree-0 channels of h:
+    q[i, h, d] = sum_c h[i, 0, c] wq[c, h*dk + d] (k likewise); (q, k) [n, H, dk]
+    in the storage type.  wq, wk float32 [C, H*dk]."""
+    shp = (shape.n, shape.H, shape.dk)
+    if q is None:
+        q = torch.empty(shp, dtype=shape.torch_dtype, device=h.device)
+    if k is None:
+        k = torch.empty(shp, dtype=shape.torch_dtype, device=h.device)
+    cs = shape.c()
+    rc = load_library().egat_qk_projection(ctypes.byref(cs), _ptr(h), _ptr(wq), _ptr(wk), _ptr(q),
+                                           _ptr(k), _stream(stream))
+    _check("egat_qk_projection", rc)
+    return q, k
+
+
+def egat_escn_num_weights(lmax: int, mmax: int) -> int:
+    return load_library().egat_escn_num_weights(lmax, mmax)
+
+
+def egat_escn_conv(shape: Shape, mmax: int, h: torch.Tensor, pos: torch.Tensor, nbr: torch.Tensor,
+                   cnt: Optional[torch.Tensor], w: torch.Tensor, order: Optional[torch.Tensor] = None,
+                   out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Edge-centric eSCN convolution out_i = sum_j D(Q_ij) SO2_w(D(Q_ij)^T h_j) over
+    the padded graph; w float32 [egat_escn_num_weights(lmax, mmax), C]; out
+    float32 [n, D, C]."""
+    if out is None:
+        out = torch.empty((shape.n, shape.D, shape.C), dtype=torch.float32, device=h.device)
+    cs = shape.c()
+    rc = load_library().egat_escn_conv(ctypes.byref(cs), mmax, _ptr(h), _ptr(pos), _ptr(nbr),
+                                       _ptr(cnt), _ptr(order), _ptr(w), _ptr(out), _stream(stream))
+    _check("egat_escn_conv", rc)
     return out
 
 

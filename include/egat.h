@@ -262,7 +262,10 @@ EGAT_API int egat_forward(const egat_shape* s, const void* d_h, const float* d_p
  *    larger problems return EGAT_ERR_SCRATCH_LIMIT without launching.
  *  - The first call on a device, made with that device current, looks up the
  *    array's device address once (cudaGetSymbolAddress); make that first call
- *    before any stream capture.
+ *    before any stream capture.  A failed lookup returns EGAT_ERR_CUDA and is
+ *    retried by the next call.  The address belongs to the device's context:
+ *    after cudaDeviceReset the entry point must not be called again in that
+ *    process.
  *  - All calls share the array: calls whose work overlaps on the GPU race
  *    on it and must be serialised by the caller.  Nothing in it needs
  *    clearing between calls.
@@ -314,6 +317,66 @@ EGAT_API int egat_backward(const egat_shape* s, const void* d_h, const float* d_
                            float* d_dq, float* d_dk, float* d_dpos, void* stream);
 
 /*
+ * Invariant query/key projection ([TS] §2.2, Eq. 6: queries and keys are
+ * SO(3)-invariant scalar projections of the node features; the equivariant
+ * geometry travels only along the value path).  The invariant scalars of
+ * atom i are its degree-0 channels h_i^(0) = d_h[i][0][0..C) (component 0 of
+ * its row); each maps linearly, without bias, to every head:
+ *   q[i][h][d] = sum_c h[i][0][c] wq[c][h*dk + d],   k likewise with wk,
+ * so the logits q_i.k_j / sqrt(dk) are invariant.  The results feed
+ * egat_otf_attention / egat_forward as d_q, d_k.
+ *  d_h        [n][D][C] in s->dtype (only component 0 is read), 16-byte aligned;
+ *             0 <= lmax <= 3 (D = (lmax+1)^2), K and graph_mode are ignored
+ *  d_wq, d_wk float32 [C][H*dk]
+ *  d_q, d_k   [n][H][dk] in s->dtype (bf16: round to nearest even)
+ * bf16 storage with C = 128 and H*dk = 256 runs on tensor cores (the weights
+ * as bf16 pairs hi + lo, float32 accumulation); other shapes (C <= 1024,
+ * H*dk <= 1024) accumulate in float32 on CUDA cores.  n = 0 is a no-op.
+ * Errors: EGAT_ERR_ARG (null or misaligned pointer, bad dtype),
+ * EGAT_ERR_UNSUPPORTED, EGAT_ERR_CUDA; a bounded wait that gave up is
+ * reported by egat_take_device_status.
+ */
+EGAT_API int egat_qk_projection(const egat_shape* s, const void* d_h, const float* d_wq,
+                                const float* d_wk, void* d_q, void* d_k, void* stream);
+
+/*
+ * Edge-centric eSCN convolution, the comparison workload (the page
+ * "EquiformerV3: Scaling Efficient, Expressive, and General SE(3)-Equivariant Graph Attention Transformers",
+ * section "eSCN卷积与SO(2)线性层": rotate by D_ij from the
+ * relative position, apply an SO(2) linear layer within each degree's
+ * components, truncated at order M_max).  It is the edge-centric formulation
+ * that the node-centric factorisation of [EX] §3.1 replaces.  For each target
+ * i and each neighbour j of its padded list:
+ *   r_ij = r_j - r_i, Q_ij its alignment rotation (Q_ij z = r_ij/|r_ij|, as
+ *   in egat_eaas_couple; identity for r_ij = 0),
+ *   x~ = D(Q_ij)^T h_j  (each degree block by its real Wigner-D matrix),
+ *   per channel c, order by order (orders above mmax are zero):
+ *     y~^lo_0  = sum_li W0[lo][li] x~^li_0
+ *     y~^lo_+m = sum_li W1_m[lo][li] x~^li_+m - W2_m[lo][li] x~^li_-m
+ *     y~^lo_-m = sum_li W2_m[lo][li] x~^li_+m + W1_m[lo][li] x~^li_-m
+ *   out_i = sum_j D(Q_ij) y~.
+ * Messages are summed on chip (nothing per edge is written).
+ *  mmax      0 <= mmax <= lmax
+ *  d_h       [n][D][C] in s->dtype, 16-byte aligned
+ *  d_pos     float32 [n][3];  d_nbr / d_cnt the padded graph (d_cnt may be NULL)
+ *  d_order   optional int32 [n] traversal order (NULL = 0..n-1)
+ *  d_w       float32 [egat_escn_num_weights(lmax, mmax)][C]: W0 at row
+ *            lo*(lmax+1) + li, then for m = 1..mmax the W1_m block followed by
+ *            the W2_m block, (lmax+1-m)^2 rows each, row (lo-m)*(lmax+1-m) +
+ *            (li-m) within a block
+ *  d_out     float32 [n][D][C]
+ * Padded graphs only (CSR returns EGAT_ERR_UNSUPPORTED).  Shapes as the
+ * module header (1 <= lmax <= 3, C in {16, 32, 64, 128}).  Errors:
+ * EGAT_ERR_ARG, EGAT_ERR_UNSUPPORTED, EGAT_ERR_CUDA.
+ * egat_escn_num_weights returns the row count of d_w, 0 for lmax or mmax out
+ * of range.
+ */
+EGAT_API int egat_escn_num_weights(int32_t lmax, int32_t mmax);
+EGAT_API int egat_escn_conv(const egat_shape* s, int32_t mmax, const void* d_h, const float* d_pos,
+                            const int32_t* d_nbr, const int32_t* d_cnt, const int32_t* d_order,
+                            const float* d_w, float* d_out, void* stream);
+
+/*
  * Row gather, the packing step of a halo exchange (a spatial domain
  * decomposition across GPUs: each rank couples its own atoms and needs the
  * h' and k rows of the neighbours it does not own; one GPU reaches about
@@ -328,8 +391,8 @@ EGAT_API int egat_gather_rows(const void* d_src, int64_t n_src, int64_t row_byte
 
 /*
  * Device status.  The tensor-core attention kernel, the tile-staged source
- * coupling and the tiled backward passes wait on mbarriers for their bulk
- * copies; every such wait is bounded (about a second).  A wait that
+ * coupling, the tensor-core query/key projection and the tiled backward
+ * passes wait on mbarriers for their bulk copies; every such wait is bounded (about a second).  A wait that
  * gives up is counted on the device, the kernel stops waiting and finishes
  * with meaningless output instead of hanging.  The pages have no
  * counterpart: this is the library's failure report.
