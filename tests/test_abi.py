@@ -195,3 +195,17 @@ def test_gather_rows_validation(lib):
     assert lib.egat_gather_rows(ok, 10, 64, ok, 4, odd, None) == egat.EGAT_ERR_ARG
     assert lib.egat_gather_rows(odd, 10, 64, ok, 4, ok, None) == egat.EGAT_ERR_ARG
     assert lib.egat_gather_rows(None, 10, 64, ok, 4, ok, None) == egat.EGAT_ERR_ARG
+
+
+def test_escn_weight_count_matches_the_oracle():
+    """The library's SO(2) weight-row count (host code, no GPU work) equals the
+    oracle's and the input generator's for every (lmax, mmax); out of range
+    gives 0."""
+    from equivariant_graph_attention_b200 import egat, synth
+    from oracle.escn import num_weights
+    lib = egat.load_library()
+    for L in (1, 2, 3):
+        for m in range(L + 1):
+            assert lib.egat_escn_num_weights(L, m) == num_weights(L, m) == synth.escn_weight_count(L, m)
+    assert lib.egat_escn_num_weights(0, 0) == 0 and lib.egat_escn_num_weights(2, 3) == 0
+    assert lib.egat_escn_num_weights(4, 1) == 0 and lib.egat_escn_num_weights(2, -1) == 0

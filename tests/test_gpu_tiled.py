@@ -20,7 +20,9 @@ from oracle.attention import aggregate, forward as oracle_forward
 from oracle import so3
 from oracle.graph import radius_graph
 from equivariant_graph_attention_b200 import synth
-from tests.parity_util import TOL, block_rel_error, device_inputs, sample_targets, shape_of
+from oracle.storage import round_bf16
+from tests.parity_util import (FLOOR, ROUNDING_FLOOR, TOL, block_rel_error, channel_rel_error,
+                               device_inputs, sample_targets, shape_of)
 
 pytestmark = pytest.mark.gpu
 
@@ -127,9 +129,11 @@ def test_tiled_attention_parity(name):
         wl, np.minimum(g["cnt"].cpu().numpy(), wl.K))
     lists, _ = radius_graph(d["pos_q"], wl.cutoff_q, K=wl.K, rows=rows)
     ref = aggregate(d["q"], d["k"], vals, lists, rows)
-    err = block_rel_error(m[torch.tensor(rows).cuda()].cpu().numpy(), ref, wl.lmax)
-    print(f"tiled m {name}: max block error {err:.2e}")
-    assert err < TOL["bf16"]
+    got = m[torch.tensor(rows).cuda()].cpu().numpy()
+    err = block_rel_error(got, ref, wl.lmax)
+    e = channel_rel_error(got, ref, wl.lmax, FLOOR["bf16"])
+    print(f"tiled m {name}: max block error {err:.2e}, per-channel {e:.2e}")
+    assert err < TOL["bf16"] and e < TOL["bf16"]
 
 
 @pytest.mark.parametrize("name", BF16)
@@ -165,6 +169,9 @@ def test_per_target_fused_kernel_parity_bf16():
     lists, _ = radius_graph(d["pos_q"], wl.cutoff_q, K=wl.K)
     ref = oracle_forward(d["h"], d["pos"], d["q"], d["k"], d["w1"], d["w2"], wl.lmax, lists)
     assert block_rel_error(out, ref, wl.lmax) < TOL["bf16"]
+    refs = oracle_forward(d["h"], d["pos"], d["q"], d["k"], d["w1"], d["w2"], wl.lmax, lists,
+                          store=round_bf16)
+    assert channel_rel_error(out, refs, wl.lmax, floor=ROUNDING_FLOOR) < TOL["bf16"]
 
 
 @pytest.mark.parametrize("lmax", [1, 2, 3])
@@ -194,3 +201,6 @@ def test_tiled_edge_cases(lmax, n):
     if n >= 4:
         assert np.all(out[3] == 0.0)
     assert block_rel_error(out, ref, lmax) < TOL["bf16"]
+    refs = oracle_forward(feats["h"], feats["pos"], feats["q"], feats["k"], feats["w1"],
+                          feats["w2"], lmax, lists, store=round_bf16)
+    assert channel_rel_error(out, refs, lmax, floor=ROUNDING_FLOOR) < TOL["bf16"]

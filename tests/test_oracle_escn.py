@@ -1,6 +1,6 @@
 """Pins of the oracle's edge-centric eSCN convolution (oracle/escn.py).
 
-"EquiformerV3" page, eSCN convolution and SO(2) linear layer: rotate by D_ij,
+"EquiformerV3: Scaling Efficient, Expressive, and General SE(3)-Equivariant Graph Attention Transformers", section "eSCN卷积与SO(2)线性层": rotate by D_ij,
 apply an SO(2) linear layer within each degree's components, rotate back.
 A plausible mistake (a transposed rotation, a wrong sign in the +-m blocks, a
 mixed-up weight row, the wrong edge direction) fails one of:

@@ -18,7 +18,7 @@ import pytest
 import torch
 
 from equivariant_graph_attention_b200 import synth
-from tests.parity_util import TOL, block_rel_error, device_inputs, shape_of
+from tests.parity_util import FLOOR, TOL, block_rel_error, channel_rel_error, device_inputs, shape_of
 
 pytestmark = pytest.mark.gpu
 
@@ -46,6 +46,8 @@ def test_noalloc_matches_forward_on_two_calls(name):
         torch.cuda.synchronize()
         err = block_rel_error(out.cpu().numpy(), ref.cpu().numpy(), wl.lmax)
         assert err < TOL[wl.dtype], (name, seed, err)
+        e = channel_rel_error(out.cpu().numpy(), ref.cpu().numpy(), wl.lmax, FLOOR[wl.dtype])
+        assert e < TOL[wl.dtype], (name, seed, e)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
