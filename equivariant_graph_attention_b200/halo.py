@@ -19,8 +19,8 @@ is the exchange of step 2; the forward needs nothing else from other ranks.
 """
 from __future__ import annotations
 
-from dataclasses import dataclass
-from typing import Callable, List, Optional
+from dataclasses import dataclass, field
+from typing import Callable, Dict, List, Optional
 
 import numpy as np
 import torch
@@ -38,10 +38,28 @@ class HaloPlan:
     send: List[np.ndarray]     # per rank: local indices (into owned) of the rows it receives from us
     local_nbr: np.ndarray      # int32 [n_owned + n_halo, K]: owned rows in local indices, halo rows -1
     local_cnt: np.ndarray      # int32 [n_owned + n_halo]
+    _dev: Dict[str, Dict[str, torch.Tensor]] = field(default_factory=dict, repr=False)
 
     @property
     def n_owned(self) -> int:
         return int(self.owned.size)
+
+    def on(self, device) -> Dict[str, torch.Tensor]:
+        """The plan's index arrays on `device`, copied once and kept: owned ids
+        (int32), local ids (owned then halo, int64), the concatenated send lists
+        (int32), the local lists and counts, and the local traversal order."""
+        key = str(device)
+        if key not in self._dev:
+            t = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to(device=device, dtype=dt)
+            self._dev[key] = {
+                "own": t(self.owned, torch.int32),
+                "loc": t(np.concatenate([self.owned, self.halo]), torch.int64),
+                "send": t(np.concatenate(self.send) if self.send else np.zeros(0), torch.int32),
+                "nbr": t(self.local_nbr, torch.int32),
+                "cnt": t(self.local_cnt, torch.int32),
+                "order": torch.arange(self.n_local, dtype=torch.int32, device=device),
+            }
+        return self._dev[key]
 
     @property
     def n_local(self) -> int:
@@ -109,52 +127,110 @@ def build_plan(nbr: np.ndarray, cnt: Optional[np.ndarray], order: np.ndarray, wo
 
 
 def exchange(plan: HaloPlan, own_rows: torch.Tensor, group=None,
-             pack: Optional[Callable[[torch.Tensor, torch.Tensor], torch.Tensor]] = None) -> torch.Tensor:
+             pack: Optional[Callable[[torch.Tensor, torch.Tensor], torch.Tensor]] = None,
+             transport: Optional[Callable] = None) -> torch.Tensor:
     """Rows of the halo atoms (in plan.halo order) from their owners, given this
     rank's own rows [n_owned, ...]: the send buffer is packed on the device
-    (egat_gather_rows) and one all-to-all moves it.  `pack(rows, idx)` replaces
-    the device packing (tests on CPU ranks)."""
-    import torch.distributed as dist
+    (egat_gather_rows, grouped by destination rank) and one all-to-all moves it.
+    `pack(rows, idx)` replaces the device packing (tests on CPU ranks);
+    `transport(send_buf, in_splits, out_splits)` replaces the all-to-all (one
+    GPU standing in for several ranks, one after the other)."""
     dev = own_rows.device
-    send_idx = torch.from_numpy(np.concatenate(plan.send).astype(np.int32)).to(dev)
+    if own_rows.is_cuda:
+        send_idx = plan.on(dev)["send"]
+    else:
+        send_idx = torch.from_numpy(np.concatenate(plan.send).astype(np.int32))
     if pack is None:
         if not own_rows.is_cuda:
             raise RuntimeError("exchange packs rows on the GPU; pass `pack` for CPU tensors")
         send_buf = egat.egat_gather_rows(own_rows.contiguous(), send_idx)
     else:
         send_buf = pack(own_rows, send_idx)
-    recv = torch.empty((sum(plan.recv_counts),) + tuple(own_rows.shape[1:]), dtype=own_rows.dtype,
+    in_splits = [int(s.size) for s in plan.send]
+    out_splits = list(plan.recv_counts)
+    if transport is not None:
+        return transport(send_buf, in_splits, out_splits)
+    import torch.distributed as dist
+    recv = torch.empty((sum(out_splits),) + tuple(own_rows.shape[1:]), dtype=own_rows.dtype,
                        device=dev)
-    dist.all_to_all_single(recv, send_buf, output_split_sizes=list(plan.recv_counts),
-                           input_split_sizes=[int(s.size) for s in plan.send], group=group)
+    dist.all_to_all_single(recv, send_buf, output_split_sizes=out_splits,
+                           input_split_sizes=in_splits, group=group)
     return recv
+
+
+@dataclass
+class RankState:
+    """One rank's device arrays for a step: its own coupled rows and keys, its
+    own queries, and the positions of its local atoms (owned, then halo)."""
+    hp_own: torch.Tensor
+    k_own: torch.Tensor
+    q_own: torch.Tensor
+    pos_loc: torch.Tensor
+
+
+def _local_shape(shape: "egat.Shape", n: int) -> "egat.Shape":
+    return egat.Shape(n=n, lmax=shape.lmax, C=shape.C, H=shape.H, dk=shape.dk, K=shape.K,
+                      dtype=shape.dtype)
+
+
+def couple_rank(plan: HaloPlan, shape: "egat.Shape", h: torch.Tensor, pos: torch.Tensor,
+                q: torch.Tensor, k: torch.Tensor, w1: torch.Tensor) -> RankState:
+    """Step 2 for this rank's own atoms (egat_eaas_couple on its rows of h); each
+    rank reads only its own rows of h, q and k and the positions of its local
+    atoms."""
+    a = plan.on(h.device)
+    own_i32, loc = a["own"], a["loc"]
+    h_own = egat.egat_gather_rows(h.contiguous(), own_i32)
+    q_own = egat.egat_gather_rows(q.contiguous(), own_i32)
+    k_own = egat.egat_gather_rows(k.contiguous(), own_i32)
+    pos_loc = pos.index_select(0, loc).contiguous()
+    hp_own = egat.egat_eaas_couple(_local_shape(shape, plan.n_owned), h_own,
+                                   pos_loc[:plan.n_owned].contiguous(), w1)
+    return RankState(hp_own, k_own, q_own, pos_loc)
+
+
+def attend_rank(plan: HaloPlan, shape: "egat.Shape", st: RankState, hp_halo: torch.Tensor,
+                k_halo: torch.Tensor, w2: torch.Tensor) -> torch.Tensor:
+    """Steps 3+4 for this rank's own atoms over its local arrays (own rows, then
+    the halo rows received): ^h float32 [n_owned, D, C] in plan.owned order.
+
+    The local system lists the owned atoms first, in the global traversal
+    order (a spatially compact block), then the halo atoms, which appear only
+    as sources (empty lists).  Shapes of the tensor-core path build the
+    attention plan over the local arrays and run the tiled kernel; its tiles of
+    halo slots have empty unions and only write zero rows, which are dropped.
+    Other shapes run the per-target kernel."""
+    dev = st.hp_own.device
+    n_loc = plan.n_local
+    hp_loc = torch.cat([st.hp_own, hp_halo])
+    k_loc = torch.cat([st.k_own, k_halo])
+    q_loc = torch.cat([st.q_own, torch.zeros((n_loc - plan.n_owned,) + tuple(st.q_own.shape[1:]),
+                                             dtype=st.q_own.dtype, device=dev)])
+    a = plan.on(dev)
+    nbr, cnt = a["nbr"], a["cnt"]
+    s_loc = _local_shape(shape, n_loc)
+    if n_loc == 0:
+        return torch.zeros((0, s_loc.D, shape.C), dtype=torch.float32, device=dev)
+    if egat.tc_attention_shape(s_loc):
+        try:
+            ap = egat.egat_build_attention_plan(s_loc, nbr, cnt, a["order"], st.pos_loc)
+            out = egat.egat_otf_attention_tiled(s_loc, q_loc, k_loc, hp_loc, ap, w2, fused=True)
+            return out[:plan.n_owned]
+        except egat.EgatError as e:   # a local system past the plan builder's size limit
+            if e.code != egat.EGAT_ERR_UNSUPPORTED:
+                raise
+    out = egat.egat_otf_attention_coupled(s_loc, q_loc, k_loc, hp_loc, nbr, cnt, st.pos_loc, w2)
+    return out[:plan.n_owned]
 
 
 def forward_rank(plan: HaloPlan, shape: "egat.Shape", h: torch.Tensor, pos: torch.Tensor,
                  q: torch.Tensor, k: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor,
                  group=None) -> torch.Tensor:
     """^h of this rank's atoms (float32 [n_owned, D, C], in plan.owned order) for the
-    global inputs h, pos, q, k of the `shape` system (each rank reads only its own
-    rows of h, q and k, and the positions of its own and its halo atoms)."""
-    dev = h.device
-    own = torch.from_numpy(plan.owned).to(dev)
-    loc = torch.from_numpy(np.concatenate([plan.owned, plan.halo])).to(dev)
-    n_own, n_loc = plan.n_owned, plan.n_local
-    own_i32 = own.to(torch.int32)
-    h_own = egat.egat_gather_rows(h.contiguous(), own_i32)
-    q_own = egat.egat_gather_rows(q.contiguous(), own_i32)
-    k_own = egat.egat_gather_rows(k.contiguous(), own_i32)
-    pos_loc = pos.index_select(0, loc).contiguous()
-    shape_own = egat.Shape(n=n_own, lmax=shape.lmax, C=shape.C, H=shape.H, dk=shape.dk, K=shape.K,
-                           dtype=shape.dtype)
-    hp_own = egat.egat_eaas_couple(shape_own, h_own, pos_loc[:n_own].contiguous(), w1)
-    hp_loc = torch.cat([hp_own, exchange(plan, hp_own, group)])
-    k_loc = torch.cat([k_own, exchange(plan, k_own, group)])
-    q_loc = torch.cat([q_own, torch.zeros((n_loc - n_own,) + tuple(q.shape[1:]), dtype=q.dtype,
-                                          device=dev)])
-    nbr = torch.from_numpy(plan.local_nbr).to(dev)
-    cnt = torch.from_numpy(plan.local_cnt).to(dev)
-    shape_loc = egat.Shape(n=n_loc, lmax=shape.lmax, C=shape.C, H=shape.H, dk=shape.dk, K=shape.K,
-                           dtype=shape.dtype)
-    out = egat.egat_otf_attention_coupled(shape_loc, q_loc, k_loc, hp_loc, nbr, cnt, pos_loc, w2)
-    return out[:n_own]
+    global inputs h, pos, q, k of the `shape` system: step 2 on the owned atoms,
+    one exchange of the boundary atoms' h' and k rows (NCCL all-to-all in
+    `group`), then steps 3+4 over the local arrays."""
+    st = couple_rank(plan, shape, h, pos, q, k, w1)
+    hp_halo = exchange(plan, st.hp_own, group)
+    k_halo = exchange(plan, st.k_own, group)
+    return attend_rank(plan, shape, st, hp_halo, k_halo, w2)
