@@ -1,7 +1,7 @@
 """Edge-centric eSCN convolution of the oracle.  Test infrastructure only.
 
-"EquiformerV3" page, section on the eSCN convolution and the SO(2) linear
-layer: eSCN splits a tensor product into two steps — rotate the features by
+"EquiformerV3: Scaling Efficient, Expressive, and General SE(3)-Equivariant
+Graph Attention Transformers", section "eSCN卷积与SO(2)线性层": eSCN splits a tensor product into two steps — rotate the features by
 D_ij, the rotation that the relative position r_ij defines, then apply an
 SO(2) linear layer that acts only within the 2l+1 components of each degree
 (with components of order |m| > M_max dropped).  It is the edge-centric
