@@ -29,13 +29,15 @@ loaded once per edge) rides along as ``effective``: the kernel serves those
 loads from L2 and shared memory, so that figure exceeds the HBM peak and is
 not a bound.
 
-Multi-GPU (torchrun): every rank runs its own independent system (same shape,
-seeded by rank) — the units are independent problems, so there is no
-data-path collective; timing is the max over ranks.  ``--decompose`` instead
-splits ONE system across the ranks by space (halo exchange of h' and k rows,
-``equivariant_graph_attention_b200.halo``) and times one decomposed forward
-step per rank.  ``--impl reference`` times the CPU oracle on the same workload
-(rank 0 only, on the host's cores).
+Multi-GPU (torchrun, N > 1): ONE system is split across the ranks by space
+(``equivariant_graph_attention_b200.halo``: each rank couples its own atoms,
+one all-to-all exchanges the boundary atoms' h' and k rows, each rank runs the
+attention of its own atoms) and the line reports the system's atoms per second
+of the slowest rank's decomposed step (strong scaling).  ``--replicas`` runs
+independent systems instead (same shape, seeded by rank; no data-path
+collective; weak scaling); ``--decompose`` forces the split at N = 1 too.
+Timing is the max over ranks.  ``--impl reference`` times the CPU oracle on the
+same workload (rank 0 only, on the host's cores).
 """
 from __future__ import annotations
 
@@ -70,6 +72,9 @@ KERNEL_SOURCES = ["equivariant_graph_attention_b200/csrc/attention.cu",
                   "equivariant_graph_attention_b200/csrc/plan.cu",
                   "equivariant_graph_attention_b200/csrc/egat_device.cuh",
                   "equivariant_graph_attention_b200/csrc/egat_async.cuh"]
+#: library kernels per decomposed step and rank: three row gathers (own h, q, k),
+#: the source coupling, two send-buffer gathers, the plan (2) and the attention
+DECOMP_LAUNCHES = 9
 #: oracle worker processes at most (each holds its own copy of a few hundred MB)
 MAX_ORACLE_WORKERS = 32
 
@@ -325,8 +330,8 @@ def run_reference(args, wl: synth.Workload):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "atoms/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * secs / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(wl, edges, args.gpus, args.decompose),
+        "scaling": "strong" if args.decompose else "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(wl, edges, args.gpus, args.decompose),
         "cpu_baseline": {"value": value, "unit": "atoms/s", "cores": workers,
                          "kind": "oracle",
                          "sample": f"{args.ref_targets} random target atoms per worker and step "
@@ -614,6 +619,40 @@ def run_decomposed(args, wl: synth.Workload):
     clk = clocks.stop()
     ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
     t_step = max_over_ranks(ms, dev)
+
+    # end to end: every step copies this rank's rows of h, q, k (pinned host
+    # memory, prepared once) and the replicated positions in, runs the
+    # decomposed forward and copies this rank's output rows out
+    own = plan.owned
+    host = {nm: torch.from_numpy(np.ascontiguousarray(data[nm][own])).to(dtype=fs.st).pin_memory()
+            for nm in ("h", "q", "k")}
+    host["pos"] = torch.from_numpy(np.ascontiguousarray(data["pos"])).pin_memory()
+    devb = {nm: torch.empty(t.shape, dtype=t.dtype, device=dev) for nm, t in host.items()}
+    out_host = torch.empty((plan.n_owned, wl.D, wl.C), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        for nm, t in host.items():
+            devb[nm].copy_(t, non_blocking=True)
+        o = halo.forward_rank(plan, fs.shape, devb["h"], devb["pos"], devb["q"], devb["k"], fs.w1,
+                              fs.w2, own_rows=True)
+        out_host.copy_(o, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ea.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    eb.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(ea.elapsed_time(eb) / args.e2e_steps, dev)
+    ref_out = halo.forward_rank(plan, fs.shape, fs.h, fs.pos, fs.q, fs.k, fs.w1, fs.w2)
+    torch.cuda.synchronize(dev)
+    e2e_ok = bool(torch.equal(out_host.to(dev), ref_out))
     edges = int(cnt.sum())
     row_bytes = wl.D * wl.C * storage_bytes(wl) + wl.H * wl.dk * storage_bytes(wl)
     halo_max = max_over_ranks(plan.halo.size, dev)
@@ -628,6 +667,13 @@ def run_decomposed(args, wl: synth.Workload):
             "dtype": wl.dtype, "data": "synthetic",
             "config": config_of(wl, edges, ws, decompose=True),
             "edges_per_s": edges / (t_step / 1000.0),
+            "e2e": {"value": wl.n / (e2e_ms / 1000.0), "unit": "atoms/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                    "what": "each rank: its rows of h, q, k and the positions in, its output rows "
+                            "out, every step", "matches_device_result": e2e_ok},
+            "gpu_launches": DECOMP_LAUNCHES * args.steps,
+            "roofline": None,
+            "roofline_note": "per-kernel rooflines are reported by the single-system line",
             "decomposition": {"owned_per_rank": int(plan.n_owned), "halo_atoms_max": int(halo_max),
                               "exchange_bytes_max": int(halo_max) * row_bytes,
                               "step": "couple own atoms, exchange h' and k halo rows (NCCL "
@@ -664,10 +710,17 @@ def main():
                     help="steps 3+4 kernel: tensor-core tiles when the shape allows (auto), or "
                          "the per-target kernel")
     ap.add_argument("--decompose", action="store_true",
-                    help="split one system across the ranks by space (halo exchange)")
+                    help="split one system across the ranks by space (halo exchange); the "
+                         "default when more than one rank runs")
+    ap.add_argument("--replicas", action="store_true",
+                    help="with more than one rank: independent systems, one per rank")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.decompose and args.replicas:
+        ap.error("--decompose and --replicas exclude each other")
+    ws0, _, _ = dist_env()
+    args.decompose = args.decompose or (ws0 > 1 and not args.replicas)
     wl = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, wl)

@@ -147,6 +147,114 @@ __global__ void __launch_bounds__(kPlanThreads) build_plan_kernel(const __grid_c
   }
 }
 
+// The same plan for large n, at a cost per tile independent of n: one CTA per
+// tile keeps a hash set of the tile's neighbour indices in shared memory
+// (open addressing, 2 * cap slots, so it never fills), collects the distinct
+// indices as they are inserted, sorts them by a block-wide bitonic sort, and
+// sets each (target, neighbour) membership bit at the position a binary
+// search of the sorted union gives.  Union, padding and mask are bit for bit
+// those of build_plan_kernel.
+__global__ void __launch_bounds__(kPlanThreads) build_plan_hash_kernel(const __grid_constant__ PlanParams p) {
+  extern __shared__ int hsm[];
+  const PlanView& pv = p.plan;
+  const int cap = pv.cap;                         // >= kTileM * K, power of two
+  const int words = cap / 32;
+  const int hs = 2 * cap;                         // hash slots
+  int* table = hsm;                               // [hs], -1 = empty
+  int* srt = hsm + hs;                            // [cap] distinct indices, then sorted
+  uint32_t* mask = reinterpret_cast<uint32_t*>(srt + cap);   // [kTileM][words]
+  __shared__ int tgt[kTileM], rowcnt[kTileM];
+  __shared__ int s_unique;
+  const int tile = blockIdx.x;
+  if (threadIdx.x < kTileM) {
+    const long long slot = (long long)tile * kTileM + threadIdx.x;
+    int t = -1;
+    if (slot < p.n) t = p.order ? p.order[slot] : int(slot);
+    if ((unsigned)t >= (unsigned)p.n) t = -1;
+    int c = 0;
+    if (t >= 0) {
+      c = p.cnt ? p.cnt[t] : p.K;
+      c = c < 0 ? 0 : (c > p.K ? p.K : c);
+    }
+    tgt[threadIdx.x] = t;
+    rowcnt[threadIdx.x] = c;
+  }
+  if (threadIdx.x == 0) s_unique = 0;
+  for (int i = threadIdx.x; i < hs; i += blockDim.x) table[i] = -1;
+  for (int i = threadIdx.x; i < kTileM * words; i += blockDim.x) mask[i] = 0u;
+  __syncthreads();
+  auto for_each_entry = [&](auto&& f) {
+    for (int r = 0; r < kTileM; ++r) {
+      const int c = rowcnt[r];
+      const int32_t* row = p.nbr + (long long)(tgt[r] < 0 ? 0 : tgt[r]) * p.K;
+      for (int e = threadIdx.x; e < c; e += blockDim.x) f(r, row[e]);
+    }
+  };
+  // 1. distinct indices (at most kTileM * K <= cap of them; the table has
+  //    twice that many slots, so every probe sequence ends within hs steps)
+  for_each_entry([&](int, int j) {
+    if ((unsigned)j >= (unsigned)p.n) return;
+    unsigned slot = (unsigned(j) * 2654435761u) & unsigned(hs - 1);
+    for (int probe = 0; probe < hs; ++probe) {
+      const int prev = atomicCAS(&table[slot], -1, j);
+      if (prev == -1) {
+        srt[atomicAdd(&s_unique, 1)] = j;
+        return;
+      }
+      if (prev == j) return;
+      slot = (slot + 1) & unsigned(hs - 1);
+    }
+  });
+  __syncthreads();
+  const int U = s_unique;
+  // 2. bitonic sort of srt[0, P2), the tail filled with INT_MAX
+  int P2 = 1;
+  while (P2 < U) P2 <<= 1;
+  for (int i = U + threadIdx.x; i < P2; i += blockDim.x) srt[i] = 0x7fffffff;
+  __syncthreads();
+  for (int k = 2; k <= P2; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < P2; i += blockDim.x) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const int a = srt[i], b = srt[ixj];
+          const bool up = (i & k) == 0;
+          if ((a > b) == up) {
+            srt[i] = b;
+            srt[ixj] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // 3. the union (ascending), padded as build_plan_kernel pads it
+  int* uni = pv.uni + (long long)tile * cap;
+  for (int i = threadIdx.x; i < U; i += blockDim.x) uni[i] = srt[i];
+  const int upad = U > 0 ? (U + kPlanPad - 1) / kPlanPad * kPlanPad : kPlanPad;
+  const int filler = U > 0 ? srt[0] : 0;
+  for (int e = U + threadIdx.x; e < upad; e += blockDim.x) uni[e] = filler;
+  if (threadIdx.x == 0) pv.ulen[tile] = U;
+  // 4. membership bits at each neighbour's union position
+  for_each_entry([&](int r, int j) {
+    if ((unsigned)j >= (unsigned)p.n) return;
+    int lo = 0, hi = U;                           // first position with srt >= j
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (srt[mid] < j) lo = mid + 1;
+      else hi = mid;
+    }
+    atomicOr(&mask[r * words + (lo >> 5)], 1u << (lo & 31));
+  });
+  __syncthreads();
+  uint32_t* gmask = pv.mask + (long long)tile * words * kTileM;
+  const int uw = upad / 32;
+  for (int i = threadIdx.x; i < kTileM * uw; i += blockDim.x) {
+    const int w = i / kTileM, r = i % kTileM;
+    gmask[i] = mask[r * words + w];
+  }
+}
+
 // One thread per target slot (tile * kTileM + r): the slot's atom, |r|^l and
 // the Wigner-D matrices of its alignment rotation (identity for an empty slot
 // or an atom at the origin), built in registers, into the tile record.
@@ -185,9 +293,18 @@ tile_records_kernel(const int32_t* __restrict__ order, const float* __restrict__
 
 }  // namespace
 
+// Systems up to this many atoms use the bitmap builder (its two bitmaps take
+// n / 4 bytes of shared memory and O(n / 32) work per tile); larger ones the
+// hash builder, whose shared memory and work per tile depend only on K.
+constexpr int kBitmapPlanAtoms = 1 << 17;
+
 size_t plan_smem_bytes(int n, int K) {
-  const size_t nw = (size_t(n) + 31) / 32;
-  return 2 * nw * sizeof(uint32_t) + size_t(kTileM) * (plan_capacity(K) / 32) * sizeof(uint32_t);
+  const size_t mask = size_t(kTileM) * (plan_capacity(K) / 32) * sizeof(uint32_t);
+  if (n <= kBitmapPlanAtoms) {
+    const size_t nw = (size_t(n) + 31) / 32;
+    return 2 * nw * sizeof(uint32_t) + mask;
+  }
+  return size_t(3) * plan_capacity(K) * sizeof(int) + mask;   // table, sorted union, mask
 }
 
 int plan_capacity(int K) {
@@ -234,12 +351,13 @@ int launch_build_plan(int n, int K, int lmax, const int32_t* d_nbr, const int32_
   p.n = n;
   p.K = K;
   const size_t shmem = plan_smem_bytes(n, K);
-  if (shmem > 48 * 1024) {
-    if (cudaFuncSetAttribute(build_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(shmem)) != cudaSuccess)
-      return EGAT_ERR_CUDA;
-  }
-  build_plan_kernel<<<p.plan.tiles, kPlanThreads, shmem, st>>>(p);
+  if (shmem > kPlanSmemLimit) return EGAT_ERR_UNSUPPORTED;
+  auto kern = n <= kBitmapPlanAtoms ? build_plan_kernel : build_plan_hash_kernel;
+  if (shmem > 48 * 1024 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(shmem)) !=
+          cudaSuccess)
+    return EGAT_ERR_CUDA;
+  kern<<<p.plan.tiles, kPlanThreads, shmem, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return EGAT_ERR_CUDA;
   const int tiles = p.plan.tiles;
   const int blocks = (tiles * kTileM + kRecThreads - 1) / kRecThreads;

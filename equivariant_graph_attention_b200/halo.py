@@ -174,15 +174,20 @@ def _local_shape(shape: "egat.Shape", n: int) -> "egat.Shape":
 
 
 def couple_rank(plan: HaloPlan, shape: "egat.Shape", h: torch.Tensor, pos: torch.Tensor,
-                q: torch.Tensor, k: torch.Tensor, w1: torch.Tensor) -> RankState:
+                q: torch.Tensor, k: torch.Tensor, w1: torch.Tensor,
+                own_rows: bool = False) -> RankState:
     """Step 2 for this rank's own atoms (egat_eaas_couple on its rows of h); each
     rank reads only its own rows of h, q and k and the positions of its local
-    atoms."""
+    atoms.  h, q, k are the whole system's arrays, or (own_rows) already this
+    rank's rows in plan.owned order; pos is always the whole system's."""
     a = plan.on(h.device)
     own_i32, loc = a["own"], a["loc"]
-    h_own = egat.egat_gather_rows(h.contiguous(), own_i32)
-    q_own = egat.egat_gather_rows(q.contiguous(), own_i32)
-    k_own = egat.egat_gather_rows(k.contiguous(), own_i32)
+    if own_rows:
+        h_own, q_own, k_own = h.contiguous(), q.contiguous(), k.contiguous()
+    else:
+        h_own = egat.egat_gather_rows(h.contiguous(), own_i32)
+        q_own = egat.egat_gather_rows(q.contiguous(), own_i32)
+        k_own = egat.egat_gather_rows(k.contiguous(), own_i32)
     pos_loc = pos.index_select(0, loc).contiguous()
     hp_own = egat.egat_eaas_couple(_local_shape(shape, plan.n_owned), h_own,
                                    pos_loc[:plan.n_owned].contiguous(), w1)
@@ -225,12 +230,13 @@ def attend_rank(plan: HaloPlan, shape: "egat.Shape", st: RankState, hp_halo: tor
 
 def forward_rank(plan: HaloPlan, shape: "egat.Shape", h: torch.Tensor, pos: torch.Tensor,
                  q: torch.Tensor, k: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor,
-                 group=None) -> torch.Tensor:
+                 group=None, own_rows: bool = False) -> torch.Tensor:
     """^h of this rank's atoms (float32 [n_owned, D, C], in plan.owned order) for the
-    global inputs h, pos, q, k of the `shape` system: step 2 on the owned atoms,
-    one exchange of the boundary atoms' h' and k rows (NCCL all-to-all in
-    `group`), then steps 3+4 over the local arrays."""
-    st = couple_rank(plan, shape, h, pos, q, k, w1)
+    inputs h, pos, q, k of the `shape` system (whole arrays, or with own_rows
+    this rank's rows of h, q, k): step 2 on the owned atoms, one exchange of the
+    boundary atoms' h' and k rows (NCCL all-to-all in `group`), then steps 3+4
+    over the local arrays."""
+    st = couple_rank(plan, shape, h, pos, q, k, w1, own_rows=own_rows)
     hp_halo = exchange(plan, st.hp_own, group)
     k_halo = exchange(plan, st.k_own, group)
     return attend_rank(plan, shape, st, hp_halo, k_halo, w2)
