@@ -36,8 +36,9 @@
 //    2^-9: P V_h runs as two mma.sync per component of the head's 8 channels
 //    (the lo products one component pair behind the hi ones, off the same
 //    accumulator's dependency chain), the value fragments by ldmatrix.trans
-//    from the staged rows; z is the mma of the same hi and lo fragments with
-//    an all-ones fragment, the row sums of exactly the weights of P V.
+//    from the staged rows; z is the float32 row sum of the weights, on the
+//    FMA pipe (the pairs equal the weights to about 2^-17), which keeps the
+//    busier tensor pipe for the products.
 // The accumulator fragment of a lane holds, for targets g and g+8 and
 // channels 2t, 2t+1 of its head, every component d — exactly what the
 // per-channel EAAS epilogue needs, so the target coupling runs from registers.
@@ -95,9 +96,12 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
 // both rounded to nearest even: hi + lo equals x to about 2^-17 relative
 __device__ __forceinline__ void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  const float2 hf = __bfloat1622float2(h);
-  __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
   hi = *reinterpret_cast<uint32_t*>(&h);
+  // (a, b) - float(hi) as one packed f32x2 FMA
+  const f32x2 r = f2_fma(bf16x2_to_f2(hi), f2_pack(-1.f, -1.f), f2_pack(a, b));
+  float ra, rb;
+  f2_unpack(r, ra, rb);
+  __nv_bfloat162 l = __floats2bfloat162_rn(ra, rb);
   lo = *reinterpret_cast<uint32_t*>(&l);
 }
 
@@ -295,10 +299,10 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
     for (int d = 0; d < D; ++d)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[d][e] = 0.f;
-    // zacc: P times an all-ones B fragment, i.e. the row sums of exactly the
-    // bf16 weights the P V product uses (zacc[0] row g, zacc[2] row g+8)
-    float zacc[4] = {0.f, 0.f, 0.f, 0.f};
-    constexpr uint32_t kOnes = 0x3f803f80u;   // bf16x2 (1, 1)
+    // z0, z1: this lane's float32 sums of the weights of rows g and g+8 (its
+    // columns of the stage); the quad's four lanes are added at the tile's end.
+    // The hi + lo pairs of P V equal these weights to about 2^-17.
+    float z0 = 0.f, z1 = 0.f;
     // reference maxima (log2 domain): a finite sentinel, so that a masked
     // entry (-inf) gives exp2(-inf) = 0 without a select
     constexpr float kNone = -1e30f;
@@ -380,10 +384,8 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
         const bool r0 = mx0 > mref0 + kLazy, r1 = mx1 > mref1 + kLazy;
         const float sc0 = r0 ? fast_exp2(mref0 - mx0) : 1.f;
         const float sc1 = r1 ? fast_exp2(mref1 - mx1) : 1.f;
-        zacc[0] *= sc0;
-        zacc[1] *= sc0;
-        zacc[2] *= sc1;
-        zacc[3] *= sc1;
+        z0 *= sc0;
+        z1 *= sc1;
 #pragma unroll
         for (int d = 0; d < D; ++d) {
           acc[d][0] *= sc0;
@@ -403,10 +405,19 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
 #pragma unroll
       for (int j = 0; j < KS; ++j) {
         float pr[8];
+        {
+          // exponents v qs - mref as packed f32x2 FMAs (pairs of one row)
+          const f32x2 q2 = f2_pack(qs, qs);
+          const f32x2 r0 = f2_pack(-mref0, -mref0), r1 = f2_pack(-mref1, -mref1);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) pr[e] = fast_exp2(fmaf(v[j][e], qs, -mref0));
-#pragma unroll
-        for (int e = 4; e < 8; ++e) pr[e] = fast_exp2(fmaf(v[j][e], qs, -mref1));
+          for (int e = 0; e < 8; e += 2) {
+            const f32x2 x = f2_fma(f2_pack(v[j][e], v[j][e + 1]), q2, e < 4 ? r0 : r1);
+            float x0, x1;
+            f2_unpack(x, x0, x1);
+            pr[e] = fast_exp2(x0);
+            pr[e + 1] = fast_exp2(x1);
+          }
+        }
         // the weights as a bf16 pair hi + lo (hi = bf16(p), lo = bf16(p - hi)):
         // 16 significant bits, so P V and the normaliser carry the float32
         // weights to about 2^-17 instead of bf16's 2^-9
@@ -415,7 +426,8 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
         split_bf16(pr[4], pr[5], pa[1], pl[1]);   // row g+8, k 2t
         split_bf16(pr[2], pr[3], pa[2], pl[2]);   // row g,   k 2t+8
         split_bf16(pr[6], pr[7], pa[3], pl[3]);   // row g+8, k 2t+8
-        mma_bf16(zacc, pa, kOnes, kOnes);
+        z0 += (pr[0] + pr[1]) + (pr[2] + pr[3]);
+        z1 += (pr[4] + pr[5]) + (pr[6] + pr[7]);
 
         // ---- O += P V (one n8 tile per component of this head's 8 channels).
         // The lo products run one component pair behind the hi products, so
@@ -446,12 +458,10 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
             mma_bf16(acc[D - 3], pl, vprev[0], vprev[1]);
             mma_bf16(acc[D - 2], pl, vprev[2], vprev[3]);
           }
-          mma_bf16(zacc, pl, kOnes, kOnes);
           mma_bf16(acc[D - 1], pl, vf[0], vf[1]);
         } else {
           mma_bf16(acc[D - 2], pl, vprev[0], vprev[1]);
           mma_bf16(acc[D - 1], pl, vprev[2], vprev[3]);
-          mma_bf16(zacc, pl, kOnes, kOnes);
         }
       }   // k-steps of the stage
     }
@@ -481,8 +491,12 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
     const int* tgt = reinterpret_cast<const int*>(rec) + kRecTgt;
     const float* rp = rec + kRecRp;             // [16][L+1]
     const float* Dq = rec + rec_off_D(L);       // [16][WS]
-    const float inv0 = zacc[0] > 0.f ? 1.f / zacc[0] : 0.f;
-    const float inv1 = zacc[2] > 0.f ? 1.f / zacc[2] : 0.f;
+    z0 += __shfl_xor_sync(0xffffffffu, z0, 1);
+    z0 += __shfl_xor_sync(0xffffffffu, z0, 2);
+    z1 += __shfl_xor_sync(0xffffffffu, z1, 1);
+    z1 += __shfl_xor_sync(0xffffffffu, z1, 2);
+    const float inv0 = z0 > 0.f ? 1.f / z0 : 0.f;
+    const float inv1 = z1 > 0.f ? 1.f / z1 : 0.f;
     const int ch = h * 8 + 2 * t;
     if constexpr (FUSED && L >= 3) {
       // register budget: m of both rows goes through this warp's slice of the

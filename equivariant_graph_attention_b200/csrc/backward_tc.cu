@@ -642,18 +642,19 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_source_tc_kernel(const __gri
       float dp[4] = {0.f, 0.f, 0.f, 0.f};
       const uint32_t db = smem_u32(fb + (8 * nt + (lane & 7)) * FSTR + h * 32 + ((lane >> 3) & 1) * 16);
       float dp2[4] = {0.f, 0.f, 0.f, 0.f};   // odd components: a second, independent chain
-      // dm rows are float32; the tf32 product takes their leading 19 bits
+      // dm rows are float32: rounded to tf32 here (the tensor core would
+      // truncate them, which doubles the error dk inherits from dalpha)
 #pragma unroll
       for (int d = 0; d + 1 < D; d += 2) {
         uint32_t r[4];
         ldsm_x4(r, db + (d + (lane >> 4)) * (kBC * 4));
-        mma_tf32(dp, ha[d], r[0], r[1]);
-        mma_tf32(dp2, ha[d + 1], r[2], r[3]);
+        mma_tf32(dp, ha[d], to_tf32(__uint_as_float(r[0])), to_tf32(__uint_as_float(r[1])));
+        mma_tf32(dp2, ha[d + 1], to_tf32(__uint_as_float(r[2])), to_tf32(__uint_as_float(r[3])));
       }
       if constexpr (D % 2) {
         uint32_t r[2];
         ldsm_x2(r, db + (D - 1) * (kBC * 4));
-        mma_tf32(dp, ha[D - 1], r[0], r[1]);
+        mma_tf32(dp, ha[D - 1], to_tf32(__uint_as_float(r[0])), to_tf32(__uint_as_float(r[1])));
       }
 #pragma unroll
       for (int e = 0; e < 4; ++e) dp[e] += dp2[e];

@@ -357,7 +357,7 @@ eaas_tile_kernel(const __grid_constant__ EaasParams p) {
     bulk_g2s(smem_u32(recs + b * REC), p.rec + (long long)tl * REC, REC * 4, bar);
   };
   // thread 0: the feature rows of a tile's targets into rows[b] (empty slots
-  // are not copied)
+  // are not copied); used for the first tile, warp 0 issues the later ones
   auto issue_rows = [&](const float* rec, int b) {
     const int* tg = reinterpret_cast<const int*>(rec) + kRecTgt;
     int valid = 0;
@@ -382,14 +382,24 @@ eaas_tile_kernel(const __grid_constant__ EaasParams p) {
     const int rb = j % 3, wb = j & 1;
     bounded_wait(smem_u32(recbar + rb), uint32_t(j / 3) & 1u, kWaitPolls, abort_flag);
     bounded_wait(smem_u32(rowbar + wb), uint32_t(j >> 1) & 1u, kWaitPolls, abort_flag);
-    if (tid == 0 && tile + grid < tiles) {
-      // the next tile's rows (its record arrived a tile ago) and the record
-      // after it; both buffers were last read by tile j - 1, before the
-      // barrier that ended it
+    if (wfirst == 0 && tile + grid < tiles) {
+      // warp 0: the next tile's rows (its record arrived a tile ago), one
+      // bulk copy per lane after lane 0 has announced their bytes, and the
+      // record after it; both buffers were last read by tile j - 1, before
+      // the barrier that ended it
       const int nb = (j + 1) % 3;
       bounded_wait(smem_u32(recbar + nb), uint32_t((j + 1) / 3) & 1u, kWaitPolls, abort_flag);
-      issue_rows(recs + nb * REC, (j + 1) & 1);
-      if (tile + 2 * grid < tiles) issue_rec(tile + 2 * grid, (j + 2) % 3);
+      const int* tg = reinterpret_cast<const int*>(recs + nb * REC) + kRecTgt;
+      const int wbn = (j + 1) & 1;
+      const uint32_t bar = smem_u32(rowbar + wbn);
+      const bool mine = lane < kTileM && (unsigned)tg[lane < kTileM ? lane : 0] < (unsigned)p.n;
+      const int valid = __popc(__ballot_sync(0xffffffffu, mine));
+      if (lane == 0) mbar_arrive_expect_tx(bar, uint32_t(valid) * ROWB);
+      __syncwarp();
+      if (mine)
+        bulk_g2s(smem_u32(rows + (size_t(wbn) * kTileM + lane) * ROWB), xb + (size_t)tg[lane] * ROWB,
+                 ROWB, bar);
+      if (lane == 0 && tile + 2 * grid < tiles) issue_rec(tile + 2 * grid, (j + 2) % 3);
     }
     const float* rec = recs + rb * REC;
     for (int w = wfirst; w < kTileM; w += kHalfWarps) {   // two slots per warp

@@ -21,10 +21,10 @@
 // shared memory (Ivanic–Ruedenberg recursion, __syncwarp only); each lane
 // owns CPL consecutive channels, holds them of the neighbour row and of the
 // running sum in registers and reads the rotation entries and its channels'
-// SO(2) weights from shared memory.  At lmax 3 with 128 channels the warp
-// walks the neighbour list twice, 64 channels a pass (the registers of four
-// channels of degree 3 would spill).  Messages are summed on chip; nothing
-// per edge reaches memory.
+// SO(2) weights from shared memory.  With 128 channels at lmax >= 2 the warp
+// walks the neighbour list twice, 64 channels a pass, so that two CTAs fit an
+// SM without spilling (four channels a lane would need more than 128
+// registers).  Messages are summed on chip; nothing per edge reaches memory.
 #include "egat_device.cuh"
 #include "egat_host.h"
 
@@ -56,8 +56,12 @@ constexpr int escn_block(int L, int m) {
   return off;
 }
 
-template <int L, typename T, int CPL, int PASSES>
-__global__ void __launch_bounds__(kEscnWarps * 32) escn_conv_kernel(const __grid_constant__ EscnParams p) {
+// M is the truncation order M_max (compile time, so the SO(2) layer is
+// straight-line code); two CTAs per SM below lmax 3, one at lmax 3 (whose
+// 16-component rows need more than 128 registers).
+template <int L, int M, typename T, int CPL, int PASSES>
+__global__ void __launch_bounds__(kEscnWarps * 32, L >= 3 ? 1 : 2)
+escn_conv_kernel(const __grid_constant__ EscnParams p) {
   constexpr int D = (L + 1) * (L + 1);
   constexpr int WS = wig_size(L);
   extern __shared__ float smem[];
@@ -136,8 +140,8 @@ __global__ void __launch_bounds__(kEscnWarps * 32) escn_conv_kernel(const __grid
           for (int k = 0; k < CPL; ++k)
             y[lo * lo + lo][k] = fmaf(w0[k], x[li * li + li][k], y[lo * lo + lo][k]);
 #pragma unroll
-          for (int m = 1; m <= L; ++m) {
-            if (m > lo || m > li || m > p.mmax) continue;
+          for (int m = 1; m <= M; ++m) {
+            if (m > lo || m > li) continue;         // compile-time after unrolling
             const int nb = L + 1 - m;
             const int r = (lo - m) * nb + (li - m);
             const float* w1 = sw + (escn_block(L, m) + r) * C + c0;
@@ -179,8 +183,8 @@ __global__ void __launch_bounds__(kEscnWarps * 32) escn_conv_kernel(const __grid
   }
 }
 
-template <int L, typename T>
-int launch_escn_t(const EscnParams& p, cudaStream_t st) {
+template <int L, int M, typename T>
+int launch_escn_m(const EscnParams& p, cudaStream_t st) {
   const size_t shmem = (size_t(p.nw) * p.C + size_t(kEscnWarps) * wig_size(L)) * sizeof(float);
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -188,15 +192,26 @@ int launch_escn_t(const EscnParams& p, cudaStream_t st) {
   const long long want = (p.n + kEscnWarps - 1) / kEscnWarps;
   const int grid = int(std::max<long long>(1, std::min<long long>(want, (long long)sms * 8)));
   switch (p.C) {
-    case 32: escn_conv_kernel<L, T, 1, 1><<<grid, kEscnWarps * 32, shmem, st>>>(p); break;
-    case 64: escn_conv_kernel<L, T, 2, 1><<<grid, kEscnWarps * 32, shmem, st>>>(p); break;
+    case 32: escn_conv_kernel<L, M, T, 1, 1><<<grid, kEscnWarps * 32, shmem, st>>>(p); break;
+    case 64: escn_conv_kernel<L, M, T, 2, 1><<<grid, kEscnWarps * 32, shmem, st>>>(p); break;
     case 128:
-      if constexpr (L >= 3) escn_conv_kernel<L, T, 2, 2><<<grid, kEscnWarps * 32, shmem, st>>>(p);
-      else escn_conv_kernel<L, T, 4, 1><<<grid, kEscnWarps * 32, shmem, st>>>(p);
+      if constexpr (L >= 2) escn_conv_kernel<L, M, T, 2, 2><<<grid, kEscnWarps * 32, shmem, st>>>(p);
+      else escn_conv_kernel<L, M, T, 4, 1><<<grid, kEscnWarps * 32, shmem, st>>>(p);
       break;
-    default: escn_conv_kernel<L, T, 1, 1><<<grid, kEscnWarps * 32, shmem, st>>>(p); break;   // C = 16
+    default: escn_conv_kernel<L, M, T, 1, 1><<<grid, kEscnWarps * 32, shmem, st>>>(p); break;   // C = 16
   }
   return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
+}
+
+template <int L, typename T>
+int launch_escn_t(const EscnParams& p, cudaStream_t st) {
+  switch (p.mmax) {
+    case 0: return launch_escn_m<L, 0, T>(p, st);
+    case 1: return launch_escn_m<L, 1, T>(p, st);
+    case 2: if constexpr (L >= 2) return launch_escn_m<L, 2, T>(p, st); else return EGAT_ERR_ARG;
+    case 3: if constexpr (L >= 3) return launch_escn_m<L, 3, T>(p, st); else return EGAT_ERR_ARG;
+    default: return EGAT_ERR_ARG;
+  }
 }
 
 }  // namespace

@@ -16,10 +16,10 @@
 //    carries the float32 weights to about 2^-17, and h is exactly bf16;
 //  * tiles of 64 atoms: one thread issues one 256-byte bulk copy per atom
 //    (the degree-0 slice of its row; cp.async.bulk, no multicast) into a
-//    double-buffered, row-padded A tile completing an mbarrier, so the next
-//    tile lands while this one is multiplied; every wait is bounded;
-//  * 8 warps, each 64 atoms x 32 output columns: per 16-channel k-step four
-//    A fragments (ldmatrix.x4), two B fragment pairs for hi and lo, and 32
+//    ring of four row-padded A tiles, each completing its own mbarrier, so
+//    three tiles are in flight while one is multiplied; every wait is bounded;
+//  * 16 warps, each 32 atoms x 32 output columns: per 16-channel k-step two
+//    A fragments (ldmatrix.x4), two B fragment pairs for hi and lo, and 16
 //    mma.sync m16n8k16 (bf16 in, float32 accumulation);
 //  * the accumulators are rounded once to the storage type and stored.
 // It moves n * (C + 2 * H*dk) * 2 bytes (degree-0 slices in, q and k out):
@@ -41,14 +41,15 @@ constexpr int kPC = 128;          // channels (the contraction length)
 constexpr int kPN = 256;          // H * dk outputs per matrix
 constexpr int kPM = 64;           // atoms per tile
 constexpr int kPRow = kPC * 2 + 16;   // padded bf16 row (272 B): ldmatrix phases hit distinct banks
-constexpr int kPWarps = 8;
+constexpr int kPWarps = 16;
+constexpr int kPBuf = 4;              // A tiles in the ring
 
 struct ProjSmem {
   static constexpr size_t whi = 0;                                   // [kPN][kPRow]
   static constexpr size_t wlo = whi + size_t(kPN) * kPRow;           // [kPN][kPRow]
-  static constexpr size_t a = wlo + size_t(kPN) * kPRow;             // [2][kPM][kPRow]
-  static constexpr size_t bars = a + size_t(2) * kPM * kPRow;        // [2] mbarriers + abort flag
-  static constexpr size_t total = bars + 2 * 8 + 16;
+  static constexpr size_t a = wlo + size_t(kPN) * kPRow;             // [kPBuf][kPM][kPRow]
+  static constexpr size_t bars = a + size_t(kPBuf) * kPM * kPRow;    // [kPBuf] mbarriers + abort flag
+  static constexpr size_t total = bars + kPBuf * 8 + 16;
   static_assert(kPRow % 16 == 0 && a % 16 == 0 && bars % 8 == 0, "bulk-copy alignment");
 };
 
@@ -81,7 +82,7 @@ __global__ void __launch_bounds__(kPWarps * 32, 1) qk_projection_tc_kernel(const
   unsigned char* wlo = smem + ProjSmem::wlo;
   unsigned char* abuf = smem + ProjSmem::a;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + ProjSmem::bars);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + kPBuf);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int sel = blockIdx.x & 1;            // 0: q from wq, 1: k from wk
@@ -90,20 +91,32 @@ __global__ void __launch_bounds__(kPWarps * 32, 1) qk_projection_tc_kernel(const
   if (slot >= p.tiles) return;               // whole CTA
 
   if (tid == 0) {
-    mbar_init(smem_u32(bar), 1);
-    mbar_init(smem_u32(bar + 1), 1);
+    for (int b = 0; b < kPBuf; ++b) mbar_init(smem_u32(bar + b), 1);
     mbar_fence_init();
     *abort_flag = 0;
   }
-  // weights: float32 [c][col] -> transposed bf16 hi/lo [col][c]
-  const float* w = p.w[sel];
-  for (int e = tid; e < kPC * kPN; e += blockDim.x) {
-    const int c = e / kPN, col = e % kPN;
-    const float x = __ldg(w + e);
-    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
-    *reinterpret_cast<__nv_bfloat16*>(whi + size_t(col) * kPRow + c * 2) = hi;
-    *reinterpret_cast<__nv_bfloat16*>(wlo + size_t(col) * kPRow + c * 2) = lo;
+  // weights: float32 [c][col] -> transposed bf16 hi/lo [col][c].  Each
+  // thread has all its 16-byte loads in flight before it converts (one L2
+  // round trip for the whole matrix, not one per element).
+  const float4* w4 = reinterpret_cast<const float4*>(p.w[sel]);
+  constexpr int kW4 = kPC * kPN / 4;                 // float4 groups of the matrix
+  constexpr int kPer = kW4 / (kPWarps * 32);         // per thread
+  static_assert(kW4 % (kPWarps * 32) == 0, "weight groups per thread");
+  float4 wv[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) wv[i] = __ldg(w4 + tid + i * kPWarps * 32);
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = 4 * (tid + i * kPWarps * 32);
+    const int c = e / kPN, col0 = e % kPN;
+    const float x[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(x[u]);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(x[u] - __bfloat162float(hi));
+      *reinterpret_cast<__nv_bfloat16*>(whi + size_t(col0 + u) * kPRow + c * 2) = hi;
+      *reinterpret_cast<__nv_bfloat16*>(wlo + size_t(col0 + u) * kPRow + c * 2) = lo;
+    }
   }
   __syncthreads();
 
@@ -119,21 +132,25 @@ __global__ void __launch_bounds__(kPWarps * 32, 1) qk_projection_tc_kernel(const
       bulk_g2s(smem_u32(abuf + (size_t(b) * kPM + r) * kPRow), hb + (long long)(a0 + r) * row_bytes,
                kPC * 2, bb);
   };
-  if (tid == 0) issue(slot, 0);
+  // the ring starts with the CTA's first kPBuf - 1 tiles in flight
+  if (tid == 0)
+    for (int q = 0; q < kPBuf - 1 && slot + q * stride < p.tiles; ++q) issue(slot + q * stride, q);
 
   const int g = lane >> 2, t = lane & 3;
-  const int n0 = warp * 32;                  // this warp's first output column
+  const int m0 = (warp & 1) * 32;            // this warp's first atom of the tile
+  const int n0 = (warp >> 1) * 32;           // this warp's first output column
   __nv_bfloat16* out = p.out[sel];
   int j = 0;
   for (int tile = slot; tile < p.tiles; tile += stride, ++j) {
-    const int b = j & 1;
-    bounded_wait(smem_u32(bar + b), uint32_t(j >> 1) & 1u, kWaitPolls, abort_flag);
-    // the next tile into the other buffer (last read by tile j - 1, which
-    // ended with a barrier)
-    if (tid == 0 && tile + stride < p.tiles) issue(tile + stride, b ^ 1);
-    float acc[4][4][4];
+    const int b = j % kPBuf;
+    bounded_wait(smem_u32(bar + b), uint32_t(j / kPBuf) & 1u, kWaitPolls, abort_flag);
+    // the tile kPBuf - 1 ahead into the buffer tile j - 1 used (it ended
+    // with a barrier)
+    const int ahead = tile + (kPBuf - 1) * stride;
+    if (tid == 0 && ahead < p.tiles) issue(ahead, (j + kPBuf - 1) % kPBuf);
+    float acc[2][4][4];
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
       for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -144,10 +161,10 @@ __global__ void __launch_bounds__(kPWarps * 32, 1) qk_projection_tc_kernel(const
     const int bhalf = (lane >> 3) & 1;
 #pragma unroll 2
     for (int kk = 0; kk < kPC / 16; ++kk) {
-      uint32_t af[4][4];
+      uint32_t af[2][4];
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt)
-        pj_ldsm_x4(af[mt], a_base + (mt * 16 + arow) * kPRow + kk * 32 + (lane >> 4) * 16);
+      for (int mt = 0; mt < 2; ++mt)
+        pj_ldsm_x4(af[mt], a_base + (m0 + mt * 16 + arow) * kPRow + kk * 32 + (lane >> 4) * 16);
 #pragma unroll
       for (int np = 0; np < 2; ++np) {       // pairs of n8 tiles
         uint32_t bh[4], bl[4];
@@ -155,7 +172,7 @@ __global__ void __launch_bounds__(kPWarps * 32, 1) qk_projection_tc_kernel(const
         pj_ldsm_x4(bh, smem_u32(whi) + off);
         pj_ldsm_x4(bl, smem_u32(wlo) + off);
 #pragma unroll
-        for (int mt = 0; mt < 4; ++mt) {
+        for (int mt = 0; mt < 2; ++mt) {
           pj_mma(acc[mt][2 * np], af[mt], bh[0], bh[1]);
           pj_mma(acc[mt][2 * np + 1], af[mt], bh[2], bh[3]);
           pj_mma(acc[mt][2 * np], af[mt], bl[0], bl[1]);
@@ -164,9 +181,9 @@ __global__ void __launch_bounds__(kPWarps * 32, 1) qk_projection_tc_kernel(const
       }
     }
     // rows g and g+8 of each m tile, columns 2t, 2t+1 of each n tile
-    const int a0 = tile * kPM;
+    const int a0 = tile * kPM + m0;
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         const int atom = a0 + mt * 16 + g + 8 * half;
@@ -178,15 +195,19 @@ __global__ void __launch_bounds__(kPWarps * 32, 1) qk_projection_tc_kernel(const
                 __floats2bfloat162_rn(acc[mt][nt][2 * half], acc[mt][nt][2 * half + 1]);
         }
       }
-    __syncthreads();   // buffer b is refilled by the next iteration's issue
+    __syncthreads();   // buffer b is refilled by a later iteration's issue
   }
   if (*abort_flag && tid == 0) {
-    // a wait gave up: give each buffer's last phase a short, bounded chance to
-    // complete before the CTA's shared memory is released
+    // a wait gave up: give each buffer's last issued phase a short, bounded
+    // chance to complete before the CTA's shared memory is released (tile
+    // sequence numbers up to j + kPBuf - 2 may have been issued)
     volatile int none = 0;
-    for (int b = 0; b < 2; ++b) {
-      const int last = j - 1 - ((j - 1 - b) & 1);
-      if (last >= 0) bounded_wait(smem_u32(bar + b), uint32_t(last >> 1) & 1u, kDrainPolls, &none);
+    for (int b = 0; b < kPBuf; ++b) {
+      int last = -1;
+      for (int q = 0; q < j + kPBuf - 1; ++q)
+        if (q % kPBuf == b && slot + q * stride < p.tiles) last = q;
+      if (last >= 0)
+        bounded_wait(smem_u32(bar + b), uint32_t(last / kPBuf) & 1u, kDrainPolls, &none);
     }
   }
 }
@@ -245,7 +266,9 @@ int launch_qk_projection(const egat_shape& s, const void* d_h, const float* d_wq
                          void* d_q, void* d_k, cudaStream_t st) {
   const long long row_elems = (long long)(s.lmax + 1) * (s.lmax + 1) * s.C;
   const int HD = s.H * s.dk;
-  if (projection_tc_supported(s)) {
+  // the tensor-core kernel reads the weights as 16-byte vectors
+  const bool w16 = ((reinterpret_cast<uintptr_t>(d_wq) | reinterpret_cast<uintptr_t>(d_wk)) & 15u) == 0;
+  if (projection_tc_supported(s) && w16) {
     ProjParams p;
     p.h = static_cast<const __nv_bfloat16*>(d_h);
     p.w[0] = d_wq;

@@ -128,3 +128,23 @@ def test_projected_forward(name):
     assert e_block < TOL[wl.dtype]
     if wl.dtype == "f32":
         assert channel_rel_error(out, ref, wl.lmax, FLOOR["f32"]) < TOL["f32"]
+
+
+def test_projection_misaligned_weights_take_the_plain_path():
+    """Weights that are only 4-byte aligned (an offset view) give the same q and
+    k through the plain kernel, within the bf16 bar of the oracle."""
+    wl, d, w = _data("uniform4096_l2_bf16")
+    egat = _egat()
+    hd = torch.from_numpy(np.ascontiguousarray(d["h"])).to("cuda", dtype=torch.bfloat16)
+    buf = torch.zeros(2 * wl.C * wl.H * wl.dk + 2, dtype=torch.float32, device="cuda")
+    n = wl.C * wl.H * wl.dk
+    wq = buf[1:1 + n].view(wl.C, wl.H * wl.dk)
+    wk = buf[1 + n:1 + 2 * n].view(wl.C, wl.H * wl.dk)
+    wq.copy_(torch.from_numpy(w["wq"]))
+    wk.copy_(torch.from_numpy(w["wk"]))
+    assert wq.data_ptr() % 16 != 0
+    q, k = egat.egat_qk_projection(shape_of(wl), hd, wq, wk)
+    rq, rk = invariant_projection(d["h"], w["wq"], w["wk"], wl.H, wl.dk)
+    f = FLOOR["bf16"]
+    assert vec_rel_error(q.float().cpu().numpy(), rq, f) < TOL["bf16"]
+    assert vec_rel_error(k.float().cpu().numpy(), rk, f) < TOL["bf16"]
