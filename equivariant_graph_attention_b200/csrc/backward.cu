@@ -1020,6 +1020,7 @@ int launch_backward(const egat_shape& s, const void* d_h, const float* d_pos, co
     switch (s.lmax) {
       case 1: return launch_backward_tiled<1>(s, w, d_h, d_pos, d_q, d_k, d_nbr, d_cnt, d_order, d_w1, d_w2, d_g, d_dh, d_dq, d_dk, d_dpos, st);
       case 2: return launch_backward_tiled<2>(s, w, d_h, d_pos, d_q, d_k, d_nbr, d_cnt, d_order, d_w1, d_w2, d_g, d_dh, d_dq, d_dk, d_dpos, st);
+      case 3: return launch_backward_tiled<3>(s, w, d_h, d_pos, d_q, d_k, d_nbr, d_cnt, d_order, d_w1, d_w2, d_g, d_dh, d_dq, d_dk, d_dpos, st);
       default: return EGAT_ERR_UNSUPPORTED;
     }
   }

@@ -28,6 +28,10 @@
 //    lists hold them (in-lists, bitmap union as for the forward plan); per 8
 //    union targets and head, S^T = K Q^T, dalpha^T = H' dm^T,
 //    dk += ds^T Q and dh' += alpha^T dm.
+// At lmax 3 (16 components: 8 KB float rows) a stage holds 8 union rows, and
+// the source pass sweeps its union twice, once for dk (with h' as the
+// register-resident operand) and once for dh' (with its accumulator), since
+// the two would not fit one thread's registers together.
 // The tile's own operand (dm of the 16 targets, or h' of the 16 sources) sits
 // in registers as tf32 fragments for the whole tile; the union rows stream
 // through shared memory in stages, one bulk copy (cp.async.bulk, no
@@ -63,8 +67,9 @@ struct BtcShape {
   static constexpr int D = (L + 1) * (L + 1);
   static constexpr int FROW = D * kBC * 4;      // float32 row of h' or dm
   static constexpr int FSTR = FROW + 16;        // staged (4 words mod 32: distinct banks)
-  static constexpr int RS = 16;                 // union rows per stage (two n8 tiles)
-  static constexpr int STAGES = L >= 2 ? 2 : 4;
+  // union rows per stage: two n8 tiles, one at lmax 3 (8 KB float rows)
+  static constexpr int RS = L >= 3 ? 8 : 16;
+  static constexpr int STAGES = L >= 3 ? 3 : (L >= 2 ? 2 : 4);
 };
 
 // Shared memory (byte offsets, 16-byte aligned): staged float rows (FR),
@@ -141,6 +146,23 @@ __device__ __forceinline__ uint32_t to_tf32(float x) {
 // a bf16 in shared memory as the bit pattern of the equal float (exact in tf32)
 __device__ __forceinline__ uint32_t bf16_bits_f32(const unsigned char* p) {
   return uint32_t(*reinterpret_cast<const unsigned short*>(p)) << 16;
+}
+
+// The head's 16 key (or query) columns of a stage's staged rows as mma B
+// fragments: {b0, b1} of n8 tile 0 in f[0], f[1] and, with 16 rows, of n8
+// tile 1 in f[2], f[3].
+template <int RS>
+__device__ __forceinline__ void stage_frags(uint32_t (&f)[4], const unsigned char* kb, int lane, int h) {
+  if constexpr (RS == 16) {
+    ldsm_x4(f, smem_u32(kb + ((lane & 7) + 8 * (lane >> 4)) * kKStr + h * 32 + ((lane >> 3) & 1) * 16));
+  } else {
+    static_assert(RS == 8, "stages of one or two n8 tiles");
+    uint32_t r[2];
+    ldsm_x2(r, smem_u32(kb + (lane & 7) * kKStr + h * 32 + ((lane >> 3) & 1) * 16));
+    f[0] = r[0];
+    f[1] = r[1];
+    f[2] = f[3] = 0u;
+  }
 }
 
 // The accumulator fragment of an n8 tile (columns 2t, 2t+1 of rows g, g+8)
@@ -320,7 +342,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_stats_tc_kernel(const __grid
     const int sh = (st * RS) & 31;
     const uint32_t m0 = mw[g] >> sh, m1 = mw[g + 8] >> sh;
     uint32_t kf[4];
-    ldsm_x4(kf, smem_u32(kb + ((lane & 7) + 8 * (lane >> 4)) * kKStr + h * 32 + ((lane >> 3) & 1) * 16));
+    stage_frags<RS>(kf, kb, lane, h);
     float v[RS / 8][4];   // masked raw logits: rows g (0, 1), g+8 (2, 3); columns 2t, 2t+1
     bool over = false;
 #pragma unroll
@@ -482,7 +504,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_target_tc_kernel(const __gri
     const uint32_t m0 = mw[g] >> sh, m1 = mw[g + 8] >> sh;
     // key fragments of both n8 tiles of the stage
     uint32_t kf[4];
-    ldsm_x4(kf, smem_u32(kb + ((lane & 7) + 8 * (lane >> 4)) * kKStr + h * 32 + ((lane >> 3) & 1) * 16));
+    stage_frags<RS>(kf, kb, lane, h);
 #pragma unroll
     for (int nt = 0; nt < RS / 8; ++nt) {
       float s[4] = {0.f, 0.f, 0.f, 0.f};
@@ -558,8 +580,13 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_target_tc_kernel(const __gri
 }
 
 // ---------------------------------------------------------------- source pass
-template <int L>
+// PART selects what one sweep accumulates: kSrcBoth dk and dh' (lmax <= 2);
+// at lmax 3 the register-resident h' operand (dk) and dh' accumulator would
+// not fit together, so the union is swept twice, kSrcDk then kSrcDh.
+enum SourcePart { kSrcBoth, kSrcDk, kSrcDh };
+template <int L, int PART>
 __global__ void __launch_bounds__(kBThreads, 1) bwd_source_tc_kernel(const __grid_constant__ BtcParams p) {
+  constexpr bool DK = PART != kSrcDh, DH = PART != kSrcDk;
   using Sh = BtcShape<L>;
   using Sm = BtcSmem<L, true>;
   constexpr int D = Sh::D, RS = Sh::RS, STAGES = Sh::STAGES, FSTR = Sh::FSTR;
@@ -585,8 +612,8 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_source_tc_kernel(const __gri
     ka[2] = sa0 >= 0 ? __ldg(k32 + (size_t)sa0 * (kBH * 8) + h * 8 + 4 + t) : 0u;
     ka[3] = sa1 >= 0 ? __ldg(k32 + (size_t)sa1 * (kBH * 8) + h * 8 + 4 + t) : 0u;
   }
-  uint32_t ha[D][4];
-  {
+  uint32_t ha[DK ? D : 1][4];
+  if constexpr (DK) {
     const uint32_t* h32 = reinterpret_cast<const uint32_t*>(p.hp);
 #pragma unroll
     for (int d = 0; d < D; ++d) {
@@ -599,13 +626,13 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_source_tc_kernel(const __gri
   }
   const float qs = p.qscale;
 
-  float dka[2][4], dha[D][4];
+  float dka[2][4], dha[DH ? D : 1][4];
 #pragma unroll
   for (int a = 0; a < 2; ++a)
 #pragma unroll
     for (int e = 0; e < 4; ++e) dka[a][e] = 0.f;
 #pragma unroll
-  for (int d = 0; d < D; ++d)
+  for (int d = 0; d < (DH ? D : 1); ++d)
 #pragma unroll
     for (int e = 0; e < 4; ++e) dha[d][e] = 0.f;
 
@@ -624,7 +651,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_source_tc_kernel(const __gri
     const int sh = (st * RS) & 31;
     const uint32_t m0 = mw[g] >> sh, m1 = mw[g + 8] >> sh;
     uint32_t qf[4];
-    ldsm_x4(qf, smem_u32(qb + ((lane & 7) + 8 * (lane >> 4)) * kKStr + h * 32 + ((lane >> 3) & 1) * 16));
+    stage_frags<RS>(qf, qb, lane, h);
 #pragma unroll
     for (int nt = 0; nt < RS / 8; ++nt) {
       // rows: sources g, g+8; columns: union targets ca = 8 nt + 2t, cb = ca + 1
@@ -639,6 +666,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_source_tc_kernel(const __gri
       P[1] = (w0 & 2u) ? fast_exp2(fmaf(s[1], qs, -lsb)) : 0.f;
       P[2] = (w1 & 1u) ? fast_exp2(fmaf(s[2], qs, -lsa)) : 0.f;
       P[3] = (w1 & 2u) ? fast_exp2(fmaf(s[3], qs, -lsb)) : 0.f;
+      if constexpr (DK) {
       float dp[4] = {0.f, 0.f, 0.f, 0.f};
       const uint32_t db = smem_u32(fb + (8 * nt + (lane & 7)) * FSTR + h * 32 + ((lane >> 3) & 1) * 16);
       float dp2[4] = {0.f, 0.f, 0.f, 0.f};   // odd components: a second, independent chain
@@ -663,15 +691,18 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_source_tc_kernel(const __gri
       ds[1] = P[1] * (dp[1] - dlb);
       ds[2] = P[2] * (dp[2] - dla);
       ds[3] = P[3] * (dp[3] - dlb);
-      uint32_t dsa[4], pa[4], pl[4];
+      uint32_t dsa[4];
       acc_as_a(dsa, ds);
-      acc_as_a_split(pa, pl, P);
       // dk += ds^T Q (B rows: union targets ca, cb)
       const unsigned char* q0 = qb + (8 * nt + 2 * t) * kKStr + h * 32;
 #pragma unroll
       for (int nd = 0; nd < 2; ++nd)
         mma_tf32(dka[nd], dsa, bf16_bits_f32(q0 + (8 * nd + g) * 2),
                  bf16_bits_f32(q0 + kKStr + (8 * nd + g) * 2));
+      }
+      if constexpr (DH) {
+      uint32_t pa[4], pl[4];
+      acc_as_a_split(pa, pl, P);
       // dh' += alpha^T dm (B rows: dm of ca, cb; columns: the head's channels)
       // in three tf32 products of the hi/lo splits of both operands,
       // alpha_hi dm_hi + alpha_lo dm_hi + alpha_hi dm_lo: float32-level
@@ -702,6 +733,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_source_tc_kernel(const __gri
         mma_tf32(dha[d], pa, la0, la1);
         if (e != d) mma_tf32(dha[e], pa, lb0, lb1);
       }
+      }
     }
   }
   S.drain(tid);
@@ -711,15 +743,19 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_source_tc_kernel(const __gri
   for (int half = 0; half < 2; ++half) {
     const int sa = half ? sa1 : sa0;
     if (sa < 0) continue;
-    float* o = p.dk + (size_t)sa * (kBH * 16) + h * 16 + 2 * t;
+    if constexpr (DK) {
+      float* o = p.dk + (size_t)sa * (kBH * 16) + h * 16 + 2 * t;
 #pragma unroll
-    for (int nd = 0; nd < 2; ++nd)
-      *reinterpret_cast<float2*>(o + 8 * nd) =
-          make_float2(dka[nd][2 * half] * ks, dka[nd][2 * half + 1] * ks);
-    float* od = p.dhp + (size_t)sa * D * kBC + h * 8 + 2 * t;
+      for (int nd = 0; nd < 2; ++nd)
+        *reinterpret_cast<float2*>(o + 8 * nd) =
+            make_float2(dka[nd][2 * half] * ks, dka[nd][2 * half + 1] * ks);
+    }
+    if constexpr (DH) {
+      float* od = p.dhp + (size_t)sa * D * kBC + h * 8 + 2 * t;
 #pragma unroll
-    for (int d = 0; d < D; ++d)
-      *reinterpret_cast<float2*>(od + d * kBC) = make_float2(dha[d][2 * half], dha[d][2 * half + 1]);
+      for (int d = 0; d < D; ++d)
+        *reinterpret_cast<float2*>(od + d * kBC) = make_float2(dha[d][2 * half], dha[d][2 * half + 1]);
+    }
   }
 }
 
@@ -845,19 +881,31 @@ int launch_pass_t(const BtcParams& p, PassKind kind, cudaStream_t st) {
   const size_t shm = kind == kSourcePass ? BtcSmem<L, true>::total
                      : lean ? BtcSmem<L, false, false>::total : BtcSmem<L, false>::total;
   if (shm > 227 * 1024) return EGAT_ERR_UNSUPPORTED;
-  auto kern = kind == kSourcePass ? bwd_source_tc_kernel<L>
-              : kind == kTargetPass ? bwd_target_tc_kernel<L>
+  auto run = [&](void (*kern)(BtcParams)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(shm)) != cudaSuccess)
+      return EGAT_ERR_CUDA;
+    kern<<<p.tiles, kBThreads, shm, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
+  };
+  if (kind == kSourcePass) {
+    if constexpr (L >= 3) {
+      // two sweeps of the source union: dk, then dh'
+      const int e = run(bwd_source_tc_kernel<L, kSrcDk>);
+      return e == EGAT_OK ? run(bwd_source_tc_kernel<L, kSrcDh>) : e;
+    } else {
+      return run(bwd_source_tc_kernel<L, kSrcBoth>);
+    }
+  }
+  auto kern = kind == kTargetPass ? bwd_target_tc_kernel<L>
               : lean ? bwd_stats_tc_kernel<L, false> : bwd_stats_tc_kernel<L, true>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(shm)) != cudaSuccess)
-    return EGAT_ERR_CUDA;
-  kern<<<p.tiles, kBThreads, shm, st>>>(p);
-  return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
+  return run(kern);
 }
 
 int launch_pass(int lmax, const BtcParams& p, PassKind kind, cudaStream_t st) {
   switch (lmax) {
     case 1: return launch_pass_t<1>(p, kind, st);
     case 2: return launch_pass_t<2>(p, kind, st);
+    case 3: return launch_pass_t<3>(p, kind, st);
     default: return EGAT_ERR_UNSUPPORTED;
   }
 }
@@ -867,9 +915,11 @@ size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 }  // namespace
 
 bool bwd_tc_supported(const egat_shape& s) {
-  return s.lmax <= 2 && tc_attention_supported(s) &&
-         (long long)s.n * s.K + (long long)kPlanPad * ((s.n + kTileM - 1) / kTileM) < (1LL << 31) &&
-         BtcSmem<2, true>::total <= 227 * 1024;
+  static_assert(BtcSmem<1, true>::total <= 227 * 1024 && BtcSmem<2, true>::total <= 227 * 1024 &&
+                    BtcSmem<3, true>::total <= 227 * 1024 && BtcSmem<3, false>::total <= 227 * 1024,
+                "stages fit the shared memory");
+  return s.lmax <= 3 && tc_attention_supported(s) &&
+         (long long)s.n * s.K + (long long)kPlanPad * ((s.n + kTileM - 1) / kTileM) < (1LL << 31);
 }
 
 size_t bwd_tc_ws_bytes(const egat_shape& s) {

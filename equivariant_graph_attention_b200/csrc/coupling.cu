@@ -422,7 +422,7 @@ eaas_tile_kernel(const __grid_constant__ EaasParams p) {
         }
         T* yr = y + (size_t)at * D * C + c0;
         const float* swc = sw + c0;
-        eaas_multi<L, CPL>(xv, rec + rec_off_D(L) + w * WS, rpow, p.tab,
+        eaas_multi<L, CPL, (CPL >= 4)>(xv, rec + rec_off_D(L) + w * WS, rpow, p.tab,
                            [&](int q, int k) { return swc[q * C + k]; },
                            [&](int d, const float (&v)[CPL]) { ChanVec<T, CPL>::store(yr + d * C, v); });
       }
@@ -531,6 +531,8 @@ int launch_eaas_source_f32out(const egat_shape& s, const void* d_x, const float*
                         : launch_eaas_t<1, float, false, Tf32Out>(s, d_x, d_pos, nullptr, n, d_w, y, st);
       case 2: return bf ? launch_eaas_t<2, __nv_bfloat16, false, Tf32Out>(s, d_x, d_pos, nullptr, n, d_w, y, st)
                         : launch_eaas_t<2, float, false, Tf32Out>(s, d_x, d_pos, nullptr, n, d_w, y, st);
+      case 3: return bf ? launch_eaas_t<3, __nv_bfloat16, false, Tf32Out>(s, d_x, d_pos, nullptr, n, d_w, y, st)
+                        : launch_eaas_t<3, float, false, Tf32Out>(s, d_x, d_pos, nullptr, n, d_w, y, st);
       default: return EGAT_ERR_UNSUPPORTED;
     }
   }

@@ -574,15 +574,112 @@ __device__ __forceinline__ void coupling_grad_channel(float (&g)[(L + 1) * (L + 
   }
 }
 
+// eaas_multi on channel pairs: the same operations in the same order per
+// channel, each pair of channels in one packed f32x2 FMA (or MUL), so the
+// results equal the scalar form bit for bit with about half the FP
+// instructions.
+template <int L, int NP, typename WFn, typename OutFn>
+__device__ __forceinline__ void eaas_multi_packed(float (&x)[2 * NP][(L + 1) * (L + 1)],
+                                                  const float* __restrict__ Dsm,
+                                                  const float (&rpow)[L + 1], const EaasTable& tab,
+                                                  WFn wgt, OutFn out) {
+  constexpr int D = (L + 1) * (L + 1);
+  f32x2 xv[NP][D], t[NP][D];
+#pragma unroll
+  for (int j = 0; j < NP; ++j)
+#pragma unroll
+    for (int d = 0; d < D; ++d) {
+      xv[j][d] = f2_pack(x[2 * j][d], x[2 * j + 1][d]);
+      t[j][d] = 0ull;   // (+0, +0)
+    }
+  static_for<1, L + 1>([&](auto lc) {
+    constexpr int l = decltype(lc)::value;
+    constexpr int w = 2 * l + 1;
+    const float* Dl = Dsm + wig_off(l);
+    f32x2 tmp[NP][w];
+#pragma unroll
+    for (int a = 0; a < w; ++a) {
+#pragma unroll
+      for (int j = 0; j < NP; ++j) tmp[j][a] = 0ull;
+#pragma unroll
+      for (int b = 0; b < w; ++b) {
+        const float dv = Dl[b * w + a];
+        const f32x2 d2 = f2_pack(dv, dv);
+#pragma unroll
+        for (int j = 0; j < NP; ++j) tmp[j][a] = f2_fma(d2, xv[j][l * l + b], tmp[j][a]);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < NP; ++j)
+#pragma unroll
+      for (int a = 0; a < w; ++a) xv[j][l * l + a] = tmp[j][a];
+  });
+  static_for<0, num_paths(L)>([&](auto pc) {
+    constexpr int p = decltype(pc)::value;
+    constexpr int li = path_info(L, p, 0);
+    constexpr int lf = path_info(L, p, 1);
+    constexpr int lo = path_info(L, p, 2);
+    constexpr bool even = ((li + lf + lo) % 2) == 0;
+    f32x2 wp[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) wp[j] = f2_pack(wgt(p, 2 * j) * rpow[lf], wgt(p, 2 * j + 1) * rpow[lf]);
+#pragma unroll
+    for (int mo = -lo; mo <= lo; ++mo) {
+      const int src = even ? mo : -mo;
+      const bool live = (iabs(mo) <= li) && (even || mo != 0);
+      if (live) {
+        const float f = tab.f[p][mo + lo];
+        const f32x2 f2 = f2_pack(f, f);
+#pragma unroll
+        for (int j = 0; j < NP; ++j)
+          t[j][lo * lo + lo + mo] = f2_fma(f2_mul(wp[j], f2), xv[j][li * li + li + src], t[j][lo * lo + lo + mo]);
+      }
+    }
+  });
+  {
+    float y[2 * NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) f2_unpack(t[j][0], y[2 * j], y[2 * j + 1]);
+    out(0, y);
+  }
+  static_for<1, L + 1>([&](auto lc) {
+    constexpr int l = decltype(lc)::value;
+    constexpr int w = 2 * l + 1;
+    const float* Dl = Dsm + wig_off(l);
+#pragma unroll
+    for (int a = 0; a < w; ++a) {
+      f32x2 y2[NP];
+#pragma unroll
+      for (int j = 0; j < NP; ++j) y2[j] = 0ull;
+#pragma unroll
+      for (int b = 0; b < w; ++b) {
+        const float dv = Dl[a * w + b];
+        const f32x2 d2 = f2_pack(dv, dv);
+#pragma unroll
+        for (int j = 0; j < NP; ++j) y2[j] = f2_fma(d2, t[j][l * l + b], y2[j]);
+      }
+      float y[2 * NP];
+#pragma unroll
+      for (int j = 0; j < NP; ++j) f2_unpack(y2[j], y[2 * j], y[2 * j + 1]);
+      out(l * l + a, y);
+    }
+  });
+}
+
 // The same operator on NCH channels at once (channels of one atom share the
 // Wigner-D matrices): each matrix entry is read once and applied to every
 // channel.  x[k][d] is overwritten; wgt(p, k) returns w[p] of channel k;
-// out(d, y) receives component d of all NCH channels.
-template <int L, int NCH, typename WFn, typename OutFn>
+// out(d, y) receives component d of all NCH channels.  PACKED (an even NCH)
+// runs the channels as packed pairs, for callers with registers to spare.
+template <int L, int NCH, bool PACKED = false, typename WFn, typename OutFn>
 __device__ __forceinline__ void eaas_multi(float (&x)[NCH][(L + 1) * (L + 1)],
                                            const float* __restrict__ Dsm,
                                            const float (&rpow)[L + 1], const EaasTable& tab,
                                            WFn wgt, OutFn out) {
+  if constexpr (PACKED) {
+    static_assert(NCH % 2 == 0, "channel pairs");
+    eaas_multi_packed<L, NCH / 2>(x, Dsm, rpow, tab, wgt, out);
+  } else {
   constexpr int D = (L + 1) * (L + 1);
   float t[NCH][D];
 #pragma unroll
@@ -655,6 +752,7 @@ __device__ __forceinline__ void eaas_multi(float (&x)[NCH][(L + 1) * (L + 1)],
       out(l * l + a, y);
     }
   });
+  }
 }
 
 }  // namespace egat

@@ -12,7 +12,7 @@
 // atoms inside their bucket by index (deterministic order) -> one warp per atom
 // sweeps the 125 surrounding cells, writes the row and counts (padded), or
 // counts, scans and writes (CSR).  Rows with more than K neighbours keep the K
-// nearest, selected on the (d^2, j) key.  No kernel waits on another
+// nearest, ranked on the (d^2, j) key.  No kernel waits on another
 // block; every loop is bounded.
 #include "egat_device.cuh"
 #include "egat_host.h"
@@ -296,21 +296,18 @@ __device__ __forceinline__ void for_each_neighbour_rounds(const Search& s, int4 
       }
       const int obeg = __shfl_sync(0xffffffffu, beg, own);
       const int oexc = __shfl_sync(0xffffffffu, exc, own);
-      const int ocx = __shfl_sync(0xffffffffu, cx, own);
-      const int ocy = __shfl_sync(0xffffffffu, cy, own);
-      const int ocz = __shfl_sync(0xffffffffu, cz, own);
       bool hit = false;
       int j = -1;
       long long d2 = 0;
       if (k < total) {
-        const int slot = obeg + (k - oexc);
-        const int4 cc = s.scell[slot];
-        const int4 q = s.spos[slot];
-        if (cc.x == ocx && cc.y == ocy && cc.z == ocz) {
-          j = q.w;
-          d2 = sq_dist(q, p);
-          hit = (j != p.w) && (d2 <= s.rc2);
-        }
+        // A bucket may also hold atoms of cells outside the 5 x 5 x 5 block
+        // (their low coordinate bits collide).  Such an atom is at least
+        // 2 cq + 1 > r_c away along one axis, so the cutoff test rejects it
+        // and the cell itself needs no check.
+        const int4 q = s.spos[obeg + (k - oexc)];
+        j = q.w;
+        d2 = sq_dist(q, p);
+        hit = (j != p.w) && (d2 <= s.rc2);
       }
       f(hit, j, d2);
     }
@@ -385,71 +382,68 @@ fill_padded(Search s, int n, int K, int32_t* __restrict__ nbr, int32_t* __restri
 // Rows with more than K neighbours: one CTA of kFixWarps warps per listed atom
 // (persistent CTAs; the loop is bounded by the device-side count).  The warps
 // split the 125-cell sweep by rounds and gather every neighbour's key
-// (d^2 << shift | j) into shared memory; a block-wide bitonic sort orders them
-// and the row is rewritten with the K smallest keys, nearest first (ties to
-// the smaller index).  Rows with more keys than fit use bisection for the K-th
-// key and one warp rewrites them in sweep order.
+// (d^2 << shift | j) into shared memory.  The keys are distinct (j is), so a
+// key's rank among them is its place in the row: the key of rank r < K writes
+// row[r], and the row lists the K nearest, nearest first, ties to the smaller
+// index.  A row with more keys than the buffer holds first finds its K-th
+// smallest key by bisection (one warp), then gathers the K keys up to it and
+// ranks those.
 constexpr int kFixWarps = 4;
 
 __global__ void __launch_bounds__(kFixWarps * 32)
 fix_truncated(Search s, int K, int32_t* __restrict__ nbr, const int* __restrict__ trunc,
               int* __restrict__ overflow) {
   __shared__ unsigned long long keys[kSelectCap];
-  __shared__ int s_total;
+  __shared__ unsigned long long s_thresh;
+  __shared__ int s_total, s_kept;
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
   const int ntr = trunc[0];
   const unsigned long long jmask = (1ull << s.key_shift) - 1ull;
+  // every warp sweeps its rounds of cells; f(hit, key) with full-warp ballots
+  auto gather = [&](const int4& p, const int4& c, int* counter, auto keep) {
+    for_each_neighbour_rounds(s, p, c, wib, kFixWarps, [&](bool hit, int j, long long d2) {
+      const unsigned long long key = (((unsigned long long)d2) << s.key_shift) | (unsigned long long)j;
+      const bool take = hit && keep(key);
+      const unsigned m = __ballot_sync(0xffffffffu, take);
+      int base = 0;
+      if (lane == 0 && m) base = atomicAdd(counter, __popc(m));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      const int pos = base + __popc(m & ((1u << lane) - 1u));
+      if (take && pos < kSelectCap) keys[pos] = key;
+    });
+  };
   for (int t = blockIdx.x; t < ntr; t += gridDim.x) {
     const int w = trunc[1 + t];
     const int4 p = s.spos[w];
     const int4 c = s.scell[w];
     int32_t* row = nbr + (long long)p.w * K;
-    if (threadIdx.x == 0) s_total = 0;
+    if (threadIdx.x == 0) {
+      s_total = 0;
+      s_kept = 0;
+    }
     __syncthreads();
-    for_each_neighbour_rounds(s, p, c, wib, kFixWarps, [&](bool hit, int j, long long d2) {
-      const unsigned m = __ballot_sync(0xffffffffu, hit);
-      int base = 0;
-      if (lane == 0 && m) base = atomicAdd(&s_total, __popc(m));
-      base = __shfl_sync(0xffffffffu, base, 0);
-      const int pos = base + __popc(m & ((1u << lane) - 1u));
-      if (hit && pos < kSelectCap)
-        keys[pos] = (((unsigned long long)d2) << s.key_shift) | (unsigned long long)j;
-    });
+    gather(p, c, &s_total, [](unsigned long long) { return true; });
     __syncthreads();
     const int total = s_total;
-    if (total <= kSelectCap) {
-      int size = 32;
-      while (size < total) size <<= 1;
-      for (int q = total + threadIdx.x; q < size; q += blockDim.x) keys[q] = ~0ull;
-      __syncthreads();
-      for (int k = 2; k <= size; k <<= 1) {
-        for (int jj = k >> 1; jj > 0; jj >>= 1) {
-          for (int i = threadIdx.x; i < size; i += blockDim.x) {
-            const int ixj = i ^ jj;
-            if (ixj > i) {
-              const unsigned long long a = keys[i], b = keys[ixj];
-              if ((a > b) == ((i & k) == 0)) {
-                keys[i] = b;
-                keys[ixj] = a;
-              }
-            }
-          }
-          __syncthreads();
-        }
+    int T = total;
+    if (total > kSelectCap) {
+      if (wib == 0) {
+        const unsigned long long th = kth_key(s, p, c, K);
+        if (lane == 0) s_thresh = th;
       }
-      for (int q = threadIdx.x; q < K; q += blockDim.x) row[q] = int32_t(keys[q] & jmask);
-    } else if (wib == 0) {
-      const unsigned long long thresh = kth_key(s, p, c, K);
-      int written = 0;
-      for_each_neighbour(s, p, c, [&](bool hit, int j, long long d2) {
-        const bool keep = hit && ((((unsigned long long)d2) << s.key_shift) |
-                                  (unsigned long long)j) <= thresh;
-        const unsigned m = __ballot_sync(0xffffffffu, keep);
-        const int pos = written + __popc(m & ((1u << lane) - 1u));
-        if (keep && pos < K) row[pos] = j;
-        written += __popc(m);
-      });
+      __syncthreads();
+      const unsigned long long th = s_thresh;
+      gather(p, c, &s_kept, [th](unsigned long long key) { return key <= th; });
+      __syncthreads();
+      T = s_kept < kSelectCap ? s_kept : kSelectCap;   // K of them
+    }
+    for (int i = threadIdx.x; i < T; i += blockDim.x) {
+      const unsigned long long key = keys[i];
+      int rank = 0;
+#pragma unroll 4
+      for (int k = 0; k < T; ++k) rank += keys[k] < key ? 1 : 0;
+      if (rank < K) row[rank] = int32_t(key & jmask);
     }
     if (threadIdx.x == 0) atomicAdd(overflow, total - K);
     __syncthreads();

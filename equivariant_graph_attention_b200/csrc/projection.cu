@@ -95,28 +95,34 @@ __global__ void __launch_bounds__(kPWarps * 32, 1) qk_projection_tc_kernel(const
     mbar_fence_init();
     *abort_flag = 0;
   }
-  // weights: float32 [c][col] -> transposed bf16 hi/lo [col][c].  Each
-  // thread has all its 16-byte loads in flight before it converts (one L2
-  // round trip for the whole matrix, not one per element).
-  const float4* w4 = reinterpret_cast<const float4*>(p.w[sel]);
-  constexpr int kW4 = kPC * kPN / 4;                 // float4 groups of the matrix
-  constexpr int kPer = kW4 / (kPWarps * 32);         // per thread
-  static_assert(kW4 % (kPWarps * 32) == 0, "weight groups per thread");
-  float4 wv[kPer];
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) wv[i] = __ldg(w4 + tid + i * kPWarps * 32);
+  // weights: float32 [c][col] -> transposed bf16 hi/lo [col][c], stored as
+  // (c, c + 1) pairs.  A warp converts a block of 8 columns x 4 channel
+  // pairs: lane -> column 8 cb + (lane & 7), pair 4 pb + (lane >> 3).  With
+  // the 68-word row pitch its 32 four-byte stores hit 32 distinct banks, and
+  // each load instruction reads 8 full 32-byte sectors.  Every load of the
+  // thread is issued before the first conversion.
+  const float* w = p.w[sel];
+  constexpr int kPer = (kPC / 2) * kPN / (kPWarps * 32);   // pairs per thread
+  static_assert((kPC / 2) * kPN % (kPWarps * 32 * 32) == 0 && kPN % 8 == 0, "weight blocks");
+  float x0[kPer], x1[kPer];
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
-    const int e = 4 * (tid + i * kPWarps * 32);
-    const int c = e / kPN, col0 = e % kPN;
-    const float x[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
+    const int blk = i * kPWarps + warp;
+    const int col = (blk % (kPN / 8)) * 8 + (lane & 7);
+    const int c = 2 * ((blk / (kPN / 8)) * 4 + (lane >> 3));
+    x0[i] = __ldg(w + c * kPN + col);
+    x1[i] = __ldg(w + (c + 1) * kPN + col);
+  }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const __nv_bfloat16 hi = __float2bfloat16_rn(x[u]);
-      const __nv_bfloat16 lo = __float2bfloat16_rn(x[u] - __bfloat162float(hi));
-      *reinterpret_cast<__nv_bfloat16*>(whi + size_t(col0 + u) * kPRow + c * 2) = hi;
-      *reinterpret_cast<__nv_bfloat16*>(wlo + size_t(col0 + u) * kPRow + c * 2) = lo;
-    }
+  for (int i = 0; i < kPer; ++i) {
+    const int blk = i * kPWarps + warp;
+    const int col = (blk % (kPN / 8)) * 8 + (lane & 7);
+    const int c = 2 * ((blk / (kPN / 8)) * 4 + (lane >> 3));
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(x0[i], x1[i]);
+    const __nv_bfloat162 lo =
+        __floats2bfloat162_rn(x0[i] - __low2float(hi), x1[i] - __high2float(hi));
+    *reinterpret_cast<__nv_bfloat162*>(whi + size_t(col) * kPRow + c * 2) = hi;
+    *reinterpret_cast<__nv_bfloat162*>(wlo + size_t(col) * kPRow + c * 2) = lo;
   }
   __syncthreads();
 
@@ -266,9 +272,7 @@ int launch_qk_projection(const egat_shape& s, const void* d_h, const float* d_wq
                          void* d_q, void* d_k, cudaStream_t st) {
   const long long row_elems = (long long)(s.lmax + 1) * (s.lmax + 1) * s.C;
   const int HD = s.H * s.dk;
-  // the tensor-core kernel reads the weights as 16-byte vectors
-  const bool w16 = ((reinterpret_cast<uintptr_t>(d_wq) | reinterpret_cast<uintptr_t>(d_wk)) & 15u) == 0;
-  if (projection_tc_supported(s) && w16) {
+  if (projection_tc_supported(s)) {
     ProjParams p;
     p.h = static_cast<const __nv_bfloat16*>(d_h);
     p.w[0] = d_wq;

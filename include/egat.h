@@ -295,11 +295,12 @@ EGAT_API int egat_forward_noalloc(const egat_shape* s, const void* d_h, const fl
  *  d_order optional int32 [n] traversal order (a permutation, as
  *          egat_build_graph returns it; NULL = 0..n-1).  It only groups atoms
  *          into tiles: results do not depend on it up to rounding, speed does.
- * Shapes of the tensor-core forward path with lmax <= 2 (bf16, C = 128,
- * H = 16, dk = 16) run tiled passes: the forward kernel unfused (m and the
+ * Shapes of the tensor-core forward path (bf16, C = 128, H = 16, dk = 16,
+ * lmax <= 3) run tiled passes: the forward kernel unfused (m and the
  * log-sum-exp), a pass over tiles of 16 targets (dq) and one over tiles of 16
- * sources and the union of the targets that list them (dk, dL/dh'), with the
- * gradient products in tf32.  Other shapes gather per target and per source
+ * sources and the union of the targets that list them (dk, dL/dh'; at
+ * lmax 3 two sweeps of that union, one for each), with the gradient
+ * products in tf32.  Other shapes gather per target and per source
  * over sorted in-lists in float32.  Either way every gradient is a sum in a
  * fixed order: deterministic, no atomics on results.  Padded graphs only (CSR
  * returns EGAT_ERR_UNSUPPORTED), n * K below 2^31; d_ws at least
@@ -330,9 +331,8 @@ EGAT_API int egat_backward(const egat_shape* s, const void* d_h, const float* d_
  *  d_wq, d_wk float32 [C][H*dk]
  *  d_q, d_k   [n][H][dk] in s->dtype (bf16: round to nearest even)
  * bf16 storage with C = 128 and H*dk = 256 runs on tensor cores (the weights
- * as bf16 pairs hi + lo, float32 accumulation; weights 16-byte aligned, else
- * the plain path); other shapes (C <= 1024, H*dk <= 1024) accumulate in
- * float32 on CUDA cores.  n = 0 is a no-op.
+ * as bf16 pairs hi + lo, float32 accumulation); other shapes (C <= 1024,
+ * H*dk <= 1024) accumulate in float32 on CUDA cores.  n = 0 is a no-op.
  * Errors: EGAT_ERR_ARG (null or misaligned pointer, bad dtype),
  * EGAT_ERR_UNSUPPORTED, EGAT_ERR_CUDA; a bounded wait that gave up is
  * reported by egat_take_device_status.

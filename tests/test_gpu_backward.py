@@ -143,8 +143,9 @@ def test_backward_edge_cases(lmax):
 def test_tiled_backward_edge_cases(lmax, n):
     """The bf16 C = 128, H = 16, dk = 16 shapes on tiny systems: a single atom
     (empty unions), and 37 atoms (a ragged last tile) with an isolated atom,
-    an atom at the origin and one on the negative z axis.  ℓmax 1-2 run the
-    tiled passes; ℓmax 3 the shape of the 100,000-atom workload."""
+    an atom at the origin and one on the negative z axis.  All three run the
+    tiled passes; ℓmax 3 is the shape of the 100,000-atom workload (8-row
+    stages, the source union swept once for dL/dk and once for dL/dh')."""
     rng = np.random.default_rng(70 + 3 * lmax + n)
     pts = rng.uniform(-3.0, 3.0, (n, 3))
     pts[0] = 0.0
@@ -173,8 +174,8 @@ def test_tiled_backward_edge_cases(lmax, n):
 @pytest.mark.parametrize("name,count", [("uniform32768_K256_l2_bf16", 12),
                                         ("uniform100000_l3_bf16", 6)])
 def test_backward_full_size_sampled(name, count):
-    """The full-size bf16 workloads (32,768 atoms, K = 256, ℓmax 2 on the tiled
-    passes; 100,000 atoms, ℓmax 3): dL/dq, dL/dk, dL/dh and dL/dr of sampled
+    """The full-size bf16 workloads on the tiled passes (32,768 atoms, K = 256,
+    ℓmax 2; 100,000 atoms, K = 96, ℓmax 3): dL/dq, dL/dk, dL/dh and dL/dr of sampled
     atoms (random ones, the highest-degree ones, the last atom) against the
     oracle evaluated at those atoms."""
     from tests.test_gpu_parity import _full_degree

@@ -73,6 +73,9 @@ def test_graph_padded_bit_exact(name):
         assert cnt[i] == len(ref)
         assert np.array_equal(np.sort(nbr[i, :cnt[i]]), np.sort(ref)), i
         assert np.all(nbr[i, cnt[i]:] == -1)
+        if full[i] > wl.K:
+            # a truncated row is listed nearest first, ties to the smaller index
+            assert np.array_equal(nbr[i], ref), i
     assert int(g["overflow"].item()) == int(np.maximum(full - wl.K, 0).sum())
     order = g["order"].cpu().numpy()
     assert np.array_equal(np.sort(order), np.arange(wl.n))
@@ -115,6 +118,35 @@ def test_graph_full_size_sampled_rows(name):
     lists, _ = radius_graph(d["pos_q"], wl.cutoff_q, K=wl.K, rows=rows)
     for i, ref in zip(rows, lists):
         assert np.array_equal(np.sort(nbr[i, :cnt[i]]), np.sort(ref)), i
+        if full[i] > wl.K:
+            # a truncated row is listed nearest first, ties to the smaller index
+            assert np.array_equal(nbr[i], ref), i
+    # the sample covers truncated rows where there are any
+    assert any(full[i] > wl.K for i in rows) or not np.any(full > wl.K)
+
+
+@pytest.mark.parametrize("n", [300, 800, 1500])
+def test_graph_dense_cluster_truncation(n):
+    """Every atom within the cutoff of every other: each row keeps its K = 64
+    nearest of n - 1, nearest first, ties (repeated positions) to the smaller
+    index.  The three sizes put the rows' key counts in the three selection
+    regimes of the padded builder: within the fill kernel's own key buffer,
+    in the block-wide sort, and above the sort's capacity (bisection)."""
+    egat = _egat()
+    rng = np.random.default_rng(11)
+    cutoff_q = 100_000
+    pos = rng.integers(0, 50_000, size=(n, 3)).astype(np.int32)   # diameter < 86,603
+    pos[n // 2:n // 2 + 20] = pos[:20]                              # repeated positions
+    pos[-5:] = pos[7]
+    K = 64
+    g = egat.egat_build_graph(torch.from_numpy(pos).cuda(), cutoff_q, K=K)
+    nbr = g["nbr"].cpu().numpy()
+    cnt = g["cnt"].cpu().numpy()
+    lists, full = radius_graph(pos, cutoff_q, K=K)
+    assert np.all(full == n - 1) and np.all(cnt == K)
+    for i, ref in enumerate(lists):
+        assert np.array_equal(nbr[i], ref), i
+    assert int(g["overflow"].item()) == n * (n - 1 - K)
 
 
 # --------------------------------------------------------------------------- steps 2, 3

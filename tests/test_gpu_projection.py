@@ -130,9 +130,9 @@ def test_projected_forward(name):
         assert channel_rel_error(out, ref, wl.lmax, FLOOR["f32"]) < TOL["f32"]
 
 
-def test_projection_misaligned_weights_take_the_plain_path():
-    """Weights that are only 4-byte aligned (an offset view) give the same q and
-    k through the plain kernel, within the bf16 bar of the oracle."""
+def test_projection_weights_at_any_float_offset():
+    """Weights that are only 4-byte aligned (an offset view) give q and k within
+    the bf16 bar of the oracle: the kernels read them as single floats."""
     wl, d, w = _data("uniform4096_l2_bf16")
     egat = _egat()
     hd = torch.from_numpy(np.ascontiguousarray(d["h"])).to("cuda", dtype=torch.bfloat16)
