@@ -9,22 +9,21 @@
 //     q[i][h*dk + d] = sum_c h[i][0][c] wq[c][h*dk + d],   k likewise with wk.
 //
 // This is a dense contraction, [n x C] . [C x H*dk] twice, so the bf16
-// shapes with C = 128 and H*dk = 256 run on tensor cores:
-//  * a persistent CTA holds one weight matrix (wq or wk, by CTA parity) in
-//    shared memory as a bf16 pair hi + lo (hi = bf16(w), lo = bf16(w - hi)),
-//    transposed [H*dk][C] so that ldmatrix yields mma B fragments; the pair
-//    carries the float32 weights to about 2^-17, and h is exactly bf16;
-//  * tiles of 64 atoms: one thread issues one 256-byte bulk copy per atom
-//    (the degree-0 slice of its row; cp.async.bulk, no multicast) into a
-//    ring of four row-padded A tiles, each completing its own mbarrier, so
-//    three tiles are in flight while one is multiplied; every wait is bounded;
-//  * 16 warps, each 32 atoms x 32 output columns: per 16-channel k-step two
-//    A fragments (ldmatrix.x4), two B fragment pairs for hi and lo, and 16
-//    mma.sync m16n8k16 (bf16 in, float32 accumulation);
-//  * the accumulators are rounded once to the storage type and stored.
+// shapes with C = 128 and H*dk = 256 run on the fifth-generation tensor
+// cores (tcgen05.mma, accumulators in tensor memory):
+//  * a persistent CTA per SM holds one weight matrix (wq or wk, by CTA
+//    parity) in shared memory as a bf16 pair hi + lo (hi = bf16(w),
+//    lo = bf16(w - hi)), transposed to [H*dk][C]; the pair carries the
+//    float32 weights to about 2^-17, and h is exactly bf16;
+//  * per 128-atom tile the degree-0 slices (256 bytes per atom) arrive by
+//    16-byte cp.async copies, two tiles in flight, and one thread issues
+//    sixteen 128 x 256 x 16 products (h W_hi and h W_lo per 16-channel step)
+//    into 256 float32 columns of tensor memory, completing an mbarrier;
+//  * eight warps read the accumulator back (tcgen05.ld), round once to the
+//    storage type and store.  Every wait is bounded.
 // It moves n * (C + 2 * H*dk) * 2 bytes (degree-0 slices in, q and k out):
-// an HBM-bound contraction (K = C = 128 gives 64 FLOP per stored byte of
-// output at most), so the kernel is measured against HBM bandwidth.
+// K = C = 128 gives at most 64 FLOP per stored byte of output, so the
+// kernel is measured against HBM bandwidth.
 //
 // Other shapes (float32 storage, other C or H*dk) take a plain kernel: a CTA
 // stages the degree-0 channels of 8 atoms and each thread forms output
@@ -37,52 +36,110 @@
 namespace egat {
 namespace {
 
-constexpr int kPC = 128;          // channels (the contraction length)
-constexpr int kPN = 256;          // H * dk outputs per matrix
-constexpr int kPM = 64;           // atoms per tile
-constexpr int kPRow = kPC * 2 + 16;   // padded bf16 row (272 B): ldmatrix phases hit distinct banks
-constexpr int kPWarps = 16;
-constexpr int kPBuf = 4;              // A tiles in the ring
-
-struct ProjSmem {
-  static constexpr size_t whi = 0;                                   // [kPN][kPRow]
-  static constexpr size_t wlo = whi + size_t(kPN) * kPRow;           // [kPN][kPRow]
-  static constexpr size_t a = wlo + size_t(kPN) * kPRow;             // [kPBuf][kPM][kPRow]
-  static constexpr size_t bars = a + size_t(kPBuf) * kPM * kPRow;    // [kPBuf] mbarriers + abort flag
-  static constexpr size_t total = bars + kPBuf * 8 + 16;
-  static_assert(kPRow % 16 == 0 && a % 16 == 0 && bars % 8 == 0, "bulk-copy alignment");
-};
-
 struct ProjParams {
   const __nv_bfloat16* h;
-  const float* w[2];      // wq, wk  [kPC][kPN]
-  __nv_bfloat16* out[2];  // q, k    [n][kPN]
+  const float* w[2];      // wq, wk  [C][H*dk]
+  __nv_bfloat16* out[2];  // q, k    [n][H*dk]
   long long row_elems;    // D * C: elements per atom row of h
   int n;
-  int tiles;
+  int tiles;              // 128-atom tiles
 };
 
-__device__ __forceinline__ void pj_ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
+// ---------------------------------------------------------------- tcgen05 path
+// One CTA per SM holds one weight matrix (wq or wk, by CTA parity) as bf16
+// hi and lo tiles and takes 128-atom tiles:
+//  * A (the tile's degree-0 slices, 128 x 128 bf16) arrives by 16-byte
+//    cp.async copies, two tiles in flight (a ragged tile's missing rows are
+//    zero-filled);
+//  * one thread issues the tile's 16 tcgen05.mma (M = 128, N = 256, K = 16:
+//    eight k-steps, each against the hi and the lo tile), accumulating
+//    h W_hi + h W_lo in float32 in tensor memory (256 columns), and commits
+//    them to an mbarrier;
+//  * eight warps read the accumulator back (tcgen05.ld, each warp its
+//    32-lane quarter and half of the columns), round to bf16 and store.
+// Shared-memory operands use the K-major no-swizzle canonical layout: 8-row
+// x 16-byte core matrices of 128 contiguous bytes, 8-row groups 128 bytes
+// apart (SBO), the two 8-channel halves of a k-step one channel chunk apart
+// (LBO).
+constexpr int kUM = 128;                 // atoms per tile (M)
+constexpr int kUN = 256;                 // outputs per matrix (N)
+constexpr int kUK = 128;                 // channels (K)
+constexpr int kUWarps = 8;
+constexpr int kUChunkA = kUM * 16;       // bytes per 8-channel chunk of an A tile
+constexpr int kUChunkB = kUN * 16;       // bytes per 8-channel chunk of a B tile
+constexpr int kUCols = 256;              // tensor-memory columns (float32 accumulator, N = 256)
+
+struct UmmaSmem {
+  static constexpr size_t bhi = 0;                                      // [16][32][8][16 B]
+  static constexpr size_t blo = bhi + size_t(kUK / 8) * kUChunkB;
+  static constexpr size_t a = blo + size_t(kUK / 8) * kUChunkB;         // [2][16][16][8][16 B]
+  static constexpr size_t bars = a + 2 * size_t(kUK / 8) * kUChunkA;    // mma mbarrier
+  static constexpr size_t tslot = bars + 8;                              // tensor-memory address
+  static constexpr size_t flag = tslot + 4;                              // abort flag
+  static constexpr size_t total = flag + 4 + 16;
+  static_assert(a % 1024 == 0 && bars % 8 == 0, "operand alignment");
+};
+
+// Shared-memory matrix descriptor: start, leading and stride byte offsets
+// (16-byte units), descriptor version 1, no swizzle.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return uint64_t((saddr >> 4) & 0x3FFFu) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) |
+         (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (uint64_t(1) << 46);
 }
-__device__ __forceinline__ void pj_mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                       uint32_t b1) {
+// Instruction descriptor, kind::f16: float32 accumulator, bf16 A and B, both
+// K-major, N = 256, M = 128.
+constexpr uint32_t kUIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kUN >> 3) << 17) |
+                             (uint32_t(kUM >> 4) << 24);
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, bool accumulate) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kUIdesc), "r"(uint32_t(accumulate))
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void tmem_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+// 32 consecutive float32 columns of this thread's lane
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+      "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, "
+      "[%32];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-__global__ void __launch_bounds__(kPWarps * 32, 1) qk_projection_tc_kernel(const __grid_constant__ ProjParams p) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  unsigned char* whi = smem + ProjSmem::whi;
-  unsigned char* wlo = smem + ProjSmem::wlo;
-  unsigned char* abuf = smem + ProjSmem::a;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + ProjSmem::bars);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + kPBuf);
+__global__ void __launch_bounds__(kUWarps * 32, 1) qk_projection_umma_kernel(const __grid_constant__ ProjParams p) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  unsigned char* bhi = smem + UmmaSmem::bhi;
+  unsigned char* blo = smem + UmmaSmem::blo;
+  unsigned char* abuf = smem + UmmaSmem::a;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + UmmaSmem::bars);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + UmmaSmem::tslot);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + UmmaSmem::flag);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int sel = blockIdx.x & 1;            // 0: q from wq, 1: k from wk
@@ -91,130 +148,145 @@ __global__ void __launch_bounds__(kPWarps * 32, 1) qk_projection_tc_kernel(const
   if (slot >= p.tiles) return;               // whole CTA
 
   if (tid == 0) {
-    for (int b = 0; b < kPBuf; ++b) mbar_init(smem_u32(bar + b), 1);
+    mbar_init(smem_u32(bar), 1);
     mbar_fence_init();
     *abort_flag = 0;
   }
-  // weights: float32 [c][col] -> transposed bf16 hi/lo [col][c], stored as
-  // (c, c + 1) pairs.  A warp converts a block of 8 columns x 4 channel
-  // pairs: lane -> column 8 cb + (lane & 7), pair 4 pb + (lane >> 3).  With
-  // the 68-word row pitch its 32 four-byte stores hit 32 distinct banks, and
-  // each load instruction reads 8 full 32-byte sectors.  Every load of the
-  // thread is issued before the first conversion.
-  const float* w = p.w[sel];
-  constexpr int kPer = (kPC / 2) * kPN / (kPWarps * 32);   // pairs per thread
-  static_assert((kPC / 2) * kPN % (kPWarps * 32 * 32) == 0 && kPN % 8 == 0, "weight blocks");
-  float x0[kPer], x1[kPer];
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int blk = i * kPWarps + warp;
-    const int col = (blk % (kPN / 8)) * 8 + (lane & 7);
-    const int c = 2 * ((blk / (kPN / 8)) * 4 + (lane >> 3));
-    x0[i] = __ldg(w + c * kPN + col);
-    x1[i] = __ldg(w + (c + 1) * kPN + col);
+  if (warp == 0) {
+    // 256 columns of tensor memory (one CTA per SM: the shared memory fills it)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tslot)),
+                 "r"(kUCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int blk = i * kPWarps + warp;
-    const int col = (blk % (kPN / 8)) * 8 + (lane & 7);
-    const int c = 2 * ((blk / (kPN / 8)) * 4 + (lane >> 3));
-    const __nv_bfloat162 hi = __floats2bfloat162_rn(x0[i], x1[i]);
-    const __nv_bfloat162 lo =
-        __floats2bfloat162_rn(x0[i] - __low2float(hi), x1[i] - __high2float(hi));
-    *reinterpret_cast<__nv_bfloat162*>(whi + size_t(col) * kPRow + c * 2) = hi;
-    *reinterpret_cast<__nv_bfloat162*>(wlo + size_t(col) * kPRow + c * 2) = lo;
-  }
-  __syncthreads();
 
   const char* hb = reinterpret_cast<const char*>(p.h);
   const long long row_bytes = p.row_elems * 2;
-  // thread 0: the degree-0 slices (first 256 bytes of each row) of tile tl
-  auto issue = [&](int tl, int b) {
-    const int a0 = tl * kPM;
-    const int valid = p.n - a0 < kPM ? p.n - a0 : kPM;
-    const uint32_t bb = smem_u32(bar + b);
-    mbar_arrive_expect_tx(bb, uint32_t(valid) * (kPC * 2));
-    for (int r = 0; r < valid; ++r)
-      bulk_g2s(smem_u32(abuf + (size_t(b) * kPM + r) * kPRow), hb + (long long)(a0 + r) * row_bytes,
-               kPC * 2, bb);
+  // the degree-0 slices of tile tl into A buffer b: 16-byte chunk (atom m,
+  // channels 8c .. 8c+7) at c * kUChunkA + (m / 8) * 128 + (m % 8) * 16;
+  // rows past n are zero-filled
+  auto load_tile = [&](int tl, int b) {
+    if (tl < p.tiles) {
+      const uint32_t base = smem_u32(abuf + size_t(b) * (kUK / 8) * kUChunkA);
+      // a warp moves 8 atoms x 4 chunks: 128 contiguous bytes of shared
+      // memory per chunk, 64 contiguous bytes of global memory per atom
+      for (int e = tid; e < kUM * (kUK / 8); e += kUWarps * 32) {
+        const int wi = e >> 5, ln = e & 31;
+        const int m = (wi & 15) * 8 + (ln & 7), c = (wi >> 4) * 4 + (ln >> 3);
+        const long long atom = (long long)tl * kUM + m;
+        const bool ok = atom < p.n;
+        const char* src = hb + (ok ? atom * row_bytes + c * 16 : 0);
+        cp_async16(base + c * kUChunkA + (m >> 3) * 128 + (m & 7) * 16, src, ok ? 16u : 0u);
+      }
+    }
+    cp_async_commit();   // one group per tile slot, empty past the last tile
   };
-  // the ring starts with the CTA's first kPBuf - 1 tiles in flight
-  if (tid == 0)
-    for (int q = 0; q < kPBuf - 1 && slot + q * stride < p.tiles; ++q) issue(slot + q * stride, q);
+  load_tile(slot, 0);
+  load_tile(slot + stride, 1);
 
-  const int g = lane >> 2, t = lane & 3;
-  const int m0 = (warp & 1) * 32;            // this warp's first atom of the tile
-  const int n0 = (warp >> 1) * 32;           // this warp's first output column
+  // weights: float32 [k][n] -> bf16 hi / lo at (k / 8) * kUChunkB +
+  // (n / 8) * 128 + (n % 8) * 16 + (k % 8) * 2, stored as (k, k + 1) pairs.
+  // A warp converts 8 columns x 4 channel pairs per step: lane -> column
+  // 8 nb + (lane & 7), pair 4 kb + (lane >> 3); its 32 four-byte stores hit
+  // 32 distinct banks.
+  {
+    const float* w = p.w[sel];
+    constexpr int kBlocks = (kUN / 8) * (kUK / 8);   // 8 x 8 blocks: 512
+    constexpr int kBatch = 16;                       // blocks in flight per warp
+#pragma unroll 1
+    for (int b0 = warp * kBatch; b0 < kBlocks; b0 += kUWarps * kBatch) {
+      float x0[kBatch], x1[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const int blk = b0 + i;
+        const int n = (blk % (kUN / 8)) * 8 + (lane & 7);
+        const int k = 2 * ((blk / (kUN / 8)) * 4 + (lane >> 3));
+        x0[i] = __ldg(w + k * kUN + n);
+        x1[i] = __ldg(w + (k + 1) * kUN + n);
+      }
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const int blk = b0 + i;
+        const int n = (blk % (kUN / 8)) * 8 + (lane & 7);
+        const int k = 2 * ((blk / (kUN / 8)) * 4 + (lane >> 3));
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(x0[i], x1[i]);
+        const __nv_bfloat162 lo =
+            __floats2bfloat162_rn(x0[i] - __low2float(hi), x1[i] - __high2float(hi));
+        const size_t off = size_t(k >> 3) * kUChunkB + (n >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2;
+        *reinterpret_cast<__nv_bfloat162*>(bhi + off) = hi;
+        *reinterpret_cast<__nv_bfloat162*>(blo + off) = lo;
+      }
+    }
+  }
+  fence_proxy_async_smem();   // the weight tiles are read by the tensor core
+  tmem_fence_before();
+  __syncthreads();
+  tmem_fence_after();
+  const uint32_t tmem = *tslot;
+
   __nv_bfloat16* out = p.out[sel];
+  const int quarter = warp & 3, colh = warp >> 2;   // TMEM lanes 32 quarter.., columns 128 colh..
+  bool ok = true;
   int j = 0;
   for (int tile = slot; tile < p.tiles; tile += stride, ++j) {
-    const int b = j % kPBuf;
-    bounded_wait(smem_u32(bar + b), uint32_t(j / kPBuf) & 1u, kWaitPolls, abort_flag);
-    // the tile kPBuf - 1 ahead into the buffer tile j - 1 used (it ended
-    // with a barrier)
-    const int ahead = tile + (kPBuf - 1) * stride;
-    if (tid == 0 && ahead < p.tiles) issue(ahead, (j + kPBuf - 1) % kPBuf);
-    float acc[2][4][4];
+    const int b = j & 1;
+    cp_async_wait<1>();          // this tile's group (the next one may still fly)
+    fence_proxy_async_smem();    // its bytes are read by the tensor core
+    tmem_fence_before();         // the previous tile's accumulator reads are done
+    __syncthreads();
+    if (tid == 0) {
+      tmem_fence_after();
+      const uint32_t a0 = smem_u32(abuf + size_t(b) * (kUK / 8) * kUChunkA);
+      const uint32_t h0 = smem_u32(bhi), l0 = smem_u32(blo);
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+      for (int s = 0; s < kUK / 16; ++s) {
+        const uint64_t ad = umma_desc(a0 + 2 * s * kUChunkA, kUChunkA, 128);
+        umma_bf16(tmem, ad, umma_desc(h0 + 2 * s * kUChunkB, kUChunkB, 128), s > 0);
+        umma_bf16(tmem, ad, umma_desc(l0 + 2 * s * kUChunkB, kUChunkB, 128), true);
+      }
+      umma_commit(smem_u32(bar));
+    }
+    // every thread leaves together if the commit never arrives
+    ok = __syncthreads_and(bounded_wait(smem_u32(bar), uint32_t(j) & 1u, kWaitPolls, abort_flag));
+    if (!ok) break;
+    tmem_fence_after();
+    // A buffer b is free: the tile two ahead goes there
+    load_tile(tile + 2 * stride, b);
+    const long long atom = (long long)tile * kUM + quarter * 32 + lane;
+    __nv_bfloat16* o = out + atom * kUN + colh * 128;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t r[32];
+      tmem_ld32(tmem + (uint32_t(quarter * 32) << 16) + uint32_t(colh * 128 + c * 32), r);
+      tmem_ld_wait();
+      if (atom < p.n) {
+        uint4* o4 = reinterpret_cast<uint4*>(o + c * 32);
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt)
+        for (int v = 0; v < 4; ++v) {
+          uint32_t wv[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
-    const uint32_t a_base = smem_u32(abuf + size_t(b) * kPM * kPRow);
-    const int arow = (lane & 7) + 8 * ((lane >> 3) & 1);
-    const int brow = (lane & 7) + 8 * (lane >> 4);
-    const int bhalf = (lane >> 3) & 1;
-#pragma unroll 2
-    for (int kk = 0; kk < kPC / 16; ++kk) {
-      uint32_t af[2][4];
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
-        pj_ldsm_x4(af[mt], a_base + (m0 + mt * 16 + arow) * kPRow + kk * 32 + (lane >> 4) * 16);
-#pragma unroll
-      for (int np = 0; np < 2; ++np) {       // pairs of n8 tiles
-        uint32_t bh[4], bl[4];
-        const uint32_t off = (n0 + np * 16 + brow) * kPRow + kk * 32 + bhalf * 16;
-        pj_ldsm_x4(bh, smem_u32(whi) + off);
-        pj_ldsm_x4(bl, smem_u32(wlo) + off);
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-          pj_mma(acc[mt][2 * np], af[mt], bh[0], bh[1]);
-          pj_mma(acc[mt][2 * np + 1], af[mt], bh[2], bh[3]);
-          pj_mma(acc[mt][2 * np], af[mt], bl[0], bl[1]);
-          pj_mma(acc[mt][2 * np + 1], af[mt], bl[2], bl[3]);
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 pr = __floats2bfloat162_rn(__uint_as_float(r[8 * v + 2 * e]),
+                                                            __uint_as_float(r[8 * v + 2 * e + 1]));
+            wv[e] = *reinterpret_cast<const uint32_t*>(&pr);
+          }
+          o4[v] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
         }
       }
     }
-    // rows g and g+8 of each m tile, columns 2t, 2t+1 of each n tile
-    const int a0 = tile * kPM + m0;
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int atom = a0 + mt * 16 + g + 8 * half;
-        if (atom < p.n) {
-          __nv_bfloat16* o = out + (long long)atom * kPN + n0 + 2 * t;
-#pragma unroll
-          for (int nt = 0; nt < 4; ++nt)
-            *reinterpret_cast<__nv_bfloat162*>(o + nt * 8) =
-                __floats2bfloat162_rn(acc[mt][nt][2 * half], acc[mt][nt][2 * half + 1]);
-        }
-      }
-    __syncthreads();   // buffer b is refilled by a later iteration's issue
   }
-  if (*abort_flag && tid == 0) {
-    // a wait gave up: give each buffer's last issued phase a short, bounded
-    // chance to complete before the CTA's shared memory is released (tile
-    // sequence numbers up to j + kPBuf - 2 may have been issued)
+  cp_async_wait<0>();
+  if (!ok && tid == 0) {
+    // the commit never arrived: a short, bounded chance for the products in
+    // flight to finish before their tensor memory is released
     volatile int none = 0;
-    for (int b = 0; b < kPBuf; ++b) {
-      int last = -1;
-      for (int q = 0; q < j + kPBuf - 1; ++q)
-        if (q % kPBuf == b && slot + q * stride < p.tiles) last = q;
-      if (last >= 0)
-        bounded_wait(smem_u32(bar + b), uint32_t(last / kPBuf) & 1u, kDrainPolls, &none);
-    }
+    bounded_wait(smem_u32(bar), uint32_t(j) & 1u, kDrainPolls, &none);
+  }
+  tmem_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tmem_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kUCols) : "memory");
   }
 }
 
@@ -265,7 +337,7 @@ __global__ void __launch_bounds__(256) qk_projection_kernel(const T* __restrict_
 }  // namespace
 
 bool projection_tc_supported(const egat_shape& s) {
-  return s.dtype == EGAT_BF16 && s.C == kPC && s.H * s.dk == kPN;
+  return s.dtype == EGAT_BF16 && s.C == kUK && s.H * s.dk == kUN;
 }
 
 int launch_qk_projection(const egat_shape& s, const void* d_h, const float* d_wq, const float* d_wk,
@@ -281,9 +353,9 @@ int launch_qk_projection(const egat_shape& s, const void* d_h, const float* d_wq
     p.out[1] = static_cast<__nv_bfloat16*>(d_k);
     p.row_elems = row_elems;
     p.n = s.n;
-    p.tiles = (s.n + kPM - 1) / kPM;
-    const size_t shmem = ProjSmem::total;
-    if (cudaFuncSetAttribute(qk_projection_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    p.tiles = (s.n + kUM - 1) / kUM;
+    const size_t shmem = UmmaSmem::total;
+    if (cudaFuncSetAttribute(qk_projection_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(shmem)) != cudaSuccess)
       return EGAT_ERR_CUDA;
     int dev = 0, sms = 148;
@@ -291,7 +363,7 @@ int launch_qk_projection(const egat_shape& s, const void* d_h, const float* d_wq
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     // one CTA per SM, an even count: CTA pairs share atom tiles, one for q, one for k
     const int pairs = p.tiles < sms / 2 ? p.tiles : sms / 2;
-    qk_projection_tc_kernel<<<2 * (pairs > 0 ? pairs : 1), kPWarps * 32, shmem, st>>>(p);
+    qk_projection_umma_kernel<<<2 * (pairs > 0 ? pairs : 1), kUWarps * 32, shmem, st>>>(p);
     return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
   }
   const int blocks = (s.n + kGenAtoms - 1) / kGenAtoms;

@@ -12,8 +12,8 @@ node features (reading: a linear map of each atom's degree-0 channels).
   rounding plus the float32 accumulation error, 2^-19 of the sum of the
   terms' magnitudes.
 * The tensor-core path (bf16, C = 128, H*dk = 256) on every bf16 workload,
-  ragged tails (1, 63, 65 and 1,000 atoms: partial 64-atom tiles) and the
-  plain path (float32 workloads, other channel counts).
+  ragged tails (1, 63, 65, 127, 129 and 1,000 atoms: partial 128-atom
+  tiles) and the plain path (float32 workloads, other channel counts).
 * Rotating every degree block of h by its Wigner-D matrix leaves the GPU's
   q and k bitwise unchanged (only degree 0 is read).
 * The projected queries and keys drive the fused forward: egat_qk_projection
@@ -80,7 +80,7 @@ def test_projection_parity(name):
     assert _egat().egat_take_device_status() == _egat().EGAT_OK
 
 
-@pytest.mark.parametrize("n", [1, 63, 65, 1000])
+@pytest.mark.parametrize("n", [1, 63, 65, 127, 129, 1000])
 @pytest.mark.parametrize("dtype,C,H,dk", [("bf16", 128, 16, 16), ("f32", 64, 4, 16),
                                           ("bf16", 32, 4, 8)])
 def test_projection_ragged(n, dtype, C, H, dk):

@@ -1,88 +1,75 @@
-"""Host-side model of the copy / wait protocol of the tensor-core query/key
-projection (`qk_projection_tc_kernel`, csrc/projection.cu).
+"""Host-side model of the copy / product protocol of the tensor-core
+query/key projection (`qk_projection_umma_kernel`, csrc/projection.cu).
 
-A CTA walks its tiles slot, slot + stride, ... .  Bulk copies fill a ring of
-kPBuf shared-memory tiles, each completing its own mbarrier; the ring starts
-with the first kPBuf - 1 tiles in flight, iteration j waits on buffer
-j % kPBuf (phase parity (j / kPBuf) & 1), then issues the tile kPBuf - 1
-ahead into the buffer iteration j - 1 read, and ends with a block barrier.
-After a wait gives up, the drain waits on the last issued phase of every
-buffer.  This model replays that control flow for many tile counts and grid
-sizes and checks:
+A CTA walks its tiles slot, slot + stride, ... .  Its threads fill two
+shared-memory A buffers with cp.async copies, one commit group per tile
+sequence number (an empty group past the last tile): groups 0 and 1 before
+the loop, group j + 2 in iteration j once the products of tile j are done.
+Iteration j waits until at most one group is pending (cp.async.wait_group 1),
+issues tile j's products from buffer j % 2, and waits on the mbarrier phase
+of parity j % 2 that their commit completes.  This model replays that
+control flow for many tile counts and grid sizes and checks:
 
-* every wait names the parity of the fill that delivers the tile it reads;
-* no buffer is refilled before the barrier that ends the iteration reading
-  its previous contents;
-* every issued fill is waited on, in the loop or by the drain, and the drain
-  waits exactly the last issued fill of each buffer.
+* the group that fills tile j's buffer is complete when its products are
+  issued, and it carries tile j;
+* no buffer is refilled before the products that read its previous tile
+  have completed;
+* one commit per tile, so the mbarrier has at most one phase pending and
+  tile j waits on parity j % 2;
+* every tile of the CTA is multiplied exactly once, and every group is
+  complete when the CTA exits (cp.async.wait_group 0).
 No GPU is involved.
 """
 import pytest
 
-K_PBUF = 4          # the kernel's kPBuf
-K_PM = 64           # atoms per tile
+K_UM = 128          # the kernel's kUM: atoms per tile
 
 
 def replay(tiles: int, slot: int, stride: int):
-    fills = {b: [] for b in range(K_PBUF)}       # buffer -> tile sequence numbers issued
-    waited = set()                               # (buffer, fill index)
-    barriers = 0
-    issued_at = {}                               # (buffer, fill index) -> barrier count at issue
+    groups = []                      # committed groups: (sequence number, buffer, tile or None)
+    complete = 0                     # groups complete so far (they complete in order)
+    buffer_busy = {0: None, 1: None}  # buffer -> sequence number whose products still read it
+    done_products = set()
+    phases = 0                       # mbarrier phases completed
 
-    def issue(seq):
-        b = seq % K_PBUF
-        if fills[b]:
-            prev = fills[b][-1]
-            # the previous contents are read by iteration prev, which must have
-            # ended with its barrier (one barrier per iteration, from 0)
-            assert barriers >= prev + 1, (seq, prev, barriers)
-            assert prev < seq
-        fills[b].append(seq)
-        issued_at[(b, len(fills[b]) - 1)] = barriers
+    def load(seq, b):
+        tile = slot + seq * stride
+        assert buffer_busy[b] is None, (seq, b, buffer_busy[b])
+        groups.append((seq, b, tile if tile < tiles else None))
 
-    for q in range(K_PBUF - 1):
-        if slot + q * stride < tiles:
-            issue(q)
+    load(0, 0)
+    load(1, 1)
     j = 0
     tile = slot
+    multiplied = []
     while tile < tiles:
-        b = j % K_PBUF
-        parity = (j // K_PBUF) & 1
-        k = fills[b].index(j)                   # the fill that carries tile j
-        assert k % 2 == parity
-        waited.add((b, k))
-        if tile + (K_PBUF - 1) * stride < tiles:
-            issue(j + K_PBUF - 1)
-        barriers += 1                           # __syncthreads ends iteration j
+        b = j % 2
+        # cp.async.wait_group 1: every group but the newest is complete
+        complete = max(complete, len(groups) - 1)
+        seq, gb, gtile = groups[j]
+        assert j < complete and seq == j and gb == b and gtile == tile
+        buffer_busy[b] = j                       # the products read buffer b
+        parity = phases & 1
+        assert parity == j % 2
+        phases += 1                              # the commit completes the phase
+        done_products.add(j)
+        buffer_busy[b] = None                    # products done: buffer b is free
+        multiplied.append(tile)
+        load(j + 2, b)
         tile += stride
         j += 1
-    # the kernel's drain after a give-up: the last issued sequence number of
-    # each buffer among 0 .. j + kPBuf - 2 (those that exist)
-    drain = {}
-    for b in range(K_PBUF):
-        last = -1
-        for q in range(j + K_PBUF - 1):
-            if q % K_PBUF == b and slot + q * stride < tiles:
-                last = q
-        if last >= 0:
-            drain[b] = (last // K_PBUF) & 1
-    for b, seqs in fills.items():
-        if seqs:
-            assert b in drain and drain[b] == ((len(seqs) - 1) % 2), (b, seqs)
-            for k in range(len(seqs)):
-                assert (b, k) in waited or k == len(seqs) - 1
-        else:
-            assert b not in drain
-    return j
+    complete = len(groups)                       # cp.async.wait_group 0 before exit
+    assert all(i < complete for i in range(len(groups)))
+    assert len(groups) == j + 2
+    return multiplied
 
 
-@pytest.mark.parametrize("n", [1, 63, 64, 65, 1000, 4096, 32768, 100000, 175616])
+@pytest.mark.parametrize("n", [1, 127, 128, 129, 1000, 4096, 32768, 100000, 175616])
 @pytest.mark.parametrize("sms", [148, 8])
-def test_projection_ring_protocol(n, sms):
-    tiles = (n + K_PM - 1) // K_PM
+def test_projection_copy_product_protocol(n, sms):
+    tiles = (n + K_UM - 1) // K_UM
     pairs = min(tiles, sms // 2)
-    stride = pairs
-    done = 0
+    seen = []
     for slot in range(pairs):
-        done += replay(tiles, slot, stride)
-    assert done == tiles                         # every tile is processed by exactly one CTA of a pair
+        seen += replay(tiles, slot, pairs)
+    assert sorted(seen) == list(range(tiles))   # every tile once per matrix (q or k)
