@@ -560,18 +560,56 @@ __device__ __forceinline__ void coupling_grad_channel(float (&g)[(L + 1) * (L + 
   };
   to_frame(g);
   to_frame(x);
+  if constexpr (L >= 3) {
+    // One pass over the paths with all five dot products at once, so that
+    // each path's weight and factors are read for one use: at lmax 3 the
+    // five separate passes keep them live across passes, past the registers.
+    float jgx[D], jxx[D], jgy[D], jxy[D];
+    gen_apply(0, g, jgx);
+    gen_apply(0, x, jxx);
+    gen_apply(1, g, jgy);
+    gen_apply(1, x, jxy);
+    float adr = 0.f, atx = 0.f, aty = 0.f;
+    static_for<0, num_paths(L)>([&](auto pc) {
+      constexpr int p = decltype(pc)::value;
+      constexpr int li = path_info(L, p, 0);
+      constexpr int lf = path_info(L, p, 1);
+      constexpr int lo = path_info(L, p, 2);
+      constexpr bool even = ((li + lf + lo) % 2) == 0;
+      const float w = wgt(p);
+      float pdr = 0.f, ptx = 0.f, pty = 0.f;
+#pragma unroll
+      for (int mo = -lo; mo <= lo; ++mo) {
+        const int src = even ? mo : -mo;
+        const bool live = (iabs(mo) <= li) && (even || mo != 0);
+        if (live) {
+          const int uo = lo * lo + lo + mo, vi = li * li + li + src;
+          const float f = tab.f[p][mo + lo];
+          pdr = fmaf(f * g[uo], x[vi], pdr);
+          ptx = fmaf(f, fmaf(jgx[uo], x[vi], g[uo] * jxx[vi]), ptx);
+          pty = fmaf(f, fmaf(jgy[uo], x[vi], g[uo] * jxy[vi]), pty);
+        }
+      }
+      adr = fmaf(w * drpow[lf], pdr, adr);
+      atx = fmaf(w * rpow[lf], ptx, atx);
+      aty = fmaf(w * rpow[lf], pty, aty);
+    });
+    dr += adr;
+    tx += atx;
+    ty += aty;
+    return;
+  }
   dr += reindex_dot(g, x, drpow);
   // <J_b g~, Rw x~> = <Rw^T J_b g~, x~> = reindex_dot(J_b g~, x~); <g~, Rw J_b x~> = reindex_dot(g~, J_b x~)
-#pragma unroll 1
-  for (int bax = 0; bax < 2; ++bax) {
+  static_for<0, 2>([&](auto bc) {
+    constexpr int bax = decltype(bc)::value;
     float jv[D];
     gen_apply(bax, g, jv);
     float s = reindex_dot(jv, x, rpow);
     gen_apply(bax, x, jv);
     s += reindex_dot(g, jv, rpow);
-    tx += bax == 0 ? s : 0.f;
-    ty += bax == 1 ? s : 0.f;
-  }
+    if constexpr (bax == 0) tx += s; else ty += s;
+  });
 }
 
 // eaas_multi on channel pairs: the same operations in the same order per
