@@ -14,13 +14,18 @@
 //  * a persistent CTA per SM holds one weight matrix (wq or wk, by CTA
 //    parity) in shared memory as a bf16 pair hi + lo (hi = bf16(w),
 //    lo = bf16(w - hi)), transposed to [H*dk][C]; the pair carries the
-//    float32 weights to about 2^-17, and h is exactly bf16;
+//    float32 weights to about 2^-17, and h is exactly bf16.  The float32
+//    matrix arrives in two 64 KB bulk copies (cp.async.bulk, no multicast)
+//    and is converted from shared memory;
 //  * per 128-atom tile the degree-0 slices (256 bytes per atom) arrive by
 //    16-byte cp.async copies, two tiles in flight, and one thread issues
 //    sixteen 128 x 256 x 16 products (h W_hi and h W_lo per 16-channel step)
-//    into 256 float32 columns of tensor memory, completing an mbarrier;
+//    into one of two 256-column float32 accumulators in tensor memory,
+//    completing that accumulator's mbarrier; tile j + 1's products run while
+//    tile j is read back;
 //  * eight warps read the accumulator back (tcgen05.ld), round once to the
-//    storage type and store.  Every wait is bounded.
+//    storage type and store through shared memory, 64 contiguous bytes of a
+//    row per four lanes.  Every wait is bounded.
 // It moves n * (C + 2 * H*dk) * 2 bytes (degree-0 slices in, q and k out):
 // K = C = 128 gives at most 64 FLOP per stored byte of output, so the
 // kernel is measured against HBM bandwidth.
@@ -67,14 +72,16 @@ constexpr int kUK = 128;                 // channels (K)
 constexpr int kUWarps = 8;
 constexpr int kUChunkA = kUM * 16;       // bytes per 8-channel chunk of an A tile
 constexpr int kUChunkB = kUN * 16;       // bytes per 8-channel chunk of a B tile
-constexpr int kUCols = 256;              // tensor-memory columns (float32 accumulator, N = 256)
+constexpr int kUCols = 512;              // tensor-memory columns: two float32 accumulators of N = 256
+constexpr int kUStageRow = 80;           // a staged 64-byte output row segment, padded (bank spread)
 
 struct UmmaSmem {
   static constexpr size_t bhi = 0;                                      // [16][32][8][16 B]
   static constexpr size_t blo = bhi + size_t(kUK / 8) * kUChunkB;
   static constexpr size_t a = blo + size_t(kUK / 8) * kUChunkB;         // [2][16][16][8][16 B]
-  static constexpr size_t bars = a + 2 * size_t(kUK / 8) * kUChunkA;    // mma mbarrier
-  static constexpr size_t tslot = bars + 8;                              // tensor-memory address
+  static constexpr size_t stage = a + 2 * size_t(kUK / 8) * kUChunkA;   // [8 warps][32 rows][80 B]
+  static constexpr size_t bars = stage + size_t(kUWarps) * 32 * kUStageRow;  // products [2], weight halves
+  static constexpr size_t tslot = bars + 24;                             // tensor-memory address
   static constexpr size_t flag = tslot + 4;                              // abort flag
   static constexpr size_t total = flag + 4 + 16;
   static_assert(a % 1024 == 0 && bars % 8 == 0, "operand alignment");
@@ -137,7 +144,9 @@ __global__ void __launch_bounds__(kUWarps * 32, 1) qk_projection_umma_kernel(con
   unsigned char* bhi = smem + UmmaSmem::bhi;
   unsigned char* blo = smem + UmmaSmem::blo;
   unsigned char* abuf = smem + UmmaSmem::a;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + UmmaSmem::bars);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + UmmaSmem::bars);        // [2] products per accumulator
+  uint64_t* wbar = bar + 2;                                                   // a weight half
+  unsigned char* stage = smem + UmmaSmem::stage;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + UmmaSmem::tslot);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + UmmaSmem::flag);
 
@@ -149,6 +158,8 @@ __global__ void __launch_bounds__(kUWarps * 32, 1) qk_projection_umma_kernel(con
 
   if (tid == 0) {
     mbar_init(smem_u32(bar), 1);
+    mbar_init(smem_u32(bar + 1), 1);
+    mbar_init(smem_u32(wbar), 1);
     mbar_fence_init();
     *abort_flag = 0;
   }
@@ -181,16 +192,43 @@ __global__ void __launch_bounds__(kUWarps * 32, 1) qk_projection_umma_kernel(con
     }
     cp_async_commit();   // one group per tile slot, empty past the last tile
   };
-  load_tile(slot, 0);
-  load_tile(slot + stride, 1);
-
   // weights: float32 [k][n] -> bf16 hi / lo at (k / 8) * kUChunkB +
   // (n / 8) * 128 + (n % 8) * 16 + (k % 8) * 2, stored as (k, k + 1) pairs.
   // A warp converts 8 columns x 4 channel pairs per step: lane -> column
   // 8 nb + (lane & 7), pair 4 kb + (lane >> 3); its 32 four-byte stores hit
   // 32 distinct banks.
-  {
-    const float* w = p.w[sel];
+  auto put = [&](int k, int n, float x0, float x1) {
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(x0, x1);
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(x0 - __low2float(hi), x1 - __high2float(hi));
+    const size_t off = size_t(k >> 3) * kUChunkB + (n >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2;
+    *reinterpret_cast<__nv_bfloat162*>(bhi + off) = hi;
+    *reinterpret_cast<__nv_bfloat162*>(blo + off) = lo;
+  };
+  const float* w = p.w[sel];
+  const bool staged = (reinterpret_cast<uintptr_t>(w) & 15u) == 0;
+  if (staged) {
+    // 16-byte aligned weights arrive as two bulk copies of 64 rows (64 KB of
+    // float32 each) into the A buffers, which are free until the first tile
+    const float* stage = reinterpret_cast<const float*>(abuf);
+    constexpr int kRows = kUK / 2;
+    static_assert(size_t(kRows) * kUN * 4 <= 2 * size_t(kUK / 8) * kUChunkA, "a weight half fits the A buffers");
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+      if (tid == 0) {
+        mbar_arrive_expect_tx(smem_u32(wbar), uint32_t(kRows) * kUN * 4);
+        bulk_g2s(smem_u32(abuf), w + size_t(half) * kRows * kUN, uint32_t(kRows) * kUN * 4, smem_u32(wbar));
+      }
+      bounded_wait(smem_u32(wbar), uint32_t(half), kWaitPolls, abort_flag);
+#pragma unroll 4
+      for (int blk = warp; blk < (kUN / 8) * (kRows / 8); blk += kUWarps) {
+        const int n = (blk % (kUN / 8)) * 8 + (lane & 7);
+        const int k = 2 * ((blk / (kUN / 8)) * 4 + (lane >> 3));   // row within the half
+        put(half * kRows + k, n, stage[k * kUN + n], stage[(k + 1) * kUN + n]);
+      }
+      __syncthreads();   // the half is consumed before the buffers are refilled
+    }
+  } else {
+    // other weights: every thread loads its pairs straight from global memory
     constexpr int kBlocks = (kUN / 8) * (kUK / 8);   // 8 x 8 blocks: 512
     constexpr int kBatch = 16;                       // blocks in flight per warp
 #pragma unroll 1
@@ -207,17 +245,12 @@ __global__ void __launch_bounds__(kUWarps * 32, 1) qk_projection_umma_kernel(con
 #pragma unroll
       for (int i = 0; i < kBatch; ++i) {
         const int blk = b0 + i;
-        const int n = (blk % (kUN / 8)) * 8 + (lane & 7);
-        const int k = 2 * ((blk / (kUN / 8)) * 4 + (lane >> 3));
-        const __nv_bfloat162 hi = __floats2bfloat162_rn(x0[i], x1[i]);
-        const __nv_bfloat162 lo =
-            __floats2bfloat162_rn(x0[i] - __low2float(hi), x1[i] - __high2float(hi));
-        const size_t off = size_t(k >> 3) * kUChunkB + (n >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2;
-        *reinterpret_cast<__nv_bfloat162*>(bhi + off) = hi;
-        *reinterpret_cast<__nv_bfloat162*>(blo + off) = lo;
+        put(2 * ((blk / (kUN / 8)) * 4 + (lane >> 3)), (blk % (kUN / 8)) * 8 + (lane & 7), x0[i], x1[i]);
       }
     }
   }
+  load_tile(slot, 0);
+  load_tile(slot + stride, 1);
   fence_proxy_async_smem();   // the weight tiles are read by the tensor core
   tmem_fence_before();
   __syncthreads();
@@ -226,61 +259,95 @@ __global__ void __launch_bounds__(kUWarps * 32, 1) qk_projection_umma_kernel(con
 
   __nv_bfloat16* out = p.out[sel];
   const int quarter = warp & 3, colh = warp >> 2;   // TMEM lanes 32 quarter.., columns 128 colh..
-  bool ok = true;
-  int j = 0;
-  for (int tile = slot; tile < p.tiles; tile += stride, ++j) {
-    const int b = j & 1;
-    cp_async_wait<1>();          // this tile's group (the next one may still fly)
+  const int J = (p.tiles - slot + stride - 1) / stride;   // this CTA's tiles
+  // tile jj's products from A buffer jj % 2 into accumulator jj % 2 (columns
+  // 256 (jj % 2) ..), completing mbarrier jj % 2; every thread takes part
+  // (the wait for the tile's copies and the barrier before the issue)
+  auto issue = [&](int jj) {
+    cp_async_wait<0>();          // the tile's copies (every older group too)
     fence_proxy_async_smem();    // its bytes are read by the tensor core
-    tmem_fence_before();         // the previous tile's accumulator reads are done
+    tmem_fence_before();         // the accumulator's previous reads are done
     __syncthreads();
     if (tid == 0) {
       tmem_fence_after();
+      const int b = jj & 1;
+      const uint32_t acc = tmem + uint32_t(b * kUN);
       const uint32_t a0 = smem_u32(abuf + size_t(b) * (kUK / 8) * kUChunkA);
       const uint32_t h0 = smem_u32(bhi), l0 = smem_u32(blo);
 #pragma unroll
       for (int s = 0; s < kUK / 16; ++s) {
         const uint64_t ad = umma_desc(a0 + 2 * s * kUChunkA, kUChunkA, 128);
-        umma_bf16(tmem, ad, umma_desc(h0 + 2 * s * kUChunkB, kUChunkB, 128), s > 0);
-        umma_bf16(tmem, ad, umma_desc(l0 + 2 * s * kUChunkB, kUChunkB, 128), true);
+        umma_bf16(acc, ad, umma_desc(h0 + 2 * s * kUChunkB, kUChunkB, 128), s > 0);
+        umma_bf16(acc, ad, umma_desc(l0 + 2 * s * kUChunkB, kUChunkB, 128), true);
       }
-      umma_commit(smem_u32(bar));
+      umma_commit(smem_u32(bar + b));
+    }
+  };
+  unsigned char* wst = stage + size_t(warp) * 32 * kUStageRow;   // this warp's staging rows
+  bool ok = true;
+  int issued = 0, j = 0;
+  if (J > 0) {
+    issue(0);
+    issued = 1;
+  }
+  for (; j < J; ++j) {
+    const int tile = slot + j * stride;
+    const int b = j & 1;
+    // the next tile's products run while this one is read back
+    if (j + 1 < J) {
+      issue(j + 1);
+      issued = j + 2;
     }
     // every thread leaves together if the commit never arrives
-    ok = __syncthreads_and(bounded_wait(smem_u32(bar), uint32_t(j) & 1u, kWaitPolls, abort_flag));
+    ok = __syncthreads_and(bounded_wait(smem_u32(bar + b), uint32_t(j >> 1) & 1u, kWaitPolls, abort_flag));
     if (!ok) break;
     tmem_fence_after();
     // A buffer b is free: the tile two ahead goes there
     load_tile(tile + 2 * stride, b);
-    const long long atom = (long long)tile * kUM + quarter * 32 + lane;
-    __nv_bfloat16* o = out + atom * kUN + colh * 128;
+    // read back 32 columns at a time: each lane its atom's row segment, as
+    // bf16 through the warp's staging rows, then stored as 8 rows x 64
+    // contiguous bytes per instruction
+    const long long row0 = (long long)tile * kUM + quarter * 32;
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
       uint32_t r[32];
-      tmem_ld32(tmem + (uint32_t(quarter * 32) << 16) + uint32_t(colh * 128 + c * 32), r);
+      tmem_ld32(tmem + uint32_t(b * kUN) + (uint32_t(quarter * 32) << 16) + uint32_t(colh * 128 + c * 32), r);
       tmem_ld_wait();
-      if (atom < p.n) {
-        uint4* o4 = reinterpret_cast<uint4*>(o + c * 32);
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          uint32_t wv[4];
+      for (int v = 0; v < 4; ++v) {
+        uint32_t wv[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 pr = __floats2bfloat162_rn(__uint_as_float(r[8 * v + 2 * e]),
-                                                            __uint_as_float(r[8 * v + 2 * e + 1]));
-            wv[e] = *reinterpret_cast<const uint32_t*>(&pr);
-          }
-          o4[v] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat162 pr = __floats2bfloat162_rn(__uint_as_float(r[8 * v + 2 * e]),
+                                                          __uint_as_float(r[8 * v + 2 * e + 1]));
+          wv[e] = *reinterpret_cast<const uint32_t*>(&pr);
         }
+        *reinterpret_cast<uint4*>(wst + lane * kUStageRow + v * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
       }
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int rr = i * 8 + (lane >> 2), seg = lane & 3;
+        const long long atom = row0 + rr;
+        const uint4 v4 = *reinterpret_cast<const uint4*>(wst + rr * kUStageRow + seg * 16);
+        if (atom < p.n)
+          *reinterpret_cast<uint4*>(out + atom * kUN + colh * 128 + c * 32 + seg * 8) = v4;
+      }
+      __syncwarp();   // the staging rows are rewritten by the next column block
     }
   }
   cp_async_wait<0>();
-  if (!ok && tid == 0) {
-    // the commit never arrived: a short, bounded chance for the products in
-    // flight to finish before their tensor memory is released
+  if (*abort_flag && tid == 0) {
+    // a wait gave up: a short, bounded chance for the products and weight
+    // copies in flight to finish before tensor and shared memory are released
     volatile int none = 0;
-    bounded_wait(smem_u32(bar), uint32_t(j) & 1u, kDrainPolls, &none);
+    for (int bb = 0; bb < 2; ++bb) {
+      int last = issued - 1;
+      while (last >= 0 && (last & 1) != bb) --last;
+      if (last >= 0) bounded_wait(smem_u32(bar + bb), uint32_t(last >> 1) & 1u, kDrainPolls, &none);
+    }
+    if (staged)
+      for (int half = 0; half < 2; ++half) bounded_wait(smem_u32(wbar), uint32_t(half), kDrainPolls, &none);
   }
   tmem_fence_before();
   __syncthreads();
