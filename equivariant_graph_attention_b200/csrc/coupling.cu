@@ -311,8 +311,8 @@ struct TileSmem {
   static constexpr size_t rows = 0;                                       // [2][16][ROWB]
   static constexpr size_t recs = rows + size_t(2) * kTileM * ROWB;        // [3][REC]
   static constexpr size_t sw = recs + size_t(3) * REC * 4;                // [P][C]
-  static constexpr size_t bars = sw + size_t(num_paths(L)) * C * 4;       // rows [2], records [3]
-  static constexpr size_t total = bars + 5 * 8 + 16;
+  static constexpr size_t bars = sw + size_t(num_paths(L)) * C * 4;       // rows [2], records [3], consumed [2]
+  static constexpr size_t total = bars + 7 * 8 + 16;
   static_assert(ROWB % 16 == 0 && REC % 4 == 0 && bars % 8 == 0, "bulk-copy alignment");
 };
 
@@ -334,7 +334,8 @@ eaas_tile_kernel(const __grid_constant__ EaasParams p) {
   float* sw = reinterpret_cast<float*>(smem + Sm::sw);
   uint64_t* rowbar = reinterpret_cast<uint64_t*>(smem + Sm::bars);   // [2] a tile's rows
   uint64_t* recbar = rowbar + 2;                                     // [3] a tile record
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(recbar + 3);
+  uint64_t* donebar = recbar + 3;                                    // [2] every warp done with a tile
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(donebar + 2);
 
   const int tid = threadIdx.x, lane = tid & 31, wfirst = tid >> 5;
   const int tiles = int(p.items / kTileM);
@@ -342,6 +343,7 @@ eaas_tile_kernel(const __grid_constant__ EaasParams p) {
   if (blockIdx.x >= tiles) return;   // whole CTA
   if (tid == 0) {
     for (int b = 0; b < 5; ++b) mbar_init(smem_u32(rowbar + b), 1);
+    for (int b = 0; b < 2; ++b) mbar_init(smem_u32(donebar + b), kHalfWarps);
     mbar_fence_init();
     *abort_flag = 0;
   }
@@ -385,8 +387,10 @@ eaas_tile_kernel(const __grid_constant__ EaasParams p) {
     if (wfirst == 0 && tile + grid < tiles) {
       // warp 0: the next tile's rows (its record arrived a tile ago), one
       // bulk copy per lane after lane 0 has announced their bytes, and the
-      // record after it; both buffers were last read by tile j - 1, before
-      // the barrier that ended it
+      // record after it; both buffers were last read by tile j - 1, which
+      // every warp has signalled done on donebar[(j - 1) & 1]
+      if (j >= 1)
+        bounded_wait(smem_u32(donebar + ((j + 1) & 1)), uint32_t((j - 1) >> 1) & 1u, kWaitPolls, abort_flag);
       const int nb = (j + 1) % 3;
       bounded_wait(smem_u32(recbar + nb), uint32_t((j + 1) / 3) & 1u, kWaitPolls, abort_flag);
       const int* tg = reinterpret_cast<const int*>(recs + nb * REC) + kRecTgt;
@@ -428,7 +432,11 @@ eaas_tile_kernel(const __grid_constant__ EaasParams p) {
       }
     }
     }
-    __syncthreads();   // rows[wb] and recs[rb] are refilled one and two tiles ahead
+    // this warp is done with rows[wb] and recs[rb]: warp 0 refills them one
+    // and two tiles ahead once every warp has said so (no block barrier, so
+    // a warp that finishes early starts the next tile)
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(donebar + wb));
   }
   if (*abort_flag && tid == 0) {
     // a wait gave up: give every barrier's last phase a short, bounded chance

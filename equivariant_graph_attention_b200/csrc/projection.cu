@@ -17,8 +17,10 @@
 //    float32 weights to about 2^-17, and h is exactly bf16.  The float32
 //    matrix arrives in two 64 KB bulk copies (cp.async.bulk, no multicast)
 //    and is converted from shared memory;
-//  * per 128-atom tile the degree-0 slices (256 bytes per atom) arrive by
-//    16-byte cp.async copies, two tiles in flight, and one thread issues
+//  * per 128-atom tile the degree-0 slices (256 bytes per atom) arrive by two
+//    TMA tensor copies (cp.async.bulk.tensor.2d, 64 channels x 128 atoms
+//    each, 128-byte swizzle, rows past n zero-filled; no multicast) on the
+//    buffer's mbarrier, two tiles in flight, and one thread issues
 //    sixteen 128 x 256 x 16 products (h W_hi and h W_lo per 16-channel step)
 //    into one of two 256-column float32 accumulators in tensor memory,
 //    completing that accumulator's mbarrier; tile j + 1's products run while
@@ -33,7 +35,11 @@
 // Other shapes (float32 storage, other C or H*dk) take a plain kernel: a CTA
 // stages the degree-0 channels of 8 atoms and each thread forms output
 // columns as float32 dot products over C, reading the weights from L2.
+#include <cuda.h>
 #include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
 
 #include "egat_async.cuh"
 #include "egat_host.h"
@@ -42,6 +48,7 @@ namespace egat {
 namespace {
 
 struct ProjParams {
+  CUtensorMap amap;       // h's degree-0 slices as a [n][C] bf16 matrix (row pitch D * C * 2 bytes)
   const __nv_bfloat16* h;
   const float* w[2];      // wq, wk  [C][H*dk]
   __nv_bfloat16* out[2];  // q, k    [n][H*dk]
@@ -62,7 +69,11 @@ struct ProjParams {
 //    them to an mbarrier;
 //  * eight warps read the accumulator back (tcgen05.ld, each warp its
 //    32-lane quarter and half of the columns), round to bf16 and store.
-// Shared-memory operands use the K-major no-swizzle canonical layout: 8-row
+// Shared-memory operands, both K-major: A (the atoms' channels) in the
+// 128-byte-swizzled layout the tensor copy writes (per 64-channel half, 128
+// rows of 128 bytes, 16-byte chunks permuted by row % 8; 8-row groups 1 KB
+// apart; a 16-channel k-step starts 32 bytes further along the row); B (the
+// weights, written by this kernel) in the no-swizzle canonical layout: 8-row
 // x 16-byte core matrices of 128 contiguous bytes, 8-row groups 128 bytes
 // apart (SBO), the two 8-channel halves of a k-step one channel chunk apart
 // (LBO).
@@ -70,7 +81,7 @@ constexpr int kUM = 128;                 // atoms per tile (M)
 constexpr int kUN = 256;                 // outputs per matrix (N)
 constexpr int kUK = 128;                 // channels (K)
 constexpr int kUWarps = 8;
-constexpr int kUChunkA = kUM * 16;       // bytes per 8-channel chunk of an A tile
+constexpr int kUHalfA = kUM * 128;       // bytes per 64-channel half of an A tile (swizzled rows)
 constexpr int kUChunkB = kUN * 16;       // bytes per 8-channel chunk of a B tile
 constexpr int kUCols = 512;              // tensor-memory columns: two float32 accumulators of N = 256
 constexpr int kUStageRow = 80;           // a staged 64-byte output row segment, padded (bank spread)
@@ -78,13 +89,13 @@ constexpr int kUStageRow = 80;           // a staged 64-byte output row segment,
 struct UmmaSmem {
   static constexpr size_t bhi = 0;                                      // [16][32][8][16 B]
   static constexpr size_t blo = bhi + size_t(kUK / 8) * kUChunkB;
-  static constexpr size_t a = blo + size_t(kUK / 8) * kUChunkB;         // [2][16][16][8][16 B]
-  static constexpr size_t stage = a + 2 * size_t(kUK / 8) * kUChunkA;   // [8 warps][32 rows][80 B]
-  static constexpr size_t bars = stage + size_t(kUWarps) * 32 * kUStageRow;  // products [2], weight halves
-  static constexpr size_t tslot = bars + 24;                             // tensor-memory address
+  static constexpr size_t a = blo + size_t(kUK / 8) * kUChunkB;         // [2][2 halves][128][128 B]
+  static constexpr size_t stage = a + 2 * size_t(2) * kUHalfA;          // [8 warps][32 rows][80 B]
+  static constexpr size_t bars = stage + size_t(kUWarps) * 32 * kUStageRow;  // products [2], A [2], weights
+  static constexpr size_t tslot = bars + 40;                             // tensor-memory address
   static constexpr size_t flag = tslot + 4;                              // abort flag
   static constexpr size_t total = flag + 4 + 16;
-  static_assert(a % 1024 == 0 && bars % 8 == 0, "operand alignment");
+  static_assert(a % 1024 == 0 && kUHalfA % 1024 == 0 && bars % 8 == 0, "operand alignment");
 };
 
 // Shared-memory matrix descriptor: start, leading and stride byte offsets
@@ -92,6 +103,18 @@ struct UmmaSmem {
 __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return uint64_t((saddr >> 4) & 0x3FFFu) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) |
          (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (uint64_t(1) << 46);
+}
+// the same for a 128-byte-swizzled K-major operand (layout type 2): 8-row
+// groups 1 KB apart, the leading offset unused (16 bytes)
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  return umma_desc(saddr, 16, 1024) | (uint64_t(2) << 61);
+}
+// 2-D tensor copy of box {x, y} of the map into shared memory, completing bar
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
 }
 // Instruction descriptor, kind::f16: float32 accumulator, bf16 A and B, both
 // K-major, N = 256, M = 128.
@@ -129,23 +152,14 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
-}
-
 __global__ void __launch_bounds__(kUWarps * 32, 1) qk_projection_umma_kernel(const __grid_constant__ ProjParams p) {
   extern __shared__ __align__(1024) unsigned char smem[];
   unsigned char* bhi = smem + UmmaSmem::bhi;
   unsigned char* blo = smem + UmmaSmem::blo;
   unsigned char* abuf = smem + UmmaSmem::a;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + UmmaSmem::bars);        // [2] products per accumulator
-  uint64_t* wbar = bar + 2;                                                   // a weight half
+  uint64_t* abar = bar + 2;                                                   // [2] an A buffer's copies
+  uint64_t* wbar = bar + 4;                                                   // a weight half
   unsigned char* stage = smem + UmmaSmem::stage;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + UmmaSmem::tslot);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + UmmaSmem::flag);
@@ -157,9 +171,7 @@ __global__ void __launch_bounds__(kUWarps * 32, 1) qk_projection_umma_kernel(con
   if (slot >= p.tiles) return;               // whole CTA
 
   if (tid == 0) {
-    mbar_init(smem_u32(bar), 1);
-    mbar_init(smem_u32(bar + 1), 1);
-    mbar_init(smem_u32(wbar), 1);
+    for (int b = 0; b < 5; ++b) mbar_init(smem_u32(bar + b), 1);
     mbar_fence_init();
     *abort_flag = 0;
   }
@@ -171,26 +183,19 @@ __global__ void __launch_bounds__(kUWarps * 32, 1) qk_projection_umma_kernel(con
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
 
-  const char* hb = reinterpret_cast<const char*>(p.h);
-  const long long row_bytes = p.row_elems * 2;
-  // the degree-0 slices of tile tl into A buffer b: 16-byte chunk (atom m,
-  // channels 8c .. 8c+7) at c * kUChunkA + (m / 8) * 128 + (m % 8) * 16;
-  // rows past n are zero-filled
-  auto load_tile = [&](int tl, int b) {
-    if (tl < p.tiles) {
-      const uint32_t base = smem_u32(abuf + size_t(b) * (kUK / 8) * kUChunkA);
-      // a warp moves 8 atoms x 4 chunks: 128 contiguous bytes of shared
-      // memory per chunk, 64 contiguous bytes of global memory per atom
-      for (int e = tid; e < kUM * (kUK / 8); e += kUWarps * 32) {
-        const int wi = e >> 5, ln = e & 31;
-        const int m = (wi & 15) * 8 + (ln & 7), c = (wi >> 4) * 4 + (ln >> 3);
-        const long long atom = (long long)tl * kUM + m;
-        const bool ok = atom < p.n;
-        const char* src = hb + (ok ? atom * row_bytes + c * 16 : 0);
-        cp_async16(base + c * kUChunkA + (m >> 3) * 128 + (m & 7) * 16, src, ok ? 16u : 0u);
-      }
+  // thread 0: tile tl's degree-0 slices into A buffer b, two 64-channel
+  // halves of 128 rows (rows past n arrive as zeros)
+  int loaded = 0;   // tiles whose copies were issued (this CTA's sequence numbers)
+  auto load_tile = [&](int jj, int b) {
+    const int tl = slot + jj * stride;
+    if (tid == 0 && tl < p.tiles) {
+      const uint32_t ab = smem_u32(abar + b);
+      const uint32_t dst = smem_u32(abuf + size_t(b) * 2 * kUHalfA);
+      mbar_arrive_expect_tx(ab, 2u * kUHalfA);
+      tma_load_2d(dst, &p.amap, 0, tl * kUM, ab);
+      tma_load_2d(dst + kUHalfA, &p.amap, 64, tl * kUM, ab);
     }
-    cp_async_commit();   // one group per tile slot, empty past the last tile
+    if (tl < p.tiles) loaded = jj + 1;
   };
   // weights: float32 [k][n] -> bf16 hi / lo at (k / 8) * kUChunkB +
   // (n / 8) * 128 + (n % 8) * 16 + (k % 8) * 2, stored as (k, k + 1) pairs.
@@ -211,7 +216,7 @@ __global__ void __launch_bounds__(kUWarps * 32, 1) qk_projection_umma_kernel(con
     // float32 each) into the A buffers, which are free until the first tile
     const float* stage = reinterpret_cast<const float*>(abuf);
     constexpr int kRows = kUK / 2;
-    static_assert(size_t(kRows) * kUN * 4 <= 2 * size_t(kUK / 8) * kUChunkA, "a weight half fits the A buffers");
+    static_assert(size_t(kRows) * kUN * 4 <= 2 * size_t(2) * kUHalfA, "a weight half fits the A buffers");
 #pragma unroll 1
     for (int half = 0; half < 2; ++half) {
       if (tid == 0) {
@@ -249,8 +254,10 @@ __global__ void __launch_bounds__(kUWarps * 32, 1) qk_projection_umma_kernel(con
       }
     }
   }
-  load_tile(slot, 0);
-  load_tile(slot + stride, 1);
+  fence_proxy_async_smem();   // the staged weights were read before the tensor copies overwrite them
+  __syncthreads();
+  load_tile(0, 0);
+  load_tile(1, 1);
   fence_proxy_async_smem();   // the weight tiles are read by the tensor core
   tmem_fence_before();
   __syncthreads();
@@ -264,19 +271,18 @@ __global__ void __launch_bounds__(kUWarps * 32, 1) qk_projection_umma_kernel(con
   // 256 (jj % 2) ..), completing mbarrier jj % 2; every thread takes part
   // (the wait for the tile's copies and the barrier before the issue)
   auto issue = [&](int jj) {
-    cp_async_wait<0>();          // the tile's copies (every older group too)
-    fence_proxy_async_smem();    // its bytes are read by the tensor core
     tmem_fence_before();         // the accumulator's previous reads are done
     __syncthreads();
     if (tid == 0) {
-      tmem_fence_after();
       const int b = jj & 1;
+      bounded_wait(smem_u32(abar + b), uint32_t(jj >> 1) & 1u, kWaitPolls, abort_flag);   // the tile's copies
+      tmem_fence_after();
       const uint32_t acc = tmem + uint32_t(b * kUN);
-      const uint32_t a0 = smem_u32(abuf + size_t(b) * (kUK / 8) * kUChunkA);
+      const uint32_t a0 = smem_u32(abuf + size_t(b) * 2 * kUHalfA);
       const uint32_t h0 = smem_u32(bhi), l0 = smem_u32(blo);
 #pragma unroll
       for (int s = 0; s < kUK / 16; ++s) {
-        const uint64_t ad = umma_desc(a0 + 2 * s * kUChunkA, kUChunkA, 128);
+        const uint64_t ad = umma_desc_sw128(a0 + (s >> 2) * kUHalfA + (s & 3) * 32);
         umma_bf16(acc, ad, umma_desc(h0 + 2 * s * kUChunkB, kUChunkB, 128), s > 0);
         umma_bf16(acc, ad, umma_desc(l0 + 2 * s * kUChunkB, kUChunkB, 128), true);
       }
@@ -303,7 +309,7 @@ __global__ void __launch_bounds__(kUWarps * 32, 1) qk_projection_umma_kernel(con
     if (!ok) break;
     tmem_fence_after();
     // A buffer b is free: the tile two ahead goes there
-    load_tile(tile + 2 * stride, b);
+    load_tile(j + 2, b);
     // read back 32 columns at a time: each lane its atom's row segment, as
     // bf16 through the warp's staging rows, then stored as 8 rows x 64
     // contiguous bytes per instruction
@@ -336,15 +342,18 @@ __global__ void __launch_bounds__(kUWarps * 32, 1) qk_projection_umma_kernel(con
       __syncwarp();   // the staging rows are rewritten by the next column block
     }
   }
-  cp_async_wait<0>();
   if (*abort_flag && tid == 0) {
-    // a wait gave up: a short, bounded chance for the products and weight
-    // copies in flight to finish before tensor and shared memory are released
+    // a wait gave up: a short, bounded chance for the products, tile copies
+    // and weight copies in flight to finish before tensor and shared memory
+    // are released
     volatile int none = 0;
     for (int bb = 0; bb < 2; ++bb) {
       int last = issued - 1;
       while (last >= 0 && (last & 1) != bb) --last;
       if (last >= 0) bounded_wait(smem_u32(bar + bb), uint32_t(last >> 1) & 1u, kDrainPolls, &none);
+      last = loaded - 1;
+      while (last >= 0 && (last & 1) != bb) --last;
+      if (last >= 0) bounded_wait(smem_u32(abar + bb), uint32_t(last >> 1) & 1u, kDrainPolls, &none);
     }
     if (staged)
       for (int half = 0; half < 2; ++half) bounded_wait(smem_u32(wbar), uint32_t(half), kDrainPolls, &none);
@@ -403,6 +412,31 @@ __global__ void __launch_bounds__(256) qk_projection_kernel(const T* __restrict_
 
 }  // namespace
 
+// The tensor map of h's degree-0 slices: a [n][C] bf16 matrix whose rows lie
+// D * C * 2 bytes apart, read in boxes of 64 channels x 128 atoms with the
+// 128-byte swizzle (the A operand layout of qk_projection_umma_kernel).  The
+// encoder comes from the driver through the runtime's entry-point query.
+int encode_degree0_map(CUtensorMap* map, const void* d_h, int n, long long row_elems) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!encode) return -1;
+  const cuuint64_t dims[2] = {cuuint64_t(kUK), cuuint64_t(n)};
+  const cuuint64_t strides[1] = {cuuint64_t(row_elems) * 2};
+  const cuuint32_t box[2] = {64, cuuint32_t(kUM)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(d_h), dims, strides, box,
+                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -1;
+}
+
 bool projection_tc_supported(const egat_shape& s) {
   return s.dtype == EGAT_BF16 && s.C == kUK && s.H * s.dk == kUN;
 }
@@ -413,6 +447,7 @@ int launch_qk_projection(const egat_shape& s, const void* d_h, const float* d_wq
   const int HD = s.H * s.dk;
   if (projection_tc_supported(s)) {
     ProjParams p;
+    if (encode_degree0_map(&p.amap, d_h, s.n, row_elems) != 0) return EGAT_ERR_CUDA;
     p.h = static_cast<const __nv_bfloat16*>(d_h);
     p.w[0] = d_wq;
     p.w[1] = d_wk;
