@@ -79,6 +79,8 @@ adjoint_coupling_kernel(const float* __restrict__ g, const float* __restrict__ p
   for (int l = 1; l <= L; ++l) rpow[l] = rpow[l - 1] * r;
   wigner_build<L>(Q, Dsm[wib], lane, 32, [] { __syncwarp(); });
   __syncwarp();
+  // two channels per lane in flight: twice the row loads outstanding per warp
+#pragma unroll 2
   for (int c = lane; c < C; c += 32) {
     float x[D];
 #pragma unroll
@@ -976,9 +978,11 @@ int launch_backward_tiled(const egat_shape& s, const BwdWs& w, const void* d_h, 
                           float* d_dk, float* d_dpos, cudaStream_t st) {
   float* hp = static_cast<float*>(w.hp);
   float* dm = static_cast<float*>(w.dm);
-  int e = launch_eaas_source_f32out(s, d_h, d_pos, d_w1, hp, st, true);
+  // the forward plan first: its tile records give the source coupling its
+  // rotations (the tile-staged kernel), then dL/dm
+  int e = launch_build_plan(s.n, s.K, s.lmax, d_nbr, d_cnt, d_order, d_pos, w.tc.plan, st);
+  if (e == EGAT_OK) e = launch_eaas_planned_tf32out(s, d_h, w.tc.plan, d_w1, hp, st);
   if (e == EGAT_OK) e = launch_adjoint<L, float>(s, d_g, d_pos, d_w2, dm, st);
-  if (e == EGAT_OK) e = launch_build_plan(s.n, s.K, s.lmax, d_nbr, d_cnt, d_order, d_pos, w.tc.plan, st);
   if (e != EGAT_OK) return e;
   // in-lists (unsorted: the source plan's union is ordered by its bitmap)
   if (cudaMemsetAsync(w.deg, 0, size_t(s.n) * 4, st) != cudaSuccess ||

@@ -320,7 +320,7 @@ struct TileSmem {
 // overlaps the other's work (one CTA per SM at lmax 3, whose rows fill the
 // shared memory)
 constexpr int kHalfWarps = kTileM / 2;
-template <int L, typename T>
+template <int L, typename T, typename TO = T>
 __global__ void __launch_bounds__(kHalfWarps * 32, L >= 3 ? 1 : 2)
 eaas_tile_kernel(const __grid_constant__ EaasParams p) {
   using Sm = TileSmem<L, T>;
@@ -351,7 +351,7 @@ eaas_tile_kernel(const __grid_constant__ EaasParams p) {
   __syncthreads();
 
   const char* xb = static_cast<const char*>(p.x);
-  T* __restrict__ y = static_cast<T*>(p.y);
+  TO* __restrict__ y = static_cast<TO*>(p.y);
   // thread 0: a tile's record into recs[b]
   auto issue_rec = [&](int tl, int b) {
     const uint32_t bar = smem_u32(recbar + b);
@@ -424,11 +424,11 @@ eaas_tile_kernel(const __grid_constant__ EaasParams p) {
 #pragma unroll
           for (int k = 0; k < CPL; ++k) xv[k][d] = v[k];
         }
-        T* yr = y + (size_t)at * D * C + c0;
+        TO* yr = y + (size_t)at * D * C + c0;
         const float* swc = sw + c0;
         eaas_multi<L, CPL, (CPL >= 4)>(xv, rec + rec_off_D(L) + w * WS, rpow, p.tab,
                            [&](int q, int k) { return swc[q * C + k]; },
-                           [&](int d, const float (&v)[CPL]) { ChanVec<T, CPL>::store(yr + d * C, v); });
+                           [&](int d, const float (&v)[CPL]) { ChanVec<TO, CPL>::store(yr + d * C, v); });
       }
     }
     }
@@ -499,7 +499,7 @@ int launch_eaas_source(const egat_shape& s, const void* d_x, const float* d_pos,
   }
 }
 
-template <int L, typename T>
+template <int L, typename T, typename TO = T>
 int launch_eaas_tile(const egat_shape& s, const void* d_x, const float* rec, long long items,
                      const float* d_w, void* d_y, cudaStream_t st) {
   EaasParams p;
@@ -513,7 +513,7 @@ int launch_eaas_tile(const egat_shape& s, const void* d_x, const float* rec, lon
   p.items = items;
   p.tab = eaas_table(L);
   constexpr size_t shmem = TileSmem<L, T>::total;
-  auto kern = eaas_tile_kernel<L, T>;
+  auto kern = eaas_tile_kernel<L, T, TO>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(shmem)) !=
       cudaSuccess)
     return EGAT_ERR_CUDA;
@@ -578,6 +578,19 @@ int launch_eaas_planned(const egat_shape& s, const void* d_x, const void* d_plan
                       : launch_eaas_t<2, float, true>(s, d_x, nullptr, pv.rec, items, d_w, d_y, st);
     case 3: return bf ? launch_eaas_t<3, __nv_bfloat16, true>(s, d_x, nullptr, pv.rec, items, d_w, d_y, st)
                       : launch_eaas_t<3, float, true>(s, d_x, nullptr, pv.rec, items, d_w, d_y, st);
+    default: return EGAT_ERR_UNSUPPORTED;
+  }
+}
+
+int launch_eaas_planned_tf32out(const egat_shape& s, const void* d_x, const void* d_plan, const float* d_w,
+                                float* d_y, cudaStream_t st) {
+  if (s.dtype != EGAT_BF16 || s.C != 128) return EGAT_ERR_UNSUPPORTED;
+  const PlanView pv = plan_view(const_cast<void*>(d_plan), s.n, s.K, s.lmax);
+  const long long items = (long long)pv.tiles * kTileM;
+  switch (s.lmax) {
+    case 1: return launch_eaas_tile<1, __nv_bfloat16, Tf32Out>(s, d_x, pv.rec, items, d_w, d_y, st);
+    case 2: return launch_eaas_tile<2, __nv_bfloat16, Tf32Out>(s, d_x, pv.rec, items, d_w, d_y, st);
+    case 3: return launch_eaas_tile<3, __nv_bfloat16, Tf32Out>(s, d_x, pv.rec, items, d_w, d_y, st);
     default: return EGAT_ERR_UNSUPPORTED;
   }
 }

@@ -77,12 +77,16 @@ int launch_build_plan(int n, int K, int lmax, const int32_t* d_nbr, const int32_
                       const int32_t* d_order, const float* d_pos, void* d_plan, cudaStream_t st);
 // Step 2 with a float32 result whatever the storage type (the backward pass
 // keeps its intermediates in float32); tf32 = true rounds the stored values
-// to tf32 (lmax <= 2).
+// to tf32.
 int launch_eaas_source_f32out(const egat_shape& s, const void* d_x, const float* d_pos,
                               const float* d_w, float* d_y, cudaStream_t st, bool tf32 = false);
 // Step 2 for every atom listed in a plan's tile records, rotations from them.
 int launch_eaas_planned(const egat_shape& s, const void* d_x, const void* d_plan, const float* d_w,
                         void* d_y, cudaStream_t st);
+// The same for bf16 features with C = 128, the result float32 rounded to tf32
+// (the backward's operand format).
+int launch_eaas_planned_tf32out(const egat_shape& s, const void* d_x, const void* d_plan, const float* d_w,
+                                float* d_y, cudaStream_t st);
 // Tiled tensor-core attention (bf16 storage, C/H = 8, dk = 16): fused = true
 // applies the target coupling and writes ^h; false writes m.
 bool tc_attention_supported(const egat_shape& s);
