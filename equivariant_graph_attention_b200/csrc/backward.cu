@@ -79,8 +79,42 @@ adjoint_coupling_kernel(const float* __restrict__ g, const float* __restrict__ p
   for (int l = 1; l <= L; ++l) rpow[l] = rpow[l - 1] * r;
   wigner_build<L>(Q, Dsm[wib], lane, 32, [] { __syncwarp(); });
   __syncwarp();
-  // two channels per lane in flight: twice the row loads outstanding per warp
-#pragma unroll 2
+  for (int c = lane; c < C; c += 32) {
+    float x[D];
+#pragma unroll
+    for (int d = 0; d < D; ++d) x[d] = g[((size_t)a * D + d) * C + c];
+    eaas_channel_adjoint<L>(x, Dsm[wib], rpow, tab, [&](int pp) { return __ldg(w + pp * C + c); },
+                            [&](int d, float v) {
+                              store_one<T>(out + ((size_t)a * D + d) * C + c, TF32 ? round_tf32(v) : v);
+                            });
+  }
+}
+
+// The same operator with each atom's rotation and |r|^l taken from the
+// attention plan's tile records instead of built per atom: one warp per tile
+// slot copies the slot's Wigner-D into its shared memory.
+template <int L, typename T, bool TF32 = false>
+__global__ void __launch_bounds__(kBwdWarps * 32)
+adjoint_planned_kernel(const float* __restrict__ g, const float* __restrict__ rec, long long items,
+                       const float* __restrict__ w, T* __restrict__ out, int n, int C,
+                       const __grid_constant__ EaasTable tab) {
+  constexpr int D = (L + 1) * (L + 1);
+  constexpr int WS = wig_size(L);
+  constexpr int REC = plan_record_words(L);
+  static_assert(WS == rec_wig_size(L), "record and shared-memory Wigner-D layouts agree");
+  __shared__ float Dsm[kBwdWarps][WS];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const long long slot = (long long)blockIdx.x * kBwdWarps + wib;
+  if (slot >= items) return;   // whole warp
+  const float* rc = rec + (slot / kTileM) * REC;
+  const int r = int(slot % kTileM);
+  const int a = reinterpret_cast<const int*>(rc)[kRecTgt + r];
+  if ((unsigned)a >= (unsigned)n) return;   // an empty slot of the last tile
+  for (int e = lane; e < WS; e += 32) Dsm[wib][e] = __ldg(rc + rec_off_D(L) + r * WS + e);
+  float rpow[L + 1];
+#pragma unroll
+  for (int l = 0; l <= L; ++l) rpow[l] = __ldg(rc + kRecRp + r * (L + 1) + l);
+  __syncwarp();
   for (int c = lane; c < C; c += 32) {
     float x[D];
 #pragma unroll
@@ -839,6 +873,17 @@ int launch_adjoint(const egat_shape& s, const float* g, const float* pos, const 
   return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
 }
 
+template <int L, typename T, bool TF32 = false>
+int launch_adjoint_planned(const egat_shape& s, const float* g, const void* plan, const float* w, void* out,
+                           cudaStream_t st) {
+  const PlanView pv = plan_view(const_cast<void*>(plan), s.n, s.K, s.lmax);
+  const long long items = (long long)pv.tiles * kTileM;
+  const long long grid = (items + kBwdWarps - 1) / kBwdWarps;
+  adjoint_planned_kernel<L, T, TF32><<<unsigned(grid), kBwdWarps * 32, 0, st>>>(
+      g, pv.rec, items, w, static_cast<T*>(out), s.n, s.C, eaas_table(L));
+  return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
+}
+
 size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // host, double precision: the Ivanic–Ruedenberg recursion of wigner_build,
@@ -982,7 +1027,7 @@ int launch_backward_tiled(const egat_shape& s, const BwdWs& w, const void* d_h, 
   // rotations (the tile-staged kernel), then dL/dm
   int e = launch_build_plan(s.n, s.K, s.lmax, d_nbr, d_cnt, d_order, d_pos, w.tc.plan, st);
   if (e == EGAT_OK) e = launch_eaas_planned_tf32out(s, d_h, w.tc.plan, d_w1, hp, st);
-  if (e == EGAT_OK) e = launch_adjoint<L, float>(s, d_g, d_pos, d_w2, dm, st);
+  if (e == EGAT_OK) e = launch_adjoint_planned<L, float>(s, d_g, w.tc.plan, d_w2, dm, st);
   if (e != EGAT_OK) return e;
   // in-lists (unsorted: the source plan's union is ordered by its bitmap)
   if (cudaMemsetAsync(w.deg, 0, size_t(s.n) * 4, st) != cudaSuccess ||
@@ -996,7 +1041,7 @@ int launch_backward_tiled(const egat_shape& s, const BwdWs& w, const void* d_h, 
   if (cudaGetLastError() != cudaSuccess) return EGAT_ERR_CUDA;
   e = launch_backward_tc(s, w.tc, d_q, d_k, hp, dm, d_order, w.ptr, w.in, d_dq, d_dk, d_dpos != nullptr,
                          st);
-  if (e == EGAT_OK) e = launch_adjoint<L, float>(s, w.tc.dhp, d_pos, d_w1, d_dh, st);
+  if (e == EGAT_OK) e = launch_adjoint_planned<L, float>(s, w.tc.dhp, w.tc.plan, d_w1, d_dh, st);
   if (e != EGAT_OK || !d_dpos) return e;
   PosGradParams pg;
   pg.g = d_g;
