@@ -601,15 +601,16 @@ __device__ __forceinline__ void coupling_grad_channel(float (&g)[(L + 1) * (L + 
   }
   dr += reindex_dot(g, x, drpow);
   // <J_b g~, Rw x~> = <Rw^T J_b g~, x~> = reindex_dot(J_b g~, x~); <g~, Rw J_b x~> = reindex_dot(g~, J_b x~)
-  static_for<0, 2>([&](auto bc) {
-    constexpr int bax = decltype(bc)::value;
+#pragma unroll 1
+  for (int bax = 0; bax < 2; ++bax) {
     float jv[D];
     gen_apply(bax, g, jv);
     float s = reindex_dot(jv, x, rpow);
     gen_apply(bax, x, jv);
     s += reindex_dot(g, jv, rpow);
-    if constexpr (bax == 0) tx += s; else ty += s;
-  });
+    tx += bax == 0 ? s : 0.f;
+    ty += bax == 1 ? s : 0.f;
+  }
 }
 
 // eaas_multi on channel pairs: the same operations in the same order per
