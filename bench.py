@@ -62,19 +62,24 @@ DEFAULT_WORKLOAD = "uniform32768_K256_l2_bf16"
 EXTRA_WORKLOADS = ["uniform4096_l2_bf16", "uniform100000_l3_bf16"]
 FLUSH_BYTES = 256 << 20
 #: kernels this library launches per step: graph (assign, scan x3, scatter,
-#: rank, fill, truncated-row fix) + attention plan (tensor-core shapes: unions
-#: and masks, tile records) + source coupling + fused attention
+#: rank, fill, truncated-row fix) + attention plan (tensor-core shapes: unions,
+#: masks and tile records in one kernel; a second for the records at lmax 3)
+#: + source coupling + fused attention
 LAUNCHES_GRAPH = 8
-LAUNCHES_PLAN = 2
+
+
+def launches_plan(lmax: int) -> int:
+    return 1 if lmax <= 2 else 2
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attention_traffic.json")
 KERNEL_SOURCES = ["equivariant_graph_attention_b200/csrc/attention.cu",
                   "equivariant_graph_attention_b200/csrc/attention_tc.cu",
                   "equivariant_graph_attention_b200/csrc/plan.cu",
                   "equivariant_graph_attention_b200/csrc/egat_device.cuh",
                   "equivariant_graph_attention_b200/csrc/egat_async.cuh"]
-#: library kernels per decomposed step and rank: three row gathers (own h, q, k),
-#: the source coupling, two send-buffer gathers, the plan (2) and the attention
-DECOMP_LAUNCHES = 9
+#: library kernels per decomposed step and rank besides the plan: three row
+#: gathers (own h, q, k), the source coupling, two send-buffer gathers and the
+#: attention
+DECOMP_LAUNCHES = 7
 #: oracle worker processes at most (each holds its own copy of a few hundred MB)
 MAX_ORACLE_WORKERS = 32
 
@@ -385,7 +390,7 @@ class ForwardStep:
             raise SystemExit("the tensor-core attention path does not support this workload")
         self.plan = torch.empty(max(plan_sz.value, 16), dtype=torch.uint8, device=dev)
         self.attn_name = "otf_attention_tiled" if self.tiled else "otf_attention_coupled"
-        self.launches = LAUNCHES_GRAPH + (LAUNCHES_PLAN if self.tiled else 0) + 2
+        self.launches = LAUNCHES_GRAPH + (launches_plan(wl.lmax) if self.tiled else 0) + 2
 
     def graph(self):
         e, w = self.egat, self.wl
@@ -671,7 +676,7 @@ def run_decomposed(args, wl: synth.Workload):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                     "what": "each rank: its rows of h, q, k and the positions in, its output rows "
                             "out, every step", "matches_device_result": e2e_ok},
-            "gpu_launches": DECOMP_LAUNCHES * args.steps,
+            "gpu_launches": (DECOMP_LAUNCHES + launches_plan(wl.lmax)) * args.steps,
             "roofline": None,
             "roofline_note": "per-kernel rooflines are reported by the single-system line",
             "decomposition": {"owned_per_rank": int(plan.n_owned), "halo_atoms_max": int(halo_max),

@@ -11,10 +11,13 @@
 // One 256-thread CTA per tile builds the union from a shared-memory bitmap
 // over atom indices (ascending atom index: a deterministic order) and sets one
 // mask bit per (target, neighbour) at the position given by the bitmap's
-// prefix counts.  A second kernel writes each tile's target record: target
+// prefix counts.  The same CTA then writes the tile's target record: target
 // ids, |r|^l and the real Wigner-D matrices of the targets' alignment
 // rotations ([EX] §2.1), which the target coupling of the attention epilogue
-// applies.
+// applies (one thread per target slot, after the union and mask; at lmax 3 a
+// separate kernel writes the slots).
+#include <type_traits>
+
 #include "egat_device.cuh"
 #include "egat_host.h"
 
@@ -24,12 +27,39 @@ namespace {
 constexpr int kPlanThreads = 256;
 
 struct PlanParams {
+  const float* pos;      // [n][3] (the tile records' rotations)
   const int32_t* nbr;    // [n][K]
   const int32_t* cnt;    // [n] or null (then every slot is scanned, -1 skipped)
   const int32_t* order;  // [n] or null
   PlanView plan;
   int n, K;
 };
+
+// The record entries of target slot r of a tile: the slot's atom (-1 for an
+// empty slot), |r|^l and the Wigner-D matrices of its alignment rotation
+// (identity for an empty slot or an atom at the origin), built in registers.
+// The header (union length, three zeros) is written by the caller.
+template <int L>
+__device__ __forceinline__ void write_slot_record(int tg, const float* __restrict__ pos, int r,
+                                                  float* __restrict__ R) {
+  constexpr int WS = wig_size(L);
+  static_assert(WS == rec_wig_size(L) && plan_record_words(L) % 4 == 0, "record layout");
+  float Q[9];
+  float rr = 0.f;
+  if (tg >= 0) rr = alignment_rotation(pos[3 * tg], pos[3 * tg + 1], pos[3 * tg + 2], Q);
+  else alignment_rotation(0.f, 0.f, 0.f, Q);
+  float D[WS];
+  wigner_regs<L>(Q, D);
+#pragma unroll
+  for (int e = 0; e < WS; ++e) R[rec_off_D(L) + r * WS + e] = D[e];
+  reinterpret_cast<int*>(R)[kRecTgt + r] = tg;
+  float a = 1.f;
+#pragma unroll
+  for (int l = 0; l <= L; ++l) {
+    R[kRecRp + r * (L + 1) + l] = a;
+    a *= rr;
+  }
+}
 
 // One CTA per tile.  Shared memory holds a bitmap over all atom indices
 // (bit j set when atom j is a neighbour of some target of the tile), the
@@ -40,6 +70,7 @@ struct PlanParams {
 //     prefix[j / 32] + popcount(bits of word j / 32 below j);
 //  3. one membership bit per (target, neighbour) at that position.
 // Cost per tile is O(n / 32) words plus O(16 K) entries; deterministic.
+template <int L, bool RECORDS>
 __global__ void __launch_bounds__(kPlanThreads) build_plan_kernel(const __grid_constant__ PlanParams p) {
   extern __shared__ uint32_t sm[];
   const PlanView& pv = p.plan;
@@ -145,6 +176,13 @@ __global__ void __launch_bounds__(kPlanThreads) build_plan_kernel(const __grid_c
     const int w = i / kTileM, r = i % kTileM;
     gmask[i] = mask[r * words + w];
   }
+  // 4. the tile record: header, then one slot per thread of the first 16
+  // (RECORDS; at lmax 3 the record's registers would cost the CTA its
+  // occupancy, and tile_records_kernel writes the slots instead)
+  float* R = pv.rec + (long long)tile * plan_record_words(L);
+  if (threadIdx.x < kRecHdr) reinterpret_cast<int*>(R)[threadIdx.x] = threadIdx.x == 0 ? U : 0;
+  if constexpr (RECORDS)
+    if (threadIdx.x < kTileM) write_slot_record<L>(tgt[threadIdx.x], p.pos, threadIdx.x, R);
 }
 
 // The same plan for large n, at a cost per tile independent of n: one CTA per
@@ -154,6 +192,7 @@ __global__ void __launch_bounds__(kPlanThreads) build_plan_kernel(const __grid_c
 // sets each (target, neighbour) membership bit at the position a binary
 // search of the sorted union gives.  Union, padding and mask are bit for bit
 // those of build_plan_kernel.
+template <int L, bool RECORDS>
 __global__ void __launch_bounds__(kPlanThreads) build_plan_hash_kernel(const __grid_constant__ PlanParams p) {
   extern __shared__ int hsm[];
   const PlanView& pv = p.plan;
@@ -253,42 +292,28 @@ __global__ void __launch_bounds__(kPlanThreads) build_plan_hash_kernel(const __g
     const int w = i / kTileM, r = i % kTileM;
     gmask[i] = mask[r * words + w];
   }
+  // 4. the tile record: header, then one slot per thread of the first 16
+  // (RECORDS; at lmax 3 the record's registers would cost the CTA its
+  // occupancy, and tile_records_kernel writes the slots instead)
+  float* R = pv.rec + (long long)tile * plan_record_words(L);
+  if (threadIdx.x < kRecHdr) reinterpret_cast<int*>(R)[threadIdx.x] = threadIdx.x == 0 ? U : 0;
+  if constexpr (RECORDS)
+    if (threadIdx.x < kTileM) write_slot_record<L>(tgt[threadIdx.x], p.pos, threadIdx.x, R);
 }
 
-// One thread per target slot (tile * kTileM + r): the slot's atom, |r|^l and
-// the Wigner-D matrices of its alignment rotation (identity for an empty slot
-// or an atom at the origin), built in registers, into the tile record.
+// The record slots of every tile, one thread per slot (tile * kTileM + r),
+// for plans whose builder does not write them (lmax 3).
 constexpr int kRecThreads = 128;
 template <int L>
 __global__ void __launch_bounds__(kRecThreads)
-tile_records_kernel(const int32_t* __restrict__ order, const float* __restrict__ pos,
-                    const int* __restrict__ ulen, int n, int tiles, float* __restrict__ rec) {
-  constexpr int WS = wig_size(L);
-  constexpr int REC = plan_record_words(L);
-  static_assert(WS == rec_wig_size(L) && REC % 4 == 0, "record layout");
+tile_records_kernel(const int32_t* __restrict__ order, const float* __restrict__ pos, int n, int tiles,
+                    float* __restrict__ rec) {
   const long long slot = (long long)blockIdx.x * kRecThreads + threadIdx.x;
   if (slot >= (long long)tiles * kTileM) return;
-  const int tile = int(slot / kTileM), r = int(slot % kTileM);
   int tg = -1;
   if (slot < n) tg = order ? order[slot] : int(slot);
   if ((unsigned)tg >= (unsigned)n) tg = -1;
-  float Q[9];
-  float rr = 0.f;
-  if (tg >= 0) rr = alignment_rotation(pos[3 * tg], pos[3 * tg + 1], pos[3 * tg + 2], Q);
-  else alignment_rotation(0.f, 0.f, 0.f, Q);
-  float D[WS];
-  wigner_regs<L>(Q, D);
-  float* R = rec + (long long)tile * REC;
-#pragma unroll
-  for (int e = 0; e < WS; ++e) R[rec_off_D(L) + r * WS + e] = D[e];
-  reinterpret_cast<int*>(R)[kRecTgt + r] = tg;
-  float a = 1.f;
-#pragma unroll
-  for (int l = 0; l <= L; ++l) {
-    R[kRecRp + r * (L + 1) + l] = a;
-    a *= rr;
-  }
-  if (r < kRecHdr) reinterpret_cast<int*>(R)[r] = r == 0 ? ulen[tile] : 0;
+  write_slot_record<L>(tg, pos, int(slot % kTileM), rec + (slot / kTileM) * plan_record_words(L));
 }
 
 }  // namespace
@@ -350,22 +375,29 @@ int launch_build_plan(int n, int K, int lmax, const int32_t* d_nbr, const int32_
   p.plan = plan_view(d_plan, n, K, lmax);
   p.n = n;
   p.K = K;
+  p.pos = d_pos;
   const size_t shmem = plan_smem_bytes(n, K);
   if (shmem > kPlanSmemLimit) return EGAT_ERR_UNSUPPORTED;
-  auto kern = n <= kBitmapPlanAtoms ? build_plan_kernel : build_plan_hash_kernel;
+  auto pick = [&](auto lc) {
+    constexpr int L = decltype(lc)::value;
+    return n <= kBitmapPlanAtoms ? build_plan_kernel<L, (L < 3)> : build_plan_hash_kernel<L, (L < 3)>;
+  };
+  void (*kern)(PlanParams) = nullptr;
+  switch (lmax) {
+    case 1: kern = pick(std::integral_constant<int, 1>{}); break;
+    case 2: kern = pick(std::integral_constant<int, 2>{}); break;
+    case 3: kern = pick(std::integral_constant<int, 3>{}); break;
+    default: return EGAT_ERR_UNSUPPORTED;
+  }
   if (shmem > 48 * 1024 &&
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(shmem)) !=
           cudaSuccess)
     return EGAT_ERR_CUDA;
   kern<<<p.plan.tiles, kPlanThreads, shmem, st>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return EGAT_ERR_CUDA;
-  const int tiles = p.plan.tiles;
-  const int blocks = (tiles * kTileM + kRecThreads - 1) / kRecThreads;
-  switch (lmax) {
-    case 1: tile_records_kernel<1><<<blocks, kRecThreads, 0, st>>>(d_order, d_pos, p.plan.ulen, n, tiles, p.plan.rec); break;
-    case 2: tile_records_kernel<2><<<blocks, kRecThreads, 0, st>>>(d_order, d_pos, p.plan.ulen, n, tiles, p.plan.rec); break;
-    case 3: tile_records_kernel<3><<<blocks, kRecThreads, 0, st>>>(d_order, d_pos, p.plan.ulen, n, tiles, p.plan.rec); break;
-    default: return EGAT_ERR_UNSUPPORTED;
+  if (lmax >= 3 && cudaGetLastError() == cudaSuccess) {
+    const long long slots = (long long)p.plan.tiles * kTileM;
+    tile_records_kernel<3><<<unsigned((slots + kRecThreads - 1) / kRecThreads), kRecThreads, 0, st>>>(
+        d_order, d_pos, n, p.plan.tiles, p.plan.rec);
   }
   return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
 }
