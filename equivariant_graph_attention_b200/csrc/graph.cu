@@ -40,10 +40,13 @@ struct GraphWs {
 constexpr int kScanTile = 4096;  // elements per scan block (1024 threads x 4)
 
 int bucket_bits(int n) {
-  // bits per axis b, table size M = 2^(3b) >= 2n, 3 <= b <= 8 (2^b >= 5
-  // keeps the 5 x 5 x 5 cells around any cell in distinct buckets)
+  // bits per axis b, table size M = 2^(3b) >= n, 3 <= b <= 8 (2^b >= 5
+  // keeps the 5 x 5 x 5 cells around any cell in distinct buckets).  With
+  // several atoms per cell, at least n buckets leave most cells a bucket of
+  // their own; atoms of other cells that share a bucket fail the distance
+  // test.
   int b = 3;
-  while (b < 8 && (int64_t(1) << (3 * b)) < 2 * int64_t(n)) ++b;
+  while (b < 8 && (int64_t(1) << (3 * b)) < int64_t(n)) ++b;
   return b;
 }
 
@@ -181,7 +184,28 @@ __global__ void __launch_bounds__(1024) scan_apply(const int* __restrict__ in, i
   }
 }
 
+// Up to kScanSingle + 1 entries: one CTA, each thread a contiguous chunk of
+// at most 9 (larger arrays take the three-phase scan, whose loads coalesce).
+constexpr int kScanSingle = 1 << 13;
+__global__ void __launch_bounds__(1024) scan_single(const int* __restrict__ in, int n, int* __restrict__ out) {
+  __shared__ int sw[32];
+  const int per = (n + 1 + 1023) / 1024;
+  const int b0 = threadIdx.x * per;
+  int s = 0;
+  for (int i = b0; i < b0 + per && i < n; ++i) s += in[i];
+  int total;
+  int ex = block_exclusive_scan(s, sw, total);
+  for (int i = b0; i < b0 + per && i <= n; ++i) {
+    out[i] = ex;
+    if (i < n) ex += in[i];
+  }
+}
+
 int launch_scan(const int* in, int n, int* partial, int* out, cudaStream_t st) {
+  if (n <= kScanSingle) {
+    scan_single<<<1, 1024, 0, st>>>(in, n, out);
+    return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
+  }
   const int nb = (n + 1 + kScanTile - 1) / kScanTile;
   scan_reduce<<<nb, 1024, 0, st>>>(in, n, partial);
   scan_partials<<<1, 1024, 0, st>>>(partial, nb);
