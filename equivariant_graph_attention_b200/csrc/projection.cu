@@ -49,10 +49,8 @@ namespace {
 
 struct ProjParams {
   CUtensorMap amap;       // h's degree-0 slices as a [n][C] bf16 matrix (row pitch D * C * 2 bytes)
-  const __nv_bfloat16* h;
   const float* w[2];      // wq, wk  [C][H*dk]
   __nv_bfloat16* out[2];  // q, k    [n][H*dk]
-  long long row_elems;    // D * C: elements per atom row of h
   int n;
   int tiles;              // 128-atom tiles
 };
@@ -60,13 +58,13 @@ struct ProjParams {
 // ---------------------------------------------------------------- tcgen05 path
 // One CTA per SM holds one weight matrix (wq or wk, by CTA parity) as bf16
 // hi and lo tiles and takes 128-atom tiles:
-//  * A (the tile's degree-0 slices, 128 x 128 bf16) arrives by 16-byte
-//    cp.async copies, two tiles in flight (a ragged tile's missing rows are
-//    zero-filled);
+//  * A (the tile's degree-0 slices, 128 x 128 bf16) arrives by two TMA
+//    tensor copies on the buffer's mbarrier, two tiles in flight (a ragged
+//    tile's missing rows arrive as zeros);
 //  * one thread issues the tile's 16 tcgen05.mma (M = 128, N = 256, K = 16:
 //    eight k-steps, each against the hi and the lo tile), accumulating
-//    h W_hi + h W_lo in float32 in tensor memory (256 columns), and commits
-//    them to an mbarrier;
+//    h W_hi + h W_lo in float32 into one of two 256-column accumulators in
+//    tensor memory, and commits them to that accumulator's mbarrier;
 //  * eight warps read the accumulator back (tcgen05.ld, each warp its
 //    32-lane quarter and half of the columns), round to bf16 and store.
 // Shared-memory operands, both K-major: A (the atoms' channels) in the
@@ -448,12 +446,10 @@ int launch_qk_projection(const egat_shape& s, const void* d_h, const float* d_wq
   if (projection_tc_supported(s)) {
     ProjParams p;
     if (encode_degree0_map(&p.amap, d_h, s.n, row_elems) != 0) return EGAT_ERR_CUDA;
-    p.h = static_cast<const __nv_bfloat16*>(d_h);
     p.w[0] = d_wq;
     p.w[1] = d_wk;
     p.out[0] = static_cast<__nv_bfloat16*>(d_q);
     p.out[1] = static_cast<__nv_bfloat16*>(d_k);
-    p.row_elems = row_elems;
     p.n = s.n;
     p.tiles = (s.n + kUM - 1) / kUM;
     const size_t shmem = UmmaSmem::total;
