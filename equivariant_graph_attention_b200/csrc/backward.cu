@@ -1010,11 +1010,12 @@ int launch_exclusive_scan(const int* d_in, int n, int* d_out, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? EGAT_OK : EGAT_ERR_CUDA;
 }
 
-// The tiled path (bwd_tc_supported): h' in float32 rounded to tf32 as it is
-// stored, dm in float32 (rounded to tf32 where it enters a single tf32
-// product, split into tf32 hi + lo where it forms dL/dh'),
-// the forward plan (target tiles), the in-lists, then the statistics, target
-// and source passes, the source coupling's adjoint and dL/dr.
+// The tiled path (bwd_tc_supported): the forward plan (target tiles) first,
+// whose tile records give every coupling below its rotations; h' in float32
+// rounded to tf32 as it is stored, dm in float32 (rounded to tf32 where it
+// enters a single tf32 product, split into tf32 hi + lo where it forms
+// dL/dh'); the in-lists, then the statistics, target and source passes, the
+// source coupling's adjoint and dL/dr.
 template <int L>
 int launch_backward_tiled(const egat_shape& s, const BwdWs& w, const void* d_h, const float* d_pos,
                           const void* d_q, const void* d_k, const int32_t* d_nbr,

@@ -292,14 +292,17 @@ eaas_source_kernel(const __grid_constant__ EaasParams p) {
     }
   }
 }
-// Planned source coupling staged by tiles, for shapes with one warp per atom
-// (C = 128 up to lmax 2).  Persistent CTAs of kTileM / 2 warps (two per SM)
-// take the plan's tiles in turn.  The tile record arrives by one bulk copy
-// two tiles ahead and the tile's 16 feature rows by 16 bulk copies one tile
-// ahead (double-buffered), so the loads stream while the previous tile is
-// coupled; warp w couples target slots w and w + kTileM / 2 from shared
-// memory (rotation and |r|^l from the record) and writes their h' rows
-// straight to global memory.  Every wait is bounded.
+// Planned source coupling staged by tiles, for C = 128 (up to lmax 2, and
+// lmax 3 in bf16, each slot in two channel halves).  Persistent CTAs of
+// kTileM / 2 warps (two per SM up to lmax 2) take the plan's tiles in turn.
+// The tile record arrives by one bulk copy two tiles ahead and the tile's 16
+// feature rows by 16 bulk copies one tile ahead (double-buffered), so the
+// loads stream while the previous tile is coupled; warp w couples target
+// slots w and w + kTileM / 2 from shared memory (rotation and |r|^l from the
+// record) and writes their h' rows (in TO) straight to global memory.  A
+// warp done with a tile arrives on that tile's done mbarrier; warp 0 refills
+// a buffer once all warps have arrived, so warps never wait on a block
+// barrier.  Every wait is bounded.
 template <int L, typename T>
 struct TileSmem {
   static constexpr int D = (L + 1) * (L + 1);
@@ -316,9 +319,8 @@ struct TileSmem {
   static_assert(ROWB % 16 == 0 && REC % 4 == 0 && bars % 8 == 0, "bulk-copy alignment");
 };
 
-// half a tile's warps per CTA, two CTAs per SM: one CTA's per-tile barrier
-// overlaps the other's work (one CTA per SM at lmax 3, whose rows fill the
-// shared memory)
+// half a tile's warps per CTA, two CTAs per SM (one at lmax 3, whose rows
+// fill the shared memory)
 constexpr int kHalfWarps = kTileM / 2;
 template <int L, typename T, typename TO = T>
 __global__ void __launch_bounds__(kHalfWarps * 32, L >= 3 ? 1 : 2)
