@@ -531,21 +531,9 @@ int launch_eaas_tile(const egat_shape& s, const void* d_x, const float* rec, lon
 }
 
 int launch_eaas_source_f32out(const egat_shape& s, const void* d_x, const float* d_pos,
-                              const float* d_w, float* d_y, cudaStream_t st, bool tf32) {
+                              const float* d_w, float* d_y, cudaStream_t st) {
   const bool bf = s.dtype == EGAT_BF16;
   const long long n = s.n;
-  if (tf32) {
-    Tf32Out* y = reinterpret_cast<Tf32Out*>(d_y);
-    switch (s.lmax) {
-      case 1: return bf ? launch_eaas_t<1, __nv_bfloat16, false, Tf32Out>(s, d_x, d_pos, nullptr, n, d_w, y, st)
-                        : launch_eaas_t<1, float, false, Tf32Out>(s, d_x, d_pos, nullptr, n, d_w, y, st);
-      case 2: return bf ? launch_eaas_t<2, __nv_bfloat16, false, Tf32Out>(s, d_x, d_pos, nullptr, n, d_w, y, st)
-                        : launch_eaas_t<2, float, false, Tf32Out>(s, d_x, d_pos, nullptr, n, d_w, y, st);
-      case 3: return bf ? launch_eaas_t<3, __nv_bfloat16, false, Tf32Out>(s, d_x, d_pos, nullptr, n, d_w, y, st)
-                        : launch_eaas_t<3, float, false, Tf32Out>(s, d_x, d_pos, nullptr, n, d_w, y, st);
-      default: return EGAT_ERR_UNSUPPORTED;
-    }
-  }
   switch (s.lmax) {
     case 1: return bf ? launch_eaas_t<1, __nv_bfloat16, false, float>(s, d_x, d_pos, nullptr, n, d_w, d_y, st)
                       : launch_eaas_t<1, float, false>(s, d_x, d_pos, nullptr, n, d_w, d_y, st);

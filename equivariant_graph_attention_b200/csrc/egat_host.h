@@ -75,11 +75,10 @@ size_t plan_bytes(int n, int K, int lmax);
 PlanView plan_view(void* base, int n, int K, int lmax);
 int launch_build_plan(int n, int K, int lmax, const int32_t* d_nbr, const int32_t* d_cnt,
                       const int32_t* d_order, const float* d_pos, void* d_plan, cudaStream_t st);
-// Step 2 with a float32 result whatever the storage type (the backward pass
-// keeps its intermediates in float32); tf32 = true rounds the stored values
-// to tf32.
+// Step 2 with a float32 result whatever the storage type (the per-target
+// backward keeps its intermediates in float32).
 int launch_eaas_source_f32out(const egat_shape& s, const void* d_x, const float* d_pos,
-                              const float* d_w, float* d_y, cudaStream_t st, bool tf32 = false);
+                              const float* d_w, float* d_y, cudaStream_t st);
 // Step 2 for every atom listed in a plan's tile records, rotations from them.
 int launch_eaas_planned(const egat_shape& s, const void* d_x, const void* d_plan, const float* d_w,
                         void* d_y, cudaStream_t st);
