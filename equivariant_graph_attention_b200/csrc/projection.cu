@@ -443,7 +443,9 @@ int launch_qk_projection(const egat_shape& s, const void* d_h, const float* d_wq
                          void* d_q, void* d_k, cudaStream_t st) {
   const long long row_elems = (long long)(s.lmax + 1) * (s.lmax + 1) * s.C;
   const int HD = s.H * s.dk;
-  if (projection_tc_supported(s)) {
+  // the tensor-core kernel stores 16-byte row segments of q and k
+  const bool out16 = ((reinterpret_cast<uintptr_t>(d_q) | reinterpret_cast<uintptr_t>(d_k)) & 15u) == 0;
+  if (projection_tc_supported(s) && out16) {
     ProjParams p;
     if (encode_degree0_map(&p.amap, d_h, s.n, row_elems) != 0) return EGAT_ERR_CUDA;
     p.w[0] = d_wq;

@@ -331,8 +331,9 @@ EGAT_API int egat_backward(const egat_shape* s, const void* d_h, const float* d_
  *  d_wq, d_wk float32 [C][H*dk]
  *  d_q, d_k   [n][H][dk] in s->dtype (bf16: round to nearest even)
  * bf16 storage with C = 128 and H*dk = 256 runs on tensor cores (the weights
- * as bf16 pairs hi + lo, float32 accumulation); other shapes (C <= 1024,
- * H*dk <= 1024) accumulate in float32 on CUDA cores.  n = 0 is a no-op.
+ * as bf16 pairs hi + lo, float32 accumulation) when d_q and d_k are 16-byte
+ * aligned; other shapes (C <= 1024, H*dk <= 1024) and 4-byte aligned outputs
+ * accumulate in float32 on CUDA cores.  n = 0 is a no-op.
  * Errors: EGAT_ERR_ARG (null or misaligned pointer, bad dtype),
  * EGAT_ERR_UNSUPPORTED, EGAT_ERR_CUDA; a bounded wait that gave up is
  * reported by egat_take_device_status.

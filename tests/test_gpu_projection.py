@@ -148,3 +148,25 @@ def test_projection_weights_at_any_float_offset():
     f = FLOOR["bf16"]
     assert vec_rel_error(q.float().cpu().numpy(), rq, f) < TOL["bf16"]
     assert vec_rel_error(k.float().cpu().numpy(), rk, f) < TOL["bf16"]
+
+
+def test_projection_outputs_at_a_float_offset():
+    """q and k buffers that are only 4-byte aligned (offset views) take the
+    plain kernel (the tensor-core kernel stores 16-byte row segments) and
+    give the same values within the bf16 bar of the oracle."""
+    wl, d, w = _data("uniform4096_l2_bf16")
+    egat = _egat()
+    hd = torch.from_numpy(np.ascontiguousarray(d["h"])).to("cuda", dtype=torch.bfloat16)
+    wq = torch.from_numpy(w["wq"]).cuda()
+    wk = torch.from_numpy(w["wk"]).cuda()
+    m = wl.n * wl.H * wl.dk
+    buf = torch.zeros(2 * m + 4, dtype=torch.bfloat16, device="cuda")
+    q = buf[2:2 + m].view(wl.n, wl.H, wl.dk)
+    k = buf[2 + m + 2:2 + 2 * m + 2].view(wl.n, wl.H, wl.dk)
+    assert q.data_ptr() % 16 != 0 and q.data_ptr() % 4 == 0 and k.data_ptr() % 4 == 0
+    egat.egat_qk_projection(shape_of(wl), hd, wq, wk, q=q, k=k)
+    torch.cuda.synchronize()
+    rq, rk = invariant_projection(d["h"], w["wq"], w["wk"], wl.H, wl.dk)
+    f = FLOOR["bf16"]
+    assert vec_rel_error(q.float().cpu().numpy(), rq, f) < TOL["bf16"]
+    assert vec_rel_error(k.float().cpu().numpy(), rk, f) < TOL["bf16"]
