@@ -11,13 +11,21 @@ scatters the products back to lanes, and checks the epilogues' dq, Delta, dk
 and dL/dh' against the direct formulas on random data (float64, no rounding).
 A wrong lane, row, channel, component or k permutation in the index
 arithmetic shows here.  It runs two heads, not sixteen: the formulas only
-offset by the head.  No GPU is involved.
+offset by the head.  Both stage shapes are modelled: 16 union rows per stage
+up to lmax 2 (key / query fragments by ldmatrix.x4) and 8 rows at lmax 3
+(ldmatrix.x2), where the source pass also runs as two sweeps, one for dk and
+one for dL/dh'.  No GPU is involved.
 """
 import numpy as np
 import pytest
 
-H, DK, RS = 2, 16, 16          # heads modelled, key dimension, union rows per stage
+H, DK = 2, 16                  # heads modelled, key dimension
 C = 8 * H
+
+
+def stage_rows(L):
+    """union rows per stage: two n8 tiles, one at lmax 3"""
+    return 8 if L >= 3 else 16
 
 
 # ----------------------------------------------------------------- PTX fragment layouts
@@ -67,9 +75,10 @@ def acc_as_a(c):
 # ----------------------------------------------------------------- data
 def _data(L, seed):
     D = (L + 1) ** 2
+    RS = stage_rows(L)
     rng = np.random.default_rng(seed)
     n = 64
-    d = dict(D=D, n=n,
+    d = dict(D=D, n=n, RS=RS,
              q=rng.standard_normal((n, H, DK)), k=rng.standard_normal((n, H, DK)),
              hp=rng.standard_normal((n, D, C)), dm=rng.standard_normal((n, D, C)),
              lse=rng.standard_normal((n, H)) + 3.0, delta=rng.standard_normal((n, H)),
@@ -90,6 +99,7 @@ def _bf16_pairs(v):
 # ----------------------------------------------------------------- target pass
 def _target_model(d):
     D, q, k, hp, dm, lse, qs = d["D"], d["q"], d["k"], d["hp"], d["dm"], d["lse"], d["qs"]
+    RS = d["RS"]
     dq = np.zeros((16, H, DK))
     dl_out = np.zeros((16, H))
     for h in range(H):
@@ -107,9 +117,10 @@ def _target_model(d):
         dl = np.zeros((32, 2))
         for st in range(d["nst"]):
             rows = d["uni"][st * RS:(st + 1) * RS]
-            # stage_key_frags<16>: row (lane & 7) + 8 (lane >> 4), half (lane >> 3) & 1
+            # stage_frags<RS>: row (lane & 7) + 8 (lane >> 4), half (lane >> 3) & 1;
+            # ldmatrix.x4 for 16 rows, .x2 (lanes 0-15 address) for 8
             kf = ldmatrix(lambda a: _bf16_pairs(k[rows[a[0]], h, 8 * a[1]:8 * a[1] + 8]),
-                          lambda l: ((l & 7) + 8 * (l >> 4), (l >> 3) & 1), 4)
+                          lambda l: ((l & 7) + 8 * (l >> 4), (l >> 3) & 1), RS // 4)
             for nt in range(RS // 8):
                 s = np.zeros((32, 4))
                 mma_bf16(s, qa, [kf[l][2 * nt] for l in range(32)], [kf[l][2 * nt + 1] for l in range(32)])
@@ -163,7 +174,7 @@ def _alpha_dalpha(d, i, j):
     return a, da
 
 
-@pytest.mark.parametrize("L", [1, 2])
+@pytest.mark.parametrize("L", [1, 2, 3])
 def test_target_pass_fragments(L):
     d = _data(L, seed=10 + L)
     dq, dl = _target_model(d)
@@ -177,9 +188,13 @@ def test_target_pass_fragments(L):
 
 
 # ----------------------------------------------------------------- source pass
-def _source_model(d):
+def _source_model(d, dk_sweep=True, dh_sweep=True):
+    """The source pass; at lmax 3 the kernel runs it twice, once with only the
+    dk sweep's work (h' fragments, dalpha, ds, dk) and once with only the
+    dL/dh' sweep's (the hi/lo weights against dm)."""
     D, q, k, hp, dm, lse, delta, qs = (d["D"], d["q"], d["k"], d["hp"], d["dm"], d["lse"],
                                        d["delta"], d["qs"])
+    RS = d["RS"]
     dk = np.zeros((16, H, DK))
     dh = np.zeros((16, D, C))
     for h in range(H):
@@ -197,20 +212,21 @@ def _source_model(d):
         for st in range(d["nst"]):
             rows = d["uni"][st * RS:(st + 1) * RS]
             qf = ldmatrix(lambda a: _bf16_pairs(q[rows[a[0]], h, 8 * a[1]:8 * a[1] + 8]),
-                          lambda l: ((l & 7) + 8 * (l >> 4), (l >> 3) & 1), 4)
+                          lambda l: ((l & 7) + 8 * (l >> 4), (l >> 3) & 1), RS // 4)
             for nt in range(RS // 8):
                 s = np.zeros((32, 4))
                 mma_bf16(s, ka, [qf[l][2 * nt] for l in range(32)], [qf[l][2 * nt + 1] for l in range(32)])
                 drow = lambda a: list(dm[rows[8 * nt + a[0]], a[1], h * 8 + 4 * a[2]:h * 8 + 4 * a[2] + 4])
                 dp, dp2 = np.zeros((32, 4)), np.zeros((32, 4))
-                for c in range(0, D - 1, 2):
-                    r = ldmatrix(drow, lambda l: (l & 7, c + (l >> 4), (l >> 3) & 1), 4)
-                    mma_tf32(dp, ha[c], [r[l][0] for l in range(32)], [r[l][1] for l in range(32)])
-                    mma_tf32(dp2, ha[c + 1], [r[l][2] for l in range(32)], [r[l][3] for l in range(32)])
-                if D % 2:
-                    r = ldmatrix(drow, lambda l: (l & 7, D - 1, (l >> 3) & 1), 2)
-                    mma_tf32(dp, ha[D - 1], [r[l][0] for l in range(32)], [r[l][1] for l in range(32)])
-                dp += dp2
+                if dk_sweep:
+                    for c in range(0, D - 1, 2):
+                        r = ldmatrix(drow, lambda l: (l & 7, c + (l >> 4), (l >> 3) & 1), 4)
+                        mma_tf32(dp, ha[c], [r[l][0] for l in range(32)], [r[l][1] for l in range(32)])
+                        mma_tf32(dp2, ha[c + 1], [r[l][2] for l in range(32)], [r[l][3] for l in range(32)])
+                    if D % 2:
+                        r = ldmatrix(drow, lambda l: (l & 7, D - 1, (l >> 3) & 1), 2)
+                        mma_tf32(dp, ha[D - 1], [r[l][0] for l in range(32)], [r[l][1] for l in range(32)])
+                    dp += dp2
                 P, ds = np.zeros((32, 4)), np.zeros((32, 4))
                 for lane in range(32):
                     g, t = lane >> 2, lane & 3
@@ -223,14 +239,16 @@ def _source_model(d):
                     ds[lane] = (P[lane, 0] * (dp[lane, 0] - delta[ca, h]), P[lane, 1] * (dp[lane, 1] - delta[cb, h]),
                                 P[lane, 2] * (dp[lane, 2] - delta[ca, h]), P[lane, 3] * (dp[lane, 3] - delta[cb, h]))
                 dsa, pa = acc_as_a(ds), acc_as_a(P)
-                for nd in range(2):
-                    b0 = [q[rows[8 * nt + 2 * (l & 3)], h, 8 * nd + (l >> 2)] for l in range(32)]
-                    b1 = [q[rows[8 * nt + 2 * (l & 3) + 1], h, 8 * nd + (l >> 2)] for l in range(32)]
-                    mma_tf32(dka[nd], dsa, b0, b1)
-                for c in range(D):
-                    b0 = [dm[rows[8 * nt + 2 * (l & 3)], c, h * 8 + (l >> 2)] for l in range(32)]
-                    b1 = [dm[rows[8 * nt + 2 * (l & 3) + 1], c, h * 8 + (l >> 2)] for l in range(32)]
-                    mma_tf32(dha[c], pa, b0, b1)
+                if dk_sweep:
+                    for nd in range(2):
+                        b0 = [q[rows[8 * nt + 2 * (l & 3)], h, 8 * nd + (l >> 2)] for l in range(32)]
+                        b1 = [q[rows[8 * nt + 2 * (l & 3) + 1], h, 8 * nd + (l >> 2)] for l in range(32)]
+                        mma_tf32(dka[nd], dsa, b0, b1)
+                if dh_sweep:
+                    for c in range(D):
+                        b0 = [dm[rows[8 * nt + 2 * (l & 3)], c, h * 8 + (l >> 2)] for l in range(32)]
+                        b1 = [dm[rows[8 * nt + 2 * (l & 3) + 1], c, h * 8 + (l >> 2)] for l in range(32)]
+                        mma_tf32(dha[c], pa, b0, b1)
         for lane in range(32):
             g, t = lane >> 2, lane & 3
             for half in range(2):
@@ -244,10 +262,14 @@ def _source_model(d):
     return dk, dh
 
 
-@pytest.mark.parametrize("L", [1, 2])
+@pytest.mark.parametrize("L", [1, 2, 3])
 def test_source_pass_fragments(L):
     d = _data(L, seed=20 + L)
-    dk, dh = _source_model(d)
+    if L >= 3:   # two sweeps: dk from the first, dL/dh' from the second
+        dk, _ = _source_model(d, dk_sweep=True, dh_sweep=False)
+        _, dh = _source_model(d, dk_sweep=False, dh_sweep=True)
+    else:
+        dk, dh = _source_model(d)
     head = np.arange(C) // 8
     for r, j in enumerate(d["tile"]):
         ref_dk = np.zeros((H, DK))
