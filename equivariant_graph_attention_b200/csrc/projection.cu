@@ -174,7 +174,8 @@ __global__ void __launch_bounds__(kUWarps * 32, 1) qk_projection_umma_kernel(con
     *abort_flag = 0;
   }
   if (warp == 0) {
-    // 256 columns of tensor memory (one CTA per SM: the shared memory fills it)
+    // 512 columns of tensor memory, two accumulators (one CTA per SM: the
+    // shared memory fills it, so the allocation never waits on another CTA)
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tslot)),
                  "r"(kUCols)
                  : "memory");
