@@ -117,8 +117,8 @@ struct TcShape {
 
 // Shared-memory layout (byte offsets; every region 16-byte aligned): staged
 // value and key rows, the tile's query rows, two tile records (current and
-// next), the target-coupling weights [P][C] (fused), the mbarriers and the
-// abort flag, then the tile's union indices [cap] and word-major membership
+// next), the target-coupling weights [P][C] (fused), the mbarriers, the
+// abort flag and the claimed next tile, then the tile's union indices [cap] and word-major membership
 // mask [cap / 32][16] (6 cap bytes, sized at launch).
 template <int L, int H, bool FUSED>
 struct TcSmem {
@@ -136,7 +136,7 @@ struct TcSmem {
   static constexpr size_t rec = sq + size_t(kTileM) * QSTR;
   static constexpr size_t sw2 = rec + 2 * size_t(REC) * 4;
   static constexpr size_t bars = sw2 + (FUSED ? size_t(num_paths(L)) * C * 4 : 0);
-  static constexpr size_t su = bars + (size_t(NBARS) * 8 + 4 + 15) / 16 * 16;
+  static constexpr size_t su = bars + (size_t(NBARS) * 8 + 8 + 15) / 16 * 16;   // + abort flag, next tile
   static size_t total(int cap) { return su + size_t(cap) * 4 + size_t(cap / 32) * kTileM * 4; }
 };
 // the fused epilogue at lmax >= 3 keeps m of the tile in the stage buffers
@@ -178,6 +178,7 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
   uint64_t* idxbar = recbar + 2;                                         // a tile's indices + queries
   uint64_t* mskbar = idxbar + 1;                                         // a tile's mask
   volatile int* abort_flag = reinterpret_cast<volatile int*>(mskbar + 1);
+  int* s_next = reinterpret_cast<int*>(mskbar + 1) + 1;                  // the CTA's next tile
   int* su = reinterpret_cast<int*>(smem + Sm::su);                       // [cap]
   uint32_t* smask = reinterpret_cast<uint32_t*>(su + p.plan.cap);        // [cap / 32][16]
 
@@ -191,6 +192,13 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
   const char* hp_bytes = reinterpret_cast<const char*>(p.hp);
   const char* k_bytes = reinterpret_cast<const char*>(p.k);
   const char* q_bytes = reinterpret_cast<const char*>(p.q);
+  // Tiles are claimed at run time (union sizes, hence tile costs, vary by
+  // about a quarter): a CTA's first tile is blockIdx.x; near the end of each
+  // tile thread 0 takes a ticket c from the plan's counter and the CTA's
+  // next tile is grid + c (past the last tile: done).  Every processed tile
+  // takes exactly one ticket, so a launch hands out tickets 0 .. tiles - 1,
+  // in that order; the CTA holding the last one sets the counter back to
+  // zero for the next launch on the plan (ordered after this one).
   if (blockIdx.x >= pv.tiles) return;   // whole CTA
 
   if (tid == 0) {
@@ -273,20 +281,33 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
   }
 
   int k = 0;   // this CTA's tile sequence number
-  for (; tile < pv.tiles; ++k, tile += grid) {
+  while (tile < pv.tiles) {
     const float* rec = recbuf + (k & 1) * REC;
     const float* nrec = recbuf + ((k + 1) & 1) * REC;
-    const int next = tile + grid;
-    const bool has_next = next < pv.tiles;
+    // thread 0 claims the tile after this one a stage before it takes the
+    // claim (the next tile's record copy), which is a stage before the next
+    // tile's indices are copied; every thread learns the next tile after
+    // the stage loop
+    int ticket = 0;
+    auto claim = [&]() { ticket = atomicAdd(pv.sched, 1); };
+    int next = pv.tiles;
+    bool has_next = false;
     // this tile's record, indices, queries and mask (all issued during the
     // previous tile, or above)
     bounded_wait(smem_u32(recbar + (k & 1)), uint32_t(k >> 1) & 1u, kWaitPolls, abort_flag);
     bounded_wait(smem_u32(idxbar), uint32_t(k) & 1u, kWaitPolls, abort_flag);
     bounded_wait(smem_u32(mskbar), uint32_t(k) & 1u, kWaitPolls, abort_flag);
-    // the next tile's record into the other buffer (its last reader, the
-    // previous tile's epilogue, finished before that tile's last barrier)
-    if (tid == 0 && has_next) issue_record(next, (k + 1) & 1);
     const int nstages = stages_of(rec);
+    // thread 0: publish the claimed tile and copy its record into the other
+    // buffer (its last reader, the previous tile's epilogue, finished before
+    // that tile's last barrier)
+    auto take_claim = [&]() {
+      if (ticket == pv.tiles - 1) atomicExch(pv.sched, 0);   // every ticket was handed out
+      next = grid + ticket;
+      has_next = next < pv.tiles;
+      *s_next = next;
+      if (has_next) issue_record(next, (k + 1) & 1);
+    };
 
     // Q fragment of this head for the tile's 16 targets
     uint32_t qa[4];
@@ -316,9 +337,13 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
     // the stage after which the indices and query rows are free for the next
     // tile: its barrier follows the last issue that reads them
     const int trig = nstages - STAGES + 1 > 0 ? nstages - STAGES + 1 : 0;
+    const int take_st = trig > 1 ? trig - 1 : 0;     // the claim is taken no later than trig
+    const int claim_st = take_st > 1 ? take_st - 1 : 0;
     for (int st = 0; st < nstages; ++st) {
       __syncthreads();   // every warp is done with the buffer about to be refilled
       if (st + STAGES - 1 < nstages) issue_rows(st + STAGES - 1, gbase + st + STAGES - 1);
+      if (st == claim_st && tid == 0) claim();
+      if (st == take_st && tid == 0) take_claim();
       if (st == trig && tid == 0 && has_next) {
         bounded_wait(smem_u32(recbar + ((k + 1) & 1)), uint32_t((k + 1) >> 1) & 1u, kWaitPolls,
                      abort_flag);
@@ -465,7 +490,13 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
         }
       }   // k-steps of the stage
     }
+    if (nstages == 0 && tid == 0) {
+      claim();
+      take_claim();
+    }
     __syncthreads();   // every warp is done with the stage buffers and the mask
+    next = *s_next;    // rewritten only after the tile's last barrier
+    has_next = next < pv.tiles;
     gbase += nstages;
     if (tid == 0 && has_next) {
       if (nstages == 0) {
@@ -561,6 +592,8 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
     if constexpr (!kEarlyRows) fence_proxy_async_smem();   // scratch before bulk copies
     __syncthreads();   // the record buffer and the stage buffers are refilled next
     if (!kEarlyRows && has_next) stage_next();
+    ++k;
+    tile = next;
   }
   if (*abort_flag && tid == 0) {
     // a wait gave up: give every barrier's last phase a short, bounded chance

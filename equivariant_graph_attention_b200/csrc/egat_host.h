@@ -52,6 +52,8 @@ struct PlanView {
   int* uni;         // [tiles][cap] union atom indices (ascending), padded to kPlanPad
   uint32_t* mask;   // [tiles][cap / 32][kTileM] word w of row r: bits of union atoms 32w..32w+31
   float* rec;       // [tiles][plan_record_words(lmax)] target ids, |r|^l, Wigner-D (see below)
+  int* sched;       // the attention kernel's tile-claim counter: zeroed by the plan
+                    // builder, zero again after every launch
   int cap;          // union capacity per tile (power of two >= kTileM * K)
   int tiles;
 };

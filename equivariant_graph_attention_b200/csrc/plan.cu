@@ -83,6 +83,7 @@ __global__ void __launch_bounds__(kPlanThreads) build_plan_kernel(const __grid_c
   __shared__ int tgt[kTileM], rowcnt[kTileM];
   __shared__ int warp_sum[kPlanThreads / 32];
   __shared__ int s_unique;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *pv.sched = 0;   // the attention kernel's claim counter
   const int tile = blockIdx.x;
 
   // the tile's targets and their neighbour counts (0 for an empty slot)
@@ -204,6 +205,7 @@ __global__ void __launch_bounds__(kPlanThreads) build_plan_hash_kernel(const __g
   uint32_t* mask = reinterpret_cast<uint32_t*>(srt + cap);   // [kTileM][words]
   __shared__ int tgt[kTileM], rowcnt[kTileM];
   __shared__ int s_unique;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *pv.sched = 0;   // the attention kernel's claim counter
   const int tile = blockIdx.x;
   if (threadIdx.x < kTileM) {
     const long long slot = (long long)tile * kTileM + threadIdx.x;
@@ -344,7 +346,7 @@ size_t plan_bytes(int n, int K, int lmax) {
   auto a256 = [](size_t x) { return (x + 255) & ~size_t(255); };
   return a256(tiles * sizeof(int)) + a256(tiles * cap * sizeof(int)) +
          a256(tiles * kTileM * (cap / 32) * sizeof(uint32_t)) +
-         a256(tiles * size_t(plan_record_words(lmax)) * sizeof(float));
+         a256(tiles * size_t(plan_record_words(lmax)) * sizeof(float)) + a256(sizeof(int));
 }
 
 PlanView plan_view(void* base, int n, int K, int lmax) {
@@ -360,7 +362,8 @@ PlanView plan_view(void* base, int n, int K, int lmax) {
   v.mask = reinterpret_cast<uint32_t*>(b);
   b += a256(tiles * kTileM * (size_t(cap) / 32) * sizeof(uint32_t));
   v.rec = reinterpret_cast<float*>(b);
-  (void)lmax;
+  b += a256(tiles * size_t(plan_record_words(lmax)) * sizeof(float));
+  v.sched = reinterpret_cast<int*>(b);
   v.cap = cap;
   v.tiles = int(tiles);
   return v;

@@ -202,14 +202,19 @@ EGAT_API int egat_otf_attention_coupled(const egat_shape* s, const void* d_q, co
  * |r|^l and the real Wigner-D matrices of their alignment rotations for the
  * target coupling), built from the padded list (d_nbr, d_cnt — d_cnt may be
  * NULL), d_order and d_pos (float32 [n][3], required) into caller memory
- * d_plan of at least the queried size.  The builder keeps a bitmap over all n
- * atoms per tile in shared memory, so it supports n up to about 800,000
- * atoms (2 * n / 8 bytes plus the tile mask within 200 KiB; larger n returns
- * EGAT_ERR_UNSUPPORTED and egat_forward falls back to the per-target kernel).
- * The plan depends only on the graph and the positions; it is reused by
- * every attention call on them.
+ * d_plan of at least the queried size.  Per tile the builder keeps, in
+ * shared memory, a bitmap over all n atoms up to n = 131,072 and beyond that
+ * a hash table of the tile's candidates whose size depends on K alone; plans
+ * whose shared memory would pass 200 KiB (K > 512 beyond 131,072 atoms)
+ * return EGAT_ERR_UNSUPPORTED, and egat_forward then falls back to the
+ * per-target kernel.  The plan depends only on the graph and the positions;
+ * it is reused by every attention call on them.
  * egat_otf_attention_tiled: fused = 1 writes ^h (d_w2 required), fused = 0
  * writes m (d_w2 unused); target order and rotations come from the plan.
+ * Its CTAs claim tiles at run time from a counter kept in the plan (the
+ * builder zeroes it and each launch leaves it zero), so one plan serves one
+ * attention launch at a time: launches that share a plan must be ordered
+ * (one stream, or events); concurrent ones need plans of their own.
  */
 EGAT_API int egat_attention_plan_bytes(const egat_shape* s, size_t* bytes);
 EGAT_API int egat_build_attention_plan(const egat_shape* s, const int32_t* d_nbr,

@@ -51,9 +51,10 @@ def test_host_only_queries(lib):
     # h' plus, for tensor-core shapes, the attention plan (2048 tiles: union
     # capacity 4096 ints, a 16 x 128-word mask and a target record of a
     # 4-word header + 16 x (1 id + 3 powers |r|^l + 35 Wigner-D entries) words
-    # each, plus lengths)
+    # each, plus lengths and the attention kernel's tile-claim counter in a
+    # 256-byte block of its own)
     plan = egat.egat_attention_plan_bytes(s)
-    assert plan == 2048 * 4 + 2048 * 4096 * 4 + 2048 * 16 * 128 * 4 + 2048 * (4 + 16 * 39) * 4
+    assert plan == 2048 * 4 + 2048 * 4096 * 4 + 2048 * 16 * 128 * 4 + 2048 * (4 + 16 * 39) * 4 + 256
     assert egat.egat_forward_workspace_bytes(s) == 32768 * 9 * 128 * 2 + plan
     f32 = egat.Shape(n=648, lmax=2, C=128, H=16, dk=16, K=64, dtype="f32")
     assert egat.egat_forward_workspace_bytes(f32) == 648 * 9 * 128 * 4

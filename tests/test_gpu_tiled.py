@@ -136,6 +136,32 @@ def test_tiled_attention_parity(name):
     assert err < TOL["bf16"] and e < TOL["bf16"]
 
 
+@pytest.mark.parametrize("name", ["uniform4096_l2_bf16", "uniform32768_K256_l2_bf16"])
+def test_tiled_relaunch_on_one_plan(name):
+    """The kernel's CTAs claim tiles at run time from a counter kept in the
+    plan (its last 256-byte block): repeated launches on one plan (m, then ^h
+    twice, then m again) give bit-identical results, and each launch leaves
+    the counter at zero."""
+    egat = _egat()
+    wl, d = _data(name)
+    dev = device_inputs(wl, d)
+    g = egat.egat_build_graph(dev["pos_q"], wl.cutoff_q, K=wl.K)
+    shape = shape_of(wl)
+    hp = egat.egat_eaas_couple(shape, dev["h"], dev["pos"], dev["w1"])
+    plan = egat.egat_build_attention_plan(shape, g["nbr"], g["cnt"], g["order"], dev["pos"])
+    nb = egat.egat_attention_plan_bytes(shape)
+    counter = lambda: int(plan[nb - 256:nb - 252].cpu().numpy().view(np.int32)[0])
+    assert counter() == 0
+    m0 = egat.egat_otf_attention_tiled(shape, dev["q"], dev["k"], hp, plan, fused=False)
+    assert counter() == 0
+    f0 = egat.egat_otf_attention_tiled(shape, dev["q"], dev["k"], hp, plan, w2=dev["w2"], fused=True)
+    f1 = egat.egat_otf_attention_tiled(shape, dev["q"], dev["k"], hp, plan, w2=dev["w2"], fused=True)
+    m1 = egat.egat_otf_attention_tiled(shape, dev["q"], dev["k"], hp, plan, fused=False)
+    assert counter() == 0
+    assert torch.equal(m0, m1) and torch.equal(f0, f1)
+    assert egat.egat_take_device_status() == 0
+
+
 @pytest.mark.parametrize("name", BF16)
 def test_tiled_fused_matches_per_target_kernel(name):
     """^h from the tiled kernel and from the per-target kernel agree (both

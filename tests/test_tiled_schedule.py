@@ -1,7 +1,8 @@
 """Host-side model of the copy / wait protocol of the tensor-core attention
 kernel (`otf_attention_tc_kernel`, csrc/attention_tc.cu).
 
-The kernel walks its CTA's tiles in order.  Bulk copies fill shared-memory
+A CTA walks the tiles it claims, in claim order (the claims themselves are
+modelled by test_tile_claims below).  Bulk copies fill shared-memory
 buffers and complete mbarrier phases: the stage buffers (rows), two tile
 record buffers (alternating), the tile's union indices + query rows, and its
 membership mask.  This model replays the kernel's control flow (tile
@@ -101,15 +102,16 @@ def replay(S, RS, ulen_of_tiles):
         m.wait("idx", k & 1, k)
         m.wait("msk", k & 1, k)
         m.read(f"recbuf{k & 1}", ("rec", k))
-        if has_next:
-            issue_record(k + 1)
         ns = stages_of(ulen_of_tiles[k])
         m.read("sq", ("q", k))
         trig = max(0, ns - S + 1)
+        take_st = trig - 1 if trig > 1 else 0    # the claimed next tile's record is copied here
         for st in range(ns):
             m.barrier()
             if st + S - 1 < ns:
                 issue_rows(k, st + S - 1, gbase + st + S - 1)
+            if st == take_st and has_next:
+                issue_record(k + 1)
             if st == trig and has_next:
                 wait_rec(k + 1)
                 m.fill("idx", "su", ("idx", k + 1))
@@ -119,6 +121,8 @@ def replay(S, RS, ulen_of_tiles):
             m.wait(stage_bar(gs), (gs // S) & 1, stage_fill[gs])
             m.read(f"stage{gs % S}", ("rows", k, st))
             m.read("smask", ("msk", k))
+        if ns == 0 and has_next:
+            issue_record(k + 1)
         m.barrier()
         gbase += ns
         if has_next:
@@ -166,3 +170,57 @@ def test_model_catches_an_early_index_prefetch():
         for seed in range(50):
             rng = random.Random(seed)
             ns["replay"](2, 32, [rng.randint(33, 400) for _ in range(4)])
+
+
+def claims(tiles: int, grid: int, seed: int):
+    """The run-time tile claims of `grid` CTAs, in a random interleaving.
+
+    A CTA's first tile is its block index; once per tile (near its end) its
+    thread 0 takes a ticket c = atomicAdd(counter, 1), and a while later it
+    takes the claim: the next tile is grid + c, past the last tile meaning
+    done, and the holder of ticket tiles - 1 sets the counter to zero.
+    Returns the tiles each CTA processed and the counter after the launch."""
+    rng = random.Random(seed)
+    box = [0]
+    got = {b: [] for b in range(grid)}
+    handed = []
+
+    def cta(b):
+        tile = b
+        while tile < tiles:
+            got[b].append(tile)
+            yield                            # the tile's work, up to the claim
+            c = box[0]                       # atomicAdd returns the old value
+            box[0] += 1
+            handed.append(c)
+            yield                            # a stage later: take the claim
+            if c == tiles - 1:
+                assert sorted(handed) == list(range(tiles)), "reset before the last claim"
+                box[0] = 0
+            yield                            # the rest of the tile
+            tile = grid + c
+
+    progs = {b: cta(b) for b in range(grid)}
+    live = set(progs)
+    while live:
+        b = rng.choice(sorted(live))
+        try:
+            next(progs[b])
+        except StopIteration:
+            live.discard(b)
+    assert handed == list(range(tiles))      # tickets are handed out in order
+    return got, box[0]
+
+
+@pytest.mark.parametrize("tiles", [1, 2, 147, 148, 149, 300, 2048])
+@pytest.mark.parametrize("seed", range(3))
+def test_tile_claims(tiles, seed):
+    """Every tile is processed exactly once, whatever the interleaving, and
+    the counter is zero again after each launch (three launches in a row on
+    one plan)."""
+    grid = min(tiles, SM_COUNT)
+    for launch in range(3):
+        got, after = claims(tiles, grid, seed * 10 + launch)
+        assert sorted(t for ts in got.values() for t in ts) == list(range(tiles))
+        assert all(ts and ts[0] == b for b, ts in got.items())
+        assert after == 0
