@@ -280,10 +280,13 @@ constexpr int kBlockCells = kWidth * kWidth * kWidth;
 // marking a neighbour within the cutoff.  Cells are taken 32 at a time: each
 // lane loads one cell's bucket range, a warp scan lays the ranges end to end,
 // and the warp walks that flat candidate list 32 at a time, each lane finding
-// its candidate's cell by a binary search over the scanned offsets.
+// its candidate's cell by a binary search over the scanned offsets.  Warps
+// that share a sweep take rounds round0, round0 + round_step, ... and, within
+// a round, candidate chunks part, part + parts, ...
 template <typename F>
 __device__ __forceinline__ void for_each_neighbour_rounds(const Search& s, int4 p, int4 c,
-                                                          int round0, int round_step, F&& f) {
+                                                          int round0, int round_step, int part,
+                                                          int parts, F&& f) {
   const int lane = threadIdx.x & 31;
   for (int r0 = round0 * 32; r0 < kBlockCells; r0 += round_step * 32) {
     const int l = r0 + lane;
@@ -309,7 +312,7 @@ __device__ __forceinline__ void for_each_neighbour_rounds(const Search& s, int4 
     }
     const int total = __shfl_sync(0xffffffffu, inc, 31);
     const int exc = inc - len;
-    for (int base = 0; base < total; base += 32) {
+    for (int base = part * 32; base < total; base += parts * 32) {
       const int k = base + lane;
       // owner: the last lane whose range starts at or before k
       int own = 0;
@@ -340,7 +343,7 @@ __device__ __forceinline__ void for_each_neighbour_rounds(const Search& s, int4 
 
 template <typename F>
 __device__ __forceinline__ void for_each_neighbour(const Search& s, int4 p, int4 c, F&& f) {
-  for_each_neighbour_rounds(s, p, c, 0, 1, f);
+  for_each_neighbour_rounds(s, p, c, 0, 1, 0, 1, f);
 }
 
 __global__ void count_neighbours(Search s, int n, int* __restrict__ deg) {
@@ -405,14 +408,17 @@ fill_padded(Search s, int n, int K, int32_t* __restrict__ nbr, int32_t* __restri
 
 // Rows with more than K neighbours: one CTA of kFixWarps warps per listed atom
 // (persistent CTAs; the loop is bounded by the device-side count).  The warps
-// split the 125-cell sweep by rounds and gather every neighbour's key
+// split the 125-cell sweep (four rounds of 32 cells, each round's candidates
+// in kFixWarps / 4 interleaved parts) and gather every neighbour's key
 // (d^2 << shift | j) into shared memory.  The keys are distinct (j is), so a
 // key's rank among them is its place in the row: the key of rank r < K writes
 // row[r], and the row lists the K nearest, nearest first, ties to the smaller
 // index.  A row with more keys than the buffer holds first finds its K-th
 // smallest key by bisection (one warp), then gathers the K keys up to it and
 // ranks those.
-constexpr int kFixWarps = 4;
+constexpr int kFixWarps = 16;
+constexpr int kFixRounds = (kBlockCells + 31) / 32;
+static_assert(kFixWarps % kFixRounds == 0, "whole rounds per group of warps");
 
 __global__ void __launch_bounds__(kFixWarps * 32)
 fix_truncated(Search s, int K, int32_t* __restrict__ nbr, const int* __restrict__ trunc,
@@ -426,7 +432,8 @@ fix_truncated(Search s, int K, int32_t* __restrict__ nbr, const int* __restrict_
   const unsigned long long jmask = (1ull << s.key_shift) - 1ull;
   // every warp sweeps its rounds of cells; f(hit, key) with full-warp ballots
   auto gather = [&](const int4& p, const int4& c, int* counter, auto keep) {
-    for_each_neighbour_rounds(s, p, c, wib, kFixWarps, [&](bool hit, int j, long long d2) {
+    for_each_neighbour_rounds(s, p, c, wib % kFixRounds, kFixRounds, wib / kFixRounds,
+                              kFixWarps / kFixRounds, [&](bool hit, int j, long long d2) {
       const unsigned long long key = (((unsigned long long)d2) << s.key_shift) | (unsigned long long)j;
       const bool take = hit && keep(key);
       const unsigned m = __ballot_sync(0xffffffffu, take);
