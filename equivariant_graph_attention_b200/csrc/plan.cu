@@ -63,15 +63,17 @@ __device__ __forceinline__ void write_slot_record(int tg, const float* __restric
 
 // One CTA per tile.  Shared memory holds a bitmap over all atom indices
 // (bit j set when atom j is a neighbour of some target of the tile), the
-// per-word prefix counts of that bitmap, and the tile's membership mask.
-//  1. set the bits of every neighbour of the tile's targets;
+// per-word prefix counts of that bitmap, the tile's membership mask and its
+// neighbour-list entries.
+//  1. load the tile's entries (a thread's entries of all 16 rows in flight
+//     together), keep them in shared memory and set the bit of every one;
 //  2. prefix-count the bitmap's words: the union, in ascending atom index, is
 //     read straight off the bitmap, and the union position of atom j is
 //     prefix[j / 32] + popcount(bits of word j / 32 below j);
 //  3. one membership bit per (target, neighbour) at that position.
 // Cost per tile is O(n / 32) words plus O(16 K) entries; deterministic.
 template <int L, bool RECORDS>
-__global__ void __launch_bounds__(kPlanThreads) build_plan_kernel(const __grid_constant__ PlanParams p) {
+__global__ void __launch_bounds__(kPlanThreads, 6) build_plan_kernel(const __grid_constant__ PlanParams p) {
   extern __shared__ uint32_t sm[];
   const PlanView& pv = p.plan;
   const int cap = pv.cap;                         // >= kTileM * K, power of two
@@ -80,6 +82,7 @@ __global__ void __launch_bounds__(kPlanThreads) build_plan_kernel(const __grid_c
   uint32_t* bitmap = sm;                          // [nw]
   uint32_t* prefix = sm + nw;                     // [nw]
   uint32_t* mask = sm + 2 * nw;                   // [kTileM][words]
+  int* ent = reinterpret_cast<int*>(mask + kTileM * words);   // [kTileM][K] the tile's entries
   __shared__ int tgt[kTileM], rowcnt[kTileM];
   __shared__ int warp_sum[kPlanThreads / 32];
   __shared__ int s_unique;
@@ -103,19 +106,24 @@ __global__ void __launch_bounds__(kPlanThreads) build_plan_kernel(const __grid_c
   for (int i = threadIdx.x; i < nw; i += blockDim.x) bitmap[i] = 0u;
   for (int i = threadIdx.x; i < kTileM * words; i += blockDim.x) mask[i] = 0u;
   __syncthreads();
-  // visit every (target row, neighbour) entry of the tile: rows in turn,
-  // the row's entries spread over the threads (coalesced loads of nbr)
-  auto for_each_entry = [&](auto&& f) {
-    for (int r = 0; r < kTileM; ++r) {
-      const int c = rowcnt[r];
-      const int32_t* row = p.nbr + (long long)(tgt[r] < 0 ? 0 : tgt[r]) * p.K;
-      for (int e = threadIdx.x; e < c; e += blockDim.x) f(r, row[e]);
+  // 1. the tile's entries and the bitmap of their union: thread t takes
+  // entry e = t, t + 256, ... of every row (coalesced loads of nbr, eight
+  // rows' loads in flight together); slots past a row's count hold -1
+  constexpr int kBatch = 8;
+  for (int e = threadIdx.x; e < p.K; e += blockDim.x) {
+#pragma unroll 1
+    for (int r0 = 0; r0 < kTileM; r0 += kBatch) {
+      int v[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i)
+        v[i] = e < rowcnt[r0 + i] ? p.nbr[(long long)tgt[r0 + i] * p.K + e] : -1;
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        ent[(r0 + i) * p.K + e] = v[i];
+        if ((unsigned)v[i] < (unsigned)p.n) atomicOr(&bitmap[v[i] >> 5], 1u << (v[i] & 31));
+      }
     }
-  };
-  // 1. bitmap of the union
-  for_each_entry([&](int, int j) {
-    if ((unsigned)j < (unsigned)p.n) atomicOr(&bitmap[j >> 5], 1u << (j & 31));
-  });
+  }
   __syncthreads();
   // 2. per-word exclusive prefix counts (contiguous chunk per thread + block scan)
   const int per = (nw + kPlanThreads - 1) / kPlanThreads;
@@ -163,12 +171,16 @@ __global__ void __launch_bounds__(kPlanThreads) build_plan_kernel(const __grid_c
   const int filler = U > 0 ? uni[0] : 0;
   for (int e = U + threadIdx.x; e < upad; e += blockDim.x) uni[e] = filler;
   if (threadIdx.x == 0) pv.ulen[tile] = U;
-  // 3. membership bits
-  for_each_entry([&](int r, int j) {
-    if ((unsigned)j >= (unsigned)p.n) return;
-    const int pos = int(prefix[j >> 5]) + __popc(bitmap[j >> 5] & ((1u << (j & 31)) - 1u));
-    atomicOr(&mask[r * words + (pos >> 5)], 1u << (pos & 31));
-  });
+  // 3. membership bits, from the cached entries
+  for (int r = 0; r < kTileM; ++r) {
+    const int c = rowcnt[r];
+    for (int e = threadIdx.x; e < c; e += blockDim.x) {
+      const int j = ent[r * p.K + e];
+      if ((unsigned)j >= (unsigned)p.n) continue;
+      const int pos = int(prefix[j >> 5]) + __popc(bitmap[j >> 5] & ((1u << (j & 31)) - 1u));
+      atomicOr(&mask[r * words + (pos >> 5)], 1u << (pos & 31));
+    }
+  }
   __syncthreads();
   // word-major in memory: the kTileM words of one 32-atom chunk are contiguous
   uint32_t* gmask = pv.mask + (long long)tile * words * kTileM;
@@ -329,7 +341,7 @@ size_t plan_smem_bytes(int n, int K) {
   const size_t mask = size_t(kTileM) * (plan_capacity(K) / 32) * sizeof(uint32_t);
   if (n <= kBitmapPlanAtoms) {
     const size_t nw = (size_t(n) + 31) / 32;
-    return 2 * nw * sizeof(uint32_t) + mask;
+    return 2 * nw * sizeof(uint32_t) + mask + size_t(kTileM) * K * sizeof(int);   // + entries
   }
   return size_t(3) * plan_capacity(K) * sizeof(int) + mask;   // table, sorted union, mask
 }
