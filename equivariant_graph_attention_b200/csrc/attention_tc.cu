@@ -92,6 +92,13 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// max(a, b, c) in one instruction (the three-input form of sm_100)
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // (a, b) as bf16x2 pairs hi + lo with hi = bf16(x) and lo = bf16(x - hi),
 // both rounded to nearest even: hi + lo equals x to about 2^-17 relative
 __device__ __forceinline__ void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
@@ -373,7 +380,7 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
       const uint32_t m0 = smask[(ub >> 5) * kTileM + g] >> ((ub & 31) + 2 * t);
       const uint32_t m1 = smask[(ub >> 5) * kTileM + g + 8] >> ((ub & 31) + 2 * t);
       float v[KS][8];   // raw logits; row g: cols 2t, 2t+1, 8+2t, 9+2t ; row g+8: same
-      bool over = false;
+      float lm0 = -INFINITY, lm1 = -INFINITY;   // this lane's largest logit of rows g, g+8
 #pragma unroll
       for (int j = 0; j < KS; ++j) {
         const uint32_t w0 = m0 >> (16 * j), w1 = m1 >> (16 * j);
@@ -385,21 +392,17 @@ otf_attention_tc_kernel(const __grid_constant__ TcParams p) {
         v[j][5] = (w1 & 2u) ? sf[j][0][3] : -INFINITY;
         v[j][6] = (w1 & 0x100u) ? sf[j][1][2] : -INFINITY;
         v[j][7] = (w1 & 0x200u) ? sf[j][1][3] : -INFINITY;
-        over |= (v[j][0] > thr0) | (v[j][1] > thr0) | (v[j][2] > thr0) | (v[j][3] > thr0) |
-                (v[j][4] > thr1) | (v[j][5] > thr1) | (v[j][6] > thr1) | (v[j][7] > thr1);
+        lm0 = max3f(max3f(lm0, v[j][0], v[j][1]), v[j][2], v[j][3]);
+        lm1 = max3f(max3f(lm1, v[j][4], v[j][5]), v[j][6], v[j][7]);
       }
+      const bool over = (lm0 > thr0) | (lm1 > thr1);
       // ---- online softmax, one test per stage.  Common case: no logit of
       // the warp's rows exceeds its row's raw threshold (mref + kLazy) / qs,
-      // tested per entry with no cross-lane traffic.  Otherwise the row
-      // maxima over the stage are formed exactly and the rows that need it
-      // are rescaled.
+      // tested on the lane's row maxima with no cross-lane traffic.
+      // Otherwise the row maxima over the stage are completed across the
+      // quad and the rows that need it are rescaled.
       if (__any_sync(0xffffffffu, over)) {
-        float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < KS; ++j) {
-          mx0 = fmaxf(mx0, fmaxf(fmaxf(v[j][0], v[j][1]), fmaxf(v[j][2], v[j][3])));
-          mx1 = fmaxf(mx1, fmaxf(fmaxf(v[j][4], v[j][5]), fmaxf(v[j][6], v[j][7])));
-        }
+        float mx0 = lm0, mx1 = lm1;
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
