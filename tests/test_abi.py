@@ -140,6 +140,33 @@ def test_plan_and_status_entry_validation(lib):
     assert lib.egat_strerror(egat.EGAT_ERR_TIMEOUT).startswith(b"a bounded device wait")
 
 
+@pytest.mark.parametrize("n,K,supported", [
+    (131072, 1024, True),     # bitmap builder: 32 KB of bitmaps + 32 KB mask + 64 KB of entries
+    (131073, 512, True),      # hash builder past 131,072 atoms: shared memory set by K alone
+    (1000000, 256, True),
+    (131073, 1024, False),    # hash builder at K = 1024: 224 KiB, past the 200 KiB limit
+])
+def test_attention_plan_size_limits(lib, n, K, supported):
+    """The documented limits of the attention plan: the bitmap builder up to
+    131,072 atoms at every K, the hash builder beyond at K <= 512, whatever
+    n is (its per-tile cost does not grow with n); the plan's size grows
+    linearly in the tile count."""
+    cs = egat.Shape(n=n, lmax=2, C=128, H=16, dk=16, K=K, dtype="bf16").c()
+    out = ctypes.c_size_t(0)
+    rc = lib.egat_attention_plan_bytes(ctypes.byref(cs), ctypes.byref(out))
+    assert rc == (egat.EGAT_OK if supported else egat.EGAT_ERR_UNSUPPORTED)
+    if supported:
+        tiles = (n + 15) // 16
+        cap = 32
+        while cap < 16 * K:
+            cap *= 2
+        a256 = lambda x: (x + 255) // 256 * 256
+        per_tile = 4 + cap * 4 + 16 * (cap // 32) * 4 + (4 + 16 * 39) * 4
+        assert out.value == a256(tiles * 4) + a256(tiles * cap * 4) + a256(tiles * 16 * (cap // 32) * 4) \
+            + a256(tiles * (4 + 16 * 39) * 4) + 256
+        assert abs(out.value - tiles * per_tile) <= 4 * 256
+
+
 def test_backward_entry_validation(lib):
     """egat_backward's host checks and workspace query (no launch on these paths)."""
     a256 = lambda x: (x + 255) // 256 * 256
